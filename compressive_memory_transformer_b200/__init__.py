@@ -1,0 +1,182 @@
+"""Python binding of libinfini_attn.so (the B200 Infini-attention forward).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library. torch supplies device memory and the stream. There is no CPU fallback:
+importing this package fails when the library is missing or cannot be loaded.
+
+Entry points (same names as the C ABI in include/infini_attn.h):
+    infini_attn_forward(q, k, v, beta, N, mode, M_in=None, z_in=None, ...)
+    infini_attn_step(q, k, v, beta, mode, M_in=None, z_in=None, ...)
+q, k, v: [B, H, L, d] CUDA tensors, bf16 (d = 128) or fp32 (d <= 128);
+beta: [H] fp32; M: [B, H, d, d] fp32; z: [B, H, d] fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LINEAR = 0
+DELTA = 1
+DTYPE_BF16 = 0
+DTYPE_F32 = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libinfini_attn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing; build it with "
+        "`python -m compressive_memory_transformer_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_ll = ctypes.c_longlong
+
+
+class Opts(ctypes.Structure):
+    _fields_ = [("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+                ("stage_events", _vp * 3)]
+
+
+_SIGS = {
+    "infini_attn_forward": [_vp] * 9 + [_i, _i, _ll, _i, _i, _i, _vp],
+    "infini_attn_step": [_vp] * 9 + [_i, _i, _i, _i, _i, _vp],
+    "infini_attn_forward_f32": [_vp] * 9 + [_i, _i, _ll, _i, _i, _i, _vp],
+    "infini_attn_step_f32": [_vp] * 9 + [_i, _i, _i, _i, _i, _vp],
+    "infini_attn_forward_ex": [_vp] * 9 + [_i, _i, _ll, _i, _i, _i, _i, ctypes.POINTER(Opts), _vp],
+    "infini_attn_workspace_size": [_i, _i, _ll, _i, _i, _i, _i],
+    "infini_attn_device_status": [],
+    "infini_attn_selftest_timeout": [_ll, _vp],
+    "infini_attn_strerror": [_i],
+    "infini_attn_version": [],
+}
+for _name, _args in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _i
+_lib.infini_attn_strerror.restype = ctypes.c_char_p
+_lib.infini_attn_workspace_size.restype = ctypes.c_size_t
+
+# every symbol the header declares (checked by the CPU tests)
+EXPORTED = tuple(_SIGS)
+
+
+class InfiniError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        super().__init__(f"infini_attn status {status}: {strerror(status)}")
+
+
+def strerror(status: int) -> str:
+    return _lib.infini_attn_strerror(int(status)).decode()
+
+
+def version() -> int:
+    return _lib.infini_attn_version()
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check(st):
+    if st != 0:
+        raise InfiniError(st)
+
+
+def _prepare(q, k, v, beta, M_in, z_in, out, M_out, z_out, state_out):
+    if q.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, L, d]")
+    B, H, L, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor shaped and typed like q")
+    if beta.dtype != torch.float32 or beta.numel() != H or not beta.is_cuda:
+        raise ValueError("beta must be a CUDA fp32 tensor with H elements")
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out and M_out is None:
+        M_out = torch.empty((B, H, d, d), device=q.device, dtype=torch.float32)
+        z_out = torch.empty((B, H, d), device=q.device, dtype=torch.float32)
+    for t in (M_in, z_in, M_out, z_out):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda):
+            raise ValueError("M and z must be contiguous CUDA fp32 tensors")
+    return B, H, L, d, out, M_out, z_out
+
+
+def infini_attn_forward(q, k, v, beta, N, mode=LINEAR, M_in=None, z_in=None, out=None,
+                        M_out=None, z_out=None, state_out=True, stream=None):
+    """Whole-sequence forward; returns (out, M_out, z_out)."""
+    B, H, L, d, out, M_out, z_out = _prepare(q, k, v, beta, M_in, z_in, out, M_out, z_out,
+                                             state_out)
+    fn = _lib.infini_attn_forward if q.dtype == torch.bfloat16 else _lib.infini_attn_forward_f32
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M_in), _ptr(z_in), _ptr(out),
+              _ptr(M_out), _ptr(z_out), B, H, L, int(N), d, int(mode), _stream_handle(stream)))
+    return out, M_out, z_out
+
+
+def infini_attn_step(q, k, v, beta, mode=LINEAR, M_in=None, z_in=None, out=None, M_out=None,
+                     z_out=None, state_out=True, stream=None):
+    """One segment (L == N) with carried state; returns (out, M_out, z_out).
+    Pass M_out=M_in, z_out=z_in to advance the state in place."""
+    B, H, L, d, out, M_out, z_out = _prepare(q, k, v, beta, M_in, z_in, out, M_out, z_out,
+                                             state_out)
+    fn = _lib.infini_attn_step if q.dtype == torch.bfloat16 else _lib.infini_attn_step_f32
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M_in), _ptr(z_in), _ptr(out),
+              _ptr(M_out), _ptr(z_out), B, H, L, d, int(mode), _stream_handle(stream)))
+    return out, M_out, z_out
+
+
+def infini_attn_forward_ex(q, k, v, beta, N, mode=LINEAR, M_in=None, z_in=None, out=None,
+                           M_out=None, z_out=None, workspace=None, stage_events=None,
+                           state_out=True, stream=None):
+    """Forward with options: a caller-owned workspace tensor (uint8, CUDA) and up to
+    three torch.cuda.Event objects recorded around the state kernels and the
+    fused attention kernel."""
+    B, H, L, d, out, M_out, z_out = _prepare(q, k, v, beta, M_in, z_in, out, M_out, z_out,
+                                             state_out)
+    dtype = DTYPE_BF16 if q.dtype == torch.bfloat16 else DTYPE_F32
+    o = Opts()
+    if workspace is not None:
+        o.workspace = workspace.data_ptr()
+        o.workspace_bytes = workspace.numel() * workspace.element_size()
+    if stage_events is not None:
+        for i_, ev in enumerate(stage_events):
+            o.stage_events[i_] = None if ev is None else ev.cuda_event
+    _check(_lib.infini_attn_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M_in),
+                                       _ptr(z_in), _ptr(out), _ptr(M_out), _ptr(z_out), B, H, L,
+                                       int(N), d, int(mode), dtype, ctypes.byref(o),
+                                       _stream_handle(stream)))
+    return out, M_out, z_out
+
+
+def workspace_size(B, H, L, N, d, mode=LINEAR, dtype=DTYPE_BF16) -> int:
+    return int(_lib.infini_attn_workspace_size(B, H, L, N, d, mode, dtype))
+
+
+def device_status() -> int:
+    """INFINI_OK (0) or INFINI_ERR_TIMEOUT (-7); synchronises the device."""
+    return _lib.infini_attn_device_status()
+
+
+def selftest_timeout(timeout_ns: int, stream=None) -> None:
+    _check(_lib.infini_attn_selftest_timeout(int(timeout_ns), _stream_handle(stream)))
+
+
+def raw_call(name, *args):
+    """Call an exported C function by name with ctypes-compatible arguments."""
+    return getattr(_lib, name)(*args)

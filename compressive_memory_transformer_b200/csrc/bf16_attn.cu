@@ -1,0 +1,441 @@
+// bf16_attn.cu — fused local attention + memory retrieval + gate (bf16, d = 128).
+//
+// One CTA computes one 128-row query tile of one segment of one (batch, head):
+//   A_dot = softmax(Q K^T / sqrt(d) + causal mask) V     over the segment's keys
+//   A_mem = sigma(Q) M_{s-1} / (sigma(Q) z_{s-1})         (0 where the denominator is 0)
+//   out   = g A_mem + (1 - g) A_dot,  g = sigmoid(beta_h)
+// ("Leave No Context Behind", arXiv 2404.07143, as quoted on
+// llm-papers-study.pages.dev: sections 3.1, 3.3, 3.5). A_dot and A_mem stay in
+// tensor memory; only `out` is written to HBM.
+//
+// Warp roles (192 threads):
+//   warp 0     TMA producer: Q tile, then the V pipeline items [M_hi, M_lo, V_0, V_1, ...]
+//              and the K pipeline items [K_0, K_1, ...], two stages each.
+//   warp 1     tensor-memory allocation and the single MMA-issuing thread.
+//   warps 2-5  softmax / epilogue: thread r owns query row r (tensor-memory lane r).
+// Tensor memory (512 columns): S0 | S1 (double-buffered scores) | O (A_dot
+// accumulator) | R (sigma(Q) M accumulator).
+// MMA order: QK_0, QK_1, R = sigma(Q)(M_hi + M_lo), then for each j: O += P_j V_j,
+// QK_{j+2}. The softmax of tile j overlaps PV_{j-1} and QK_{j+1}.
+// Online softmax keeps a per-row reference max and rescales O only when the
+// running max grows by more than 2^8 (in exp2 units), so most tiles skip the
+// tensor-memory round trip of O.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda.h>
+#include <cstdint>
+
+#include "bf16_path.h"
+#include "sm100.cuh"
+
+namespace infini {
+namespace {
+
+constexpr int D = 128;
+constexpr int BM = 128;   // query rows per CTA
+constexpr int BN = 128;   // keys per tile
+constexpr int kTile = 32768;     // one 128 x 128 bf16 tile
+constexpr int kSub = 16384;      // one 128 x 64 box (128-byte rows)
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = kTile;         // 2 stages
+constexpr int OFF_V = 3 * kTile;     // 2 stages
+constexpr int OFF_P = 5 * kTile;
+constexpr int OFF_Z = 6 * kTile;     // 128 floats
+constexpr int OFF_BAR = OFF_Z + 512;
+constexpr int kAttnSmem = OFF_BAR + 256 + 1024;  // + alignment slack
+constexpr int kThreads = 192;
+
+enum {
+  B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9,
+  B_PFULL = 11, B_PVDONE = 12, B_DRAIN = 13, B_COUNT = 14
+};
+
+// Bounded wait used only while draining after an error: ignores the error flag.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) break;  // 200 ms
+  }
+}
+
+// K-major operand (rows = M or N index, 64 bf16 of K per 128-byte row, two boxes
+// of 64 columns 16 KB apart): k-step kk covers K elements [16 kk, 16 kk + 16).
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk) {
+  return sdesc(base + (uint32_t)(kk >> 2) * kSub + (uint32_t)(kk & 3) * 32, 16, 1024);
+}
+// MN-major operand (rows = K index, 64 bf16 of N per 128-byte row, two boxes of
+// 64 columns 16 KB apart): k-step kk covers K rows [16 kk, 16 kk + 16).
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kk) {
+  return sdesc(base + (uint32_t)kk * 2048, kSub, 1024);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+            const __grid_constant__ CUtensorMap tm_m, const float* __restrict__ beta,
+            const float* __restrict__ zprev, __nv_bfloat16* __restrict__ out, long long L, int N,
+            int S, int H, int T, int BH) {
+  // ---- work item: heaviest query tiles first ----
+  const long long x = blockIdx.x;
+  const long long per = (long long)S * BH;
+  const int i = T - 1 - (int)(x / per);
+  const long long rem = x % per;
+  const int s = (int)(rem % S);
+  const int bh = (int)(rem / S);
+  const long long seg0 = (long long)s * N;
+  const int n_s = (int)min((long long)N, L - seg0);
+  const int T_s = (n_s + BM - 1) / BM;
+  if (i >= T_s) return;  // uniform for the whole CTA, before any barrier
+  const int nkv = i + 1;
+  const int q_row = (int)(seg0 + (long long)i * BM);
+  const int rows_valid = min(BM, n_s - i * BM);
+  const bool tma_store_ok = rows_valid == BM || seg0 + n_s == L;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + OFF_Q;
+  uint8_t* sK = smem + OFF_K;
+  uint8_t* sV = smem + OFF_V;
+  uint8_t* sP = smem + OFF_P;
+  float* sZ = reinterpret_cast<float*>(smem + OFF_Z);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < B_COUNT; ++b) mbar_init(&bars[b], b == B_PFULL ? 128u : 1u);
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_m);
+    tma_prefetch_desc(&tm_o);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + 256, tR = tmem + 384;
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      int k_iss[2] = {0, 0}, v_iss[2] = {0, 0};
+      auto issue_k = [&](int j) -> bool {
+        const int st = j & 1, use = j >> 1;
+        if (use > 0 && !mbar_wait(&bars[B_KEMPTY + st], (uint32_t)((use - 1) & 1))) return false;
+        mbar_arrive_expect_tx(&bars[B_KFULL + st], kTile);
+        const int row = (int)(seg0 + (long long)j * BN);
+        tma_load_3d(sK + st * kTile, &tm_k, &bars[B_KFULL + st], 0, row, bh);
+        tma_load_3d(sK + st * kTile + kSub, &tm_k, &bars[B_KFULL + st], 64, row, bh);
+        ++k_iss[st];
+        return true;
+      };
+      auto issue_v = [&](int item) -> bool {
+        const int st = item & 1, use = item >> 1;
+        if (use > 0 && !mbar_wait(&bars[B_VEMPTY + st], (uint32_t)((use - 1) & 1))) return false;
+        mbar_arrive_expect_tx(&bars[B_VFULL + st], kTile);
+        if (item < 2) {
+          const int zc = (bh * S + s) * 2 + item;
+          tma_load_3d(sV + st * kTile, &tm_m, &bars[B_VFULL + st], 0, 0, zc);
+          tma_load_3d(sV + st * kTile + kSub, &tm_m, &bars[B_VFULL + st], 64, 0, zc);
+        } else {
+          const int row = (int)(seg0 + (long long)(item - 2) * BN);
+          tma_load_3d(sV + st * kTile, &tm_v, &bars[B_VFULL + st], 0, row, bh);
+          tma_load_3d(sV + st * kTile + kSub, &tm_v, &bars[B_VFULL + st], 64, row, bh);
+        }
+        ++v_iss[st];
+        return true;
+      };
+      mbar_arrive_expect_tx(&bars[B_QFULL], kTile);
+      tma_load_3d(sQ, &tm_q, &bars[B_QFULL], 0, q_row, bh);
+      tma_load_3d(sQ + kSub, &tm_q, &bars[B_QFULL], 64, q_row, bh);
+      bool ok = issue_k(0) && (nkv < 2 || issue_k(1)) && issue_v(0) && issue_v(1);
+      for (int j = 0; ok && j < nkv; ++j) {
+        ok = issue_v(j + 2);
+        if (ok && j + 2 < nkv) ok = issue_k(j + 2);
+      }
+      if (!ok) {  // let the copies already issued land before the CTA exits
+        drain_wait(&bars[B_QFULL], 0);
+        for (int st = 0; st < 2; ++st) {
+          if (k_iss[st] > 0) drain_wait(&bars[B_KFULL + st], (uint32_t)((k_iss[st] - 1) & 1));
+          if (v_iss[st] > 0) drain_wait(&bars[B_VFULL + st], (uint32_t)((v_iss[st] - 1) & 1));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      const uint32_t id_qk = idesc_f32acc(1, 0, 0, BM, BN);
+      const uint32_t id_pv = idesc_f32acc(1, 0, 1, BM, D);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      auto qk = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!mbar_wait(&bars[B_KFULL + st], (uint32_t)((j >> 1) & 1))) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tS + st * BN, kmajor_desc(aQ, kk), kmajor_desc(aK + st * kTile, kk), id_qk,
+                      kk > 0 ? 1u : 0u);
+        mma_commit(&bars[B_KEMPTY + st]);
+        mma_commit(&bars[B_SFULL + st]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars[B_QFULL], 0);
+      ok = ok && qk(0) && (nkv < 2 || qk(1));
+      // retrieval: R = sigma(Q) M_hi + sigma(Q) M_lo
+      ok = ok && mbar_wait(&bars[B_PFULL], 0) && mbar_wait(&bars[B_VFULL + 0], 0) &&
+           mbar_wait(&bars[B_VFULL + 1], 0);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tR, kmajor_desc(aP, kk), mnmajor_desc(aV, kk), id_pv, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tR, kmajor_desc(aP, kk), mnmajor_desc(aV + kTile, kk), id_pv, 1u);
+        mma_commit(&bars[B_VEMPTY + 0]);
+        mma_commit(&bars[B_VEMPTY + 1]);
+        mma_commit(&bars[B_PVDONE]);
+      }
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int item = j + 2, st = item & 1;
+        ok = mbar_wait(&bars[B_PFULL], (uint32_t)((j + 1) & 1)) &&
+             mbar_wait(&bars[B_VFULL + st], (uint32_t)((item >> 1) & 1));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_bf16_ss(tO, kmajor_desc(aP, kk), mnmajor_desc(aV + st * kTile, kk), id_pv,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[B_VEMPTY + st]);
+        mma_commit(&bars[B_PVDONE]);
+        if (j + 2 < nkv) ok = qk(j + 2);
+      }
+      // no MMA may still be running when the CTA frees tensor memory
+      mma_commit(&bars[B_DRAIN]);
+      drain_wait(&bars[B_DRAIN], 0);
+    }
+  } else {
+    // ================= softmax / epilogue (warps 2..5) =================
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // query row inside the tile == tensor-memory lane
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const float bta = beta[bh % H];
+    const float g = 1.f / (1.f + expf(-bta));
+    sZ[r] = zprev[((size_t)bh * S + s) * D + r];
+    named_bar_sync(1, 128);
+
+    bool ok = mbar_wait(&bars[B_QFULL], 0);
+    float den = 0.f;
+    if (ok) {
+      // sigma(Q) row -> P buffer (same swizzled position), den = sigma(Q_r) . z_{s-1}
+#pragma unroll 4
+      for (int u = 0; u < 16; ++u) {
+        const uint32_t off = (uint32_t)(u >> 3) * kSub + sw128(r, u & 7);
+        const uint4 raw = *reinterpret_cast<const uint4*>(sQ + off);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h[e]);
+          const float p0 = elu1(f.x), p1 = elu1(f.y);
+          den = fmaf(p0, sZ[u * 8 + 2 * e], den);
+          den = fmaf(p1, sZ[u * 8 + 2 * e + 1], den);
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[B_PFULL]);
+    }
+
+    const float sl = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+    float m_use = -INFINITY, l = 0.f;
+    for (int j = 0; ok && j < nkv; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(&bars[B_SFULL + b], (uint32_t)((j >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[BN];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(tS + lane_off + b * BN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+      tmem_wait_ld();
+      float mt = -INFINITY;
+      if (j == i) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          if (c > r) sr[c] = __float_as_uint(-INFINITY);
+          mt = fmaxf(mt, __uint_as_float(sr[c]));
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) mt = fmaxf(mt, __uint_as_float(sr[c]));
+      }
+      bool need = false;
+      float alpha = 1.f;
+      if (j == 0) {
+        m_use = mt;
+      } else if ((mt - m_use) * sl > 8.f) {
+        need = true;
+        alpha = ex2_approx((m_use - mt) * sl);
+        m_use = mt;
+      }
+      const float mb = m_use * sl;
+      float rs = 0.f;
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int c = 0; c < BN / 2; ++c) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), sl, -mb));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), sl, -mb));
+        rs += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      // PV_{j-1} (or the retrieval, for j = 0) must be done before O or P is touched
+      if (!mbar_wait(&bars[B_PVDONE], (uint32_t)(j & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + lane_off + c * 32, o);
+        }
+        tmem_wait_st();
+      }
+      l = l * alpha + rs;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const uint32_t off = (uint32_t)(u >> 3) * kSub + sw128(r, u & 7);
+        *reinterpret_cast<uint4*>(sP + off) =
+            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars[B_PFULL]);
+    }
+
+    // ---- epilogue: out = (1 - g) O / l + g R / den ----
+    if (ok) ok = mbar_wait(&bars[B_PVDONE], (uint32_t)(nkv & 1));
+    tc_fence_after();
+    if (ok) {
+      const float go = (1.f - g) / l;
+      const float gr = den != 0.f ? g / den : 0.f;
+      __nv_bfloat16* orow = out + ((size_t)bh * L + q_row + r) * D;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32], rr[32];
+        tmem_ld32(tO + lane_off + c * 32, o);
+        tmem_ld32(tR + lane_off + c * 32, rr);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a0 = go * __uint_as_float(o[2 * e]) + gr * __uint_as_float(rr[2 * e]);
+          const float a1 = go * __uint_as_float(o[2 * e + 1]) + gr * __uint_as_float(rr[2 * e + 1]);
+          w[e] = pack_bf16x2(a0, a1);
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 val = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+          const int u = c * 4 + q4;  // 16-byte unit of the row (8 columns)
+          if (tma_store_ok) {
+            *reinterpret_cast<uint4*>(sQ + (uint32_t)(u >> 3) * kSub + sw128(r, u & 7)) = val;
+          } else if (r < rows_valid) {
+            *reinterpret_cast<uint4*>(orow + u * 8) = val;
+          }
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    named_bar_sync(1, 128);
+    if (ok && tma_store_ok && r == 0) {
+      tma_store_3d(&tm_o, sQ, 0, q_row, bh);
+      tma_store_3d(&tm_o, sQ + kSub, 64, q_row, bh);
+      tma_store_commit();
+      tma_store_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 map: (128 columns, rows, planes), box 64 x 128 x 1, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t planes) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, rows, planes};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * rows};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t bf16_attn_set_attributes() {
+  return cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kAttnSmem);
+}
+
+cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
+                             const __nv_bfloat16* v, const float* beta, __nv_bfloat16* out,
+                             const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
+                             cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mo, mm;
+  if (!make_map(&mq, q, (uint64_t)L, BH) || !make_map(&mk, k, (uint64_t)L, BH) ||
+      !make_map(&mv, v, (uint64_t)L, BH) || !make_map(&mo, out, (uint64_t)L, BH) ||
+      !make_map(&mm, ws.Mhl, D, (uint64_t)BH * S * 2))
+    return cudaErrorInvalidValue;
+  const int T = (int)((min((long long)N, L) + BM - 1) / BM);
+  const unsigned grid = (unsigned)((long long)T * S * BH);
+  attn_kernel<<<grid, kThreads, kAttnSmem, stream>>>(mq, mk, mv, mo, mm, beta, ws.zprev, out, L, N,
+                                                     S, H, T, BH);
+  return cudaGetLastError();
+}
+
+}  // namespace infini

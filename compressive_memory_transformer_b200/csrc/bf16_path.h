@@ -1,0 +1,42 @@
+// bf16_path.h — internal interface of the bf16 forward (d = 128): the state
+// kernels (bf16_state.cu) and the fused attention kernel (bf16_attn.cu).
+#pragma once
+#include <cstddef>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace infini {
+
+// Scratch of one bf16 forward call, carved from one allocation.
+//   zpart [BH][S][CH][128] f32   partial sums of sigma(K) per token chunk
+//   zprev [BH][S][128]     f32   z_{s-1} for every segment
+//   dpart [BH][S][CH][2][128][128] f32   per-chunk [dM | G] of the state GEMM
+//   Mhl   [BH][S][2][128][128] bf16      M_{s-1} as hi and lo bf16 parts
+struct Bf16Workspace {
+  float* zpart;
+  float* zprev;
+  float* dpart;
+  __nv_bfloat16* Mhl;
+};
+
+void bf16_state_plan(int BH, int S, int N, int* CH, int* CL);
+size_t bf16_workspace_bytes(int BH, int S, int CH);
+Bf16Workspace bf16_workspace_carve(void* base, int BH, int S, int CH);
+
+cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, const float* M_in,
+                              const float* z_in, float* M_out, float* z_out,
+                              const Bf16Workspace& ws, int BH, long long L, int N, int S, int CH,
+                              int CL, int mode, cudaStream_t stream);
+
+// The fused local-attention + retrieval + gate kernel. Reads q, k, v, beta and
+// the workspace's zprev / Mhl; writes out.
+cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
+                             const __nv_bfloat16* v, const float* beta, __nv_bfloat16* out,
+                             const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
+                             cudaStream_t stream);
+
+// Sets the dynamic shared-memory limits of the kernels on the current device
+// (once per device).
+cudaError_t bf16_prepare_device();
+
+}  // namespace infini

@@ -1,0 +1,294 @@
+// infini_attn.cu — the C ABI (include/infini_attn.h): argument checks, scratch
+// memory, and the launch sequence of the forward.
+//
+// bf16 (d = 128): zpart -> zscan -> state (tcgen05 tf32) -> chain -> attn (tcgen05 bf16)
+// fp32 (d <= 128): f32_state -> f32_attn (CUDA cores)
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "infini_attn.h"
+#include "bf16_path.h"
+#include "f32_path.h"
+#include "sm100.cuh"
+
+namespace infini {
+
+__device__ int g_device_error = 0;
+__device__ unsigned long long g_wait_timeout_ns = 4000000000ull;  // 4 s per wait
+
+cudaError_t bf16_state_set_attributes();
+cudaError_t bf16_attn_set_attributes();
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_prepared[kMaxDevices];
+
+cudaError_t prepare_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (g_prepared[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = bf16_state_set_attributes();
+  if (e == cudaSuccess) e = bf16_attn_set_attributes();
+  if (e == cudaSuccess) g_prepared[dev].store(1, std::memory_order_release);
+  return e;
+}
+
+// Copies (or zero-fills) the state when there is nothing to process.
+__global__ void pass_state_kernel(const float* M_in, const float* z_in, float* M_out,
+                                  float* z_out, long long nM, long long nz) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nM;
+       i += (long long)gridDim.x * blockDim.x) {
+    if (i < nz && z_out) z_out[i] = z_in ? z_in[i] : 0.f;
+    if (M_out) M_out[i] = M_in ? M_in[i] : 0.f;
+  }
+}
+
+__global__ void timeout_selftest_kernel(unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // nothing ever arrives on this barrier: the wait must run out and report
+    const uint32_t a = smem_u32(&bar);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(a, 0)) {
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        raise_device_error(kDevErrTimeout);
+        break;
+      }
+    }
+  }
+}
+
+bool overflows(long long a, long long b) { return a != 0 && b > (long long)(INT64_MAX / a); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+int check_common(const void* q, const void* k, const void* v, const float* beta,
+                 const float* M_in, const float* z_in, const void* out, const float* M_out,
+                 const float* z_out, int B, int H, long long L, int N, int d, int mode,
+                 size_t esize) {
+  if (!q || !k || !v || !beta || !out) return INFINI_ERR_NULL;
+  if ((M_in == nullptr) != (z_in == nullptr)) return INFINI_ERR_NULL;
+  if ((M_out == nullptr) != (z_out == nullptr)) return INFINI_ERR_NULL;
+  if (B < 1 || H < 1 || N < 1 || L < 0 || d < 1) return INFINI_ERR_SHAPE;
+  if (mode != INFINI_LINEAR && mode != INFINI_DELTA) return INFINI_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > (1LL << 30)) return INFINI_ERR_SHAPE;
+  if (overflows(BH, L) || overflows(BH * L, d) || overflows(BH * L * d, (long long)esize))
+    return INFINI_ERR_SHAPE;
+  if (L >= (1LL << 31)) return INFINI_ERR_SHAPE;
+  const size_t nio = (size_t)(BH * L * d) * esize;
+  const size_t nM = (size_t)BH * d * d * sizeof(float), nz = (size_t)BH * d * sizeof(float);
+  if (overlap(out, nio, q, nio) || overlap(out, nio, k, nio) || overlap(out, nio, v, nio) ||
+      overlap(out, nio, M_in, nM) || overlap(out, nio, z_in, nz) ||
+      overlap(out, nio, M_out, nM) || overlap(out, nio, z_out, nz))
+    return INFINI_ERR_ALIAS;
+  return INFINI_OK;
+}
+
+int pass_state(const float* M_in, const float* z_in, float* M_out, float* z_out, long long BH,
+               int d, cudaStream_t stream) {
+  if (!M_out) return INFINI_OK;
+  const long long nM = BH * d * d, nz = BH * d;
+  pass_state_kernel<<<(unsigned)min((nM + 255) / 256, 4096LL), 256, 0, stream>>>(M_in, z_in,
+                                                                                  M_out, z_out,
+                                                                                  nM, nz);
+  return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+struct Scratch {
+  void* ptr = nullptr;
+  bool owned = false;
+  cudaStream_t stream = nullptr;
+  ~Scratch() {
+    if (owned && ptr) cudaFreeAsync(ptr, stream);
+  }
+};
+
+int get_scratch(Scratch& s, size_t bytes, const infini_attn_opts_t* opts, cudaStream_t stream) {
+  if (bytes == 0) return INFINI_OK;
+  if (opts && opts->workspace) {
+    if (opts->workspace_bytes < bytes) return INFINI_ERR_NOMEM;
+    if ((reinterpret_cast<uintptr_t>(opts->workspace) & 255u) != 0) return INFINI_ERR_ALIGN;
+    s.ptr = opts->workspace;
+    return INFINI_OK;
+  }
+  if (cudaMallocAsync(&s.ptr, bytes, stream) != cudaSuccess) {
+    cudaGetLastError();
+    s.ptr = nullptr;
+    return INFINI_ERR_NOMEM;
+  }
+  s.owned = true;
+  s.stream = stream;
+  return INFINI_OK;
+}
+
+void record(const infini_attn_opts_t* opts, int i, cudaStream_t stream) {
+  if (opts && opts->stage_events[i])
+    cudaEventRecord(static_cast<cudaEvent_t>(opts->stage_events[i]), stream);
+}
+
+int forward_impl(const void* q, const void* k, const void* v, const float* beta,
+                 const float* M_in, const float* z_in, void* out, float* M_out, float* z_out,
+                 int B, int H, long long L, int N, int d, int mode, int dtype,
+                 const infini_attn_opts_t* opts, cudaStream_t stream) {
+  if (dtype != INFINI_DTYPE_BF16 && dtype != INFINI_DTYPE_F32) return INFINI_ERR_UNSUPPORTED;
+  const size_t esize = dtype == INFINI_DTYPE_BF16 ? 2 : 4;
+  int st = check_common(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, L, N, d, mode, esize);
+  if (st != INFINI_OK) return st;
+  if (dtype == INFINI_DTYPE_BF16 && d != 128) return INFINI_ERR_UNSUPPORTED;
+  if (dtype == INFINI_DTYPE_F32 && d > 128) return INFINI_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return INFINI_ERR_ALIGN;
+  if ((M_in && !aligned16(M_in)) || (M_out && !aligned16(M_out))) return INFINI_ERR_ALIGN;
+  const int BH = B * H;
+  if (L == 0) {
+    record(opts, 0, stream);
+    st = pass_state(M_in, z_in, M_out, z_out, BH, d, stream);
+    record(opts, 1, stream);
+    record(opts, 2, stream);
+    return st;
+  }
+  if (prepare_device() != cudaSuccess) return INFINI_ERR_CUDA;
+  const int S = (int)((L + N - 1) / N);
+  if (dtype == INFINI_DTYPE_F32) {
+    Scratch sc;
+    st = get_scratch(sc, f32_workspace_bytes(BH, S, d), opts, stream);
+    if (st != INFINI_OK) return st;
+    record(opts, 0, stream);
+    const cudaError_t e = f32_forward_launch(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        beta, M_in, z_in, static_cast<float*>(out), M_out, z_out, BH, H, L, N, d, mode, sc.ptr,
+        stream);
+    record(opts, 1, stream);
+    record(opts, 2, stream);
+    return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+  }
+  int CH = 1, CL = N;
+  bf16_state_plan(BH, S, N, &CH, &CL);
+  if ((long long)BH * S * CH >= (1LL << 31)) return INFINI_ERR_SHAPE;
+  Scratch sc;
+  st = get_scratch(sc, bf16_workspace_bytes(BH, S, CH), opts, stream);
+  if (st != INFINI_OK) return st;
+  const Bf16Workspace ws = bf16_workspace_carve(sc.ptr, BH, S, CH);
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  record(opts, 0, stream);
+  cudaError_t e = bf16_state_launch(kb, vb, M_in, z_in, M_out, z_out, ws, BH, L, N, S, CH, CL,
+                                    mode, stream);
+  if (e != cudaSuccess) return INFINI_ERR_CUDA;
+  record(opts, 1, stream);
+  e = bf16_attn_launch(qb, kb, vb, beta, static_cast<__nv_bfloat16*>(out), ws, BH, H, L, N, S,
+                       stream);
+  record(opts, 2, stream);
+  return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace infini
+
+using namespace infini;
+
+extern "C" {
+
+int infini_attn_forward(const void* q, const void* k, const void* v, const float* beta,
+                        const float* M_in, const float* z_in, void* out, float* M_out,
+                        float* z_out, int B, int H, long long L, int N, int d, int mode,
+                        void* stream) {
+  return forward_impl(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, L, N, d, mode,
+                      INFINI_DTYPE_BF16, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int infini_attn_step(const void* q, const void* k, const void* v, const float* beta,
+                     const float* M_in, const float* z_in, void* out, float* M_out,
+                     float* z_out, int B, int H, int N, int d, int mode, void* stream) {
+  return forward_impl(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, N, N < 1 ? 1 : N, d,
+                      mode, INFINI_DTYPE_BF16, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int infini_attn_forward_f32(const float* q, const float* k, const float* v, const float* beta,
+                            const float* M_in, const float* z_in, float* out, float* M_out,
+                            float* z_out, int B, int H, long long L, int N, int d, int mode,
+                            void* stream) {
+  return forward_impl(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, L, N, d, mode,
+                      INFINI_DTYPE_F32, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int infini_attn_step_f32(const float* q, const float* k, const float* v, const float* beta,
+                         const float* M_in, const float* z_in, float* out, float* M_out,
+                         float* z_out, int B, int H, int N, int d, int mode, void* stream) {
+  return forward_impl(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, N, N < 1 ? 1 : N, d,
+                      mode, INFINI_DTYPE_F32, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+size_t infini_attn_workspace_size(int B, int H, long long L, int N, int d, int mode, int dtype) {
+  (void)mode;
+  if (B < 1 || H < 1 || N < 1 || L <= 0 || d < 1) return 0;
+  const int BH = B * H;
+  const int S = (int)((L + N - 1) / N);
+  if (dtype == INFINI_DTYPE_F32) return f32_workspace_bytes(BH, S, d);
+  int CH = 1, CL = N;
+  bf16_state_plan(BH, S, N, &CH, &CL);
+  return bf16_workspace_bytes(BH, S, CH);
+}
+
+int infini_attn_forward_ex(const void* q, const void* k, const void* v, const float* beta,
+                           const float* M_in, const float* z_in, void* out, float* M_out,
+                           float* z_out, int B, int H, long long L, int N, int d, int mode,
+                           int dtype, const infini_attn_opts_t* opts, void* stream) {
+  return forward_impl(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, L, N, d, mode, dtype,
+                      opts, static_cast<cudaStream_t>(stream));
+}
+
+int infini_attn_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return INFINI_ERR_CUDA;
+  int flag = 0;
+  if (cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int)) != cudaSuccess)
+    return INFINI_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess)
+    return INFINI_ERR_CUDA;
+  return flag == kDevErrTimeout ? INFINI_ERR_TIMEOUT : INFINI_OK;
+}
+
+int infini_attn_selftest_timeout(long long timeout_ns, void* stream) {
+  if (timeout_ns < 0 || timeout_ns > 10000000000LL) return INFINI_ERR_SHAPE;
+  timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+const char* infini_attn_strerror(int status) {
+  switch (status) {
+    case INFINI_OK: return "ok";
+    case INFINI_ERR_NULL: return "a required pointer is NULL (or M/z NULL-ness differs)";
+    case INFINI_ERR_SHAPE: return "invalid or overflowing sizes";
+    case INFINI_ERR_UNSUPPORTED: return "unsupported head width, mode or dtype";
+    case INFINI_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case INFINI_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case INFINI_ERR_NOMEM: return "scratch memory could not be obtained";
+    case INFINI_ERR_TIMEOUT: return "a bounded device wait ran out";
+    case INFINI_ERR_ALIAS: return "out overlaps an input or the state";
+    default: return "unknown status";
+  }
+}
+
+int infini_attn_version(void) { return 100; }
+
+}  // extern "C"

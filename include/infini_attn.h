@@ -1,0 +1,158 @@
+/*
+ * infini_attn.h — C ABI of the B200 (sm_100a) Infini-attention forward library.
+ *
+ * The operation is the Infini-attention layer of "Leave No Context Behind:
+ * Efficient Infinite Context Transformers with Infini-attention" (Munkhdalai,
+ * Faruqui, Golovnev; arXiv 2404.07143), as quoted on the close-reading note
+ * llm-papers-study.pages.dev ("精读笔记：Infini-attention"), section 3.
+ * For every (batch b, head h) the sequence of L tokens is cut into segments of N
+ * tokens (the last one may be shorter). For segment s, with sigma = ELU + 1 and
+ * g_h = sigmoid(beta_h):
+ *
+ *   A_dot = softmax(Q_s K_s^T / sqrt(d) + causal mask) V_s          (section 3.1)
+ *   A_mem = sigma(Q_s) M_{s-1} / (sigma(Q_s) z_{s-1})                 (section 3.3)
+ *   out_s = g_h * A_mem + (1 - g_h) * A_dot                           (section 3.5)
+ *   Linear:       M_s = M_{s-1} + sigma(K_s)^T V_s                    (section 3.4)
+ *   Linear+Delta: M_s = M_{s-1} + sigma(K_s)^T (V_s - sigma(K_s) M_{s-1}
+ *                                                 / (sigma(K_s) z_{s-1}))
+ *   both modes:   z_s = z_{s-1} + sum_t sigma(K_{s,t})
+ *
+ * The output of a segment is formed from the state before that segment's update
+ * (read, then write: section 3.8 summary; waylandz.com chapter 24, section 24.5).
+ * Conventions fixed by this library: the softmax scale is 1/sqrt(d); the causal
+ * mask is inside the segment and includes the diagonal; a row whose denominator
+ * sigma(x) . z is exactly 0 (the zero state, e.g. the first segment from
+ * M_0 = 0, z_0 = 0) retrieves 0 and contributes no delta term; the gate is still
+ * applied to such rows.
+ *
+ * Layouts (all contiguous, row-major):
+ *   q, k, v, out : [B, H, L, d]     (bf16 for the plain names, fp32 for *_f32)
+ *   beta         : [H] fp32         one gate logit per head, shared by the batch
+ *   M            : [B, H, d, d] fp32, row = key feature, column = value feature
+ *   z            : [B, H, d] fp32
+ *
+ * Pointers are device pointers owned by the caller; the library keeps none of
+ * them after the call returns. M_in/z_in may be NULL (zero state, both must be
+ * NULL together). M_out/z_out may be NULL (state not written; both together) and
+ * may equal M_in/z_in (in-place carry: the library reads the old state before it
+ * writes the new one). out must not overlap q, k, v, M or z.
+ *
+ * Execution: every call is asynchronous on `stream` (a cudaStream_t, NULL = the
+ * legacy default stream). The return value reports argument errors (checked on
+ * the host before any launch) and launch errors. Faults during execution surface
+ * at the caller's next synchronisation. No call synchronises with the host and
+ * none falls back to the CPU.
+ */
+#ifndef INFINI_ATTN_H
+#define INFINI_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  INFINI_LINEAR = 0, /* section 3.4, Linear update */
+  INFINI_DELTA = 1   /* section 3.4, Linear + Delta update */
+} infini_mode_t;
+
+typedef enum {
+  INFINI_OK = 0,
+  INFINI_ERR_NULL = -1,        /* a required pointer is NULL, or M/z NULL-ness mismatched */
+  INFINI_ERR_SHAPE = -2,       /* B, H, N < 1, L < 0, or a size product overflows */
+  INFINI_ERR_UNSUPPORTED = -3, /* d or mode not supported by this entry point */
+  INFINI_ERR_ALIGN = -4,       /* q, k, v or out not 16-byte aligned */
+  INFINI_ERR_CUDA = -5,        /* a CUDA runtime call or a launch failed */
+  INFINI_ERR_NOMEM = -6,       /* the stream-ordered scratch allocation failed */
+  INFINI_ERR_TIMEOUT = -7,     /* a bounded device wait ran out (infini_attn_device_status) */
+  INFINI_ERR_ALIAS = -8        /* out overlaps an input or the state */
+} infini_status_t;
+
+/*
+ * Whole-sequence forward, bf16 q/k/v/out (__nv_bfloat16), fp32 beta/M/z.
+ * Requires d == 128. L may be 0 (the state is passed through) and need not be a
+ * multiple of N (the last segment is shorter). Scratch memory for the per-segment
+ * states is taken from the stream-ordered allocator on `stream` and returned on
+ * the same stream before the call returns (INFINI_ERR_NOMEM if that fails).
+ */
+int infini_attn_forward(const void* q, const void* k, const void* v, const float* beta,
+                        const float* M_in, const float* z_in, void* out, float* M_out,
+                        float* z_out, int B, int H, long long L, int N, int d, int mode,
+                        void* stream);
+
+/*
+ * One segment of a stream with carried state (section 3.4: the new state is
+ * passed to the next segment). Same as infini_attn_forward with L == N; the
+ * output uses (M_in, z_in), then the state advances to (M_out, z_out), which may
+ * be the same buffers. bf16 q/k/v/out [B, H, N, d].
+ */
+int infini_attn_step(const void* q, const void* k, const void* v, const float* beta,
+                     const float* M_in, const float* z_in, void* out, float* M_out,
+                     float* z_out, int B, int H, int N, int d, int mode, void* stream);
+
+/* fp32 q/k/v/out variants of the two calls above; 1 <= d <= 128. */
+int infini_attn_forward_f32(const float* q, const float* k, const float* v, const float* beta,
+                            const float* M_in, const float* z_in, float* out, float* M_out,
+                            float* z_out, int B, int H, long long L, int N, int d, int mode,
+                            void* stream);
+int infini_attn_step_f32(const float* q, const float* k, const float* v, const float* beta,
+                         const float* M_in, const float* z_in, float* out, float* M_out,
+                         float* z_out, int B, int H, int N, int d, int mode, void* stream);
+
+/*
+ * Options for the extended forward. All fields may be zero.
+ *   workspace / workspace_bytes: caller-owned device scratch of at least
+ *     infini_attn_workspace_size(...) bytes, 256-byte aligned; when NULL the
+ *     library uses the stream-ordered allocator as infini_attn_forward does.
+ *   stage_events[0..2]: cudaEvent_t handles (or NULL) recorded on `stream`
+ *     before the state kernels, between the state kernels and the fused
+ *     attention kernel, and after the fused attention kernel.
+ */
+typedef struct {
+  void* workspace;
+  size_t workspace_bytes;
+  void* stage_events[3];
+} infini_attn_opts_t;
+
+/* dtype codes for the extended calls */
+#define INFINI_DTYPE_BF16 0
+#define INFINI_DTYPE_F32 1
+
+/* Scratch bytes the forward needs for these sizes (0 when none is needed). */
+size_t infini_attn_workspace_size(int B, int H, long long L, int N, int d, int mode,
+                                  int dtype);
+
+/* infini_attn_forward / _f32 with options (dtype selects the element type). */
+int infini_attn_forward_ex(const void* q, const void* k, const void* v, const float* beta,
+                           const float* M_in, const float* z_in, void* out, float* M_out,
+                           float* z_out, int B, int H, long long L, int N, int d, int mode,
+                           int dtype, const infini_attn_opts_t* opts, void* stream);
+
+/*
+ * Device-side status of earlier calls on the current device: INFINI_OK, or
+ * INFINI_ERR_TIMEOUT when a bounded wait inside a kernel ran out (the kernel
+ * then stopped early and its outputs are invalid). Synchronises the device,
+ * then clears the flag.
+ */
+int infini_attn_device_status(void);
+
+/*
+ * Runs one kernel whose only work is a bounded wait, on a barrier that nothing
+ * arrives at, for about timeout_ns nanoseconds; it exists to exercise the
+ * timeout path above (expected result: INFINI_ERR_TIMEOUT from
+ * infini_attn_device_status afterwards).
+ */
+int infini_attn_selftest_timeout(long long timeout_ns, void* stream);
+
+/* Text for a status code (static storage). */
+const char* infini_attn_strerror(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int infini_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INFINI_ATTN_H */

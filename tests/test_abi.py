@@ -1,0 +1,104 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from compressive_memory_transformer_b200 import build
+    build.build()
+    import compressive_memory_transformer_b200 as m
+    return m
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "infini_attn.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(infini_attn_\w+)\s*\(", txt)))
+
+
+def test_header_symbols_exported(lib):
+    names = header_functions()
+    assert len(names) >= 10
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for n in names:
+        assert hasattr(so, n), f"{n} declared in the header but not exported"
+    assert set(names) == set(lib.EXPORTED)
+
+
+def test_version_and_strerror(lib):
+    assert lib.version() >= 100
+    for code in range(-8, 1):
+        s = lib.strerror(code)
+        assert s and s != "unknown status"
+    assert lib.strerror(-99) == "unknown status"
+
+
+FAKE = 1 << 20  # a 16-byte aligned, never dereferenced address
+
+
+def call_fwd(lib, q=FAKE, k=FAKE + 4096, v=FAKE + 8192, beta=FAKE + 12288, M_in=None, z_in=None,
+             out=FAKE * 2, M_out=None, z_out=None, B=1, H=1, L=128, N=128, d=128, mode=0,
+             name="infini_attn_forward"):
+    return lib.raw_call(name, q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, L, N, d, mode,
+                        None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(k=None), -1), (dict(v=None), -1), (dict(beta=None), -1),
+    (dict(out=None), -1),
+    (dict(M_in=FAKE * 4), -1),            # M_in without z_in
+    (dict(M_out=FAKE * 4), -1),           # M_out without z_out
+    (dict(B=0), -2), (dict(H=-1), -2), (dict(N=0), -2), (dict(L=-5), -2),
+    (dict(L=1 << 31), -2),
+    (dict(d=64), -3), (dict(d=256), -3), (dict(mode=2), -3),
+    (dict(q=FAKE + 2), -4), (dict(out=FAKE * 2 + 8), -4),
+    (dict(out=FAKE + 64), -8),            # out overlaps q
+])
+def test_forward_rejects_bad_arguments(lib, kw, code):
+    assert call_fwd(lib, **kw) == code
+
+
+def test_f32_rejects_wide_heads(lib):
+    assert call_fwd(lib, d=129, name="infini_attn_forward_f32") == -3
+    assert call_fwd(lib, d=0, name="infini_attn_forward_f32") == -2
+
+
+def test_step_rejects_bad_arguments(lib):
+    st = lib.raw_call("infini_attn_step", None, FAKE, FAKE, FAKE, None, None, FAKE * 2, None,
+                      None, 1, 1, 128, 128, 0, None)
+    assert st == -1
+    st = lib.raw_call("infini_attn_step", FAKE, FAKE, FAKE, FAKE, None, None, FAKE * 2, None,
+                      None, 1, 1, 128, 64, 0, None)
+    assert st == -3
+
+
+def test_workspace_size_is_host_only(lib):
+    assert lib.workspace_size(1, 1, 0, 128, 128) == 0
+    w1 = lib.workspace_size(4, 8, 32768, 2048, 128, 0, 0)
+    w2 = lib.workspace_size(4, 8, 32768, 2048, 128, 1, 0)
+    assert w1 > 0 and w1 == w2
+    # per (head, segment): z partials + z_{s-1} + [dM | G] + hi/lo M
+    assert w1 >= 32 * 16 * (2 * 128 * 128 * 4 + 2 * 128 * 128 * 2)
+    assert lib.workspace_size(1, 2, 256, 64, 64, 0, 1) > 0
+
+
+def test_package_fails_loudly_without_library(tmp_path):
+    import subprocess
+    import sys
+    code = ("import sys, shutil, os; sys.path.insert(0, %r); "
+            "import importlib.util as u; "
+            "spec = u.spec_from_file_location('pkgcopy', %r); m = u.module_from_spec(spec); "
+            "spec.loader.exec_module(m)") % (
+        str(tmp_path), str(tmp_path / "pkgcopy" / "__init__.py"))
+    (tmp_path / "pkgcopy").mkdir()
+    src = open(os.path.join(ROOT, "compressive_memory_transformer_b200", "__init__.py")).read()
+    (tmp_path / "pkgcopy" / "__init__.py").write_text(src)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True)
+    assert r.returncode != 0 and "ImportError" in r.stderr and "missing" in r.stderr
