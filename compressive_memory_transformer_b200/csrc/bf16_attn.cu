@@ -27,6 +27,7 @@
 
 #include "bf16_path.h"
 #include "sm100.cuh"
+#include "tma_map.h"
 
 namespace infini {
 namespace {
@@ -380,41 +381,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   }
 }
 
-// ---------------------------------------------------------------------------
-// Host side: tensor maps
-// ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 3-D bf16 map: (128 columns, rows, planes), box 64 x 128 x 1, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t planes) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, rows, planes};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * rows};
-  const cuuint32_t box[3] = {64, 128, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 cudaError_t bf16_attn_set_attributes() {
@@ -427,9 +393,10 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                              const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
                              cudaStream_t stream) {
   CUtensorMap mq, mk, mv, mo, mm;
-  if (!make_map(&mq, q, (uint64_t)L, BH) || !make_map(&mk, k, (uint64_t)L, BH) ||
-      !make_map(&mv, v, (uint64_t)L, BH) || !make_map(&mo, out, (uint64_t)L, BH) ||
-      !make_map(&mm, ws.Mhl, D, (uint64_t)BH * S * 2))
+  if (!make_bf16_map(&mq, q, (uint64_t)L, BH, 128) || !make_bf16_map(&mk, k, (uint64_t)L, BH, 128) ||
+      !make_bf16_map(&mv, v, (uint64_t)L, BH, 128) ||
+      !make_bf16_map(&mo, out, (uint64_t)L, BH, 128) ||
+      !make_bf16_map(&mm, ws.Mhl, D, (uint64_t)BH * S * 2, 128))
     return cudaErrorInvalidValue;
   const int T = (int)((min((long long)N, L) + BM - 1) / BM);
   const unsigned grid = (unsigned)((long long)T * S * BH);

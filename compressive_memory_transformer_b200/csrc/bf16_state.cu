@@ -17,7 +17,7 @@
 // Kernels (launch order):
 //   zpart_kernel  : partial sums of sigma(K) per (head, segment, token chunk)
 //   zscan_kernel  : z_{s-1} for every segment (fixed order), z_out
-//   state_kernel  : tf32 tcgen05 GEMM per (head, segment, chunk):
+//   state_kernel  : bf16 tcgen05 GEMMs per (head, segment, chunk):
 //                   [dM | G] = sigma(K)^T [V | diag(inv) sigma(K)]
 //   chain_kernel  : per (head, 32-column block of M): M_{s-1} for every segment
 //                   (written as a bf16 hi/lo pair for the retrieval GEMM), M_out.
@@ -27,6 +27,7 @@
 
 #include "bf16_path.h"
 #include "sm100.cuh"
+#include "tma_map.h"
 
 namespace infini {
 namespace {
@@ -99,42 +100,54 @@ __global__ void __launch_bounds__(D) zscan_kernel(const float* __restrict__ zpar
 }
 
 // ---------------------------------------------------------------------------
-// state_kernel: grid = BH * S * CH, block 256, one CTA per (head, segment, chunk).
+// state_kernel: grid = BH * S * CH, one CTA per (head, segment, chunk of tokens).
 //
-// Operands in shared memory, fp32 (read as tf32 by kind::tf32), 128-byte swizzle,
-// MN-major (the feature index is contiguous, tokens are rows):
-//   A slab = sigma(K)          [32 tokens x 128 features]   4 chunks of 32 features
-//   B slab = [V | inv*sigma(K)] [32 tokens x 256 features]  8 chunks (Delta) / 4 (Linear)
-// Each chunk is 32 rows x 128 B = 4 KB (LBO = 4096), 8-row groups 1024 B apart
-// (SBO = 1024). One tf32 MMA covers 8 tokens (K = 8): M = 128, N = 128 or 256.
-// The accumulator D[feature i][j] lives in tensor memory: columns 0..127 hold
-// dM, columns 128..255 hold G.
+// For the chunk's tokens it accumulates, in tensor memory,
+//   columns   0..127: dM = sigma(K)^T V
+//   columns 128..255: G  = sigma(K)^T diag(inv) sigma(K)      (Delta only)
+// with bf16 tcgen05 MMAs (fp32 accumulation). sigma(K) is split into
+// hi = rn_bf16(sigma) and lo = rn_bf16(sigma - hi), and dM = hi^T V + lo^T V
+// (V is exact in bf16), which keeps dM within ~2^-16 relative per term. G sums
+// only positive terms, so its bf16 rounding errors average out: G = hi^T (inv sigma)_bf16.
+//
+// Tokens move in slabs of 64. Per slab and pipeline stage (64 KB):
+//   KH  [64 x 128] bf16: K as loaded by TMA, overwritten in place by sigma(K)_hi
+//   V   [64 x 128] bf16: loaded by TMA, used as is
+//   GH  [64 x 128] bf16: (inv * sigma(K))_bf16            (Delta only)
+//   KL  [64 x 128] bf16: sigma(K)_lo
+// each as two boxes of 64 features (8 KB), 128-byte swizzle, rows = tokens. As
+// MMA operands they are MN-major (features contiguous, tokens = K); V and GH are
+// adjacent so that hi^T [V | GH] is one N = 256 MMA.
+// Warps 0..7 convert; warp 8 issues the TMA copies and the MMAs.
 // ---------------------------------------------------------------------------
-constexpr int kSlab = 32;
-constexpr int kStages = 2;
-constexpr int kAChunkBytes = kSlab * 128;             // 4 KB
-constexpr int kABytes = 4 * kAChunkBytes;             // 16 KB
-constexpr int kBBytes = 8 * kAChunkBytes;             // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;        // 48 KB
-constexpr int kStateSmem = kStages * kStageBytes + 2048;  // + alignment slack, barriers, z
+constexpr int kSlab = 64;
+constexpr int kStages = 3;
+constexpr int kBox = kSlab * 128;          // one 64-row x 64-feature box: 8 KB
+constexpr int kMat = 2 * kBox;             // one [64 x 128] bf16 matrix: 16 KB
+constexpr int OFF_KH = 0, OFF_V = kMat, OFF_GH = 2 * kMat, OFF_KL = 3 * kMat;
+constexpr int kStageBytes = 4 * kMat;      // 64 KB
+constexpr int kStateThreads = 288;
+constexpr int kStateSmem = kStages * kStageBytes + 1024 + 1024;  // + alignment, barriers, z
 
-__device__ __forceinline__ uint32_t tf32_round(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
+__device__ __forceinline__ uint64_t slab_desc(uint32_t base, int kk) {
+  // MN-major: 16 token rows per k-step (2048 B), 64-feature boxes kBox apart
+  return sdesc(base + (uint32_t)kk * 2048, kBox, 1024);
 }
 
-__global__ void __launch_bounds__(256, 1)
-state_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+__global__ void __launch_bounds__(kStateThreads, 1)
+state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const float* __restrict__ zprev, float* __restrict__ dpart, long long L, int N, int S,
              int CH, int CL, int mode) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bar_mma = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);  // [kStages]
-  uint64_t* bar_done = bar_mma + kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_done + 1);
-  float* sZ = reinterpret_cast<float*>(smem + kStages * kStageBytes + 128);     // [128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* bar_full = bars;                 // [kStages] TMA landed
+  uint64_t* bar_conv = bars + kStages;       // [kStages] operands converted (256 arrivals)
+  uint64_t* bar_mma = bars + 2 * kStages;    // [kStages] MMAs of the stage done
+  uint64_t* bar_done = bars + 3 * kStages;   // all MMAs done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
+  float* sZ = reinterpret_cast<float*>(smem + kStages * kStageBytes + 512);  // [128]
 
   const long long idx = blockIdx.x;
   const int c = (int)(idx % CH);
@@ -144,18 +157,22 @@ state_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restric
   const int n = (int)min((long long)N, L - t0);
   const int beg = min(n, c * CL), end = min(n, (c + 1) * CL);
   const int len = end - beg;
-  const int nslab = len > 0 ? (len + kSlab - 1) / kSlab : 1;
+  const int nslab = len > 0 ? (len + kSlab - 1) / kSlab : 0;
   const bool delta = mode == 1;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t ncols = delta ? 256u : 128u;
 
   if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) mbar_init(&bar_mma[i], 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_conv[i], 256);
+      mbar_init(&bar_mma[i], 1);
+    }
     mbar_init(bar_done, 1);
     fence_barrier_init();
   }
   if (tid < D) sZ[tid] = delta ? zprev[((size_t)bh * S + s) * D + tid] : 0.f;
-  if (warp == 0) {
+  if (warp == 8) {
     tmem_alloc(tmem_slot, ncols);
     tmem_relinquish();
   }
@@ -165,118 +182,141 @@ state_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restric
   const uint32_t tmem_d = *tmem_slot;
   bool ok = true;
 
-  // conversion mapping: item = tid + 256*it, token row r = item / 16, 8-feature group cg
-  const __nv_bfloat16* kbase = k + ((size_t)bh * L + t0 + beg) * D;
-  const __nv_bfloat16* vbase = v + ((size_t)bh * L + t0 + beg) * D;
-  uint4 kr[2], vr[2];
-  auto load_slab = [&](int sl) {
+  if (warp == 8) {
+    // ---------------- producer + MMA issuer ----------------
+    if (lane == 0 && nslab > 0) {
+      const int row0 = (int)(t0 + beg);
+      auto load = [&](int sl) {
+        uint8_t* st = smem + (sl % kStages) * kStageBytes;
+        uint64_t* fb = &bar_full[sl % kStages];
+        mbar_arrive_expect_tx(fb, 2 * kMat);
+        const int row = row0 + sl * kSlab;
+        tma_load_3d(st + OFF_KH, &tm_k, fb, 0, row, (int)bh);
+        tma_load_3d(st + OFF_KH + kBox, &tm_k, fb, 64, row, (int)bh);
+        tma_load_3d(st + OFF_V, &tm_v, fb, 0, row, (int)bh);
+        tma_load_3d(st + OFF_V + kBox, &tm_v, fb, 64, row, (int)bh);
+      };
+      int issued = 0;
+      for (; issued < nslab && issued < kStages; ++issued) load(issued);
+      const uint32_t id256 = idesc_f32acc(1, 1, 1, 128, 256);
+      const uint32_t id128 = idesc_f32acc(1, 1, 1, 128, 128);
+      for (int sl = 0; sl < nslab && ok; ++sl) {
+        const int stg = sl % kStages;
+        if (!mbar_wait(&bar_conv[stg], (uint32_t)((sl / kStages) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t base = smem_u32(smem + stg * kStageBytes);
 #pragma unroll
-    for (int it = 0; it < 2; ++it) {
-      const int item = tid + 256 * it;
-      const int r = item >> 4, cg = item & 15;
-      const int t = sl * kSlab + r;
-      if (t < len) {
-        kr[it] = __ldg(reinterpret_cast<const uint4*>(kbase + (size_t)t * D + cg * 8));
-        vr[it] = __ldg(reinterpret_cast<const uint4*>(vbase + (size_t)t * D + cg * 8));
-      } else {
-        kr[it] = make_uint4(0, 0, 0, 0);
-        vr[it] = make_uint4(0, 0, 0, 0);
+        for (int kk = 0; kk < kSlab / 16; ++kk) {
+          const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t a_hi = slab_desc(base + OFF_KH, kk);
+          const uint64_t a_lo = slab_desc(base + OFF_KL, kk);
+          const uint64_t b_v = slab_desc(base + OFF_V, kk);
+          if (delta) {
+            mma_bf16_ss(tmem_d, a_hi, b_v, id256, acc);  // [dM | G] += hi^T [V | GH]
+          } else {
+            mma_bf16_ss(tmem_d, a_hi, b_v, id128, acc);  // dM += hi^T V
+          }
+          mma_bf16_ss(tmem_d, a_lo, b_v, id128, 1u);     // dM += lo^T V
+        }
+        mma_commit(&bar_mma[stg]);
+        // refill the stage used by slab sl - 1 once its MMAs are done
+        if (sl >= 1 && issued < nslab) {
+          const int prev = sl - 1;
+          if (!mbar_wait(&bar_mma[prev % kStages], (uint32_t)((prev / kStages) & 1))) {
+            ok = false;
+            break;
+          }
+          load(issued++);
+        }
       }
+      mma_commit(bar_done);
+    } else if (lane == 0) {
+      mma_commit(bar_done);  // nothing issued: completes at once
     }
-  };
-  load_slab(0);
-
-  const uint32_t idesc = idesc_f32acc(2, 1, 1, 128, ncols);
-  for (int sl = 0; sl < nslab; ++sl) {
-    const int st = sl % kStages;
-    uint8_t* sA = smem + st * kStageBytes;
-    uint8_t* sB = sA + kABytes;
-    if (sl >= kStages) {
-      if (!mbar_wait(&bar_mma[st], (uint32_t)((sl / kStages - 1) & 1))) ok = false;
-    }
-    uint4 kc[2] = {kr[0], kr[1]}, vc[2] = {vr[0], vr[1]};
-    if (sl + 1 < nslab) load_slab(sl + 1);  // prefetch the next slab into registers
-    if (ok) {
+  } else {
+    // ---------------- converters (warps 0..7) ----------------
+    for (int sl = 0; sl < nslab && ok; ++sl) {
+      const int stg = sl % kStages;
+      uint8_t* st = smem + stg * kStageBytes;
+      if (!mbar_wait(&bar_full[stg], (uint32_t)((sl / kStages) & 1))) {
+        ok = false;
+        break;
+      }
 #pragma unroll
-      for (int it = 0; it < 2; ++it) {
+      for (int it = 0; it < 4; ++it) {
         const int item = tid + 256 * it;
-        const int r = item >> 4, cg = item & 15;
+        const int r = item >> 4, cg = item & 15;  // token row in the slab, 8-feature group
         const bool valid = sl * kSlab + r < len;
-        float f[8], g[8];
-        bf16x8_to_f32(kc[it], f);
-        bf16x8_to_f32(vc[it], g);
+        const uint32_t off = (uint32_t)(cg >> 3) * kBox + sw128(r, cg & 7);
+        const uint4 raw = *reinterpret_cast<const uint4*>(st + OFF_KH + off);
+        float f[8];
+        bf16x8_to_f32(raw, f);
         float den = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           f[e] = valid ? elu1(f[e]) : 0.f;
           den = fmaf(f[e], sZ[cg * 8 + e], den);
         }
-        // row sum over the 16 lanes of this half-warp (same token)
+        // 16 lanes of a half-warp hold the 128 features of one token
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        uint32_t hi[4], lo[4], gh[4];
         const float inv = (delta && den != 0.f) ? 1.f / den : 0.f;
-        const uint32_t chunk_off = (uint32_t)(cg >> 2) * kAChunkBytes;
-        const uint32_t u0 = (uint32_t)(cg & 3) * 2;
-        uint4 a0, a1, b0, b1;
-        a0 = make_uint4(tf32_round(f[0]), tf32_round(f[1]), tf32_round(f[2]), tf32_round(f[3]));
-        a1 = make_uint4(tf32_round(f[4]), tf32_round(f[5]), tf32_round(f[6]), tf32_round(f[7]));
-        b0 = make_uint4(__float_as_uint(g[0]), __float_as_uint(g[1]), __float_as_uint(g[2]),
-                        __float_as_uint(g[3]));
-        b1 = make_uint4(__float_as_uint(g[4]), __float_as_uint(g[5]), __float_as_uint(g[6]),
-                        __float_as_uint(g[7]));
-        *reinterpret_cast<uint4*>(sA + chunk_off + sw128(r, u0)) = a0;
-        *reinterpret_cast<uint4*>(sA + chunk_off + sw128(r, u0 + 1)) = a1;
-        *reinterpret_cast<uint4*>(sB + chunk_off + sw128(r, u0)) = b0;
-        *reinterpret_cast<uint4*>(sB + chunk_off + sw128(r, u0 + 1)) = b1;
-        if (delta) {
-          uint4 h0 = make_uint4(tf32_round(f[0] * inv), tf32_round(f[1] * inv),
-                                tf32_round(f[2] * inv), tf32_round(f[3] * inv));
-          uint4 h1 = make_uint4(tf32_round(f[4] * inv), tf32_round(f[5] * inv),
-                                tf32_round(f[6] * inv), tf32_round(f[7] * inv));
-          *reinterpret_cast<uint4*>(sB + 4 * kAChunkBytes + chunk_off + sw128(r, u0)) = h0;
-          *reinterpret_cast<uint4*>(sB + 4 * kAChunkBytes + chunk_off + sw128(r, u0 + 1)) = h1;
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0 && ok) {
-      tc_fence_after();
-      const uint32_t a_addr = smem_u32(sA), b_addr = smem_u32(sB);
 #pragma unroll
-      for (int kk = 0; kk < kSlab / 8; ++kk) {
-        const uint64_t ad = sdesc(a_addr + kk * 1024, kAChunkBytes, 1024);
-        const uint64_t bd = sdesc(b_addr + kk * 1024, kAChunkBytes, 1024);
-        mma_tf32_ss(tmem_d, ad, bd, idesc, (sl > 0 || kk > 0) ? 1u : 0u);
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+          const float2 hf = __bfloat1622float2(h);
+          const __nv_bfloat162 l = __floats2bfloat162_rn(f[2 * e] - hf.x, f[2 * e + 1] - hf.y);
+          const __nv_bfloat162 g = __floats2bfloat162_rn(f[2 * e] * inv, f[2 * e + 1] * inv);
+          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+          lo[e] = *reinterpret_cast<const uint32_t*>(&l);
+          gh[e] = *reinterpret_cast<const uint32_t*>(&g);
+        }
+        *reinterpret_cast<uint4*>(st + OFF_KH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(st + OFF_KL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        if (delta)
+          *reinterpret_cast<uint4*>(st + OFF_GH + off) = make_uint4(gh[0], gh[1], gh[2], gh[3]);
       }
-      mma_commit(&bar_mma[st]);
+      fence_proxy_async_smem();
+      mbar_arrive(&bar_conv[stg]);
     }
   }
-  if (tid == 0) mma_commit(bar_done);  // tracks every MMA issued above
+
   const bool done = mbar_wait(bar_done, 0);
   tc_fence_after();
-
   // epilogue: warps 0-3 write dM rows, warps 4-7 write G rows (Delta)
-  const int lane_base = (warp & 3) * 32;
-  const int row = lane_base + (tid & 31);
-  const int half = warp >> 2;
-  if (done && ok && (half == 0 || delta)) {
-    float* dst = dpart + ((size_t)idx * 2 + half) * D * D + (size_t)row * D;
+  if (warp < 8) {
+    const int lane_base = (warp & 3) * 32;
+    const int row = lane_base + lane;
+    const int half = warp >> 2;
+    if (half == 0 || delta) {
+      float* dst = dpart + ((size_t)idx * 2 + half) * D * D + (size_t)row * D;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t r[32];
-      tmem_ld32(tmem_d + ((uint32_t)lane_base << 16) + half * 128 + cc * 32, r);
-      tmem_wait_ld();
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t rr[32];
+        if (nslab > 0) {
+          tmem_ld32(tmem_d + ((uint32_t)lane_base << 16) + half * 128 + cc * 32, rr);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(dst + cc * 32 + e) =
-            make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                        __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+          for (int e = 0; e < 32; ++e) rr[e] = 0u;
+        }
+        if (done && ok) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + cc * 32 + e) =
+                make_float4(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1]),
+                            __uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3]));
+        }
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem_d, ncols);
   }
@@ -437,8 +477,11 @@ cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, co
   const unsigned nunits = (unsigned)((long long)BH * S * CH);
   zpart_kernel<<<nunits, 256, 0, stream>>>(k, ws.zpart, L, N, S, CH, CL);
   zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH);
-  state_kernel<<<nunits, 256, kStateSmem, stream>>>(k, v, ws.zprev, ws.dpart, L, N, S, CH, CL,
-                                                     mode);
+  CUtensorMap mk, mv;
+  if (!make_bf16_map(&mk, k, (uint64_t)L, BH, kSlab) || !make_bf16_map(&mv, v, (uint64_t)L, BH, kSlab))
+    return cudaErrorInvalidValue;
+  state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(mk, mv, ws.zprev, ws.dpart, L, N, S,
+                                                               CH, CL, mode);
   chain_kernel<<<dim3(BH, 4), 256, mode == 1 ? kChainSmem : 0, stream>>>(ws.dpart, M_in, M_out,
                                                                         ws.Mhl, S, CH, mode);
   return cudaGetLastError();

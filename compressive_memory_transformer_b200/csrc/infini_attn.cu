@@ -83,7 +83,8 @@ int check_common(const void* q, const void* k, const void* v, const float* beta,
                  const float* M_in, const float* z_in, const void* out, const float* M_out,
                  const float* z_out, int B, int H, long long L, int N, int d, int mode,
                  size_t esize) {
-  if (!q || !k || !v || !beta || !out) return INFINI_ERR_NULL;
+  if (!beta) return INFINI_ERR_NULL;
+  if (L > 0 && (!q || !k || !v || !out)) return INFINI_ERR_NULL;
   if ((M_in == nullptr) != (z_in == nullptr)) return INFINI_ERR_NULL;
   if ((M_out == nullptr) != (z_out == nullptr)) return INFINI_ERR_NULL;
   if (B < 1 || H < 1 || N < 1 || L < 0 || d < 1) return INFINI_ERR_SHAPE;
