@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the Infini-attention forward on B200.
+
+Workload: the 1B-LM layer shape, B=4, H=8, d=128, segment N=2048, L=32768
+(16 segments), bf16 q/k/v i.i.d. N(0,1), beta ~ N(0,1) per head, fp32 state
+from zero. One step is one pass of the whole forward path in both memory-update
+modes over the same batch: infini_attn_forward in Linear mode, then in
+Linear+Delta mode (each = sigma(K) sums, z scan, per-segment state GEMMs, state
+chain, fused attention + retrieval + gate). Tokens per step = 2 * B * L.
+
+Prints one JSON line (rank 0). Under torchrun (N > 1) every rank runs its own
+batch (the path shards by (batch, head) with no exchange: weak scaling), the
+ranks meet at barriers around the timed region, and the time is the max over
+ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (bounded
+samples of the same workload) and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "Infini-attn fwd tokens/s on 1 B200 (N=2048,d=128); % bf16 tensor peak"
+UNIT = "tokens/s"
+B, H, D, N, L = 4, 8, 128, 2048, 32768
+WORKLOAD = (f"1B-LM layer shape: B={B}, H={H}, d={D}, N={N}, L={L} ({L // N} segments), "
+            "bf16 q/k/v, fp32 state from zero; step = Linear forward + Linear+Delta forward")
+LAUNCHES_PER_FORWARD = 5   # zpart, zscan, state, chain, attn
+
+
+def attn_flops_per_launch():
+    """Algorithmic FLOPs of the fused attention + retrieval kernel for one forward:
+    per token-head 2d(N+1) for the causal QK^T and PV pairs plus 2d^2 for sigma(Q)M."""
+    return B * H * L * (2 * D * (N + 1) + 2 * D * D)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return j["bf16_tflops"], j.get("bf16_tflops_sustained", j["bf16_tflops"]), j["hbm_gbs"], "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def measured_traffic(kernel_src, record):
+    """dram read + write bytes per launch from the committed ncu capture, or None
+    when the kernel source has changed since the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", record)
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    with open(os.path.join(ROOT, kernel_src), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if sha != rec.get("source_sha256"):
+        return None
+    return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+
+
+def usable_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.sel = str(device)
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[3][1:5])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows),
+                "samples": len(load), "reasons": reasons}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reported baseline; the oracle is timed as it stands)
+# ---------------------------------------------------------------------------
+def oracle_sample(q, k, v, beta, heads, modes):
+    """Run the fp64 oracle on the given heads (full length) and modes; returns
+    (seconds, token-heads processed)."""
+    import oracle
+    t0 = time.perf_counter()
+    th = 0
+    for (b, h) in heads:
+        qh = q[b, h].to(torch.float64).numpy()
+        kh = k[b, h].to(torch.float64).numpy()
+        vh = v[b, h].to(torch.float64).numpy()
+        g = oracle.gate_value(float(beta[h]))
+        for mode in modes:
+            oracle.head_forward(qh, kh, vh, g, N, mode)
+            th += qh.shape[0]
+    return time.perf_counter() - t0, th
+
+
+def cpu_baseline(inp_cpu):
+    heads = [(0, 0), (1, 3), (2, 5), (3, 7)]
+    secs, th = oracle_sample(inp_cpu["q"], inp_cpu["k"], inp_cpu["v"], inp_cpu["beta"], heads,
+                             (0, 1))
+    return {"value": (th / H) / secs, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{len(heads)} of {B * H} heads (full L={L}) x Linear and Linear+Delta, "
+                      f"fp64 numpy oracle, {secs:.1f} s; tokens = token-heads / H"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, device):
+    import compressive_memory_transformer_b200 as ia
+    from synthetic_inputs import make_inputs
+
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream()
+    inp = make_inputs(B, H, L, D, torch.bfloat16, seed=rank, device=device, gen_device=device)
+    q, k, v, beta = inp["q"], inp["k"], inp["v"], inp["beta"]
+    outs = {m: (torch.empty_like(q), torch.empty((B, H, D, D), device=device),
+                torch.empty((B, H, D), device=device)) for m in (ia.LINEAR, ia.DELTA)}
+    ws = torch.empty(ia.workspace_size(B, H, L, N, D, ia.DELTA), dtype=torch.uint8, device=device)
+
+    def forward(mode, evs=None):
+        o, M, z = outs[mode]
+        ia.infini_attn_forward_ex(q, k, v, beta, N, mode, out=o, M_out=M, z_out=z,
+                                  workspace=ws, stage_events=evs)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        forward(ia.LINEAR)
+        forward(ia.DELTA)
+    torch.cuda.synchronize()
+    assert ia.device_status() == 0
+
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(2)]
+          for _ in range(args.steps)]
+    # torch creates the CUDA event on its first record; the library then re-records
+    # the same handles around its launches inside the timed region
+    for e in (e for step in ev for mode in step for e in mode):
+        e.record(stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(device)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        forward(ia.LINEAR, ev[i][0])
+        forward(ia.DELTA, ev[i][1])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    assert ia.device_status() == 0, "a bounded device wait ran out during the timed region"
+
+    attn_ms = [ev[i][m][1].elapsed_time(ev[i][m][2]) for i in range(args.steps) for m in (0, 1)]
+    state_ms = {m: statistics.mean(ev[i][m][0].elapsed_time(ev[i][m][1])
+                                   for i in range(args.steps)) for m in (0, 1)}
+    fwd_ms = {m: statistics.mean(ev[i][m][0].elapsed_time(ev[i][m][2])
+                                 for i in range(args.steps)) for m in (0, 1)}
+
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # ---- end to end through the public call with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+        oh = {m: torch.empty(q.shape, dtype=q.dtype).pin_memory() for m in (0, 1)}
+        Mh = {m: torch.empty((B, H, D, D)).pin_memory() for m in (0, 1)}
+        zh = {m: torch.empty((B, H, D)).pin_memory() for m in (0, 1)}
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            for m in (ia.LINEAR, ia.DELTA):
+                o, M, z = ia.infini_attn_forward(qd, kd, vd, beta, N, m, out=outs[m][0],
+                                                 M_out=outs[m][1], z_out=outs[m][2])
+                oh[m].copy_(o, non_blocking=True)
+                Mh[m].copy_(M, non_blocking=True)
+                zh[m].copy_(z, non_blocking=True)
+
+        e_steps = max(3, args.steps // 4)
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        te = torch.tensor([a.elapsed_time(b_)], device=device, dtype=torch.float64)
+        if world > 1:
+            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+        h2d = 3 * q.numel() * q.element_size()
+        d2h = 2 * (q.numel() * q.element_size() + B * H * (D * D + D) * 4)
+        e2e = {"value": world * e_steps * 2 * B * L / (float(te.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
+               "ms_per_step": float(te.item()) / e_steps}
+        assert ia.device_status() == 0
+
+    if rank != 0:
+        return None
+    peak_burst, peak_sust, hbm, peak_src = load_peaks()
+    avg_attn_s = statistics.mean(attn_ms) / 1e3
+    achieved = attn_flops_per_launch() / avg_attn_s / 1e12
+    tokens = world * args.steps * 2 * B * L
+    line = {
+        "metric": METRIC, "value": tokens / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/k/v, N(0,1) beta)",
+        "config": {"workload": WORKLOAD, "B": B, "H": H, "d": D, "N": N, "L": L,
+                   "modes": ["linear", "delta"], "per_rank_batch": B,
+                   "l2": "inputs larger than L2 (q/k/v 768 MiB per forward), no flush"},
+        "roofline": {"kernel": "attn_kernel (fused local attention + retrieval + gate)",
+                     "bound": "tensor", "achieved": achieved, "peak": peak_sust,
+                     "unit": "TFLOP/s", "frac": achieved / peak_sust,
+                     "traffic": measured_traffic(
+                         "compressive_memory_transformer_b200/csrc/bf16_attn.cu",
+                         "attn_kernel_c2_traffic.json"),
+                     "peak_kind": f"bf16 dense, sustained, {peak_src}",
+                     "frac_of_burst_peak": achieved / peak_burst,
+                     "flops_per_launch": attn_flops_per_launch(),
+                     "avg_launch_ms": avg_attn_s * 1e3},
+        "modes": {
+            "linear": {"tokens_per_s": B * L / (fwd_ms[0] / 1e3), "forward_ms": fwd_ms[0],
+                       "state_kernels_ms": state_ms[0]},
+            "delta": {"tokens_per_s": B * L / (fwd_ms[1] / 1e3), "forward_ms": fwd_ms[1],
+                      "state_kernels_ms": state_ms[1]},
+        },
+        "gpu_launches": args.steps * 2 * LAUNCHES_PER_FORWARD,
+        "clocks": clk,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline({"q": q.cpu(), "k": k.cpu(), "v": v.cpu(),
+                                             "beta": beta.cpu()})
+    return line
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    from synthetic_inputs import make_inputs
+    import oracle
+    inp = make_inputs(B, H, L, D, torch.bfloat16, seed=0, device="cpu")
+    # one step = one head of the workload, full length, Linear and Linear+Delta; the
+    # number of segments per step is cut so that the whole run stays within ~3 min
+    q, k, v, beta = inp["q"], inp["k"], inp["v"], inp["beta"]
+    t_cal, _ = oracle_sample(q[:, :, :N], k[:, :, :N], v[:, :, :N], beta, [(0, 0)], (0, 1))
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    segs = int(max(1, min(L // N, budget // max(t_cal, 1e-3))))
+    Ls = segs * N
+    heads = [(b, h) for b in range(B) for h in range(H)]
+    for i in range(args.warmup):
+        b, h = heads[i % len(heads)]
+        oracle_sample(q[:, :, :Ls], k[:, :, :Ls], v[:, :, :Ls], beta, [(b, h)], (0, 1))
+    tot_s, tot_th = 0.0, 0
+    for i in range(args.steps):
+        b, h = heads[i % len(heads)]
+        s_, th = oracle_sample(q[:, :, :Ls], k[:, :, :Ls], v[:, :, :Ls], beta, [(b, h)], (0, 1))
+        tot_s += s_
+        tot_th += th
+    value = (tot_th / H) / tot_s
+    sample = (f"per step one head of {B * H}, first {segs} of {L // N} segments, Linear and "
+              f"Linear+Delta, fp64 numpy oracle; tokens = token-heads / H")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_s / max(1, args.steps) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "H": H, "d": D, "N": N, "L": L,
+                   "modes": ["linear", "delta"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    try:
+        line = run_ours(args, rank, world, device)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
