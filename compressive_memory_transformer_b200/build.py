@@ -1,6 +1,8 @@
 """Build libinfini_attn.so in-tree with nvcc for sm_100a.
 
-Usage: python -m compressive_memory_transformer_b200.build [-v] [--ptxas-info]
+Usage: python compressive_memory_transformer_b200/build.py [-v] [--ptxas-info] [--force]
+
+This file imports nothing from the package (whose __init__ needs the built library).
 """
 from __future__ import annotations
 

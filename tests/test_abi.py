@@ -11,8 +11,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def lib():
-    from compressive_memory_transformer_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._build_module().build()
     import compressive_memory_transformer_b200 as m
     return m
 
