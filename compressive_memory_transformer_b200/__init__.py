@@ -45,6 +45,7 @@ class Opts(ctypes.Structure):
 _SIGS = {
     "infini_attn_forward": [_vp] * 9 + [_i, _i, _ll, _i, _i, _i, _vp],
     "infini_attn_step": [_vp] * 9 + [_i, _i, _i, _i, _i, _vp],
+    "infini_attn_step_static": [_vp] * 9 + [_i, _i, _i, _i, _i, _vp],
     "infini_attn_forward_f32": [_vp] * 9 + [_i, _i, _ll, _i, _i, _i, _vp],
     "infini_attn_step_f32": [_vp] * 9 + [_i, _i, _i, _i, _i, _vp],
     "infini_attn_forward_ex": [_vp] * 9 + [_i, _i, _ll, _i, _i, _i, _i, ctypes.POINTER(Opts), _vp],

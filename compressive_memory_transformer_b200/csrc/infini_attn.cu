@@ -286,6 +286,7 @@ const char* infini_attn_strerror(int status) {
     case INFINI_ERR_NOMEM: return "scratch memory could not be obtained";
     case INFINI_ERR_TIMEOUT: return "a bounded device wait ran out";
     case INFINI_ERR_ALIAS: return "out overlaps an input or the state";
+    case INFINI_ERR_SCRATCH_LIMIT: return "sizes need more scratch than the fixed static array holds";
     default: return "unknown status";
   }
 }

@@ -66,7 +66,8 @@ typedef enum {
   INFINI_ERR_CUDA = -5,        /* a CUDA runtime call or a launch failed */
   INFINI_ERR_NOMEM = -6,       /* the stream-ordered scratch allocation failed */
   INFINI_ERR_TIMEOUT = -7,     /* a bounded device wait ran out (infini_attn_device_status) */
-  INFINI_ERR_ALIAS = -8        /* out overlaps an input or the state */
+  INFINI_ERR_ALIAS = -8,       /* out overlaps an input or the state */
+  INFINI_ERR_SCRATCH_LIMIT = -9 /* infini_attn_step_static: sizes need more than its fixed scratch */
 } infini_status_t;
 
 /*
@@ -91,7 +92,27 @@ int infini_attn_step(const void* q, const void* k, const void* v, const float* b
                      const float* M_in, const float* z_in, void* out, float* M_out,
                      float* z_out, int B, int H, int N, int d, int mode, void* stream);
 
-/* fp32 q/k/v/out variants of the two calls above; 1 <= d <= 128. */
+/*
+ * infini_attn_step without any device-memory allocation. The paper has no
+ * counterpart to this call; it exists for callers that must not allocate on
+ * their hot path: a serving loop that reserved its whole memory budget at
+ * start-up, or a framework whose own allocator owns all device memory (an
+ * allocation made behind its back sits outside its accounting and can fail or
+ * fragment). Arguments, layouts and results are those of infini_attn_step
+ * (bf16, d == 128); the caller still passes every input and output.
+ * Scratch: one fixed 8 MiB array per device, reserved for the life of the
+ * process on every GPU that loads the library. Sizes whose scratch does not fit
+ * (roughly B*H above 40 heads for one segment) return INFINI_ERR_SCRATCH_LIMIT
+ * before any launch. The first call on a device looks up the array's address
+ * for that device; make that first call before any stream capture begins. All
+ * calls on a device share the array: calls whose GPU work may overlap in time
+ * race on it, so order them on one stream or synchronise between them.
+ */
+int infini_attn_step_static(const void* q, const void* k, const void* v, const float* beta,
+                            const float* M_in, const float* z_in, void* out, float* M_out,
+                            float* z_out, int B, int H, int N, int d, int mode, void* stream);
+
+/* fp32 q/k/v/out variants of infini_attn_forward and infini_attn_step; 1 <= d <= 128. */
 int infini_attn_forward_f32(const float* q, const float* k, const float* v, const float* beta,
                             const float* M_in, const float* z_in, float* out, float* M_out,
                             float* z_out, int B, int H, long long L, int N, int d, int mode,
