@@ -366,6 +366,134 @@ def run_reference(args):
     }
 
 
+# ---------------------------------------------------------------------------
+# the other workloads of the configuration list (extra lines, not the headline)
+# ---------------------------------------------------------------------------
+def _timed(fn, reps, stream):
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b_.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b_) / reps
+
+
+def run_extra(args, device):
+    """C3: 1M-token stream through 512 infini_attn_step calls (graph-captured),
+    C4: 8B 500K single forward, C5: segment-length sweep. One JSON line each."""
+    import compressive_memory_transformer_b200 as ia
+    from synthetic_inputs import make_inputs
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream()
+    peak_burst, peak_sust, _, src = load_peaks()
+    lines = []
+    which = args.config
+
+    def attn_tflops(Bc, Hc, Lc, Nc, ms):
+        return Bc * Hc * Lc * (2 * D * (Nc + 1) + 2 * D * D) / (ms / 1e3) / 1e12
+
+    if which in ("c5", "all"):
+        Bc, Hc, Lc = 8, 16, 65536
+        inp = make_inputs(Bc, Hc, Lc, D, torch.bfloat16, seed=0, device=device, gen_device=device)
+        res = []
+        for Nc in (512, 1024, 2048, 4096):
+            for mode in (ia.LINEAR, ia.DELTA):
+                ws = torch.empty(ia.workspace_size(Bc, Hc, Lc, Nc, D, mode), dtype=torch.uint8,
+                                 device=device)
+                out = torch.empty_like(inp["q"])
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                for e in ev:
+                    e.record(stream)
+
+                def f():
+                    ia.infini_attn_forward_ex(inp["q"], inp["k"], inp["v"], inp["beta"], Nc, mode,
+                                              out=out, workspace=ws, stage_events=ev)
+                for _ in range(3):
+                    f()
+                torch.cuda.synchronize()
+                tot = st = at = 0.0
+                reps = max(3, args.steps // 3)
+                for _ in range(reps):
+                    f()
+                    torch.cuda.synchronize()
+                    tot += ev[0].elapsed_time(ev[2])
+                    st += ev[0].elapsed_time(ev[1])
+                    at += ev[1].elapsed_time(ev[2])
+                tot, st, at = tot / reps, st / reps, at / reps
+                res.append({"N": Nc, "mode": "delta" if mode else "linear",
+                            "tokens_per_s": Bc * Lc / (tot / 1e3), "forward_ms": tot,
+                            "state_ms": st, "attn_ms": at,
+                            "attn_tflops": attn_tflops(Bc, Hc, Lc, Nc, at),
+                            "attn_frac_sustained": attn_tflops(Bc, Hc, Lc, Nc, at) / peak_sust,
+                            "attn_hbm_gbs": Bc * Hc * Lc * 1024 / (at / 1e3) / 1e9})
+        assert ia.device_status() == 0
+        lines.append({"config": "C5 segment-length sweep: B=8, H=16, d=128, L=65536, bf16",
+                      "peak": f"{peak_sust} TFLOP/s sustained ({src})", "results": res})
+        del inp
+        torch.cuda.empty_cache()
+
+    if which in ("c4", "all"):
+        Bc, Hc, Lc, Nc = 1, 32, 524288, 2048
+        inp = make_inputs(Bc, Hc, Lc, D, torch.bfloat16, seed=0, device=device, gen_device=device)
+        out = torch.empty_like(inp["q"])
+        ws = torch.empty(ia.workspace_size(Bc, Hc, Lc, Nc, D, ia.DELTA), dtype=torch.uint8,
+                         device=device)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        for e in ev:
+            e.record(stream)
+
+        def f4():
+            ia.infini_attn_forward_ex(inp["q"], inp["k"], inp["v"], inp["beta"], Nc, ia.DELTA,
+                                      out=out, workspace=ws, stage_events=ev)
+        f4()
+        torch.cuda.synchronize()
+        ms = _timed(f4, 3, stream)
+        at = ev[1].elapsed_time(ev[2])
+        assert ia.device_status() == 0
+        lines.append({"config": "C4 8B-model 500K stream: B=1, H=32, d=128, N=2048, L=524288, "
+                                "Linear+Delta, one forward",
+                      "tokens_per_s": Bc * Lc / (ms / 1e3), "forward_ms": ms,
+                      "state_ms": ev[0].elapsed_time(ev[1]), "attn_ms": at,
+                      "attn_tflops": attn_tflops(Bc, Hc, Lc, Nc, at),
+                      "attn_frac_sustained": attn_tflops(Bc, Hc, Lc, Nc, at) / peak_sust})
+        del inp, out, ws
+        torch.cuda.empty_cache()
+
+    if which in ("c3", "all"):
+        Bc, Hc, Nc, S = 1, 8, 2048, 512
+        # the stream arrives segment by segment: [S][B, H, N, d], each segment contiguous
+        seg = [make_inputs(Bc, Hc, Nc, D, torch.bfloat16, seed=1000 + i, device=device,
+                           gen_device=device) for i in range(S)]
+        beta = seg[0]["beta"]
+        M = torch.zeros((Bc, Hc, D, D), device=device)
+        z = torch.zeros((Bc, Hc, D), device=device)
+        outs = [torch.empty_like(seg[0]["q"]) for _ in range(S)]
+
+        def run_stream():
+            for i in range(S):
+                ia.infini_attn_step(seg[i]["q"], seg[i]["k"], seg[i]["v"], beta, ia.DELTA, M, z,
+                                    out=outs[i], M_out=M, z_out=z)
+        run_stream()
+        torch.cuda.synchronize()
+        plain_ms = _timed(run_stream, 2, stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run_stream()
+        g.replay()
+        torch.cuda.synchronize()
+        graph_ms = _timed(g.replay, 3, stream)
+        del g
+        assert ia.device_status() == 0
+        lines.append({"config": "C3 1M-token stream: B=1, H=8, d=128, N=2048, L=1048576 via 512 "
+                                "infini_attn_step calls, Linear+Delta, state carried in place",
+                      "tokens_per_s_graph": Bc * S * Nc / (graph_ms / 1e3),
+                      "stream_ms_graph": graph_ms, "us_per_step_graph": graph_ms * 1e3 / S,
+                      "tokens_per_s_plain": Bc * S * Nc / (plain_ms / 1e3),
+                      "stream_ms_plain": plain_ms})
+    return lines
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -374,6 +502,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", choices=["c2", "c3", "c4", "c5", "all"], default="c2",
+                    help="c2 (default) prints the headline line; the others print one extra "
+                         "line per workload of the configuration list")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -392,6 +523,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
+    if args.config != "c2":
+        for ln in run_extra(args, device):
+            print(json.dumps(ln), flush=True)
+        return
     try:
         line = run_ours(args, rank, world, device)
         if rank == 0:

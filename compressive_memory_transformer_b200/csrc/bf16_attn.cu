@@ -8,11 +8,18 @@
 // llm-papers-study.pages.dev: sections 3.1, 3.3, 3.5). A_dot and A_mem stay in
 // tensor memory; only `out` is written to HBM.
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0     TMA producer: Q tile, then the V pipeline items [M_hi, M_lo, V_0, V_1, ...]
 //              and the K pipeline items [K_0, K_1, ...], two stages each.
 //   warp 1     tensor-memory allocation and the single MMA-issuing thread.
-//   warps 2-5  softmax / epilogue: thread r owns query row r (tensor-memory lane r).
+//   warps 2-9  softmax / epilogue, two warpgroups: query row r (tensor-memory lane r)
+//              is shared by one thread of each; warpgroup h owns key columns
+//              [64h, 64h + 64) of S and value columns [64h, 64h + 64) of O, R and out.
+//              The two threads of a row exchange their partial row max every tile
+//              (and row sum / denominator at the end) through shared memory,
+//              synchronised by an mbarrier per warp pair.
+// Grid order: the query tiles of one segment are consecutive (heaviest first), so
+// the segment's K/V tiles are reused from L2 while they are in flight.
 // Tensor memory (512 columns): S0 | S1 (double-buffered scores) | O (A_dot
 // accumulator) | R (sigma(Q) M accumulator).
 // MMA order: QK_0, QK_1, R = sigma(Q)(M_hi + M_lo), then for each j: O += P_j V_j,
@@ -42,13 +49,15 @@ constexpr int OFF_K = kTile;         // 2 stages
 constexpr int OFF_V = 3 * kTile;     // 2 stages
 constexpr int OFF_P = 5 * kTile;
 constexpr int OFF_Z = 6 * kTile;     // 128 floats
-constexpr int OFF_BAR = OFF_Z + 512;
+constexpr int OFF_X = OFF_Z + 512;   // exchange: max [2 slots][2 halves][128], den, l [2][128]
+constexpr int OFF_BAR = OFF_X + 4096;
 constexpr int kAttnSmem = OFF_BAR + 256 + 1024;  // + alignment slack
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = 256;
 
 enum {
   B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9,
-  B_PFULL = 11, B_PVDONE = 12, B_DRAIN = 13, B_COUNT = 14
+  B_PFULL = 11, B_PVDONE = 12, B_DRAIN = 13, B_PAIR = 14 /* 4 */, B_GROUP = 18, B_COUNT = 19
 };
 
 // Bounded wait used only while draining after an error: ignores the error flag.
@@ -77,13 +86,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const __grid_constant__ CUtensorMap tm_m, const float* __restrict__ beta,
             const float* __restrict__ zprev, __nv_bfloat16* __restrict__ out, long long L, int N,
             int S, int H, int T, int BH) {
-  // ---- work item: heaviest query tiles first ----
+  // ---- work item: segment-major, heaviest query tile of the segment first ----
   const long long x = blockIdx.x;
-  const long long per = (long long)S * BH;
-  const int i = T - 1 - (int)(x / per);
-  const long long rem = x % per;
-  const int s = (int)(rem % S);
-  const int bh = (int)(rem / S);
+  const long long seg = x / T;
+  const int i = T - 1 - (int)(x % T);
+  const int s = (int)(seg % S);
+  const int bh = (int)(seg / S);
   const long long seg0 = (long long)s * N;
   const int n_s = (int)min((long long)N, L - seg0);
   const int T_s = (n_s + BM - 1) / BM;
@@ -101,12 +109,18 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   uint8_t* sV = smem + OFF_V;
   uint8_t* sP = smem + OFF_P;
   float* sZ = reinterpret_cast<float*>(smem + OFF_Z);
+  float* sX = reinterpret_cast<float*>(smem + OFF_X);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int b = 0; b < B_COUNT; ++b) mbar_init(&bars[b], b == B_PFULL ? 128u : 1u);
+    for (int b = 0; b < B_COUNT; ++b) {
+      uint32_t cnt = 1;
+      if (b == B_PFULL || b == B_GROUP) cnt = kSoftmaxThreads;
+      if (b >= B_PAIR && b < B_PAIR + 4) cnt = 64;
+      mbar_init(&bars[b], cnt);
+    }
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -118,6 +132,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + D) sZ[threadIdx.x - 64] = zprev[((size_t)bh * S + s) * D + threadIdx.x - 64];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -224,22 +239,28 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       drain_wait(&bars[B_DRAIN], 0);
     }
   } else {
-    // ================= softmax / epilogue (warps 2..5) =================
+    // ================= softmax / epilogue (warps 2..9) =================
     const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // query row inside the tile == tensor-memory lane
+    const int half = (warp - 2) >> 2;  // key / value columns [64 half, 64 half + 64)
+    const int r = wq * 32 + lane;      // query row inside the tile == tensor-memory lane
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t col0 = (uint32_t)half * 64;
+    uint64_t* pair = &bars[B_PAIR + wq];  // the two warps that share these rows
+    uint32_t pair_phase = 0;
+    float* xmax = sX;            // [2 slots][2 halves][128]
+    float* xden = sX + 512;      // [2 halves][128]
+    float* xl = sX + 768;        // [2 halves][128]
     const float bta = beta[bh % H];
     const float g = 1.f / (1.f + expf(-bta));
-    sZ[r] = zprev[((size_t)bh * S + s) * D + r];
-    named_bar_sync(1, 128);
 
     bool ok = mbar_wait(&bars[B_QFULL], 0);
     float den = 0.f;
     if (ok) {
-      // sigma(Q) row -> P buffer (same swizzled position), den = sigma(Q_r) . z_{s-1}
+      // sigma(Q) of this thread's 64 columns -> P buffer (same swizzled position);
+      // partial denominator sigma(Q_r) . z_{s-1} over those columns
 #pragma unroll 4
-      for (int u = 0; u < 16; ++u) {
-        const uint32_t off = (uint32_t)(u >> 3) * kSub + sw128(r, u & 7);
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t off = (uint32_t)half * kSub + sw128(r, u);
         const uint4 raw = *reinterpret_cast<const uint4*>(sQ + off);
         const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
         uint32_t pk[4];
@@ -247,8 +268,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int e = 0; e < 4; ++e) {
           const float2 f = __bfloat1622float2(h[e]);
           const float p0 = elu1(f.x), p1 = elu1(f.y);
-          den = fmaf(p0, sZ[u * 8 + 2 * e], den);
-          den = fmaf(p1, sZ[u * 8 + 2 * e + 1], den);
+          den = fmaf(p0, sZ[col0 + u * 8 + 2 * e], den);
+          den = fmaf(p1, sZ[col0 + u * 8 + 2 * e + 1], den);
           pk[e] = pack_bf16x2(p0, p1);
         }
         *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -266,22 +287,32 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         break;
       }
       tc_fence_after();
-      uint32_t sr[BN];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(tS + lane_off + b * BN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+      uint32_t sr[64];
+      tmem_ld32(tS + lane_off + b * BN + col0, *reinterpret_cast<uint32_t(*)[32]>(sr));
+      tmem_ld32(tS + lane_off + b * BN + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
       tmem_wait_ld();
-      float mt = -INFINITY;
       if (j == i) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          if (c > r) sr[c] = __float_as_uint(-INFINITY);
-          mt = fmaxf(mt, __uint_as_float(sr[c]));
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < BN; ++c) mt = fmaxf(mt, __uint_as_float(sr[c]));
+        for (int c = 0; c < 64; ++c)
+          if ((int)col0 + c > r) sr[c] = __float_as_uint(-INFINITY);
       }
+      float mx[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        mx[t] = __uint_as_float(sr[t]);
+#pragma unroll
+        for (int c = 1; c < 8; ++c) mx[t] = fmaxf(mx[t], __uint_as_float(sr[8 * c + t]));
+      }
+      const float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      xmax[b * 256 + half * 128 + r] = mh;
+      mbar_arrive(pair);
+      if (!mbar_wait(pair, pair_phase & 1)) {
+        ok = false;
+        break;
+      }
+      ++pair_phase;
+      const float mt = fmaxf(mh, xmax[b * 256 + (1 - half) * 128 + r]);
       bool need = false;
       float alpha = 1.f;
       if (j == 0) {
@@ -292,15 +323,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         m_use = mt;
       }
       const float mb = m_use * sl;
-      float rs = 0.f;
-      uint32_t pk[BN / 2];
+      float rsum[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < BN / 2; ++c) {
+      for (int c = 0; c < 32; ++c) {
         const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), sl, -mb));
         const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), sl, -mb));
-        rs += p0 + p1;
+        rsum[c & 3] += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
       }
+      const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
       // PV_{j-1} (or the retrieval, for j = 0) must be done before O or P is touched
       if (!mbar_wait(&bars[B_PVDONE], (uint32_t)(j & 1))) {
         ok = false;
@@ -309,20 +341,20 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       tc_fence_after();
       if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t o[32];
-          tmem_ld32(tO + lane_off + c * 32, o);
+          tmem_ld32(tO + lane_off + col0 + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + lane_off + c * 32, o);
+          tmem_st32(tO + lane_off + col0 + c * 32, o);
         }
         tmem_wait_st();
       }
       l = l * alpha + rs;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const uint32_t off = (uint32_t)(u >> 3) * kSub + sw128(r, u & 7);
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t off = (uint32_t)half * kSub + sw128(r, u);
         *reinterpret_cast<uint4*>(sP + off) =
             make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       }
@@ -335,14 +367,22 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (ok) ok = mbar_wait(&bars[B_PVDONE], (uint32_t)(nkv & 1));
     tc_fence_after();
     if (ok) {
-      const float go = (1.f - g) / l;
-      const float gr = den != 0.f ? g / den : 0.f;
-      __nv_bfloat16* orow = out + ((size_t)bh * L + q_row + r) * D;
+      xden[half * 128 + r] = den;
+      xl[half * 128 + r] = l;
+      mbar_arrive(pair);
+      ok = mbar_wait(pair, pair_phase & 1);
+    }
+    if (ok) {
+      const float den_t = den + xden[(1 - half) * 128 + r];
+      const float l_t = l + xl[(1 - half) * 128 + r];
+      const float go = (1.f - g) / l_t;
+      const float gr = den_t != 0.f ? g / den_t : 0.f;
+      __nv_bfloat16* orow = out + ((size_t)bh * L + q_row + r) * D + col0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t o[32], rr[32];
-        tmem_ld32(tO + lane_off + c * 32, o);
-        tmem_ld32(tR + lane_off + c * 32, rr);
+        tmem_ld32(tO + lane_off + col0 + c * 32, o);
+        tmem_ld32(tR + lane_off + col0 + c * 32, rr);
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
@@ -354,9 +394,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const uint4 val = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
-          const int u = c * 4 + q4;  // 16-byte unit of the row (8 columns)
+          const int u = c * 4 + q4;  // 16-byte unit (8 columns) inside this half's box
           if (tma_store_ok) {
-            *reinterpret_cast<uint4*>(sQ + (uint32_t)(u >> 3) * kSub + sw128(r, u & 7)) = val;
+            *reinterpret_cast<uint4*>(sQ + (uint32_t)half * kSub + sw128(r, u)) = val;
           } else if (r < rows_valid) {
             *reinterpret_cast<uint4*>(orow + u * 8) = val;
           }
@@ -364,8 +404,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
       fence_proxy_async_smem();
     }
-    named_bar_sync(1, 128);
-    if (ok && tma_store_ok && r == 0) {
+    mbar_arrive(&bars[B_GROUP]);
+    const bool all_done = mbar_wait(&bars[B_GROUP], 0);
+    if (ok && all_done && tma_store_ok && threadIdx.x == 64) {
       tma_store_3d(&tm_o, sQ, 0, q_row, bh);
       tma_store_3d(&tm_o, sQ + kSub, 64, q_row, bh);
       tma_store_commit();
