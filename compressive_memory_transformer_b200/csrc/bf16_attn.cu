@@ -1,6 +1,6 @@
 // bf16_attn.cu — fused local attention + memory retrieval + gate (bf16, d = 128).
 //
-// One CTA computes one 128-row query tile of one segment of one (batch, head):
+// For every 128-row query tile of every segment of every (batch, head):
 //   A_dot = softmax(Q K^T / sqrt(d) + causal mask) V     over the segment's keys
 //   A_mem = sigma(Q) M_{s-1} / (sigma(Q) z_{s-1})         (0 where the denominator is 0)
 //   out   = g A_mem + (1 - g) A_dot,  g = sigmoid(beta_h)
@@ -8,25 +8,32 @@
 // llm-papers-study.pages.dev: sections 3.1, 3.3, 3.5). A_dot and A_mem stay in
 // tensor memory; only `out` is written to HBM.
 //
+// Persistent kernel: one CTA per SM walks a list of work units. A unit is a pair
+// of query tiles of one segment, i and T-1-i (T tiles per segment), so every unit
+// holds T+1 key tiles of work; units are dealt out round-robin in segment order,
+// so the ~150 units in flight touch ~20 segments and their K/V stay in L2.
+// Every pipeline runs on across tiles: while the softmax warps finish one tile,
+// the producer already loads the next Q and K tiles and the MMA thread issues
+// the next tile's first two Q K^T products.
+//
 // Warp roles (320 threads):
-//   warp 0     TMA producer: Q tile, then the V pipeline items [M_hi, M_lo, V_0, V_1, ...]
-//              and the K pipeline items [K_0, K_1, ...], two stages each.
+//   warp 0     TMA producer: Q per tile (reloaded once the last Q K^T of the tile
+//              and sigma(Q) are done); a K ring (2 stages); a V ring (2 stages)
+//              whose items per tile are M_hi, M_lo (the state, hi and lo bf16
+//              halves), then V_0, V_1, ...
 //   warp 1     tensor-memory allocation and the single MMA-issuing thread.
 //   warps 2-9  softmax / epilogue, two warpgroups: query row r (tensor-memory lane r)
 //              is shared by one thread of each; warpgroup h owns key columns
 //              [64h, 64h + 64) of S and value columns [64h, 64h + 64) of O, R and out.
-//              The two threads of a row exchange their partial row max every tile
-//              (and row sum / denominator at the end) through shared memory,
+//              The two threads of a row exchange their partial row max every key
+//              tile (and row sum / denominator at the end) through shared memory,
 //              synchronised by an mbarrier per warp pair.
-// Grid order: the query tiles of one segment are consecutive (heaviest first), so
-// the segment's K/V tiles are reused from L2 while they are in flight.
-// Tensor memory (512 columns): S0 | S1 (double-buffered scores) | O (A_dot
-// accumulator) | R (sigma(Q) M accumulator).
-// MMA order: QK_0, QK_1, R = sigma(Q)(M_hi + M_lo), then for each j: O += P_j V_j,
-// QK_{j+2}. The softmax of tile j overlaps PV_{j-1} and QK_{j+1}.
+// Tensor memory (512 columns): S0 | S1 (scores, alternating over the global key-tile
+// sequence) | O (A_dot accumulator) | R (sigma(Q) M accumulator).
+// MMA order per tile: R = sigma(Q)(M_hi + M_lo); for each j: O += P_j V_j, then
+// Q K_{j+2}^T; after the last PV, the next tile's Q K_0^T and Q K_1^T.
 // Online softmax keeps a per-row reference max and rescales O only when the
-// running max grows by more than 2^8 (in exp2 units), so most tiles skip the
-// tensor-memory round trip of O.
+// running max grows by more than 2^8 (in exp2 units).
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda.h>
@@ -40,7 +47,7 @@ namespace infini {
 namespace {
 
 constexpr int D = 128;
-constexpr int BM = 128;   // query rows per CTA
+constexpr int BM = 128;   // query rows per tile
 constexpr int BN = 128;   // keys per tile
 constexpr int kTile = 32768;     // one 128 x 128 bf16 tile
 constexpr int kSub = 16384;      // one 128 x 64 box (128-byte rows)
@@ -48,16 +55,64 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K = kTile;         // 2 stages
 constexpr int OFF_V = 3 * kTile;     // 2 stages
 constexpr int OFF_P = 5 * kTile;
-constexpr int OFF_Z = 6 * kTile;     // 128 floats
-constexpr int OFF_X = OFF_Z + 512;   // exchange: max [2 slots][2 halves][128], den, l [2][128]
+constexpr int OFF_X = 6 * kTile;     // exchange: max [2][2][128], den [2][128], l [2][128]
 constexpr int OFF_BAR = OFF_X + 4096;
 constexpr int kAttnSmem = OFF_BAR + 256 + 1024;  // + alignment slack
 constexpr int kThreads = 320;
 constexpr int kSoftmaxThreads = 256;
 
 enum {
-  B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9,
-  B_PFULL = 11, B_PVDONE = 12, B_DRAIN = 13, B_PAIR = 14 /* 4 */, B_GROUP = 18, B_COUNT = 19
+  B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = 4, B_VFULL = 6, B_VEMPTY = 8,
+  B_SFULL = 10, B_PFULL = 12, B_PVDONE = 13, B_DRAIN = 14, B_PAIR = 15 /* 4 */, B_COUNT = 19
+};
+
+struct Params {
+  long long L;
+  int N, S, H, T, U, BH;
+  long long units;
+};
+
+// One query tile of the work list.
+struct Tile {
+  int bh, s, i, nkv, q_row, rows_valid;
+  long long seg0;
+};
+
+// Walks the CTA's tiles: units blockIdx.x, blockIdx.x + gridDim.x, ...; unit u of
+// a segment holds tiles T-1-u and u (one tile when they coincide); tiles past the
+// end of a short final segment are skipped.
+struct TileIter {
+  long long unit;
+  int k;  // 0: tile T-1-u, 1: tile u
+  __device__ void init() {
+    unit = blockIdx.x;
+    k = 0;
+  }
+  __device__ bool next(const Params& p, Tile& t) {
+    while (unit < p.units) {
+      const long long seg = unit / p.U;
+      const int u = (int)(unit % p.U);
+      const int kk = k;
+      if (++k == 2) {
+        k = 0;
+        unit += gridDim.x;
+      }
+      const int i = kk == 0 ? p.T - 1 - u : u;
+      if (kk == 1 && u >= p.T - 1 - u) continue;  // the pair collapsed to one tile
+      t.s = (int)(seg % p.S);
+      t.bh = (int)(seg / p.S);
+      t.seg0 = (long long)t.s * p.N;
+      const int n_s = (int)min((long long)p.N, p.L - t.seg0);
+      const int T_s = (n_s + BM - 1) / BM;
+      if (i >= T_s) continue;
+      t.i = i;
+      t.nkv = i + 1;
+      t.q_row = (int)(t.seg0 + (long long)i * BM);
+      t.rows_valid = min(BM, n_s - i * BM);
+      return true;
+    }
+    return false;
+  }
 };
 
 // Bounded wait used only while draining after an error: ignores the error flag.
@@ -82,25 +137,9 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kk) {
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-            const __grid_constant__ CUtensorMap tm_m, const float* __restrict__ beta,
-            const float* __restrict__ zprev, __nv_bfloat16* __restrict__ out, long long L, int N,
-            int S, int H, int T, int BH) {
-  // ---- work item: segment-major, heaviest query tile of the segment first ----
-  const long long x = blockIdx.x;
-  const long long seg = x / T;
-  const int i = T - 1 - (int)(x % T);
-  const int s = (int)(seg % S);
-  const int bh = (int)(seg / S);
-  const long long seg0 = (long long)s * N;
-  const int n_s = (int)min((long long)N, L - seg0);
-  const int T_s = (n_s + BM - 1) / BM;
-  if (i >= T_s) return;  // uniform for the whole CTA, before any barrier
-  const int nkv = i + 1;
-  const int q_row = (int)(seg0 + (long long)i * BM);
-  const int rows_valid = min(BM, n_s - i * BM);
-  const bool tma_store_ok = rows_valid == BM || seg0 + n_s == L;
-
+            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
+            const float* __restrict__ beta, const float* __restrict__ zprev,
+            __nv_bfloat16* __restrict__ out, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -108,7 +147,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   uint8_t* sK = smem + OFF_K;
   uint8_t* sV = smem + OFF_V;
   uint8_t* sP = smem + OFF_P;
-  float* sZ = reinterpret_cast<float*>(smem + OFF_Z);
   float* sX = reinterpret_cast<float*>(smem + OFF_X);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
@@ -117,7 +155,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   if (threadIdx.x == 0) {
     for (int b = 0; b < B_COUNT; ++b) {
       uint32_t cnt = 1;
-      if (b == B_PFULL || b == B_GROUP) cnt = kSoftmaxThreads;
+      if (b == B_PFULL) cnt = kSoftmaxThreads;
+      // Q is free once the tile's last Q K^T is done and every softmax thread has
+      // read its row of Q for sigma(Q)
+      if (b == B_QEMPTY) cnt = 1 + kSoftmaxThreads;
       if (b >= B_PAIR && b < B_PAIR + 4) cnt = 64;
       mbar_init(&bars[b], cnt);
     }
@@ -126,13 +167,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_m);
-    tma_prefetch_desc(&tm_o);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (threadIdx.x >= 64 && threadIdx.x < 64 + D) sZ[threadIdx.x - 64] = zprev[((size_t)bh * S + s) * D + threadIdx.x - 64];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -142,43 +181,61 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0) {
-      int k_iss[2] = {0, 0}, v_iss[2] = {0, 0};
-      auto issue_k = [&](int j) -> bool {
-        const int st = j & 1, use = j >> 1;
+      int q_iss = 0, k_iss[2] = {0, 0}, v_iss[2] = {0, 0};
+      long long kc = 0, vc = 0;
+      bool ok = true;
+      auto issue_k = [&](const Tile& t, int j) -> bool {
+        const int st = (int)(kc & 1);
+        const long long use = kc >> 1;
         if (use > 0 && !mbar_wait(&bars[B_KEMPTY + st], (uint32_t)((use - 1) & 1))) return false;
         mbar_arrive_expect_tx(&bars[B_KFULL + st], kTile);
-        const int row = (int)(seg0 + (long long)j * BN);
-        tma_load_3d(sK + st * kTile, &tm_k, &bars[B_KFULL + st], 0, row, bh);
-        tma_load_3d(sK + st * kTile + kSub, &tm_k, &bars[B_KFULL + st], 64, row, bh);
+        const int row = (int)(t.seg0 + (long long)j * BN);
+        tma_load_3d(sK + st * kTile, &tm_k, &bars[B_KFULL + st], 0, row, t.bh);
+        tma_load_3d(sK + st * kTile + kSub, &tm_k, &bars[B_KFULL + st], 64, row, t.bh);
         ++k_iss[st];
+        ++kc;
         return true;
       };
-      auto issue_v = [&](int item) -> bool {
-        const int st = item & 1, use = item >> 1;
+      auto issue_v = [&](const Tile& t, int item) -> bool {  // item 0,1: M_hi, M_lo; 2+j: V_j
+        const int st = (int)(vc & 1);
+        const long long use = vc >> 1;
         if (use > 0 && !mbar_wait(&bars[B_VEMPTY + st], (uint32_t)((use - 1) & 1))) return false;
         mbar_arrive_expect_tx(&bars[B_VFULL + st], kTile);
         if (item < 2) {
-          const int zc = (bh * S + s) * 2 + item;
+          const int zc = (t.bh * p.S + t.s) * 2 + item;
           tma_load_3d(sV + st * kTile, &tm_m, &bars[B_VFULL + st], 0, 0, zc);
           tma_load_3d(sV + st * kTile + kSub, &tm_m, &bars[B_VFULL + st], 64, 0, zc);
         } else {
-          const int row = (int)(seg0 + (long long)(item - 2) * BN);
-          tma_load_3d(sV + st * kTile, &tm_v, &bars[B_VFULL + st], 0, row, bh);
-          tma_load_3d(sV + st * kTile + kSub, &tm_v, &bars[B_VFULL + st], 64, row, bh);
+          const int row = (int)(t.seg0 + (long long)(item - 2) * BN);
+          tma_load_3d(sV + st * kTile, &tm_v, &bars[B_VFULL + st], 0, row, t.bh);
+          tma_load_3d(sV + st * kTile + kSub, &tm_v, &bars[B_VFULL + st], 64, row, t.bh);
         }
         ++v_iss[st];
+        ++vc;
         return true;
       };
-      mbar_arrive_expect_tx(&bars[B_QFULL], kTile);
-      tma_load_3d(sQ, &tm_q, &bars[B_QFULL], 0, q_row, bh);
-      tma_load_3d(sQ + kSub, &tm_q, &bars[B_QFULL], 64, q_row, bh);
-      bool ok = issue_k(0) && (nkv < 2 || issue_k(1)) && issue_v(0) && issue_v(1);
-      for (int j = 0; ok && j < nkv; ++j) {
-        ok = issue_v(j + 2);
-        if (ok && j + 2 < nkv) ok = issue_k(j + 2);
+      TileIter it;
+      it.init();
+      Tile t;
+      int tc = 0;
+      while (ok && it.next(p, t)) {
+        if (tc > 0 && !mbar_wait(&bars[B_QEMPTY], (uint32_t)((tc - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&bars[B_QFULL], kTile);
+        tma_load_3d(sQ, &tm_q, &bars[B_QFULL], 0, t.q_row, t.bh);
+        tma_load_3d(sQ + kSub, &tm_q, &bars[B_QFULL], 64, t.q_row, t.bh);
+        ++q_iss;
+        ok = issue_k(t, 0) && (t.nkv < 2 || issue_k(t, 1)) && issue_v(t, 0) && issue_v(t, 1);
+        for (int j = 0; ok && j < t.nkv; ++j) {
+          ok = issue_v(t, j + 2);
+          if (ok && j + 2 < t.nkv) ok = issue_k(t, j + 2);
+        }
+        ++tc;
       }
       if (!ok) {  // let the copies already issued land before the CTA exits
-        drain_wait(&bars[B_QFULL], 0);
+        if (q_iss > 0) drain_wait(&bars[B_QFULL], (uint32_t)((q_iss - 1) & 1));
         for (int st = 0; st < 2; ++st) {
           if (k_iss[st] > 0) drain_wait(&bars[B_KFULL + st], (uint32_t)((k_iss[st] - 1) & 1));
           if (v_iss[st] > 0) drain_wait(&bars[B_VFULL + st], (uint32_t)((v_iss[st] - 1) & 1));
@@ -191,9 +248,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       const uint32_t id_qk = idesc_f32acc(1, 0, 0, BM, BN);
       const uint32_t id_pv = idesc_f32acc(1, 0, 1, BM, D);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-      auto qk = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&bars[B_KFULL + st], (uint32_t)((j >> 1) & 1))) return false;
+      long long kq = 0, vc = 0, pi = 0;
+      int tc = 0;
+      auto qk = [&](const Tile& t, int j, int tile_no) -> bool {
+        if (j == 0 && !mbar_wait(&bars[B_QFULL], (uint32_t)(tile_no & 1))) return false;
+        const int st = (int)(kq & 1);
+        if (!mbar_wait(&bars[B_KFULL + st], (uint32_t)((kq >> 1) & 1))) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
@@ -201,38 +261,60 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                       kk > 0 ? 1u : 0u);
         mma_commit(&bars[B_KEMPTY + st]);
         mma_commit(&bars[B_SFULL + st]);
+        if (j == t.nkv - 1) mma_commit(&bars[B_QEMPTY]);
+        ++kq;
         return true;
       };
-      bool ok = mbar_wait(&bars[B_QFULL], 0);
-      ok = ok && qk(0) && (nkv < 2 || qk(1));
-      // retrieval: R = sigma(Q) M_hi + sigma(Q) M_lo
-      ok = ok && mbar_wait(&bars[B_PFULL], 0) && mbar_wait(&bars[B_VFULL + 0], 0) &&
-           mbar_wait(&bars[B_VFULL + 1], 0);
-      if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tR, kmajor_desc(aP, kk), mnmajor_desc(aV, kk), id_pv, kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tR, kmajor_desc(aP, kk), mnmajor_desc(aV + kTile, kk), id_pv, 1u);
-        mma_commit(&bars[B_VEMPTY + 0]);
-        mma_commit(&bars[B_VEMPTY + 1]);
-        mma_commit(&bars[B_PVDONE]);
-      }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int item = j + 2, st = item & 1;
-        ok = mbar_wait(&bars[B_PFULL], (uint32_t)((j + 1) & 1)) &&
-             mbar_wait(&bars[B_VFULL + st], (uint32_t)((item >> 1) & 1));
+      TileIter it;
+      it.init();
+      Tile t, tn;
+      bool have = it.next(p, t);
+      bool ok = true;
+      if (have) ok = qk(t, 0, 0) && (t.nkv < 2 || qk(t, 1, 0));
+      while (ok && have) {
+        // retrieval: R = sigma(Q) M_hi + sigma(Q) M_lo
+        const int s0 = (int)(vc & 1), s1 = (int)((vc + 1) & 1);
+        ok = mbar_wait(&bars[B_PFULL], (uint32_t)(pi & 1)) &&
+             mbar_wait(&bars[B_VFULL + s0], (uint32_t)((vc >> 1) & 1)) &&
+             mbar_wait(&bars[B_VFULL + s1], (uint32_t)(((vc + 1) >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_bf16_ss(tO, kmajor_desc(aP, kk), mnmajor_desc(aV + st * kTile, kk), id_pv,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars[B_VEMPTY + st]);
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tR, kmajor_desc(aP, kk), mnmajor_desc(aV + s0 * kTile, kk), id_pv,
+                      kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tR, kmajor_desc(aP, kk), mnmajor_desc(aV + s1 * kTile, kk), id_pv, 1u);
+        mma_commit(&bars[B_VEMPTY + s0]);
+        mma_commit(&bars[B_VEMPTY + s1]);
         mma_commit(&bars[B_PVDONE]);
-        if (j + 2 < nkv) ok = qk(j + 2);
+        vc += 2;
+        ++pi;
+        const bool has_next = it.next(p, tn);
+        for (int j = 0; ok && j < t.nkv; ++j) {
+          const int st = (int)(vc & 1);
+          ok = mbar_wait(&bars[B_PFULL], (uint32_t)(pi & 1)) &&
+               mbar_wait(&bars[B_VFULL + st], (uint32_t)((vc >> 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_bf16_ss(tO, kmajor_desc(aP, kk), mnmajor_desc(aV + st * kTile, kk), id_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars[B_VEMPTY + st]);
+          mma_commit(&bars[B_PVDONE]);
+          ++vc;
+          ++pi;
+          if (j + 2 < t.nkv) {
+            ok = qk(t, j + 2, tc);
+          } else if (j == t.nkv - 1 && has_next) {
+            ok = qk(tn, 0, tc + 1) && (tn.nkv < 2 || qk(tn, 1, tc + 1));
+          }
+        }
+        t = tn;
+        have = has_next;
+        ++tc;
       }
       // no MMA may still be running when the CTA frees tensor memory
       mma_commit(&bars[B_DRAIN]);
@@ -250,134 +332,155 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     float* xmax = sX;            // [2 slots][2 halves][128]
     float* xden = sX + 512;      // [2 halves][128]
     float* xl = sX + 768;        // [2 halves][128]
-    const float bta = beta[bh % H];
-    const float g = 1.f / (1.f + expf(-bta));
-
-    bool ok = mbar_wait(&bars[B_QFULL], 0);
-    float den = 0.f;
-    if (ok) {
+    const float sl = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+    long long kc = 0, pi = 0;
+    int tc = 0;
+    bool ok = true;
+    TileIter it;
+    it.init();
+    Tile t;
+    while (ok && it.next(p, t)) {
+      const float g = 1.f / (1.f + expf(-beta[t.bh % p.H]));
+      const float* zs = zprev + ((size_t)t.bh * p.S + t.s) * D + col0;
+      if (!mbar_wait(&bars[B_QFULL], (uint32_t)(tc & 1))) {
+        ok = false;
+        break;
+      }
       // sigma(Q) of this thread's 64 columns -> P buffer (same swizzled position);
       // partial denominator sigma(Q_r) . z_{s-1} over those columns
-#pragma unroll 4
+      float den = 0.f;
+#pragma unroll 2
       for (int u = 0; u < 8; ++u) {
         const uint32_t off = (uint32_t)half * kSub + sw128(r, u);
         const uint4 raw = *reinterpret_cast<const uint4*>(sQ + off);
+        const float4 z0 = __ldg(reinterpret_cast<const float4*>(zs + u * 8));
+        const float4 z1 = __ldg(reinterpret_cast<const float4*>(zs + u * 8 + 4));
+        const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
         const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __bfloat1622float2(h[e]);
           const float p0 = elu1(f.x), p1 = elu1(f.y);
-          den = fmaf(p0, sZ[col0 + u * 8 + 2 * e], den);
-          den = fmaf(p1, sZ[col0 + u * 8 + 2 * e + 1], den);
+          den = fmaf(p0, zz[2 * e], den);
+          den = fmaf(p1, zz[2 * e + 1], den);
           pk[e] = pack_bf16x2(p0, p1);
         }
         *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
+      mbar_arrive(&bars[B_QEMPTY]);  // this thread is done reading Q
       fence_proxy_async_smem();
+      tc_fence_before();
       mbar_arrive(&bars[B_PFULL]);
-    }
+      ++pi;
 
-    const float sl = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
-    float m_use = -INFINITY, l = 0.f;
-    for (int j = 0; ok && j < nkv; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(&bars[B_SFULL + b], (uint32_t)((j >> 1) & 1))) {
+      float m_use = -INFINITY, l = 0.f;
+      for (int j = 0; j < t.nkv; ++j) {
+        const int b = (int)(kc & 1);
+        if (!mbar_wait(&bars[B_SFULL + b], (uint32_t)((kc >> 1) & 1))) {
+          ok = false;
+          break;
+        }
+        ++kc;
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld32(tS + lane_off + b * BN + col0, *reinterpret_cast<uint32_t(*)[32]>(sr));
+        tmem_ld32(tS + lane_off + b * BN + col0 + 32,
+                  *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+        tmem_wait_ld();
+        if (j == t.i) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if ((int)col0 + c > r) sr[c] = __float_as_uint(-INFINITY);
+        }
+        float mx[8];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+          mx[q8] = __uint_as_float(sr[q8]);
+#pragma unroll
+          for (int c = 1; c < 8; ++c) mx[q8] = fmaxf(mx[q8], __uint_as_float(sr[8 * c + q8]));
+        }
+        const float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        xmax[b * 256 + half * 128 + r] = mh;
+        mbar_arrive(pair);
+        if (!mbar_wait(pair, pair_phase & 1)) {
+          ok = false;
+          break;
+        }
+        ++pair_phase;
+        const float mt = fmaxf(mh, xmax[b * 256 + (1 - half) * 128 + r]);
+        bool need = false;
+        float alpha = 1.f;
+        if (j == 0) {
+          m_use = mt;
+        } else if ((mt - m_use) * sl > 8.f) {
+          need = true;
+          alpha = ex2_approx((m_use - mt) * sl);
+          m_use = mt;
+        }
+        const float mb = m_use * sl;
+        float rsum[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), sl, -mb));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), sl, -mb));
+          rsum[c & 3] += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+        // the previous P item (sigma(Q) or P_{j-1}) must be consumed before O or P is touched
+        if (!mbar_wait(&bars[B_PVDONE], (uint32_t)((pi - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + lane_off + col0 + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + lane_off + col0 + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+        l = l * alpha + rs;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t off = (uint32_t)half * kSub + sw128(r, u);
+          *reinterpret_cast<uint4*>(sP + off) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars[B_PFULL]);
+        ++pi;
+      }
+      if (!ok) break;
+
+      // ---- epilogue: out = (1 - g) O / l + g R / den, stored from registers ----
+      if (!mbar_wait(&bars[B_PVDONE], (uint32_t)((pi - 1) & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(tS + lane_off + b * BN + col0, *reinterpret_cast<uint32_t(*)[32]>(sr));
-      tmem_ld32(tS + lane_off + b * BN + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-      tmem_wait_ld();
-      if (j == i) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if ((int)col0 + c > r) sr[c] = __float_as_uint(-INFINITY);
-      }
-      float mx[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        mx[t] = __uint_as_float(sr[t]);
-#pragma unroll
-        for (int c = 1; c < 8; ++c) mx[t] = fmaxf(mx[t], __uint_as_float(sr[8 * c + t]));
-      }
-      const float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      xmax[b * 256 + half * 128 + r] = mh;
+      xden[half * 128 + r] = den;
+      xl[half * 128 + r] = l;
       mbar_arrive(pair);
       if (!mbar_wait(pair, pair_phase & 1)) {
         ok = false;
         break;
       }
       ++pair_phase;
-      const float mt = fmaxf(mh, xmax[b * 256 + (1 - half) * 128 + r]);
-      bool need = false;
-      float alpha = 1.f;
-      if (j == 0) {
-        m_use = mt;
-      } else if ((mt - m_use) * sl > 8.f) {
-        need = true;
-        alpha = ex2_approx((m_use - mt) * sl);
-        m_use = mt;
-      }
-      const float mb = m_use * sl;
-      float rsum[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), sl, -mb));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), sl, -mb));
-        rsum[c & 3] += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
-      }
-      const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
-      // PV_{j-1} (or the retrieval, for j = 0) must be done before O or P is touched
-      if (!mbar_wait(&bars[B_PVDONE], (uint32_t)(j & 1))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + lane_off + col0 + c * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + lane_off + col0 + c * 32, o);
-        }
-        tmem_wait_st();
-      }
-      l = l * alpha + rs;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t off = (uint32_t)half * kSub + sw128(r, u);
-        *reinterpret_cast<uint4*>(sP + off) =
-            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars[B_PFULL]);
-    }
-
-    // ---- epilogue: out = (1 - g) O / l + g R / den ----
-    if (ok) ok = mbar_wait(&bars[B_PVDONE], (uint32_t)(nkv & 1));
-    tc_fence_after();
-    if (ok) {
-      xden[half * 128 + r] = den;
-      xl[half * 128 + r] = l;
-      mbar_arrive(pair);
-      ok = mbar_wait(pair, pair_phase & 1);
-    }
-    if (ok) {
       const float den_t = den + xden[(1 - half) * 128 + r];
       const float l_t = l + xl[(1 - half) * 128 + r];
       const float go = (1.f - g) / l_t;
       const float gr = den_t != 0.f ? g / den_t : 0.f;
-      __nv_bfloat16* orow = out + ((size_t)bh * L + q_row + r) * D + col0;
+      __nv_bfloat16* orow = out + ((size_t)t.bh * p.L + t.q_row + r) * D + col0;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t o[32], rr[32];
@@ -391,26 +494,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           const float a1 = go * __uint_as_float(o[2 * e + 1]) + gr * __uint_as_float(rr[2 * e + 1]);
           w[e] = pack_bf16x2(a0, a1);
         }
+        if (r < t.rows_valid) {
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint4 val = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
-          const int u = c * 4 + q4;  // 16-byte unit (8 columns) inside this half's box
-          if (tma_store_ok) {
-            *reinterpret_cast<uint4*>(sQ + (uint32_t)half * kSub + sw128(r, u)) = val;
-          } else if (r < rows_valid) {
-            *reinterpret_cast<uint4*>(orow + u * 8) = val;
-          }
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) =
+                make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
         }
       }
-      fence_proxy_async_smem();
-    }
-    mbar_arrive(&bars[B_GROUP]);
-    const bool all_done = mbar_wait(&bars[B_GROUP], 0);
-    if (ok && all_done && tma_store_ok && threadIdx.x == 64) {
-      tma_store_3d(&tm_o, sQ, 0, q_row, bh);
-      tma_store_3d(&tm_o, sQ + kSub, 64, q_row, bh);
-      tma_store_commit();
-      tma_store_wait_all();
+      tc_fence_before();
+      ++tc;
     }
   }
 
@@ -433,16 +525,25 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                              const __nv_bfloat16* v, const float* beta, __nv_bfloat16* out,
                              const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
                              cudaStream_t stream) {
-  CUtensorMap mq, mk, mv, mo, mm;
+  CUtensorMap mq, mk, mv, mm;
   if (!make_bf16_map(&mq, q, (uint64_t)L, BH, 128) || !make_bf16_map(&mk, k, (uint64_t)L, BH, 128) ||
       !make_bf16_map(&mv, v, (uint64_t)L, BH, 128) ||
-      !make_bf16_map(&mo, out, (uint64_t)L, BH, 128) ||
       !make_bf16_map(&mm, ws.Mhl, D, (uint64_t)BH * S * 2, 128))
     return cudaErrorInvalidValue;
-  const int T = (int)((min((long long)N, L) + BM - 1) / BM);
-  const unsigned grid = (unsigned)((long long)T * S * BH);
-  attn_kernel<<<grid, kThreads, kAttnSmem, stream>>>(mq, mk, mv, mo, mm, beta, ws.zprev, out, L, N,
-                                                     S, H, T, BH);
+  Params p;
+  p.L = L;
+  p.N = N;
+  p.S = S;
+  p.H = H;
+  p.BH = BH;
+  p.T = (int)((min((long long)N, L) + BM - 1) / BM);
+  p.U = (p.T + 1) / 2;
+  p.units = (long long)BH * S * p.U;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const unsigned grid = (unsigned)(p.units < (long long)sms ? p.units : (long long)sms);
+  attn_kernel<<<grid, kThreads, kAttnSmem, stream>>>(mq, mk, mv, mm, beta, ws.zprev, out, p);
   return cudaGetLastError();
 }
 
