@@ -18,7 +18,7 @@
 //
 // Warp roles (320 threads):
 //   warp 0     TMA producer: Q per tile (reloaded once the last Q K^T of the tile
-//              and sigma(Q) are done); a K ring (2 stages); a V ring (2 stages)
+//              and sigma(Q) are done); a K ring (2 stages); a V ring (3 stages)
 //              whose items per tile are M_hi, M_lo (the state, hi and lo bf16
 //              halves), then V_0, V_1, ...
 //   warp 1     tensor-memory allocation and the single MMA-issuing thread.
@@ -27,13 +27,20 @@
 //              [64h, 64h + 64) of S and value columns [64h, 64h + 64) of O, R and out.
 //              The two threads of a row exchange their partial row max every key
 //              tile (and row sum / denominator at the end) through shared memory,
-//              synchronised by an mbarrier per warp pair.
+//              synchronised by an mbarrier per warp pair. Softmax barriers count
+//              one arrival per warp.
 // Tensor memory (512 columns): S0 | S1 (scores, alternating over the global key-tile
-// sequence) | O (A_dot accumulator) | R (sigma(Q) M accumulator).
+// sequence) | O (A_dot accumulator) | R (sigma(Q) M accumulator). P (bf16) is
+// written over the first 64 columns of its S buffer and read from there by the PV
+// MMA; sigma(Q) (bf16) is staged in O, each half in its own columns, for the
+// retrieval MMA before the tile's first PV overwrites O. Tensor-core operations
+// issued by the one MMA thread execute in issue order, which orders every read of
+// an aliased region before the next write to it.
 // MMA order per tile: R = sigma(Q)(M_hi + M_lo); for each j: O += P_j V_j, then
 // Q K_{j+2}^T; after the last PV, the next tile's Q K_0^T and Q K_1^T.
 // Online softmax keeps a per-row reference max and rescales O only when the
-// running max grows by more than 2^8 (in exp2 units).
+// running max grows by more than 2^8 (in exp2 units). One exponential in four is
+// evaluated on the FMA pipe (ex2_poly2) to offload the MUFU unit.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda.h>
@@ -51,19 +58,20 @@ constexpr int BM = 128;   // query rows per tile
 constexpr int BN = 128;   // keys per tile
 constexpr int kTile = 32768;     // one 128 x 128 bf16 tile
 constexpr int kSub = 16384;      // one 128 x 64 box (128-byte rows)
+constexpr int kVStages = 3;
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = kTile;         // 2 stages
-constexpr int OFF_V = 3 * kTile;     // 2 stages
-constexpr int OFF_P = 5 * kTile;
+constexpr int OFF_V = 3 * kTile;     // kVStages stages
 constexpr int OFF_X = 6 * kTile;     // exchange: max [2][2][128], den [2][128], l [2][128]
 constexpr int OFF_BAR = OFF_X + 4096;
 constexpr int kAttnSmem = OFF_BAR + 256 + 1024;  // + alignment slack
 constexpr int kThreads = 320;
 constexpr int kSoftmaxThreads = 256;
+constexpr int kSoftmaxWarps = 8;
 
 enum {
-  B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = 4, B_VFULL = 6, B_VEMPTY = 8,
-  B_SFULL = 10, B_PFULL = 12, B_PVDONE = 13, B_DRAIN = 14, B_PAIR = 15 /* 4 */, B_COUNT = 19
+  B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = 4, B_VFULL = 6 /* 3 */, B_VEMPTY = 9 /* 3 */,
+  B_SFULL = 12, B_PFULL = 14, B_PVDONE = 15, B_DRAIN = 16, B_PAIR = 17 /* 4 */, B_COUNT = 21
 };
 
 struct Params {
@@ -146,7 +154,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   uint8_t* sQ = smem + OFF_Q;
   uint8_t* sK = smem + OFF_K;
   uint8_t* sV = smem + OFF_V;
-  uint8_t* sP = smem + OFF_P;
   float* sX = reinterpret_cast<float*>(smem + OFF_X);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
@@ -155,11 +162,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   if (threadIdx.x == 0) {
     for (int b = 0; b < B_COUNT; ++b) {
       uint32_t cnt = 1;
-      if (b == B_PFULL) cnt = kSoftmaxThreads;
-      // Q is free once the tile's last Q K^T is done and every softmax thread has
-      // read its row of Q for sigma(Q)
-      if (b == B_QEMPTY) cnt = 1 + kSoftmaxThreads;
-      if (b >= B_PAIR && b < B_PAIR + 4) cnt = 64;
+      // arrivals are counted per warp (mbar_arrive_warp)
+      if (b == B_PFULL) cnt = kSoftmaxWarps;
+      // Q is free once the tile's last Q K^T is done and every softmax warp has
+      // read its rows of Q for sigma(Q)
+      if (b == B_QEMPTY) cnt = 1 + kSoftmaxWarps;
+      if (b >= B_PAIR && b < B_PAIR + 4) cnt = 2;
       mbar_init(&bars[b], cnt);
     }
     fence_barrier_init();
@@ -181,7 +189,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0) {
-      int q_iss = 0, k_iss[2] = {0, 0}, v_iss[2] = {0, 0};
+      int q_iss = 0, k_iss[2] = {0, 0}, v_iss[kVStages] = {0, 0, 0};
       long long kc = 0, vc = 0;
       bool ok = true;
       auto issue_k = [&](const Tile& t, int j) -> bool {
@@ -197,8 +205,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         return true;
       };
       auto issue_v = [&](const Tile& t, int item) -> bool {  // item 0,1: M_hi, M_lo; 2+j: V_j
-        const int st = (int)(vc & 1);
-        const long long use = vc >> 1;
+        const int st = (int)(vc % kVStages);
+        const long long use = vc / kVStages;
         if (use > 0 && !mbar_wait(&bars[B_VEMPTY + st], (uint32_t)((use - 1) & 1))) return false;
         mbar_arrive_expect_tx(&bars[B_VFULL + st], kTile);
         if (item < 2) {
@@ -236,10 +244,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
       if (!ok) {  // let the copies already issued land before the CTA exits
         if (q_iss > 0) drain_wait(&bars[B_QFULL], (uint32_t)((q_iss - 1) & 1));
-        for (int st = 0; st < 2; ++st) {
+        for (int st = 0; st < 2; ++st)
           if (k_iss[st] > 0) drain_wait(&bars[B_KFULL + st], (uint32_t)((k_iss[st] - 1) & 1));
+        for (int st = 0; st < kVStages; ++st)
           if (v_iss[st] > 0) drain_wait(&bars[B_VFULL + st], (uint32_t)((v_iss[st] - 1) & 1));
-        }
       }
     }
   } else if (warp == 1) {
@@ -247,8 +255,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (lane == 0) {
       const uint32_t id_qk = idesc_f32acc(1, 0, 0, BM, BN);
       const uint32_t id_pv = idesc_f32acc(1, 0, 1, BM, D);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-      long long kq = 0, vc = 0, pi = 0;
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      long long kq = 0, kp = 0, vc = 0, pi = 0;
       int tc = 0;
       auto qk = [&](const Tile& t, int j, int tile_no) -> bool {
         if (j == 0 && !mbar_wait(&bars[B_QFULL], (uint32_t)(tile_no & 1))) return false;
@@ -272,20 +280,22 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       bool ok = true;
       if (have) ok = qk(t, 0, 0) && (t.nkv < 2 || qk(t, 1, 0));
       while (ok && have) {
-        // retrieval: R = sigma(Q) M_hi + sigma(Q) M_lo
-        const int s0 = (int)(vc & 1), s1 = (int)((vc + 1) & 1);
+        // retrieval: R = sigma(Q) M_hi + sigma(Q) M_lo, sigma(Q) read from tensor memory
+        // (features 0..63 at O + [0, 32), features 64..127 at O + [64, 96))
+        const int s0 = (int)(vc % kVStages), s1 = (int)((vc + 1) % kVStages);
         ok = mbar_wait(&bars[B_PFULL], (uint32_t)(pi & 1)) &&
-             mbar_wait(&bars[B_VFULL + s0], (uint32_t)((vc >> 1) & 1)) &&
-             mbar_wait(&bars[B_VFULL + s1], (uint32_t)(((vc + 1) >> 1) & 1));
+             mbar_wait(&bars[B_VFULL + s0], (uint32_t)((vc / kVStages) & 1)) &&
+             mbar_wait(&bars[B_VFULL + s1], (uint32_t)(((vc + 1) / kVStages) & 1));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tR, kmajor_desc(aP, kk), mnmajor_desc(aV + s0 * kTile, kk), id_pv,
-                      kk > 0 ? 1u : 0u);
+          mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)),
+                      mnmajor_desc(aV + s0 * kTile, kk), id_pv, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tR, kmajor_desc(aP, kk), mnmajor_desc(aV + s1 * kTile, kk), id_pv, 1u);
+          mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)),
+                      mnmajor_desc(aV + s1 * kTile, kk), id_pv, 1u);
         mma_commit(&bars[B_VEMPTY + s0]);
         mma_commit(&bars[B_VEMPTY + s1]);
         mma_commit(&bars[B_PVDONE]);
@@ -293,19 +303,22 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         ++pi;
         const bool has_next = it.next(p, tn);
         for (int j = 0; ok && j < t.nkv; ++j) {
-          const int st = (int)(vc & 1);
+          const int st = (int)(vc % kVStages);
           ok = mbar_wait(&bars[B_PFULL], (uint32_t)(pi & 1)) &&
-               mbar_wait(&bars[B_VFULL + st], (uint32_t)((vc >> 1) & 1));
+               mbar_wait(&bars[B_VFULL + st], (uint32_t)((vc / kVStages) & 1));
           if (!ok) break;
           tc_fence_after();
+          // P_j lives in the first 64 columns of its S buffer
+          const uint32_t tP = tS + (uint32_t)(kp & 1) * BN;
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
-            mma_bf16_ss(tO, kmajor_desc(aP, kk), mnmajor_desc(aV + st * kTile, kk), id_pv,
+            mma_bf16_ts(tO, tP + 8 * kk, mnmajor_desc(aV + st * kTile, kk), id_pv,
                         (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bars[B_VEMPTY + st]);
           mma_commit(&bars[B_PVDONE]);
           ++vc;
           ++pi;
+          ++kp;
           if (j + 2 < t.nkv) {
             ok = qk(t, j + 2, tc);
           } else if (j == t.nkv - 1 && has_next) {
@@ -342,14 +355,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     while (ok && it.next(p, t)) {
       const float g = 1.f / (1.f + expf(-beta[t.bh % p.H]));
       const float* zs = zprev + ((size_t)t.bh * p.S + t.s) * D + col0;
-      if (!mbar_wait(&bars[B_QFULL], (uint32_t)(tc & 1))) {
+      if (!mbar_wait_warp(&bars[B_QFULL], (uint32_t)(tc & 1))) {
         ok = false;
         break;
       }
-      // sigma(Q) of this thread's 64 columns -> P buffer (same swizzled position);
-      // partial denominator sigma(Q_r) . z_{s-1} over those columns
+      // sigma(Q) of this thread's 64 columns -> tensor memory (O + 64 half, 32 packed
+      // columns); partial denominator sigma(Q_r) . z_{s-1} over those columns
       float den = 0.f;
-#pragma unroll 2
+      uint32_t sq[32];
+#pragma unroll
       for (int u = 0; u < 8; ++u) {
         const uint32_t off = (uint32_t)half * kSub + sw128(r, u);
         const uint4 raw = *reinterpret_cast<const uint4*>(sQ + off);
@@ -366,18 +380,20 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           den = fmaf(p1, zz[2 * e + 1], den);
           pk[e] = pack_bf16x2(p0, p1);
         }
-        *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sq[4 * u + e] = pk[e];
       }
-      mbar_arrive(&bars[B_QEMPTY]);  // this thread is done reading Q
-      fence_proxy_async_smem();
+      mbar_arrive_warp(&bars[B_QEMPTY]);  // this warp is done reading Q
+      tmem_st32_(tO + lane_off + 64 * half, sq);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[B_PFULL]);
+      mbar_arrive_warp(&bars[B_PFULL]);
       ++pi;
 
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < t.nkv; ++j) {
         const int b = (int)(kc & 1);
-        if (!mbar_wait(&bars[B_SFULL + b], (uint32_t)((kc >> 1) & 1))) {
+        if (!mbar_wait_warp(&bars[B_SFULL + b], (uint32_t)((kc >> 1) & 1))) {
           ok = false;
           break;
         }
@@ -403,8 +419,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         xmax[b * 256 + half * 128 + r] = mh;
-        mbar_arrive(pair);
-        if (!mbar_wait(pair, pair_phase & 1)) {
+        mbar_arrive_warp(pair);
+        if (!mbar_wait_warp(pair, pair_phase & 1)) {
           ok = false;
           break;
         }
@@ -420,18 +436,30 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           m_use = mt;
         }
         const float mb = m_use * sl;
-        float rsum[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint64_t sl2 = f2pack(sl, sl), nmb2 = f2pack(-mb, -mb);
+        uint64_t rsum2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), sl, -mb));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), sl, -mb));
-          rsum[c & 3] += p0 + p1;
+          float a0, a1, p0, p1;
+          f2unpack(fma2(f2pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2,
+                        nmb2),
+                   a0, a1);
+          if ((c & 3) == 3) {
+            ex2_poly2(a0, a1, p0, p1);
+          } else {
+            p0 = ex2_approx(a0);
+            p1 = ex2_approx(a1);
+          }
+          rsum2[c & 1] = add2(rsum2[c & 1], f2pack(p0, p1));
           pk[c] = pack_bf16x2(p0, p1);
         }
-        const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+        float r0, r1, r2, r3;
+        f2unpack(rsum2[0], r0, r1);
+        f2unpack(rsum2[1], r2, r3);
+        const float rs = (r0 + r1) + (r2 + r3);
         // the previous P item (sigma(Q) or P_{j-1}) must be consumed before O or P is touched
-        if (!mbar_wait(&bars[B_PVDONE], (uint32_t)((pi - 1) & 1))) {
+        if (!mbar_wait_warp(&bars[B_PVDONE], (uint32_t)((pi - 1) & 1))) {
           ok = false;
           break;
         }
@@ -449,29 +477,26 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           tmem_wait_st();
         }
         l = l * alpha + rs;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t off = (uint32_t)half * kSub + sw128(r, u);
-          *reinterpret_cast<uint4*>(sP + off) =
-              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        }
-        fence_proxy_async_smem();
+        // P (bf16) over the first 64 columns of this S buffer: half h at [32h, 32h + 32).
+        // Both halves of every row have read their S values (the max exchange above).
+        tmem_st32_(tS + lane_off + b * BN + 32 * half, pk);
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars[B_PFULL]);
+        mbar_arrive_warp(&bars[B_PFULL]);
         ++pi;
       }
       if (!ok) break;
 
       // ---- epilogue: out = (1 - g) O / l + g R / den, stored from registers ----
-      if (!mbar_wait(&bars[B_PVDONE], (uint32_t)((pi - 1) & 1))) {
+      if (!mbar_wait_warp(&bars[B_PVDONE], (uint32_t)((pi - 1) & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
       xden[half * 128 + r] = den;
       xl[half * 128 + r] = l;
-      mbar_arrive(pair);
-      if (!mbar_wait(pair, pair_phase & 1)) {
+      mbar_arrive_warp(pair);
+      if (!mbar_wait_warp(pair, pair_phase & 1)) {
         ok = false;
         break;
       }

@@ -14,7 +14,8 @@
 // with G_s = 0. This is the same function as the per-token formula, evaluated in
 // a different association order.
 //
-// Kernels (launch order):
+// Kernels (launch order; Linear+Delta: zpart, zscan, state, chain;
+// Linear: state (which also sums sigma(K)), zscan, chain):
 //   zpart_kernel  : partial sums of sigma(K) per (head, segment, token chunk)
 //   zscan_kernel  : z_{s-1} for every segment (fixed order), z_out
 //   state_kernel  : bf16 tcgen05 GEMMs per (head, segment, chunk):
@@ -24,6 +25,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <cstring>
 
 #include "bf16_path.h"
 #include "sm100.cuh"
@@ -109,25 +111,36 @@ __global__ void __launch_bounds__(D) zscan_kernel(const float* __restrict__ zpar
 // hi = rn_bf16(sigma) and lo = rn_bf16(sigma - hi), and dM = hi^T V + lo^T V
 // (V is exact in bf16), which keeps dM within ~2^-16 relative per term. G sums
 // only positive terms, so its bf16 rounding errors average out: G = hi^T (inv sigma)_bf16.
+// In Linear mode the kernel also writes the chunk's sum of sigma(K) (zpart), so
+// K is read once.
 //
-// Tokens move in slabs of 64. Per slab and pipeline stage (64 KB):
-//   KH  [64 x 128] bf16: K as loaded by TMA, overwritten in place by sigma(K)_hi
-//   V   [64 x 128] bf16: loaded by TMA, used as is
-//   GH  [64 x 128] bf16: (inv * sigma(K))_bf16            (Delta only)
-//   KL  [64 x 128] bf16: sigma(K)_lo
-// each as two boxes of 64 features (8 KB), 128-byte swizzle, rows = tokens. As
+// Tokens move in slabs of 32 through a ring of 6 stages. Per stage (32 KB):
+//   KH  [32 x 128] bf16: K as loaded by TMA, overwritten in place by sigma(K)_hi
+//   V   [32 x 128] bf16: loaded by TMA, used as is
+//   GH  [32 x 128] bf16: (inv * sigma(K))_bf16            (Delta only)
+//   KL  [32 x 128] bf16: sigma(K)_lo
+// each as two boxes of 64 features (4 KB), 128-byte swizzle, rows = tokens. As
 // MMA operands they are MN-major (features contiguous, tokens = K); V and GH are
 // adjacent so that hi^T [V | GH] is one N = 256 MMA.
-// Warps 0..7 convert; warp 8 issues the TMA copies and the MMAs.
+// Warps 0..15 convert (one 8-feature group of one token each per slab), warp 16
+// issues the TMA copies, warp 17 issues the MMAs.
 // ---------------------------------------------------------------------------
-constexpr int kSlab = 64;
-constexpr int kStages = 3;
-constexpr int kBox = kSlab * 128;          // one 64-row x 64-feature box: 8 KB
-constexpr int kMat = 2 * kBox;             // one [64 x 128] bf16 matrix: 16 KB
+constexpr int kSlab = 32;
+constexpr int kStages = 6;
+constexpr int kBox = kSlab * 128;          // one 32-row x 64-feature box: 4 KB
+constexpr int kMat = 2 * kBox;             // one [32 x 128] bf16 matrix: 8 KB
 constexpr int OFF_KH = 0, OFF_V = kMat, OFF_GH = 2 * kMat, OFF_KL = 3 * kMat;
-constexpr int kStageBytes = 4 * kMat;      // 64 KB
-constexpr int kStateThreads = 288;
-constexpr int kStateSmem = kStages * kStageBytes + 1024 + 1024;  // + alignment, barriers, z
+constexpr int kStageBytes = 4 * kMat;      // 32 KB
+constexpr int kConvWarps = 16;
+constexpr int kStateThreads = (kConvWarps + 2) * 32;
+constexpr int kProdWarp = kConvWarps, kMmaWarp = kConvWarps + 1;
+constexpr int kStateSmem = kStages * kStageBytes + 1024 + 256;  // + alignment, barriers
+
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
 
 __device__ __forceinline__ uint64_t slab_desc(uint32_t base, int kk) {
   // MN-major: 16 token rows per k-step (2048 B), 64-feature boxes kBox apart
@@ -136,18 +149,19 @@ __device__ __forceinline__ uint64_t slab_desc(uint32_t base, int kk) {
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-             const float* __restrict__ zprev, float* __restrict__ dpart, long long L, int N, int S,
-             int CH, int CL, int mode) {
+             const float* __restrict__ zprev, float* __restrict__ dpart,
+             float* __restrict__ zpart, long long L, int N, int S, int CH, int CL, int mode) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
   uint64_t* bar_full = bars;                 // [kStages] TMA landed
-  uint64_t* bar_conv = bars + kStages;       // [kStages] operands converted (256 arrivals)
+  uint64_t* bar_conv = bars + kStages;       // [kStages] operands converted (warp arrivals)
   uint64_t* bar_mma = bars + 2 * kStages;    // [kStages] MMAs of the stage done
   uint64_t* bar_done = bars + 3 * kStages;   // all MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
-  float* sZ = reinterpret_cast<float*>(smem + kStages * kStageBytes + 512);  // [128]
+  // [32][128] partial sums of sigma(K); reuses stage memory once every MMA is done
+  float* sZred = reinterpret_cast<float*>(smem);
 
   const long long idx = blockIdx.x;
   const int c = (int)(idx % CH);
@@ -165,14 +179,13 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_conv[i], 256);
+      mbar_init(&bar_conv[i], kConvWarps);  // one arrival per converter warp
       mbar_init(&bar_mma[i], 1);
     }
     mbar_init(bar_done, 1);
     fence_barrier_init();
   }
-  if (tid < D) sZ[tid] = delta ? zprev[((size_t)bh * S + s) * D + tid] : 0.f;
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, ncols);
     tmem_relinquish();
   }
@@ -181,26 +194,36 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   bool ok = true;
+  float dz[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // Linear: sum of sigma(K)
+  const int cg = tid & 15;  // this converter's 8-feature group
+  const int r = tid >> 4;   // this converter's token row in each slab
 
-  if (warp == 8) {
-    // ---------------- producer + MMA issuer ----------------
-    if (lane == 0 && nslab > 0) {
+  if (warp == kProdWarp) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
       const int row0 = (int)(t0 + beg);
-      auto load = [&](int sl) {
-        uint8_t* st = smem + (sl % kStages) * kStageBytes;
-        uint64_t* fb = &bar_full[sl % kStages];
-        mbar_arrive_expect_tx(fb, 2 * kMat);
+      for (int sl = 0; sl < nslab; ++sl) {
+        const int stg = sl % kStages;
+        if (sl >= kStages &&
+            !mbar_wait(&bar_mma[stg], (uint32_t)((sl / kStages - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + stg * kStageBytes;
+        mbar_arrive_expect_tx(&bar_full[stg], 2 * kMat);
         const int row = row0 + sl * kSlab;
-        tma_load_3d(st + OFF_KH, &tm_k, fb, 0, row, (int)bh);
-        tma_load_3d(st + OFF_KH + kBox, &tm_k, fb, 64, row, (int)bh);
-        tma_load_3d(st + OFF_V, &tm_v, fb, 0, row, (int)bh);
-        tma_load_3d(st + OFF_V + kBox, &tm_v, fb, 64, row, (int)bh);
-      };
-      int issued = 0;
-      for (; issued < nslab && issued < kStages; ++issued) load(issued);
+        tma_load_3d(st + OFF_KH, &tm_k, &bar_full[stg], 0, row, (int)bh);
+        tma_load_3d(st + OFF_KH + kBox, &tm_k, &bar_full[stg], 64, row, (int)bh);
+        tma_load_3d(st + OFF_V, &tm_v, &bar_full[stg], 0, row, (int)bh);
+        tma_load_3d(st + OFF_V + kBox, &tm_v, &bar_full[stg], 64, row, (int)bh);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
       const uint32_t id256 = idesc_f32acc(1, 1, 1, 128, 256);
       const uint32_t id128 = idesc_f32acc(1, 1, 1, 128, 128);
-      for (int sl = 0; sl < nslab && ok; ++sl) {
+      for (int sl = 0; sl < nslab; ++sl) {
         const int stg = sl % kStages;
         if (!mbar_wait(&bar_conv[stg], (uint32_t)((sl / kStages) & 1))) {
           ok = false;
@@ -214,41 +237,26 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           const uint64_t a_hi = slab_desc(base + OFF_KH, kk);
           const uint64_t a_lo = slab_desc(base + OFF_KL, kk);
           const uint64_t b_v = slab_desc(base + OFF_V, kk);
-          if (delta) {
-            mma_bf16_ss(tmem_d, a_hi, b_v, id256, acc);  // [dM | G] += hi^T [V | GH]
-          } else {
-            mma_bf16_ss(tmem_d, a_hi, b_v, id128, acc);  // dM += hi^T V
-          }
-          mma_bf16_ss(tmem_d, a_lo, b_v, id128, 1u);     // dM += lo^T V
+          mma_bf16_ss(tmem_d, a_hi, b_v, delta ? id256 : id128, acc);  // [dM | G] += hi^T [V | GH]
+          mma_bf16_ss(tmem_d, a_lo, b_v, id128, 1u);                  // dM += lo^T V
         }
         mma_commit(&bar_mma[stg]);
-        // refill the stage used by slab sl - 1 once its MMAs are done
-        if (sl >= 1 && issued < nslab) {
-          const int prev = sl - 1;
-          if (!mbar_wait(&bar_mma[prev % kStages], (uint32_t)((prev / kStages) & 1))) {
-            ok = false;
-            break;
-          }
-          load(issued++);
-        }
       }
-      mma_commit(bar_done);
-    } else if (lane == 0) {
-      mma_commit(bar_done);  // nothing issued: completes at once
+      mma_commit(bar_done);  // tracks every MMA issued above (completes at once if none)
     }
   } else {
-    // ---------------- converters (warps 0..7) ----------------
+    // ---------------- converters (warps 0..15) ----------------
+    float zr[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) zr[e] = delta ? zprev[((size_t)bh * S + s) * D + cg * 8 + e] : 0.f;
     for (int sl = 0; sl < nslab && ok; ++sl) {
       const int stg = sl % kStages;
       uint8_t* st = smem + stg * kStageBytes;
-      if (!mbar_wait(&bar_full[stg], (uint32_t)((sl / kStages) & 1))) {
+      if (!mbar_wait_warp(&bar_full[stg], (uint32_t)((sl / kStages) & 1))) {
         ok = false;
         break;
       }
-#pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int item = tid + 256 * it;
-        const int r = item >> 4, cg = item & 15;  // token row in the slab, 8-feature group
+      {
         const bool valid = sl * kSlab + r < len;
         const uint32_t off = (uint32_t)(cg >> 3) * kBox + sw128(r, cg & 7);
         const uint4 raw = *reinterpret_cast<const uint4*>(st + OFF_KH + off);
@@ -258,41 +266,49 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           f[e] = valid ? elu1(f[e]) : 0.f;
-          den = fmaf(f[e], sZ[cg * 8 + e], den);
+          den = fmaf(f[e], zr[e], den);
+          dz[e] += f[e];
         }
-        // 16 lanes of a half-warp hold the 128 features of one token
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        uint32_t hi[4], lo[4], gh[4];
-        const float inv = (delta && den != 0.f) ? 1.f / den : 0.f;
+        uint32_t hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
           const float2 hf = __bfloat1622float2(h);
           const __nv_bfloat162 l = __floats2bfloat162_rn(f[2 * e] - hf.x, f[2 * e + 1] - hf.y);
-          const __nv_bfloat162 g = __floats2bfloat162_rn(f[2 * e] * inv, f[2 * e + 1] * inv);
           hi[e] = *reinterpret_cast<const uint32_t*>(&h);
           lo[e] = *reinterpret_cast<const uint32_t*>(&l);
-          gh[e] = *reinterpret_cast<const uint32_t*>(&g);
         }
         *reinterpret_cast<uint4*>(st + OFF_KH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4*>(st + OFF_KL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        if (delta)
+        if (delta) {
+          // 16 lanes of a half-warp hold the 128 features of one token
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+          const float inv = den != 0.f ? 1.f / den : 0.f;
+          uint32_t gh[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 g = __floats2bfloat162_rn(f[2 * e] * inv, f[2 * e + 1] * inv);
+            gh[e] = *reinterpret_cast<const uint32_t*>(&g);
+          }
           *reinterpret_cast<uint4*>(st + OFF_GH + off) = make_uint4(gh[0], gh[1], gh[2], gh[3]);
+        }
       }
       fence_proxy_async_smem();
-      mbar_arrive(&bar_conv[stg]);
+      mbar_arrive_warp(&bar_conv[stg]);
     }
   }
 
-  const bool done = mbar_wait(bar_done, 0);
+  // Only the converter warps wait for the MMAs: the idle lanes of the producer and
+  // MMA warps must not spin next to the lane that drives the pipeline.
+  const bool done = warp < kConvWarps ? mbar_wait_warp(bar_done, 0) : true;
   tc_fence_after();
-  // epilogue: warps 0-3 write dM rows, warps 4-7 write G rows (Delta)
-  if (warp < 8) {
+  if (warp < kConvWarps) {
+    // epilogue: warps 0-3 write dM rows, warps 4-7 write G rows (Delta)
     const int lane_base = (warp & 3) * 32;
     const int row = lane_base + lane;
     const int half = warp >> 2;
-    if (half == 0 || delta) {
+    if (warp < 8 && (half == 0 || delta)) {
       float* dst = dpart + ((size_t)idx * 2 + half) * D * D + (size_t)row * D;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
@@ -306,6 +322,11 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         }
         if (done && ok) {
 #pragma unroll
+          if (half == 1) {  // G feeds a tf32 MMA in the chain: round it here, unbiased
+#pragma unroll
+            for (int e = 0; e < 32; ++e) rr[e] = tf32_rna(__uint_as_float(rr[e]));
+          }
+#pragma unroll
           for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4*>(dst + cc * 32 + e) =
                 make_float4(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1]),
@@ -313,117 +334,223 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         }
       }
     }
+    if (!delta) {
+      // chunk sum of sigma(K): threads with the same feature group add up
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sZred[r * 128 + cg * 8 + e] = dz[e];
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (!delta && tid < D) {
+    float sum = 0.f;
+#pragma unroll
+    for (int rr = 0; rr < kSlab; ++rr) sum += sZred[rr * 128 + tid];
+    zpart[idx * D + tid] = sum;
+  }
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_d, ncols);
   }
 }
 
 // ---------------------------------------------------------------------------
-// chain_kernel: grid = (BH, 4), block 256. Column block cb covers M[:, 32cb .. 32cb+31].
-// Thread t owns a 4x4 tile: rows 4*(t/8) .. +3, columns 32cb + 4*(t%8) .. +3.
+// chain_kernel: grid = (BH, 4), block 160. Column block cb covers M[:, 32cb .. 32cb+31].
+// Threads 0..127 own one row r of the block (32 fp32 values in registers);
+// warp 4 issues the TMA copies of G and the MMAs.
 // For s = 0..S-1: write M_{s-1} as hi/lo bf16 into Mhl[bh][s] (hi = rn(M),
-// lo = rn(M - hi)), then M += dM_s - G_s M (Delta) or M += dM_s (Linear).
-// G_s is symmetric, so row k of G_s serves as column k.
+// lo = rn(M - hi)), then M += dM_s (Linear) or M += dM_s - G_s M (Delta).
+// G_s M runs on the tensor cores as tf32 (both operands K-major): A = G_s as
+// stored (row-major, rounded to tf32 by the state kernel), B = the block of M
+// transposed in shared memory (rounded to tf32); D [128 x 32] in tensor memory.
+// G_s of the next segment is prefetched by TMA while the current one is used.
 // ---------------------------------------------------------------------------
-constexpr int kChainSmem = (D * D + D * 32) * 4;
+constexpr int kChainThreads = 160;
+constexpr int kGBytes = D * D * 4;                 // 64 KB
+constexpr int kMtBytes = 32 * D * 4;               // 16 KB: M block transposed [32][128]
+constexpr int kChainSmem = 2 * kGBytes + kMtBytes + 1024 + 256;
 
-__global__ void __launch_bounds__(256, 1)
-chain_kernel(const float* __restrict__ dpart, const float* M_in, float* M_out,
-             __nv_bfloat16* __restrict__ Mhl, int S, int CH, int mode) {
-  extern __shared__ __align__(16) float csm[];
-  float* sG = csm;            // [128][128]
-  float* sM = csm + D * D;    // [128][32]
-  const int bh = blockIdx.x, cb = blockIdx.y, tid = threadIdx.x;
-  const int r0 = 4 * (tid >> 3), cl = 4 * (tid & 7), c0 = 32 * cb + cl;
+__global__ void __launch_bounds__(kChainThreads, 1)
+chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__ dpart,
+             const float* M_in, float* M_out, __nv_bfloat16* __restrict__ Mhl, int S, int CH,
+             int mode) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sG = smem;                         // 2 buffers x [4 boxes of 128 rows x 32 fp32]
+  uint8_t* sMt = smem + 2 * kGBytes;          // [4 boxes of 32 rows x 32 fp32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kGBytes + kMtBytes);
+  uint64_t* bar_g = bars;       // [2] G landed
+  uint64_t* bar_mt = bars + 2;  // M^T written (4 warp arrivals)
+  uint64_t* bar_mma = bars + 3; // one G_c M product done (per chunk; the MMA thread waits it)
+  uint64_t* bar_seg = bars + 4; // G_s M of a whole segment done (once per segment)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+
+  const int bh = blockIdx.x, cb = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c0 = 32 * cb;
   const bool delta = mode == 1;
-  float m[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float4 t = M_in ? *reinterpret_cast<const float4*>(M_in + ((size_t)bh * D + r0 + i) * D + c0)
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
-    m[i][0] = t.x; m[i][1] = t.y; m[i][2] = t.z; m[i][3] = t.w;
+  if (tid == 0) {
+    mbar_init(&bar_g[0], 1);
+    mbar_init(&bar_g[1], 1);
+    mbar_init(bar_mt, 4);  // one arrival per row warp
+    mbar_init(bar_mma, 1);
+    mbar_init(bar_seg, 1);
+    fence_barrier_init();
   }
-  for (int s = 0; s < S; ++s) {
-    __nv_bfloat16* hi = Mhl + ((size_t)bh * S + s) * 2 * D * D;
-    __nv_bfloat16* lo = hi + D * D;
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 4) {
+    if (lane == 0 && delta) {
+      // G_s of chunk c: plane (bh*S + s)*CH*2 + 2c + 1 of dpart
+      auto load_g = [&](int s, int c, int buf) {
+        mbar_arrive_expect_tx(&bar_g[buf], kGBytes);
+        const int plane = ((bh * S + s) * CH + c) * 2 + 1;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __nv_bfloat162 h01 = __floats2bfloat162_rn(m[i][0], m[i][1]);
-      __nv_bfloat162 h23 = __floats2bfloat162_rn(m[i][2], m[i][3]);
-      const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
-      __nv_bfloat162 l01 = __floats2bfloat162_rn(m[i][0] - f01.x, m[i][1] - f01.y);
-      __nv_bfloat162 l23 = __floats2bfloat162_rn(m[i][2] - f23.x, m[i][3] - f23.y);
-      uint2 hv, lv;
-      hv.x = *reinterpret_cast<uint32_t*>(&h01); hv.y = *reinterpret_cast<uint32_t*>(&h23);
-      lv.x = *reinterpret_cast<uint32_t*>(&l01); lv.y = *reinterpret_cast<uint32_t*>(&l23);
-      *reinterpret_cast<uint2*>(hi + (size_t)(r0 + i) * D + c0) = hv;
-      *reinterpret_cast<uint2*>(lo + (size_t)(r0 + i) * D + c0) = lv;
-    }
-    float dm[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dm[i][j] = 0.f;
-    const float* dp = dpart + ((size_t)bh * S + s) * CH * 2 * D * D;
-    for (int c = 0; c < CH; ++c) {
-      const float* p = dp + (size_t)c * 2 * D * D;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 t = *reinterpret_cast<const float4*>(p + (size_t)(r0 + i) * D + c0);
-        dm[i][0] += t.x; dm[i][1] += t.y; dm[i][2] += t.z; dm[i][3] += t.w;
-      }
-    }
-    if (delta) {
-      __syncthreads();  // previous iteration's readers of sG / sM are done
-      for (int e = tid * 4; e < D * D; e += 256 * 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int c = 0; c < CH; ++c) {
-          const float4 t = *reinterpret_cast<const float4*>(dp + (size_t)c * 2 * D * D + D * D + e);
-          acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
+        for (int bx = 0; bx < 4; ++bx)
+          tma_load_3d(sG + buf * kGBytes + bx * (D * 128), &tm_g, &bar_g[buf], bx * 32, 0, plane);
+      };
+      const uint32_t idesc = idesc_f32acc(2, 0, 0, 128, 32);
+      int n = 0;  // G loads consumed so far
+      const int total = S * CH;
+      load_g(0, 0, 0);
+      for (int s = 0; s < S && ok; ++s) {
+        // M^T of this segment's M_{s-1} must be in shared memory
+        if (!mbar_wait(bar_mt, (uint32_t)(s & 1))) {
+          ok = false;
+          break;
         }
-        *reinterpret_cast<float4*>(sG + e) = acc;
+        for (int c = 0; c < CH; ++c, ++n) {
+          const int buf = n & 1;
+          if (n + 1 < total) {
+            // the other buffer was last read by the MMA of load n-1, finished before
+            // this point (its commit was awaited below)
+            load_g((n + 1) / CH, (n + 1) % CH, buf ^ 1);
+          }
+          if (!mbar_wait(&bar_g[buf], (uint32_t)((n >> 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ga = smem_u32(sG + buf * kGBytes), mb = smem_u32(sMt);
+#pragma unroll
+          for (int kk = 0; kk < D / 8; ++kk) {
+            const uint32_t koff = (uint32_t)(kk >> 2) * (D * 128) + (uint32_t)(kk & 3) * 32;
+            const uint32_t moff = (uint32_t)(kk >> 2) * (32 * 128) + (uint32_t)(kk & 3) * 32;
+            mma_tf32_ss(tmem_d, sdesc(ga + koff, 16, 1024), sdesc(mb + moff, 16, 1024), idesc,
+                        (c > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar_mma);
+          if (c == CH - 1) mma_commit(bar_seg);
+          if (!mbar_wait(bar_mma, (uint32_t)(n & 1))) {
+            ok = false;
+            break;
+          }
+        }
       }
+    }
+  } else {
+    const int r = tid;  // row of M
+    float m[32];
+    if (M_in) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<float4*>(sM + (r0 + i) * 32 + cl) =
-            make_float4(m[i][0], m[i][1], m[i][2], m[i][3]);
-      __syncthreads();
-      float gm[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) gm[i][j] = 0.f;
-#pragma unroll 4
-      for (int kk = 0; kk < D; ++kk) {
-        const float4 g4 = *reinterpret_cast<const float4*>(sG + kk * D + r0);   // G[r0..r0+3][kk]
-        const float4 m4 = *reinterpret_cast<const float4*>(sM + kk * 32 + cl);  // M[kk][c..c+3]
-        const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
-        const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) gm[i][j] = fmaf(gv[i], mv[j], gm[i][j]);
+      for (int e = 0; e < 32; e += 4) {
+        const float4 t = *reinterpret_cast<const float4*>(M_in + ((size_t)bh * D + r) * D + c0 + e);
+        m[e] = t.x; m[e + 1] = t.y; m[e + 2] = t.z; m[e + 3] = t.w;
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) m[i][j] += dm[i][j] - gm[i][j];
     } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int e = 0; e < 32; ++e) m[e] = 0.f;
+    }
+    // dM of the next segment, prefetched into registers. Chunk 0 is loaded by plain
+    // assignment so that nothing waits on the loads until the next segment uses
+    // them; further chunks (only when a segment is split, e.g. one-segment steps)
+    // are added at once.
+    float nx[32];
+    auto load_dm = [&](int s) {
+      const float* src = dpart + ((size_t)((bh * S + s) * CH) * 2) * D * D + (size_t)r * D + c0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) m[i][j] += dm[i][j];
+      for (int e = 0; e < 32; e += 4) {
+        const float4 t = __ldg(reinterpret_cast<const float4*>(src + e));
+        nx[e] = t.x; nx[e + 1] = t.y; nx[e + 2] = t.z; nx[e + 3] = t.w;
+      }
+      for (int c = 1; c < CH; ++c) {
+        const float* sc = src + (size_t)c * 2 * D * D;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 t = __ldg(reinterpret_cast<const float4*>(sc + e));
+          nx[e] += t.x; nx[e + 1] += t.y; nx[e + 2] += t.z; nx[e + 3] += t.w;
+        }
+      }
+    };
+    if (S > 0) load_dm(0);
+    for (int s = 0; s < S; ++s) {
+      // M_{s-1} -> hi / lo bf16
+      __nv_bfloat16* hi = Mhl + ((size_t)bh * S + s) * 2 * D * D + (size_t)r * D + c0;
+      __nv_bfloat16* lo = hi + D * D;
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        uint32_t h4[4], l4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(m[e + 2 * q], m[e + 2 * q + 1]);
+          const float2 hf = __bfloat1622float2(h);
+          const __nv_bfloat162 l = __floats2bfloat162_rn(m[e + 2 * q] - hf.x, m[e + 2 * q + 1] - hf.y);
+          h4[q] = *reinterpret_cast<const uint32_t*>(&h);
+          l4[q] = *reinterpret_cast<const uint32_t*>(&l);
+        }
+        *reinterpret_cast<uint4*>(hi + e) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+        *reinterpret_cast<uint4*>(lo + e) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+      }
+      float dm[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) dm[e] = nx[e];
+      if (s + 1 < S) load_dm(s + 1);
+      if (delta) {
+        // M^T block (tf32) -> shared memory: row c, K-major, 4 boxes of 32 k
+        const uint32_t kb = (uint32_t)(r >> 5), kin = (uint32_t)(r & 31);
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) {
+          const uint32_t off = kb * (32 * 128) + sw128((uint32_t)cc, kin >> 2) + (kin & 3) * 4;
+          *reinterpret_cast<uint32_t*>(sMt + off) = tf32_rna(m[cc]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive_warp(bar_mt);
+        if (!mbar_wait_warp(bar_seg, (uint32_t)(s & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t gm[32];
+        tmem_ld32(tmem_d + ((uint32_t)(warp * 32) << 16), gm);
+        tmem_wait_ld();
+        tc_fence_before();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) m[e] += dm[e] - __uint_as_float(gm[e]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) m[e] += dm[e];
+      }
+    }
+    if (M_out && ok) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(M_out + ((size_t)bh * D + r) * D + c0 + e) =
+            make_float4(m[e], m[e + 1], m[e + 2], m[e + 3]);
     }
   }
-  if (M_out) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<float4*>(M_out + ((size_t)bh * D + r0 + i) * D + c0) =
-          make_float4(m[i][0], m[i][1], m[i][2], m[i][3]);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, 32);
   }
 }
 
@@ -475,15 +602,39 @@ cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, co
                               const Bf16Workspace& ws, int BH, long long L, int N, int S, int CH,
                               int CL, int mode, cudaStream_t stream) {
   const unsigned nunits = (unsigned)((long long)BH * S * CH);
-  zpart_kernel<<<nunits, 256, 0, stream>>>(k, ws.zpart, L, N, S, CH, CL);
-  zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH);
   CUtensorMap mk, mv;
   if (!make_bf16_map(&mk, k, (uint64_t)L, BH, kSlab) || !make_bf16_map(&mv, v, (uint64_t)L, BH, kSlab))
     return cudaErrorInvalidValue;
-  state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(mk, mv, ws.zprev, ws.dpart, L, N, S,
-                                                               CH, CL, mode);
-  chain_kernel<<<dim3(BH, 4), 256, mode == 1 ? kChainSmem : 0, stream>>>(ws.dpart, M_in, M_out,
-                                                                        ws.Mhl, S, CH, mode);
+  if (mode == 1) {
+    // Linear+Delta needs z_{s-1} (hence every segment's sum of sigma(K)) first
+    zpart_kernel<<<nunits, 256, 0, stream>>>(k, ws.zpart, L, N, S, CH, CL);
+    zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH);
+    state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(mk, mv, ws.zprev, ws.dpart,
+                                                                 ws.zpart, L, N, S, CH, CL, mode);
+  } else {
+    // Linear: the state GEMM also produces the sums of sigma(K)
+    state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(mk, mv, ws.zprev, ws.dpart,
+                                                                 ws.zpart, L, N, S, CH, CL, mode);
+    zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH);
+  }
+  CUtensorMap mg;
+  if (mode == 1) {
+    // G planes of dpart, fp32 [planes][128][128]; box 32 columns x 128 rows
+    EncodeTiledFn enc = get_encode_fn();
+    const cuuint64_t dims[3] = {128, 128, (cuuint64_t)nunits * 2};
+    const cuuint64_t strides[2] = {128 * 4, 128 * 128 * 4};
+    const cuuint32_t box[3] = {32, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (!enc || enc(&mg, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ws.dpart, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    memset(&mg, 0, sizeof(mg));
+  }
+  chain_kernel<<<dim3(BH, 4), kChainThreads, kChainSmem, stream>>>(mg, ws.dpart, M_in, M_out,
+                                                                    ws.Mhl, S, CH, mode);
   return cudaGetLastError();
 }
 

@@ -54,6 +54,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One arrival for the whole warp: every lane's earlier shared-memory writes are
+// ordered before the arrival by the warp barrier, then lane 0 arrives. Barriers
+// waited on this way count warps, not threads (a few arrivals instead of hundreds
+// of serialised atomic updates on one barrier word).
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
@@ -90,6 +99,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
       }
     }
   }
+}
+
+// mbar_wait for code run by a whole warp: the outcome is made warp-uniform, so
+// that a wait that gave up in one lane makes the whole warp leave together (no
+// lane is left behind at a later warp-wide barrier).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
 // ----------------------------------------------------------------------------
@@ -228,6 +244,34 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// 32 lanes x 32 columns store, the mirror of tmem_ld32.
+__device__ __forceinline__ void tmem_st32_(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16. A in tensor memory: row m in
+// lane m, K elements packed two per 32-bit column (element 2c in the low half of
+// column c), one MMA (K = 16) reading 8 columns from a_tmem.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -271,6 +315,54 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction for two lanes' worth.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+  return v;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe (x <= 126; -inf allowed), so that
+// the MUFU unit is not the only pipe evaluating softmax exponentials.
+// Range reduction: x = n + f with n = round-to-nearest(x) (obtained by adding and
+// subtracting 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial,
+// then n is added to the exponent field. The polynomial is this library's own
+// minimax fit of 2^f on [-1/2, 1/2] for relative error (Remez exchange):
+// max relative error 7.5e-5, far below the bf16 rounding (2^-9) the result gets.
+// Inputs below -126 are clamped there (the result is then below 2^-126).
+__device__ __forceinline__ void ex2_poly2(float a, float b, float& ra, float& rb) {
+  const float kRound = 12582912.f;  // 1.5 * 2^23
+  a = fmaxf(a, -126.f);
+  b = fmaxf(b, -126.f);
+  const uint64_t x = f2pack(a, b);
+  const uint64_t t = add2(x, f2pack(kRound, kRound));
+  const uint64_t n = add2(t, f2pack(-kRound, -kRound));
+  const uint64_t f = fma2(n, f2pack(-1.f, -1.f), x);
+  uint64_t p = fma2(f, f2pack(0.05517167f, 0.05517167f), f2pack(0.24261113f, 0.24261113f));
+  p = fma2(p, f, f2pack(0.69326097f, 0.69326097f));
+  p = fma2(p, f, f2pack(0.99992806f, 0.99992806f));
+  float pa, pb, ta, tb;
+  f2unpack(p, pa, pb);
+  f2unpack(t, ta, tb);
+  const int na = __float_as_int(ta) - __float_as_int(kRound);
+  const int nb = __float_as_int(tb) - __float_as_int(kRound);
+  ra = __int_as_float(__float_as_int(pa) + (na << 23));
+  rb = __int_as_float(__float_as_int(pb) + (nb << 23));
 }
 
 // sigma(x) = ELU(x) + 1 = x + 1 for x > 0, e^x otherwise.
