@@ -38,6 +38,11 @@
 // an aliased region before the next write to it.
 // MMA order per tile: R = sigma(Q)(M_hi + M_lo); for each j: O += P_j V_j, then
 // Q K_{j+2}^T; after the last PV, the next tile's Q K_0^T and Q K_1^T.
+// Every mbarrier is waited on in completion order and can never complete twice
+// before its waiter has seen the first completion (a parity wait would then
+// miss it): sigma(Q) and P have separate barriers; P_{j+1} is written only after
+// the softmax saw PV_j done, the next tile's sigma(Q) only after the epilogue saw
+// R and the last PV done. z_{s-1} (512 B) rides on the Q barrier.
 // Online softmax keeps a per-row reference max and rescales O only when the
 // running max grows by more than 2^8 (in exp2 units). One exponential in four is
 // evaluated on the FMA pipe (ex2_poly2) to offload the MUFU unit.
@@ -63,7 +68,8 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K = kTile;         // 2 stages
 constexpr int OFF_V = 3 * kTile;     // kVStages stages
 constexpr int OFF_X = 6 * kTile;     // exchange: max [2][2][128], den [2][128], l [2][128]
-constexpr int OFF_BAR = OFF_X + 4096;
+constexpr int OFF_Z = OFF_X + 4096;   // z_{s-1} of the current tile (128 floats), loaded with Q
+constexpr int OFF_BAR = OFF_Z + 512;
 constexpr int kAttnSmem = OFF_BAR + 256 + 1024;  // + alignment slack
 constexpr int kThreads = 320;
 constexpr int kSoftmaxThreads = 256;
@@ -71,7 +77,8 @@ constexpr int kSoftmaxWarps = 8;
 
 enum {
   B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = 4, B_VFULL = 6 /* 3 */, B_VEMPTY = 9 /* 3 */,
-  B_SFULL = 12, B_PFULL = 14, B_PVDONE = 15, B_DRAIN = 16, B_PAIR = 17 /* 4 */, B_COUNT = 21
+  B_SFULL = 12, B_PFULL = 14, B_PVDONE = 15, B_DRAIN = 16, B_PAIR = 17 /* 4 */, B_RDONE = 21,
+  B_SQFULL = 22, B_COUNT = 23
 };
 
 struct Params {
@@ -142,6 +149,11 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kk) {
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kk) {
   return sdesc(base + (uint32_t)kk * 2048, kSub, 1024);
 }
+// The same two layouts as offsets added to the descriptor of k-step 0.
+__device__ __forceinline__ constexpr uint32_t kdesc_off(int kk) {
+  return (uint32_t)((kk >> 2) * (kSub >> 4) + (kk & 3) * 2);
+}
+__device__ __forceinline__ constexpr uint32_t mndesc_off(int kk) { return (uint32_t)kk * 128u; }
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -155,6 +167,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   uint8_t* sK = smem + OFF_K;
   uint8_t* sV = smem + OFF_V;
   float* sX = reinterpret_cast<float*>(smem + OFF_X);
+  float* sZ = reinterpret_cast<float*>(smem + OFF_Z);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
 
@@ -163,10 +176,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     for (int b = 0; b < B_COUNT; ++b) {
       uint32_t cnt = 1;
       // arrivals are counted per warp (mbar_arrive_warp)
-      if (b == B_PFULL) cnt = kSoftmaxWarps;
+      if (b == B_PFULL || b == B_SQFULL) cnt = kSoftmaxWarps;
       // Q is free once the tile's last Q K^T is done and every softmax warp has
       // read its rows of Q for sigma(Q)
       if (b == B_QEMPTY) cnt = 1 + kSoftmaxWarps;
+      // B_RDONE: one commit per tile (retrieval MMAs)
       if (b >= B_PAIR && b < B_PAIR + 4) cnt = 2;
       mbar_init(&bars[b], cnt);
     }
@@ -190,36 +204,41 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // ================= TMA producer =================
     if (lane == 0) {
       int q_iss = 0, k_iss[2] = {0, 0}, v_iss[kVStages] = {0, 0, 0};
-      long long kc = 0, vc = 0;
+      uint32_t kst = 0, kph = 0, vst = 0, vph = 0;  // next K / V ring stage and phase
+      bool k_wrapped = false, v_wrapped = false;     // every stage used at least once
       bool ok = true;
       auto issue_k = [&](const Tile& t, int j) -> bool {
-        const int st = (int)(kc & 1);
-        const long long use = kc >> 1;
-        if (use > 0 && !mbar_wait(&bars[B_KEMPTY + st], (uint32_t)((use - 1) & 1))) return false;
-        mbar_arrive_expect_tx(&bars[B_KFULL + st], kTile);
+        if (k_wrapped && !mbar_wait(&bars[B_KEMPTY + kst], kph ^ 1u)) return false;
+        mbar_arrive_expect_tx(&bars[B_KFULL + kst], kTile);
         const int row = (int)(t.seg0 + (long long)j * BN);
-        tma_load_3d(sK + st * kTile, &tm_k, &bars[B_KFULL + st], 0, row, t.bh);
-        tma_load_3d(sK + st * kTile + kSub, &tm_k, &bars[B_KFULL + st], 64, row, t.bh);
-        ++k_iss[st];
-        ++kc;
+        uint8_t* dst = sK + kst * kTile;
+        tma_load_3d(dst, &tm_k, &bars[B_KFULL + kst], 0, row, t.bh);
+        tma_load_3d(dst + kSub, &tm_k, &bars[B_KFULL + kst], 64, row, t.bh);
+        ++k_iss[kst];
+        kph ^= kst;
+        k_wrapped |= (kst == 1u);
+        kst ^= 1u;
         return true;
       };
       auto issue_v = [&](const Tile& t, int item) -> bool {  // item 0,1: M_hi, M_lo; 2+j: V_j
-        const int st = (int)(vc % kVStages);
-        const long long use = vc / kVStages;
-        if (use > 0 && !mbar_wait(&bars[B_VEMPTY + st], (uint32_t)((use - 1) & 1))) return false;
-        mbar_arrive_expect_tx(&bars[B_VFULL + st], kTile);
+        if (v_wrapped && !mbar_wait(&bars[B_VEMPTY + vst], vph ^ 1u)) return false;
+        mbar_arrive_expect_tx(&bars[B_VFULL + vst], kTile);
+        uint8_t* dst = sV + vst * kTile;
         if (item < 2) {
           const int zc = (t.bh * p.S + t.s) * 2 + item;
-          tma_load_3d(sV + st * kTile, &tm_m, &bars[B_VFULL + st], 0, 0, zc);
-          tma_load_3d(sV + st * kTile + kSub, &tm_m, &bars[B_VFULL + st], 64, 0, zc);
+          tma_load_3d(dst, &tm_m, &bars[B_VFULL + vst], 0, 0, zc);
+          tma_load_3d(dst + kSub, &tm_m, &bars[B_VFULL + vst], 64, 0, zc);
         } else {
           const int row = (int)(t.seg0 + (long long)(item - 2) * BN);
-          tma_load_3d(sV + st * kTile, &tm_v, &bars[B_VFULL + st], 0, row, t.bh);
-          tma_load_3d(sV + st * kTile + kSub, &tm_v, &bars[B_VFULL + st], 64, row, t.bh);
+          tma_load_3d(dst, &tm_v, &bars[B_VFULL + vst], 0, row, t.bh);
+          tma_load_3d(dst + kSub, &tm_v, &bars[B_VFULL + vst], 64, row, t.bh);
         }
-        ++v_iss[st];
-        ++vc;
+        ++v_iss[vst];
+        if (++vst == (uint32_t)kVStages) {
+          vst = 0;
+          vph ^= 1u;
+          v_wrapped = true;
+        }
         return true;
       };
       TileIter it;
@@ -231,9 +250,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&bars[B_QFULL], kTile);
+        mbar_arrive_expect_tx(&bars[B_QFULL], kTile + D * 4);
         tma_load_3d(sQ, &tm_q, &bars[B_QFULL], 0, t.q_row, t.bh);
         tma_load_3d(sQ + kSub, &tm_q, &bars[B_QFULL], 64, t.q_row, t.bh);
+        bulk_load(sZ, zprev + ((size_t)t.bh * p.S + t.s) * D, D * 4, &bars[B_QFULL]);
         ++q_iss;
         ok = issue_k(t, 0) && (t.nkv < 2 || issue_k(t, 1)) && issue_v(t, 0) && issue_v(t, 1);
         for (int j = 0; ok && j < t.nkv; ++j) {
@@ -252,26 +272,44 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
+    // One thread issues every tensor-core operation, so everything between two
+    // MMAs is on the critical path: shared-memory descriptors are built once per
+    // buffer and moved by a constant add (a descriptor holds the address / 16 in
+    // its low 14 bits and every operand lies below 256 KB, so an offset inside a
+    // buffer never carries out of that field), and ring positions are kept as
+    // 32-bit stage / phase pairs.
     if (lane == 0) {
       const uint32_t id_qk = idesc_f32acc(1, 0, 0, BM, BN);
       const uint32_t id_pv = idesc_f32acc(1, 0, 1, BM, D);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      long long kq = 0, kp = 0, vc = 0, pi = 0;
+      const uint64_t dQ = kmajor_desc(smem_u32(sQ), 0);
+      const uint64_t dK0 = kmajor_desc(smem_u32(sK), 0);
+      const uint64_t dV0 = mnmajor_desc(smem_u32(sV), 0);
+      constexpr uint32_t kTileD = kTile >> 4;  // one tile, in descriptor units
+      uint32_t kst = 0, kph = 0;  // K ring: stage and phase of the next Q K^T
+      uint32_t vst = 0, vph = 0;  // V ring: stage and phase of the next item
+      uint32_t pb = 0;            // S buffer (and p_full parity) of the next P
       int tc = 0;
       auto qk = [&](const Tile& t, int j, int tile_no) -> bool {
         if (j == 0 && !mbar_wait(&bars[B_QFULL], (uint32_t)(tile_no & 1))) return false;
-        const int st = (int)(kq & 1);
-        if (!mbar_wait(&bars[B_KFULL + st], (uint32_t)((kq >> 1) & 1))) return false;
+        if (!mbar_wait(&bars[B_KFULL + kst], kph)) return false;
         tc_fence_after();
+        const uint64_t dk = dK0 + kst * kTileD;
+        const uint32_t dS = tS + kst * BN;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tS + st * BN, kmajor_desc(aQ, kk), kmajor_desc(aK + st * kTile, kk), id_qk,
-                      kk > 0 ? 1u : 0u);
-        mma_commit(&bars[B_KEMPTY + st]);
-        mma_commit(&bars[B_SFULL + st]);
+          mma_bf16_ss(dS, dQ + kdesc_off(kk), dk + kdesc_off(kk), id_qk, kk > 0 ? 1u : 0u);
+        mma_commit(&bars[B_KEMPTY + kst]);
+        mma_commit(&bars[B_SFULL + kst]);
         if (j == t.nkv - 1) mma_commit(&bars[B_QEMPTY]);
-        ++kq;
+        kph ^= kst;
+        kst ^= 1u;
         return true;
+      };
+      auto v_next = [&]() {
+        if (++vst == (uint32_t)kVStages) {
+          vst = 0;
+          vph ^= 1u;
+        }
       };
       TileIter it;
       it.init();
@@ -282,43 +320,42 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       while (ok && have) {
         // retrieval: R = sigma(Q) M_hi + sigma(Q) M_lo, sigma(Q) read from tensor memory
         // (features 0..63 at O + [0, 32), features 64..127 at O + [64, 96))
-        const int s0 = (int)(vc % kVStages), s1 = (int)((vc + 1) % kVStages);
-        ok = mbar_wait(&bars[B_PFULL], (uint32_t)(pi & 1)) &&
-             mbar_wait(&bars[B_VFULL + s0], (uint32_t)((vc / kVStages) & 1)) &&
-             mbar_wait(&bars[B_VFULL + s1], (uint32_t)(((vc + 1) / kVStages) & 1));
+        const uint32_t s0 = vst, p0 = vph;
+        v_next();
+        const uint32_t s1 = vst, p1 = vph;
+        v_next();
+        ok = mbar_wait(&bars[B_SQFULL], (uint32_t)(tc & 1)) &&
+             mbar_wait(&bars[B_VFULL + s0], p0) && mbar_wait(&bars[B_VFULL + s1], p1);
         if (!ok) break;
         tc_fence_after();
+        const uint64_t dm0 = dV0 + s0 * kTileD, dm1 = dV0 + s1 * kTileD;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)),
-                      mnmajor_desc(aV + s0 * kTile, kk), id_pv, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)), dm0 + mndesc_off(kk), id_pv,
+                      kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)),
-                      mnmajor_desc(aV + s1 * kTile, kk), id_pv, 1u);
+          mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)), dm1 + mndesc_off(kk), id_pv,
+                      1u);
         mma_commit(&bars[B_VEMPTY + s0]);
         mma_commit(&bars[B_VEMPTY + s1]);
-        mma_commit(&bars[B_PVDONE]);
-        vc += 2;
-        ++pi;
+        mma_commit(&bars[B_RDONE]);
         const bool has_next = it.next(p, tn);
         for (int j = 0; ok && j < t.nkv; ++j) {
-          const int st = (int)(vc % kVStages);
-          ok = mbar_wait(&bars[B_PFULL], (uint32_t)(pi & 1)) &&
-               mbar_wait(&bars[B_VFULL + st], (uint32_t)((vc / kVStages) & 1));
+          const uint32_t st = vst, ph = vph;
+          v_next();
+          ok = mbar_wait(&bars[B_PFULL], pb) && mbar_wait(&bars[B_VFULL + st], ph);
           if (!ok) break;
           tc_fence_after();
           // P_j lives in the first 64 columns of its S buffer
-          const uint32_t tP = tS + (uint32_t)(kp & 1) * BN;
+          const uint32_t tP = tS + pb * BN;
+          const uint64_t dv = dV0 + st * kTileD;
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
-            mma_bf16_ts(tO, tP + 8 * kk, mnmajor_desc(aV + st * kTile, kk), id_pv,
-                        (j > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ts(tO, tP + 8 * kk, dv + mndesc_off(kk), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bars[B_VEMPTY + st]);
           mma_commit(&bars[B_PVDONE]);
-          ++vc;
-          ++pi;
-          ++kp;
+          pb ^= 1u;
           if (j + 2 < t.nkv) {
             ok = qk(t, j + 2, tc);
           } else if (j == t.nkv - 1 && has_next) {
@@ -346,15 +383,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     float* xden = sX + 512;      // [2 halves][128]
     float* xl = sX + 768;        // [2 halves][128]
     const float sl = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
-    long long kc = 0, pi = 0;
+    long long kc = 0;
     int tc = 0;
     bool ok = true;
     TileIter it;
     it.init();
     Tile t;
     while (ok && it.next(p, t)) {
-      const float g = 1.f / (1.f + expf(-beta[t.bh % p.H]));
-      const float* zs = zprev + ((size_t)t.bh * p.S + t.s) * D + col0;
+      const float bta = __ldg(beta + t.bh % p.H);  // used in the epilogue
+      const float* zs = sZ + col0;
       if (!mbar_wait_warp(&bars[B_QFULL], (uint32_t)(tc & 1))) {
         ok = false;
         break;
@@ -367,8 +404,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       for (int u = 0; u < 8; ++u) {
         const uint32_t off = (uint32_t)half * kSub + sw128(r, u);
         const uint4 raw = *reinterpret_cast<const uint4*>(sQ + off);
-        const float4 z0 = __ldg(reinterpret_cast<const float4*>(zs + u * 8));
-        const float4 z1 = __ldg(reinterpret_cast<const float4*>(zs + u * 8 + 4));
+        const float4 z0 = *reinterpret_cast<const float4*>(zs + u * 8);
+        const float4 z1 = *reinterpret_cast<const float4*>(zs + u * 8 + 4);
         const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
         const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
         uint32_t pk[4];
@@ -387,8 +424,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       tmem_st32_(tO + lane_off + 64 * half, sq);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive_warp(&bars[B_PFULL]);
-      ++pi;
+      mbar_arrive_warp(&bars[B_SQFULL]);
 
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < t.nkv; ++j) {
@@ -458,8 +494,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         f2unpack(rsum2[0], r0, r1);
         f2unpack(rsum2[1], r2, r3);
         const float rs = (r0 + r1) + (r2 + r3);
-        // the previous P item (sigma(Q) or P_{j-1}) must be consumed before O or P is touched
-        if (!mbar_wait_warp(&bars[B_PVDONE], (uint32_t)((pi - 1) & 1))) {
+        // PV_{j-1} must be done before O is touched (a rescale). Every PV completion
+        // is consumed once, in order: PV of the previous tile's last step in its
+        // epilogue, PV_{j-1} here for j >= 1.
+        if (j > 0 && !mbar_wait_warp(&bars[B_PVDONE], (uint32_t)((kc - 2) & 1))) {
           ok = false;
           break;
         }
@@ -483,15 +521,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive_warp(&bars[B_PFULL]);
-        ++pi;
       }
       if (!ok) break;
 
-      // ---- epilogue: out = (1 - g) O / l + g R / den, stored from registers ----
-      if (!mbar_wait_warp(&bars[B_PVDONE], (uint32_t)((pi - 1) & 1))) {
+      // ---- epilogue: out = (1 - g) O / l + g R / den ----
+      if (!mbar_wait_warp(&bars[B_PVDONE], (uint32_t)((kc - 1) & 1)) ||
+          !mbar_wait_warp(&bars[B_RDONE], (uint32_t)(tc & 1))) {
         ok = false;
         break;
       }
+      const float g = 1.f / (1.f + expf(-bta));
       tc_fence_after();
       xden[half * 128 + r] = den;
       xl[half * 128 + r] = l;
