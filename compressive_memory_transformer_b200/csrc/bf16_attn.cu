@@ -21,7 +21,7 @@
 //              and sigma(Q) are done); a K ring (2 stages); a V ring (3 stages)
 //              whose items per tile are M_hi, M_lo (the state, hi and lo bf16
 //              halves), then V_0, V_1, ...
-//   warp 1     tensor-memory allocation and the single MMA-issuing thread.
+//   warp 1     tensor-memory allocation and the MMA issue (one elected lane).
 //   warps 2-9  softmax / epilogue, two warpgroups: query row r (tensor-memory lane r)
 //              is shared by one thread of each; warpgroup h owns key columns
 //              [64h, 64h + 64) of S and value columns [64h, 64h + 64) of O, R and out.
@@ -272,13 +272,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
-    // One thread issues every tensor-core operation, so everything between two
-    // MMAs is on the critical path: shared-memory descriptors are built once per
-    // buffer and moved by a constant add (a descriptor holds the address / 16 in
-    // its low 14 bits and every operand lies below 256 KB, so an offset inside a
-    // buffer never carries out of that field), and ring positions are kept as
-    // 32-bit stage / phase pairs.
-    if (lane == 0) {
+    // The whole warp runs the issue loop (waits, ring positions, descriptors), so
+    // every value is warp-uniform, and one elected lane (always lane 0) issues the
+    // tensor-core operations and commits: issuing from a diverged single thread
+    // was several times slower while the softmax warps on the same scheduler were
+    // busy. Everything between two MMAs is on the critical path: shared-memory
+    // descriptors are built once per buffer and moved by a constant add (a
+    // descriptor holds the address / 16 in its low 14 bits and every operand lies
+    // below 256 KB, so an offset inside a buffer never carries out of that field),
+    // and ring positions are kept as 32-bit stage / phase pairs.
+    {
       const uint32_t id_qk = idesc_f32acc(1, 0, 0, BM, BN);
       const uint32_t id_pv = idesc_f32acc(1, 0, 1, BM, D);
       const uint64_t dQ = kmajor_desc(smem_u32(sQ), 0);
@@ -290,17 +293,20 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       uint32_t pb = 0;            // S buffer (and p_full parity) of the next P
       int tc = 0;
       auto qk = [&](const Tile& t, int j, int tile_no) -> bool {
-        if (j == 0 && !mbar_wait(&bars[B_QFULL], (uint32_t)(tile_no & 1))) return false;
-        if (!mbar_wait(&bars[B_KFULL + kst], kph)) return false;
+        if (j == 0 && !mbar_wait_warp(&bars[B_QFULL], (uint32_t)(tile_no & 1))) return false;
+        if (!mbar_wait_warp(&bars[B_KFULL + kst], kph)) return false;
         tc_fence_after();
         const uint64_t dk = dK0 + kst * kTileD;
         const uint32_t dS = tS + kst * BN;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(dS, dQ + kdesc_off(kk), dk + kdesc_off(kk), id_qk, kk > 0 ? 1u : 0u);
-        mma_commit(&bars[B_KEMPTY + kst]);
-        mma_commit(&bars[B_SFULL + kst]);
-        if (j == t.nkv - 1) mma_commit(&bars[B_QEMPTY]);
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(dS, dQ + kdesc_off(kk), dk + kdesc_off(kk), id_qk, kk > 0 ? 1u : 0u);
+          mma_commit(&bars[B_KEMPTY + kst]);
+          mma_commit(&bars[B_SFULL + kst]);
+          if (j == t.nkv - 1) mma_commit(&bars[B_QEMPTY]);
+        }
+        __syncwarp();
         kph ^= kst;
         kst ^= 1u;
         return true;
@@ -324,37 +330,43 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         v_next();
         const uint32_t s1 = vst, p1 = vph;
         v_next();
-        ok = mbar_wait(&bars[B_SQFULL], (uint32_t)(tc & 1)) &&
-             mbar_wait(&bars[B_VFULL + s0], p0) && mbar_wait(&bars[B_VFULL + s1], p1);
+        ok = mbar_wait_warp(&bars[B_SQFULL], (uint32_t)(tc & 1)) &&
+             mbar_wait_warp(&bars[B_VFULL + s0], p0) && mbar_wait_warp(&bars[B_VFULL + s1], p1);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dm0 = dV0 + s0 * kTileD, dm1 = dV0 + s1 * kTileD;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)), dm0 + mndesc_off(kk), id_pv,
-                      kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)), dm0 + mndesc_off(kk), id_pv,
+                        kk > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)), dm1 + mndesc_off(kk), id_pv,
-                      1u);
-        mma_commit(&bars[B_VEMPTY + s0]);
-        mma_commit(&bars[B_VEMPTY + s1]);
-        mma_commit(&bars[B_RDONE]);
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)), dm1 + mndesc_off(kk), id_pv,
+                        1u);
+          mma_commit(&bars[B_VEMPTY + s0]);
+          mma_commit(&bars[B_VEMPTY + s1]);
+          mma_commit(&bars[B_RDONE]);
+        }
+        __syncwarp();
         const bool has_next = it.next(p, tn);
         for (int j = 0; ok && j < t.nkv; ++j) {
           const uint32_t st = vst, ph = vph;
           v_next();
-          ok = mbar_wait(&bars[B_PFULL], pb) && mbar_wait(&bars[B_VFULL + st], ph);
+          ok = mbar_wait_warp(&bars[B_PFULL], pb) && mbar_wait_warp(&bars[B_VFULL + st], ph);
           if (!ok) break;
           tc_fence_after();
           // P_j lives in the first 64 columns of its S buffer
           const uint32_t tP = tS + pb * BN;
           const uint64_t dv = dV0 + st * kTileD;
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            mma_bf16_ts(tO, tP + 8 * kk, dv + mndesc_off(kk), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&bars[B_VEMPTY + st]);
-          mma_commit(&bars[B_PVDONE]);
+            for (int kk = 0; kk < BN / 16; ++kk)
+              mma_bf16_ts(tO, tP + 8 * kk, dv + mndesc_off(kk), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&bars[B_VEMPTY + st]);
+            mma_commit(&bars[B_PVDONE]);
+          }
+          __syncwarp();
           pb ^= 1u;
           if (j + 2 < t.nkv) {
             ok = qk(t, j + 2, tc);
@@ -367,7 +379,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         ++tc;
       }
       // no MMA may still be running when the CTA frees tensor memory
-      mma_commit(&bars[B_DRAIN]);
+      if (elect_one()) mma_commit(&bars[B_DRAIN]);
+      __syncwarp();
       drain_wait(&bars[B_DRAIN], 0);
     }
   } else {

@@ -270,6 +270,21 @@ __device__ __forceinline__ void tmem_st32_(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+// One lane of a converged warp (the lowest active one, so always the same lane
+// when the whole warp is active) gets true. Tensor-core work is issued this way
+// from a warp whose other lanes run the same bookkeeping: values computed by the
+// whole warp stay warp-uniform, which keeps the issue path short even when other
+// warps compete for the same scheduler.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .b32 r;\n\t.reg .pred p;\n\t"
+      "elect.sync r|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc], kind::f16. A in tensor memory: row m in
 // lane m, K elements packed two per 32-bit column (element 2c in the low half of
 // column c), one MMA (K = 16) reading 8 columns from a_tmem.
