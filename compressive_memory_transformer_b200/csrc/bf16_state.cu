@@ -220,17 +220,20 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      const uint32_t id256 = idesc_f32acc(1, 1, 1, 128, 256);
-      const uint32_t id128 = idesc_f32acc(1, 1, 1, 128, 128);
-      for (int sl = 0; sl < nslab; ++sl) {
-        const int stg = sl % kStages;
-        if (!mbar_wait(&bar_conv[stg], (uint32_t)((sl / kStages) & 1))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t base = smem_u32(smem + stg * kStageBytes);
+    // The whole warp runs the loop and waits; one elected lane (always lane 0)
+    // issues and commits, which keeps the issue path short next to the busy
+    // converter warps on the same scheduler.
+    const uint32_t id256 = idesc_f32acc(1, 1, 1, 128, 256);
+    const uint32_t id128 = idesc_f32acc(1, 1, 1, 128, 128);
+    for (int sl = 0; sl < nslab; ++sl) {
+      const int stg = sl % kStages;
+      if (!mbar_wait_warp(&bar_conv[stg], (uint32_t)((sl / kStages) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t base = smem_u32(smem + stg * kStageBytes);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < kSlab / 16; ++kk) {
           const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
@@ -242,8 +245,10 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         }
         mma_commit(&bar_mma[stg]);
       }
-      mma_commit(bar_done);  // tracks every MMA issued above (completes at once if none)
+      __syncwarp();
     }
+    if (elect_one()) mma_commit(bar_done);  // tracks every MMA issued above
+    __syncwarp();
   } else {
     // ---------------- converters (warps 0..15) ----------------
     float zr[8];
@@ -408,14 +413,20 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
   bool ok = true;
 
   if (warp == 4) {
-    if (lane == 0 && delta) {
+    // The whole warp runs the loop and waits; one elected lane (always lane 0)
+    // issues the copies, MMAs and commits.
+    if (delta) {
       // G_s of chunk c: plane (bh*S + s)*CH*2 + 2c + 1 of dpart
       auto load_g = [&](int s, int c, int buf) {
-        mbar_arrive_expect_tx(&bar_g[buf], kGBytes);
-        const int plane = ((bh * S + s) * CH + c) * 2 + 1;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(&bar_g[buf], kGBytes);
+          const int plane = ((bh * S + s) * CH + c) * 2 + 1;
 #pragma unroll
-        for (int bx = 0; bx < 4; ++bx)
-          tma_load_3d(sG + buf * kGBytes + bx * (D * 128), &tm_g, &bar_g[buf], bx * 32, 0, plane);
+          for (int bx = 0; bx < 4; ++bx)
+            tma_load_3d(sG + buf * kGBytes + bx * (D * 128), &tm_g, &bar_g[buf], bx * 32, 0,
+                        plane);
+        }
+        __syncwarp();
       };
       const uint32_t idesc = idesc_f32acc(2, 0, 0, 128, 32);
       int n = 0;  // G loads consumed so far
@@ -423,7 +434,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
       load_g(0, 0, 0);
       for (int s = 0; s < S && ok; ++s) {
         // M^T of this segment's M_{s-1} must be in shared memory
-        if (!mbar_wait(bar_mt, (uint32_t)(s & 1))) {
+        if (!mbar_wait_warp(bar_mt, (uint32_t)(s & 1))) {
           ok = false;
           break;
         }
@@ -434,22 +445,25 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
             // this point (its commit was awaited below)
             load_g((n + 1) / CH, (n + 1) % CH, buf ^ 1);
           }
-          if (!mbar_wait(&bar_g[buf], (uint32_t)((n >> 1) & 1))) {
+          if (!mbar_wait_warp(&bar_g[buf], (uint32_t)((n >> 1) & 1))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t ga = smem_u32(sG + buf * kGBytes), mb = smem_u32(sMt);
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 8; ++kk) {
-            const uint32_t koff = (uint32_t)(kk >> 2) * (D * 128) + (uint32_t)(kk & 3) * 32;
-            const uint32_t moff = (uint32_t)(kk >> 2) * (32 * 128) + (uint32_t)(kk & 3) * 32;
-            mma_tf32_ss(tmem_d, sdesc(ga + koff, 16, 1024), sdesc(mb + moff, 16, 1024), idesc,
-                        (c > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < D / 8; ++kk) {
+              const uint32_t koff = (uint32_t)(kk >> 2) * (D * 128) + (uint32_t)(kk & 3) * 32;
+              const uint32_t moff = (uint32_t)(kk >> 2) * (32 * 128) + (uint32_t)(kk & 3) * 32;
+              mma_tf32_ss(tmem_d, sdesc(ga + koff, 16, 1024), sdesc(mb + moff, 16, 1024), idesc,
+                          (c > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(bar_mma);
+            if (c == CH - 1) mma_commit(bar_seg);
           }
-          mma_commit(bar_mma);
-          if (c == CH - 1) mma_commit(bar_seg);
-          if (!mbar_wait(bar_mma, (uint32_t)(n & 1))) {
+          __syncwarp();
+          if (!mbar_wait_warp(bar_mma, (uint32_t)(n & 1))) {
             ok = false;
             break;
           }
