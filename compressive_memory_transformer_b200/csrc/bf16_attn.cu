@@ -399,19 +399,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     long long kc = 0;
     int tc = 0;
     bool ok = true;
-    TileIter it;
-    it.init();
-    Tile t;
-    while (ok && it.next(p, t)) {
-      const float bta = __ldg(beta + t.bh % p.H);  // used in the epilogue
+    // sigma(Q) of tile number tile_no (this thread's 64 columns) -> tensor memory
+    // (O + 64 half, 32 packed columns) for the retrieval MMA; partial denominator
+    // sigma(Q_r) . z_{s-1} over those columns.
+    auto sigma_q = [&](int tile_no, float& den) -> bool {
+      if (!mbar_wait_warp(&bars[B_QFULL], (uint32_t)(tile_no & 1))) return false;
       const float* zs = sZ + col0;
-      if (!mbar_wait_warp(&bars[B_QFULL], (uint32_t)(tc & 1))) {
-        ok = false;
-        break;
-      }
-      // sigma(Q) of this thread's 64 columns -> tensor memory (O + 64 half, 32 packed
-      // columns); partial denominator sigma(Q_r) . z_{s-1} over those columns
-      float den = 0.f;
+      den = 0.f;
       uint32_t sq[32];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -421,24 +415,30 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const float4 z1 = *reinterpret_cast<const float4*>(zs + u * 8 + 4);
         const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
         const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-        uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __bfloat1622float2(h[e]);
           const float p0 = elu1(f.x), p1 = elu1(f.y);
           den = fmaf(p0, zz[2 * e], den);
           den = fmaf(p1, zz[2 * e + 1], den);
-          pk[e] = pack_bf16x2(p0, p1);
+          sq[4 * u + e] = pack_bf16x2(p0, p1);
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sq[4 * u + e] = pk[e];
       }
       mbar_arrive_warp(&bars[B_QEMPTY]);  // this warp is done reading Q
       tmem_st32_(tO + lane_off + 64 * half, sq);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(&bars[B_SQFULL]);
-
+      return true;
+    };
+    TileIter it;
+    it.init();
+    Tile t, tn;
+    bool have = it.next(p, t);
+    float den = 0.f;
+    if (have) ok = sigma_q(0, den);
+    while (ok && have) {
+      const float bta = __ldg(beta + t.bh % p.H);  // used in the epilogue
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < t.nkv; ++j) {
         const int b = (int)(kc & 1);
@@ -538,13 +538,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       if (!ok) break;
 
       // ---- epilogue: out = (1 - g) O / l + g R / den ----
-      if (!mbar_wait_warp(&bars[B_PVDONE], (uint32_t)((kc - 1) & 1)) ||
-          !mbar_wait_warp(&bars[B_RDONE], (uint32_t)(tc & 1))) {
-        ok = false;
-        break;
-      }
-      const float g = 1.f / (1.f + expf(-bta));
-      tc_fence_after();
+      // The row sum and denominator halves do not depend on the MMAs: exchange
+      // them first. Then O and R become packed outputs in registers, the next
+      // tile's sigma(Q) goes into O (the retrieval MMA waits for it), and the
+      // global stores of this tile come last, overlapping the next tile's MMAs.
       xden[half * 128 + r] = den;
       xl[half * 128 + r] = l;
       mbar_arrive_warp(pair);
@@ -553,32 +550,46 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         break;
       }
       ++pair_phase;
+      const float g = 1.f / (1.f + expf(-bta));
       const float den_t = den + xden[(1 - half) * 128 + r];
       const float l_t = l + xl[(1 - half) * 128 + r];
       const float go = (1.f - g) / l_t;
       const float gr = den_t != 0.f ? g / den_t : 0.f;
-      __nv_bfloat16* orow = out + ((size_t)t.bh * p.L + t.q_row + r) * D + col0;
+      if (!mbar_wait_warp(&bars[B_PVDONE], (uint32_t)((kc - 1) & 1)) ||
+          !mbar_wait_warp(&bars[B_RDONE], (uint32_t)(tc & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t w[32];  // this row's 64 outputs, bf16 pairs
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t o[32], rr[32];
         tmem_ld32(tO + lane_off + col0 + c * 32, o);
         tmem_ld32(tR + lane_off + col0 + c * 32, rr);
         tmem_wait_ld();
-        uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float a0 = go * __uint_as_float(o[2 * e]) + gr * __uint_as_float(rr[2 * e]);
           const float a1 = go * __uint_as_float(o[2 * e + 1]) + gr * __uint_as_float(rr[2 * e + 1]);
-          w[e] = pack_bf16x2(a0, a1);
-        }
-        if (r < t.rows_valid) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) =
-                make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+          w[16 * c + e] = pack_bf16x2(a0, a1);
         }
       }
       tc_fence_before();
+      const bool has_next = it.next(p, tn);
+      if (has_next && !sigma_q(tc + 1, den)) {
+        ok = false;
+        break;
+      }
+      if (r < t.rows_valid) {
+        __nv_bfloat16* orow = out + ((size_t)t.bh * p.L + t.q_row + r) * D + col0;
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<uint4*>(orow + q4 * 8) =
+              make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+      }
+      t = tn;
+      have = has_next;
       ++tc;
     }
   }
