@@ -23,10 +23,16 @@ void bf16_state_plan(int BH, int S, int N, int* CH, int* CL);
 size_t bf16_workspace_bytes(int BH, int S, int CH);
 Bf16Workspace bf16_workspace_carve(void* base, int BH, int S, int CH);
 
+// The state path. Segments s < first (0 or 1) of the workspace's M_{s-1} hi/lo
+// and z_{s-1} are taken as already written (by bf16_prep_first) and not rewritten.
 cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, const float* M_in,
                               const float* z_in, float* M_out, float* z_out,
                               const Bf16Workspace& ws, int BH, long long L, int N, int S, int CH,
-                              int CL, int mode, cudaStream_t stream);
+                              int CL, int mode, int first, cudaStream_t stream);
+
+// Writes the workspace's first-segment M_{-1} hi/lo and z_{-1} from M_in / z_in.
+cudaError_t bf16_prep_first(const float* M_in, const float* z_in, const Bf16Workspace& ws,
+                            int BH, int S, cudaStream_t stream);
 
 // The fused local-attention + retrieval + gate kernel. Reads q, k, v, beta and
 // the workspace's zprev / Mhl; writes out.
@@ -35,8 +41,5 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                              const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
                              cudaStream_t stream);
 
-// Sets the dynamic shared-memory limits of the kernels on the current device
-// (once per device).
-cudaError_t bf16_prepare_device();
 
 }  // namespace infini

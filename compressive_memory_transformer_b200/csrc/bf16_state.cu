@@ -90,11 +90,12 @@ __global__ void __launch_bounds__(256) zpart_kernel(const __nv_bfloat16* __restr
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(D) zscan_kernel(const float* __restrict__ zpart,
                                                   const float* z_in, float* z_out,
-                                                  float* __restrict__ zprev, int S, int CH) {
+                                                  float* __restrict__ zprev, int S, int CH,
+                                                  int first) {
   const int bh = blockIdx.x, kf = threadIdx.x;
   float z = z_in ? z_in[(size_t)bh * D + kf] : 0.f;
   for (int s = 0; s < S; ++s) {
-    zprev[((size_t)bh * S + s) * D + kf] = z;
+    if (s >= first) zprev[((size_t)bh * S + s) * D + kf] = z;
     const float* zp = zpart + ((size_t)bh * S + s) * CH * D + kf;
     for (int c = 0; c < CH; ++c) z += zp[(size_t)c * D];
   }
@@ -383,7 +384,7 @@ constexpr int kChainSmem = 2 * kGBytes + kMtBytes + 1024 + 256;
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__ dpart,
              const float* M_in, float* M_out, __nv_bfloat16* __restrict__ Mhl, int S, int CH,
-             int mode) {
+             int mode, int first) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -511,22 +512,25 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
     };
     if (S > 0) load_dm(0);
     for (int s = 0; s < S; ++s) {
-      // M_{s-1} -> hi / lo bf16
-      __nv_bfloat16* hi = Mhl + ((size_t)bh * S + s) * 2 * D * D + (size_t)r * D + c0;
-      __nv_bfloat16* lo = hi + D * D;
+      // M_{s-1} -> hi / lo bf16 (segments below `first` were written by prep_first_kernel)
+      if (s >= first) {
+        __nv_bfloat16* hi = Mhl + ((size_t)bh * S + s) * 2 * D * D + (size_t)r * D + c0;
+        __nv_bfloat16* lo = hi + D * D;
 #pragma unroll
-      for (int e = 0; e < 32; e += 8) {
-        uint32_t h4[4], l4[4];
+        for (int e = 0; e < 32; e += 8) {
+          uint32_t h4[4], l4[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const __nv_bfloat162 h = __floats2bfloat162_rn(m[e + 2 * q], m[e + 2 * q + 1]);
-          const float2 hf = __bfloat1622float2(h);
-          const __nv_bfloat162 l = __floats2bfloat162_rn(m[e + 2 * q] - hf.x, m[e + 2 * q + 1] - hf.y);
-          h4[q] = *reinterpret_cast<const uint32_t*>(&h);
-          l4[q] = *reinterpret_cast<const uint32_t*>(&l);
+          for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(m[e + 2 * q], m[e + 2 * q + 1]);
+            const float2 hf = __bfloat1622float2(h);
+            const __nv_bfloat162 l =
+                __floats2bfloat162_rn(m[e + 2 * q] - hf.x, m[e + 2 * q + 1] - hf.y);
+            h4[q] = *reinterpret_cast<const uint32_t*>(&h);
+            l4[q] = *reinterpret_cast<const uint32_t*>(&l);
+          }
+          *reinterpret_cast<uint4*>(hi + e) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+          *reinterpret_cast<uint4*>(lo + e) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
         }
-        *reinterpret_cast<uint4*>(hi + e) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-        *reinterpret_cast<uint4*>(lo + e) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
       }
       float dm[32];
 #pragma unroll
@@ -573,14 +577,54 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
   }
 }
 
+// prep_first_kernel: grid = BH, block 128. Writes what the attention kernel reads
+// for the first segment, M_{-1} = M_in as hi / lo bf16 and z_{-1} = z_in (zero when
+// absent), exactly as chain_kernel and zscan_kernel would, so that a one-segment
+// call can run the attention beside the state update.
+__global__ void __launch_bounds__(D) prep_first_kernel(const float* M_in, const float* z_in,
+                                                       __nv_bfloat16* __restrict__ Mhl,
+                                                       float* __restrict__ zprev, int S) {
+  const int bh = blockIdx.x, r = threadIdx.x;
+  __nv_bfloat16* hi = Mhl + (size_t)bh * S * 2 * D * D + (size_t)r * D;
+  __nv_bfloat16* lo = hi + D * D;
+  const float* src = M_in ? M_in + ((size_t)bh * D + r) * D : nullptr;
+#pragma unroll 4
+  for (int e = 0; e < D; e += 8) {
+    float m[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) m[q] = src ? src[e + q] : 0.f;
+    uint32_t h4[4], l4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(m[2 * q], m[2 * q + 1]);
+      const float2 hf = __bfloat1622float2(h);
+      const __nv_bfloat162 l = __floats2bfloat162_rn(m[2 * q] - hf.x, m[2 * q + 1] - hf.y);
+      h4[q] = *reinterpret_cast<const uint32_t*>(&h);
+      l4[q] = *reinterpret_cast<const uint32_t*>(&l);
+    }
+    *reinterpret_cast<uint4*>(hi + e) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+    *reinterpret_cast<uint4*>(lo + e) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+  }
+  zprev[(size_t)bh * S * D + r] = z_in ? z_in[(size_t)bh * D + r] : 0.f;
+}
+
 }  // namespace
+
+cudaError_t bf16_prep_first(const float* M_in, const float* z_in, const Bf16Workspace& ws,
+                            int BH, int S, cudaStream_t stream) {
+  prep_first_kernel<<<BH, D, 0, stream>>>(M_in, z_in, ws.Mhl, ws.zprev, S);
+  return cudaGetLastError();
+}
 
 void bf16_state_plan(int BH, int S, int N, int* CH, int* CL) {
   // Chunk the segments so that the state GEMM has at least ~2 CTAs per SM, with
   // chunks of at least 128 tokens.
   const long long units = (long long)BH * S;
   int ch = 1;
-  const int maxch = N >= 128 ? N / 128 : 1;
+  // At most 8 chunks: the chain adds each chunk's G M in turn (one segment's
+  // chunks in sequence), which outweighs a more parallel state GEMM beyond that
+  // (one-segment steps of 2048 tokens: 8 chunks 69 us per step, 16 chunks 75 us).
+  const int maxch = N >= 128 ? (N / 128 < 8 ? N / 128 : 8) : 1;
   while (units * ch < 296 && ch * 2 <= maxch) ch *= 2;
   *CH = ch;
   *CL = (N + ch - 1) / ch;
@@ -619,7 +663,7 @@ Bf16Workspace bf16_workspace_carve(void* base, int BH, int S, int CH) {
 cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, const float* M_in,
                               const float* z_in, float* M_out, float* z_out,
                               const Bf16Workspace& ws, int BH, long long L, int N, int S, int CH,
-                              int CL, int mode, cudaStream_t stream) {
+                              int CL, int mode, int first, cudaStream_t stream) {
   const unsigned nunits = (unsigned)((long long)BH * S * CH);
   CUtensorMap mk, mv;
   if (!make_bf16_map(&mk, k, (uint64_t)L, BH, kSlab) || !make_bf16_map(&mv, v, (uint64_t)L, BH, kSlab))
@@ -627,14 +671,14 @@ cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, co
   if (mode == 1) {
     // Linear+Delta needs z_{s-1} (hence every segment's sum of sigma(K)) first
     zpart_kernel<<<nunits, 256, 0, stream>>>(k, ws.zpart, L, N, S, CH, CL);
-    zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH);
+    zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH, first);
     state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(mk, mv, ws.zprev, ws.dpart,
                                                                  ws.zpart, L, N, S, CH, CL, mode);
   } else {
     // Linear: the state GEMM also produces the sums of sigma(K)
     state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(mk, mv, ws.zprev, ws.dpart,
                                                                  ws.zpart, L, N, S, CH, CL, mode);
-    zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH);
+    zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH, first);
   }
   CUtensorMap mg;
   if (mode == 1) {
@@ -653,7 +697,7 @@ cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, co
     memset(&mg, 0, sizeof(mg));
   }
   chain_kernel<<<dim3(BH, 4), kChainThreads, kChainSmem, stream>>>(mg, ws.dpart, M_in, M_out,
-                                                                    ws.Mhl, S, CH, mode);
+                                                                    ws.Mhl, S, CH, mode, first);
   return cudaGetLastError();
 }
 

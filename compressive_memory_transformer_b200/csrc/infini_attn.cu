@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "infini_attn.h"
 #include "bf16_path.h"
@@ -26,15 +27,34 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_prepared[kMaxDevices];
+std::mutex g_prepare_mu;
 
-cudaError_t prepare_device() {
+// A second stream of each device, for one-segment calls: the state update runs on
+// it beside the attention kernel, forked from and joined back into the caller's
+// stream inside the call. The mutex keeps each fork..join sequence whole when
+// several host threads call at once.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex mu;
+};
+SideStream g_side[kMaxDevices];
+
+cudaError_t prepare_device(int* dev_out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  *dev_out = dev;
+  if (g_prepared[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  std::lock_guard<std::mutex> lk(g_prepare_mu);
   if (g_prepared[dev].load(std::memory_order_acquire)) return cudaSuccess;
   e = bf16_state_set_attributes();
   if (e == cudaSuccess) e = bf16_attn_set_attributes();
+  SideStream& sd = g_side[dev];
+  if (e == cudaSuccess && !sd.stream) e = cudaStreamCreateWithFlags(&sd.stream, cudaStreamNonBlocking);
+  if (e == cudaSuccess && !sd.fork) e = cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming);
+  if (e == cudaSuccess && !sd.join) e = cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming);
   if (e == cudaSuccess) g_prepared[dev].store(1, std::memory_order_release);
   return e;
 }
@@ -165,7 +185,8 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
     record(opts, 2, stream);
     return st;
   }
-  if (prepare_device() != cudaSuccess) return INFINI_ERR_CUDA;
+  int dev = 0;
+  if (prepare_device(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
   const int S = (int)((L + N - 1) / N);
   if (dtype == INFINI_DTYPE_F32) {
     Scratch sc;
@@ -191,8 +212,31 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
   const auto* vb = static_cast<const __nv_bfloat16*>(v);
   record(opts, 0, stream);
+  if (S == 1) {
+    // One segment: the attention reads only the incoming state (M_in, z_in), so it
+    // runs beside the state update, which goes to the side stream and is joined
+    // back before the call returns.
+    SideStream& sd = g_side[dev];
+    std::lock_guard<std::mutex> lk(sd.mu);
+    cudaError_t e = bf16_prep_first(M_in, z_in, ws, BH, S, stream);
+    if (e == cudaSuccess) e = cudaEventRecord(sd.fork, stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sd.stream, sd.fork, 0);
+    if (e != cudaSuccess) return INFINI_ERR_CUDA;
+    const cudaError_t es = bf16_state_launch(kb, vb, M_in, z_in, M_out, z_out, ws, BH, L, N, S,
+                                             CH, CL, mode, 1, sd.stream);
+    record(opts, 1, stream);
+    const cudaError_t ea = bf16_attn_launch(qb, kb, vb, beta, static_cast<__nv_bfloat16*>(out),
+                                            ws, BH, H, L, N, S, stream);
+    // joined even after a launch error, so that the side stream never runs ahead of
+    // the caller's stream
+    cudaError_t ej = cudaEventRecord(sd.join, sd.stream);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(stream, sd.join, 0);
+    record(opts, 2, stream);
+    return es == cudaSuccess && ea == cudaSuccess && ej == cudaSuccess ? INFINI_OK
+                                                                        : INFINI_ERR_CUDA;
+  }
   cudaError_t e = bf16_state_launch(kb, vb, M_in, z_in, M_out, z_out, ws, BH, L, N, S, CH, CL,
-                                    mode, stream);
+                                    mode, 0, stream);
   if (e != cudaSuccess) return INFINI_ERR_CUDA;
   record(opts, 1, stream);
   e = bf16_attn_launch(qb, kb, vb, beta, static_cast<__nv_bfloat16*>(out), ws, BH, H, L, N, S,

@@ -111,7 +111,7 @@ extern "C" int infini_attn_step_static(const void* q, const void* k, const void*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
   const auto* vb = static_cast<const __nv_bfloat16*>(v);
-  if (bf16_state_launch(kb, vb, M_in, z_in, M_out, z_out, ws, BH, N, N, S, CH, CL, mode, st) !=
+  if (bf16_state_launch(kb, vb, M_in, z_in, M_out, z_out, ws, BH, N, N, S, CH, CL, mode, 0, st) !=
       cudaSuccess)
     return INFINI_ERR_CUDA;
   if (bf16_attn_launch(static_cast<const __nv_bfloat16*>(q), kb, vb, beta,

@@ -128,7 +128,11 @@ int infini_attn_step_f32(const float* q, const float* k, const float* v, const f
  *     library uses the stream-ordered allocator as infini_attn_forward does.
  *   stage_events[0..2]: cudaEvent_t handles (or NULL) recorded on `stream`
  *     before the state kernels, between the state kernels and the fused
- *     attention kernel, and after the fused attention kernel.
+ *     attention kernel, and after the fused attention kernel. When the call
+ *     holds a single segment (L <= N), the attention reads only the incoming
+ *     state and the state update runs beside it on a second stream of the
+ *     library (forked from and joined back into `stream` within the call):
+ *     event 1 then marks the fork, event 2 the point where both are done.
  */
 typedef struct {
   void* workspace;
