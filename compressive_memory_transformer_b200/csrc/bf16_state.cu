@@ -154,7 +154,8 @@ __device__ __forceinline__ uint64_t slab_desc(uint32_t base, int kk) {
 __global__ void __launch_bounds__(kStateThreads, 1)
 state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const float* __restrict__ zprev, float* __restrict__ dpart,
-             float* __restrict__ zpart, long long L, int N, int S, int CH, int CL, int mode) {
+             float* __restrict__ zpart, long long L, int N, int S, int CH, int CL, int mode,
+             int zsum) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -345,7 +346,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         }
       }
     }
-    if (!delta) {
+    if (zsum) {
       // chunk sum of sigma(K): threads with the same feature group add up
 #pragma unroll
       for (int e = 0; e < 8; ++e) sZred[r * 128 + cg * 8 + e] = dz[e];
@@ -353,7 +354,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   }
   tc_fence_before();
   __syncthreads();
-  if (!delta && tid < D) {
+  if (zsum && tid < D) {
     float sum = 0.f;
 #pragma unroll
     for (int rr = 0; rr < kConvRows; ++rr) sum += sZred[rr * 128 + tid];
@@ -577,42 +578,48 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
   }
 }
 
-// prep_first_kernel: grid = BH, block 128. Writes what the attention kernel reads
-// for the first segment, M_{-1} = M_in as hi / lo bf16 and z_{-1} = z_in (zero when
-// absent), exactly as chain_kernel and zscan_kernel would, so that a one-segment
-// call can run the attention beside the state update.
+// prep_first_kernel: grid = (BH, 16), block 128; block y covers rows 8y .. 8y+7.
+// Writes what the attention kernel reads for the first segment, M_{-1} = M_in as
+// hi / lo bf16 and z_{-1} = z_in (zero when absent), exactly as chain_kernel and
+// zscan_kernel would, so that a one-segment call can run the attention beside the
+// state update.
 __global__ void __launch_bounds__(D) prep_first_kernel(const float* M_in, const float* z_in,
                                                        __nv_bfloat16* __restrict__ Mhl,
                                                        float* __restrict__ zprev, int S) {
-  const int bh = blockIdx.x, r = threadIdx.x;
-  __nv_bfloat16* hi = Mhl + (size_t)bh * S * 2 * D * D + (size_t)r * D;
-  __nv_bfloat16* lo = hi + D * D;
-  const float* src = M_in ? M_in + ((size_t)bh * D + r) * D : nullptr;
-#pragma unroll 4
-  for (int e = 0; e < D; e += 8) {
-    float m[8];
+  const int bh = blockIdx.x, r = blockIdx.y * 8 + (threadIdx.x >> 4), c = (threadIdx.x & 15) * 8;
+  float m[8];
+  if (M_in) {
+    const float4* src = reinterpret_cast<const float4*>(M_in + ((size_t)bh * D + r) * D + c);
+    const float4 a0 = src[0], a1 = src[1];
+    m[0] = a0.x; m[1] = a0.y; m[2] = a0.z; m[3] = a0.w;
+    m[4] = a1.x; m[5] = a1.y; m[6] = a1.z; m[7] = a1.w;
+  } else {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) m[q] = src ? src[e + q] : 0.f;
-    uint32_t h4[4], l4[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const __nv_bfloat162 h = __floats2bfloat162_rn(m[2 * q], m[2 * q + 1]);
-      const float2 hf = __bfloat1622float2(h);
-      const __nv_bfloat162 l = __floats2bfloat162_rn(m[2 * q] - hf.x, m[2 * q + 1] - hf.y);
-      h4[q] = *reinterpret_cast<const uint32_t*>(&h);
-      l4[q] = *reinterpret_cast<const uint32_t*>(&l);
-    }
-    *reinterpret_cast<uint4*>(hi + e) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-    *reinterpret_cast<uint4*>(lo + e) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+    for (int q = 0; q < 8; ++q) m[q] = 0.f;
   }
-  zprev[(size_t)bh * S * D + r] = z_in ? z_in[(size_t)bh * D + r] : 0.f;
+  uint32_t h4[4], l4[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(m[2 * q], m[2 * q + 1]);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(m[2 * q] - hf.x, m[2 * q + 1] - hf.y);
+    h4[q] = *reinterpret_cast<const uint32_t*>(&h);
+    l4[q] = *reinterpret_cast<const uint32_t*>(&l);
+  }
+  __nv_bfloat16* hi = Mhl + (size_t)bh * S * 2 * D * D + (size_t)r * D + c;
+  *reinterpret_cast<uint4*>(hi) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+  *reinterpret_cast<uint4*>(hi + D * D) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+  if (blockIdx.y == 0) {
+    const int f = threadIdx.x;
+    zprev[(size_t)bh * S * D + f] = z_in ? z_in[(size_t)bh * D + f] : 0.f;
+  }
 }
 
 }  // namespace
 
 cudaError_t bf16_prep_first(const float* M_in, const float* z_in, const Bf16Workspace& ws,
                             int BH, int S, cudaStream_t stream) {
-  prep_first_kernel<<<BH, D, 0, stream>>>(M_in, z_in, ws.Mhl, ws.zprev, S);
+  prep_first_kernel<<<dim3(BH, D / 8), D, 0, stream>>>(M_in, z_in, ws.Mhl, ws.zprev, S);
   return cudaGetLastError();
 }
 
@@ -668,16 +675,17 @@ cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, co
   CUtensorMap mk, mv;
   if (!make_bf16_map(&mk, k, (uint64_t)L, BH, kSlab) || !make_bf16_map(&mv, v, (uint64_t)L, BH, kSlab))
     return cudaErrorInvalidValue;
-  if (mode == 1) {
+  if (mode == 1 && !(first == 1 && S == 1)) {
     // Linear+Delta needs z_{s-1} (hence every segment's sum of sigma(K)) first
     zpart_kernel<<<nunits, 256, 0, stream>>>(k, ws.zpart, L, N, S, CH, CL);
     zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH, first);
-    state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(mk, mv, ws.zprev, ws.dpart,
-                                                                 ws.zpart, L, N, S, CH, CL, mode);
+    state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(
+        mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 0);
   } else {
-    // Linear: the state GEMM also produces the sums of sigma(K)
-    state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(mk, mv, ws.zprev, ws.dpart,
-                                                                 ws.zpart, L, N, S, CH, CL, mode);
+    // The state GEMM also produces the sums of sigma(K): always in Linear mode, and
+    // in Linear+Delta mode for a lone segment whose z_{-1} is already in place
+    state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(
+        mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 1);
     zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH, first);
   }
   CUtensorMap mg;
