@@ -38,7 +38,9 @@ UNIT = "tokens/s"
 B, H, D, N, L = 4, 8, 128, 2048, 32768
 WORKLOAD = (f"1B-LM layer shape: B={B}, H={H}, d={D}, N={N}, L={L} ({L // N} segments), "
             "bf16 q/k/v, fp32 state from zero; step = Linear forward + Linear+Delta forward")
-LAUNCHES_PER_FORWARD = 5   # zpart, zscan, state, chain, attn
+# kernels per forward of the workload (several segments): Linear state, zscan, chain,
+# attn; Linear+Delta zpart, zscan, state, chain, attn
+LAUNCHES_PER_STEP = 4 + 5
 
 
 def attn_flops_per_launch():
@@ -326,7 +328,7 @@ def run_ours(args, rank, world, device):
             "delta": {"tokens_per_s": B * L / (fwd_ms[1] / 1e3), "forward_ms": fwd_ms[1],
                       "state_kernels_ms": state_ms[1]},
         },
-        "gpu_launches": args.steps * 2 * LAUNCHES_PER_FORWARD,
+        "gpu_launches": args.steps * LAUNCHES_PER_STEP,
         "clocks": clk,
     }
     if e2e is not None:
