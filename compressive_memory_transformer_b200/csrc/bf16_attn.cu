@@ -85,6 +85,7 @@ struct Params {
   long long L;
   int N, S, H, T, U, BH;
   long long units;
+  int out32;  // out is 32-byte aligned: rows are stored as whole 32-byte sectors
 };
 
 // One query tile of the work list.
@@ -583,10 +584,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
       if (r < t.rows_valid) {
         __nv_bfloat16* orow = out + ((size_t)t.bh * p.L + t.q_row + r) * D + col0;
+        if (p.out32) {
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          *reinterpret_cast<uint4*>(orow + q4 * 8) =
-              make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+          for (int q8 = 0; q8 < 4; ++q8) st_global_v8(orow + q8 * 16, w + 8 * q8);
+        } else {
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            *reinterpret_cast<uint4*>(orow + q4 * 8) =
+                make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+        }
       }
       t = tn;
       have = has_next;
@@ -627,6 +633,7 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   p.T = (int)((min((long long)N, L) + BM - 1) / BM);
   p.U = (p.T + 1) / 2;
   p.units = (long long)BH * S * p.U;
+  p.out32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

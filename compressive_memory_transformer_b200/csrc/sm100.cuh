@@ -403,6 +403,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// One 32-byte global store (a whole L2 sector); the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 // Byte offset of the 16-byte unit u (0..7) of row r inside a 128B-swizzled
 // region whose rows are 128 bytes apart (region base 1024-byte aligned).
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t u) {

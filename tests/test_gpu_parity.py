@@ -219,6 +219,22 @@ def test_bf16_steps_under_graph_capture(ia, mode):
     check_bf16(torch.cat(o1, dim=2), M1, z1, ref, what=f"graph steps mode={mode}")
 
 
+def test_bf16_output_only_16_byte_aligned(ia):
+    """The attention kernel stores rows as 32-byte sectors when `out` allows it;
+    an `out` aligned to 16 bytes only takes the 16-byte stores, same result."""
+    B, H, L, N = 1, 2, 512, 256
+    inp = make_inputs(B, H, L, 128, torch.bfloat16, seed=51, device="cuda", gen_device="cpu")
+    n = B * H * L * 128
+    buf = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    out16 = buf[8:].view(B, H, L, 128)
+    assert out16.data_ptr() % 32 == 16
+    for mode in (LIN, DEL):
+        ref_out, _, _ = ia.infini_attn_forward(inp["q"], inp["k"], inp["v"], inp["beta"], N, mode)
+        ia.infini_attn_forward(inp["q"], inp["k"], inp["v"], inp["beta"], N, mode, out=out16)
+        sync_ok(ia)
+        assert torch.equal(out16, ref_out)
+
+
 def test_bf16_empty_sequence_passes_state(ia):
     B, H = 1, 2
     e = torch.empty((B, H, 0, 128), dtype=torch.bfloat16, device="cuda")
