@@ -13,15 +13,18 @@
 // holds T+1 key tiles of work; units are dealt out round-robin in segment order,
 // so the ~150 units in flight touch ~20 segments and their K/V stay in L2.
 // Every pipeline runs on across tiles: while the softmax warps finish one tile,
-// the producer already loads the next Q and K tiles and the MMA thread issues
-// the next tile's first two Q K^T products.
+// the producer already loads the next Q (prefetched into L2 a tile earlier) and K
+// tiles and the next tile's first Q K^T products are issued.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warp 0     TMA producer: Q per tile (reloaded once the last Q K^T of the tile
-//              and sigma(Q) are done); a K ring (2 stages); a V ring (3 stages)
-//              whose items per tile are M_hi, M_lo (the state, hi and lo bf16
-//              halves), then V_0, V_1, ...
-//   warp 1     tensor-memory allocation and the MMA issue (one elected lane).
+//              and sigma(Q) are done) together with the tile's descriptor (a shared
+//              memory slot, so no other role walks the work list); a K ring (2
+//              stages); a V ring (3 stages) whose items per tile are M_hi (the
+//              state rounded to bf16), then V_0, V_1, ...
+//   warp 1     tensor-memory allocation; issues the retrieval and P V products.
+//   warp 10    issues the Q K^T products (another scheduler than warp 1, so each
+//              issuing warp carries half of the per-key-tile instruction stream).
 //   warps 2-9  softmax / epilogue, two warpgroups: query row r (tensor-memory lane r)
 //              is shared by one thread of each; warpgroup h owns key columns
 //              [64h, 64h + 64) of S and value columns [64h, 64h + 64) of O, R and out.
@@ -33,11 +36,12 @@
 // sequence) | O (A_dot accumulator) | R (sigma(Q) M accumulator). P (bf16) is
 // written over the first 64 columns of its S buffer and read from there by the PV
 // MMA; sigma(Q) (bf16) is staged in O, each half in its own columns, for the
-// retrieval MMA before the tile's first PV overwrites O. Tensor-core operations
-// issued by the one MMA thread execute in issue order, which orders every read of
-// an aliased region before the next write to it.
-// MMA order per tile: R = sigma(Q)(M_hi + M_lo); for each j: O += P_j V_j, then
-// Q K_{j+2}^T; after the last PV, the next tile's Q K_0^T and Q K_1^T.
+// retrieval MMA before the tile's first PV overwrites O.
+// Tensor-core operations from one issuing thread execute in issue order: warp 1's
+// retrieval precedes the tile's first P V (which overwrites the staged sigma(Q)).
+// Across the two issuing warps the order is explicit: the Q K^T of key step n
+// overwrites the S buffer that held P of step n - 2, so it waits for that step's
+// P V through the buffer's S-free barrier.
 // Every mbarrier is waited on in completion order and can never complete twice
 // before its waiter has seen the first completion (a parity wait would then
 // miss it): sigma(Q) and P have separate barriers; P_{j+1} is written only after
@@ -45,7 +49,10 @@
 // R and the last PV done. z_{s-1} (512 B) rides on the Q barrier.
 // Online softmax keeps a per-row reference max and rescales O only when the
 // running max grows by more than 2^8 (in exp2 units). One exponential in four is
-// evaluated on the FMA pipe (ex2_poly2) to offload the MUFU unit.
+// evaluated on the FMA pipe (ex2_poly2) to offload the MUFU unit. The retrieval
+// uses M rounded to one bf16 term: A_mem is a weighted average over the 128 rows
+// of M, so the independent per-element roundings (relative 2^-9) average out to
+// ~5e-5 of the output, far inside the bf16 output tolerance.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda.h>
@@ -70,13 +77,14 @@ constexpr int OFF_V = 3 * kTile;     // kVStages stages
 constexpr int OFF_X = 6 * kTile;     // exchange: max [2][2][128], den [2][128], l [2][128]
 constexpr int OFF_Z = OFF_X + 4096;   // z_{s-1} of the current tile (128 floats), loaded with Q
 constexpr int OFF_BAR = OFF_Z + 512;
-constexpr int kAttnSmem = OFF_BAR + 256 + 1024;  // + alignment slack
-constexpr int kThreads = 320;
+constexpr int OFF_SLOT = OFF_BAR + 256;  // two tile descriptors
+constexpr int kAttnSmem = OFF_SLOT + 128 + 1024;  // + alignment slack
+constexpr int kThreads = 352;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kSoftmaxWarps = 8;
 
 enum {
-  B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = 4, B_VFULL = 6 /* 3 */, B_VEMPTY = 9 /* 3 */,
+  B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_SFREE = 4 /* 2 */, B_VFULL = 6 /* 3 */, B_VEMPTY = 9 /* 3 */,
   B_SFULL = 12, B_PFULL = 14, B_PVDONE = 15, B_DRAIN = 16, B_PAIR = 17 /* 4 */, B_RDONE = 21,
   B_SQFULL = 22, B_COUNT = 23
 };
@@ -84,21 +92,22 @@ enum {
 struct Params {
   long long L;
   int N, S, H, T, U, BH;
-  long long units;
+  unsigned units;  // BH * S * U, below 2^31
+  FastDiv divU, divS;
   int out32;  // out is 32-byte aligned: rows are stored as whole 32-byte sectors
 };
 
-// One query tile of the work list.
+// One query tile of the work list (valid = 0: the end of the CTA's list).
 struct Tile {
-  int bh, s, i, nkv, q_row, rows_valid;
   long long seg0;
+  int bh, s, i, nkv, q_row, rows_valid, h, valid;
 };
 
 // Walks the CTA's tiles: units blockIdx.x, blockIdx.x + gridDim.x, ...; unit u of
 // a segment holds tiles T-1-u and u (one tile when they coincide); tiles past the
 // end of a short final segment are skipped.
 struct TileIter {
-  long long unit;
+  unsigned unit;
   int k;  // 0: tile T-1-u, 1: tile u
   __device__ void init() {
     unit = blockIdx.x;
@@ -106,8 +115,8 @@ struct TileIter {
   }
   __device__ bool next(const Params& p, Tile& t) {
     while (unit < p.units) {
-      const long long seg = unit / p.U;
-      const int u = (int)(unit % p.U);
+      const unsigned seg = p.divU.div(unit);
+      const int u = (int)(unit - seg * (unsigned)p.U);
       const int kk = k;
       if (++k == 2) {
         k = 0;
@@ -115,14 +124,17 @@ struct TileIter {
       }
       const int i = kk == 0 ? p.T - 1 - u : u;
       if (kk == 1 && u >= p.T - 1 - u) continue;  // the pair collapsed to one tile
-      t.s = (int)(seg % p.S);
-      t.bh = (int)(seg / p.S);
+      const unsigned bh = p.divS.div(seg);
+      t.s = (int)(seg - bh * (unsigned)p.S);
+      t.bh = (int)bh;
       t.seg0 = (long long)t.s * p.N;
       const int n_s = (int)min((long long)p.N, p.L - t.seg0);
       const int T_s = (n_s + BM - 1) / BM;
       if (i >= T_s) continue;
       t.i = i;
       t.nkv = i + 1;
+      t.h = t.bh % p.H;
+      t.valid = 1;
       t.q_row = (int)(t.seg0 + (long long)i * BM);
       t.rows_valid = min(BM, n_s - i * BM);
       return true;
@@ -171,6 +183,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   float* sZ = reinterpret_cast<float*>(smem + OFF_Z);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+  // Tile descriptors: the producer writes tile c's into slots[c & 1] before it arms
+  // Q's full barrier for that tile (release), and after the last tile it writes an
+  // end marker and arrives on the barrier without a copy. The other roles read a
+  // slot only after a wait that orders them behind that arrival.
+  Tile* slots = reinterpret_cast<Tile*>(smem + OFF_SLOT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -183,6 +200,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       if (b == B_QEMPTY) cnt = 1 + kSoftmaxWarps;
       // B_RDONE: one commit per tile (retrieval MMAs)
       if (b >= B_PAIR && b < B_PAIR + 4) cnt = 2;
+      if (b == B_DRAIN) cnt = 2;  // one commit from each MMA-issuing warp
       mbar_init(&bars[b], cnt);
     }
     fence_barrier_init();
@@ -209,7 +227,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       bool k_wrapped = false, v_wrapped = false;     // every stage used at least once
       bool ok = true;
       auto issue_k = [&](const Tile& t, int j) -> bool {
-        if (k_wrapped && !mbar_wait(&bars[B_KEMPTY + kst], kph ^ 1u)) return false;
+        // the Q K^T that read this stage signalled the same stage's scores barrier
+        if (k_wrapped && !mbar_wait(&bars[B_SFULL + kst], kph ^ 1u)) return false;
         mbar_arrive_expect_tx(&bars[B_KFULL + kst], kTile);
         const int row = (int)(t.seg0 + (long long)j * BN);
         uint8_t* dst = sK + kst * kTile;
@@ -221,16 +240,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         kst ^= 1u;
         return true;
       };
-      auto issue_v = [&](const Tile& t, int item) -> bool {  // item 0,1: M_hi, M_lo; 2+j: V_j
+      auto issue_v = [&](const Tile& t, int item) -> bool {  // item 0: M_hi; 1+j: V_j
         if (v_wrapped && !mbar_wait(&bars[B_VEMPTY + vst], vph ^ 1u)) return false;
         mbar_arrive_expect_tx(&bars[B_VFULL + vst], kTile);
         uint8_t* dst = sV + vst * kTile;
-        if (item < 2) {
-          const int zc = (t.bh * p.S + t.s) * 2 + item;
+        if (item == 0) {
+          const int zc = (t.bh * p.S + t.s) * 2;
           tma_load_3d(dst, &tm_m, &bars[B_VFULL + vst], 0, 0, zc);
           tma_load_3d(dst + kSub, &tm_m, &bars[B_VFULL + vst], 64, 0, zc);
         } else {
-          const int row = (int)(t.seg0 + (long long)(item - 2) * BN);
+          const int row = (int)(t.seg0 + (long long)(item - 1) * BN);
           tma_load_3d(dst, &tm_v, &bars[B_VFULL + vst], 0, row, t.bh);
           tma_load_3d(dst + kSub, &tm_v, &bars[B_VFULL + vst], 64, row, t.bh);
         }
@@ -251,17 +270,33 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           ok = false;
           break;
         }
+        slots[tc & 1] = t;
         mbar_arrive_expect_tx(&bars[B_QFULL], kTile + D * 4);
         tma_load_3d(sQ, &tm_q, &bars[B_QFULL], 0, t.q_row, t.bh);
         tma_load_3d(sQ + kSub, &tm_q, &bars[B_QFULL], 64, t.q_row, t.bh);
         bulk_load(sZ, zprev + ((size_t)t.bh * p.S + t.s) * D, D * 4, &bars[B_QFULL]);
         ++q_iss;
-        ok = issue_k(t, 0) && (t.nkv < 2 || issue_k(t, 1)) && issue_v(t, 0) && issue_v(t, 1);
+        {  // the next tile's Q has a whole tile of work to reach L2
+          TileIter ahead = it;
+          Tile tn;
+          if (ahead.next(p, tn)) {
+            tma_prefetch_l2_3d(&tm_q, 0, tn.q_row, tn.bh);
+            tma_prefetch_l2_3d(&tm_q, 64, tn.q_row, tn.bh);
+          }
+        }
+        ok = issue_k(t, 0) && (t.nkv < 2 || issue_k(t, 1)) && issue_v(t, 0);
         for (int j = 0; ok && j < t.nkv; ++j) {
-          ok = issue_v(t, j + 2);
+          ok = issue_v(t, j + 1);
           if (ok && j + 2 < t.nkv) ok = issue_k(t, j + 2);
         }
         ++tc;
+      }
+      // end of the list: a descriptor with valid = 0 and a plain arrival
+      if (ok && (tc == 0 || mbar_wait(&bars[B_QEMPTY], (uint32_t)((tc - 1) & 1)))) {
+        Tile e;
+        e.valid = 0;
+        slots[tc & 1] = e;
+        mbar_arrive(&bars[B_QFULL]);
       }
       if (!ok) {  // let the copies already issued land before the CTA exits
         if (q_iss > 0) drain_wait(&bars[B_QFULL], (uint32_t)((q_iss - 1) & 1));
@@ -272,85 +307,56 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
     }
   } else if (warp == 1) {
-    // ================= MMA issuer =================
+    // ================= retrieval and P V issuer =================
     // The whole warp runs the issue loop (waits, ring positions, descriptors), so
-    // every value is warp-uniform, and one elected lane (always lane 0) issues the
-    // tensor-core operations and commits: issuing from a diverged single thread
-    // was several times slower while the softmax warps on the same scheduler were
-    // busy. Everything between two MMAs is on the critical path: shared-memory
-    // descriptors are built once per buffer and moved by a constant add (a
-    // descriptor holds the address / 16 in its low 14 bits and every operand lies
-    // below 256 KB, so an offset inside a buffer never carries out of that field),
-    // and ring positions are kept as 32-bit stage / phase pairs.
+    // every value is warp-uniform, and one elected lane issues the tensor-core
+    // operations and commits: issuing from a diverged single thread was several
+    // times slower while the softmax warps on the same scheduler were busy. The
+    // Q K^T products come from warp 10 on another scheduler, so each issuing warp
+    // has half of the per-key-tile instruction stream. Shared-memory descriptors are
+    // built once per buffer and moved by a constant add (a descriptor holds the
+    // address / 16 in its low 14 bits and every operand lies below 256 KB, so an
+    // offset inside a buffer never carries out of that field).
     {
-      const uint32_t id_qk = idesc_f32acc(1, 0, 0, BM, BN);
       const uint32_t id_pv = idesc_f32acc(1, 0, 1, BM, D);
-      const uint64_t dQ = kmajor_desc(smem_u32(sQ), 0);
-      const uint64_t dK0 = kmajor_desc(smem_u32(sK), 0);
       const uint64_t dV0 = mnmajor_desc(smem_u32(sV), 0);
       constexpr uint32_t kTileD = kTile >> 4;  // one tile, in descriptor units
-      uint32_t kst = 0, kph = 0;  // K ring: stage and phase of the next Q K^T
       uint32_t vst = 0, vph = 0;  // V ring: stage and phase of the next item
       uint32_t pb = 0;            // S buffer (and p_full parity) of the next P
       int tc = 0;
-      auto qk = [&](const Tile& t, int j, int tile_no) -> bool {
-        if (j == 0 && !mbar_wait_warp(&bars[B_QFULL], (uint32_t)(tile_no & 1))) return false;
-        if (!mbar_wait_warp(&bars[B_KFULL + kst], kph)) return false;
-        tc_fence_after();
-        const uint64_t dk = dK0 + kst * kTileD;
-        const uint32_t dS = tS + kst * BN;
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_bf16_ss(dS, dQ + kdesc_off(kk), dk + kdesc_off(kk), id_qk, kk > 0 ? 1u : 0u);
-          mma_commit(&bars[B_KEMPTY + kst]);
-          mma_commit(&bars[B_SFULL + kst]);
-          if (j == t.nkv - 1) mma_commit(&bars[B_QEMPTY]);
-        }
-        __syncwarp();
-        kph ^= kst;
-        kst ^= 1u;
-        return true;
-      };
       auto v_next = [&]() {
         if (++vst == (uint32_t)kVStages) {
           vst = 0;
           vph ^= 1u;
         }
       };
-      TileIter it;
-      it.init();
-      Tile t, tn;
-      bool have = it.next(p, t);
       bool ok = true;
-      if (have) ok = qk(t, 0, 0) && (t.nkv < 2 || qk(t, 1, 0));
-      while (ok && have) {
-        // retrieval: R = sigma(Q) M_hi + sigma(Q) M_lo, sigma(Q) read from tensor memory
-        // (features 0..63 at O + [0, 32), features 64..127 at O + [64, 96))
+      for (;;) {
+        // sigma(Q) of tile tc (or the softmax warps' end-of-list arrival) also orders
+        // this read of its descriptor after the producer's write
+        if (!mbar_wait_warp(&bars[B_SQFULL], (uint32_t)(tc & 1))) {
+          ok = false;
+          break;
+        }
+        const Tile t = slots[tc & 1];
+        if (!t.valid) break;
+        // retrieval: R = sigma(Q) M_hi, sigma(Q) read from tensor memory (features
+        // 0..63 at O + [0, 32), features 64..127 at O + [64, 96))
         const uint32_t s0 = vst, p0 = vph;
         v_next();
-        const uint32_t s1 = vst, p1 = vph;
-        v_next();
-        ok = mbar_wait_warp(&bars[B_SQFULL], (uint32_t)(tc & 1)) &&
-             mbar_wait_warp(&bars[B_VFULL + s0], p0) && mbar_wait_warp(&bars[B_VFULL + s1], p1);
+        ok = mbar_wait_warp(&bars[B_VFULL + s0], p0);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t dm0 = dV0 + s0 * kTileD, dm1 = dV0 + s1 * kTileD;
+        const uint64_t dm0 = dV0 + s0 * kTileD;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)), dm0 + mndesc_off(kk), id_pv,
                         kk > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_bf16_ts(tR, tO + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4)), dm1 + mndesc_off(kk), id_pv,
-                        1u);
           mma_commit(&bars[B_VEMPTY + s0]);
-          mma_commit(&bars[B_VEMPTY + s1]);
           mma_commit(&bars[B_RDONE]);
         }
         __syncwarp();
-        const bool has_next = it.next(p, tn);
         for (int j = 0; ok && j < t.nkv; ++j) {
           const uint32_t st = vst, ph = vph;
           v_next();
@@ -366,20 +372,64 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
               mma_bf16_ts(tO, tP + 8 * kk, dv + mndesc_off(kk), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&bars[B_VEMPTY + st]);
             mma_commit(&bars[B_PVDONE]);
+            mma_commit(&bars[B_SFREE + pb]);  // the S buffer may take the next Q K^T
           }
           __syncwarp();
           pb ^= 1u;
-          if (j + 2 < t.nkv) {
-            ok = qk(t, j + 2, tc);
-          } else if (j == t.nkv - 1 && has_next) {
-            ok = qk(tn, 0, tc + 1) && (tn.nkv < 2 || qk(tn, 1, tc + 1));
-          }
         }
-        t = tn;
-        have = has_next;
+        if (!ok) break;
         ++tc;
       }
       // no MMA may still be running when the CTA frees tensor memory
+      if (elect_one()) mma_commit(&bars[B_DRAIN]);
+      __syncwarp();
+      drain_wait(&bars[B_DRAIN], 0);
+    }
+  } else if (warp == 2 + kSoftmaxWarps) {
+    // ================= Q K^T issuer (warp 10) =================
+    // Key step n (counted over the CTA's whole tile sequence) uses K stage and S
+    // buffer n & 1. Its product overwrites the S buffer that held P of step n - 2,
+    // so it waits for that step's P V (the S-free barrier of the buffer, committed by
+    // warp 1); each S-free barrier completes once per use of its buffer and cannot
+    // run two phases ahead of this warp, whose product the next P V needs.
+    {
+      const uint32_t id_qk = idesc_f32acc(1, 0, 0, BM, BN);
+      const uint64_t dQ = kmajor_desc(smem_u32(sQ), 0);
+      const uint64_t dK0 = kmajor_desc(smem_u32(sK), 0);
+      constexpr uint32_t kTileD = kTile >> 4;
+      uint32_t kst = 0, kph = 0;  // K stage / S buffer of the next step, and its use parity
+      uint32_t n = 0;
+      int tc = 0;
+      bool ok = true;
+      for (;;) {
+        if (!mbar_wait_warp(&bars[B_QFULL], (uint32_t)(tc & 1))) {
+          ok = false;
+          break;
+        }
+        const Tile t = slots[tc & 1];
+        if (!t.valid) break;
+        for (int j = 0; j < t.nkv; ++j) {
+          ok = (n < 2 || mbar_wait_warp(&bars[B_SFREE + kst], kph ^ 1u)) &&
+               mbar_wait_warp(&bars[B_KFULL + kst], kph);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dk = dK0 + kst * kTileD;
+          const uint32_t dS = tS + kst * BN;
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_bf16_ss(dS, dQ + kdesc_off(kk), dk + kdesc_off(kk), id_qk, kk > 0 ? 1u : 0u);
+            mma_commit(&bars[B_SFULL + kst]);  // also frees the K stage
+            if (j == t.nkv - 1) mma_commit(&bars[B_QEMPTY]);
+          }
+          __syncwarp();
+          kph ^= kst;
+          kst ^= 1u;
+          ++n;
+        }
+        if (!ok) break;
+        ++tc;
+      }
       if (elect_one()) mma_commit(&bars[B_DRAIN]);
       __syncwarp();
       drain_wait(&bars[B_DRAIN], 0);
@@ -403,10 +453,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // sigma(Q) of tile number tile_no (this thread's 64 columns) -> tensor memory
     // (O + 64 half, 32 packed columns) for the retrieval MMA; partial denominator
     // sigma(Q_r) . z_{s-1} over those columns.
+    // the next tile's descriptor, after Q's full barrier: 1 a tile, 0 the end of the
+    // list (arrive on sigma(Q)'s barrier once more so the P V warp sees it too),
+    // -1 the wait gave up
+    auto fetch = [&](int tile_no, Tile& tt) -> int {
+      if (!mbar_wait_warp(&bars[B_QFULL], (uint32_t)(tile_no & 1))) return -1;
+      tt = slots[tile_no & 1];
+      if (tt.valid) return 1;
+      mbar_arrive_warp(&bars[B_SQFULL]);
+      return 0;
+    };
     auto sigma_q = [&](int tile_no, float& den) -> bool {
-      if (!mbar_wait_warp(&bars[B_QFULL], (uint32_t)(tile_no & 1))) return false;
       const float* zs = sZ + col0;
-      den = 0.f;
+      float dp[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t sq[32];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -420,11 +479,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int e = 0; e < 4; ++e) {
           const float2 f = __bfloat1622float2(h[e]);
           const float p0 = elu1(f.x), p1 = elu1(f.y);
-          den = fmaf(p0, zz[2 * e], den);
-          den = fmaf(p1, zz[2 * e + 1], den);
+          dp[e] = fmaf(p0, zz[2 * e], dp[e]);
+          dp[e] = fmaf(p1, zz[2 * e + 1], dp[e]);
           sq[4 * u + e] = pack_bf16x2(p0, p1);
         }
       }
+      den = (dp[0] + dp[1]) + (dp[2] + dp[3]);
       mbar_arrive_warp(&bars[B_QEMPTY]);  // this warp is done reading Q
       tmem_st32_(tO + lane_off + 64 * half, sq);
       tmem_wait_st();
@@ -432,14 +492,14 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       mbar_arrive_warp(&bars[B_SQFULL]);
       return true;
     };
-    TileIter it;
-    it.init();
     Tile t, tn;
-    bool have = it.next(p, t);
     float den = 0.f;
+    const int got = fetch(0, t);
+    ok = got >= 0;
+    bool have = got == 1;
     if (have) ok = sigma_q(0, den);
     while (ok && have) {
-      const float bta = __ldg(beta + t.bh % p.H);  // used in the epilogue
+      const float bta = __ldg(beta + t.h);  // used in the epilogue
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < t.nkv; ++j) {
         const int b = (int)(kc & 1);
@@ -462,12 +522,14 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         float mx[8];
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) {
-          mx[q8] = __uint_as_float(sr[q8]);
-#pragma unroll
-          for (int c = 1; c < 8; ++c) mx[q8] = fmaxf(mx[q8], __uint_as_float(sr[8 * c + q8]));
+          const float* v = reinterpret_cast<const float*>(sr);
+          mx[q8] = fmax3(v[q8], v[8 + q8], v[16 + q8]);
+          mx[q8] = fmax3(mx[q8], v[24 + q8], v[32 + q8]);
+          mx[q8] = fmax3(mx[q8], v[40 + q8], v[48 + q8]);
+          mx[q8] = fmaxf(mx[q8], v[56 + q8]);
         }
-        const float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mh = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                               fmaxf(mx[6], mx[7]));
         xmax[b * 256 + half * 128 + r] = mh;
         mbar_arrive_warp(pair);
         if (!mbar_wait_warp(pair, pair_phase & 1)) {
@@ -577,8 +639,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
       }
       tc_fence_before();
-      const bool has_next = it.next(p, tn);
-      if (has_next && !sigma_q(tc + 1, den)) {
+      const int gn = fetch(tc + 1, tn);
+      const bool has_next = gn == 1;
+      if (gn < 0 || (has_next && !sigma_q(tc + 1, den))) {
         ok = false;
         break;
       }
@@ -632,12 +695,16 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   p.BH = BH;
   p.T = (int)((min((long long)N, L) + BM - 1) / BM);
   p.U = (p.T + 1) / 2;
-  p.units = (long long)BH * S * p.U;
+  const long long units = (long long)BH * S * p.U;
+  if (units >= (1ll << 31)) return cudaErrorInvalidValue;
+  p.units = (unsigned)units;
+  p.divU = FastDiv((uint32_t)p.U);
+  p.divS = FastDiv((uint32_t)S);
   p.out32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const unsigned grid = (unsigned)(p.units < (long long)sms ? p.units : (long long)sms);
+  const unsigned grid = p.units < (unsigned)sms ? p.units : (unsigned)sms;
   attn_kernel<<<grid, kThreads, kAttnSmem, stream>>>(mq, mk, mv, mm, beta, ws.zprev, out, p);
   return cudaGetLastError();
 }

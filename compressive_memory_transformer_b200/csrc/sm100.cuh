@@ -128,6 +128,14 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
+// Asks the TMA unit to bring a box into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m, uint64_t* bar,
                                             int c0, int c1, int c2) {
   asm volatile(
@@ -397,6 +405,13 @@ __device__ __forceinline__ float elu1(float x) {
   return x > 0.f ? x + 1.f : ex2_approx(fminf(x, 0.f) * kLog2e);
 }
 
+// Three-input maximum (one sm_100 instruction).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -409,6 +424,27 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v) {
                "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
                : "memory");
 }
+
+// Unsigned 32-bit division by a divisor fixed at launch, as a multiply-high and
+// two shifts (Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication", PLDI 1994, section 4): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, q = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0)
+// where t = mulhi(m, n), exact for every 32-bit n and 1 <= d < 2^31.
+struct FastDiv {
+  uint32_t d, m, s1, s2;
+  __host__ __device__ FastDiv() : d(1), m(1), s1(0), s2(0) {}
+  explicit FastDiv(uint32_t div) : d(div) {
+    uint32_t l = 0;
+    while (l < 32 && (1ull << l) < div) ++l;
+    m = (uint32_t)((((1ull << l) - div) << 32) / div + 1);
+    s1 = l < 1 ? l : 1;
+    s2 = l > 1 ? l - 1 : 0;
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    const uint32_t t = __umulhi(m, n);
+    return (t + ((n - t) >> s1)) >> s2;
+  }
+};
 
 // Byte offset of the 16-byte unit u (0..7) of row r inside a 128B-swizzled
 // region whose rows are 128 bytes apart (region base 1024-byte aligned).

@@ -164,22 +164,26 @@ def test_bf16_carried_state_and_step(ia, mode):
 
 
 @pytest.mark.parametrize("mode", [LIN, DEL])
-def test_bf16_rescale_every_key_tile(ia, mode):
-    """Scores that grow along the segment (keys k_t ~ 0.05 t + N(0,1), queries
-    ~ 1 + 0.1 N(0,1)): every later key tile raises each row's running max far past
-    the 2^8 threshold, so the online softmax rescales O at every key tile."""
+@pytest.mark.parametrize("growth", [0.0045, 0.008, 0.015, 0.05])
+def test_bf16_rescale_every_key_tile(ia, mode, growth):
+    """Scores that grow along the segment (keys k_t ~ growth t + N(0,1), queries
+    ~ 1 + 0.1 N(0,1)): each key tile raises each row's running max by about
+    2089 growth in exp2 units (128 features x 128 keys x log2(e)/sqrt(128)), i.e.
+    about 9, 17, 31 and 104 for the four rates: past the 2^8 rescale threshold at
+    every key tile, below and above the 2^24 bound under which a step keeps the P it
+    computed against the previous step's maximum."""
     B, H, L, N = 1, 2, 1024, 512
     g = torch.Generator().manual_seed(41)
     t = torch.arange(L, dtype=torch.float32).view(1, 1, L, 1)
     q = (1.0 + 0.1 * torch.randn((B, H, L, 128), generator=g)).to(torch.bfloat16)
-    k = (0.05 * (t % N) + torch.randn((B, H, L, 128), generator=g)).to(torch.bfloat16)
+    k = (growth * (t % N) + torch.randn((B, H, L, 128), generator=g)).to(torch.bfloat16)
     v = torch.randn((B, H, L, 128), generator=g).to(torch.bfloat16)
     beta = torch.tensor([0.3, -0.7])
     inp = {"q": q.cuda(), "k": k.cuda(), "v": v.cuda(), "beta": beta.cuda()}
     out, M, z = ia.infini_attn_forward(inp["q"], inp["k"], inp["v"], inp["beta"], N, mode)
     sync_ok(ia)
     ref = run_oracle(inp, N, mode)
-    check_bf16(out, M, z, ref, what=f"rescale mode={mode}")
+    check_bf16(out, M, z, ref, what=f"rescale mode={mode} growth={growth}")
 
 
 @pytest.mark.parametrize("mode", [LIN, DEL])
