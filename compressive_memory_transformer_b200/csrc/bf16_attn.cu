@@ -70,10 +70,11 @@ constexpr int BM = 128;   // query rows per tile
 constexpr int BN = 128;   // keys per tile
 constexpr int kTile = 32768;     // one 128 x 128 bf16 tile
 constexpr int kSub = 16384;      // one 128 x 64 box (128-byte rows)
-constexpr int kVStages = 3;
+constexpr int kVStages = 2;
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = kTile;         // 2 stages
 constexpr int OFF_V = 3 * kTile;     // kVStages stages
+constexpr int OFF_OUT = 5 * kTile;   // output tile staged for the TMA store (half h at h * kSub)
 constexpr int OFF_X = 6 * kTile;     // exchange: max [2][2][128], den [2][128], l [2][128]
 constexpr int OFF_Z = OFF_X + 4096;   // z_{s-1} of the current tile (128 floats), loaded with Q
 constexpr int OFF_BAR = OFF_Z + 512;
@@ -86,7 +87,7 @@ constexpr int kSoftmaxWarps = 8;
 enum {
   B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_SFREE = 4 /* 2 */, B_VFULL = 6 /* 3 */, B_VEMPTY = 9 /* 3 */,
   B_SFULL = 12, B_PFULL = 14, B_PVDONE = 15, B_DRAIN = 16, B_PAIR = 17 /* 4 */, B_RDONE = 21,
-  B_SQFULL = 22, B_COUNT = 23
+  B_SQFULL = 22, B_OFULL = 23 /* 2 */, B_OFREE = 25 /* 2 */, B_COUNT = 27
 };
 
 struct Params {
@@ -94,7 +95,8 @@ struct Params {
   int N, S, H, T, U, BH;
   unsigned units;  // BH * S * U, below 2^31
   FastDiv divU, divS;
-  int out32;  // out is 32-byte aligned: rows are stored as whole 32-byte sectors
+  int out32;    // out is 32-byte aligned: rows are stored as whole 32-byte sectors
+  int tma_out;  // out has a TMA map: whole tiles leave through shared memory
 };
 
 // One query tile of the work list (valid = 0: the end of the CTA's list).
@@ -171,6 +173,7 @@ __device__ __forceinline__ constexpr uint32_t mndesc_off(int kk) { return (uint3
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
+            const __grid_constant__ CUtensorMap tm_o,
             const float* __restrict__ beta, const float* __restrict__ zprev,
             __nv_bfloat16* __restrict__ out, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -179,6 +182,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   uint8_t* sQ = smem + OFF_Q;
   uint8_t* sK = smem + OFF_K;
   uint8_t* sV = smem + OFF_V;
+  uint8_t* sOut = smem + OFF_OUT;
   float* sX = reinterpret_cast<float*>(smem + OFF_X);
   float* sZ = reinterpret_cast<float*>(smem + OFF_Z);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -201,6 +205,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // B_RDONE: one commit per tile (retrieval MMAs)
       if (b >= B_PAIR && b < B_PAIR + 4) cnt = 2;
       if (b == B_DRAIN) cnt = 2;  // one commit from each MMA-issuing warp
+      if (b == B_OFULL || b == B_OFULL + 1) cnt = 4;  // the four warps of a half
       mbar_init(&bars[b], cnt);
     }
     fence_barrier_init();
@@ -208,6 +213,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_m);
+    if (p.tma_out) tma_prefetch_desc(&tm_o);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -222,7 +228,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0) {
-      int q_iss = 0, k_iss[2] = {0, 0}, v_iss[kVStages] = {0, 0, 0};
+      int q_iss = 0, k_iss[2] = {0, 0}, v_iss[kVStages] = {0, 0};
       uint32_t kst = 0, kph = 0, vst = 0, vph = 0;  // next K / V ring stage and phase
       bool k_wrapped = false, v_wrapped = false;     // every stage used at least once
       bool ok = true;
@@ -286,8 +292,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         ok = issue_k(t, 0) && (t.nkv < 2 || issue_k(t, 1)) && issue_v(t, 0);
         for (int j = 0; ok && j < t.nkv; ++j) {
-          ok = issue_v(t, j + 1);
-          if (ok && j + 2 < t.nkv) ok = issue_k(t, j + 2);
+          // K of step j + 2 (its stage frees when Q K^T_j is done) goes before V_j,
+          // whose stage frees one P V later
+          if (j + 2 < t.nkv) ok = issue_k(t, j + 2);
+          if (ok) ok = issue_v(t, j + 1);
         }
         ++tc;
       }
@@ -494,6 +502,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     };
     Tile t, tn;
     float den = 0.f;
+    int oc = 0;  // tiles stored through shared memory so far
     const int got = fetch(0, t);
     ok = got >= 0;
     bool have = got == 1;
@@ -639,13 +648,51 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
       }
       tc_fence_before();
+      // A whole tile (or one whose missing rows lie past the end of the tensor, where
+      // TMA drops them) leaves through shared memory: each half writes its 128 x 64
+      // box, 128B-swizzled, and the half's first warp issues the TMA store. Before a
+      // half rewrites its box, that warp has seen its previous store finish reading.
+      const bool tma_tile =
+          p.tma_out && (t.rows_valid == BM || (long long)t.q_row + t.rows_valid == p.L);
+      const bool issuer = warp == 2 + 4 * half;
+      if (tma_tile) {
+        if (oc > 0) {
+          if (issuer && lane == 0) {
+            bulk_wait_group_read0();
+            mbar_arrive(&bars[B_OFREE + half]);
+          }
+          __syncwarp();
+          if (!mbar_wait_warp(&bars[B_OFREE + half], (uint32_t)((oc - 1) & 1))) {
+            ok = false;
+            break;
+          }
+        }
+        const uint32_t ob = smem_u32(sOut + half * kSub);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          st_shared_v4(ob + sw128(r, u), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        fence_proxy_async_smem();
+        mbar_arrive_warp(&bars[B_OFULL + half]);
+        if (issuer) {
+          if (!mbar_wait_warp(&bars[B_OFULL + half], (uint32_t)(oc & 1))) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            tma_store_3d(&tm_o, sOut + half * kSub, 64 * half, t.q_row, t.bh);
+            tma_store_commit();
+          }
+          __syncwarp();
+        }
+        ++oc;
+      }
       const int gn = fetch(tc + 1, tn);
       const bool has_next = gn == 1;
       if (gn < 0 || (has_next && !sigma_q(tc + 1, den))) {
         ok = false;
         break;
       }
-      if (r < t.rows_valid) {
+      if (!tma_tile && r < t.rows_valid) {
         __nv_bfloat16* orow = out + ((size_t)t.bh * p.L + t.q_row + r) * D + col0;
         if (p.out32) {
 #pragma unroll
@@ -661,6 +708,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       have = has_next;
       ++tc;
     }
+    // the TMA stores must be done with shared memory (and global) before the CTA ends
+    if (warp == 2 + 4 * half && lane == 0) tma_store_wait_all();
   }
 
   tc_fence_before();
@@ -682,7 +731,7 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                              const __nv_bfloat16* v, const float* beta, __nv_bfloat16* out,
                              const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
                              cudaStream_t stream) {
-  CUtensorMap mq, mk, mv, mm;
+  CUtensorMap mq, mk, mv, mm, mo;
   if (!make_bf16_map(&mq, q, (uint64_t)L, BH, 128) || !make_bf16_map(&mk, k, (uint64_t)L, BH, 128) ||
       !make_bf16_map(&mv, v, (uint64_t)L, BH, 128) ||
       !make_bf16_map(&mm, ws.Mhl, D, (uint64_t)BH * S * 2, 128))
@@ -701,11 +750,14 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   p.divU = FastDiv((uint32_t)p.U);
   p.divS = FastDiv((uint32_t)S);
   p.out32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
+  // a TMA map needs a 16-byte aligned base; otherwise every tile is stored directly
+  p.tma_out = make_bf16_map(&mo, out, (uint64_t)L, BH, 128) ? 1 : 0;
+  if (!p.tma_out) mo = mq;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const unsigned grid = p.units < (unsigned)sms ? p.units : (unsigned)sms;
-  attn_kernel<<<grid, kThreads, kAttnSmem, stream>>>(mq, mk, mv, mm, beta, ws.zprev, out, p);
+  attn_kernel<<<grid, kThreads, kAttnSmem, stream>>>(mq, mk, mv, mm, mo, beta, ws.zprev, out, p);
   return cudaGetLastError();
 }
 
