@@ -7,6 +7,7 @@ importing this package fails when the library is missing or cannot be loaded.
 Entry points (same names as the C ABI in include/infini_attn.h):
     infini_attn_forward(q, k, v, beta, N, mode, M_in=None, z_in=None, ...)
     infini_attn_step(q, k, v, beta, mode, M_in=None, z_in=None, ...)
+    infini_attn_decode(q, k, v, beta, k_cache, v_cache, M, z, pos, mode, ...)
 q, k, v: [B, H, L, d] CUDA tensors, bf16 (d = 128) or fp32 (d <= 128);
 beta: [H] fp32; M: [B, H, d, d] fp32; z: [B, H, d] fp32.
 """
@@ -49,6 +50,7 @@ _SIGS = {
     "infini_attn_forward_f32": [_vp] * 9 + [_i, _i, _ll, _i, _i, _i, _vp],
     "infini_attn_step_f32": [_vp] * 9 + [_i, _i, _i, _i, _i, _vp],
     "infini_attn_forward_ex": [_vp] * 9 + [_i, _i, _ll, _i, _i, _i, _i, ctypes.POINTER(Opts), _vp],
+    "infini_attn_decode": [_vp] * 9 + [_i] * 7 + [_vp],
     "infini_attn_workspace_size": [_i, _i, _ll, _i, _i, _i, _i],
     "infini_attn_device_status": [],
     "infini_attn_selftest_timeout": [_ll, _vp],
@@ -163,6 +165,39 @@ def infini_attn_forward_ex(q, k, v, beta, N, mode=LINEAR, M_in=None, z_in=None, 
                                        int(N), d, int(mode), dtype, ctypes.byref(o),
                                        _stream_handle(stream)))
     return out, M_out, z_out
+
+
+def infini_attn_decode(q, k, v, beta, k_cache, v_cache, M, z, pos, mode=LINEAR, out=None,
+                       stream=None):
+    """Token-level streaming decode: n new tokens (q, k, v: [B, H, n, d] bf16) join the
+    current segment, whose first `pos` tokens are in k_cache / v_cache ([B, H, N, d]
+    bf16). Writes the new rows into the caches, returns out ([B, H, n, d] bf16), and
+    when pos + n == N folds the segment into M / z ([B, H, d, d] / [B, H, d] fp32) in
+    place."""
+    if q.dim() != 4 or q.dtype != torch.bfloat16:
+        raise ValueError("q, k, v must be [B, H, n, d] bf16")
+    B, H, n, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor shaped and typed like q")
+    if k_cache.dim() != 4 or k_cache.shape[:2] != (B, H) or k_cache.shape[3] != d:
+        raise ValueError("k_cache must be [B, H, N, d]")
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        if (t.shape != k_cache.shape or t.dtype != torch.bfloat16 or not t.is_cuda
+                or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor shaped like k_cache")
+    for t in (M, z):
+        if t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("M and z must be contiguous CUDA fp32 tensors")
+    if beta.dtype != torch.float32 or beta.numel() != H or not beta.is_cuda:
+        raise ValueError("beta must be a CUDA fp32 tensor with H elements")
+    N = k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_lib.infini_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(k_cache),
+                                   _ptr(v_cache), _ptr(M), _ptr(z), _ptr(out), B, H, n, int(pos),
+                                   N, d, int(mode), _stream_handle(stream)))
+    return out
 
 
 def workspace_size(B, H, L, N, d, mode=LINEAR, dtype=DTYPE_BF16) -> int:

@@ -20,7 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_NAME = "libinfini_attn.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
-SOURCES = ["infini_attn.cu", "bf16_state.cu", "bf16_attn.cu", "f32_path.cu", "step_static.cu"]
+SOURCES = ["infini_attn.cu", "bf16_state.cu", "bf16_attn.cu", "f32_path.cu", "step_static.cu",
+           "bf16_decode.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -245,6 +245,69 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
+// Token-level decode: append the new rows to the caches, attention + retrieval +
+// gate for the new tokens against the cache and the state as it stands, then, when
+// the segment is complete, the segment's state update in place (the same calls as
+// a one-segment step with M_out == M_in).
+int decode_impl(const void* q, const void* k, const void* v, const float* beta, void* k_cache,
+                void* v_cache, float* M, float* z, void* out, int B, int H, int n, int pos,
+                int N, int d, int mode, cudaStream_t stream) {
+  if (!q || !k || !v || !beta || !k_cache || !v_cache || !M || !z || !out) return INFINI_ERR_NULL;
+  if (B < 1 || H < 1 || n < 1 || pos < 0 || N < 1 || (long long)pos + n > N)
+    return INFINI_ERR_SHAPE;
+  if (mode != INFINI_LINEAR && mode != INFINI_DELTA) return INFINI_ERR_UNSUPPORTED;
+  if (d != 128) return INFINI_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > (1LL << 30) || overflows(BH, (long long)N * d * 2)) return INFINI_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(M) || !aligned16(z))
+    return INFINI_ERR_ALIGN;
+  const size_t nio = (size_t)(BH * n * d) * 2, ncache = (size_t)(BH * N * d) * 2;
+  const size_t nM = (size_t)BH * d * d * sizeof(float), nz = (size_t)BH * d * sizeof(float);
+  const void* ins[] = {q, k, v};
+  for (const void* x : ins)
+    if (overlap(out, nio, x, nio) || overlap(k_cache, ncache, x, nio) ||
+        overlap(v_cache, ncache, x, nio))
+      return INFINI_ERR_ALIAS;
+  if (overlap(out, nio, k_cache, ncache) || overlap(out, nio, v_cache, ncache) ||
+      overlap(out, nio, M, nM) || overlap(out, nio, z, nz) ||
+      overlap(k_cache, ncache, v_cache, ncache) || overlap(k_cache, ncache, M, nM) ||
+      overlap(v_cache, ncache, M, nM) || overlap(M, nM, z, nz))
+    return INFINI_ERR_ALIAS;
+  int dev = 0, sms = 148;
+  if (prepare_device(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // the new keys and values go to cache rows [pos, pos + n) of every head
+  const size_t row = (size_t)d * 2;
+  if (cudaMemcpy2DAsync(static_cast<char*>(k_cache) + (size_t)pos * row, (size_t)N * row, k,
+                        (size_t)n * row, (size_t)n * row, (size_t)BH, cudaMemcpyDeviceToDevice,
+                        stream) != cudaSuccess ||
+      cudaMemcpy2DAsync(static_cast<char*>(v_cache) + (size_t)pos * row, (size_t)N * row, v,
+                        (size_t)n * row, (size_t)n * row, (size_t)BH, cudaMemcpyDeviceToDevice,
+                        stream) != cudaSuccess)
+    return INFINI_ERR_CUDA;
+  Scratch sp;
+  int st = get_scratch(sp, bf16_decode_workspace_bytes((int)BH, n, pos, sms), nullptr, stream);
+  if (st != INFINI_OK) return st;
+  const auto* kcb = static_cast<const __nv_bfloat16*>(k_cache);
+  const auto* vcb = static_cast<const __nv_bfloat16*>(v_cache);
+  if (bf16_decode_launch(static_cast<const __nv_bfloat16*>(q), kcb, vcb, beta, M, z,
+                         static_cast<__nv_bfloat16*>(out), static_cast<float*>(sp.ptr), (int)BH, H,
+                         n, pos, N, sms, stream) != cudaSuccess)
+    return INFINI_ERR_CUDA;
+  if (pos + n < N) return INFINI_OK;
+  int CH = 1, CL = N;
+  bf16_state_plan((int)BH, 1, N, &CH, &CL);
+  Scratch sc;
+  st = get_scratch(sc, bf16_workspace_bytes((int)BH, 1, CH), nullptr, stream);
+  if (st != INFINI_OK) return st;
+  const Bf16Workspace ws = bf16_workspace_carve(sc.ptr, (int)BH, 1, CH);
+  cudaError_t e = bf16_prep_first(M, z, ws, (int)BH, 1, stream);
+  if (e == cudaSuccess)
+    e = bf16_state_launch(kcb, vcb, M, z, M, z, ws, (int)BH, N, N, 1, CH, CL, mode, 1, stream);
+  return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace infini
 
@@ -280,6 +343,13 @@ int infini_attn_step_f32(const float* q, const float* k, const float* v, const f
                          float* z_out, int B, int H, int N, int d, int mode, void* stream) {
   return forward_impl(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, N, N < 1 ? 1 : N, d,
                       mode, INFINI_DTYPE_F32, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int infini_attn_decode(const void* q, const void* k, const void* v, const float* beta,
+                       void* k_cache, void* v_cache, float* M, float* z, void* out, int B, int H,
+                       int n, int pos, int N, int d, int mode, void* stream) {
+  return decode_impl(q, k, v, beta, k_cache, v_cache, M, z, out, B, H, n, pos, N, d, mode,
+                     static_cast<cudaStream_t>(stream));
 }
 
 size_t infini_attn_workspace_size(int B, int H, long long L, int N, int d, int mode, int dtype) {

@@ -112,6 +112,37 @@ int infini_attn_step_static(const void* q, const void* k, const void* v, const f
                             const float* M_in, const float* z_in, void* out, float* M_out,
                             float* z_out, int B, int H, int N, int d, int mode, void* stream);
 
+/*
+ * Token-level streaming decode (the pages' "fast streaming inference": section 3.1
+ * attention and section 3.3 retrieval for tokens that arrive one or a few at a
+ * time inside a segment). n new tokens of every (b, h) join the current segment,
+ * whose first `pos` tokens the caller's KV cache already holds.
+ *   q, k, v            [B, H, n, d] bf16, the new tokens (device, read).
+ *   beta               [H] fp32 (device, read).
+ *   k_cache, v_cache   [B, H, N, d] bf16, the current segment's keys and values
+ *                      (device, caller-owned): rows [0, pos) are read, rows
+ *                      [pos, pos + n) are written with k and v by this call.
+ *   M, z               [B, H, d, d] and [B, H, d] fp32 (device): the memory of the
+ *                      segments before this one (M_{s-1}, z_{s-1}; zeros at the start
+ *                      of a stream). Read for the retrieval; when pos + n == N the
+ *                      call then folds the completed segment in with the Linear or
+ *                      Linear+Delta rule, in place, so the next call starts the next
+ *                      segment with pos = 0.
+ *   out                [B, H, n, d] bf16 (device, written): for new token i (segment
+ *                      position t = pos + i), g A_mem + (1 - g) A_dot with A_dot the
+ *                      causal softmax attention over cache rows 0..t and A_mem the
+ *                      retrieval from (M, z) as passed in. Every token gets what
+ *                      infini_attn_forward gives it on the same stream of tokens.
+ * Requires d == 128, n >= 1, pos >= 0, pos + n <= N, mode 0 or 1, 16-byte aligned
+ * pointers and no overlap between out, the caches, the state and the inputs
+ * (INFINI_ERR_NULL / SHAPE / UNSUPPORTED / ALIGN / ALIAS before any launch).
+ * Scratch comes from the stream-ordered allocator on `stream` (INFINI_ERR_NOMEM).
+ * Built for small n; a whole segment at once is cheaper through infini_attn_step.
+ */
+int infini_attn_decode(const void* q, const void* k, const void* v, const float* beta,
+                       void* k_cache, void* v_cache, float* M, float* z, void* out, int B, int H,
+                       int n, int pos, int N, int d, int mode, void* stream);
+
 /* fp32 q/k/v/out variants of infini_attn_forward and infini_attn_step; 1 <= d <= 128. */
 int infini_attn_forward_f32(const float* q, const float* k, const float* v, const float* beta,
                             const float* M_in, const float* z_in, float* out, float* M_out,

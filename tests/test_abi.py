@@ -102,3 +102,29 @@ def test_package_fails_loudly_without_library(tmp_path):
     (tmp_path / "pkgcopy" / "__init__.py").write_text(src)
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True)
     assert r.returncode != 0 and "ImportError" in r.stderr and "missing" in r.stderr
+
+
+def call_decode(lib, q=FAKE, k=FAKE + 4096, v=FAKE + 8192, beta=FAKE + 12288, k_cache=FAKE * 3,
+                v_cache=FAKE * 3 + 65536, M=FAKE * 4, z=FAKE * 4 + 65536, out=FAKE * 2, B=1, H=1,
+                n=1, pos=0, N=128, d=128, mode=0):
+    return lib.raw_call("infini_attn_decode", q, k, v, beta, k_cache, v_cache, M, z, out, B, H,
+                        n, pos, N, d, mode, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(k=None), -1), (dict(v=None), -1), (dict(beta=None), -1),
+    (dict(k_cache=None), -1), (dict(v_cache=None), -1), (dict(M=None), -1), (dict(z=None), -1),
+    (dict(out=None), -1),
+    (dict(B=0), -2), (dict(H=0), -2), (dict(n=0), -2), (dict(pos=-1), -2), (dict(N=0), -2),
+    (dict(pos=120, n=9), -2),             # pos + n > N
+    (dict(d=64), -3), (dict(mode=2), -3),
+    (dict(q=FAKE + 8), -4), (dict(k_cache=FAKE * 3 + 8), -4), (dict(M=FAKE * 4 + 4), -4),
+    (dict(out=FAKE), -8),                 # out is q
+    (dict(v_cache=FAKE * 3 + 16384), -8), # the caches overlap
+    (dict(out=FAKE * 3 + 256), -8),       # out inside k_cache
+    (dict(k=FAKE * 3), -8),               # the new keys inside the cache
+    (dict(z=FAKE * 4 + 4096), -8),        # z inside M
+])
+def test_decode_rejects_bad_arguments(lib, kw, code):
+    """Every argument error is reported on the host, before any CUDA call."""
+    assert call_decode(lib, **kw) == code
