@@ -504,6 +504,75 @@ def run_extra(args, device):
                       "stream_ms_graph": graph_ms, "us_per_step_graph": graph_ms * 1e3 / S,
                       "tokens_per_s_plain": Bc * S * Nc / (plain_ms / 1e3),
                       "stream_ms_plain": plain_ms})
+    if which in ("decode", "all"):
+        # token-level streaming decode on the 1B-layer heads: one segment of N tokens fed
+        # one token per infini_attn_decode call (the segment-end call also folds the
+        # segment into the state), and single calls in the middle of the segment
+        Bc, Hc, Nc = 4, 8, 2048
+        inp = make_inputs(Bc, Hc, Nc, D, torch.bfloat16, seed=7, device=device, gen_device=device)
+        kc = torch.zeros((Bc, Hc, Nc, D), device=device, dtype=torch.bfloat16)
+        vc = torch.zeros_like(kc)
+        M = torch.zeros((Bc, Hc, D, D), device=device)
+        z = torch.zeros((Bc, Hc, D), device=device)
+        tok = [{x: inp[x][:, :, t:t + 1].contiguous() for x in ("q", "k", "v")}
+               for t in range(Nc)]
+        outs = [torch.empty_like(tok[0]["q"]) for _ in range(Nc)]
+        beta = inp["beta"]
+
+        def segment():
+            for t in range(Nc):
+                ia.infini_attn_decode(tok[t]["q"], tok[t]["k"], tok[t]["v"], beta, kc, vc, M, z,
+                                      t, ia.DELTA, out=outs[t])
+        segment()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            segment()
+        g.replay()
+        torch.cuda.synchronize()
+        seg_ms = _timed(g.replay, 2, stream)
+        del g
+
+        def calls_at(pos, n, reps=64):
+            q_ = inp["q"][:, :, pos:pos + n].contiguous()
+            k_ = inp["k"][:, :, pos:pos + n].contiguous()
+            v_ = inp["v"][:, :, pos:pos + n].contiguous()
+            o_ = torch.empty_like(q_)
+
+            def f():
+                for _ in range(reps):
+                    ia.infini_attn_decode(q_, k_, v_, beta, kc, vc, M, z, pos, ia.DELTA, out=o_)
+            f()
+            torch.cuda.synchronize()
+            gg = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gg):
+                f()
+            gg.replay()
+            torch.cuda.synchronize()
+            ms = _timed(gg.replay, 3, stream) / reps
+            del gg
+            # bytes one call must move: the cache rows it attends to (K and V), the fp32
+            # state, the new tokens' q/k/v in, their cache rows and outputs out
+            byts = Bc * Hc * ((pos + n) * 2 * D * 2 + D * D * 4 + D * 4 + n * D * 2 * 6)
+            return ms, byts
+        ms1, by1 = calls_at(1024, 1)
+        ms16, by16 = calls_at(1024, 16)
+        assert ia.device_status() == 0
+        hbm_peak = load_peaks()[2]
+        lines.append({"config": "decode: B=4, H=8, d=128, N=2048, bf16, Linear+Delta, "
+                                "infini_attn_decode",
+                      "segment_one_token_per_call": {
+                          "tokens_per_s": Bc * Nc / (seg_ms / 1e3),
+                          "us_per_call": seg_ms * 1e3 / Nc, "graph_captured": True},
+                      "one_token_at_pos1024": {
+                          "us_per_call": ms1 * 1e3, "bytes": by1,
+                          "hbm_gbs": by1 / (ms1 / 1e3) / 1e9,
+                          "frac_hbm": by1 / (ms1 / 1e3) / 1e9 / hbm_peak},
+                      "16_tokens_at_pos1024": {
+                          "us_per_call": ms16 * 1e3, "tokens_per_s": Bc * 16 / (ms16 / 1e3),
+                          "hbm_gbs": by16 / (ms16 / 1e3) / 1e9,
+                          "frac_hbm": by16 / (ms16 / 1e3) / 1e9 / hbm_peak},
+                      "hbm_peak_gbs": hbm_peak})
     return lines
 
 
@@ -515,7 +584,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--config", choices=["c2", "c3", "c4", "c5", "all"], default="c2",
+    ap.add_argument("--config", choices=["c2", "c3", "c4", "c5", "decode", "all"], default="c2",
                     help="c2 (default) prints the headline line; the others print one extra "
                          "line per workload of the configuration list")
     args = ap.parse_args()

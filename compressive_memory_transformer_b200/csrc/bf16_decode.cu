@@ -12,16 +12,21 @@
 // The work is a batch of short matrix-vector products over the cache: it is bound
 // by reading the cache (512 B per cached token-head) and the fp32 memory (64 KiB per
 // head), so it runs on CUDA cores, split over the cache like flash decoding:
-//   decode_partial_kernel  grid (splits, BH, query groups of 16). A CTA stages
+//   decode_partial_kernel  grid (splits, BH, query groups of up to 16). A CTA stages
 //                          64-row chunks of K and V in shared memory (16-byte loads,
-//                          coalesced), scores every query of its group against them
-//                          (two threads per row, 64 features each), and keeps one
-//                          online-softmax partial (max, sum, 128 accumulators) per
-//                          query in exp2 units.
+//                          coalesced): cache rows below pos from the cache, the new
+//                          rows straight from the call's k and v (the last query
+//                          group also writes those into the cache; nothing in the
+//                          call reads them from there). It scores every query of
+//                          its group against the chunk (two threads per row, 64
+//                          features each) and keeps one online-softmax partial
+//                          (max, sum, 128 accumulators) per query in exp2 units.
 //   decode_combine_kernel  grid (BH, query groups). Merges the splits' partials,
-//                          adds the retrieval from the fp32 state (one thread per
-//                          output feature walks M's column, shared by the group's
-//                          queries) and the gate, writes out in bf16.
+//                          adds the retrieval from the fp32 state (M read once per
+//                          group, row-coalesced float4 loads spread over the four
+//                          warps) and the gate, writes out in bf16.
+// Both kernels are compiled for query-group widths 1, 2, 4, 8 and 16, so a single
+// token carries no idle accumulators.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -45,9 +50,11 @@ struct DecodeParams {
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
+template <int NQ>
 __global__ void __launch_bounds__(kThreads)
-decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
-                      const __nv_bfloat16* __restrict__ vc, float* __restrict__ part,
+decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ knew,
+                      const __nv_bfloat16* __restrict__ vnew, __nv_bfloat16* __restrict__ kc,
+                      __nv_bfloat16* __restrict__ vc, float* __restrict__ part,
                       const DecodeParams p) {
   __shared__ __align__(16) float sq[kGroup][D];    // queries, scaled by log2(e) / sqrt(d)
   __shared__ __align__(16) uint32_t sk[kRows][D / 2];  // bf16 pairs
@@ -71,9 +78,10 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
   const int rows = p.pos + q0 + nq;
   const int r_begin = split * p.chunks_per_split * kRows;
   const int r_end = min(rows, r_begin + p.chunks_per_split * kRows);
-  float acc[kGroup];
+  float acc[NQ];
 #pragma unroll
-  for (int i = 0; i < kGroup; ++i) acc[i] = 0.f;
+  for (int i = 0; i < NQ; ++i) acc[i] = 0.f;
+  const bool writer = grp == p.groups - 1;  // this group loads every new row
 
   const size_t base = (size_t)bh * p.N * D;
   for (int r0 = r_begin; r0 < r_end; r0 += kRows) {
@@ -82,8 +90,20 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
     // K and V rows [r0, r0 + nr): 16 bytes per thread per step, row-contiguous
     for (int e = t; e < nr * (D / 8); e += kThreads) {
       const int row = e / (D / 8), c = e % (D / 8);
-      const uint4 kk = *reinterpret_cast<const uint4*>(kc + base + (size_t)(r0 + row) * D + c * 8);
-      const uint4 vv = *reinterpret_cast<const uint4*>(vc + base + (size_t)(r0 + row) * D + c * 8);
+      const int R = r0 + row;
+      uint4 kk, vv;
+      if (R < p.pos) {
+        kk = *reinterpret_cast<const uint4*>(kc + base + (size_t)R * D + c * 8);
+        vv = *reinterpret_cast<const uint4*>(vc + base + (size_t)R * D + c * 8);
+      } else {
+        const size_t src = ((size_t)bh * p.n + (R - p.pos)) * D + c * 8;
+        kk = *reinterpret_cast<const uint4*>(knew + src);
+        vv = *reinterpret_cast<const uint4*>(vnew + src);
+        if (writer) {
+          *reinterpret_cast<uint4*>(kc + base + (size_t)R * D + c * 8) = kk;
+          *reinterpret_cast<uint4*>(vc + base + (size_t)R * D + c * 8) = vv;
+        }
+      }
       *reinterpret_cast<uint4*>(&sk[row][c * 4]) = kk;
       *reinterpret_cast<uint4*>(&sv[row][c * 4]) = vv;
     }
@@ -150,13 +170,14 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
     // P V: thread t owns feature t
     {
 #pragma unroll
-      for (int i = 0; i < kGroup; ++i)
+      for (int i = 0; i < NQ; ++i)
         if (i < nq) acc[i] *= sm_a[i];
+#pragma unroll 4
       for (int r = 0; r < nr; ++r) {
         const uint32_t u = sv[r][t >> 1];
         const float vf = (t & 1) ? bf_hi(u) : bf_lo(u);
 #pragma unroll
-        for (int i = 0; i < kGroup; ++i)
+        for (int i = 0; i < NQ; ++i)
           if (i < nq) acc[i] = fmaf(ss[i][r], vf, acc[i]);
       }
     }
@@ -164,7 +185,7 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
   __syncthreads();
   float* out = part + (((size_t)bh * p.groups + grp) * p.splits + split) * kGroup * kPart;
 #pragma unroll
-  for (int i = 0; i < kGroup; ++i) {
+  for (int i = 0; i < NQ; ++i) {
     if (i >= nq) break;
     if (t == 0) {
       out[i * kPart] = sm_m[i];
@@ -174,16 +195,18 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
   }
 }
 
+template <int NQ>
 __global__ void __launch_bounds__(kThreads)
 decode_combine_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ part,
                       const float* __restrict__ beta, const float* __restrict__ M,
                       const float* __restrict__ z, __nv_bfloat16* __restrict__ out,
                       const DecodeParams p) {
-  __shared__ float sphi[kGroup][D];  // sigma(q)
-  __shared__ float sden[kGroup][kThreads / 32];
+  __shared__ float sphi[NQ][D];  // sigma(q)
+  __shared__ float sden[NQ][kThreads / 32];
+  __shared__ __align__(16) float sr[kThreads / 32][NQ][D];  // per-warp partial retrievals
   const int bh = blockIdx.x, grp = blockIdx.y, t = threadIdx.x, lane = t & 31, w = t >> 5;
   const int q0 = grp * kGroup;
-  const int nq = min(kGroup, p.n - q0);
+  const int nq = min(NQ, p.n - q0);
   const float zt = z[(size_t)bh * D + t];
   for (int i = 0; i < nq; ++i) {
     const float phi = elu1(__bfloat162float(q[((size_t)bh * p.n + q0 + i) * D + t]));
@@ -194,23 +217,37 @@ decode_combine_kernel(const __nv_bfloat16* __restrict__ q, const float* __restri
     if (lane == 0) sden[i][w] = dp;
   }
   __syncthreads();
-  // retrieval: R[i][t] = sum_k sigma(q_i)[k] M[k][t]; the column of M is read once
-  float rr[kGroup];
+  // retrieval R[i][c] = sum_k sigma(q_i)[k] M[k][c]: warp w takes rows k = w, w + 4, ...,
+  // lane takes columns [4 lane, 4 lane + 4) (one 512-byte row per warp load), eight
+  // rows in flight per thread
+  {
+    float4 rr[NQ];
 #pragma unroll
-  for (int i = 0; i < kGroup; ++i) rr[i] = 0.f;
-  const float* Mb = M + (size_t)bh * D * D;
-  for (int k = 0; k < D; ++k) {
-    const float m = Mb[(size_t)k * D + t];
+    for (int i = 0; i < NQ; ++i) rr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* Mb = reinterpret_cast<const float4*>(M + (size_t)bh * D * D);
+#pragma unroll 8
+    for (int k = w; k < D; k += kThreads / 32) {
+      const float4 m = Mb[(size_t)k * (D / 4) + lane];
 #pragma unroll
-    for (int i = 0; i < kGroup; ++i)
-      if (i < nq) rr[i] = fmaf(sphi[i][k], m, rr[i]);
+      for (int i = 0; i < NQ; ++i) {
+        if (i < nq) {
+          const float ph = sphi[i][k];
+          rr[i].x = fmaf(ph, m.x, rr[i].x);
+          rr[i].y = fmaf(ph, m.y, rr[i].y);
+          rr[i].z = fmaf(ph, m.z, rr[i].z);
+          rr[i].w = fmaf(ph, m.w, rr[i].w);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NQ; ++i)
+      if (i < nq) *reinterpret_cast<float4*>(&sr[w][i][4 * lane]) = rr[i];
   }
+  __syncthreads();
   const float bt = beta[bh % p.H];
   const float g = 1.f / (1.f + expf(-bt));
   const float* pb = part + ((size_t)bh * p.groups + grp) * p.splits * kGroup * kPart;
-#pragma unroll
-  for (int i = 0; i < kGroup; ++i) {
-    if (i >= nq) break;
+  for (int i = 0; i < nq; ++i) {
     float m = -INFINITY;
     for (int s = 0; s < p.splits; ++s) m = fmaxf(m, pb[(s * kGroup + i) * kPart]);
     float l = 0.f, a = 0.f;
@@ -222,7 +259,8 @@ decode_combine_kernel(const __nv_bfloat16* __restrict__ q, const float* __restri
       a = fmaf(ps[2 + t], f, a);
     }
     const float den = (sden[i][0] + sden[i][1]) + (sden[i][2] + sden[i][3]);
-    const float amem = den != 0.f ? rr[i] / den : 0.f;
+    const float r = (sr[0][i][t] + sr[1][i][t]) + (sr[2][i][t] + sr[3][i][t]);
+    const float amem = den != 0.f ? r / den : 0.f;
     const float adot = a / l;
     out[((size_t)bh * p.n + q0 + i) * D + t] = __float2bfloat16(g * amem + (1.f - g) * adot);
   }
@@ -241,8 +279,9 @@ size_t bf16_decode_workspace_bytes(int BH, int n, int pos, int sms) {
   return (size_t)BH * groups * splits * kGroup * kPart * sizeof(float);
 }
 
-cudaError_t bf16_decode_launch(const __nv_bfloat16* q, const __nv_bfloat16* k_cache,
-                               const __nv_bfloat16* v_cache, const float* beta, const float* M,
+cudaError_t bf16_decode_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
+                               const __nv_bfloat16* v, __nv_bfloat16* k_cache,
+                               __nv_bfloat16* v_cache, const float* beta, const float* M,
                                const float* z, __nv_bfloat16* out, float* part, int BH, int H,
                                int n, int pos, int N, int sms, cudaStream_t stream) {
   DecodeParams p;
@@ -257,11 +296,24 @@ cudaError_t bf16_decode_launch(const __nv_bfloat16* q, const __nv_bfloat16* k_ca
   if (splits > chunks) splits = chunks;
   p.chunks_per_split = (chunks + splits - 1) / splits;
   p.splits = (chunks + p.chunks_per_split - 1) / p.chunks_per_split;
-  decode_partial_kernel<<<dim3(p.splits, BH, p.groups), kThreads, 0, stream>>>(q, k_cache, v_cache,
-                                                                             part, p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<dim3(BH, p.groups), kThreads, 0, stream>>>(q, part, beta, M, z, out, p);
+  const dim3 gp(p.splits, BH, p.groups), gc(BH, p.groups);
+  // the compiled width must hold the widest group: min(n, 16) queries
+  const int w = n > 8 ? kGroup : n > 4 ? 8 : n > 2 ? 4 : n;
+  switch (w) {
+#define DECODE_CASE(W)                                                                      \
+  case W:                                                                                   \
+    decode_partial_kernel<W><<<gp, kThreads, 0, stream>>>(q, k, v, k_cache, v_cache, part, p); \
+    decode_combine_kernel<W><<<gc, kThreads, 0, stream>>>(q, part, beta, M, z, out, p);      \
+    break;
+    DECODE_CASE(1)
+    DECODE_CASE(2)
+    DECODE_CASE(4)
+    DECODE_CASE(8)
+    DECODE_CASE(16)
+#undef DECODE_CASE
+    default:
+      return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -41,12 +41,14 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                              const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
                              cudaStream_t stream);
 
-// Token-level decode (bf16_decode.cu): partial attention over the KV cache, split
-// like flash decoding, then merge + retrieval from the fp32 state + gate. `part`
-// holds bf16_decode_workspace_bytes(...) bytes.
+// Token-level decode (bf16_decode.cu): partial attention over the KV cache (rows
+// below pos) and the new rows (k, v, also written into the caches), split like flash
+// decoding, then merge + retrieval from the fp32 state + gate. `part` holds
+// bf16_decode_workspace_bytes(...) bytes.
 size_t bf16_decode_workspace_bytes(int BH, int n, int pos, int sms);
-cudaError_t bf16_decode_launch(const __nv_bfloat16* q, const __nv_bfloat16* k_cache,
-                               const __nv_bfloat16* v_cache, const float* beta, const float* M,
+cudaError_t bf16_decode_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
+                               const __nv_bfloat16* v, __nv_bfloat16* k_cache,
+                               __nv_bfloat16* v_cache, const float* beta, const float* M,
                                const float* z, __nv_bfloat16* out, float* part, int BH, int H,
                                int n, int pos, int N, int sms, cudaStream_t stream);
 

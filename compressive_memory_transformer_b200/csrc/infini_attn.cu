@@ -245,10 +245,10 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
-// Token-level decode: append the new rows to the caches, attention + retrieval +
-// gate for the new tokens against the cache and the state as it stands, then, when
-// the segment is complete, the segment's state update in place (the same calls as
-// a one-segment step with M_out == M_in).
+// Token-level decode: attention + retrieval + gate for the new tokens against the
+// cache and the state as it stands (the new rows are also written into the caches),
+// then, when the segment is complete, the segment's state update in place (the same
+// calls as a one-segment step with M_out == M_in).
 int decode_impl(const void* q, const void* k, const void* v, const float* beta, void* k_cache,
                 void* v_cache, float* M, float* z, void* out, int B, int H, int n, int pos,
                 int N, int d, int mode, cudaStream_t stream) {
@@ -277,23 +277,16 @@ int decode_impl(const void* q, const void* k, const void* v, const float* beta, 
   int dev = 0, sms = 148;
   if (prepare_device(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // the new keys and values go to cache rows [pos, pos + n) of every head
-  const size_t row = (size_t)d * 2;
-  if (cudaMemcpy2DAsync(static_cast<char*>(k_cache) + (size_t)pos * row, (size_t)N * row, k,
-                        (size_t)n * row, (size_t)n * row, (size_t)BH, cudaMemcpyDeviceToDevice,
-                        stream) != cudaSuccess ||
-      cudaMemcpy2DAsync(static_cast<char*>(v_cache) + (size_t)pos * row, (size_t)N * row, v,
-                        (size_t)n * row, (size_t)n * row, (size_t)BH, cudaMemcpyDeviceToDevice,
-                        stream) != cudaSuccess)
-    return INFINI_ERR_CUDA;
   Scratch sp;
   int st = get_scratch(sp, bf16_decode_workspace_bytes((int)BH, n, pos, sms), nullptr, stream);
   if (st != INFINI_OK) return st;
   const auto* kcb = static_cast<const __nv_bfloat16*>(k_cache);
   const auto* vcb = static_cast<const __nv_bfloat16*>(v_cache);
-  if (bf16_decode_launch(static_cast<const __nv_bfloat16*>(q), kcb, vcb, beta, M, z,
-                         static_cast<__nv_bfloat16*>(out), static_cast<float*>(sp.ptr), (int)BH, H,
-                         n, pos, N, sms, stream) != cudaSuccess)
+  if (bf16_decode_launch(static_cast<const __nv_bfloat16*>(q),
+                         static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+                         static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache),
+                         beta, M, z, static_cast<__nv_bfloat16*>(out), static_cast<float*>(sp.ptr),
+                         (int)BH, H, n, pos, N, sms, stream) != cudaSuccess)
     return INFINI_ERR_CUDA;
   if (pos + n < N) return INFINI_OK;
   int CH = 1, CL = N;
