@@ -21,10 +21,12 @@
 //                          its group against the chunk (two threads per row, 64
 //                          features each) and keeps one online-softmax partial
 //                          (max, sum, 128 accumulators) per query in exp2 units.
+//                          Four more CTAs per (head, group) compute the retrieval
+//                          sigma(q) M_{s-1} (32 columns each, M read row-coalesced)
+//                          and sigma(q) z_{s-1}, beside the cache reads.
 //   decode_combine_kernel  grid (BH, query groups). Merges the splits' partials,
-//                          adds the retrieval from the fp32 state (M read once per
-//                          group, row-coalesced float4 loads spread over the four
-//                          warps) and the gate, writes out in bf16.
+//                          divides the retrieval by its denominator, applies the
+//                          gate and writes out in bf16.
 // Both kernels are compiled for query-group widths 1, 2, 4, 8 and 16, so a single
 // token carries no idle accumulators.
 #include <cuda_runtime.h>
@@ -42,6 +44,9 @@ constexpr int kRows = 64;     // cache rows per chunk
 constexpr int kGroup = 16;    // queries per CTA
 constexpr int kThreads = 128;
 constexpr int kPart = 2 + D;  // one partial: max, sum, 128 accumulators
+constexpr int kMaxSplits = 512;
+constexpr int kRetCTAs = 4;   // retrieval CTAs per (head, group), 32 columns of M each
+constexpr int kRet = D + 1;   // one retrieval record: sigma(q) M (128), sigma(q) z
 
 struct DecodeParams {
   int n, pos, N, H, splits, chunks_per_split, groups;
@@ -51,11 +56,12 @@ __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u <<
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
 template <int NQ>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)  // four CTAs per SM (shared memory allows four)
 decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ knew,
                       const __nv_bfloat16* __restrict__ vnew, __nv_bfloat16* __restrict__ kc,
-                      __nv_bfloat16* __restrict__ vc, float* __restrict__ part,
-                      const DecodeParams p) {
+                      __nv_bfloat16* __restrict__ vc, const float* __restrict__ M,
+                      const float* __restrict__ z, float* __restrict__ part,
+                      float* __restrict__ ret, const DecodeParams p) {
   __shared__ __align__(16) float sq[kGroup][D];    // queries, scaled by log2(e) / sqrt(d)
   __shared__ __align__(16) uint32_t sk[kRows][D / 2];  // bf16 pairs
   __shared__ __align__(16) uint32_t sv[kRows][D / 2];
@@ -67,6 +73,51 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
   const int q0 = grp * kGroup;
   const int nq = min(kGroup, p.n - q0);
   const float sl = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+
+  if (split >= p.splits) {
+    // retrieval CTA cb: columns [32 cb, 32 cb + 32) of sigma(q) M_{s-1}; cb 0 also
+    // forms sigma(q) z_{s-1}
+    const int cb = split - p.splits, lane = t & 31, w = t >> 5;
+    float (*sphi)[D] = sq;
+    for (int i = 0; i < nq; ++i)
+      sphi[i][t] = elu1(__bfloat162float(q[((size_t)bh * p.n + q0 + i) * D + t]));
+    __syncthreads();
+    float* rec = ret + ((size_t)bh * p.groups + grp) * kGroup * kRet;
+    if (cb == 0) {
+      const float zt = z[(size_t)bh * D + t];
+      for (int i = 0; i < nq; ++i) {
+        float dp = sphi[i][t] * zt;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dp += __shfl_xor_sync(0xffffffffu, dp, o);
+        if (lane == 0) ss[i][w] = dp;
+      }
+    }
+    float acc[NQ];
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) acc[i] = 0.f;
+    const float* Mc = M + (size_t)bh * D * D + 32 * cb + lane;
+#pragma unroll 8
+    for (int k = w; k < D; k += kThreads / 32) {
+      const float m = Mc[(size_t)k * D];
+#pragma unroll
+      for (int i = 0; i < NQ; ++i)
+        if (i < nq) acc[i] = fmaf(sphi[i][k], m, acc[i]);
+    }
+    float (*red)[NQ][32] = reinterpret_cast<float (*)[NQ][32]>(&sk[0][0]);
+#pragma unroll
+    for (int i = 0; i < NQ; ++i)
+      if (i < nq) red[w][i][lane] = acc[i];
+    __syncthreads();
+    if (w == 0) {
+#pragma unroll
+      for (int i = 0; i < NQ; ++i)
+        if (i < nq)
+          rec[i * kRet + 32 * cb + lane] = (red[0][i][lane] + red[1][i][lane]) +
+                                           (red[2][i][lane] + red[3][i][lane]);
+    }
+    if (cb == 0 && t < nq) rec[t * kRet + D] = (ss[t][0] + ss[t][1]) + (ss[t][2] + ss[t][3]);
+    return;
+  }
 
   for (int i = 0; i < nq; ++i)
     sq[i][t] = __bfloat162float(q[((size_t)bh * p.n + q0 + i) * D + t]) * sl;
@@ -88,53 +139,69 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
     const int nr = min(kRows, r_end - r0);
     __syncthreads();  // the previous chunk's readers are done
     // K and V rows [r0, r0 + nr): 16 bytes per thread per step, row-contiguous
-    for (int e = t; e < nr * (D / 8); e += kThreads) {
+    // asynchronous 16-byte copies, all in flight before one wait
+#pragma unroll
+    for (int it = 0; it < kRows * (D / 8) / kThreads; ++it) {
+      const int e = t + it * kThreads;
       const int row = e / (D / 8), c = e % (D / 8);
       const int R = r0 + row;
-      uint4 kk, vv;
-      if (R < p.pos) {
-        kk = *reinterpret_cast<const uint4*>(kc + base + (size_t)R * D + c * 8);
-        vv = *reinterpret_cast<const uint4*>(vc + base + (size_t)R * D + c * 8);
-      } else {
-        const size_t src = ((size_t)bh * p.n + (R - p.pos)) * D + c * 8;
-        kk = *reinterpret_cast<const uint4*>(knew + src);
-        vv = *reinterpret_cast<const uint4*>(vnew + src);
-        if (writer) {
-          *reinterpret_cast<uint4*>(kc + base + (size_t)R * D + c * 8) = kk;
-          *reinterpret_cast<uint4*>(vc + base + (size_t)R * D + c * 8) = vv;
+      if (row < nr) {
+        const __nv_bfloat16* ks;
+        const __nv_bfloat16* vs;
+        if (R < p.pos) {
+          ks = kc + base + (size_t)R * D + c * 8;
+          vs = vc + base + (size_t)R * D + c * 8;
+        } else {
+          const size_t src = ((size_t)bh * p.n + (R - p.pos)) * D + c * 8;
+          ks = knew + src;
+          vs = vnew + src;
         }
+        cp_async16(&sk[row][c * 4], ks);
+        cp_async16(&sv[row][c * 4], vs);
       }
-      *reinterpret_cast<uint4*>(&sk[row][c * 4]) = kk;
-      *reinterpret_cast<uint4*>(&sv[row][c * 4]) = vv;
     }
+    cp_async_wait_all();
     __syncthreads();
-    // scores: thread pair (2r, 2r + 1) covers row r, features [64h, 64h + 64); the
-    // pair word read at step j is rotated by 2r + h, so a warp's 32 reads fall in 32
+    // the last group also writes the new rows it staged into the caches
+    if (writer && r0 + nr > p.pos) {
+      const int first = max(0, p.pos - r0);
+      for (int e = first * (D / 8) + t; e < nr * (D / 8); e += kThreads) {
+        const int row = e / (D / 8), c = e % (D / 8);
+        const size_t dst = base + (size_t)(r0 + row) * D + c * 8;
+        *reinterpret_cast<uint4*>(kc + dst) = *reinterpret_cast<const uint4*>(&sk[row][c * 4]);
+        *reinterpret_cast<uint4*>(vc + dst) = *reinterpret_cast<const uint4*>(&sv[row][c * 4]);
+      }
+    }
+    // scores: thread pair (2r, 2r + 1) covers row r, features [64h, 64h + 64); each
+    // key pair is read from shared memory once for all the group's queries; the pair
+    // word read at step j is rotated by 2r + h, so a warp's 32 reads fall in 32
     // different banks
     {
       const int r = t >> 1, h = t & 1;
-      float kf[64];
+      float sc[NQ];
+#pragma unroll
+      for (int i = 0; i < NQ; ++i) sc[i] = 0.f;
       if (r < nr) {
-#pragma unroll
+#pragma unroll 8
         for (int j = 0; j < 32; ++j) {
-          const uint32_t u = sk[r][32 * h + ((j + 2 * r + h) & 31)];
-          kf[2 * j] = bf_lo(u);
-          kf[2 * j + 1] = bf_hi(u);
-        }
-      }
-      for (int i = 0; i < nq; ++i) {
-        float s = 0.f;
-        if (r < nr) {
+          const int jj = (j + 2 * r + h) & 31;
+          const uint32_t u = sk[r][32 * h + jj];
+          const float k0 = bf_lo(u), k1 = bf_hi(u);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int f = 64 * h + 2 * ((j + 2 * r + h) & 31);
-            const float2 qf = *reinterpret_cast<const float2*>(&sq[i][f]);
-            s = fmaf(qf.x, kf[2 * j], s);
-            s = fmaf(qf.y, kf[2 * j + 1], s);
+          for (int i = 0; i < NQ; ++i) {
+            if (i < nq) {
+              const float2 qf = *reinterpret_cast<const float2*>(&sq[i][64 * h + 2 * jj]);
+              sc[i] = fmaf(qf.x, k0, fmaf(qf.y, k1, sc[i]));
+            }
           }
         }
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        if (h == 0) ss[i][r] = (r < nr && r0 + r <= p.pos + q0 + i) ? s : -INFINITY;
+      }
+#pragma unroll
+      for (int i = 0; i < NQ; ++i) {
+        if (i < nq) {
+          const float sv2 = sc[i] + __shfl_xor_sync(0xffffffffu, sc[i], 1);
+          if (h == 0) ss[i][r] = (r < nr && r0 + r <= p.pos + q0 + i) ? sv2 : -INFINITY;
+        }
       }
     }
     __syncthreads();
@@ -197,86 +264,62 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
 
 template <int NQ>
 __global__ void __launch_bounds__(kThreads)
-decode_combine_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ part,
-                      const float* __restrict__ beta, const float* __restrict__ M,
-                      const float* __restrict__ z, __nv_bfloat16* __restrict__ out,
+decode_combine_kernel(const float* __restrict__ part, const float* __restrict__ ret,
+                      const float* __restrict__ beta, __nv_bfloat16* __restrict__ out,
                       const DecodeParams p) {
-  __shared__ float sphi[NQ][D];  // sigma(q)
-  __shared__ float sden[NQ][kThreads / 32];
-  __shared__ __align__(16) float sr[kThreads / 32][NQ][D];  // per-warp partial retrievals
-  const int bh = blockIdx.x, grp = blockIdx.y, t = threadIdx.x, lane = t & 31, w = t >> 5;
+  __shared__ float sml[kMaxSplits][2];  // splits' (max, sum)
+  const int bh = blockIdx.x, grp = blockIdx.y, t = threadIdx.x;
   const int q0 = grp * kGroup;
   const int nq = min(NQ, p.n - q0);
-  const float zt = z[(size_t)bh * D + t];
-  for (int i = 0; i < nq; ++i) {
-    const float phi = elu1(__bfloat162float(q[((size_t)bh * p.n + q0 + i) * D + t]));
-    sphi[i][t] = phi;
-    float dp = phi * zt;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) dp += __shfl_xor_sync(0xffffffffu, dp, o);
-    if (lane == 0) sden[i][w] = dp;
-  }
-  __syncthreads();
-  // retrieval R[i][c] = sum_k sigma(q_i)[k] M[k][c]: warp w takes rows k = w, w + 4, ...,
-  // lane takes columns [4 lane, 4 lane + 4) (one 512-byte row per warp load), eight
-  // rows in flight per thread
-  {
-    float4 rr[NQ];
-#pragma unroll
-    for (int i = 0; i < NQ; ++i) rr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4* Mb = reinterpret_cast<const float4*>(M + (size_t)bh * D * D);
-#pragma unroll 8
-    for (int k = w; k < D; k += kThreads / 32) {
-      const float4 m = Mb[(size_t)k * (D / 4) + lane];
-#pragma unroll
-      for (int i = 0; i < NQ; ++i) {
-        if (i < nq) {
-          const float ph = sphi[i][k];
-          rr[i].x = fmaf(ph, m.x, rr[i].x);
-          rr[i].y = fmaf(ph, m.y, rr[i].y);
-          rr[i].z = fmaf(ph, m.z, rr[i].z);
-          rr[i].w = fmaf(ph, m.w, rr[i].w);
-        }
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < NQ; ++i)
-      if (i < nq) *reinterpret_cast<float4*>(&sr[w][i][4 * lane]) = rr[i];
-  }
-  __syncthreads();
   const float bt = beta[bh % p.H];
   const float g = 1.f / (1.f + expf(-bt));
   const float* pb = part + ((size_t)bh * p.groups + grp) * p.splits * kGroup * kPart;
+  const float* rec = ret + ((size_t)bh * p.groups + grp) * kGroup * kRet;
   for (int i = 0; i < nq; ++i) {
-    float m = -INFINITY;
-    for (int s = 0; s < p.splits; ++s) m = fmaxf(m, pb[(s * kGroup + i) * kPart]);
-    float l = 0.f, a = 0.f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float* ps = pb + (s * kGroup + i) * kPart;
-      if (ps[0] == -INFINITY) continue;  // this split saw none of the query's rows
-      const float f = exp2f(ps[0] - m);
-      l = fmaf(ps[1], f, l);
-      a = fmaf(ps[2 + t], f, a);
+    // every split's (max, sum) in parallel, then the weights
+    for (int s = t; s < p.splits; s += kThreads) {
+      sml[s][0] = pb[(s * kGroup + i) * kPart];
+      sml[s][1] = pb[(s * kGroup + i) * kPart + 1];
     }
-    const float den = (sden[i][0] + sden[i][1]) + (sden[i][2] + sden[i][3]);
-    const float r = (sr[0][i][t] + sr[1][i][t]) + (sr[2][i][t] + sr[3][i][t]);
-    const float amem = den != 0.f ? r / den : 0.f;
+    __syncthreads();
+    float m = -INFINITY;
+    for (int s = 0; s < p.splits; ++s) m = fmaxf(m, sml[s][0]);
+    float l = 0.f, a = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < p.splits; ++s) {
+      // a split that saw none of the query's rows has max -inf and weight 0
+      const float f = sml[s][0] == -INFINITY ? 0.f : exp2f(sml[s][0] - m);
+      l = fmaf(sml[s][1], f, l);
+      a = fmaf(pb[(s * kGroup + i) * kPart + 2 + t], f, a);
+    }
+    __syncthreads();
+    const float den = rec[i * kRet + D];
+    const float amem = den != 0.f ? rec[i * kRet + t] / den : 0.f;
     const float adot = a / l;
     out[((size_t)bh * p.n + q0 + i) * D + t] = __float2bfloat16(g * amem + (1.f - g) * adot);
   }
 }
 
+// Cache split: one 64-row chunk per CTA while that keeps the grid within four CTAs
+// per SM, more chunks per CTA beyond; at most kMaxSplits splits.
+void decode_splits(int BH, int n, int pos, int sms, int* splits, int* cps) {
+  const int groups = (n + kGroup - 1) / kGroup;
+  const int chunks = (pos + n + kRows - 1) / kRows;
+  const long long want = (4LL * sms + (long long)BH * groups - 1) / ((long long)BH * groups);
+  int s = want < 1 ? 1 : (want > kMaxSplits ? kMaxSplits : (int)want);
+  if (s > chunks) s = chunks;
+  *cps = (chunks + s - 1) / s;
+  *splits = (chunks + *cps - 1) / *cps;
+}
+
 }  // namespace
 
 size_t bf16_decode_workspace_bytes(int BH, int n, int pos, int sms) {
+  int splits = 0, cps = 0;
+  decode_splits(BH, n, pos, sms, &splits, &cps);
   const int groups = (n + kGroup - 1) / kGroup;
-  const int chunks = (pos + n + kRows - 1) / kRows;
-  const int want = (2 * sms + BH * groups - 1) / (BH * groups);
-  int splits = want < 1 ? 1 : want;
-  if (splits > chunks) splits = chunks;
-  const int cps = (chunks + splits - 1) / splits;
-  splits = (chunks + cps - 1) / cps;
-  return (size_t)BH * groups * splits * kGroup * kPart * sizeof(float);
+  return ((size_t)BH * groups * splits * kGroup * kPart + (size_t)BH * groups * kGroup * kRet) *
+         sizeof(float);
 }
 
 cudaError_t bf16_decode_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
@@ -290,20 +333,17 @@ cudaError_t bf16_decode_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   p.N = N;
   p.H = H;
   p.groups = (n + kGroup - 1) / kGroup;
-  const int chunks = (pos + n + kRows - 1) / kRows;
-  const int want = (2 * sms + BH * p.groups - 1) / (BH * p.groups);
-  int splits = want < 1 ? 1 : want;
-  if (splits > chunks) splits = chunks;
-  p.chunks_per_split = (chunks + splits - 1) / splits;
-  p.splits = (chunks + p.chunks_per_split - 1) / p.chunks_per_split;
-  const dim3 gp(p.splits, BH, p.groups), gc(BH, p.groups);
+  decode_splits(BH, n, pos, sms, &p.splits, &p.chunks_per_split);
+  const dim3 gp(p.splits + kRetCTAs, BH, p.groups), gc(BH, p.groups);
+  float* ret = part + (size_t)BH * p.groups * p.splits * kGroup * kPart;
   // the compiled width must hold the widest group: min(n, 16) queries
   const int w = n > 8 ? kGroup : n > 4 ? 8 : n > 2 ? 4 : n;
   switch (w) {
 #define DECODE_CASE(W)                                                                      \
   case W:                                                                                   \
-    decode_partial_kernel<W><<<gp, kThreads, 0, stream>>>(q, k, v, k_cache, v_cache, part, p); \
-    decode_combine_kernel<W><<<gc, kThreads, 0, stream>>>(q, part, beta, M, z, out, p);      \
+    decode_partial_kernel<W><<<gp, kThreads, 0, stream>>>(q, k, v, k_cache, v_cache, M, z,    \
+                                                          part, ret, p);                    \
+    decode_combine_kernel<W><<<gc, kThreads, 0, stream>>>(part, ret, beta, out, p);          \
     break;
     DECODE_CASE(1)
     DECODE_CASE(2)

@@ -136,6 +136,17 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0,
                : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (no register round trip), and the
+// wait for all of this thread's outstanding ones.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(reinterpret_cast<uint64_t>(gsrc))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Wait until every committed bulk store of this thread has finished reading its
 // shared-memory source (the source may then be rewritten).
 __device__ __forceinline__ void bulk_wait_group_read0() {
