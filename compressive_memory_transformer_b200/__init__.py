@@ -8,6 +8,8 @@ Entry points (same names as the C ABI in include/infini_attn.h):
     infini_attn_forward(q, k, v, beta, N, mode, M_in=None, z_in=None, ...)
     infini_attn_step(q, k, v, beta, mode, M_in=None, z_in=None, ...)
     infini_attn_decode(q, k, v, beta, k_cache, v_cache, M, z, pos, mode, ...)
+    infini_attn_state_update(k, v, N, mode, M_in=None, z_in=None, ...)
+    infini_attn_state_sum(dM, dz, M_in=None, z_in=None, ...)
 q, k, v: [B, H, L, d] CUDA tensors, bf16 (d = 128) or fp32 (d <= 128);
 beta: [H] fp32; M: [B, H, d, d] fp32; z: [B, H, d] fp32.
 """
@@ -51,6 +53,8 @@ _SIGS = {
     "infini_attn_step_f32": [_vp] * 9 + [_i, _i, _i, _i, _i, _vp],
     "infini_attn_forward_ex": [_vp] * 9 + [_i, _i, _ll, _i, _i, _i, _i, ctypes.POINTER(Opts), _vp],
     "infini_attn_decode": [_vp] * 9 + [_i] * 7 + [_vp],
+    "infini_attn_state_update": [_vp] * 6 + [_i, _i, _ll, _i, _i, _i, _vp],
+    "infini_attn_state_sum": [_vp, _vp, _i] + [_vp] * 4 + [_i, _i, _i, _vp],
     "infini_attn_workspace_size": [_i, _i, _ll, _i, _i, _i, _i],
     "infini_attn_device_status": [],
     "infini_attn_selftest_timeout": [_ll, _vp],
@@ -165,6 +169,46 @@ def infini_attn_forward_ex(q, k, v, beta, N, mode=LINEAR, M_in=None, z_in=None, 
                                        int(N), d, int(mode), dtype, ctypes.byref(o),
                                        _stream_handle(stream)))
     return out, M_out, z_out
+
+
+def infini_attn_state_update(k, v, N, mode=LINEAR, M_in=None, z_in=None, M_out=None, z_out=None,
+                             stream=None):
+    """The memory update alone over k, v [B, H, L, d] (bf16, segments of N) from
+    (M_in, z_in) (None: the zero state); returns (M_out, z_out)."""
+    if k.dim() != 4 or k.dtype != torch.bfloat16:
+        raise ValueError("k, v must be [B, H, L, d] bf16")
+    B, H, L, d = k.shape
+    if v.shape != k.shape or v.dtype != k.dtype or not (k.is_cuda and v.is_cuda) or not (
+            k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("k and v must be contiguous CUDA tensors of the same shape")
+    if M_out is None:
+        M_out = torch.empty((B, H, d, d), device=k.device, dtype=torch.float32)
+        z_out = torch.empty((B, H, d), device=k.device, dtype=torch.float32)
+    for t in (M_in, z_in, M_out, z_out):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda):
+            raise ValueError("M and z must be contiguous CUDA fp32 tensors")
+    _check(_lib.infini_attn_state_update(_ptr(k), _ptr(v), _ptr(M_in), _ptr(z_in), _ptr(M_out),
+                                         _ptr(z_out), B, H, L, int(N), d, int(mode),
+                                         _stream_handle(stream)))
+    return M_out, z_out
+
+
+def infini_attn_state_sum(dM, dz, M_in=None, z_in=None, M_out=None, z_out=None, stream=None):
+    """(M_in, z_in) (None: zero) plus the sum of the blocks dM [count, B, H, d, d],
+    dz [count, B, H, d] (fp32, CUDA), in block order; returns (M_out, z_out)."""
+    count, B, H, d = dM.shape[0], dM.shape[1], dM.shape[2], dM.shape[3]
+    if dM.shape != (count, B, H, d, d) or dz.shape != (count, B, H, d):
+        raise ValueError("dM must be [count, B, H, d, d] and dz [count, B, H, d]")
+    if M_out is None:
+        M_out = torch.empty((B, H, d, d), device=dM.device, dtype=torch.float32)
+        z_out = torch.empty((B, H, d), device=dM.device, dtype=torch.float32)
+    for t in (dM, dz, M_in, z_in, M_out, z_out):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda):
+            raise ValueError("states must be contiguous CUDA fp32 tensors")
+    _check(_lib.infini_attn_state_sum(_ptr(dM) if count else None, _ptr(dz) if count else None,
+                                      count, _ptr(M_in), _ptr(z_in), _ptr(M_out), _ptr(z_out), B,
+                                      H, d, _stream_handle(stream)))
+    return M_out, z_out
 
 
 def infini_attn_decode(q, k, v, beta, k_cache, v_cache, M, z, pos, mode=LINEAR, out=None,

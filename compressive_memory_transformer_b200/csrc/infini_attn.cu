@@ -69,6 +69,24 @@ __global__ void pass_state_kernel(const float* M_in, const float* z_in, float* M
   }
 }
 
+// (M_out, z_out) = (M_in, z_in) (or zero) + the sum of `count` state blocks, added in
+// block order (the Linear memory is a plain sum over segments, section 3.4).
+__global__ void state_sum_kernel(const float* dM, const float* dz, int count, const float* M_in,
+                                 const float* z_in, float* M_out, float* z_out, long long nM,
+                                 long long nz) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nM;
+       i += (long long)gridDim.x * blockDim.x) {
+    float m = M_in ? M_in[i] : 0.f;
+    for (int c = 0; c < count; ++c) m += dM[(long long)c * nM + i];
+    M_out[i] = m;
+    if (i < nz) {
+      float zz = z_in ? z_in[i] : 0.f;
+      for (int c = 0; c < count; ++c) zz += dz[(long long)c * nz + i];
+      z_out[i] = zz;
+    }
+  }
+}
+
 __global__ void timeout_selftest_kernel(unsigned long long timeout_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -245,6 +263,46 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
+// The state path alone: (M_out, z_out) after L tokens (segments of N) from (M_in,
+// z_in), without the attention outputs.
+int state_update_impl(const void* k, const void* v, const float* M_in, const float* z_in,
+                      float* M_out, float* z_out, int B, int H, long long L, int N, int d,
+                      int mode, cudaStream_t stream) {
+  if (!M_out || !z_out) return INFINI_ERR_NULL;
+  if (L > 0 && (!k || !v)) return INFINI_ERR_NULL;
+  if ((M_in == nullptr) != (z_in == nullptr)) return INFINI_ERR_NULL;
+  if (B < 1 || H < 1 || N < 1 || L < 0 || d < 1) return INFINI_ERR_SHAPE;
+  if (mode != INFINI_LINEAR && mode != INFINI_DELTA) return INFINI_ERR_UNSUPPORTED;
+  if (d != 128) return INFINI_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > (1LL << 30) || overflows(BH, L) || overflows(BH * L, (long long)d * 2) ||
+      L >= (1LL << 31))
+    return INFINI_ERR_SHAPE;
+  if ((L > 0 && (!aligned16(k) || !aligned16(v))) || (M_in && !aligned16(M_in)) ||
+      !aligned16(M_out))
+    return INFINI_ERR_ALIGN;
+  const size_t nio = (size_t)(BH * L * d) * 2;
+  const size_t nM = (size_t)BH * d * d * sizeof(float), nz = (size_t)BH * d * sizeof(float);
+  if (overlap(M_out, nM, k, nio) || overlap(M_out, nM, v, nio) || overlap(z_out, nz, k, nio) ||
+      overlap(z_out, nz, v, nio) || overlap(M_out, nM, z_out, nz))
+    return INFINI_ERR_ALIAS;
+  if (L == 0) return pass_state(M_in, z_in, M_out, z_out, BH, d, stream);
+  int dev = 0;
+  if (prepare_device(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
+  const int S = (int)((L + N - 1) / N);
+  int CH = 1, CL = N;
+  bf16_state_plan((int)BH, S, N, &CH, &CL);
+  if (BH * S * CH >= (1LL << 31)) return INFINI_ERR_SHAPE;
+  Scratch sc;
+  const int st = get_scratch(sc, bf16_workspace_bytes((int)BH, S, CH), nullptr, stream);
+  if (st != INFINI_OK) return st;
+  const Bf16Workspace ws = bf16_workspace_carve(sc.ptr, (int)BH, S, CH);
+  const cudaError_t e = bf16_state_launch(static_cast<const __nv_bfloat16*>(k),
+                                          static_cast<const __nv_bfloat16*>(v), M_in, z_in, M_out,
+                                          z_out, ws, (int)BH, L, N, S, CH, CL, mode, 0, stream);
+  return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
 // Token-level decode: attention + retrieval + gate for the new tokens against the
 // cache and the state as it stands (the new rows are also written into the caches),
 // then, when the segment is complete, the segment's state update in place (the same
@@ -336,6 +394,37 @@ int infini_attn_step_f32(const float* q, const float* k, const float* v, const f
                          float* z_out, int B, int H, int N, int d, int mode, void* stream) {
   return forward_impl(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, N, N < 1 ? 1 : N, d,
                       mode, INFINI_DTYPE_F32, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int infini_attn_state_sum(const float* dM, const float* dz, int count, const float* M_in,
+                          const float* z_in, float* M_out, float* z_out, int B, int H, int d,
+                          void* stream) {
+  if (!M_out || !z_out || (count > 0 && (!dM || !dz))) return INFINI_ERR_NULL;
+  if ((M_in == nullptr) != (z_in == nullptr)) return INFINI_ERR_NULL;
+  if (B < 1 || H < 1 || d < 1 || count < 0) return INFINI_ERR_SHAPE;
+  const long long BH = (long long)B * H;
+  if (BH > (1LL << 30) || overflows(BH * d, (long long)d) || overflows(BH * d * d, (long long)count + 1))
+    return INFINI_ERR_SHAPE;
+  const long long nM = BH * d * d, nz = BH * d;
+  const size_t bM = (size_t)nM * sizeof(float), bz = (size_t)nz * sizeof(float);
+  if (overlap(M_out, bM, dM, bM * count) || overlap(M_out, bM, dz, bz * count) ||
+      overlap(z_out, bz, dM, bM * count) || overlap(z_out, bz, dz, bz * count) ||
+      overlap(M_out, bM, z_out, bz))
+    return INFINI_ERR_ALIAS;
+  int dev = 0;
+  if (prepare_device(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  state_sum_kernel<<<(unsigned)min((nM + 255) / 256, 4096LL), 256, 0, st>>>(dM, dz, count, M_in,
+                                                                           z_in, M_out, z_out,
+                                                                           nM, nz);
+  return cudaGetLastError() == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+int infini_attn_state_update(const void* k, const void* v, const float* M_in, const float* z_in,
+                             float* M_out, float* z_out, int B, int H, long long L, int N, int d,
+                             int mode, void* stream) {
+  return state_update_impl(k, v, M_in, z_in, M_out, z_out, B, H, L, N, d, mode,
+                           static_cast<cudaStream_t>(stream));
 }
 
 int infini_attn_decode(const void* q, const void* k, const void* v, const float* beta,

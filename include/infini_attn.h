@@ -113,6 +113,34 @@ int infini_attn_step_static(const void* q, const void* k, const void* v, const f
                             float* z_out, int B, int H, int N, int d, int mode, void* stream);
 
 /*
+ * The memory update alone (section 3.4, Linear or Linear+Delta, applied segment by
+ * segment): (M_out, z_out) after L tokens of bf16 k, v [B, H, L, d] cut into
+ * segments of N (the last may be shorter), starting from (M_in, z_in) (NULL: the
+ * zero state); no attention outputs. For Linear the result is M_in + sum over
+ * segments of sigma(K_s)^T V_s and z_in + sum of sigma(K_s) rows, so a sequence split
+ * into consecutive ranges can be processed range by range, or on several GPUs: each
+ * range's sum from the zero state, an all-gather, and every range's forward from the
+ * sum of the ranges before it. Requires d == 128; M_out, z_out required (they may
+ * be M_in, z_in); 16-byte aligned k, v, M_in, M_out; the state must not overlap k, v.
+ * Scratch from the stream-ordered allocator on `stream` (INFINI_ERR_NOMEM).
+ */
+int infini_attn_state_update(const void* k, const void* v, const float* M_in, const float* z_in,
+                             float* M_out, float* z_out, int B, int H, long long L, int N, int d,
+                             int mode, void* stream);
+
+/*
+ * (M_out, z_out) = (M_in, z_in) + the sum of `count` state blocks dM [count, B, H, d, d]
+ * and dz [count, B, H, d] (fp32, device), added in block order (deterministic).
+ * M_in / z_in NULL: the zero state; count may be 0. With infini_attn_state_update this
+ * composes Linear-mode states of consecutive ranges of a sequence (section 3.4: the
+ * Linear memory is a plain sum over segments). M_out, z_out must not overlap the
+ * blocks (they may be M_in, z_in).
+ */
+int infini_attn_state_sum(const float* dM, const float* dz, int count, const float* M_in,
+                          const float* z_in, float* M_out, float* z_out, int B, int H, int d,
+                          void* stream);
+
+/*
  * Token-level streaming decode (the pages' "fast streaming inference": section 3.1
  * attention and section 3.3 retrieval for tokens that arrive one or a few at a
  * time inside a segment). n new tokens of every (b, h) join the current segment,

@@ -128,3 +128,38 @@ def call_decode(lib, q=FAKE, k=FAKE + 4096, v=FAKE + 8192, beta=FAKE + 12288, k_
 def test_decode_rejects_bad_arguments(lib, kw, code):
     """Every argument error is reported on the host, before any CUDA call."""
     assert call_decode(lib, **kw) == code
+
+
+def call_state_update(lib, k=FAKE, v=FAKE + 65536, M_in=None, z_in=None, M_out=FAKE * 4,
+                      z_out=FAKE * 4 + 65536, B=1, H=1, L=128, N=128, d=128, mode=0):
+    return lib.raw_call("infini_attn_state_update", k, v, M_in, z_in, M_out, z_out, B, H, L, N, d,
+                        mode, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), -1), (dict(v=None), -1), (dict(M_out=None), -1), (dict(z_out=None), -1),
+    (dict(M_in=FAKE * 8), -1),            # M_in without z_in
+    (dict(B=0), -2), (dict(N=0), -2), (dict(L=-1), -2), (dict(L=1 << 31), -2),
+    (dict(d=64), -3), (dict(mode=2), -3),
+    (dict(k=FAKE + 8), -4), (dict(M_out=FAKE * 4 + 4), -4),
+    (dict(M_out=FAKE), -8),               # the state over k
+    (dict(z_out=FAKE * 4 + 1024), -8),    # z inside M
+])
+def test_state_update_rejects_bad_arguments(lib, kw, code):
+    assert call_state_update(lib, **kw) == code
+
+
+def test_state_sum_rejects_bad_arguments(lib):
+    ok = dict(dM=FAKE, dz=FAKE * 2, count=2, M_in=None, z_in=None, M_out=FAKE * 4,
+              z_out=FAKE * 5, B=1, H=1, d=128)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.raw_call("infini_attn_state_sum", a["dM"], a["dz"], a["count"], a["M_in"],
+                            a["z_in"], a["M_out"], a["z_out"], a["B"], a["H"], a["d"], None)
+    assert call(M_out=None) == -1
+    assert call(dM=None) == -1
+    assert call(M_in=FAKE * 6) == -1      # M_in without z_in
+    assert call(count=-1) == -2
+    assert call(B=0) == -2
+    assert call(M_out=FAKE + 4096) == -8  # M_out inside the blocks
