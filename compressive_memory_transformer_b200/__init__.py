@@ -8,6 +8,7 @@ Entry points (same names as the C ABI in include/infini_attn.h):
     infini_attn_forward(q, k, v, beta, N, mode, M_in=None, z_in=None, ...)
     infini_attn_step(q, k, v, beta, mode, M_in=None, z_in=None, ...)
     infini_attn_decode(q, k, v, beta, k_cache, v_cache, M, z, pos, mode, ...)
+    infini_attn_forward_gqa(q, k, v, beta, N, mode, layout, ...)
     infini_attn_state_update(k, v, N, mode, M_in=None, z_in=None, ...)
     infini_attn_state_sum(dM, dz, M_in=None, z_in=None, ...)
 q, k, v: [B, H, L, d] CUDA tensors, bf16 (d = 128) or fp32 (d <= 128);
@@ -22,6 +23,8 @@ import torch
 
 LINEAR = 0
 DELTA = 1
+LAYOUT_BHLD = 0  # [B, H, L, d]
+LAYOUT_BLHD = 1  # [B, L, H, d]
 DTYPE_BF16 = 0
 DTYPE_F32 = 1
 
@@ -54,6 +57,7 @@ _SIGS = {
     "infini_attn_forward_ex": [_vp] * 9 + [_i, _i, _ll, _i, _i, _i, _i, ctypes.POINTER(Opts), _vp],
     "infini_attn_decode": [_vp] * 9 + [_i] * 7 + [_vp],
     "infini_attn_state_update": [_vp] * 6 + [_i, _i, _ll, _i, _i, _i, _vp],
+    "infini_attn_forward_gqa": [_vp] * 9 + [_i, _i, _i, _ll, _i, _i, _i, _i, _vp],
     "infini_attn_state_sum": [_vp, _vp, _i] + [_vp] * 4 + [_i, _i, _i, _vp],
     "infini_attn_workspace_size": [_i, _i, _ll, _i, _i, _i, _i],
     "infini_attn_device_status": [],
@@ -168,6 +172,47 @@ def infini_attn_forward_ex(q, k, v, beta, N, mode=LINEAR, M_in=None, z_in=None, 
                                        _ptr(z_in), _ptr(out), _ptr(M_out), _ptr(z_out), B, H, L,
                                        int(N), d, int(mode), dtype, ctypes.byref(o),
                                        _stream_handle(stream)))
+    return out, M_out, z_out
+
+
+def infini_attn_forward_gqa(q, k, v, beta, N, mode=LINEAR, layout=LAYOUT_BHLD, M_in=None,
+                            z_in=None, out=None, M_out=None, z_out=None, state_out=True,
+                            stream=None):
+    """Forward with grouped key/value heads and a choice of layout (bf16, d = 128).
+    LAYOUT_BHLD: q [B, H, L, d], k/v [B, H_kv, L, d]; LAYOUT_BLHD: q [B, L, H, d], k/v
+    [B, L, H_kv, d]; out is laid out as q. M/z are per key/value head: [B, H_kv, d, d]
+    and [B, H_kv, d]. Returns (out, M_out, z_out)."""
+    if q.dim() != 4 or q.dtype != torch.bfloat16:
+        raise ValueError("q, k, v must be 4-d bf16 tensors")
+    if layout == LAYOUT_BHLD:
+        B, H, L, d = q.shape
+        H_kv = k.shape[1]
+        kv_shape = (B, H_kv, L, d)
+    elif layout == LAYOUT_BLHD:
+        B, L, H, d = q.shape
+        H_kv = k.shape[2]
+        kv_shape = (B, L, H_kv, d)
+    else:
+        raise ValueError("layout must be LAYOUT_BHLD or LAYOUT_BLHD")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor")
+    if tuple(k.shape) != kv_shape or tuple(v.shape) != kv_shape:
+        raise ValueError(f"k and v must be {kv_shape}")
+    if beta.dtype != torch.float32 or beta.numel() != H or not beta.is_cuda:
+        raise ValueError("beta must be a CUDA fp32 tensor with H elements")
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out and M_out is None:
+        M_out = torch.empty((B, H_kv, d, d), device=q.device, dtype=torch.float32)
+        z_out = torch.empty((B, H_kv, d), device=q.device, dtype=torch.float32)
+    for t in (M_in, z_in, M_out, z_out):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda):
+            raise ValueError("M and z must be contiguous CUDA fp32 tensors")
+    _check(_lib.infini_attn_forward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M_in),
+                                        _ptr(z_in), _ptr(out), _ptr(M_out), _ptr(z_out), B, H,
+                                        H_kv, L, int(N), d, int(mode), int(layout),
+                                        _stream_handle(stream)))
     return out, M_out, z_out
 
 

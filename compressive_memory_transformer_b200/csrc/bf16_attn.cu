@@ -94,7 +94,9 @@ struct Params {
   long long L;
   int N, S, H, T, U, BH;
   unsigned units;  // BH * S * U, below 2^31
-  FastDiv divU, divS;
+  FastDiv divU, divS, divH, divG;  // G = H / Hkv query heads per key/value head
+  int Hkv;
+  long long o_sb, o_sh, o_sl;  // out strides (elements): batch row, head, row
   int out32;    // out is 32-byte aligned: rows are stored as whole 32-byte sectors
   int tma_out;  // out has a TMA map: whole tiles leave through shared memory
 };
@@ -103,6 +105,7 @@ struct Params {
 struct Tile {
   long long seg0;
   int bh, s, i, nkv, q_row, rows_valid, h, valid;
+  int b, hk, bhk;  // batch row, key/value head, and its index b * Hkv + hk
 };
 
 // Walks the CTA's tiles: units blockIdx.x, blockIdx.x + gridDim.x, ...; unit u of
@@ -135,7 +138,10 @@ struct TileIter {
       if (i >= T_s) continue;
       t.i = i;
       t.nkv = i + 1;
-      t.h = t.bh % p.H;
+      t.b = (int)p.divH.div((uint32_t)t.bh);
+      t.h = t.bh - t.b * p.H;
+      t.hk = (int)p.divG.div((uint32_t)t.h);
+      t.bhk = t.b * p.Hkv + t.hk;
       t.valid = 1;
       t.q_row = (int)(t.seg0 + (long long)i * BM);
       t.rows_valid = min(BM, n_s - i * BM);
@@ -238,8 +244,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_arrive_expect_tx(&bars[B_KFULL + kst], kTile);
         const int row = (int)(t.seg0 + (long long)j * BN);
         uint8_t* dst = sK + kst * kTile;
-        tma_load_3d(dst, &tm_k, &bars[B_KFULL + kst], 0, row, t.bh);
-        tma_load_3d(dst + kSub, &tm_k, &bars[B_KFULL + kst], 64, row, t.bh);
+        tma_load_4d(dst, &tm_k, &bars[B_KFULL + kst], 0, row, t.hk, t.b);
+        tma_load_4d(dst + kSub, &tm_k, &bars[B_KFULL + kst], 64, row, t.hk, t.b);
         ++k_iss[kst];
         kph ^= kst;
         k_wrapped |= (kst == 1u);
@@ -251,13 +257,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_arrive_expect_tx(&bars[B_VFULL + vst], kTile);
         uint8_t* dst = sV + vst * kTile;
         if (item == 0) {
-          const int zc = (t.bh * p.S + t.s) * 2;
+          const int zc = (t.bhk * p.S + t.s) * 2;
           tma_load_3d(dst, &tm_m, &bars[B_VFULL + vst], 0, 0, zc);
           tma_load_3d(dst + kSub, &tm_m, &bars[B_VFULL + vst], 64, 0, zc);
         } else {
           const int row = (int)(t.seg0 + (long long)(item - 1) * BN);
-          tma_load_3d(dst, &tm_v, &bars[B_VFULL + vst], 0, row, t.bh);
-          tma_load_3d(dst + kSub, &tm_v, &bars[B_VFULL + vst], 64, row, t.bh);
+          tma_load_4d(dst, &tm_v, &bars[B_VFULL + vst], 0, row, t.hk, t.b);
+          tma_load_4d(dst + kSub, &tm_v, &bars[B_VFULL + vst], 64, row, t.hk, t.b);
         }
         ++v_iss[vst];
         if (++vst == (uint32_t)kVStages) {
@@ -278,16 +284,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         slots[tc & 1] = t;
         mbar_arrive_expect_tx(&bars[B_QFULL], kTile + D * 4);
-        tma_load_3d(sQ, &tm_q, &bars[B_QFULL], 0, t.q_row, t.bh);
-        tma_load_3d(sQ + kSub, &tm_q, &bars[B_QFULL], 64, t.q_row, t.bh);
-        bulk_load(sZ, zprev + ((size_t)t.bh * p.S + t.s) * D, D * 4, &bars[B_QFULL]);
+        tma_load_4d(sQ, &tm_q, &bars[B_QFULL], 0, t.q_row, t.h, t.b);
+        tma_load_4d(sQ + kSub, &tm_q, &bars[B_QFULL], 64, t.q_row, t.h, t.b);
+        bulk_load(sZ, zprev + ((size_t)t.bhk * p.S + t.s) * D, D * 4, &bars[B_QFULL]);
         ++q_iss;
         {  // the next tile's Q has a whole tile of work to reach L2
           TileIter ahead = it;
           Tile tn;
           if (ahead.next(p, tn)) {
-            tma_prefetch_l2_3d(&tm_q, 0, tn.q_row, tn.bh);
-            tma_prefetch_l2_3d(&tm_q, 64, tn.q_row, tn.bh);
+            tma_prefetch_l2_4d(&tm_q, 0, tn.q_row, tn.h, tn.b);
+            tma_prefetch_l2_4d(&tm_q, 64, tn.q_row, tn.h, tn.b);
           }
         }
         ok = issue_k(t, 0) && (t.nkv < 2 || issue_k(t, 1)) && issue_v(t, 0);
@@ -679,7 +685,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             break;
           }
           if (lane == 0) {
-            tma_store_3d(&tm_o, sOut + half * kSub, 64 * half, t.q_row, t.bh);
+            tma_store_4d(&tm_o, sOut + half * kSub, 64 * half, t.q_row, t.h, t.b);
             tma_store_commit();
           }
           __syncwarp();
@@ -693,7 +699,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         break;
       }
       if (!tma_tile && r < t.rows_valid) {
-        __nv_bfloat16* orow = out + ((size_t)t.bh * p.L + t.q_row + r) * D + col0;
+        __nv_bfloat16* orow = out + t.b * p.o_sb + t.h * p.o_sh + (t.q_row + r) * p.o_sl + col0;
         if (p.out32) {
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) st_global_v8(orow + q8 * 16, w + 8 * q8);
@@ -730,18 +736,26 @@ cudaError_t bf16_attn_set_attributes() {
 cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                              const __nv_bfloat16* v, const float* beta, __nv_bfloat16* out,
                              const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const Bf16Layout* lay) {
+  // query head (b, h) reads key/value head (b, h / (H / H_kv)); out is laid out as q
+  const Bf16Layout l = lay ? *lay : Bf16Layout::bhld(BH / H, H, L);
+  if ((long long)l.B * l.H != BH || l.H_kv < 1 || l.H % l.H_kv != 0) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv, mm, mo;
-  if (!make_bf16_map(&mq, q, (uint64_t)L, BH, 128) || !make_bf16_map(&mk, k, (uint64_t)L, BH, 128) ||
-      !make_bf16_map(&mv, v, (uint64_t)L, BH, 128) ||
-      !make_bf16_map(&mm, ws.Mhl, D, (uint64_t)BH * S * 2, 128))
+  if (!make_bf16_map4(&mq, q, (uint64_t)L, l.H, l.B, l.q_sl, l.q_sh, l.q_sb, 128) ||
+      !make_bf16_map4(&mk, k, (uint64_t)L, l.H_kv, l.B, l.kv_sl, l.kv_sh, l.kv_sb, 128) ||
+      !make_bf16_map4(&mv, v, (uint64_t)L, l.H_kv, l.B, l.kv_sl, l.kv_sh, l.kv_sb, 128) ||
+      !make_bf16_map(&mm, ws.Mhl, D, (uint64_t)l.B * l.H_kv * S * 2, 128))
     return cudaErrorInvalidValue;
   Params p;
   p.L = L;
   p.N = N;
   p.S = S;
-  p.H = H;
+  p.H = l.H;
+  p.Hkv = l.H_kv;
   p.BH = BH;
+  p.o_sb = l.q_sb;
+  p.o_sh = l.q_sh;
+  p.o_sl = l.q_sl;
   p.T = (int)((min((long long)N, L) + BM - 1) / BM);
   p.U = (p.T + 1) / 2;
   const long long units = (long long)BH * S * p.U;
@@ -749,9 +763,11 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   p.units = (unsigned)units;
   p.divU = FastDiv((uint32_t)p.U);
   p.divS = FastDiv((uint32_t)S);
+  p.divH = FastDiv((uint32_t)l.H);
+  p.divG = FastDiv((uint32_t)(l.H / l.H_kv));
   p.out32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
   // a TMA map needs a 16-byte aligned base; otherwise every tile is stored directly
-  p.tma_out = make_bf16_map(&mo, out, (uint64_t)L, BH, 128) ? 1 : 0;
+  p.tma_out = make_bf16_map4(&mo, out, (uint64_t)L, l.H, l.B, l.q_sl, l.q_sh, l.q_sb, 128) ? 1 : 0;
   if (!p.tma_out) mo = mq;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)

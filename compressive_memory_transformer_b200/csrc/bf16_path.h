@@ -19,16 +19,36 @@ struct Bf16Workspace {
   __nv_bfloat16* Mhl;
 };
 
+// Where q/k/v/out sit: element (b, h, l, f) of q and out at b*q_sb + h*q_sh + l*q_sl + f,
+// of k and v at b*kv_sb + h*kv_sh + l*kv_sl + f (strides in elements). H query heads
+// share H_kv key/value heads (query head h reads key/value head h / (H / H_kv)); the
+// memory state is per key/value head. bhld() is the contiguous [B, H, L, d] case.
+struct Bf16Layout {
+  int B, H, H_kv;
+  long long q_sb, q_sh, q_sl, kv_sb, kv_sh, kv_sl;
+  static Bf16Layout bhld(int B, int H, long long L) {
+    const long long d = 128;
+    return Bf16Layout{B, H, H, (long long)H * L * d, L * d, d, (long long)H * L * d, L * d, d};
+  }
+  static Bf16Layout blhd(int B, int H, int H_kv, long long L) {
+    const long long d = 128;
+    return Bf16Layout{B, H, H_kv, L * H * d, d, (long long)H * d, L * H_kv * d, d,
+                      (long long)H_kv * d};
+  }
+};
+
 void bf16_state_plan(int BH, int S, int N, int* CH, int* CL);
 size_t bf16_workspace_bytes(int BH, int S, int CH);
 Bf16Workspace bf16_workspace_carve(void* base, int BH, int S, int CH);
 
 // The state path. Segments s < first (0 or 1) of the workspace's M_{s-1} hi/lo
 // and z_{s-1} are taken as already written (by bf16_prep_first) and not rewritten.
+// BH here counts key/value heads (B * H_kv); k and v are read through the layout.
 cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, const float* M_in,
                               const float* z_in, float* M_out, float* z_out,
                               const Bf16Workspace& ws, int BH, long long L, int N, int S, int CH,
-                              int CL, int mode, int first, cudaStream_t stream);
+                              int CL, int mode, int first, cudaStream_t stream,
+                              const Bf16Layout* lay = nullptr);
 
 // Writes the workspace's first-segment M_{-1} hi/lo and z_{-1} from M_in / z_in.
 cudaError_t bf16_prep_first(const float* M_in, const float* z_in, const Bf16Workspace& ws,
@@ -36,10 +56,11 @@ cudaError_t bf16_prep_first(const float* M_in, const float* z_in, const Bf16Work
 
 // The fused local-attention + retrieval + gate kernel. Reads q, k, v, beta and
 // the workspace's zprev / Mhl; writes out.
+// BH counts query heads (B * H); the workspace holds the key/value heads' states.
 cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                              const __nv_bfloat16* v, const float* beta, __nv_bfloat16* out,
                              const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
-                             cudaStream_t stream);
+                             cudaStream_t stream, const Bf16Layout* lay = nullptr);
 
 // Token-level decode (bf16_decode.cu): partial attention over the KV cache (rows
 // below pos) and the new rows (k, v, also written into the caches), split like flash

@@ -52,7 +52,8 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& raw, float (&f)[8]) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) zpart_kernel(const __nv_bfloat16* __restrict__ k,
                                                     float* __restrict__ zpart, long long L, int N,
-                                                    int S, int CH, int CL) {
+                                                    int S, int CH, int CL, int Hkv, long long sb,
+                                                    long long sh, long long sl) {
   __shared__ float red[16][D + 4];
   const long long idx = blockIdx.x;
   const int c = (int)(idx % CH);
@@ -65,7 +66,8 @@ __global__ void __launch_bounds__(256) zpart_kernel(const __nv_bfloat16* __restr
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  const __nv_bfloat16* base = k + ((size_t)bh * L + t0) * D + cg * 8;
+  // key/value head bh = (batch row, head); rows of K are sl elements apart
+  const __nv_bfloat16* base = k + (bh / Hkv) * sb + (bh % Hkv) * sh + t0 * sl + cg * 8;
   // four rows per thread in flight: one outstanding load per thread would cap the
   // stream at ~4 TB/s
   int t = beg + rg;
@@ -73,7 +75,7 @@ __global__ void __launch_bounds__(256) zpart_kernel(const __nv_bfloat16* __restr
     uint4 raw[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-      raw[u] = __ldg(reinterpret_cast<const uint4*>(base + (size_t)(t + 16 * u) * D));
+      raw[u] = __ldg(reinterpret_cast<const uint4*>(base + (t + 16 * u) * sl));
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       float f[8];
@@ -83,7 +85,7 @@ __global__ void __launch_bounds__(256) zpart_kernel(const __nv_bfloat16* __restr
     }
   }
   for (; t < end; t += 16) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(base + (size_t)t * D));
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(base + t * sl));
     float f[8];
     bf16x8_to_f32(raw, f);
 #pragma unroll
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const float* __restrict__ zprev, float* __restrict__ dpart,
              float* __restrict__ zpart, long long L, int N, int S, int CH, int CL, int mode,
-             int zsum) {
+             int zsum, int Hkv) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -234,10 +236,11 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         uint8_t* st = smem + stg * kStageBytes;
         mbar_arrive_expect_tx(&bar_full[stg], 2 * kMat);
         const int row = row0 + sl * kSlab;
-        tma_load_3d(st + OFF_KH, &tm_k, &bar_full[stg], 0, row, (int)bh);
-        tma_load_3d(st + OFF_KH + kBox, &tm_k, &bar_full[stg], 64, row, (int)bh);
-        tma_load_3d(st + OFF_V, &tm_v, &bar_full[stg], 0, row, (int)bh);
-        tma_load_3d(st + OFF_V + kBox, &tm_v, &bar_full[stg], 64, row, (int)bh);
+        const int hh = (int)(bh % Hkv), bb = (int)(bh / Hkv);
+        tma_load_4d(st + OFF_KH, &tm_k, &bar_full[stg], 0, row, hh, bb);
+        tma_load_4d(st + OFF_KH + kBox, &tm_k, &bar_full[stg], 64, row, hh, bb);
+        tma_load_4d(st + OFF_V, &tm_v, &bar_full[stg], 0, row, hh, bb);
+        tma_load_4d(st + OFF_V + kBox, &tm_v, &bar_full[stg], 64, row, hh, bb);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -702,22 +705,29 @@ Bf16Workspace bf16_workspace_carve(void* base, int BH, int S, int CH) {
 cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, const float* M_in,
                               const float* z_in, float* M_out, float* z_out,
                               const Bf16Workspace& ws, int BH, long long L, int N, int S, int CH,
-                              int CL, int mode, int first, cudaStream_t stream) {
+                              int CL, int mode, int first, cudaStream_t stream,
+                              const Bf16Layout* lay) {
   const unsigned nunits = (unsigned)((long long)BH * S * CH);
+  // key/value head i = (batch row i / Hkv, head i % Hkv); without a layout, BH
+  // contiguous [L, 128] planes
+  const Bf16Layout l = lay ? *lay : Bf16Layout::bhld(BH, 1, L);
+  const int Hkv = l.H_kv;
   CUtensorMap mk, mv;
-  if (!make_bf16_map(&mk, k, (uint64_t)L, BH, kSlab) || !make_bf16_map(&mv, v, (uint64_t)L, BH, kSlab))
+  if (!make_bf16_map4(&mk, k, (uint64_t)L, Hkv, l.B, l.kv_sl, l.kv_sh, l.kv_sb, kSlab) ||
+      !make_bf16_map4(&mv, v, (uint64_t)L, Hkv, l.B, l.kv_sl, l.kv_sh, l.kv_sb, kSlab))
     return cudaErrorInvalidValue;
   if (mode == 1 && !(first == 1 && S == 1)) {
     // Linear+Delta needs z_{s-1} (hence every segment's sum of sigma(K)) first
-    zpart_kernel<<<nunits, 256, 0, stream>>>(k, ws.zpart, L, N, S, CH, CL);
+    zpart_kernel<<<nunits, 256, 0, stream>>>(k, ws.zpart, L, N, S, CH, CL, Hkv, l.kv_sb, l.kv_sh,
+                                             l.kv_sl);
     zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH, first);
     state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(
-        mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 0);
+        mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 0, Hkv);
   } else {
     // The state GEMM also produces the sums of sigma(K): always in Linear mode, and
     // in Linear+Delta mode for a lone segment whose z_{-1} is already in place
     state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(
-        mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 1);
+        mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 1, Hkv);
     zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH, first);
   }
   CUtensorMap mg;

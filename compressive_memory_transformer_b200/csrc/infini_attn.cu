@@ -120,7 +120,8 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 int check_common(const void* q, const void* k, const void* v, const float* beta,
                  const float* M_in, const float* z_in, const void* out, const float* M_out,
                  const float* z_out, int B, int H, long long L, int N, int d, int mode,
-                 size_t esize) {
+                 size_t esize, int H_kv = 0) {
+  if (H_kv == 0) H_kv = H;
   if (!beta) return INFINI_ERR_NULL;
   if (L > 0 && (!q || !k || !v || !out)) return INFINI_ERR_NULL;
   if ((M_in == nullptr) != (z_in == nullptr)) return INFINI_ERR_NULL;
@@ -132,9 +133,11 @@ int check_common(const void* q, const void* k, const void* v, const float* beta,
   if (overflows(BH, L) || overflows(BH * L, d) || overflows(BH * L * d, (long long)esize))
     return INFINI_ERR_SHAPE;
   if (L >= (1LL << 31)) return INFINI_ERR_SHAPE;
-  const size_t nio = (size_t)(BH * L * d) * esize;
-  const size_t nM = (size_t)BH * d * d * sizeof(float), nz = (size_t)BH * d * sizeof(float);
-  if (overlap(out, nio, q, nio) || overlap(out, nio, k, nio) || overlap(out, nio, v, nio) ||
+  if (H_kv < 1 || H % H_kv != 0) return INFINI_ERR_SHAPE;
+  const long long BHkv = (long long)B * H_kv;
+  const size_t nio = (size_t)(BH * L * d) * esize, nkv = (size_t)(BHkv * L * d) * esize;
+  const size_t nM = (size_t)BHkv * d * d * sizeof(float), nz = (size_t)BHkv * d * sizeof(float);
+  if (overlap(out, nio, q, nio) || overlap(out, nio, k, nkv) || overlap(out, nio, v, nkv) ||
       overlap(out, nio, M_in, nM) || overlap(out, nio, z_in, nz) ||
       overlap(out, nio, M_out, nM) || overlap(out, nio, z_out, nz))
     return INFINI_ERR_ALIAS;
@@ -186,19 +189,29 @@ void record(const infini_attn_opts_t* opts, int i, cudaStream_t stream) {
 int forward_impl(const void* q, const void* k, const void* v, const float* beta,
                  const float* M_in, const float* z_in, void* out, float* M_out, float* z_out,
                  int B, int H, long long L, int N, int d, int mode, int dtype,
-                 const infini_attn_opts_t* opts, cudaStream_t stream) {
+                 const infini_attn_opts_t* opts, cudaStream_t stream, int H_kv = 0,
+                 int layout = INFINI_LAYOUT_BHLD) {
   if (dtype != INFINI_DTYPE_BF16 && dtype != INFINI_DTYPE_F32) return INFINI_ERR_UNSUPPORTED;
+  if (H_kv == 0) H_kv = H;
   const size_t esize = dtype == INFINI_DTYPE_BF16 ? 2 : 4;
-  int st = check_common(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, L, N, d, mode, esize);
+  int st = check_common(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, L, N, d, mode, esize,
+                        H_kv);
   if (st != INFINI_OK) return st;
+  if (layout != INFINI_LAYOUT_BHLD && layout != INFINI_LAYOUT_BLHD) return INFINI_ERR_UNSUPPORTED;
+  if (dtype == INFINI_DTYPE_F32 && (layout != INFINI_LAYOUT_BHLD || H_kv != H))
+    return INFINI_ERR_UNSUPPORTED;
   if (dtype == INFINI_DTYPE_BF16 && d != 128) return INFINI_ERR_UNSUPPORTED;
   if (dtype == INFINI_DTYPE_F32 && d > 128) return INFINI_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return INFINI_ERR_ALIGN;
   if ((M_in && !aligned16(M_in)) || (M_out && !aligned16(M_out))) return INFINI_ERR_ALIGN;
-  const int BH = B * H;
+  const int BH = B * H, BHkv = B * H_kv;
+  const Bf16Layout lay = layout == INFINI_LAYOUT_BLHD ? Bf16Layout::blhd(B, H, H_kv, L)
+                                                      : Bf16Layout{B, H, H_kv, (long long)H * L * d,
+                                                                   L * d, d, (long long)H_kv * L * d,
+                                                                   L * d, d};
   if (L == 0) {
     record(opts, 0, stream);
-    st = pass_state(M_in, z_in, M_out, z_out, BH, d, stream);
+    st = pass_state(M_in, z_in, M_out, z_out, BHkv, d, stream);
     record(opts, 1, stream);
     record(opts, 2, stream);
     return st;
@@ -220,12 +233,12 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
     return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
   }
   int CH = 1, CL = N;
-  bf16_state_plan(BH, S, N, &CH, &CL);
-  if ((long long)BH * S * CH >= (1LL << 31)) return INFINI_ERR_SHAPE;
+  bf16_state_plan(BHkv, S, N, &CH, &CL);
+  if ((long long)BHkv * S * CH >= (1LL << 31)) return INFINI_ERR_SHAPE;
   Scratch sc;
-  st = get_scratch(sc, bf16_workspace_bytes(BH, S, CH), opts, stream);
+  st = get_scratch(sc, bf16_workspace_bytes(BHkv, S, CH), opts, stream);
   if (st != INFINI_OK) return st;
-  const Bf16Workspace ws = bf16_workspace_carve(sc.ptr, BH, S, CH);
+  const Bf16Workspace ws = bf16_workspace_carve(sc.ptr, BHkv, S, CH);
   const auto* qb = static_cast<const __nv_bfloat16*>(q);
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
   const auto* vb = static_cast<const __nv_bfloat16*>(v);
@@ -236,15 +249,15 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
     // back before the call returns.
     SideStream& sd = g_side[dev];
     std::lock_guard<std::mutex> lk(sd.mu);
-    cudaError_t e = bf16_prep_first(M_in, z_in, ws, BH, S, stream);
+    cudaError_t e = bf16_prep_first(M_in, z_in, ws, BHkv, S, stream);
     if (e == cudaSuccess) e = cudaEventRecord(sd.fork, stream);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(sd.stream, sd.fork, 0);
     if (e != cudaSuccess) return INFINI_ERR_CUDA;
-    const cudaError_t es = bf16_state_launch(kb, vb, M_in, z_in, M_out, z_out, ws, BH, L, N, S,
-                                             CH, CL, mode, 1, sd.stream);
+    const cudaError_t es = bf16_state_launch(kb, vb, M_in, z_in, M_out, z_out, ws, BHkv, L, N, S,
+                                             CH, CL, mode, 1, sd.stream, &lay);
     record(opts, 1, stream);
     const cudaError_t ea = bf16_attn_launch(qb, kb, vb, beta, static_cast<__nv_bfloat16*>(out),
-                                            ws, BH, H, L, N, S, stream);
+                                            ws, BH, H, L, N, S, stream, &lay);
     // joined even after a launch error, so that the side stream never runs ahead of
     // the caller's stream
     cudaError_t ej = cudaEventRecord(sd.join, sd.stream);
@@ -253,12 +266,12 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
     return es == cudaSuccess && ea == cudaSuccess && ej == cudaSuccess ? INFINI_OK
                                                                         : INFINI_ERR_CUDA;
   }
-  cudaError_t e = bf16_state_launch(kb, vb, M_in, z_in, M_out, z_out, ws, BH, L, N, S, CH, CL,
-                                    mode, 0, stream);
+  cudaError_t e = bf16_state_launch(kb, vb, M_in, z_in, M_out, z_out, ws, BHkv, L, N, S, CH, CL,
+                                    mode, 0, stream, &lay);
   if (e != cudaSuccess) return INFINI_ERR_CUDA;
   record(opts, 1, stream);
   e = bf16_attn_launch(qb, kb, vb, beta, static_cast<__nv_bfloat16*>(out), ws, BH, H, L, N, S,
-                       stream);
+                       stream, &lay);
   record(opts, 2, stream);
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
@@ -394,6 +407,15 @@ int infini_attn_step_f32(const float* q, const float* k, const float* v, const f
                          float* z_out, int B, int H, int N, int d, int mode, void* stream) {
   return forward_impl(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, N, N < 1 ? 1 : N, d,
                       mode, INFINI_DTYPE_F32, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int infini_attn_forward_gqa(const void* q, const void* k, const void* v, const float* beta,
+                            const float* M_in, const float* z_in, void* out, float* M_out,
+                            float* z_out, int B, int H, int H_kv, long long L, int N, int d,
+                            int mode, int layout, void* stream) {
+  if (H_kv < 1) return INFINI_ERR_SHAPE;
+  return forward_impl(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, L, N, d, mode,
+                      INFINI_DTYPE_BF16, nullptr, static_cast<cudaStream_t>(stream), H_kv, layout);
 }
 
 int infini_attn_state_sum(const float* dM, const float* dz, int count, const float* M_in,

@@ -43,4 +43,24 @@ inline bool make_bf16_map(CUtensorMap* m, const void* base, uint64_t rows, uint6
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D bf16 map over d = 128 features x L rows x H heads x B batch rows, element
+// (b, h, l, f) at base + b * sb + h * sh + l * sl + f (strides in elements, each a
+// multiple of 8, i.e. 16 bytes): [B, H, L, 128] contiguous and [B, L, H, 128] are
+// both such maps. Box = 64 features x box_rows rows x one head x one batch row,
+// 128-byte swizzle, as make_bf16_map. Rows past L read as zeros; stores there are
+// dropped.
+inline bool make_bf16_map4(CUtensorMap* m, const void* base, uint64_t L, uint64_t H, uint64_t B,
+                           uint64_t sl, uint64_t sh, uint64_t sb, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {128, L, H, B};
+  const cuuint64_t strides[3] = {sl * 2, sh * 2, sb * 2};
+  const cuuint32_t box[4] = {64, box_rows, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace infini

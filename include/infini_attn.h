@@ -112,6 +112,28 @@ int infini_attn_step_static(const void* q, const void* k, const void* v, const f
                             const float* M_in, const float* z_in, void* out, float* M_out,
                             float* z_out, int B, int H, int N, int d, int mode, void* stream);
 
+/* Memory layouts of q, k, v and out for infini_attn_forward_gqa. */
+typedef enum {
+  INFINI_LAYOUT_BHLD = 0, /* [B, H, L, d] contiguous (every other entry point) */
+  INFINI_LAYOUT_BLHD = 1  /* [B, L, H, d] contiguous: the rows of a [B, L, H * d] projection */
+} infini_layout_t;
+
+/*
+ * infini_attn_forward with grouped key/value heads and a choice of layout (bf16,
+ * d == 128). q and out have H heads, k and v have H_kv heads (H % H_kv == 0); query
+ * head h reads key/value head h / (H / H_kv) for its local attention and retrieves
+ * from that head's memory, so M and z are [B, H_kv, d, d] and [B, H_kv, d] (the
+ * memory is built from K and V only, section 3.4). With H_kv == H and
+ * INFINI_LAYOUT_BHLD this is infini_attn_forward. The layout applies to all four of
+ * q, k, v, out: [B, H or H_kv, L, d] or [B, L, H or H_kv, d]. beta has H entries.
+ * Errors: INFINI_ERR_SHAPE for H_kv < 1 or H % H_kv != 0, INFINI_ERR_UNSUPPORTED for
+ * an unknown layout or d != 128; otherwise as infini_attn_forward.
+ */
+int infini_attn_forward_gqa(const void* q, const void* k, const void* v, const float* beta,
+                            const float* M_in, const float* z_in, void* out, float* M_out,
+                            float* z_out, int B, int H, int H_kv, long long L, int N, int d,
+                            int mode, int layout, void* stream);
+
 /*
  * The memory update alone (section 3.4, Linear or Linear+Delta, applied segment by
  * segment): (M_out, z_out) after L tokens of bf16 k, v [B, H, L, d] cut into

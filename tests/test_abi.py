@@ -163,3 +163,17 @@ def test_state_sum_rejects_bad_arguments(lib):
     assert call(count=-1) == -2
     assert call(B=0) == -2
     assert call(M_out=FAKE + 4096) == -8  # M_out inside the blocks
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(H=4, H_kv=3), -2), (dict(H=4, H_kv=0), -2), (dict(layout=2), -3), (dict(d=64), -3),
+    (dict(q=None), -1),
+])
+def test_forward_gqa_rejects_bad_arguments(lib, kw, code):
+    a = dict(q=FAKE, k=FAKE + (1 << 20), v=FAKE + (2 << 20), beta=FAKE + (3 << 20), M_in=None,
+             z_in=None, out=FAKE * 8, M_out=None, z_out=None, B=1, H=4, H_kv=2, L=128, N=128,
+             d=128, mode=0, layout=0)
+    a.update(kw)
+    assert lib.raw_call("infini_attn_forward_gqa", a["q"], a["k"], a["v"], a["beta"], a["M_in"],
+                        a["z_in"], a["out"], a["M_out"], a["z_out"], a["B"], a["H"], a["H_kv"],
+                        a["L"], a["N"], a["d"], a["mode"], a["layout"], None) == code
