@@ -11,6 +11,7 @@ Entry points (same names as the C ABI in include/infini_attn.h):
     infini_attn_forward_gqa(q, k, v, beta, N, mode, layout, ...)
     infini_attn_state_update(k, v, N, mode, M_in=None, z_in=None, ...)
     infini_attn_state_sum(dM, dz, M_in=None, z_in=None, ...)
+    infini_attn_backward(q, k, v, beta, N, mode, dout, M_in=None, z_in=None, ...)
 q, k, v: [B, H, L, d] CUDA tensors, bf16 (d = 128) or fp32 (d <= 128);
 beta: [H] fp32; M: [B, H, d, d] fp32; z: [B, H, d] fp32.
 """
@@ -59,6 +60,7 @@ _SIGS = {
     "infini_attn_state_update": [_vp] * 6 + [_i, _i, _ll, _i, _i, _i, _vp],
     "infini_attn_forward_gqa": [_vp] * 9 + [_i, _i, _i, _ll, _i, _i, _i, _i, _vp],
     "infini_attn_state_sum": [_vp, _vp, _i] + [_vp] * 4 + [_i, _i, _i, _vp],
+    "infini_attn_backward": [_vp] * 15 + [_i, _i, _ll, _i, _i, _i, _vp],
     "infini_attn_workspace_size": [_i, _i, _ll, _i, _i, _i, _i],
     "infini_attn_device_status": [],
     "infini_attn_selftest_timeout": [_ll, _vp],
@@ -254,6 +256,31 @@ def infini_attn_state_sum(dM, dz, M_in=None, z_in=None, M_out=None, z_out=None, 
                                       count, _ptr(M_in), _ptr(z_in), _ptr(M_out), _ptr(z_out), B,
                                       H, d, _stream_handle(stream)))
     return M_out, z_out
+
+
+def infini_attn_backward(q, k, v, beta, N, mode, dout, M_in=None, z_in=None, dM_out=None,
+                         dz_out=None, state_grad=True, stream=None):
+    """Gradient of infini_attn_forward (bf16, [B, H, L, 128], N a multiple of 128, L a
+    multiple of N) for the loss sum(dout * out) + sum(dM_out * M_out) + sum(dz_out *
+    z_out). Returns (dq, dk, dv, dbeta, dM_in, dz_in); dM_in, dz_in are None when
+    state_grad is False."""
+    B, H, L, d, _, _, _ = _prepare(q, k, v, beta, M_in, z_in, None, None, None, False)
+    if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_cuda or not dout.is_contiguous():
+        raise ValueError("dout must be a contiguous CUDA tensor shaped and typed like q")
+    for t in (dM_out, dz_out):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or not t.is_cuda):
+            raise ValueError("dM_out and dz_out must be contiguous CUDA fp32 tensors")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dbeta = torch.empty((H,), device=q.device, dtype=torch.float32)
+    dM_in = dz_in = None
+    if state_grad:
+        dM_in = torch.empty((B, H, d, d), device=q.device, dtype=torch.float32)
+        dz_in = torch.empty((B, H, d), device=q.device, dtype=torch.float32)
+    _check(_lib.infini_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M_in),
+                                     _ptr(z_in), _ptr(dout), _ptr(dM_out), _ptr(dz_out), _ptr(dq),
+                                     _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dM_in), _ptr(dz_in), B,
+                                     H, L, int(N), d, int(mode), _stream_handle(stream)))
+    return dq, dk, dv, dbeta, dM_in, dz_in
 
 
 def infini_attn_decode(q, k, v, beta, k_cache, v_cache, M, z, pos, mode=LINEAR, out=None,

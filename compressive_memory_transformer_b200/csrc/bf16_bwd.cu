@@ -1,0 +1,1274 @@
+// bf16_bwd.cu — gradient of the bf16 forward (d = 128, [B, H, L, d], N a multiple of
+// 128 and L a multiple of N).
+//
+// The layer ("Leave No Context Behind", arXiv 2404.07143, as quoted on
+// llm-papers-study.pages.dev, sections 3.1, 3.3-3.5) is, per head and segment s,
+//   out = g A_mem + (1 - g) A_dot,   A_dot = softmax(Q K^T / sqrt(d) + mask) V,
+//   A_mem = sigma(Q) M_{s-1} / (sigma(Q) z_{s-1}),
+//   M_s = M_{s-1} + sigma(K)^T V                 (Linear)
+//   M_s = M_{s-1} + sigma(K)^T (V - R),  R = sigma(K) M_{s-1} / (sigma(K) z_{s-1})  (Delta)
+//   z_s = z_{s-1} + sum_t sigma(K_t).
+// Its gradient is the chain rule through those steps in reverse segment order. With
+// dM_s, dz_s the gradients of the state after segment s:
+//   retrieval: dnum = g dout / den, dden = -rowsum(g dout * A_mem) / den,
+//              dsigma(Q) = dnum M^T + dden z^T, and (M_{s-1}, z_{s-1}) receive
+//              GM_s = sigma(Q)^T dnum and Gz_s = sigma(Q)^T dden;
+//   Linear:    dM_{s-1} = dM_s + GM_s;  dsigma(K) = V dM_s^T + dz_s;  dV += sigma(K) dM_s;
+//   Delta:     dU = sigma(K) dM_s (U = V - R), dV += dU, and through R
+//              dM_{s-1} = dM_s - G_s dM_s + GM_s with G_s = sigma(K)^T diag(1/den_K) sigma(K)
+//              (the same symmetric matrix the forward's state kernel builds),
+//              dsigma(K) = U dM_s^T - (dU / den_K) M^T + ddenR z^T + dz_s,
+//              ddenR = rowsum(dU * R) / den_K, dz_{s-1} = dz_s + sigma(K)^T ddenR + Gz_s;
+//   attention: the usual softmax backward of the local causal attention, scaled by
+//              (1 - g); dbeta = g (1 - g) sum dout * (A_mem - A_dot).
+// Rows whose denominator is exactly 0 retrieve the constant 0 and pass no gradient.
+//
+// Kernels, in launch order (after the forward's state path has rebuilt M_{s-1} as
+// bf16 hi/lo, z_{s-1} and, for Delta, every segment's G_s):
+//   retr   (head, segment): retrieval backward over the segment's query tiles ->
+//          dq_mem (fp32), GM_s, Gz_s, the segment's sum of dout * A_mem.
+//   chain  (head, 32-column block): dM_s for s = S-1 .. 0 (bf16 hi/lo stack), dM_in.
+//   kside  (head, segment, key tile): the memory update's backward per key row ->
+//          dk_mem (dsigma(K) without dz_s), dv_mem, per-tile sigma(K)^T ddenR.
+//   dz     (head): dz_s for every segment, dz_in.
+//   dq     (head, segment, query tile): two sweeps over the key tiles; the first
+//          gives each row's log-sum-exp and D' = dout . A_dot, the second
+//          dQ = sum_j dS_j K_j; adds dq_mem, writes dq, the row statistics and the
+//          tile's sum of D' (for dbeta).
+//   dkdv   (head, segment, key tile): over the query tiles at or after it,
+//          dV = sum_i (1-g) P_i^T dout_i and dK = sum_i dS_i^T Q_i from S^T = K Q^T
+//          and dP'^T = V dout^T; adds dv_mem, (dk_mem + dz_s) * sigma'(K); writes dk, dv.
+//   dbeta  : per head, summed over batch rows and segments in a fixed order.
+// Every product is a 128 x 128 x 128 bf16 tcgen05 MMA (fp32 accumulation in tensor
+// memory) on 128B-swizzled shared-memory tiles, in the operand forms the forward
+// uses: A, B both K-major (Q K^T), A in tensor memory with B MN-major (P V), and
+// A, B both MN-major (sigma(K)^T V); the Delta chain uses the forward chain's tf32
+// form. Each CTA has 128 threads, thread r owning tile row r (tensor-memory lane r).
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda.h>
+#include <cstdint>
+#include <cstring>
+
+#include "bf16_path.h"
+#include "sm100.cuh"
+#include "tma_map.h"
+
+namespace infini {
+namespace {
+
+constexpr int D = 128;
+constexpr int kTile = 32768;  // 128 x 128 bf16
+constexpr int kSub = 16384;   // one 128 x 64 box (128-byte rows)
+constexpr int kThreads = 128;
+
+// ---------------------------------------------------------------------------
+// tiles, descriptors, products
+// ---------------------------------------------------------------------------
+// Byte offset of 16-byte unit u (0..15: features 8u .. 8u+7) of row r of a tile
+// stored as two 64-column boxes with the 128-byte swizzle (the TMA layout).
+__device__ __forceinline__ uint32_t toff(int r, int u) {
+  return (uint32_t)(u >> 3) * kSub + sw128((uint32_t)r, (uint32_t)(u & 7));
+}
+__device__ __forceinline__ uint4 ld_unit(const uint8_t* t, int r, int u) {
+  return *reinterpret_cast<const uint4*>(t + toff(r, u));
+}
+__device__ __forceinline__ void st_unit(uint8_t* t, int r, int u, const float (&f)[8]) {
+  *reinterpret_cast<uint4*>(t + toff(r, u)) =
+      make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                 pack_bf16x2(f[6], f[7]));
+}
+__device__ __forceinline__ void unpack8(const uint4& raw, float (&f)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 t = __bfloat1622float2(h[e]);
+    f[2 * e] = t.x;
+    f[2 * e + 1] = t.y;
+  }
+}
+// element (r, c) of a tile
+__device__ __forceinline__ float ld_elem(const uint8_t* t, int r, int c) {
+  const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(t + toff(r, c >> 3)) + (c & 7);
+  return __bfloat162float(*p);
+}
+
+// sigma = ELU + 1 and its derivative (1 for x > 0, e^x otherwise), full-precision exp
+__device__ __forceinline__ float sig(float x) { return x > 0.f ? x + 1.f : expf(x); }
+__device__ __forceinline__ float dsig(float x) { return x > 0.f ? 1.f : expf(x); }
+
+__device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk) {
+  return sdesc(base + (uint32_t)(kk >> 2) * kSub + (uint32_t)(kk & 3) * 32, 16, 1024);
+}
+__device__ __forceinline__ uint64_t mdesc(uint32_t base, int kk) {
+  return sdesc(base + (uint32_t)kk * 2048, kSub, 1024);
+}
+constexpr uint32_t kIdKK = idesc_f32acc(1, 0, 0, 128, 128);
+constexpr uint32_t kIdKM = idesc_f32acc(1, 0, 1, 128, 128);
+constexpr uint32_t kIdMM = idesc_f32acc(1, 1, 1, 128, 128);
+
+// D (+)= A B^T: A[m][k] and B[n][k] are tiles (rows m and n, 128 k each)
+__device__ __forceinline__ void gemm_kk(uint32_t d, const uint8_t* a, const uint8_t* b, bool acc) {
+  const uint32_t sa = smem_u32(a), sb = smem_u32(b);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_bf16_ss(d, kdesc(sa, kk), kdesc(sb, kk), kIdKK, (acc || kk > 0) ? 1u : 0u);
+}
+// D (+)= A X: A[m][k] and X[k][n] are tiles
+__device__ __forceinline__ void gemm_km(uint32_t d, const uint8_t* a, const uint8_t* x, bool acc) {
+  const uint32_t sa = smem_u32(a), sx = smem_u32(x);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_bf16_ss(d, kdesc(sa, kk), mdesc(sx, kk), kIdKM, (acc || kk > 0) ? 1u : 0u);
+}
+// D (+)= X^T Y: X[k][m] and Y[k][n] are tiles (the contraction runs over tile rows)
+__device__ __forceinline__ void gemm_mm(uint32_t d, const uint8_t* x, const uint8_t* y, bool acc) {
+  const uint32_t sx = smem_u32(x), sy = smem_u32(y);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_bf16_ss(d, mdesc(sx, kk), mdesc(sy, kk), kIdMM, (acc || kk > 0) ? 1u : 0u);
+}
+// D (+)= A X: A[m][k] in tensor memory (bf16 pairs, 64 columns from ta), X[k][n] a tile
+__device__ __forceinline__ void gemm_tm(uint32_t d, uint32_t ta, const uint8_t* x, bool acc) {
+  const uint32_t sx = smem_u32(x);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_bf16_ts(d, ta + 8 * kk, mdesc(sx, kk), kIdKM, (acc || kk > 0) ? 1u : 0u);
+}
+
+// Both boxes of a 128-row tile of a [B, H, L, 128] tensor.
+__device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* m, uint64_t* bar, int row,
+                                          int h, int b) {
+  tma_load_4d(dst, m, bar, 0, row, h, b);
+  tma_load_4d(dst + kSub, m, bar, 64, row, h, b);
+}
+// Both boxes of a [128][128] plane of a 3-D map.
+__device__ __forceinline__ void load_plane(uint8_t* dst, const CUtensorMap* m, uint64_t* bar,
+                                           int plane) {
+  tma_load_3d(dst, m, bar, 0, 0, plane);
+  tma_load_3d(dst + kSub, m, bar, 64, 0, plane);
+}
+
+// A wait by all 128 threads whose outcome is the same in every thread (and a CTA
+// barrier): a wait that gave up anywhere makes every thread leave its loop.
+__device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity) {
+  const bool w = mbar_wait(bar, parity);
+  return __syncthreads_and(w ? 1 : 0) != 0;
+}
+
+// Bounded wait used only while draining after an error.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) break;  // 200 ms
+  }
+}
+
+// Issues the product(s) from one elected lane of warp 0, then commits to bar.
+#define ISSUE_MMA(bar, ...)                 \
+  do {                                      \
+    if (warp == 0) {                        \
+      tc_fence_after();                     \
+      if (elect_one()) {                    \
+        __VA_ARGS__;                        \
+        mma_commit(bar);                    \
+      }                                     \
+      __syncwarp();                         \
+    }                                       \
+  } while (0)
+
+// Threads' shared- and tensor-memory writes -> visible to the tensor cores.
+__device__ __forceinline__ void publish_writes() {
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+}
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  return (red[0] + red[1]) + (red[2] + red[3]);
+}
+
+struct BwdParams {
+  long long L;       // tokens per (batch row, head)
+  int N, S, T, H;    // T = N / 128 tiles per segment
+  unsigned tiles;    // BH * S * T
+  FastDiv divT, divS;
+  float sl;          // log2(e) / sqrt(d)
+  float rsd;         // 1 / sqrt(d)
+};
+
+// grid index -> (bh, s, tile)
+__device__ __forceinline__ void decode3(const BwdParams& p, unsigned u, int& bh, int& s, int& t) {
+  const unsigned seg = p.divT.div(u);
+  t = (int)(u - seg * (unsigned)p.T);
+  const unsigned b = p.divS.div(seg);
+  s = (int)(seg - b * (unsigned)p.S);
+  bh = (int)b;
+}
+
+// ---------------------------------------------------------------------------
+// retr: grid = BH * S, one CTA per (head, segment), looping over its query tiles.
+// Tensor memory: num = sigma(Q) M | dsigma(Q) = dnum M^T | GM (accumulated).
+// ---------------------------------------------------------------------------
+constexpr int kRetrSmem = 5 * kTile + 1024 + 64 + 256 + 1024;
+
+__global__ void __launch_bounds__(kThreads, 1)
+retr_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                const __grid_constant__ CUtensorMap tm_m, const float* __restrict__ beta,
+                const float* __restrict__ zprev, float* __restrict__ dq_mem,
+                float* __restrict__ GM, float* __restrict__ Gz, float* __restrict__ mem_part,
+                const BwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sM = smem;
+  uint8_t* sQ = smem + kTile;
+  uint8_t* sDO = smem + 2 * kTile;
+  uint8_t* sSQ = smem + 3 * kTile;  // sigma(Q), bf16
+  uint8_t* sDN = smem + 4 * kTile;  // dnum, bf16
+  float* sZ = reinterpret_cast<float*>(smem + 5 * kTile);
+  float* sDD = sZ + D;              // dden per row
+  float* red = sDD + D;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 16);  // 0 M/z, 1 Q/dout, 2 MMA, 3 drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+
+  const int seg = blockIdx.x;
+  const int bh = (int)p.divS.div((unsigned)seg), s = seg - bh * p.S;
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int tid = threadIdx.x, warp = tid >> 5, r = tid;
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot, tN = tmem, tD = tmem + 128, tG = tmem + 256;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  int q_iss = 0, q_cons = 0;
+  bool m_pending = true;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], kTile + D * 4);
+    load_plane(sM, &tm_m, &bars[0], (bh * p.S + s) * 2);
+    bulk_load(sZ, zprev + ((size_t)bh * p.S + s) * D, D * 4, &bars[0]);
+  }
+  const float g = 1.f / (1.f + expf(-beta[h]));
+  float gz = 0.f, memt = 0.f;
+  uint32_t mph = 0;
+  bool ok = cta_wait(&bars[0], 0);
+  if (ok) m_pending = false;
+  for (int i = 0; ok && i < p.T; ++i) {
+    const int row = s * p.N + i * 128;
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&bars[1], 2 * kTile);
+      load_rows(sQ, &tm_q, &bars[1], row, h, b);
+      load_rows(sDO, &tm_do, &bars[1], row, h, b);
+    }
+    ++q_iss;
+    ok = cta_wait(&bars[1], (uint32_t)(i & 1));
+    if (!ok) break;
+    ++q_cons;
+    // sigma(Q) row r (bf16 operand) and its denominator in fp32
+    float den = 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      float f[8];
+      unpack8(ld_unit(sQ, r, u), f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        f[e] = sig(f[e]);
+        den = fmaf(f[e], sZ[8 * u + e], den);
+      }
+      st_unit(sSQ, r, u, f);
+    }
+    publish_writes();
+    ISSUE_MMA(&bars[2], gemm_km(tN, sSQ, sM, false));
+    ok = cta_wait(&bars[2], mph & 1);
+    ++mph;
+    if (!ok) break;
+    tc_fence_after();
+    const float inv = den != 0.f ? 1.f / den : 0.f;
+    float dd = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t nv[32];
+      tmem_ld32(tN + lane_off + 32 * c, nv);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const int u = 4 * c + u4;
+        float o[8], dn[8];
+        unpack8(ld_unit(sDO, r, u), o);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float a = __uint_as_float(nv[8 * u4 + e]) * inv;  // A_mem
+          const float da = g * o[e];
+          dn[e] = da * inv;
+          dd = fmaf(da, a, dd);
+          memt = fmaf(o[e], a, memt);
+        }
+        st_unit(sDN, r, u, dn);
+      }
+    }
+    const float dden = -dd * inv;
+    sDD[r] = dden;
+    publish_writes();
+    ISSUE_MMA(&bars[2], gemm_kk(tD, sDN, sM, false); gemm_mm(tG, sSQ, sDN, i > 0));
+    // Gz: column r of sigma(Q)^T dden, from the exact sigma of the bf16 inputs
+    {
+      float acc = 0.f;
+      for (int rr = 0; rr < 128; ++rr) acc = fmaf(sig(ld_elem(sQ, rr, r)), sDD[rr], acc);
+      gz += acc;
+    }
+    ok = cta_wait(&bars[2], mph & 1);
+    ++mph;
+    if (!ok) break;
+    tc_fence_after();
+    float* dst = dq_mem + ((size_t)bh * p.L + row + r) * D;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t dv[32];
+      tmem_ld32(tD + lane_off + 32 * c, dv);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const int u = 4 * c + u4;
+        float qf[8], o[8];
+        unpack8(ld_unit(sQ, r, u), qf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          o[e] = fmaf(dden, sZ[8 * u + e], __uint_as_float(dv[8 * u4 + e])) * dsig(qf[e]);
+        *reinterpret_cast<float4*>(dst + 8 * u) = make_float4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<float4*>(dst + 8 * u + 4) = make_float4(o[4], o[5], o[6], o[7]);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // Q, dout and tensor-memory reads done before the next tile
+  }
+  if (ok) {
+    float* gm = GM + (((size_t)bh * p.S + s) * D + r) * D;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tG + lane_off + 32 * c, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(gm + 32 * c + e) =
+            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+    }
+    Gz[((size_t)bh * p.S + s) * D + r] = gz;
+    const float tot = block_sum(memt, red);
+    if (tid == 0) mem_part[(size_t)bh * p.S + s] = tot;
+  } else if (tid == 0) {
+    if (m_pending) drain_wait(&bars[0], 0);
+    if (q_iss > q_cons) drain_wait(&bars[1], (uint32_t)((q_iss - 1) & 1));
+  }
+  if (!ok && warp == 0) {
+    if (elect_one()) mma_commit(&bars[3]);
+    __syncwarp();
+    drain_wait(&bars[3], 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// chain: grid = (BH, 4), block 160. Column block cb covers dM[:, 32cb .. 32cb+31];
+// threads 0..127 own one row (32 fp32 values); warp 4 issues the copies of G and the
+// tf32 products (Delta). For s = S-1 .. 0: write X = dM_s as bf16 hi/lo into the
+// stack, then X += GM_s (Linear) or X += GM_s - G_s X (Delta); finally dM_in = X.
+// ---------------------------------------------------------------------------
+constexpr int kChainThreads = 160;
+constexpr int kGBytes = D * D * 4;    // 64 KB
+constexpr int kXtBytes = 32 * D * 4;  // 16 KB: the X block transposed [32][128], tf32
+constexpr int kChainSmem = 2 * kGBytes + kXtBytes + 1024 + 256;
+
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+__global__ void __launch_bounds__(kChainThreads, 1)
+chain_bwd_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__ GM,
+                 const float* dM_out, float* dM_in, __nv_bfloat16* __restrict__ dMs, int S,
+                 int CH, int mode) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sG = smem;
+  uint8_t* sXt = smem + 2 * kGBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kGBytes + kXtBytes);
+  uint64_t* bar_g = bars;        // [2] G chunk landed
+  uint64_t* bar_xt = bars + 2;   // X^T written (4 warp arrivals)
+  uint64_t* bar_mma = bars + 3;  // one G_c X product done
+  uint64_t* bar_seg = bars + 4;  // G_s X of a whole segment done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+
+  const int bh = blockIdx.x, cb = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+  const int c0 = 32 * cb;
+  const bool delta = mode == 1;
+  if (tid == 0) {
+    mbar_init(&bar_g[0], 1);
+    mbar_init(&bar_g[1], 1);
+    mbar_init(bar_xt, 4);
+    mbar_init(bar_mma, 1);
+    mbar_init(bar_seg, 1);
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 4) {
+    if (delta) {
+      // load n of the sequence (s = S-1-n/CH, chunk n%CH): G plane of dpart
+      int g_iss[2] = {0, 0}, g_cons[2] = {0, 0};
+      auto load_g = [&](int n, int buf) {
+        if (elect_one()) {
+          const int s = S - 1 - n / CH, c = n % CH;
+          mbar_arrive_expect_tx(&bar_g[buf], kGBytes);
+          const int plane = ((bh * S + s) * CH + c) * 2 + 1;
+#pragma unroll
+          for (int bx = 0; bx < 4; ++bx)
+            tma_load_3d(sG + buf * kGBytes + bx * (D * 128), &tm_g, &bar_g[buf], bx * 32, 0,
+                        plane);
+        }
+        __syncwarp();
+        ++g_iss[buf];
+      };
+      const uint32_t idesc = idesc_f32acc(2, 0, 0, 128, 32);
+      const int total = S * CH;
+      int n = 0;
+      load_g(0, 0);
+      for (int q = 0; q < S && ok; ++q) {
+        if (!mbar_wait_warp(bar_xt, (uint32_t)(q & 1))) {
+          ok = false;
+          break;
+        }
+        for (int c = 0; c < CH; ++c, ++n) {
+          const int buf = n & 1;
+          if (n + 1 < total) load_g(n + 1, buf ^ 1);
+          if (!mbar_wait_warp(&bar_g[buf], (uint32_t)((n >> 1) & 1))) {
+            ok = false;
+            break;
+          }
+          ++g_cons[buf];
+          tc_fence_after();
+          const uint32_t ga = smem_u32(sG + buf * kGBytes), xb = smem_u32(sXt);
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < D / 8; ++kk) {
+              const uint32_t koff = (uint32_t)(kk >> 2) * (D * 128) + (uint32_t)(kk & 3) * 32;
+              const uint32_t xoff = (uint32_t)(kk >> 2) * (32 * 128) + (uint32_t)(kk & 3) * 32;
+              mma_tf32_ss(tmem_d, sdesc(ga + koff, 16, 1024), sdesc(xb + xoff, 16, 1024), idesc,
+                          (c > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(bar_mma);
+            if (c == CH - 1) mma_commit(bar_seg);
+          }
+          __syncwarp();
+          if (!mbar_wait_warp(bar_mma, (uint32_t)(n & 1))) {
+            ok = false;
+            break;
+          }
+        }
+      }
+      if (!ok) {
+        if (elect_one()) {
+          for (int bf = 0; bf < 2; ++bf)
+            if (g_iss[bf] > g_cons[bf]) drain_wait(&bar_g[bf], (uint32_t)((g_iss[bf] - 1) & 1));
+        }
+        __syncwarp();
+      }
+    }
+  } else {
+    const int r = tid;
+    float x[32];
+    if (dM_out) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 t = *reinterpret_cast<const float4*>(dM_out + ((size_t)bh * D + r) * D + c0 + e);
+        x[e] = t.x; x[e + 1] = t.y; x[e + 2] = t.z; x[e + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] = 0.f;
+    }
+    for (int q = 0; q < S; ++q) {
+      const int s = S - 1 - q;
+      {  // dM_s -> hi / lo bf16
+        __nv_bfloat16* hi = dMs + ((size_t)bh * S + s) * 2 * D * D + (size_t)r * D + c0;
+        __nv_bfloat16* lo = hi + D * D;
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint32_t h4[4], l4[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const __nv_bfloat162 hv = __floats2bfloat162_rn(x[e + 2 * t], x[e + 2 * t + 1]);
+            const float2 hf = __bfloat1622float2(hv);
+            const __nv_bfloat162 lv = __floats2bfloat162_rn(x[e + 2 * t] - hf.x, x[e + 2 * t + 1] - hf.y);
+            h4[t] = *reinterpret_cast<const uint32_t*>(&hv);
+            l4[t] = *reinterpret_cast<const uint32_t*>(&lv);
+          }
+          *reinterpret_cast<uint4*>(hi + e) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+          *reinterpret_cast<uint4*>(lo + e) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+        }
+      }
+      float gm[32];
+      const float* src = GM + (((size_t)bh * S + s) * D + r) * D + c0;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 t = __ldg(reinterpret_cast<const float4*>(src + e));
+        gm[e] = t.x; gm[e + 1] = t.y; gm[e + 2] = t.z; gm[e + 3] = t.w;
+      }
+      if (delta) {
+        // X^T block (tf32) -> shared memory: row c, K-major, 4 boxes of 32 k
+        const uint32_t kb = (uint32_t)(r >> 5), kin = (uint32_t)(r & 31);
+#pragma unroll
+        for (int cc = 0; cc < 32; ++cc) {
+          const uint32_t off = kb * (32 * 128) + sw128((uint32_t)cc, kin >> 2) + (kin & 3) * 4;
+          *reinterpret_cast<uint32_t*>(sXt + off) = tf32_rna(x[cc]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive_warp(bar_xt);
+        if (!mbar_wait_warp(bar_seg, (uint32_t)(q & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t gx[32];
+        tmem_ld32(tmem_d + ((uint32_t)(warp * 32) << 16), gx);
+        tmem_wait_ld();
+        tc_fence_before();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] += gm[e] - __uint_as_float(gx[e]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] += gm[e];
+      }
+    }
+    if (dM_in && ok) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dM_in + ((size_t)bh * D + r) * D + c0 + e) =
+            make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, 32);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// kside: grid = BH * S * T, one CTA per key tile. Tensor memory: A (dV_u = dU) |
+// B (dsigma(K) without dz_s) | R (sigma(K) M_{s-1}, Delta).
+// ---------------------------------------------------------------------------
+constexpr int kKsideSmem = 5 * kTile + 1024 + 64 + 256 + 1024;
+
+__global__ void __launch_bounds__(kThreads, 1)
+kside_bwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_m, const __grid_constant__ CUtensorMap tm_x,
+                 const float* __restrict__ zprev, float* __restrict__ dk_mem,
+                 float* __restrict__ dv_mem, float* __restrict__ gzk, const BwdParams p, int mode) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sK = smem;               // K, then U (Delta)
+  uint8_t* sV = smem + kTile;       // V, then dnumR (Delta)
+  uint8_t* sSK = smem + 2 * kTile;  // sigma(K), bf16
+  uint8_t* sX = smem + 3 * kTile;   // dM_s (hi)
+  uint8_t* sM = smem + 4 * kTile;   // M_{s-1} (hi), Delta
+  float* sZ = reinterpret_cast<float*>(smem + 5 * kTile);
+  float* sDD = sZ + D;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDD + D + 16);  // 0 loads, 1 MMA, 2 drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+
+  int bh, s, j;
+  decode3(p, blockIdx.x, bh, s, j);
+  const int b = bh / p.H, h = bh - b * p.H;
+  const bool delta = mode == 1;
+  const int tid = threadIdx.x, warp = tid >> 5, r = tid;
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot, tA = tmem, tB = tmem + 128, tR = tmem + 256;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int row = s * p.N + j * 128;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], (delta ? 4 * kTile + D * 4 : 3 * kTile));
+    load_rows(sK, &tm_k, &bars[0], row, h, b);
+    load_rows(sV, &tm_v, &bars[0], row, h, b);
+    load_plane(sX, &tm_x, &bars[0], (bh * p.S + s) * 2);
+    if (delta) {
+      load_plane(sM, &tm_m, &bars[0], (bh * p.S + s) * 2);
+      bulk_load(sZ, zprev + ((size_t)bh * p.S + s) * D, D * 4, &bars[0]);
+    }
+  }
+  bool ok = cta_wait(&bars[0], 0);
+  bool loads_pending = !ok;
+  uint32_t mph = 0;
+  float denK = 0.f;
+  if (ok) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      float f[8];
+      unpack8(ld_unit(sK, r, u), f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        f[e] = sig(f[e]);
+        if (delta) denK = fmaf(f[e], sZ[8 * u + e], denK);
+      }
+      st_unit(sSK, r, u, f);
+    }
+    publish_writes();
+    if (delta) {
+      ISSUE_MMA(&bars[1], gemm_km(tR, sSK, sM, false); gemm_km(tA, sSK, sX, false));
+    } else {
+      ISSUE_MMA(&bars[1], gemm_km(tA, sSK, sX, false); gemm_kk(tB, sV, sX, false));
+    }
+    ok = cta_wait(&bars[1], mph & 1);
+    ++mph;
+  }
+  const size_t base = ((size_t)bh * p.L + row + r) * D;
+  if (ok && !delta) {
+    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t a[32], bb[32];
+      tmem_ld32(tA + lane_off + 32 * c, a);
+      tmem_ld32(tB + lane_off + 32 * c, bb);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        *reinterpret_cast<float4*>(dv_mem + base + 32 * c + e) =
+            make_float4(__uint_as_float(a[e]), __uint_as_float(a[e + 1]),
+                        __uint_as_float(a[e + 2]), __uint_as_float(a[e + 3]));
+        *reinterpret_cast<float4*>(dk_mem + base + 32 * c + e) =
+            make_float4(__uint_as_float(bb[e]), __uint_as_float(bb[e + 1]),
+                        __uint_as_float(bb[e + 2]), __uint_as_float(bb[e + 3]));
+      }
+    }
+  } else if (ok && delta) {
+    tc_fence_after();
+    const float inv = denK != 0.f ? 1.f / denK : 0.f;
+    float dd = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t rn[32], du[32];
+      tmem_ld32(tR + lane_off + 32 * c, rn);
+      tmem_ld32(tA + lane_off + 32 * c, du);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const int u = 4 * c + u4;
+        float vv[8], uu[8], dn[8];
+        unpack8(ld_unit(sV, r, u), vv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float rr = __uint_as_float(rn[8 * u4 + e]) * inv;
+          const float dU = __uint_as_float(du[8 * u4 + e]);
+          uu[e] = vv[e] - rr;
+          dn[e] = -dU * inv;
+          dd = fmaf(dU, rr, dd);
+        }
+        st_unit(sK, r, u, uu);  // U over K (no longer needed)
+        st_unit(sV, r, u, dn);  // dnumR over V (this row's V is read)
+      }
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dv_mem + base + 32 * c + e) =
+            make_float4(__uint_as_float(du[e]), __uint_as_float(du[e + 1]),
+                        __uint_as_float(du[e + 2]), __uint_as_float(du[e + 3]));
+    }
+    const float dden = dd * inv;
+    sDD[r] = dden;
+    publish_writes();
+    ISSUE_MMA(&bars[1], gemm_kk(tB, sK, sX, false); gemm_kk(tB, sV, sM, true));
+    {  // column r of sigma(K)^T ddenR over this tile's rows
+      float acc = 0.f;
+      for (int rr = 0; rr < 128; ++rr) acc = fmaf(ld_elem(sSK, rr, r), sDD[rr], acc);
+      gzk[(((size_t)bh * p.S + s) * p.T + j) * D + r] = acc;
+    }
+    ok = cta_wait(&bars[1], mph & 1);
+    ++mph;
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tB + lane_off + 32 * c, v);
+        tmem_wait_ld();
+        float o[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = fmaf(dden, sZ[32 * c + e], __uint_as_float(v[e]));
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dk_mem + base + 32 * c + e) =
+              make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+      }
+    }
+  }
+  if (tid == 0 && loads_pending) drain_wait(&bars[0], 0);
+  if (!ok && warp == 0) {
+    if (elect_one()) mma_commit(&bars[2]);
+    __syncwarp();
+    drain_wait(&bars[2], 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dz: grid = BH, block 128 (feature t). dz_s for s = S-1 .. 0, then dz_in.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(D)
+dz_bwd_kernel(const float* __restrict__ Gz, const float* __restrict__ gzk, const float* dz_out,
+              float* __restrict__ dzs, float* dz_in, int S, int T, int mode) {
+  const int bh = blockIdx.x, t = threadIdx.x;
+  float x = dz_out ? dz_out[(size_t)bh * D + t] : 0.f;
+  for (int s = S - 1; s >= 0; --s) {
+    const size_t i = ((size_t)bh * S + s) * D + t;
+    dzs[i] = x;
+    x += Gz[i];
+    if (mode == 1)
+      for (int jj = 0; jj < T; ++jj) x += gzk[(((size_t)bh * S + s) * T + jj) * D + t];
+  }
+  if (dz_in) dz_in[(size_t)bh * D + t] = x;
+}
+
+// ---------------------------------------------------------------------------
+// dq: grid = BH * S * T, one CTA per query tile. Tensor memory: S | dP' | dQ.
+// Key tiles stream through a 2-stage K/V ring, twice (the two sweeps).
+// ---------------------------------------------------------------------------
+constexpr int kDqSmem = 6 * kTile + 1024 + 64 + 256;
+
+__global__ void __launch_bounds__(kThreads, 1)
+dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+              const float* __restrict__ beta, const float* __restrict__ dq_mem,
+              float* __restrict__ lse_out, float* __restrict__ dp_out,
+              float* __restrict__ dot_part, __nv_bfloat16* __restrict__ dq, const BwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sDO = smem + kTile;
+  uint8_t* sK = smem + 2 * kTile;  // 2 stages
+  uint8_t* sV = smem + 4 * kTile;  // 2 stages
+  float* red = reinterpret_cast<float*>(smem + 6 * kTile);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 16);  // 0 Q, 1-2 K/V, 3 MMA, 4 drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+
+  int bh, s, i;
+  decode3(p, blockIdx.x, bh, s, i);
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int tid = threadIdx.x, warp = tid >> 5, r = tid;
+  const int nk = i + 1, total = 2 * nk;
+  const int row0 = s * p.N + i * 128;
+  if (tid == 0) {
+    for (int x = 0; x < 5; ++x) mbar_init(&bars[x], 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot, tS = tmem, tP = tmem + 128, tQ = tmem + 256;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  int kv_iss[2] = {0, 0}, kv_cons[2] = {0, 0};
+  auto issue_kv = [&](int n) {
+    const int st = n & 1, j = n % nk;
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&bars[1 + st], 2 * kTile);
+      load_rows(sK + st * kTile, &tm_k, &bars[1 + st], s * p.N + j * 128, h, b);
+      load_rows(sV + st * kTile, &tm_v, &bars[1 + st], s * p.N + j * 128, h, b);
+    }
+    ++kv_iss[st];
+  };
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], 2 * kTile);
+    load_rows(sQ, &tm_q, &bars[0], row0, h, b);
+    load_rows(sDO, &tm_do, &bars[0], row0, h, b);
+  }
+  issue_kv(0);
+  if (total > 1) issue_kv(1);
+  const float g = 1.f / (1.f + expf(-beta[h]));
+  const float cds = (1.f - g) * p.rsd, sl = p.sl;
+  float m = -INFINITY, l = 0.f, dacc = 0.f, lse2 = 0.f, dpv = 0.f;
+  uint32_t mph = 0;
+  bool q_pending = true;
+  bool ok = cta_wait(&bars[0], 0);
+  if (ok) q_pending = false;
+  for (int n = 0; ok && n < total; ++n) {
+    const int st = n & 1, j = n % nk;
+    const bool sweep2 = n >= nk, diag = j == i;
+    ok = cta_wait(&bars[1 + st], (uint32_t)((n >> 1) & 1));
+    if (!ok) break;
+    ++kv_cons[st];
+    ISSUE_MMA(&bars[3], gemm_kk(tS, sQ, sK + st * kTile, false);
+              gemm_kk(tP, sDO, sV + st * kTile, false));
+    ok = cta_wait(&bars[3], mph & 1);
+    ++mph;
+    if (!ok) break;
+    tc_fence_after();
+    if (!sweep2) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32];
+        tmem_ld32(tS + lane_off + 32 * c, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const bool masked = diag && (32 * c + e) > r;
+          if (!masked) mx = fmaxf(mx, __uint_as_float(sv[e]));
+        }
+      }
+      const float mn = fmaxf(m, mx);
+      const float alpha = ex2_approx((m - mn) * sl);  // 0 on the first key tile (m = -inf)
+      l *= alpha;
+      dacc *= alpha;
+      m = mn;
+      const float mb = m * sl;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], pv[32];
+        tmem_ld32(tS + lane_off + 32 * c, sv);
+        tmem_ld32(tP + lane_off + 32 * c, pv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const bool masked = diag && (32 * c + e) > r;
+          const float pe = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[e]), sl, -mb));
+          l += pe;
+          dacc = fmaf(pe, __uint_as_float(pv[e]), dacc);
+        }
+      }
+      if (n == nk - 1) {
+        lse2 = mb + log2f(l);
+        dpv = dacc / l;
+      }
+    } else {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sv[64], pv[64];
+        tmem_ld32(tS + lane_off + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(sv));
+        tmem_ld32(tS + lane_off + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+        tmem_ld32(tP + lane_off + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(pv));
+        tmem_ld32(tP + lane_off + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(pv + 32));
+        tmem_wait_ld();
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float ds[2];
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const int c = 64 * hh + 2 * e + w;
+            const bool masked = diag && c > r;
+            const float pe =
+                masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[2 * e + w]), sl, -lse2));
+            ds[w] = cds * pe * (__uint_as_float(pv[2 * e + w]) - dpv);
+          }
+          pk[e] = pack_bf16x2(ds[0], ds[1]);
+        }
+        // dS (bf16 pairs) over S's first 64 columns; half hh covers [32 hh, 32 hh + 32),
+        // which this thread has already read
+        tmem_st32_(tS + lane_off + 32 * hh, pk);
+      }
+      tmem_wait_st();
+      publish_writes();
+      ISSUE_MMA(&bars[3], gemm_tm(tQ, tS, sK + st * kTile, j > 0));
+      ok = cta_wait(&bars[3], mph & 1);
+      ++mph;
+      if (!ok) break;
+      tc_fence_after();
+    }
+    tc_fence_before();
+    __syncthreads();  // tensor-memory reads of S and dP' done; stage st is free
+    if (n + 2 < total) issue_kv(n + 2);
+  }
+  if (ok) {
+    const size_t rowi = (size_t)bh * p.L + row0 + r;
+    const float* src = dq_mem + rowi * D;
+    __nv_bfloat16* dst = dq + rowi * D;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tQ + lane_off + 32 * c, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const float4 a = *reinterpret_cast<const float4*>(src + 32 * c + 8 * u4);
+        const float4 bq = *reinterpret_cast<const float4*>(src + 32 * c + 8 * u4 + 4);
+        const float* w = reinterpret_cast<const float*>(v) + 8 * u4;
+        *reinterpret_cast<uint4*>(dst + 32 * c + 8 * u4) =
+            make_uint4(pack_bf16x2(w[0] + a.x, w[1] + a.y), pack_bf16x2(w[2] + a.z, w[3] + a.w),
+                       pack_bf16x2(w[4] + bq.x, w[5] + bq.y), pack_bf16x2(w[6] + bq.z, w[7] + bq.w));
+      }
+    }
+    lse_out[rowi] = lse2;
+    dp_out[rowi] = dpv;
+    const float tot = block_sum(dpv, red);
+    if (tid == 0) dot_part[blockIdx.x] = tot;
+  } else if (tid == 0) {
+    if (q_pending) drain_wait(&bars[0], 0);
+    for (int st = 0; st < 2; ++st)
+      if (kv_iss[st] > kv_cons[st]) drain_wait(&bars[1 + st], (uint32_t)((kv_iss[st] - 1) & 1));
+  }
+  if (!ok && warp == 0) {
+    if (elect_one()) mma_commit(&bars[4]);
+    __syncwarp();
+    drain_wait(&bars[4], 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dkdv: grid = BH * S * T, one CTA per key tile. Tensor memory: S^T | dP'^T | dV | dK.
+// Query tiles i >= j stream through a 2-stage Q/dout ring with their row statistics.
+// ---------------------------------------------------------------------------
+constexpr int kDkdvSmem = 6 * kTile + 2 * 2 * D * 4 + 1024 + 64 + 256;
+
+__global__ void __launch_bounds__(kThreads, 1)
+dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const float* __restrict__ beta, const float* __restrict__ lse,
+                const float* __restrict__ dpr, const float* __restrict__ dk_mem,
+                const float* __restrict__ dv_mem, const float* __restrict__ dzs,
+                __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, const BwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + kTile;
+  uint8_t* sQ = smem + 2 * kTile;   // 2 stages
+  uint8_t* sDO = smem + 4 * kTile;  // 2 stages
+  float* sLD = reinterpret_cast<float*>(smem + 6 * kTile);  // [stage][lse | D'][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sLD + 4 * D);  // 0 K/V, 1-2 Q, 3 MMA, 4 drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+
+  int bh, s, j;
+  decode3(p, blockIdx.x, bh, s, j);
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int tid = threadIdx.x, warp = tid >> 5, r = tid;
+  const int nq = p.T - j;
+  if (tid == 0) {
+    for (int x = 0; x < 5; ++x) mbar_init(&bars[x], 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot, tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 384;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int krow = s * p.N + j * 128;
+  int q_iss[2] = {0, 0}, q_cons[2] = {0, 0};
+  auto issue_q = [&](int n) {
+    const int st = n & 1, rq = s * p.N + (j + n) * 128;
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&bars[1 + st], 2 * kTile + 2 * D * 4);
+      load_rows(sQ + st * kTile, &tm_q, &bars[1 + st], rq, h, b);
+      load_rows(sDO + st * kTile, &tm_do, &bars[1 + st], rq, h, b);
+      bulk_load(sLD + st * 2 * D, lse + (size_t)bh * p.L + rq, D * 4, &bars[1 + st]);
+      bulk_load(sLD + st * 2 * D + D, dpr + (size_t)bh * p.L + rq, D * 4, &bars[1 + st]);
+    }
+    ++q_iss[st];
+  };
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], 2 * kTile);
+    load_rows(sK, &tm_k, &bars[0], krow, h, b);
+    load_rows(sV, &tm_v, &bars[0], krow, h, b);
+  }
+  issue_q(0);
+  if (nq > 1) issue_q(1);
+  const float g = 1.f / (1.f + expf(-beta[h]));
+  const float cp = 1.f - g, cds = (1.f - g) * p.rsd, sl = p.sl;
+  uint32_t mph = 0;
+  bool kv_pending = true;
+  bool ok = cta_wait(&bars[0], 0);
+  if (ok) kv_pending = false;
+  for (int n = 0; ok && n < nq; ++n) {
+    const int st = n & 1;
+    const bool diag = n == 0;
+    ok = cta_wait(&bars[1 + st], (uint32_t)((n >> 1) & 1));
+    if (!ok) break;
+    ++q_cons[st];
+    ISSUE_MMA(&bars[3], gemm_kk(tS, sK, sQ + st * kTile, false);
+              gemm_kk(tP, sV, sDO + st * kTile, false));
+    ok = cta_wait(&bars[3], mph & 1);
+    ++mph;
+    if (!ok) break;
+    tc_fence_after();
+    const float* ls = sLD + st * 2 * D;
+    const float* dps = ls + D;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t sv[64], pv[64];
+      tmem_ld32(tS + lane_off + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(sv));
+      tmem_ld32(tS + lane_off + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+      tmem_ld32(tP + lane_off + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(pv));
+      tmem_ld32(tP + lane_off + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(pv + 32));
+      tmem_wait_ld();
+      uint32_t pk1[32], pk2[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        float pg[2], ds[2];
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int c = 64 * hh + 2 * e + w;  // query row of the tile
+          const bool masked = diag && c < r;  // key r after query c
+          const float pe = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[2 * e + w]), sl, -ls[c]));
+          pg[w] = cp * pe;
+          ds[w] = cds * pe * (__uint_as_float(pv[2 * e + w]) - dps[c]);
+        }
+        pk1[e] = pack_bf16x2(pg[0], pg[1]);
+        pk2[e] = pack_bf16x2(ds[0], ds[1]);
+      }
+      tmem_st32_(tS + lane_off + 32 * hh, pk1);
+      tmem_st32_(tP + lane_off + 32 * hh, pk2);
+    }
+    tmem_wait_st();
+    publish_writes();
+    ISSUE_MMA(&bars[3], gemm_tm(tV, tS, sDO + st * kTile, n > 0);
+              gemm_tm(tK, tP, sQ + st * kTile, n > 0));
+    ok = cta_wait(&bars[3], mph & 1);
+    ++mph;
+    if (!ok) break;
+    tc_fence_after();
+    tc_fence_before();
+    __syncthreads();
+    if (n + 2 < nq) issue_q(n + 2);
+  }
+  if (ok) {
+    const size_t rowk = (size_t)bh * p.L + krow + r;
+    const float* dz = dzs + ((size_t)bh * p.S + s) * D;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t a[32], bb[32];
+      tmem_ld32(tV + lane_off + 32 * c, a);
+      tmem_ld32(tK + lane_off + 32 * c, bb);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const int u = 4 * c + u4;
+        float kf[8], ov[8], ok8[8];
+        unpack8(ld_unit(sK, r, u), kf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int f = 8 * u + e;
+          ov[e] = __uint_as_float(a[8 * u4 + e]) + dv_mem[rowk * D + f];
+          ok8[e] = __uint_as_float(bb[8 * u4 + e]) + (dk_mem[rowk * D + f] + dz[f]) * dsig(kf[e]);
+        }
+        *reinterpret_cast<uint4*>(dv + rowk * D + 8 * u) =
+            make_uint4(pack_bf16x2(ov[0], ov[1]), pack_bf16x2(ov[2], ov[3]),
+                       pack_bf16x2(ov[4], ov[5]), pack_bf16x2(ov[6], ov[7]));
+        *reinterpret_cast<uint4*>(dk + rowk * D + 8 * u) =
+            make_uint4(pack_bf16x2(ok8[0], ok8[1]), pack_bf16x2(ok8[2], ok8[3]),
+                       pack_bf16x2(ok8[4], ok8[5]), pack_bf16x2(ok8[6], ok8[7]));
+      }
+    }
+  } else if (tid == 0) {
+    if (kv_pending) drain_wait(&bars[0], 0);
+    for (int st = 0; st < 2; ++st)
+      if (q_iss[st] > q_cons[st]) drain_wait(&bars[1 + st], (uint32_t)((q_iss[st] - 1) & 1));
+  }
+  if (!ok && warp == 0) {
+    if (elect_one()) mma_commit(&bars[4]);
+    __syncwarp();
+    drain_wait(&bars[4], 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// dbeta[h] = g (1 - g) sum over batch rows and segments of (sum dout * A_mem - sum D').
+__global__ void dbeta_bwd_kernel(const float* __restrict__ beta, const float* __restrict__ mem_part,
+                                 const float* __restrict__ dot_part, float* __restrict__ dbeta,
+                                 int B, int H, int S, int T) {
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    double acc = 0.0;
+    for (int b = 0; b < B; ++b)
+      for (int s = 0; s < S; ++s) {
+        const size_t seg = ((size_t)b * H + h) * S + s;
+        double t = mem_part[seg];
+        for (int i = 0; i < T; ++i) t -= dot_part[seg * T + i];
+        acc += t;
+      }
+    const float g = 1.f / (1.f + expf(-beta[h]));
+    dbeta[h] = (float)(acc * (double)g * (1.0 - (double)g));
+  }
+}
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+cudaError_t bf16_bwd_set_attributes() {
+  cudaError_t e = cudaFuncSetAttribute(retr_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kRetrSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(chain_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kChainSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kside_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kKsideSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(dq_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(dkdv_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kDkdvSmem);
+  return e;
+}
+
+// Backward scratch after the state path's: per-row statistics, the memory path's
+// fp32 contributions to dq / dk / dv, the per-segment gradients of the state.
+size_t bf16_bwd_workspace_bytes(int BH, long long L, int S, int T, int CH) {
+  const size_t bh = (size_t)BH, rows = bh * (size_t)L, bhs = bh * S;
+  return up256(bf16_workspace_bytes(BH, S, CH)) + 2 * up256(rows * 4) + 3 * up256(rows * D * 4) +
+         up256(bhs * D * D * 4) + up256(bhs * D * 4) + up256(bhs * 2 * D * D * 2) +
+         up256(bhs * D * 4) + up256(bhs * T * D * 4) + up256(bhs * 4) + up256(bhs * T * 4);
+}
+
+cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                 const __nv_bfloat16* v, const float* beta, const float* M_in,
+                                 const float* z_in, const __nv_bfloat16* dout,
+                                 const float* dM_out, const float* dz_out, __nv_bfloat16* dq,
+                                 __nv_bfloat16* dk, __nv_bfloat16* dv, float* dbeta, float* dM_in,
+                                 float* dz_in, int B, int H, long long L, int N, int mode,
+                                 void* scratch, int CH, int CL, cudaStream_t stream) {
+  const int BH = B * H, S = (int)(L / N), T = N / 128;
+  char* ptr = static_cast<char*>(scratch);
+  const Bf16Workspace ws = bf16_workspace_carve(ptr, BH, S, CH);
+  ptr += up256(bf16_workspace_bytes(BH, S, CH));
+  const size_t rows = (size_t)BH * L, bhs = (size_t)BH * S;
+  auto take = [&](size_t bytes) {
+    char* r = ptr;
+    ptr += up256(bytes);
+    return r;
+  };
+  float* lse2 = reinterpret_cast<float*>(take(rows * 4));
+  float* dpr = reinterpret_cast<float*>(take(rows * 4));
+  float* dq_mem = reinterpret_cast<float*>(take(rows * D * 4));
+  float* dk_mem = reinterpret_cast<float*>(take(rows * D * 4));
+  float* dv_mem = reinterpret_cast<float*>(take(rows * D * 4));
+  float* GM = reinterpret_cast<float*>(take(bhs * D * D * 4));
+  float* Gz = reinterpret_cast<float*>(take(bhs * D * 4));
+  __nv_bfloat16* dMs = reinterpret_cast<__nv_bfloat16*>(take(bhs * 2 * D * D * 2));
+  float* dzs = reinterpret_cast<float*>(take(bhs * D * 4));
+  float* gzk = reinterpret_cast<float*>(take(bhs * T * D * 4));
+  float* mem_part = reinterpret_cast<float*>(take(bhs * 4));
+  float* dot_part = reinterpret_cast<float*>(take(bhs * T * 4));
+
+  // M_{s-1} (bf16 hi/lo), z_{s-1} and, for Delta, every segment's G_s
+  cudaError_t e = bf16_state_launch(k, v, M_in, z_in, nullptr, nullptr, ws, BH, L, N, S, CH, CL,
+                                    mode, 0, stream);
+  if (e != cudaSuccess) return e;
+
+  const Bf16Layout lay = Bf16Layout::bhld(B, H, L);
+  CUtensorMap mq, mk, mv, mdo, mm, mx, mg;
+  if (!make_bf16_map4(&mq, q, (uint64_t)L, H, B, lay.q_sl, lay.q_sh, lay.q_sb, 128) ||
+      !make_bf16_map4(&mk, k, (uint64_t)L, H, B, lay.q_sl, lay.q_sh, lay.q_sb, 128) ||
+      !make_bf16_map4(&mv, v, (uint64_t)L, H, B, lay.q_sl, lay.q_sh, lay.q_sb, 128) ||
+      !make_bf16_map4(&mdo, dout, (uint64_t)L, H, B, lay.q_sl, lay.q_sh, lay.q_sb, 128) ||
+      !make_bf16_map(&mm, ws.Mhl, D, (uint64_t)bhs * 2, 128) ||
+      !make_bf16_map(&mx, dMs, D, (uint64_t)bhs * 2, 128))
+    return cudaErrorInvalidValue;
+  if (mode == 1) {
+    // G planes of the state path's dpart, fp32 [planes][128][128]; box 32 x 128
+    EncodeTiledFn enc = get_encode_fn();
+    const cuuint64_t dims[3] = {128, 128, (cuuint64_t)bhs * CH * 2};
+    const cuuint64_t strides[2] = {128 * 4, 128 * 128 * 4};
+    const cuuint32_t box[3] = {32, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (!enc || enc(&mg, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ws.dpart, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    memset(&mg, 0, sizeof(mg));
+  }
+  BwdParams p;
+  p.L = L;
+  p.N = N;
+  p.S = S;
+  p.T = T;
+  p.H = H;
+  const long long tiles = (long long)BH * S * T;
+  if (tiles >= (1ll << 31) || bhs >= (1ull << 31)) return cudaErrorInvalidValue;
+  p.tiles = (unsigned)tiles;
+  p.divT = FastDiv((uint32_t)T);
+  p.divS = FastDiv((uint32_t)S);
+  p.rsd = 0.08838834764831845f;
+  p.sl = 1.4426950408889634f * p.rsd;
+
+  retr_bwd_kernel<<<(unsigned)bhs, kThreads, kRetrSmem, stream>>>(mq, mdo, mm, beta, ws.zprev,
+                                                                  dq_mem, GM, Gz, mem_part, p);
+  chain_bwd_kernel<<<dim3(BH, 4), kChainThreads, kChainSmem, stream>>>(mg, GM, dM_out, dM_in, dMs,
+                                                                        S, CH, mode);
+  kside_bwd_kernel<<<p.tiles, kThreads, kKsideSmem, stream>>>(mk, mv, mm, mx, ws.zprev, dk_mem,
+                                                               dv_mem, gzk, p, mode);
+  dz_bwd_kernel<<<BH, D, 0, stream>>>(Gz, gzk, dz_out, dzs, dz_in, S, T, mode);
+  dq_bwd_kernel<<<p.tiles, kThreads, kDqSmem, stream>>>(mq, mk, mv, mdo, beta, dq_mem, lse2, dpr,
+                                                         dot_part, dq, p);
+  dkdv_bwd_kernel<<<p.tiles, kThreads, kDkdvSmem, stream>>>(mq, mk, mv, mdo, beta, lse2, dpr,
+                                                             dk_mem, dv_mem, dzs, dk, dv, p);
+  dbeta_bwd_kernel<<<1, 128, 0, stream>>>(beta, mem_part, dot_part, dbeta, B, H, S, T);
+  return cudaGetLastError();
+}
+
+}  // namespace infini

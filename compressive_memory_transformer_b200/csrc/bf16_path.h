@@ -62,6 +62,18 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                              const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
                              cudaStream_t stream, const Bf16Layout* lay = nullptr);
 
+// Gradient of the bf16 forward (bf16_bwd.cu): [B, H, L, 128] contiguous, N a multiple
+// of 128, L a multiple of N. `scratch` holds bf16_bwd_workspace_bytes(...) bytes; CH /
+// CL are the state path's token chunking (bf16_state_plan).
+size_t bf16_bwd_workspace_bytes(int BH, long long L, int S, int T, int CH);
+cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                 const __nv_bfloat16* v, const float* beta, const float* M_in,
+                                 const float* z_in, const __nv_bfloat16* dout,
+                                 const float* dM_out, const float* dz_out, __nv_bfloat16* dq,
+                                 __nv_bfloat16* dk, __nv_bfloat16* dv, float* dbeta, float* dM_in,
+                                 float* dz_in, int B, int H, long long L, int N, int mode,
+                                 void* scratch, int CH, int CL, cudaStream_t stream);
+
 // Token-level decode (bf16_decode.cu): partial attention over the KV cache (rows
 // below pos) and the new rows (k, v, also written into the caches), split like flash
 // decoding, then merge + retrieval from the fp32 state + gate. `part` holds

@@ -22,6 +22,7 @@ __device__ unsigned long long g_wait_timeout_ns = 4000000000ull;  // 4 s per wai
 
 cudaError_t bf16_state_set_attributes();
 cudaError_t bf16_attn_set_attributes();
+cudaError_t bf16_bwd_set_attributes();
 
 namespace {
 
@@ -51,6 +52,7 @@ cudaError_t prepare_device(int* dev_out) {
   if (g_prepared[dev].load(std::memory_order_acquire)) return cudaSuccess;
   e = bf16_state_set_attributes();
   if (e == cudaSuccess) e = bf16_attn_set_attributes();
+  if (e == cudaSuccess) e = bf16_bwd_set_attributes();
   SideStream& sd = g_side[dev];
   if (e == cudaSuccess && !sd.stream) e = cudaStreamCreateWithFlags(&sd.stream, cudaStreamNonBlocking);
   if (e == cudaSuccess && !sd.fork) e = cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming);
@@ -372,6 +374,68 @@ int decode_impl(const void* q, const void* k, const void* v, const float* beta, 
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
+// Gradient of the bf16 forward: the state path rebuilds every segment's incoming
+// state, then the backward kernels (bf16_bwd.cu) run in order on the caller's stream.
+int backward_impl(const void* q, const void* k, const void* v, const float* beta,
+                  const float* M_in, const float* z_in, const void* dout, const float* dM_out,
+                  const float* dz_out, void* dq, void* dk, void* dv, float* dbeta, float* dM_in,
+                  float* dz_in, int B, int H, long long L, int N, int d, int mode,
+                  cudaStream_t stream) {
+  if (!beta || !dbeta) return INFINI_ERR_NULL;
+  if (L > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv)) return INFINI_ERR_NULL;
+  if ((M_in == nullptr) != (z_in == nullptr)) return INFINI_ERR_NULL;
+  if ((dM_out == nullptr) != (dz_out == nullptr)) return INFINI_ERR_NULL;
+  if ((dM_in == nullptr) != (dz_in == nullptr)) return INFINI_ERR_NULL;
+  if (B < 1 || H < 1 || N < 1 || L < 0 || d < 1) return INFINI_ERR_SHAPE;
+  if (mode != INFINI_LINEAR && mode != INFINI_DELTA) return INFINI_ERR_UNSUPPORTED;
+  if (d != 128 || N % 128 != 0 || L % N != 0) return INFINI_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > (1LL << 30) || overflows(BH, L) || overflows(BH * L, (long long)d * 4) ||
+      L >= (1LL << 31))
+    return INFINI_ERR_SHAPE;
+  const void* tok[] = {q, k, v, dout, dq, dk, dv};
+  for (const void* p : tok)
+    if (L > 0 && !aligned16(p)) return INFINI_ERR_ALIGN;
+  const void* st_ptrs[] = {M_in, z_in, dM_out, dz_out, dM_in, dz_in};
+  for (const void* p : st_ptrs)
+    if (p && !aligned16(p)) return INFINI_ERR_ALIGN;
+  const size_t nio = (size_t)(BH * L * d) * 2;
+  const size_t nM = (size_t)BH * d * d * sizeof(float), nz = (size_t)BH * d * sizeof(float);
+  const size_t nb = (size_t)H * sizeof(float);
+  const void* ins[] = {q, k, v, dout, M_in, z_in, dM_out, dz_out, beta};
+  const size_t in_n[] = {nio, nio, nio, nio, nM, nz, nM, nz, nb};
+  void* outs[] = {dq, dk, dv, dM_in, dz_in, dbeta};
+  const size_t out_n[] = {nio, nio, nio, nM, nz, nb};
+  for (int a = 0; a < 6; ++a) {
+    if (L == 0 && a < 3) continue;
+    for (int c = 0; c < 9; ++c)
+      if (overlap(outs[a], out_n[a], ins[c], in_n[c])) return INFINI_ERR_ALIAS;
+    for (int c = a + 1; c < 6; ++c)
+      if (overlap(outs[a], out_n[a], outs[c], out_n[c])) return INFINI_ERR_ALIAS;
+  }
+  int dev = 0;
+  if (prepare_device(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
+  if (L == 0) {
+    // no tokens: the state passes through unchanged, beta has no influence
+    if (cudaMemsetAsync(dbeta, 0, nb, stream) != cudaSuccess) return INFINI_ERR_CUDA;
+    return pass_state(dM_out, dz_out, dM_in, dz_in, BH, d, stream);
+  }
+  const int S = (int)(L / N), T = N / 128;
+  int CH = 1, CL = N;
+  bf16_state_plan((int)BH, S, N, &CH, &CL);
+  if (BH * S * CH >= (1LL << 31) || BH * S * T >= (1LL << 31)) return INFINI_ERR_SHAPE;
+  Scratch sc;
+  const int st = get_scratch(sc, bf16_bwd_workspace_bytes((int)BH, L, S, T, CH), nullptr, stream);
+  if (st != INFINI_OK) return st;
+  const cudaError_t e = bf16_backward_launch(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), beta, M_in, z_in,
+      static_cast<const __nv_bfloat16*>(dout), dM_out, dz_out, static_cast<__nv_bfloat16*>(dq),
+      static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), dbeta, dM_in, dz_in, B, H,
+      L, N, mode, sc.ptr, CH, CL, stream);
+  return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace infini
 
@@ -473,6 +537,15 @@ int infini_attn_forward_ex(const void* q, const void* k, const void* v, const fl
                            int dtype, const infini_attn_opts_t* opts, void* stream) {
   return forward_impl(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, L, N, d, mode, dtype,
                       opts, static_cast<cudaStream_t>(stream));
+}
+
+int infini_attn_backward(const void* q, const void* k, const void* v, const float* beta,
+                         const float* M_in, const float* z_in, const void* dout,
+                         const float* dM_out, const float* dz_out, void* dq, void* dk, void* dv,
+                         float* dbeta, float* dM_in, float* dz_in, int B, int H, long long L,
+                         int N, int d, int mode, void* stream) {
+  return backward_impl(q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv, dbeta, dM_in,
+                       dz_in, B, H, L, N, d, mode, static_cast<cudaStream_t>(stream));
 }
 
 int infini_attn_device_status(void) {

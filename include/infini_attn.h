@@ -193,6 +193,40 @@ int infini_attn_decode(const void* q, const void* k, const void* v, const float*
                        void* k_cache, void* v_cache, float* M, float* z, void* out, int B, int H,
                        int n, int pos, int N, int d, int mode, void* stream);
 
+/*
+ * Gradient of infini_attn_forward (bf16) with respect to q, k, v, beta and the
+ * incoming state, for the loss sum(dout * out) + sum(dM_out * M_out) +
+ * sum(dz_out * z_out). The pages define only the forward ("Leave No Context
+ * Behind", arXiv 2404.07143, sections 3.1, 3.3-3.5 as quoted on
+ * llm-papers-study.pages.dev); this is the chain rule through its steps. A row whose
+ * retrieval denominator is exactly 0 (the zero state) retrieves the constant 0 and
+ * passes no gradient; sigma'(x) = 1 for x > 0, e^x otherwise.
+ *
+ *   q, k, v, dout      device, bf16 [B, H, L, d] contiguous, the forward's inputs and
+ *                      the gradient of its output
+ *   beta               device, fp32 [H]
+ *   M_in, z_in         device, fp32 [B, H, d, d] / [B, H, d], the forward's incoming
+ *                      state (both NULL: the zero state)
+ *   dM_out, dz_out     device, fp32, gradients of the forward's final state (both
+ *                      NULL: zero)
+ *   dq, dk, dv         device, bf16 [B, H, L, d], written
+ *   dbeta              device, fp32 [H], written (summed over the batch)
+ *   dM_in, dz_in       device, fp32, gradients of the incoming state (both NULL: not
+ *                      written)
+ * Requires d = 128, N a multiple of 128 and L a multiple of N
+ * (INFINI_ERR_UNSUPPORTED otherwise); every pointer 16-byte aligned; no output may
+ * overlap an input or another output (INFINI_ERR_ALIAS). L = 0 writes dbeta = 0 and
+ * passes (dM_out, dz_out) through to (dM_in, dz_in). Asynchronous on `stream`;
+ * scratch (about 1.6 KB per token and head) comes from the stream-ordered
+ * allocator (INFINI_ERR_NOMEM). The forward's state path runs again inside the call
+ * to rebuild every segment's incoming state.
+ */
+int infini_attn_backward(const void* q, const void* k, const void* v, const float* beta,
+                         const float* M_in, const float* z_in, const void* dout,
+                         const float* dM_out, const float* dz_out, void* dq, void* dk, void* dv,
+                         float* dbeta, float* dM_in, float* dz_in, int B, int H, long long L,
+                         int N, int d, int mode, void* stream);
+
 /* fp32 q/k/v/out variants of infini_attn_forward and infini_attn_step; 1 <= d <= 128. */
 int infini_attn_forward_f32(const float* q, const float* k, const float* v, const float* beta,
                             const float* M_in, const float* z_in, float* out, float* M_out,

@@ -177,3 +177,34 @@ def test_forward_gqa_rejects_bad_arguments(lib, kw, code):
     assert lib.raw_call("infini_attn_forward_gqa", a["q"], a["k"], a["v"], a["beta"], a["M_in"],
                         a["z_in"], a["out"], a["M_out"], a["z_out"], a["B"], a["H"], a["H_kv"],
                         a["L"], a["N"], a["d"], a["mode"], a["layout"], None) == code
+
+
+IN0, OUT0 = 1 << 24, 1 << 28  # inputs and outputs of the gradient, 1 MiB apart each
+
+
+def call_backward(lib, q=IN0, k=IN0 + (1 << 20), v=IN0 + (2 << 20), beta=IN0 + (3 << 20),
+                  M_in=None, z_in=None, dout=IN0 + (4 << 20), dM_out=None, dz_out=None,
+                  dq=OUT0, dk=OUT0 + (1 << 20), dv=OUT0 + (2 << 20), dbeta=OUT0 + (3 << 20),
+                  dM_in=None, dz_in=None, B=1, H=1, L=256, N=128, d=128, mode=0):
+    return lib.raw_call("infini_attn_backward", q, k, v, beta, M_in, z_in, dout, dM_out, dz_out,
+                        dq, dk, dv, dbeta, dM_in, dz_in, B, H, L, N, d, mode, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(dout=None), -1), (dict(dbeta=None), -1), (dict(dq=None), -1),
+    (dict(M_in=OUT0 * 2), -1),            # M_in without z_in
+    (dict(dM_out=OUT0 * 2), -1),          # dM_out without dz_out
+    (dict(dM_in=OUT0 * 2), -1),           # dM_in without dz_in
+    (dict(B=0), -2), (dict(N=0), -2), (dict(L=-1), -2),
+    (dict(d=64), -3), (dict(mode=2), -3),
+    (dict(N=192, L=384), -3),             # N not a multiple of 128
+    (dict(L=384, N=256), -3),             # L not a multiple of N
+    (dict(dq=OUT0 + 8), -4), (dict(dM_in=OUT0 * 2 + 4, dz_in=OUT0 * 3), -4),
+    (dict(dq=IN0), -8),                   # dq is q
+    (dict(dk=OUT0 + 4096), -8),           # dk inside dq
+    (dict(dbeta=IN0 + (3 << 20)), -8),    # dbeta is beta
+    (dict(dM_in=IN0 + (4 << 20), dz_in=OUT0 * 2), -8),  # dM_in over dout
+])
+def test_backward_rejects_bad_arguments(lib, kw, code):
+    """Every argument error of the gradient entry point is reported on the host."""
+    assert call_backward(lib, **kw) == code
