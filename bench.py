@@ -573,6 +573,62 @@ def run_extra(args, device):
                           "hbm_gbs": by16 / (ms16 / 1e3) / 1e9,
                           "frac_hbm": by16 / (ms16 / 1e3) / 1e9 / hbm_peak},
                       "hbm_peak_gbs": hbm_peak})
+    if which in ("backward", "all"):
+        # infini_attn_backward on the 1B-layer shape: gradients of q, k, v, beta and the
+        # incoming state for a loss through the output (dout ~ N(0, 1), bf16)
+        from synthetic_inputs import normal
+        Bc, Hc, Lc, Nc = 4, 8, 32768, 2048
+        inp = make_inputs(Bc, Hc, Lc, D, torch.bfloat16, seed=0, device=device, gen_device="cuda")
+        dout = normal((Bc, Hc, Lc, D), torch.bfloat16, 0, 7, device="cuda").to(device)
+        res = {}
+        ws = torch.empty(ia.backward_workspace_size(Bc, Hc, Lc, Nc, D, ia.DELTA), dtype=torch.uint8,
+                         device=device)
+        for mode, name in ((ia.LINEAR, "linear"), (ia.DELTA, "delta")):
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(3)]
+            for e in (e for row in evs for e in row):
+                e.record(stream)  # torch creates the CUDA event on its first record
+            it = [0]
+
+            def f():
+                e = evs[it[0] % 3]
+                it[0] += 1
+                e[0].record(stream)
+                ia.infini_attn_backward(inp["q"], inp["k"], inp["v"], inp["beta"], Nc, mode, dout,
+                                        workspace=ws, stage_events=e[1:])
+            for _ in range(2):
+                f()
+            torch.cuda.synchronize()
+            it[0] = 0
+            ms = _timed(f, 3, stream)
+            # per stage, averaged over the three timed calls: memory path, dq, dk/dv
+            st_ms = [sum(e[k].elapsed_time(e[k + 1]) for e in evs) / 3 for k in range(3)]
+            pairs = Bc * Hc * (Lc // Nc) * (Nc // 128) * (Nc // 128 + 1) // 2  # tile pairs
+            att = pairs * 2 * 128 * 128 * D  # one 128 x 128 x 128 product over every pair
+            # algorithmic products per token and head: the four gradient products of the
+            # causal attention (dP = dout V^T, dV = P^T dout, dQ = dS K, dK = dS^T Q) over
+            # (N + 1) / 2 keys on average, and the memory's d x d products (Linear: dnum M^T,
+            # sigma(Q)^T dnum, V dM^T, sigma(K) dM; Delta adds U dM^T, dnumR M^T in place of
+            # V dM^T and the chain's G_s dM_s, 2 d^3 per segment)
+            mem = 8 * D * D if mode == ia.LINEAR else 10 * D * D + 2 * D ** 3 / Nc
+            flops = Bc * Hc * Lc * (4 * D * (Nc + 1) + mem)
+            tf = flops / (ms / 1e3) / 1e12
+            res[name] = {"ms_per_call": ms, "tokens_per_s": Bc * Lc / (ms / 1e3),
+                         "algorithmic_tflops": tf, "frac_of_sustained_bf16": tf / peak_sust,
+                         "frac_of_burst_bf16": tf / peak_burst,
+                         "stage_ms": {"memory_path": st_ms[0], "dq_kernel": st_ms[1],
+                                      "dkdv_kernel": st_ms[2]},
+                         # executed tile products: dq 5 per tile pair (S, dP' twice, dQ),
+                         # dk/dv 4 (S^T, dP'^T, dV, dK)
+                         "dq_kernel_executed_tflops": 5 * att / (st_ms[1] / 1e3) / 1e12,
+                         "dkdv_kernel_executed_tflops": 4 * att / (st_ms[2] / 1e3) / 1e12}
+        assert ia.device_status() == 0
+        del inp, dout, ws
+        lines.append({"config": "backward: B=4, H=8, d=128, N=2048, L=32768, bf16, "
+                                "infini_attn_backward (loss through out)",
+                      **res, "peak_source": src,
+                      "note": "one call: the state path rebuilt, then the seven backward "
+                              "kernels; executed tensor work is about 2.3x the algorithmic "
+                              "count (S and dP' are recomputed in both attention kernels)"})
     return lines
 
 
@@ -584,7 +640,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--config", choices=["c2", "c3", "c4", "c5", "decode", "all"], default="c2",
+    ap.add_argument("--config", choices=["c2", "c3", "c4", "c5", "decode", "backward", "all"],
+                    default="c2",
                     help="c2 (default) prints the headline line; the others print one extra "
                          "line per workload of the configuration list")
     args = ap.parse_args()

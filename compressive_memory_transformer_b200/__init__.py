@@ -61,6 +61,8 @@ _SIGS = {
     "infini_attn_forward_gqa": [_vp] * 9 + [_i, _i, _i, _ll, _i, _i, _i, _i, _vp],
     "infini_attn_state_sum": [_vp, _vp, _i] + [_vp] * 4 + [_i, _i, _i, _vp],
     "infini_attn_backward": [_vp] * 15 + [_i, _i, _ll, _i, _i, _i, _vp],
+    "infini_attn_backward_ex": [_vp] * 15 + [_i, _i, _ll, _i, _i, _i, ctypes.POINTER(Opts), _vp],
+    "infini_attn_backward_workspace_size": [_i, _i, _ll, _i, _i, _i],
     "infini_attn_workspace_size": [_i, _i, _ll, _i, _i, _i, _i],
     "infini_attn_device_status": [],
     "infini_attn_selftest_timeout": [_ll, _vp],
@@ -73,6 +75,7 @@ for _name, _args in _SIGS.items():
     _f.restype = _i
 _lib.infini_attn_strerror.restype = ctypes.c_char_p
 _lib.infini_attn_workspace_size.restype = ctypes.c_size_t
+_lib.infini_attn_backward_workspace_size.restype = ctypes.c_size_t
 
 # every symbol the header declares (checked by the CPU tests)
 EXPORTED = tuple(_SIGS)
@@ -259,11 +262,14 @@ def infini_attn_state_sum(dM, dz, M_in=None, z_in=None, M_out=None, z_out=None, 
 
 
 def infini_attn_backward(q, k, v, beta, N, mode, dout, M_in=None, z_in=None, dM_out=None,
-                         dz_out=None, state_grad=True, stream=None):
+                         dz_out=None, state_grad=True, workspace=None, stage_events=None,
+                         stream=None):
     """Gradient of infini_attn_forward (bf16, [B, H, L, 128], N a multiple of 128, L a
     multiple of N) for the loss sum(dout * out) + sum(dM_out * M_out) + sum(dz_out *
     z_out). Returns (dq, dk, dv, dbeta, dM_in, dz_in); dM_in, dz_in are None when
-    state_grad is False."""
+    state_grad is False. workspace: optional uint8 CUDA tensor of at least
+    backward_workspace_size(...) bytes; stage_events: up to three torch.cuda.Event
+    recorded after the memory path, the dq kernel and the dk/dv kernel."""
     B, H, L, d, _, _, _ = _prepare(q, k, v, beta, M_in, z_in, None, None, None, False)
     if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_cuda or not dout.is_contiguous():
         raise ValueError("dout must be a contiguous CUDA tensor shaped and typed like q")
@@ -276,11 +282,24 @@ def infini_attn_backward(q, k, v, beta, N, mode, dout, M_in=None, z_in=None, dM_
     if state_grad:
         dM_in = torch.empty((B, H, d, d), device=q.device, dtype=torch.float32)
         dz_in = torch.empty((B, H, d), device=q.device, dtype=torch.float32)
-    _check(_lib.infini_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M_in),
-                                     _ptr(z_in), _ptr(dout), _ptr(dM_out), _ptr(dz_out), _ptr(dq),
-                                     _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dM_in), _ptr(dz_in), B,
-                                     H, L, int(N), d, int(mode), _stream_handle(stream)))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(M_in), _ptr(z_in), _ptr(dout),
+            _ptr(dM_out), _ptr(dz_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dM_in),
+            _ptr(dz_in), B, H, L, int(N), d, int(mode))
+    if workspace is None and stage_events is None:
+        _check(_lib.infini_attn_backward(*args, _stream_handle(stream)))
+    else:
+        o = Opts()
+        if workspace is not None:
+            o.workspace = workspace.data_ptr()
+            o.workspace_bytes = workspace.numel() * workspace.element_size()
+        for i, ev in enumerate(stage_events or ()):
+            o.stage_events[i] = ev.cuda_event if ev is not None else None
+        _check(_lib.infini_attn_backward_ex(*args, ctypes.byref(o), _stream_handle(stream)))
     return dq, dk, dv, dbeta, dM_in, dz_in
+
+
+def backward_workspace_size(B, H, L, N, d, mode=LINEAR) -> int:
+    return int(_lib.infini_attn_backward_workspace_size(B, H, L, N, d, mode))
 
 
 def infini_attn_decode(q, k, v, beta, k_cache, v_cache, M, z, pos, mode=LINEAR, out=None,

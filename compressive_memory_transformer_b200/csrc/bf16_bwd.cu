@@ -775,12 +775,78 @@ dz_bwd_kernel(const float* __restrict__ Gz, const float* __restrict__ gzk, const
 }
 
 // ---------------------------------------------------------------------------
-// dq: grid = BH * S * T, one CTA per query tile. Tensor memory: S | dP' | dQ.
-// Key tiles stream through a 2-stage K/V ring, twice (the two sweeps).
+// The two attention kernels below share one pipeline. Every 128-wide key (dq) or
+// query (dk/dv) tile is taken as two 64-column halves, h = 2 n + a for load n and
+// half a, alternating between two tensor-memory buffers (scores and dP' side by
+// side, 64 fp32 columns each). Warpgroup a (warps 4a .. 4a+3) does the softmax
+// arithmetic of every half a, so while one warpgroup works on half h the tensor
+// cores compute half h + 1 (and the gradient products of half h - 1). Warp 8 is the
+// TMA producer, warp 9 allocates tensor memory and issues every MMA from one
+// elected lane. Barriers: SFULL[b] (scores of a half in buffer b ready, one
+// tcgen05.commit), PFULL[b] (the half's bf16 operand written over the buffer, four
+// warp arrivals); each completes once per use of its buffer and cannot run a phase
+// ahead of its waiter (the next use of a buffer is issued only after the previous
+// one's PFULL, and its PFULL needs the next SFULL).
 // ---------------------------------------------------------------------------
-constexpr int kDqSmem = 6 * kTile + 1024 + 64 + 256;
+constexpr int kPipeThreads = 320;
+constexpr uint32_t kIdN64 = idesc_f32acc(1, 0, 0, 128, 64);
 
-__global__ void __launch_bounds__(kThreads, 1)
+// 32 lanes x 16 columns store (bf16 pairs of 32 values per thread)
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+// D = A B^T with N = 64: A[m][k] a full tile, B the 64 rows starting at row 64 a of
+// a tile (both K-major, K = 128)
+__device__ __forceinline__ void gemm_kk_n64(uint32_t d, const uint8_t* a, const uint8_t* b_tile,
+                                            int half) {
+  const uint32_t sa = smem_u32(a), sb = smem_u32(b_tile) + (uint32_t)half * 64 * 128;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    mma_bf16_ss(d, kdesc(sa, kk), kdesc(sb, kk), kIdN64, kk > 0 ? 1u : 0u);
+}
+// D (+)= A X with K = 64: A in tensor memory (32 columns of bf16 pairs), X the 64 rows
+// starting at row 64 a of a tile (MN-major, N = 128)
+__device__ __forceinline__ void gemm_tm_k64(uint32_t d, uint32_t ta, const uint8_t* x_tile,
+                                            int half, bool acc) {
+  const uint32_t sx = smem_u32(x_tile) + (uint32_t)half * 64 * 128;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    mma_bf16_ts(d, ta + 8 * kk, mdesc(sx, kk), kIdKM, (acc || kk > 0) ? 1u : 0u);
+}
+
+enum {
+  P_ONCE = 0,     // tiles loaded once (Q/dout or K/V)
+  P_FULL = 1,     // [2] ring stage loaded
+  P_FREE = 3,     // [2] ring stage no longer read by the tensor cores
+  P_SFULL = 5,    // [2]
+  P_PFULL = 7,    // [2]
+  P_DONE = 9,     // every MMA finished
+  P_COUNT = 10
+};
+
+__device__ __forceinline__ void pipe_init(uint64_t* bars) {
+  for (int x = 0; x < P_COUNT; ++x)
+    mbar_init(&bars[x], (x == P_PFULL || x == P_PFULL + 1) ? 4u : 1u);
+  fence_barrier_init();
+}
+
+// ---------------------------------------------------------------------------
+// dq: grid = BH * S * T, one CTA per query tile i. Loads n = 0 .. 2 (i+1) - 1 stream
+// the key tiles j = n mod (i+1) through a 2-stage K/V ring, twice: the first sweep
+// gives each row's log-sum-exp and D' = dout . A_dot (a running maximum, sum and
+// dP'-weighted sum per warpgroup, merged once), the second dS and dQ = sum dS K.
+// Tensor memory: buffer 0 [0, 128), buffer 1 [128, 256), dQ [256, 384).
+// ---------------------------------------------------------------------------
+constexpr int kDqSmem = 6 * kTile + 3 * 2 * D * 4 + 64 + 256 + 1024;
+
+__global__ void __launch_bounds__(kPipeThreads, 1)
 dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
               const float* __restrict__ beta, const float* __restrict__ dq_mem,
@@ -793,189 +859,236 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   uint8_t* sDO = smem + kTile;
   uint8_t* sK = smem + 2 * kTile;  // 2 stages
   uint8_t* sV = smem + 4 * kTile;  // 2 stages
-  float* red = reinterpret_cast<float*>(smem + 6 * kTile);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 16);  // 0 Q, 1-2 K/V, 3 MMA, 4 drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+  float* xs = reinterpret_cast<float*>(smem + 6 * kTile);  // [wg][m | l | dacc][128]
+  float* red = xs + 3 * 2 * D;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 16);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_COUNT);
 
   int bh, s, i;
   decode3(p, blockIdx.x, bh, s, i);
   const int b = bh / p.H, h = bh - b * p.H;
-  const int tid = threadIdx.x, warp = tid >> 5, r = tid;
-  const int nk = i + 1, total = 2 * nk;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = i + 1, nl = 2 * nk, nh = 2 * nl;
   const int row0 = s * p.N + i * 128;
-  if (tid == 0) {
-    for (int x = 0; x < 5; ++x) mbar_init(&bars[x], 1);
-    fence_barrier_init();
-  }
-  if (warp == 0) {
+  if (threadIdx.x == 0) pipe_init(bars);
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot, tS = tmem, tP = tmem + 128, tQ = tmem + 256;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  int kv_iss[2] = {0, 0}, kv_cons[2] = {0, 0};
-  auto issue_kv = [&](int n) {
-    const int st = n & 1, j = n % nk;
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&bars[1 + st], 2 * kTile);
-      load_rows(sK + st * kTile, &tm_k, &bars[1 + st], s * p.N + j * 128, h, b);
-      load_rows(sV + st * kTile, &tm_v, &bars[1 + st], s * p.N + j * 128, h, b);
+  const uint32_t tmem = *tmem_slot, tQ = tmem + 256;
+  bool ok = true;
+
+  if (warp == 8) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int iss[2] = {0, 0};
+      mbar_arrive_expect_tx(&bars[P_ONCE], 2 * kTile);
+      load_rows(sQ, &tm_q, &bars[P_ONCE], row0, h, b);
+      load_rows(sDO, &tm_do, &bars[P_ONCE], row0, h, b);
+      for (int n = 0; n < nl; ++n) {
+        const int st = n & 1, j = n % nk;
+        if (n >= 2 && !mbar_wait(&bars[P_FREE + st], (uint32_t)(((n >> 1) - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&bars[P_FULL + st], 2 * kTile);
+        load_rows(sK + st * kTile, &tm_k, &bars[P_FULL + st], s * p.N + j * 128, h, b);
+        load_rows(sV + st * kTile, &tm_v, &bars[P_FULL + st], s * p.N + j * 128, h, b);
+        ++iss[st];
+      }
+      if (!ok) {
+        drain_wait(&bars[P_ONCE], 0);
+        for (int st = 0; st < 2; ++st)
+          if (iss[st] > 0) drain_wait(&bars[P_FULL + st], (uint32_t)((iss[st] - 1) & 1));
+      }
     }
-    ++kv_iss[st];
-  };
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], 2 * kTile);
-    load_rows(sQ, &tm_q, &bars[0], row0, h, b);
-    load_rows(sDO, &tm_do, &bars[0], row0, h, b);
-  }
-  issue_kv(0);
-  if (total > 1) issue_kv(1);
-  const float g = 1.f / (1.f + expf(-beta[h]));
-  const float cds = (1.f - g) * p.rsd, sl = p.sl;
-  float m = -INFINITY, l = 0.f, dacc = 0.f, lse2 = 0.f, dpv = 0.f;
-  uint32_t mph = 0;
-  bool q_pending = true;
-  bool ok = cta_wait(&bars[0], 0);
-  if (ok) q_pending = false;
-  for (int n = 0; ok && n < total; ++n) {
-    const int st = n & 1, j = n % nk;
-    const bool sweep2 = n >= nk, diag = j == i;
-    ok = cta_wait(&bars[1 + st], (uint32_t)((n >> 1) & 1));
-    if (!ok) break;
-    ++kv_cons[st];
-    ISSUE_MMA(&bars[3], gemm_kk(tS, sQ, sK + st * kTile, false);
-              gemm_kk(tP, sDO, sV + st * kTile, false));
-    ok = cta_wait(&bars[3], mph & 1);
-    ++mph;
-    if (!ok) break;
-    tc_fence_after();
-    if (!sweep2) {
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    auto issue_sdp = [&](int hh) -> bool {
+      const int n = hh >> 1, a = hh & 1, st = n & 1;
+      if (a == 0 && !mbar_wait_warp(&bars[P_FULL + st], (uint32_t)((n >> 1) & 1))) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t tb = tmem + (uint32_t)a * 128;
+        gemm_kk_n64(tb, sQ, sK + st * kTile, a);        // S  = Q K_j[64a..]^T
+        gemm_kk_n64(tb + 64, sDO, sV + st * kTile, a);  // dP' = dout V_j[64a..]^T
+        mma_commit(&bars[P_SFULL + a]);
+        if (n < nk && a == 1) mma_commit(&bars[P_FREE + st]);  // first sweep: done with K/V
+      }
+      __syncwarp();
+      return true;
+    };
+    ok = mbar_wait_warp(&bars[P_ONCE], 0) && issue_sdp(0) && issue_sdp(1);
+    for (int hh = 0; ok && hh < nh; ++hh) {
+      const int n = hh >> 1, a = hh & 1, st = n & 1;
+      if (!mbar_wait_warp(&bars[P_PFULL + a], (uint32_t)(n & 1))) {
+        ok = false;
+        break;
+      }
+      if (n >= nk) {
+        tc_fence_after();
+        if (elect_one()) {
+          // dQ += dS_h K_j[64a..]  (dS in the first 32 columns of the buffer)
+          gemm_tm_k64(tQ, tmem + (uint32_t)a * 128, sK + st * kTile, a, n > nk || a == 1);
+          if (a == 1) mma_commit(&bars[P_FREE + st]);
+        }
+        __syncwarp();
+      }
+      if (hh + 2 < nh && !issue_sdp(hh + 2)) ok = false;
+    }
+    if (elect_one()) mma_commit(&bars[P_DONE]);
+    __syncwarp();
+    if (!ok) drain_wait(&bars[P_DONE], 0);
+  } else {
+    // ---------------- softmax warpgroups ----------------
+    const int wg = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tb = tmem + (uint32_t)wg * 128 + lane_off;
+    const float g = 1.f / (1.f + expf(-beta[h]));
+    const float cds = (1.f - g) * p.rsd, sl = p.sl;
+    float m = -INFINITY, l = 0.f, dacc = 0.f;
+    for (int n = 0; ok && n < nk; ++n) {
+      if (!mbar_wait_warp(&bars[P_SFULL + wg], (uint32_t)(n & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = n == i;
+      uint32_t sv[64], pv[64];
+      tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(sv));
+      tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+      tmem_ld32(tb + 64, *reinterpret_cast<uint32_t(*)[32]>(pv));
+      tmem_ld32(tb + 96, *reinterpret_cast<uint32_t(*)[32]>(pv + 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive_warp(&bars[P_PFULL + wg]);  // the buffer may take the next half
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32];
-        tmem_ld32(tS + lane_off + 32 * c, sv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const bool masked = diag && (32 * c + e) > r;
-          if (!masked) mx = fmaxf(mx, __uint_as_float(sv[e]));
-        }
-      }
+      for (int c = 0; c < 64; ++c)
+        if (!(diag && 64 * wg + c > r)) mx = fmaxf(mx, __uint_as_float(sv[c]));
+      if (mx == -INFINITY) continue;  // every key of this half is after the row
       const float mn = fmaxf(m, mx);
-      const float alpha = ex2_approx((m - mn) * sl);  // 0 on the first key tile (m = -inf)
+      const float alpha = ex2_approx((m - mn) * sl);  // 0 while m = -inf
       l *= alpha;
       dacc *= alpha;
       m = mn;
       const float mb = m * sl;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32], pv[32];
-        tmem_ld32(tS + lane_off + 32 * c, sv);
-        tmem_ld32(tP + lane_off + 32 * c, pv);
+      for (int c = 0; c < 64; ++c) {
+        const bool masked = diag && 64 * wg + c > r;
+        const float pe = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[c]), sl, -mb));
+        l += pe;
+        dacc = fmaf(pe, __uint_as_float(pv[c]), dacc);
+      }
+    }
+    // merge the two warpgroups' running statistics of row r
+    if (ok) {
+      xs[(wg * 3 + 0) * D + r] = m;
+      xs[(wg * 3 + 1) * D + r] = l;
+      xs[(wg * 3 + 2) * D + r] = dacc;
+    }
+    named_bar_sync(1, 256);
+    float lse2 = 0.f, dpv = 0.f;
+    {
+      const float m0 = xs[0 * D + r], l0 = xs[1 * D + r], d0 = xs[2 * D + r];
+      const float m1 = xs[3 * D + r], l1 = xs[4 * D + r], d1 = xs[5 * D + r];
+      const float mt = fmaxf(m0, m1);
+      const float e0 = ex2_approx((m0 - mt) * sl), e1 = ex2_approx((m1 - mt) * sl);
+      const float lt = l0 * e0 + l1 * e1;
+      lse2 = mt * sl + log2f(lt);
+      dpv = (d0 * e0 + d1 * e1) / lt;
+    }
+    for (int n = nk; ok && n < nl; ++n) {
+      if (!mbar_wait_warp(&bars[P_SFULL + wg], (uint32_t)(n & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = n == nl - 1;
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t sv[32], pv[32], pk[16];
+        tmem_ld32(tb + 32 * c2, sv);
+        tmem_ld32(tb + 64 + 32 * c2, pv);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const bool masked = diag && (32 * c + e) > r;
-          const float pe = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[e]), sl, -mb));
-          l += pe;
-          dacc = fmaf(pe, __uint_as_float(pv[e]), dacc);
-        }
-      }
-      if (n == nk - 1) {
-        lse2 = mb + log2f(l);
-        dpv = dacc / l;
-      }
-    } else {
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t sv[64], pv[64];
-        tmem_ld32(tS + lane_off + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(sv));
-        tmem_ld32(tS + lane_off + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-        tmem_ld32(tP + lane_off + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(pv));
-        tmem_ld32(tP + lane_off + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(pv + 32));
-        tmem_wait_ld();
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < 16; ++e) {
           float ds[2];
 #pragma unroll
           for (int w = 0; w < 2; ++w) {
-            const int c = 64 * hh + 2 * e + w;
-            const bool masked = diag && c > r;
-            const float pe =
-                masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[2 * e + w]), sl, -lse2));
+            const int c = 32 * c2 + 2 * e + w;
+            const bool masked = diag && 64 * wg + c > r;
+            const float pe = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[2 * e + w]), sl, -lse2));
             ds[w] = cds * pe * (__uint_as_float(pv[2 * e + w]) - dpv);
           }
           pk[e] = pack_bf16x2(ds[0], ds[1]);
         }
-        // dS (bf16 pairs) over S's first 64 columns; half hh covers [32 hh, 32 hh + 32),
-        // which this thread has already read
-        tmem_st32_(tS + lane_off + 32 * hh, pk);
+        // columns [16 c2, 16 c2 + 16): scores this thread has already read
+        tmem_st16(tb + 16 * c2, pk);
       }
       tmem_wait_st();
-      publish_writes();
-      ISSUE_MMA(&bars[3], gemm_tm(tQ, tS, sK + st * kTile, j > 0));
-      ok = cta_wait(&bars[3], mph & 1);
-      ++mph;
-      if (!ok) break;
-      tc_fence_after();
+      tc_fence_before();
+      mbar_arrive_warp(&bars[P_PFULL + wg]);
     }
-    tc_fence_before();
-    __syncthreads();  // tensor-memory reads of S and dP' done; stage st is free
-    if (n + 2 < total) issue_kv(n + 2);
-  }
-  if (ok) {
-    const size_t rowi = (size_t)bh * p.L + row0 + r;
-    const float* src = dq_mem + rowi * D;
-    __nv_bfloat16* dst = dq + rowi * D;
+    ok = ok && mbar_wait_warp(&bars[P_DONE], 0);
+    if (ok) {
+      tc_fence_after();
+      const size_t rowi = (size_t)bh * p.L + row0 + r;
+      const float* src = dq_mem + rowi * D + 64 * wg;
+      __nv_bfloat16* dst = dq + rowi * D + 64 * wg;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t v[32];
-      tmem_ld32(tQ + lane_off + 32 * c, v);
-      tmem_wait_ld();
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tQ + lane_off + 64 * wg + 32 * c, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4) {
-        const float4 a = *reinterpret_cast<const float4*>(src + 32 * c + 8 * u4);
-        const float4 bq = *reinterpret_cast<const float4*>(src + 32 * c + 8 * u4 + 4);
-        const float* w = reinterpret_cast<const float*>(v) + 8 * u4;
-        *reinterpret_cast<uint4*>(dst + 32 * c + 8 * u4) =
-            make_uint4(pack_bf16x2(w[0] + a.x, w[1] + a.y), pack_bf16x2(w[2] + a.z, w[3] + a.w),
-                       pack_bf16x2(w[4] + bq.x, w[5] + bq.y), pack_bf16x2(w[6] + bq.z, w[7] + bq.w));
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const float4 x0 = *reinterpret_cast<const float4*>(src + 32 * c + 8 * u4);
+          const float4 x1 = *reinterpret_cast<const float4*>(src + 32 * c + 8 * u4 + 4);
+          const float* w = reinterpret_cast<const float*>(v) + 8 * u4;
+          *reinterpret_cast<uint4*>(dst + 32 * c + 8 * u4) = make_uint4(
+              pack_bf16x2(w[0] + x0.x, w[1] + x0.y), pack_bf16x2(w[2] + x0.z, w[3] + x0.w),
+              pack_bf16x2(w[4] + x1.x, w[5] + x1.y), pack_bf16x2(w[6] + x1.z, w[7] + x1.w));
+        }
+      }
+      if (wg == 0) {
+        lse_out[rowi] = lse2;
+        dp_out[rowi] = dpv;
       }
     }
-    lse_out[rowi] = lse2;
-    dp_out[rowi] = dpv;
-    const float tot = block_sum(dpv, red);
-    if (tid == 0) dot_part[blockIdx.x] = tot;
-  } else if (tid == 0) {
-    if (q_pending) drain_wait(&bars[0], 0);
-    for (int st = 0; st < 2; ++st)
-      if (kv_iss[st] > kv_cons[st]) drain_wait(&bars[1 + st], (uint32_t)((kv_iss[st] - 1) & 1));
-  }
-  if (!ok && warp == 0) {
-    if (elect_one()) mma_commit(&bars[4]);
-    __syncwarp();
-    drain_wait(&bars[4], 0);
+    // the tile's sum of D' (for dbeta); every thread of warpgroup 0 reaches the
+    // barrier, whatever its waits returned
+    if (wg == 0) {
+      float t = ok ? dpv : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) red[warp] = t;
+      named_bar_sync(2, 128);
+      if (threadIdx.x == 0 && ok) dot_part[blockIdx.x] = (red[0] + red[1]) + (red[2] + red[3]);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
 // ---------------------------------------------------------------------------
-// dkdv: grid = BH * S * T, one CTA per key tile. Tensor memory: S^T | dP'^T | dV | dK.
-// Query tiles i >= j stream through a 2-stage Q/dout ring with their row statistics.
+// dkdv: grid = BH * S * T, one CTA per key tile j. Loads n = 0 .. T-1-j stream the
+// query tiles i = j + n (Q, dout and their rows' statistics) through a 2-stage ring.
+// Half a of load n is queries [64a, 64a + 64): S^T = K_j Q^T and dP'^T = V_j dout^T
+// (128 keys x 64 queries), then dV += (1-g) P^T dout and dK += dS^T Q over those 64
+// queries. Tensor memory: buffer 0 [0, 128), buffer 1 [128, 256), dV, dK.
 // ---------------------------------------------------------------------------
-constexpr int kDkdvSmem = 6 * kTile + 2 * 2 * D * 4 + 1024 + 64 + 256;
+constexpr int kDkdvSmem = 6 * kTile + 2 * 2 * D * 4 + 64 + 256 + 1024;
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPipeThreads, 1)
 dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const float* __restrict__ beta, const float* __restrict__ lse,
@@ -990,146 +1103,167 @@ dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint8_t* sQ = smem + 2 * kTile;   // 2 stages
   uint8_t* sDO = smem + 4 * kTile;  // 2 stages
   float* sLD = reinterpret_cast<float*>(smem + 6 * kTile);  // [stage][lse | D'][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sLD + 4 * D);  // 0 K/V, 1-2 Q, 3 MMA, 4 drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sLD + 4 * D + 16);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_COUNT);
 
   int bh, s, j;
   decode3(p, blockIdx.x, bh, s, j);
   const int b = bh / p.H, h = bh - b * p.H;
-  const int tid = threadIdx.x, warp = tid >> 5, r = tid;
-  const int nq = p.T - j;
-  if (tid == 0) {
-    for (int x = 0; x < 5; ++x) mbar_init(&bars[x], 1);
-    fence_barrier_init();
-  }
-  if (warp == 0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nl = p.T - j, nh = 2 * nl;
+  const int krow = s * p.N + j * 128;
+  if (threadIdx.x == 0) pipe_init(bars);
+  if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot, tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 384;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int krow = s * p.N + j * 128;
-  int q_iss[2] = {0, 0}, q_cons[2] = {0, 0};
-  auto issue_q = [&](int n) {
-    const int st = n & 1, rq = s * p.N + (j + n) * 128;
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&bars[1 + st], 2 * kTile + 2 * D * 4);
-      load_rows(sQ + st * kTile, &tm_q, &bars[1 + st], rq, h, b);
-      load_rows(sDO + st * kTile, &tm_do, &bars[1 + st], rq, h, b);
-      bulk_load(sLD + st * 2 * D, lse + (size_t)bh * p.L + rq, D * 4, &bars[1 + st]);
-      bulk_load(sLD + st * 2 * D + D, dpr + (size_t)bh * p.L + rq, D * 4, &bars[1 + st]);
-    }
-    ++q_iss[st];
-  };
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], 2 * kTile);
-    load_rows(sK, &tm_k, &bars[0], krow, h, b);
-    load_rows(sV, &tm_v, &bars[0], krow, h, b);
-  }
-  issue_q(0);
-  if (nq > 1) issue_q(1);
-  const float g = 1.f / (1.f + expf(-beta[h]));
-  const float cp = 1.f - g, cds = (1.f - g) * p.rsd, sl = p.sl;
-  uint32_t mph = 0;
-  bool kv_pending = true;
-  bool ok = cta_wait(&bars[0], 0);
-  if (ok) kv_pending = false;
-  for (int n = 0; ok && n < nq; ++n) {
-    const int st = n & 1;
-    const bool diag = n == 0;
-    ok = cta_wait(&bars[1 + st], (uint32_t)((n >> 1) & 1));
-    if (!ok) break;
-    ++q_cons[st];
-    ISSUE_MMA(&bars[3], gemm_kk(tS, sK, sQ + st * kTile, false);
-              gemm_kk(tP, sV, sDO + st * kTile, false));
-    ok = cta_wait(&bars[3], mph & 1);
-    ++mph;
-    if (!ok) break;
-    tc_fence_after();
-    const float* ls = sLD + st * 2 * D;
-    const float* dps = ls + D;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      uint32_t sv[64], pv[64];
-      tmem_ld32(tS + lane_off + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(sv));
-      tmem_ld32(tS + lane_off + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-      tmem_ld32(tP + lane_off + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(pv));
-      tmem_ld32(tP + lane_off + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(pv + 32));
-      tmem_wait_ld();
-      uint32_t pk1[32], pk2[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        float pg[2], ds[2];
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          const int c = 64 * hh + 2 * e + w;  // query row of the tile
-          const bool masked = diag && c < r;  // key r after query c
-          const float pe = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[2 * e + w]), sl, -ls[c]));
-          pg[w] = cp * pe;
-          ds[w] = cds * pe * (__uint_as_float(pv[2 * e + w]) - dps[c]);
+  const uint32_t tmem = *tmem_slot, tV = tmem + 256, tK = tmem + 384;
+  bool ok = true;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      int iss[2] = {0, 0};
+      mbar_arrive_expect_tx(&bars[P_ONCE], 2 * kTile);
+      load_rows(sK, &tm_k, &bars[P_ONCE], krow, h, b);
+      load_rows(sV, &tm_v, &bars[P_ONCE], krow, h, b);
+      for (int n = 0; n < nl; ++n) {
+        const int st = n & 1, rq = s * p.N + (j + n) * 128;
+        if (n >= 2 && !mbar_wait(&bars[P_FREE + st], (uint32_t)(((n >> 1) - 1) & 1))) {
+          ok = false;
+          break;
         }
-        pk1[e] = pack_bf16x2(pg[0], pg[1]);
-        pk2[e] = pack_bf16x2(ds[0], ds[1]);
+        mbar_arrive_expect_tx(&bars[P_FULL + st], 2 * kTile + 2 * D * 4);
+        load_rows(sQ + st * kTile, &tm_q, &bars[P_FULL + st], rq, h, b);
+        load_rows(sDO + st * kTile, &tm_do, &bars[P_FULL + st], rq, h, b);
+        bulk_load(sLD + st * 2 * D, lse + (size_t)bh * p.L + rq, D * 4, &bars[P_FULL + st]);
+        bulk_load(sLD + st * 2 * D + D, dpr + (size_t)bh * p.L + rq, D * 4, &bars[P_FULL + st]);
+        ++iss[st];
       }
-      tmem_st32_(tS + lane_off + 32 * hh, pk1);
-      tmem_st32_(tP + lane_off + 32 * hh, pk2);
-    }
-    tmem_wait_st();
-    publish_writes();
-    ISSUE_MMA(&bars[3], gemm_tm(tV, tS, sDO + st * kTile, n > 0);
-              gemm_tm(tK, tP, sQ + st * kTile, n > 0));
-    ok = cta_wait(&bars[3], mph & 1);
-    ++mph;
-    if (!ok) break;
-    tc_fence_after();
-    tc_fence_before();
-    __syncthreads();
-    if (n + 2 < nq) issue_q(n + 2);
-  }
-  if (ok) {
-    const size_t rowk = (size_t)bh * p.L + krow + r;
-    const float* dz = dzs + ((size_t)bh * p.S + s) * D;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t a[32], bb[32];
-      tmem_ld32(tV + lane_off + 32 * c, a);
-      tmem_ld32(tK + lane_off + 32 * c, bb);
-      tmem_wait_ld();
-#pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4) {
-        const int u = 4 * c + u4;
-        float kf[8], ov[8], ok8[8];
-        unpack8(ld_unit(sK, r, u), kf);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int f = 8 * u + e;
-          ov[e] = __uint_as_float(a[8 * u4 + e]) + dv_mem[rowk * D + f];
-          ok8[e] = __uint_as_float(bb[8 * u4 + e]) + (dk_mem[rowk * D + f] + dz[f]) * dsig(kf[e]);
-        }
-        *reinterpret_cast<uint4*>(dv + rowk * D + 8 * u) =
-            make_uint4(pack_bf16x2(ov[0], ov[1]), pack_bf16x2(ov[2], ov[3]),
-                       pack_bf16x2(ov[4], ov[5]), pack_bf16x2(ov[6], ov[7]));
-        *reinterpret_cast<uint4*>(dk + rowk * D + 8 * u) =
-            make_uint4(pack_bf16x2(ok8[0], ok8[1]), pack_bf16x2(ok8[2], ok8[3]),
-                       pack_bf16x2(ok8[4], ok8[5]), pack_bf16x2(ok8[6], ok8[7]));
+      if (!ok) {
+        drain_wait(&bars[P_ONCE], 0);
+        for (int st = 0; st < 2; ++st)
+          if (iss[st] > 0) drain_wait(&bars[P_FULL + st], (uint32_t)((iss[st] - 1) & 1));
       }
     }
-  } else if (tid == 0) {
-    if (kv_pending) drain_wait(&bars[0], 0);
-    for (int st = 0; st < 2; ++st)
-      if (q_iss[st] > q_cons[st]) drain_wait(&bars[1 + st], (uint32_t)((q_iss[st] - 1) & 1));
-  }
-  if (!ok && warp == 0) {
-    if (elect_one()) mma_commit(&bars[4]);
+  } else if (warp == 9) {
+    auto issue_sdp = [&](int hh) -> bool {
+      const int n = hh >> 1, a = hh & 1, st = n & 1;
+      if (a == 0 && !mbar_wait_warp(&bars[P_FULL + st], (uint32_t)((n >> 1) & 1))) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t tb = tmem + (uint32_t)a * 128;
+        gemm_kk_n64(tb, sK, sQ + st * kTile, a);        // S^T  = K_j Q[64a..]^T
+        gemm_kk_n64(tb + 64, sV, sDO + st * kTile, a);  // dP'^T = V_j dout[64a..]^T
+        mma_commit(&bars[P_SFULL + a]);
+      }
+      __syncwarp();
+      return true;
+    };
+    ok = mbar_wait_warp(&bars[P_ONCE], 0) && issue_sdp(0) && issue_sdp(1);
+    for (int hh = 0; ok && hh < nh; ++hh) {
+      const int n = hh >> 1, a = hh & 1, st = n & 1;
+      if (!mbar_wait_warp(&bars[P_PFULL + a], (uint32_t)(n & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t tb = tmem + (uint32_t)a * 128;
+        gemm_tm_k64(tV, tb, sDO + st * kTile, a, hh > 0);      // dV += (1-g) P^T dout
+        gemm_tm_k64(tK, tb + 64, sQ + st * kTile, a, hh > 0);  // dK += dS^T Q
+        if (a == 1) mma_commit(&bars[P_FREE + st]);
+      }
+      __syncwarp();
+      if (hh + 2 < nh && !issue_sdp(hh + 2)) ok = false;
+    }
+    if (elect_one()) mma_commit(&bars[P_DONE]);
     __syncwarp();
-    drain_wait(&bars[4], 0);
+    if (!ok) drain_wait(&bars[P_DONE], 0);
+  } else {
+    const int wg = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;  // key row of the tile
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tb = tmem + (uint32_t)wg * 128 + lane_off;
+    const float g = 1.f / (1.f + expf(-beta[h]));
+    const float cp = 1.f - g, cds = (1.f - g) * p.rsd, sl = p.sl;
+    for (int n = 0; ok && n < nl; ++n) {
+      const int st = n & 1;
+      // the stage's row statistics (written by TMA) and this half's scores
+      if (!mbar_wait_warp(&bars[P_FULL + st], (uint32_t)((n >> 1) & 1)) ||
+          !mbar_wait_warp(&bars[P_SFULL + wg], (uint32_t)(n & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = n == 0;
+      const float* ls = sLD + st * 2 * D + 64 * wg;
+      const float* dps = ls + D;
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t sv[32], pv[32], pk1[16], pk2[16];
+        tmem_ld32(tb + 32 * c2, sv);
+        tmem_ld32(tb + 64 + 32 * c2, pv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float pg[2], ds[2];
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const int c = 32 * c2 + 2 * e + w;  // query 64 wg + c of the tile
+            const bool masked = diag && 64 * wg + c < r;
+            const float pe = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[2 * e + w]), sl, -ls[c]));
+            pg[w] = cp * pe;
+            ds[w] = cds * pe * (__uint_as_float(pv[2 * e + w]) - dps[c]);
+          }
+          pk1[e] = pack_bf16x2(pg[0], pg[1]);
+          pk2[e] = pack_bf16x2(ds[0], ds[1]);
+        }
+        tmem_st16(tb + 16 * c2, pk1);
+        tmem_st16(tb + 64 + 16 * c2, pk2);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive_warp(&bars[P_PFULL + wg]);
+    }
+    ok = ok && mbar_wait_warp(&bars[P_DONE], 0);
+    if (ok) {
+      tc_fence_after();
+      const size_t rowk = (size_t)bh * p.L + krow + r;
+      const float* dz = dzs + ((size_t)bh * p.S + s) * D;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t a[32], bb[32];
+        const uint32_t col = 64 * wg + 32 * c;
+        tmem_ld32(tV + lane_off + col, a);
+        tmem_ld32(tK + lane_off + col, bb);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const int u = (int)(col >> 3) + u4;
+          float kf[8], ov[8], ok8[8];
+          unpack8(ld_unit(sK, r, u), kf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int f = 8 * u + e;
+            ov[e] = __uint_as_float(a[8 * u4 + e]) + dv_mem[rowk * D + f];
+            ok8[e] = __uint_as_float(bb[8 * u4 + e]) + (dk_mem[rowk * D + f] + dz[f]) * dsig(kf[e]);
+          }
+          *reinterpret_cast<uint4*>(dv + rowk * D + 8 * u) =
+              make_uint4(pack_bf16x2(ov[0], ov[1]), pack_bf16x2(ov[2], ov[3]),
+                         pack_bf16x2(ov[4], ov[5]), pack_bf16x2(ov[6], ov[7]));
+          *reinterpret_cast<uint4*>(dk + rowk * D + 8 * u) =
+              make_uint4(pack_bf16x2(ok8[0], ok8[1]), pack_bf16x2(ok8[2], ok8[3]),
+                         pack_bf16x2(ok8[4], ok8[5]), pack_bf16x2(ok8[6], ok8[7]));
+        }
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -1189,7 +1323,11 @@ cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                                  const float* dM_out, const float* dz_out, __nv_bfloat16* dq,
                                  __nv_bfloat16* dk, __nv_bfloat16* dv, float* dbeta, float* dM_in,
                                  float* dz_in, int B, int H, long long L, int N, int mode,
-                                 void* scratch, int CH, int CL, cudaStream_t stream) {
+                                 void* scratch, int CH, int CL, cudaStream_t stream,
+                                 cudaEvent_t const* events) {
+  auto mark = [&](int i) {
+    if (events && events[i]) cudaEventRecord(events[i], stream);
+  };
   const int BH = B * H, S = (int)(L / N), T = N / 128;
   char* ptr = static_cast<char*>(scratch);
   const Bf16Workspace ws = bf16_workspace_carve(ptr, BH, S, CH);
@@ -1263,10 +1401,13 @@ cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   kside_bwd_kernel<<<p.tiles, kThreads, kKsideSmem, stream>>>(mk, mv, mm, mx, ws.zprev, dk_mem,
                                                                dv_mem, gzk, p, mode);
   dz_bwd_kernel<<<BH, D, 0, stream>>>(Gz, gzk, dz_out, dzs, dz_in, S, T, mode);
-  dq_bwd_kernel<<<p.tiles, kThreads, kDqSmem, stream>>>(mq, mk, mv, mdo, beta, dq_mem, lse2, dpr,
+  mark(0);
+  dq_bwd_kernel<<<p.tiles, kPipeThreads, kDqSmem, stream>>>(mq, mk, mv, mdo, beta, dq_mem, lse2, dpr,
                                                          dot_part, dq, p);
-  dkdv_bwd_kernel<<<p.tiles, kThreads, kDkdvSmem, stream>>>(mq, mk, mv, mdo, beta, lse2, dpr,
+  mark(1);
+  dkdv_bwd_kernel<<<p.tiles, kPipeThreads, kDkdvSmem, stream>>>(mq, mk, mv, mdo, beta, lse2, dpr,
                                                              dk_mem, dv_mem, dzs, dk, dv, p);
+  mark(2);
   dbeta_bwd_kernel<<<1, 128, 0, stream>>>(beta, mem_part, dot_part, dbeta, B, H, S, T);
   return cudaGetLastError();
 }

@@ -72,7 +72,8 @@ cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                                  const float* dM_out, const float* dz_out, __nv_bfloat16* dq,
                                  __nv_bfloat16* dk, __nv_bfloat16* dv, float* dbeta, float* dM_in,
                                  float* dz_in, int B, int H, long long L, int N, int mode,
-                                 void* scratch, int CH, int CL, cudaStream_t stream);
+                                 void* scratch, int CH, int CL, cudaStream_t stream,
+                                 cudaEvent_t const* events = nullptr);
 
 // Token-level decode (bf16_decode.cu): partial attention over the KV cache (rows
 // below pos) and the new rows (k, v, also written into the caches), split like flash

@@ -380,7 +380,7 @@ int backward_impl(const void* q, const void* k, const void* v, const float* beta
                   const float* M_in, const float* z_in, const void* dout, const float* dM_out,
                   const float* dz_out, void* dq, void* dk, void* dv, float* dbeta, float* dM_in,
                   float* dz_in, int B, int H, long long L, int N, int d, int mode,
-                  cudaStream_t stream) {
+                  const infini_attn_opts_t* opts, cudaStream_t stream) {
   if (!beta || !dbeta) return INFINI_ERR_NULL;
   if (L > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv)) return INFINI_ERR_NULL;
   if ((M_in == nullptr) != (z_in == nullptr)) return INFINI_ERR_NULL;
@@ -425,14 +425,17 @@ int backward_impl(const void* q, const void* k, const void* v, const float* beta
   bf16_state_plan((int)BH, S, N, &CH, &CL);
   if (BH * S * CH >= (1LL << 31) || BH * S * T >= (1LL << 31)) return INFINI_ERR_SHAPE;
   Scratch sc;
-  const int st = get_scratch(sc, bf16_bwd_workspace_bytes((int)BH, L, S, T, CH), nullptr, stream);
+  const int st = get_scratch(sc, bf16_bwd_workspace_bytes((int)BH, L, S, T, CH), opts, stream);
   if (st != INFINI_OK) return st;
+  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+  if (opts)
+    for (int i = 0; i < 3; ++i) ev[i] = static_cast<cudaEvent_t>(opts->stage_events[i]);
   const cudaError_t e = bf16_backward_launch(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), beta, M_in, z_in,
       static_cast<const __nv_bfloat16*>(dout), dM_out, dz_out, static_cast<__nv_bfloat16*>(dq),
       static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), dbeta, dM_in, dz_in, B, H,
-      L, N, mode, sc.ptr, CH, CL, stream);
+      L, N, mode, sc.ptr, CH, CL, stream, ev);
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
@@ -545,7 +548,28 @@ int infini_attn_backward(const void* q, const void* k, const void* v, const floa
                          float* dbeta, float* dM_in, float* dz_in, int B, int H, long long L,
                          int N, int d, int mode, void* stream) {
   return backward_impl(q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv, dbeta, dM_in,
-                       dz_in, B, H, L, N, d, mode, static_cast<cudaStream_t>(stream));
+                       dz_in, B, H, L, N, d, mode, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int infini_attn_backward_ex(const void* q, const void* k, const void* v, const float* beta,
+                            const float* M_in, const float* z_in, const void* dout,
+                            const float* dM_out, const float* dz_out, void* dq, void* dk,
+                            void* dv, float* dbeta, float* dM_in, float* dz_in, int B, int H,
+                            long long L, int N, int d, int mode, const infini_attn_opts_t* opts,
+                            void* stream) {
+  return backward_impl(q, k, v, beta, M_in, z_in, dout, dM_out, dz_out, dq, dk, dv, dbeta, dM_in,
+                       dz_in, B, H, L, N, d, mode, opts, static_cast<cudaStream_t>(stream));
+}
+
+size_t infini_attn_backward_workspace_size(int B, int H, long long L, int N, int d, int mode) {
+  (void)mode;
+  if (B < 1 || H < 1 || N < 128 || L <= 0 || d != 128 || N % 128 != 0 || L % N != 0) return 0;
+  const long long BH = (long long)B * H;
+  if (BH > (1LL << 30) || L >= (1LL << 31)) return 0;
+  const int S = (int)(L / N);
+  int CH = 1, CL = N;
+  bf16_state_plan((int)BH, S, N, &CH, &CL);
+  return bf16_bwd_workspace_bytes((int)BH, L, S, N / 128, CH);
 }
 
 int infini_attn_device_status(void) {

@@ -270,6 +270,24 @@ int infini_attn_forward_ex(const void* q, const void* k, const void* v, const fl
                            int dtype, const infini_attn_opts_t* opts, void* stream);
 
 /*
+ * infini_attn_backward with options: opts->workspace (256-byte aligned, at least
+ * infini_attn_backward_workspace_size(...) bytes) replaces the stream-ordered
+ * allocation; opts->stage_events[0..2] (cudaEvent_t or NULL) are recorded on
+ * `stream` after the memory path's kernels (state rebuild, retrieval, state
+ * gradients, update backward), after the dq kernel, and after the dk/dv kernel.
+ */
+int infini_attn_backward_ex(const void* q, const void* k, const void* v, const float* beta,
+                            const float* M_in, const float* z_in, const void* dout,
+                            const float* dM_out, const float* dz_out, void* dq, void* dk,
+                            void* dv, float* dbeta, float* dM_in, float* dz_in, int B, int H,
+                            long long L, int N, int d, int mode, const infini_attn_opts_t* opts,
+                            void* stream);
+
+/* Scratch bytes infini_attn_backward needs for these sizes (0 when the sizes are
+ * not supported or L = 0). */
+size_t infini_attn_backward_workspace_size(int B, int H, long long L, int N, int d, int mode);
+
+/*
  * Device-side status of earlier calls on the current device: INFINI_OK, or
  * INFINI_ERR_TIMEOUT when a bounded wait inside a kernel ran out (the kernel
  * then stopped early and its outputs are invalid). Synchronises the device,
