@@ -28,22 +28,24 @@
 //   retr   (head, segment): retrieval backward over the segment's query tiles ->
 //          dq_mem (fp32), GM_s, Gz_s, the segment's sum of dout * A_mem.
 //   chain  (head, 32-column block): dM_s for s = S-1 .. 0 (bf16 hi/lo stack), dM_in.
-//   kside  (head, segment, key tile): the memory update's backward per key row ->
-//          dk_mem (dsigma(K) without dz_s), dv_mem, per-tile sigma(K)^T ddenR.
-//   dz     (head): dz_s for every segment, dz_in.
+//   dz     (head, Linear): dz_s for every segment, dz_in.
 //   dq     (head, segment, query tile): two sweeps over the key tiles; the first
 //          gives each row's log-sum-exp and D' = dout . A_dot, the second
 //          dQ = sum_j dS_j K_j; adds dq_mem, writes dq, the row statistics and the
 //          tile's sum of D' (for dbeta).
 //   dkdv   (head, segment, key tile): over the query tiles at or after it,
 //          dV = sum_i (1-g) P_i^T dout_i and dK = sum_i dS_i^T Q_i from S^T = K Q^T
-//          and dP'^T = V dout^T; adds dv_mem, (dk_mem + dz_s) * sigma'(K); writes dk, dv.
+//          and dP'^T = V dout^T; then the memory update's backward of its key rows
+//          (dV += sigma(K) dM_s, dsigma(K), and for Delta sigma(K)^T ddenR per tile);
+//          writes dk, dv.
+//   dz, dk_dz (Delta): dz_s for every segment (it needs every tile's sigma(K)^T
+//          ddenR), dz_in, then dk += dz_s * sigma'(K).
 //   dbeta  : per head, summed over batch rows and segments in a fixed order.
 // Every product is a 128 x 128 x 128 bf16 tcgen05 MMA (fp32 accumulation in tensor
 // memory) on 128B-swizzled shared-memory tiles, in the operand forms the forward
 // uses: A, B both K-major (Q K^T), A in tensor memory with B MN-major (P V), and
 // A, B both MN-major (sigma(K)^T V); the Delta chain uses the forward chain's tf32
-// form. Each CTA has 128 threads, thread r owning tile row r (tensor-memory lane r).
+// form. Thread r of a 128-thread group owns tile row r (tensor-memory lane r).
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda.h>
@@ -586,177 +588,6 @@ chain_bwd_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restri
 }
 
 // ---------------------------------------------------------------------------
-// kside: grid = BH * S * T, one CTA per key tile. Tensor memory: A (dV_u = dU) |
-// B (dsigma(K) without dz_s) | R (sigma(K) M_{s-1}, Delta).
-// ---------------------------------------------------------------------------
-constexpr int kKsideSmem = 5 * kTile + 1024 + 64 + 256 + 1024;
-
-__global__ void __launch_bounds__(kThreads, 1)
-kside_bwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const __grid_constant__ CUtensorMap tm_m, const __grid_constant__ CUtensorMap tm_x,
-                 const float* __restrict__ zprev, float* __restrict__ dk_mem,
-                 float* __restrict__ dv_mem, float* __restrict__ gzk, const BwdParams p, int mode) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint8_t* sK = smem;               // K, then U (Delta)
-  uint8_t* sV = smem + kTile;       // V, then dnumR (Delta)
-  uint8_t* sSK = smem + 2 * kTile;  // sigma(K), bf16
-  uint8_t* sX = smem + 3 * kTile;   // dM_s (hi)
-  uint8_t* sM = smem + 4 * kTile;   // M_{s-1} (hi), Delta
-  float* sZ = reinterpret_cast<float*>(smem + 5 * kTile);
-  float* sDD = sZ + D;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDD + D + 16);  // 0 loads, 1 MMA, 2 drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
-
-  int bh, s, j;
-  decode3(p, blockIdx.x, bh, s, j);
-  const int b = bh / p.H, h = bh - b * p.H;
-  const bool delta = mode == 1;
-  const int tid = threadIdx.x, warp = tid >> 5, r = tid;
-  if (tid == 0) {
-    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
-    fence_barrier_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot, tA = tmem, tB = tmem + 128, tR = tmem + 256;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int row = s * p.N + j * 128;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], (delta ? 4 * kTile + D * 4 : 3 * kTile));
-    load_rows(sK, &tm_k, &bars[0], row, h, b);
-    load_rows(sV, &tm_v, &bars[0], row, h, b);
-    load_plane(sX, &tm_x, &bars[0], (bh * p.S + s) * 2);
-    if (delta) {
-      load_plane(sM, &tm_m, &bars[0], (bh * p.S + s) * 2);
-      bulk_load(sZ, zprev + ((size_t)bh * p.S + s) * D, D * 4, &bars[0]);
-    }
-  }
-  bool ok = cta_wait(&bars[0], 0);
-  bool loads_pending = !ok;
-  uint32_t mph = 0;
-  float denK = 0.f;
-  if (ok) {
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      float f[8];
-      unpack8(ld_unit(sK, r, u), f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        f[e] = sig(f[e]);
-        if (delta) denK = fmaf(f[e], sZ[8 * u + e], denK);
-      }
-      st_unit(sSK, r, u, f);
-    }
-    publish_writes();
-    if (delta) {
-      ISSUE_MMA(&bars[1], gemm_km(tR, sSK, sM, false); gemm_km(tA, sSK, sX, false));
-    } else {
-      ISSUE_MMA(&bars[1], gemm_km(tA, sSK, sX, false); gemm_kk(tB, sV, sX, false));
-    }
-    ok = cta_wait(&bars[1], mph & 1);
-    ++mph;
-  }
-  const size_t base = ((size_t)bh * p.L + row + r) * D;
-  if (ok && !delta) {
-    tc_fence_after();
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t a[32], bb[32];
-      tmem_ld32(tA + lane_off + 32 * c, a);
-      tmem_ld32(tB + lane_off + 32 * c, bb);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        *reinterpret_cast<float4*>(dv_mem + base + 32 * c + e) =
-            make_float4(__uint_as_float(a[e]), __uint_as_float(a[e + 1]),
-                        __uint_as_float(a[e + 2]), __uint_as_float(a[e + 3]));
-        *reinterpret_cast<float4*>(dk_mem + base + 32 * c + e) =
-            make_float4(__uint_as_float(bb[e]), __uint_as_float(bb[e + 1]),
-                        __uint_as_float(bb[e + 2]), __uint_as_float(bb[e + 3]));
-      }
-    }
-  } else if (ok && delta) {
-    tc_fence_after();
-    const float inv = denK != 0.f ? 1.f / denK : 0.f;
-    float dd = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t rn[32], du[32];
-      tmem_ld32(tR + lane_off + 32 * c, rn);
-      tmem_ld32(tA + lane_off + 32 * c, du);
-      tmem_wait_ld();
-#pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4) {
-        const int u = 4 * c + u4;
-        float vv[8], uu[8], dn[8];
-        unpack8(ld_unit(sV, r, u), vv);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float rr = __uint_as_float(rn[8 * u4 + e]) * inv;
-          const float dU = __uint_as_float(du[8 * u4 + e]);
-          uu[e] = vv[e] - rr;
-          dn[e] = -dU * inv;
-          dd = fmaf(dU, rr, dd);
-        }
-        st_unit(sK, r, u, uu);  // U over K (no longer needed)
-        st_unit(sV, r, u, dn);  // dnumR over V (this row's V is read)
-      }
-#pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(dv_mem + base + 32 * c + e) =
-            make_float4(__uint_as_float(du[e]), __uint_as_float(du[e + 1]),
-                        __uint_as_float(du[e + 2]), __uint_as_float(du[e + 3]));
-    }
-    const float dden = dd * inv;
-    sDD[r] = dden;
-    publish_writes();
-    ISSUE_MMA(&bars[1], gemm_kk(tB, sK, sX, false); gemm_kk(tB, sV, sM, true));
-    {  // column r of sigma(K)^T ddenR over this tile's rows
-      float acc = 0.f;
-      for (int rr = 0; rr < 128; ++rr) acc = fmaf(ld_elem(sSK, rr, r), sDD[rr], acc);
-      gzk[(((size_t)bh * p.S + s) * p.T + j) * D + r] = acc;
-    }
-    ok = cta_wait(&bars[1], mph & 1);
-    ++mph;
-    if (ok) {
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tB + lane_off + 32 * c, v);
-        tmem_wait_ld();
-        float o[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = fmaf(dden, sZ[32 * c + e], __uint_as_float(v[e]));
-#pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dk_mem + base + 32 * c + e) =
-              make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
-      }
-    }
-  }
-  if (tid == 0 && loads_pending) drain_wait(&bars[0], 0);
-  if (!ok && warp == 0) {
-    if (elect_one()) mma_commit(&bars[2]);
-    __syncwarp();
-    drain_wait(&bars[2], 0);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
-// ---------------------------------------------------------------------------
 // dz: grid = BH, block 128 (feature t). dz_s for s = S-1 .. 0, then dz_in.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(D)
@@ -1085,16 +916,28 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 // Half a of load n is queries [64a, 64a + 64): S^T = K_j Q^T and dP'^T = V_j dout^T
 // (128 keys x 64 queries), then dV += (1-g) P^T dout and dK += dS^T Q over those 64
 // queries. Tensor memory: buffer 0 [0, 128), buffer 1 [128, 256), dV, dK.
+// After the loop the same CTA runs the memory update's backward for its key rows,
+// with K and V still in shared memory and dM_s (bf16, the reverse chain's stack)
+// loaded into the ring stage that frees first: sigma(K) replaces K in place, and
+//   Linear: dV += sigma(K) dM_s;  dsigma(K) = V dM_s^T (+ dz_s)
+//   Delta:  R = sigma(K) M_{s-1} / den_K, dU = sigma(K) dM_s, dV += dU, U = V - R
+//           (over V), dnumR = -dU / den_K, ddenR = rowsum(dU * R) / den_K,
+//           dsigma(K) = U dM_s^T + dnumR M^T + ddenR z, and the tile's sigma(K)^T ddenR
+//           for the z gradients (dz_s, which needs every later segment's, is added
+//           to dk by dk_dz_kernel afterwards).
 // ---------------------------------------------------------------------------
-constexpr int kDkdvSmem = 6 * kTile + 2 * 2 * D * 4 + 64 + 256 + 1024;
+enum { P_X = P_COUNT, P_SK, P_M1, P_SK2, P_M2, P_COUNT2 };
+constexpr int kDkdvSmem = 6 * kTile + 2 * 2 * D * 4 + 5 * D * 4 + 64 + 256 + 1024;
 
 __global__ void __launch_bounds__(kPipeThreads, 1)
 dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const float* __restrict__ beta, const float* __restrict__ lse,
-                const float* __restrict__ dpr, const float* __restrict__ dk_mem,
-                const float* __restrict__ dv_mem, const float* __restrict__ dzs,
-                __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, const BwdParams p) {
+                const __grid_constant__ CUtensorMap tm_m, const __grid_constant__ CUtensorMap tm_x,
+                const float* __restrict__ beta, const float* __restrict__ zprev,
+                const float* __restrict__ lse, const float* __restrict__ dpr,
+                const float* __restrict__ dzs, float* __restrict__ gzk,
+                __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, const BwdParams p,
+                int mode) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -1103,8 +946,11 @@ dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint8_t* sQ = smem + 2 * kTile;   // 2 stages
   uint8_t* sDO = smem + 4 * kTile;  // 2 stages
   float* sLD = reinterpret_cast<float*>(smem + 6 * kTile);  // [stage][lse | D'][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sLD + 4 * D + 16);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_COUNT);
+  float* xs = sLD + 4 * D;    // [2][128] per-warpgroup partial row sums
+  float* sDD = xs + 2 * D;    // [128] ddenR
+  float* gzp = sDD + D;       // [2][128] partial column sums
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gzp + 2 * D + 16);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_COUNT2);
 
   int bh, s, j;
   decode3(p, blockIdx.x, bh, s, j);
@@ -1112,7 +958,21 @@ dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nl = p.T - j, nh = 2 * nl;
   const int krow = s * p.N + j * 128;
-  if (threadIdx.x == 0) pipe_init(bars);
+  const bool delta = mode == 1;
+  const int sx = nl & 1;  // ring stage that holds dM_s (and M_{s-1}, z_{s-1}) at the end
+  uint8_t* sX = sQ + sx * kTile;         // dM_s (hi)
+  uint8_t* sMp = sDO + sx * kTile;       // M_{s-1} (hi), Delta
+  uint8_t* sDN = sQ + (sx ^ 1) * kTile;  // dnumR, Delta (the last load's stage)
+  const float* sZ = sLD + sx * 2 * D;    // z_{s-1}, Delta
+  if (threadIdx.x == 0) {
+    pipe_init(bars);
+    mbar_init(&bars[P_X], 1);
+    mbar_init(&bars[P_SK], 8);
+    mbar_init(&bars[P_M1], 1);
+    mbar_init(&bars[P_SK2], 8);
+    mbar_init(&bars[P_M2], 1);
+    fence_barrier_init();
+  }
   if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -1126,6 +986,7 @@ dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == 8) {
     if (lane == 0) {
       int iss[2] = {0, 0};
+      bool x_iss = false;
       mbar_arrive_expect_tx(&bars[P_ONCE], 2 * kTile);
       load_rows(sK, &tm_k, &bars[P_ONCE], krow, h, b);
       load_rows(sV, &tm_v, &bars[P_ONCE], krow, h, b);
@@ -1142,10 +1003,24 @@ dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bulk_load(sLD + st * 2 * D + D, dpr + (size_t)bh * p.L + rq, D * 4, &bars[P_FULL + st]);
         ++iss[st];
       }
+      // stage sx was last used by load nl - 2 (never when nl == 1)
+      if (ok && nl >= 2 && !mbar_wait(&bars[P_FREE + sx], (uint32_t)(((nl - 2) >> 1) & 1)))
+        ok = false;
+      if (ok) {
+        const int plane = (bh * p.S + s) * 2;
+        mbar_arrive_expect_tx(&bars[P_X], delta ? 2 * kTile + D * 4 : kTile);
+        load_plane(sX, &tm_x, &bars[P_X], plane);
+        if (delta) {
+          load_plane(sMp, &tm_m, &bars[P_X], plane);
+          bulk_load(sLD + sx * 2 * D, zprev + ((size_t)bh * p.S + s) * D, D * 4, &bars[P_X]);
+        }
+        x_iss = true;
+      }
       if (!ok) {
         drain_wait(&bars[P_ONCE], 0);
         for (int st = 0; st < 2; ++st)
           if (iss[st] > 0) drain_wait(&bars[P_FULL + st], (uint32_t)((iss[st] - 1) & 1));
+        if (x_iss) drain_wait(&bars[P_X], 0);
       }
     }
   } else if (warp == 9) {
@@ -1181,7 +1056,39 @@ dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     if (elect_one()) mma_commit(&bars[P_DONE]);
     __syncwarp();
-    if (!ok) drain_wait(&bars[P_DONE], 0);
+    // the memory update's backward: sigma(K) written over K, dM_s (and M, z) loaded
+    ok = ok && mbar_wait_warp(&bars[P_X], 0) && mbar_wait_warp(&bars[P_SK], 0);
+    if (ok) {
+      tc_fence_after();
+      if (elect_one()) {
+        if (delta) {
+          gemm_km(tmem, sK, sMp, false);       // R_num = sigma(K) M_{s-1}
+          gemm_km(tmem + 128, sK, sX, false);  // dU = sigma(K) dM_s
+        } else {
+          gemm_kk(tmem, sV, sX, false);        // V dM_s^T
+        }
+        gemm_km(tV, sK, sX, true);             // dV += sigma(K) dM_s
+        mma_commit(&bars[P_M1]);
+      }
+      __syncwarp();
+      if (delta) {
+        ok = mbar_wait_warp(&bars[P_SK2], 0);
+        if (ok) {
+          tc_fence_after();
+          if (elect_one()) {
+            gemm_kk(tmem, sV, sX, false);     // U dM_s^T   (U written over V)
+            gemm_kk(tmem, sDN, sMp, true);    // + dnumR M^T
+            mma_commit(&bars[P_M2]);
+          }
+          __syncwarp();
+        }
+      }
+    }
+    if (!ok) {
+      if (elect_one()) mma_commit(&bars[P_M2]);
+      __syncwarp();
+      drain_wait(&bars[P_M2], 0);
+    }
   } else {
     const int wg = warp >> 2;
     const int r = (warp & 3) * 32 + lane;  // key row of the tile
@@ -1228,28 +1135,104 @@ dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_before();
       mbar_arrive_warp(&bars[P_PFULL + wg]);
     }
-    ok = ok && mbar_wait_warp(&bars[P_DONE], 0);
+    // ---- the memory update's backward ----
+    // every MMA of the loop is done (K may be overwritten); z_{s-1} is needed for Delta
+    ok = ok && mbar_wait_warp(&bars[P_DONE], 0) && (!delta || mbar_wait_warp(&bars[P_X], 0));
+    float denp = 0.f;
+    if (ok) {
+#pragma unroll
+      for (int u = 8 * wg; u < 8 * wg + 8; ++u) {
+        float f[8];
+        unpack8(ld_unit(sK, r, u), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          f[e] = sig(f[e]);
+          if (delta) denp = fmaf(f[e], sZ[8 * u + e], denp);
+        }
+        st_unit(sK, r, u, f);
+      }
+    }
+    fence_proxy_async_smem();
+    xs[wg * D + r] = denp;
+    named_bar_sync(1, 256);
+    const float denK = xs[r] + xs[D + r];
+    tc_fence_before();
+    mbar_arrive_warp(&bars[P_SK]);
+    const size_t rowk = (size_t)bh * p.L + krow + r;
+    float ddenR = 0.f;
+    if (delta) {
+      ok = ok && mbar_wait_warp(&bars[P_M1], 0);
+      float ddp = 0.f;
+      if (ok) {
+        tc_fence_after();
+        const float inv = denK != 0.f ? 1.f / denK : 0.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t rn[32], du[32];
+          tmem_ld32(tmem + lane_off + 64 * wg + 32 * c, rn);
+          tmem_ld32(tmem + 128 + lane_off + 64 * wg + 32 * c, du);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u4 = 0; u4 < 4; ++u4) {
+            const int u = 8 * wg + 4 * c + u4;
+            float vv[8], uu[8], dn[8];
+            unpack8(ld_unit(sV, r, u), vv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float rr = __uint_as_float(rn[8 * u4 + e]) * inv;
+              const float dU = __uint_as_float(du[8 * u4 + e]);
+              uu[e] = vv[e] - rr;
+              dn[e] = -dU * inv;
+              ddp = fmaf(dU, rr, ddp);
+            }
+            st_unit(sV, r, u, uu);   // U over V (this row's V is read)
+            st_unit(sDN, r, u, dn);
+          }
+        }
+        ddp *= inv;
+      }
+      fence_proxy_async_smem();
+      xs[wg * D + r] = ddp;
+      named_bar_sync(1, 256);
+      ddenR = xs[r] + xs[D + r];
+      if (wg == 0) sDD[r] = ddenR;
+      tc_fence_before();
+      mbar_arrive_warp(&bars[P_SK2]);
+      named_bar_sync(1, 256);
+      {  // sigma(K)^T ddenR over this tile's rows: column r, rows [64 wg, 64 wg + 64)
+        float acc = 0.f;
+        for (int rr = 64 * wg; rr < 64 * wg + 64; ++rr) acc = fmaf(ld_elem(sK, rr, r), sDD[rr], acc);
+        gzp[wg * D + r] = acc;
+      }
+      named_bar_sync(1, 256);
+      if (wg == 0 && ok) gzk[(((size_t)bh * p.S + s) * p.T + j) * D + r] = gzp[r] + gzp[D + r];
+      ok = ok && mbar_wait_warp(&bars[P_M2], 0);
+    } else {
+      ok = ok && mbar_wait_warp(&bars[P_M1], 0);
+    }
     if (ok) {
       tc_fence_after();
-      const size_t rowk = (size_t)bh * p.L + krow + r;
       const float* dz = dzs + ((size_t)bh * p.S + s) * D;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t a[32], bb[32];
+        uint32_t a[32], bb[32], xk[32];
         const uint32_t col = 64 * wg + 32 * c;
         tmem_ld32(tV + lane_off + col, a);
         tmem_ld32(tK + lane_off + col, bb);
+        tmem_ld32(tmem + lane_off + col, xk);
         tmem_wait_ld();
 #pragma unroll
         for (int u4 = 0; u4 < 4; ++u4) {
           const int u = (int)(col >> 3) + u4;
-          float kf[8], ov[8], ok8[8];
-          unpack8(ld_unit(sK, r, u), kf);
+          float sk[8], ov[8], ok8[8];
+          unpack8(ld_unit(sK, r, u), sk);  // sigma(K), bf16
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int f = 8 * u + e;
-            ov[e] = __uint_as_float(a[8 * u4 + e]) + dv_mem[rowk * D + f];
-            ok8[e] = __uint_as_float(bb[8 * u4 + e]) + (dk_mem[rowk * D + f] + dz[f]) * dsig(kf[e]);
+            float dsk = __uint_as_float(xk[8 * u4 + e]);
+            dsk = delta ? fmaf(ddenR, sZ[f], dsk) : dsk + dz[f];
+            ov[e] = __uint_as_float(a[8 * u4 + e]);
+            ok8[e] = fmaf(dsk, fminf(sk[e], 1.f), __uint_as_float(bb[8 * u4 + e]));  // sigma' = min(sigma, 1)
           }
           *reinterpret_cast<uint4*>(dv + rowk * D + 8 * u) =
               make_uint4(pack_bf16x2(ov[0], ov[1]), pack_bf16x2(ov[2], ov[3]),
@@ -1266,6 +1249,29 @@ dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// Delta: dk += dz_s * sigma'(K), once every segment's z gradient is known.
+// grid-stride over the [BH][L][128] elements in units of 8.
+__global__ void __launch_bounds__(256)
+dk_dz_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict__ dzs,
+             __nv_bfloat16* __restrict__ dk, long long L, int N, int S, long long units) {
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < units;
+       u += (long long)gridDim.x * blockDim.x) {
+    const long long row = u >> 4;  // 16 units of 8 per row
+    const int f0 = (int)(u & 15) * 8;
+    const long long bh = row / L;
+    const int s = (int)((row - bh * L) / N);
+    const float* dz = dzs + ((size_t)bh * S + s) * D + f0;
+    float kf[8], df[8];
+    unpack8(*reinterpret_cast<const uint4*>(k + u * 8), kf);
+    unpack8(*reinterpret_cast<const uint4*>(dk + u * 8), df);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) df[e] = fmaf(dz[e], dsig(kf[e]), df[e]);
+    *reinterpret_cast<uint4*>(dk + u * 8) =
+        make_uint4(pack_bf16x2(df[0], df[1]), pack_bf16x2(df[2], df[3]),
+                   pack_bf16x2(df[4], df[5]), pack_bf16x2(df[6], df[7]));
   }
 }
 
@@ -1298,9 +1304,6 @@ cudaError_t bf16_bwd_set_attributes() {
     e = cudaFuncSetAttribute(chain_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kChainSmem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kside_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kKsideSmem);
-  if (e == cudaSuccess)
     e = cudaFuncSetAttribute(dq_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(dkdv_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1308,11 +1311,11 @@ cudaError_t bf16_bwd_set_attributes() {
   return e;
 }
 
-// Backward scratch after the state path's: per-row statistics, the memory path's
-// fp32 contributions to dq / dk / dv, the per-segment gradients of the state.
+// Backward scratch after the state path's: per-row statistics, the retrieval's fp32
+// contribution to dq, the per-segment gradients of the state.
 size_t bf16_bwd_workspace_bytes(int BH, long long L, int S, int T, int CH) {
   const size_t bh = (size_t)BH, rows = bh * (size_t)L, bhs = bh * S;
-  return up256(bf16_workspace_bytes(BH, S, CH)) + 2 * up256(rows * 4) + 3 * up256(rows * D * 4) +
+  return up256(bf16_workspace_bytes(BH, S, CH)) + 2 * up256(rows * 4) + up256(rows * D * 4) +
          up256(bhs * D * D * 4) + up256(bhs * D * 4) + up256(bhs * 2 * D * D * 2) +
          up256(bhs * D * 4) + up256(bhs * T * D * 4) + up256(bhs * 4) + up256(bhs * T * 4);
 }
@@ -1341,8 +1344,6 @@ cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   float* lse2 = reinterpret_cast<float*>(take(rows * 4));
   float* dpr = reinterpret_cast<float*>(take(rows * 4));
   float* dq_mem = reinterpret_cast<float*>(take(rows * D * 4));
-  float* dk_mem = reinterpret_cast<float*>(take(rows * D * 4));
-  float* dv_mem = reinterpret_cast<float*>(take(rows * D * 4));
   float* GM = reinterpret_cast<float*>(take(bhs * D * D * 4));
   float* Gz = reinterpret_cast<float*>(take(bhs * D * 4));
   __nv_bfloat16* dMs = reinterpret_cast<__nv_bfloat16*>(take(bhs * 2 * D * D * 2));
@@ -1398,16 +1399,20 @@ cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                                                                   dq_mem, GM, Gz, mem_part, p);
   chain_bwd_kernel<<<dim3(BH, 4), kChainThreads, kChainSmem, stream>>>(mg, GM, dM_out, dM_in, dMs,
                                                                         S, CH, mode);
-  kside_bwd_kernel<<<p.tiles, kThreads, kKsideSmem, stream>>>(mk, mv, mm, mx, ws.zprev, dk_mem,
-                                                               dv_mem, gzk, p, mode);
-  dz_bwd_kernel<<<BH, D, 0, stream>>>(Gz, gzk, dz_out, dzs, dz_in, S, T, mode);
+  if (mode == 0) dz_bwd_kernel<<<BH, D, 0, stream>>>(Gz, gzk, dz_out, dzs, dz_in, S, T, mode);
   mark(0);
   dq_bwd_kernel<<<p.tiles, kPipeThreads, kDqSmem, stream>>>(mq, mk, mv, mdo, beta, dq_mem, lse2, dpr,
                                                          dot_part, dq, p);
   mark(1);
-  dkdv_bwd_kernel<<<p.tiles, kPipeThreads, kDkdvSmem, stream>>>(mq, mk, mv, mdo, beta, lse2, dpr,
-                                                             dk_mem, dv_mem, dzs, dk, dv, p);
+  dkdv_bwd_kernel<<<p.tiles, kPipeThreads, kDkdvSmem, stream>>>(
+      mq, mk, mv, mdo, mm, mx, beta, ws.zprev, lse2, dpr, dzs, gzk, dk, dv, p, mode);
   mark(2);
+  if (mode == 1) {
+    dz_bwd_kernel<<<BH, D, 0, stream>>>(Gz, gzk, dz_out, dzs, dz_in, S, T, mode);
+    const long long units = (long long)rows * (D / 8);
+    const unsigned grid = (unsigned)min((units + 255) / 256, 148LL * 16);
+    dk_dz_kernel<<<grid, 256, 0, stream>>>(k, dzs, dk, L, N, S, units);
+  }
   dbeta_bwd_kernel<<<1, 128, 0, stream>>>(beta, mem_part, dot_part, dbeta, B, H, S, T);
   return cudaGetLastError();
 }
