@@ -797,24 +797,33 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive_warp(&bars[P_PFULL + wg]);  // the buffer may take the next half
-      float mx = -INFINITY;
+      float* sf = reinterpret_cast<float*>(sv);
+      if (diag) {  // keys after the row do not count
 #pragma unroll
-      for (int c = 0; c < 64; ++c)
-        if (!(diag && 64 * wg + c > r)) mx = fmaxf(mx, __uint_as_float(sv[c]));
+        for (int c = 0; c < 64; ++c)
+          if (64 * wg + c > r) sf[c] = -INFINITY;
+      }
+      float mx8[8];
+#pragma unroll
+      for (int q8 = 0; q8 < 8; ++q8)
+        mx8[q8] = fmaxf(fmax3(sf[q8], sf[8 + q8], sf[16 + q8]),
+                        fmax3(sf[24 + q8], sf[32 + q8], fmax3(sf[40 + q8], sf[48 + q8], sf[56 + q8])));
+      const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                             fmaxf(fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       if (mx == -INFINITY) continue;  // every key of this half is after the row
       const float mn = fmaxf(m, mx);
       const float alpha = ex2_approx((m - mn) * sl);  // 0 while m = -inf
-      l *= alpha;
-      dacc *= alpha;
-      m = mn;
-      const float mb = m * sl;
+      const float mb = mn * sl;
+      float la[4] = {0.f, 0.f, 0.f, 0.f}, da[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const bool masked = diag && 64 * wg + c > r;
-        const float pe = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[c]), sl, -mb));
-        l += pe;
-        dacc = fmaf(pe, __uint_as_float(pv[c]), dacc);
+        const float pe = ex2_approx(fmaf(sf[c], sl, -mb));  // 0 where masked (-inf)
+        la[c & 3] += pe;
+        da[c & 3] = fmaf(pe, __uint_as_float(pv[c]), da[c & 3]);
       }
+      l = fmaf(l, alpha, (la[0] + la[1]) + (la[2] + la[3]));
+      dacc = fmaf(dacc, alpha, (da[0] + da[1]) + (da[2] + da[3]));
+      m = mn;
     }
     // merge the two warpgroups' running statistics of row r
     if (ok) {
@@ -839,28 +848,27 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         break;
       }
       tc_fence_after();
-      const bool diag = n == nl - 1;
+      uint32_t sv[64], pv[64], pk[32];
+      tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(sv));
+      tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+      tmem_ld32(tb + 64, *reinterpret_cast<uint32_t(*)[32]>(pv));
+      tmem_ld32(tb + 96, *reinterpret_cast<uint32_t(*)[32]>(pv + 32));
+      tmem_wait_ld();
+      float* sf = reinterpret_cast<float*>(sv);
+      if (n == nl - 1) {  // the diagonal tile: keys after the row get P = 0
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        uint32_t sv[32], pv[32], pk[16];
-        tmem_ld32(tb + 32 * c2, sv);
-        tmem_ld32(tb + 64 + 32 * c2, pv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float ds[2];
-#pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            const int c = 32 * c2 + 2 * e + w;
-            const bool masked = diag && 64 * wg + c > r;
-            const float pe = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[2 * e + w]), sl, -lse2));
-            ds[w] = cds * pe * (__uint_as_float(pv[2 * e + w]) - dpv);
-          }
-          pk[e] = pack_bf16x2(ds[0], ds[1]);
-        }
-        // columns [16 c2, 16 c2 + 16): scores this thread has already read
-        tmem_st16(tb + 16 * c2, pk);
+        for (int c = 0; c < 64; ++c)
+          if (64 * wg + c > r) sf[c] = -INFINITY;
       }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float p0 = ex2_approx(fmaf(sf[2 * e], sl, -lse2));
+        const float p1 = ex2_approx(fmaf(sf[2 * e + 1], sl, -lse2));
+        pk[e] = pack_bf16x2(cds * p0 * (__uint_as_float(pv[2 * e]) - dpv),
+                            cds * p1 * (__uint_as_float(pv[2 * e + 1]) - dpv));
+      }
+      // dS over the first 32 columns of the buffer: scores this thread has read
+      tmem_st32_(tb, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(&bars[P_PFULL + wg]);
@@ -1105,32 +1113,33 @@ dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         break;
       }
       tc_fence_after();
-      const bool diag = n == 0;
       const float* ls = sLD + st * 2 * D + 64 * wg;
       const float* dps = ls + D;
+      uint32_t sv[64], pv[64], pk1[32], pk2[32];
+      tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(sv));
+      tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+      tmem_ld32(tb + 64, *reinterpret_cast<uint32_t(*)[32]>(pv));
+      tmem_ld32(tb + 96, *reinterpret_cast<uint32_t(*)[32]>(pv + 32));
+      tmem_wait_ld();
+      float* sf = reinterpret_cast<float*>(sv);
+      if (n == 0) {  // the diagonal tile: queries before key r get P = 0
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        uint32_t sv[32], pv[32], pk1[16], pk2[16];
-        tmem_ld32(tb + 32 * c2, sv);
-        tmem_ld32(tb + 64 + 32 * c2, pv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float pg[2], ds[2];
-#pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            const int c = 32 * c2 + 2 * e + w;  // query 64 wg + c of the tile
-            const bool masked = diag && 64 * wg + c < r;
-            const float pe = masked ? 0.f : ex2_approx(fmaf(__uint_as_float(sv[2 * e + w]), sl, -ls[c]));
-            pg[w] = cp * pe;
-            ds[w] = cds * pe * (__uint_as_float(pv[2 * e + w]) - dps[c]);
-          }
-          pk1[e] = pack_bf16x2(pg[0], pg[1]);
-          pk2[e] = pack_bf16x2(ds[0], ds[1]);
-        }
-        tmem_st16(tb + 16 * c2, pk1);
-        tmem_st16(tb + 64 + 16 * c2, pk2);
+        for (int c = 0; c < 64; ++c)
+          if (64 * wg + c < r) sf[c] = -INFINITY;
       }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float2 lq = *reinterpret_cast<const float2*>(ls + 2 * e);
+        const float2 dq2 = *reinterpret_cast<const float2*>(dps + 2 * e);
+        const float p0 = ex2_approx(fmaf(sf[2 * e], sl, -lq.x));
+        const float p1 = ex2_approx(fmaf(sf[2 * e + 1], sl, -lq.y));
+        pk1[e] = pack_bf16x2(cp * p0, cp * p1);
+        pk2[e] = pack_bf16x2(cds * p0 * (__uint_as_float(pv[2 * e]) - dq2.x),
+                             cds * p1 * (__uint_as_float(pv[2 * e + 1]) - dq2.y));
+      }
+      // P^T and dS^T over the first 32 columns of the scores and of dP'^T (read)
+      tmem_st32_(tb, pk1);
+      tmem_st32_(tb + 64, pk2);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(&bars[P_PFULL + wg]);
