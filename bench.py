@@ -600,7 +600,9 @@ def run_extra(args, device):
             torch.cuda.synchronize()
             it[0] = 0
             ms = _timed(f, 3, stream)
-            # per stage, averaged over the three timed calls: memory path, dq, dk/dv
+            # per stage, averaged over the three timed calls: state rebuild, dq (with the
+            # retrieval's backward), dk/dv (with the reverse state chain and the update's
+            # backward)
             st_ms = [sum(e[k].elapsed_time(e[k + 1]) for e in evs) / 3 for k in range(3)]
             pairs = Bc * Hc * (Lc // Nc) * (Nc // 128) * (Nc // 128 + 1) // 2  # tile pairs
             att = pairs * 2 * 128 * 128 * D  # one 128 x 128 x 128 product over every pair
@@ -615,8 +617,8 @@ def run_extra(args, device):
             res[name] = {"ms_per_call": ms, "tokens_per_s": Bc * Lc / (ms / 1e3),
                          "algorithmic_tflops": tf, "frac_of_sustained_bf16": tf / peak_sust,
                          "frac_of_burst_bf16": tf / peak_burst,
-                         "stage_ms": {"memory_path": st_ms[0], "dq_kernel": st_ms[1],
-                                      "dkdv_kernel": st_ms[2]},
+                         "stage_ms": {"state_rebuild": st_ms[0], "dq_kernel": st_ms[1],
+                                      "chain_and_dkdv_kernel": st_ms[2]},
                          # executed tile products: dq 5 per tile pair (S, dP' twice, dQ),
                          # dk/dv 4 (S^T, dP'^T, dV, dK)
                          "dq_kernel_executed_tflops": 5 * att / (st_ms[1] / 1e3) / 1e12,
@@ -626,9 +628,11 @@ def run_extra(args, device):
         lines.append({"config": "backward: B=4, H=8, d=128, N=2048, L=32768, bf16, "
                                 "infini_attn_backward (loss through out)",
                       **res, "peak_source": src,
-                      "note": "one call: the state path rebuilt, then the seven backward "
-                              "kernels; executed tensor work is about 2.3x the algorithmic "
-                              "count (S and dP' are recomputed in both attention kernels)"})
+                      "note": "one call: the state path rebuilt, then the dq kernel, the "
+                              "reverse state chain, the dk/dv kernel (Delta: the z-gradient "
+                              "scan and the dk fix-up) and the dbeta sum; executed tensor "
+                              "work is about 2.3x the algorithmic count (S and dP' are "
+                              "recomputed in both attention kernels)"})
     return lines
 
 

@@ -269,7 +269,8 @@ def infini_attn_backward(q, k, v, beta, N, mode, dout, M_in=None, z_in=None, dM_
     z_out). Returns (dq, dk, dv, dbeta, dM_in, dz_in); dM_in, dz_in are None when
     state_grad is False. workspace: optional uint8 CUDA tensor of at least
     backward_workspace_size(...) bytes; stage_events: up to three torch.cuda.Event
-    recorded after the memory path, the dq kernel and the dk/dv kernel."""
+    recorded after the state rebuild, after the dq kernel (with the retrieval's
+    backward) and after the dk/dv kernel (with the reverse state chain)."""
     B, H, L, d, _, _, _ = _prepare(q, k, v, beta, M_in, z_in, None, None, None, False)
     if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_cuda or not dout.is_contiguous():
         raise ValueError("dout must be a contiguous CUDA tensor shaped and typed like q")

@@ -25,14 +25,13 @@
 //
 // Kernels, in launch order (after the forward's state path has rebuilt M_{s-1} as
 // bf16 hi/lo, z_{s-1} and, for Delta, every segment's G_s):
-//   retr   (head, segment): retrieval backward over the segment's query tiles ->
-//          dq_mem (fp32), GM_s, Gz_s, the segment's sum of dout * A_mem.
-//   chain  (head, 32-column block): dM_s for s = S-1 .. 0 (bf16 hi/lo stack), dM_in.
-//   dz     (head, Linear): dz_s for every segment, dz_in.
 //   dq     (head, segment, query tile): two sweeps over the key tiles; the first
 //          gives each row's log-sum-exp and D' = dout . A_dot, the second
-//          dQ = sum_j dS_j K_j; adds dq_mem, writes dq, the row statistics and the
-//          tile's sum of D' (for dbeta).
+//          dQ = sum_j dS_j K_j; then the retrieval's backward of its query rows
+//          (dsigma(Q), and the tile's partials of GM_s and Gz_s); writes dq, the row
+//          statistics and the tile's sums for dbeta.
+//   chain  (head, 32-column block): dM_s for s = S-1 .. 0 (bf16 hi/lo stack), dM_in.
+//   dz     (head, Linear): dz_s for every segment, dz_in.
 //   dkdv   (head, segment, key tile): over the query tiles at or after it,
 //          dV = sum_i (1-g) P_i^T dout_i and dK = sum_i dS_i^T Q_i from S^T = K Q^T
 //          and dP'^T = V dout^T; then the memory update's backward of its key rows
@@ -40,12 +39,12 @@
 //          writes dk, dv.
 //   dz, dk_dz (Delta): dz_s for every segment (it needs every tile's sigma(K)^T
 //          ddenR), dz_in, then dk += dz_s * sigma'(K).
-//   dbeta  : per head, summed over batch rows and segments in a fixed order.
-// Every product is a 128 x 128 x 128 bf16 tcgen05 MMA (fp32 accumulation in tensor
-// memory) on 128B-swizzled shared-memory tiles, in the operand forms the forward
-// uses: A, B both K-major (Q K^T), A in tensor memory with B MN-major (P V), and
-// A, B both MN-major (sigma(K)^T V); the Delta chain uses the forward chain's tf32
-// form. Thread r of a 128-thread group owns tile row r (tensor-memory lane r).
+//   dbeta  : per head, summed over batch rows, segments and tiles in a fixed order.
+// Every product is a bf16 tcgen05 MMA (fp32 accumulation in tensor memory) on
+// 128B-swizzled shared-memory tiles, in the operand forms the forward uses: A, B
+// both K-major (Q K^T), A in tensor memory with B MN-major (P V), and A, B both
+// MN-major (sigma(K)^T V); the Delta chain uses the forward chain's tf32 form.
+// Thread r of a 128-thread warpgroup owns tile row r (tensor-memory lane r).
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda.h>
@@ -62,7 +61,6 @@ namespace {
 constexpr int D = 128;
 constexpr int kTile = 32768;  // 128 x 128 bf16
 constexpr int kSub = 16384;   // one 128 x 64 box (128-byte rows)
-constexpr int kThreads = 128;
 
 // ---------------------------------------------------------------------------
 // tiles, descriptors, products
@@ -123,21 +121,6 @@ __device__ __forceinline__ void gemm_km(uint32_t d, const uint8_t* a, const uint
   for (int kk = 0; kk < D / 16; ++kk)
     mma_bf16_ss(d, kdesc(sa, kk), mdesc(sx, kk), kIdKM, (acc || kk > 0) ? 1u : 0u);
 }
-// D (+)= X^T Y: X[k][m] and Y[k][n] are tiles (the contraction runs over tile rows)
-__device__ __forceinline__ void gemm_mm(uint32_t d, const uint8_t* x, const uint8_t* y, bool acc) {
-  const uint32_t sx = smem_u32(x), sy = smem_u32(y);
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk)
-    mma_bf16_ss(d, mdesc(sx, kk), mdesc(sy, kk), kIdMM, (acc || kk > 0) ? 1u : 0u);
-}
-// D (+)= A X: A[m][k] in tensor memory (bf16 pairs, 64 columns from ta), X[k][n] a tile
-__device__ __forceinline__ void gemm_tm(uint32_t d, uint32_t ta, const uint8_t* x, bool acc) {
-  const uint32_t sx = smem_u32(x);
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk)
-    mma_bf16_ts(d, ta + 8 * kk, mdesc(sx, kk), kIdKM, (acc || kk > 0) ? 1u : 0u);
-}
-
 // Both boxes of a 128-row tile of a [B, H, L, 128] tensor.
 __device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* m, uint64_t* bar, int row,
                                           int h, int b) {
@@ -151,13 +134,6 @@ __device__ __forceinline__ void load_plane(uint8_t* dst, const CUtensorMap* m, u
   tma_load_3d(dst + kSub, m, bar, 64, 0, plane);
 }
 
-// A wait by all 128 threads whose outcome is the same in every thread (and a CTA
-// barrier): a wait that gave up anywhere makes every thread leave its loop.
-__device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity) {
-  const bool w = mbar_wait(bar, parity);
-  return __syncthreads_and(w ? 1 : 0) != 0;
-}
-
 // Bounded wait used only while draining after an error.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
@@ -165,35 +141,6 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   while (!mbar_try_wait(a, parity)) {
     if (globaltimer_ns() - t0 > 200000000ull) break;  // 200 ms
   }
-}
-
-// Issues the product(s) from one elected lane of warp 0, then commits to bar.
-#define ISSUE_MMA(bar, ...)                 \
-  do {                                      \
-    if (warp == 0) {                        \
-      tc_fence_after();                     \
-      if (elect_one()) {                    \
-        __VA_ARGS__;                        \
-        mma_commit(bar);                    \
-      }                                     \
-      __syncwarp();                         \
-    }                                       \
-  } while (0)
-
-// Threads' shared- and tensor-memory writes -> visible to the tensor cores.
-__device__ __forceinline__ void publish_writes() {
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-}
-
-__device__ __forceinline__ float block_sum(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  return (red[0] + red[1]) + (red[2] + red[3]);
 }
 
 struct BwdParams {
@@ -215,186 +162,11 @@ __device__ __forceinline__ void decode3(const BwdParams& p, unsigned u, int& bh,
 }
 
 // ---------------------------------------------------------------------------
-// retr: grid = BH * S, one CTA per (head, segment), looping over its query tiles.
-// Tensor memory: num = sigma(Q) M | dsigma(Q) = dnum M^T | GM (accumulated).
-// ---------------------------------------------------------------------------
-constexpr int kRetrSmem = 5 * kTile + 1024 + 64 + 256 + 1024;
-
-__global__ void __launch_bounds__(kThreads, 1)
-retr_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                const __grid_constant__ CUtensorMap tm_m, const float* __restrict__ beta,
-                const float* __restrict__ zprev, float* __restrict__ dq_mem,
-                float* __restrict__ GM, float* __restrict__ Gz, float* __restrict__ mem_part,
-                const BwdParams p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint8_t* sM = smem;
-  uint8_t* sQ = smem + kTile;
-  uint8_t* sDO = smem + 2 * kTile;
-  uint8_t* sSQ = smem + 3 * kTile;  // sigma(Q), bf16
-  uint8_t* sDN = smem + 4 * kTile;  // dnum, bf16
-  float* sZ = reinterpret_cast<float*>(smem + 5 * kTile);
-  float* sDD = sZ + D;              // dden per row
-  float* red = sDD + D;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 16);  // 0 M/z, 1 Q/dout, 2 MMA, 3 drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
-
-  const int seg = blockIdx.x;
-  const int bh = (int)p.divS.div((unsigned)seg), s = seg - bh * p.S;
-  const int b = bh / p.H, h = bh - b * p.H;
-  const int tid = threadIdx.x, warp = tid >> 5, r = tid;
-  if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
-    fence_barrier_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot, tN = tmem, tD = tmem + 128, tG = tmem + 256;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  int q_iss = 0, q_cons = 0;
-  bool m_pending = true;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], kTile + D * 4);
-    load_plane(sM, &tm_m, &bars[0], (bh * p.S + s) * 2);
-    bulk_load(sZ, zprev + ((size_t)bh * p.S + s) * D, D * 4, &bars[0]);
-  }
-  const float g = 1.f / (1.f + expf(-beta[h]));
-  float gz = 0.f, memt = 0.f;
-  uint32_t mph = 0;
-  bool ok = cta_wait(&bars[0], 0);
-  if (ok) m_pending = false;
-  for (int i = 0; ok && i < p.T; ++i) {
-    const int row = s * p.N + i * 128;
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&bars[1], 2 * kTile);
-      load_rows(sQ, &tm_q, &bars[1], row, h, b);
-      load_rows(sDO, &tm_do, &bars[1], row, h, b);
-    }
-    ++q_iss;
-    ok = cta_wait(&bars[1], (uint32_t)(i & 1));
-    if (!ok) break;
-    ++q_cons;
-    // sigma(Q) row r (bf16 operand) and its denominator in fp32
-    float den = 0.f;
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      float f[8];
-      unpack8(ld_unit(sQ, r, u), f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        f[e] = sig(f[e]);
-        den = fmaf(f[e], sZ[8 * u + e], den);
-      }
-      st_unit(sSQ, r, u, f);
-    }
-    publish_writes();
-    ISSUE_MMA(&bars[2], gemm_km(tN, sSQ, sM, false));
-    ok = cta_wait(&bars[2], mph & 1);
-    ++mph;
-    if (!ok) break;
-    tc_fence_after();
-    const float inv = den != 0.f ? 1.f / den : 0.f;
-    float dd = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t nv[32];
-      tmem_ld32(tN + lane_off + 32 * c, nv);
-      tmem_wait_ld();
-#pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4) {
-        const int u = 4 * c + u4;
-        float o[8], dn[8];
-        unpack8(ld_unit(sDO, r, u), o);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float a = __uint_as_float(nv[8 * u4 + e]) * inv;  // A_mem
-          const float da = g * o[e];
-          dn[e] = da * inv;
-          dd = fmaf(da, a, dd);
-          memt = fmaf(o[e], a, memt);
-        }
-        st_unit(sDN, r, u, dn);
-      }
-    }
-    const float dden = -dd * inv;
-    sDD[r] = dden;
-    publish_writes();
-    ISSUE_MMA(&bars[2], gemm_kk(tD, sDN, sM, false); gemm_mm(tG, sSQ, sDN, i > 0));
-    // Gz: column r of sigma(Q)^T dden, from the exact sigma of the bf16 inputs
-    {
-      float acc = 0.f;
-      for (int rr = 0; rr < 128; ++rr) acc = fmaf(sig(ld_elem(sQ, rr, r)), sDD[rr], acc);
-      gz += acc;
-    }
-    ok = cta_wait(&bars[2], mph & 1);
-    ++mph;
-    if (!ok) break;
-    tc_fence_after();
-    float* dst = dq_mem + ((size_t)bh * p.L + row + r) * D;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t dv[32];
-      tmem_ld32(tD + lane_off + 32 * c, dv);
-      tmem_wait_ld();
-#pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4) {
-        const int u = 4 * c + u4;
-        float qf[8], o[8];
-        unpack8(ld_unit(sQ, r, u), qf);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          o[e] = fmaf(dden, sZ[8 * u + e], __uint_as_float(dv[8 * u4 + e])) * dsig(qf[e]);
-        *reinterpret_cast<float4*>(dst + 8 * u) = make_float4(o[0], o[1], o[2], o[3]);
-        *reinterpret_cast<float4*>(dst + 8 * u + 4) = make_float4(o[4], o[5], o[6], o[7]);
-      }
-    }
-    tc_fence_before();
-    __syncthreads();  // Q, dout and tensor-memory reads done before the next tile
-  }
-  if (ok) {
-    float* gm = GM + (((size_t)bh * p.S + s) * D + r) * D;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t v[32];
-      tmem_ld32(tG + lane_off + 32 * c, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(gm + 32 * c + e) =
-            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-    }
-    Gz[((size_t)bh * p.S + s) * D + r] = gz;
-    const float tot = block_sum(memt, red);
-    if (tid == 0) mem_part[(size_t)bh * p.S + s] = tot;
-  } else if (tid == 0) {
-    if (m_pending) drain_wait(&bars[0], 0);
-    if (q_iss > q_cons) drain_wait(&bars[1], (uint32_t)((q_iss - 1) & 1));
-  }
-  if (!ok && warp == 0) {
-    if (elect_one()) mma_commit(&bars[3]);
-    __syncwarp();
-    drain_wait(&bars[3], 0);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
-// ---------------------------------------------------------------------------
 // chain: grid = (BH, 4), block 160. Column block cb covers dM[:, 32cb .. 32cb+31];
 // threads 0..127 own one row (32 fp32 values); warp 4 issues the copies of G and the
 // tf32 products (Delta). For s = S-1 .. 0: write X = dM_s as bf16 hi/lo into the
-// stack, then X += GM_s (Linear) or X += GM_s - G_s X (Delta); finally dM_in = X.
+// stack, then X += GM_s (Linear) or X += GM_s - G_s X (Delta), GM_s being the sum of
+// the segment's per-query-tile partials; finally dM_in = X.
 // ---------------------------------------------------------------------------
 constexpr int kChainThreads = 160;
 constexpr int kGBytes = D * D * 4;    // 64 KB
@@ -408,9 +180,9 @@ __device__ __forceinline__ uint32_t tf32_rna(float x) {
 }
 
 __global__ void __launch_bounds__(kChainThreads, 1)
-chain_bwd_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__ GM,
+chain_bwd_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__ GMp,
                  const float* dM_out, float* dM_in, __nv_bfloat16* __restrict__ dMs, int S,
-                 int CH, int mode) {
+                 int CH, int T, int mode) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -539,12 +311,17 @@ chain_bwd_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restri
           *reinterpret_cast<uint4*>(lo + e) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
         }
       }
+      // GM_s: the segment's query tiles' partials, added in tile order
       float gm[32];
-      const float* src = GM + (((size_t)bh * S + s) * D + r) * D + c0;
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const float4 t = __ldg(reinterpret_cast<const float4*>(src + e));
-        gm[e] = t.x; gm[e + 1] = t.y; gm[e + 2] = t.z; gm[e + 3] = t.w;
+      for (int e = 0; e < 32; ++e) gm[e] = 0.f;
+      for (int t = 0; t < T; ++t) {
+        const float* src = GMp + ((((size_t)bh * S + s) * T + t) * D + r) * D + c0;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 v4 = __ldg(reinterpret_cast<const float4*>(src + e));
+          gm[e] += v4.x; gm[e + 1] += v4.y; gm[e + 2] += v4.z; gm[e + 3] += v4.w;
+        }
       }
       if (delta) {
         // X^T block (tf32) -> shared memory: row c, K-major, 4 boxes of 32 k
@@ -591,14 +368,13 @@ chain_bwd_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restri
 // dz: grid = BH, block 128 (feature t). dz_s for s = S-1 .. 0, then dz_in.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(D)
-dz_bwd_kernel(const float* __restrict__ Gz, const float* __restrict__ gzk, const float* dz_out,
+dz_bwd_kernel(const float* __restrict__ Gzp, const float* __restrict__ gzk, const float* dz_out,
               float* __restrict__ dzs, float* dz_in, int S, int T, int mode) {
   const int bh = blockIdx.x, t = threadIdx.x;
   float x = dz_out ? dz_out[(size_t)bh * D + t] : 0.f;
   for (int s = S - 1; s >= 0; --s) {
-    const size_t i = ((size_t)bh * S + s) * D + t;
-    dzs[i] = x;
-    x += Gz[i];
+    dzs[((size_t)bh * S + s) * D + t] = x;
+    for (int jj = 0; jj < T; ++jj) x += Gzp[(((size_t)bh * S + s) * T + jj) * D + t];
     if (mode == 1)
       for (int jj = 0; jj < T; ++jj) x += gzk[(((size_t)bh * S + s) * T + jj) * D + t];
   }
@@ -621,17 +397,6 @@ dz_bwd_kernel(const float* __restrict__ Gz, const float* __restrict__ gzk, const
 // ---------------------------------------------------------------------------
 constexpr int kPipeThreads = 320;
 constexpr uint32_t kIdN64 = idesc_f32acc(1, 0, 0, 128, 64);
-
-// 32 lanes x 16 columns store (bf16 pairs of 32 values per thread)
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
 
 // D = A B^T with N = 64: A[m][k] a full tile, B the 64 rows starting at row 64 a of
 // a tile (both K-major, K = 128)
@@ -662,9 +427,17 @@ enum {
   P_COUNT = 10
 };
 
+// the epilogue's steps: memory-path tiles loaded, operand written by the softmax
+// warps (8 warp arrivals), products done
+enum { P_X = P_COUNT, P_SK, P_M1, P_SK2, P_M2, P_COUNT2 };
+
 __device__ __forceinline__ void pipe_init(uint64_t* bars) {
-  for (int x = 0; x < P_COUNT; ++x)
-    mbar_init(&bars[x], (x == P_PFULL || x == P_PFULL + 1) ? 4u : 1u);
+  for (int x = 0; x < P_COUNT2; ++x) {
+    uint32_t c = 1;
+    if (x == P_PFULL || x == P_PFULL + 1) c = 4;
+    if (x == P_SK || x == P_SK2) c = 8;
+    mbar_init(&bars[x], c);
+  }
   fence_barrier_init();
 }
 
@@ -674,15 +447,24 @@ __device__ __forceinline__ void pipe_init(uint64_t* bars) {
 // gives each row's log-sum-exp and D' = dout . A_dot (a running maximum, sum and
 // dP'-weighted sum per warpgroup, merged once), the second dS and dQ = sum dS K.
 // Tensor memory: buffer 0 [0, 128), buffer 1 [128, 256), dQ [256, 384).
+// After the loop the same CTA runs the retrieval's backward for its query rows,
+// with Q and dout still in shared memory and M_{s-1} (bf16 hi) loaded into the K
+// ring stage that frees first: sigma(Q) replaces Q, num = sigma(Q) M -> buffer 0,
+// dnum = g dout / den over the other K stage, dden = -rowsum(g dout * A_mem) / den
+// as a 129th column right after it; dsigma(Q) = dnum M^T -> [384, 512) and
+// sigma(Q)^T [dnum | dden] (N = 144) -> [0, 144), the tile's GM and Gz partials.
+// dq = dQ + (dsigma(Q) + dden z) * sigma'(Q) is written once, in bf16.
 // ---------------------------------------------------------------------------
-constexpr int kDqSmem = 6 * kTile + 3 * 2 * D * 4 + 64 + 256 + 1024;
+constexpr int kDqSmem = 6 * kTile + 3 * 2 * D * 4 + 64 + D * 4 + 256 + 1024;
 
 __global__ void __launch_bounds__(kPipeThreads, 1)
 dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-              const float* __restrict__ beta, const float* __restrict__ dq_mem,
-              float* __restrict__ lse_out, float* __restrict__ dp_out,
-              float* __restrict__ dot_part, __nv_bfloat16* __restrict__ dq, const BwdParams p) {
+              const __grid_constant__ CUtensorMap tm_m, const float* __restrict__ beta,
+              const float* __restrict__ zprev, float* __restrict__ lse_out,
+              float* __restrict__ dp_out, float* __restrict__ dot_part,
+              float* __restrict__ mem_part, float* __restrict__ GMp, float* __restrict__ Gzp,
+              __nv_bfloat16* __restrict__ dq, const BwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -692,8 +474,11 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   uint8_t* sV = smem + 4 * kTile;  // 2 stages
   float* xs = reinterpret_cast<float*>(smem + 6 * kTile);  // [wg][m | l | dacc][128]
   float* red = xs + 3 * 2 * D;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 16);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_COUNT);
+  float* sZ = red + 16;                                     // z_{s-1}
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sZ + D);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_COUNT2);
+  uint8_t* sM = sK;           // M_{s-1} (hi): K stage 0, free once load nl - 2 is done
+  uint8_t* sDN = sK + kTile;  // dnum: K stage 1; dden in the next 64-column box (V stage 0)
 
   int bh, s, i;
   decode3(p, blockIdx.x, bh, s, i);
@@ -730,10 +515,20 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         load_rows(sV + st * kTile, &tm_v, &bars[P_FULL + st], s * p.N + j * 128, h, b);
         ++iss[st];
       }
+      // K stage 0 was last used by load nl - 2 (nl is even)
+      bool x_iss = false;
+      if (ok && !mbar_wait(&bars[P_FREE], (uint32_t)(((nl - 2) >> 1) & 1))) ok = false;
+      if (ok) {
+        mbar_arrive_expect_tx(&bars[P_X], kTile + D * 4);
+        load_plane(sM, &tm_m, &bars[P_X], (bh * p.S + s) * 2);
+        bulk_load(sZ, zprev + ((size_t)bh * p.S + s) * D, D * 4, &bars[P_X]);
+        x_iss = true;
+      }
       if (!ok) {
         drain_wait(&bars[P_ONCE], 0);
         for (int st = 0; st < 2; ++st)
           if (iss[st] > 0) drain_wait(&bars[P_FULL + st], (uint32_t)((iss[st] - 1) & 1));
+        if (x_iss) drain_wait(&bars[P_X], 0);
       }
     }
   } else if (warp == 9) {
@@ -772,7 +567,36 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     if (elect_one()) mma_commit(&bars[P_DONE]);
     __syncwarp();
-    if (!ok) drain_wait(&bars[P_DONE], 0);
+    // the retrieval's backward
+    ok = ok && mbar_wait_warp(&bars[P_X], 0) && mbar_wait_warp(&bars[P_SK], 0);
+    if (ok) {
+      tc_fence_after();
+      if (elect_one()) {
+        gemm_km(tmem, sQ, sM, false);  // num = sigma(Q) M
+        mma_commit(&bars[P_M1]);
+      }
+      __syncwarp();
+      ok = mbar_wait_warp(&bars[P_SK2], 0);
+    }
+    if (ok) {
+      tc_fence_after();
+      if (elect_one()) {
+        gemm_kk(tmem + 384, sDN, sM, false);  // dsigma(Q) = dnum M^T
+        // [GM | Gz] = sigma(Q)^T [dnum | dden]: both operands MN-major, N = 144
+        const uint32_t sa = smem_u32(sQ), sb = smem_u32(sDN);
+        constexpr uint32_t kIdG = idesc_f32acc(1, 1, 1, 128, 144);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tmem, mdesc(sa, kk), mdesc(sb, kk), kIdG, kk > 0 ? 1u : 0u);
+        mma_commit(&bars[P_M2]);
+      }
+      __syncwarp();
+    }
+    if (!ok) {
+      if (elect_one()) mma_commit(&bars[P_M2]);
+      __syncwarp();
+      drain_wait(&bars[P_M2], 0);
+    }
   } else {
     // ---------------- softmax warpgroups ----------------
     const int wg = warp >> 2;
@@ -873,41 +697,128 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive_warp(&bars[P_PFULL + wg]);
     }
-    ok = ok && mbar_wait_warp(&bars[P_DONE], 0);
+    // ---- the retrieval's backward (every product of the loop done: Q may change) ----
+    ok = ok && mbar_wait_warp(&bars[P_DONE], 0) && mbar_wait_warp(&bars[P_X], 0);
+    float denp = 0.f;
+    if (ok) {
+#pragma unroll
+      for (int u = 8 * wg; u < 8 * wg + 8; ++u) {
+        float f[8];
+        unpack8(ld_unit(sQ, r, u), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          f[e] = sig(f[e]);
+          denp = fmaf(f[e], sZ[8 * u + e], denp);
+        }
+        st_unit(sQ, r, u, f);  // sigma(Q) over Q
+      }
+    }
+    fence_proxy_async_smem();
+    xs[wg * D + r] = denp;
+    named_bar_sync(1, 256);
+    const float den = xs[r] + xs[D + r];
+    const float inv = den != 0.f ? 1.f / den : 0.f;
+    tc_fence_before();
+    mbar_arrive_warp(&bars[P_SK]);
+    float dd = 0.f, memt = 0.f;
+    ok = ok && mbar_wait_warp(&bars[P_M1], 0);
     if (ok) {
       tc_fence_after();
-      const size_t rowi = (size_t)bh * p.L + row0 + r;
-      const float* src = dq_mem + rowi * D + 64 * wg;
-      __nv_bfloat16* dst = dq + rowi * D + 64 * wg;
+      uint32_t nv[64];
+      tmem_ld32(tmem + lane_off + 64 * wg, *reinterpret_cast<uint32_t(*)[32]>(nv));
+      tmem_ld32(tmem + lane_off + 64 * wg + 32, *reinterpret_cast<uint32_t(*)[32]>(nv + 32));
+      tmem_wait_ld();
+#pragma unroll
+      for (int u8 = 0; u8 < 8; ++u8) {
+        const int u = 8 * wg + u8;
+        float o[8], dn[8];
+        unpack8(ld_unit(sDO, r, u), o);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float am = __uint_as_float(nv[8 * u8 + e]) * inv;  // A_mem
+          const float da = g * o[e];
+          dn[e] = da * inv;
+          dd = fmaf(da, am, dd);
+          memt = fmaf(o[e], am, memt);
+        }
+        st_unit(sDN, r, u, dn);
+      }
+    }
+    xs[wg * D + r] = dd;  // every thread has read den above (P_M1 needs all P_SK arrivals)
+    named_bar_sync(1, 256);
+    const float dden = -(xs[r] + xs[D + r]) * inv;
+    if (wg == 0)  // the 129th column of the product's right operand: (row r, column 0) of box 2
+      *reinterpret_cast<__nv_bfloat16*>(sDN + 2 * kSub + sw128((uint32_t)r, 0)) =
+          __float2bfloat16_rn(dden);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    mbar_arrive_warp(&bars[P_SK2]);
+    ok = ok && mbar_wait_warp(&bars[P_M2], 0);
+    const size_t rowi = (size_t)bh * p.L + row0 + r;
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* dst = dq + rowi * D;
+      float* gm = GMp + ((size_t)blockIdx.x * D + r) * D;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tQ + lane_off + 64 * wg + 32 * c, v);
+        const uint32_t col = 64 * wg + 32 * c;
+        uint32_t qv[32], sv[32], gv[32];
+        tmem_ld32(tQ + lane_off + col, qv);
+        tmem_ld32(tmem + 384 + lane_off + col, sv);
+        tmem_ld32(tmem + lane_off + col, gv);
         tmem_wait_ld();
 #pragma unroll
         for (int u4 = 0; u4 < 4; ++u4) {
-          const float4 x0 = *reinterpret_cast<const float4*>(src + 32 * c + 8 * u4);
-          const float4 x1 = *reinterpret_cast<const float4*>(src + 32 * c + 8 * u4 + 4);
-          const float* w = reinterpret_cast<const float*>(v) + 8 * u4;
-          *reinterpret_cast<uint4*>(dst + 32 * c + 8 * u4) = make_uint4(
-              pack_bf16x2(w[0] + x0.x, w[1] + x0.y), pack_bf16x2(w[2] + x0.z, w[3] + x0.w),
-              pack_bf16x2(w[4] + x1.x, w[5] + x1.y), pack_bf16x2(w[6] + x1.z, w[7] + x1.w));
+          const int u = (int)(col >> 3) + u4;
+          float sq[8], o[8];
+          unpack8(ld_unit(sQ, r, u), sq);  // sigma(Q), bf16
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float dsq = fmaf(dden, sZ[8 * u + e], __uint_as_float(sv[8 * u4 + e]));
+            o[e] = fmaf(dsq, fminf(sq[e], 1.f), __uint_as_float(qv[8 * u4 + e]));  // sigma' = min(sigma, 1)
+          }
+          *reinterpret_cast<uint4*>(dst + 8 * u) =
+              make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                         pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
         }
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(gm + col + e) =
+              make_float4(__uint_as_float(gv[e]), __uint_as_float(gv[e + 1]),
+                          __uint_as_float(gv[e + 2]), __uint_as_float(gv[e + 3]));
       }
       if (wg == 0) {
+        uint32_t zv[32];
+        tmem_ld32(tmem + lane_off + 128, zv);  // column 128: sigma(Q)^T dden
+        tmem_wait_ld();
+        Gzp[(size_t)blockIdx.x * D + r] = __uint_as_float(zv[0]);
         lse_out[rowi] = lse2;
         dp_out[rowi] = dpv;
       }
     }
-    // the tile's sum of D' (for dbeta); every thread of warpgroup 0 reaches the
-    // barrier, whatever its waits returned
-    if (wg == 0) {
-      float t = ok ? dpv : 0.f;
+    // the tile's sums of D' and of dout * A_mem (for dbeta); every softmax thread
+    // reaches the barrier, whatever its waits returned
+    {
+      float t0 = (ok && wg == 0) ? dpv : 0.f, t1 = ok ? memt : 0.f;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-      if (lane == 0) red[warp] = t;
-      named_bar_sync(2, 128);
-      if (threadIdx.x == 0 && ok) dot_part[blockIdx.x] = (red[0] + red[1]) + (red[2] + red[3]);
+      for (int o = 16; o > 0; o >>= 1) {
+        t0 += __shfl_xor_sync(0xffffffffu, t0, o);
+        t1 += __shfl_xor_sync(0xffffffffu, t1, o);
+      }
+      if (lane == 0) {
+        red[warp] = t0;
+        red[8 + warp] = t1;
+      }
+      named_bar_sync(2, 256);
+      if (threadIdx.x == 0 && ok) {
+        float a0 = 0.f, a1 = 0.f;
+        for (int w = 0; w < 8; ++w) {
+          a0 += red[w];
+          a1 += red[8 + w];
+        }
+        dot_part[blockIdx.x] = a0;
+        mem_part[blockIdx.x] = a1;
+      }
     }
   }
   tc_fence_before();
@@ -934,7 +845,6 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 //           for the z gradients (dz_s, which needs every later segment's, is added
 //           to dk by dk_dz_kernel afterwards).
 // ---------------------------------------------------------------------------
-enum { P_X = P_COUNT, P_SK, P_M1, P_SK2, P_M2, P_COUNT2 };
 constexpr int kDkdvSmem = 6 * kTile + 2 * 2 * D * 4 + 5 * D * 4 + 64 + 256 + 1024;
 
 __global__ void __launch_bounds__(kPipeThreads, 1)
@@ -974,12 +884,6 @@ dkdv_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const float* sZ = sLD + sx * 2 * D;    // z_{s-1}, Delta
   if (threadIdx.x == 0) {
     pipe_init(bars);
-    mbar_init(&bars[P_X], 1);
-    mbar_init(&bars[P_SK], 8);
-    mbar_init(&bars[P_M1], 1);
-    mbar_init(&bars[P_SK2], 8);
-    mbar_init(&bars[P_M2], 1);
-    fence_barrier_init();
   }
   if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
@@ -1293,8 +1197,8 @@ __global__ void dbeta_bwd_kernel(const float* __restrict__ beta, const float* __
     for (int b = 0; b < B; ++b)
       for (int s = 0; s < S; ++s) {
         const size_t seg = ((size_t)b * H + h) * S + s;
-        double t = mem_part[seg];
-        for (int i = 0; i < T; ++i) t -= dot_part[seg * T + i];
+        double t = 0.0;
+        for (int i = 0; i < T; ++i) t += (double)mem_part[seg * T + i] - dot_part[seg * T + i];
         acc += t;
       }
     const float g = 1.f / (1.f + expf(-beta[h]));
@@ -1307,11 +1211,8 @@ size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 }  // namespace
 
 cudaError_t bf16_bwd_set_attributes() {
-  cudaError_t e = cudaFuncSetAttribute(retr_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kRetrSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(chain_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kChainSmem);
+  cudaError_t e = cudaFuncSetAttribute(chain_bwd_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kChainSmem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(dq_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
   if (e == cudaSuccess)
@@ -1320,13 +1221,13 @@ cudaError_t bf16_bwd_set_attributes() {
   return e;
 }
 
-// Backward scratch after the state path's: per-row statistics, the retrieval's fp32
-// contribution to dq, the per-segment gradients of the state.
+// Backward scratch after the state path's: per-row statistics, per-query-tile
+// partials of the state gradients, the dM_s stack, dz_s, per-tile sums for dbeta.
 size_t bf16_bwd_workspace_bytes(int BH, long long L, int S, int T, int CH) {
   const size_t bh = (size_t)BH, rows = bh * (size_t)L, bhs = bh * S;
-  return up256(bf16_workspace_bytes(BH, S, CH)) + 2 * up256(rows * 4) + up256(rows * D * 4) +
-         up256(bhs * D * D * 4) + up256(bhs * D * 4) + up256(bhs * 2 * D * D * 2) +
-         up256(bhs * D * 4) + up256(bhs * T * D * 4) + up256(bhs * 4) + up256(bhs * T * 4);
+  return up256(bf16_workspace_bytes(BH, S, CH)) + 2 * up256(rows * 4) +
+         up256(bhs * T * D * D * 4) + up256(bhs * T * D * 4) + up256(bhs * 2 * D * D * 2) +
+         up256(bhs * D * 4) + up256(bhs * T * D * 4) + 2 * up256(bhs * T * 4);
 }
 
 cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
@@ -1352,13 +1253,12 @@ cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   };
   float* lse2 = reinterpret_cast<float*>(take(rows * 4));
   float* dpr = reinterpret_cast<float*>(take(rows * 4));
-  float* dq_mem = reinterpret_cast<float*>(take(rows * D * 4));
-  float* GM = reinterpret_cast<float*>(take(bhs * D * D * 4));
-  float* Gz = reinterpret_cast<float*>(take(bhs * D * 4));
+  float* GMp = reinterpret_cast<float*>(take(bhs * T * D * D * 4));
+  float* Gzp = reinterpret_cast<float*>(take(bhs * T * D * 4));
   __nv_bfloat16* dMs = reinterpret_cast<__nv_bfloat16*>(take(bhs * 2 * D * D * 2));
   float* dzs = reinterpret_cast<float*>(take(bhs * D * 4));
   float* gzk = reinterpret_cast<float*>(take(bhs * T * D * 4));
-  float* mem_part = reinterpret_cast<float*>(take(bhs * 4));
+  float* mem_part = reinterpret_cast<float*>(take(bhs * T * 4));
   float* dot_part = reinterpret_cast<float*>(take(bhs * T * 4));
 
   // M_{s-1} (bf16 hi/lo), z_{s-1} and, for Delta, every segment's G_s
@@ -1404,20 +1304,18 @@ cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   p.rsd = 0.08838834764831845f;
   p.sl = 1.4426950408889634f * p.rsd;
 
-  retr_bwd_kernel<<<(unsigned)bhs, kThreads, kRetrSmem, stream>>>(mq, mdo, mm, beta, ws.zprev,
-                                                                  dq_mem, GM, Gz, mem_part, p);
-  chain_bwd_kernel<<<dim3(BH, 4), kChainThreads, kChainSmem, stream>>>(mg, GM, dM_out, dM_in, dMs,
-                                                                        S, CH, mode);
-  if (mode == 0) dz_bwd_kernel<<<BH, D, 0, stream>>>(Gz, gzk, dz_out, dzs, dz_in, S, T, mode);
   mark(0);
-  dq_bwd_kernel<<<p.tiles, kPipeThreads, kDqSmem, stream>>>(mq, mk, mv, mdo, beta, dq_mem, lse2, dpr,
-                                                         dot_part, dq, p);
+  dq_bwd_kernel<<<p.tiles, kPipeThreads, kDqSmem, stream>>>(
+      mq, mk, mv, mdo, mm, beta, ws.zprev, lse2, dpr, dot_part, mem_part, GMp, Gzp, dq, p);
   mark(1);
+  chain_bwd_kernel<<<dim3(BH, 4), kChainThreads, kChainSmem, stream>>>(mg, GMp, dM_out, dM_in, dMs,
+                                                                        S, CH, T, mode);
+  if (mode == 0) dz_bwd_kernel<<<BH, D, 0, stream>>>(Gzp, gzk, dz_out, dzs, dz_in, S, T, mode);
   dkdv_bwd_kernel<<<p.tiles, kPipeThreads, kDkdvSmem, stream>>>(
       mq, mk, mv, mdo, mm, mx, beta, ws.zprev, lse2, dpr, dzs, gzk, dk, dv, p, mode);
   mark(2);
   if (mode == 1) {
-    dz_bwd_kernel<<<BH, D, 0, stream>>>(Gz, gzk, dz_out, dzs, dz_in, S, T, mode);
+    dz_bwd_kernel<<<BH, D, 0, stream>>>(Gzp, gzk, dz_out, dzs, dz_in, S, T, mode);
     const long long units = (long long)rows * (D / 8);
     const unsigned grid = (unsigned)min((units + 255) / 256, 148LL * 16);
     dk_dz_kernel<<<grid, 256, 0, stream>>>(k, dzs, dk, L, N, S, units);

@@ -273,8 +273,9 @@ int infini_attn_forward_ex(const void* q, const void* k, const void* v, const fl
  * infini_attn_backward with options: opts->workspace (256-byte aligned, at least
  * infini_attn_backward_workspace_size(...) bytes) replaces the stream-ordered
  * allocation; opts->stage_events[0..2] (cudaEvent_t or NULL) are recorded on
- * `stream` after the memory path's kernels (state rebuild, retrieval, state
- * gradients, update backward), after the dq kernel, and after the dk/dv kernel.
+ * `stream` after the state rebuild, after the dq kernel (which also runs the
+ * retrieval's backward) and after the dk/dv kernel (preceded by the reverse state
+ * chain; it also runs the memory update's backward).
  */
 int infini_attn_backward_ex(const void* q, const void* k, const void* v, const float* beta,
                             const float* M_in, const float* z_in, const void* dout,
