@@ -480,8 +480,11 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   uint8_t* sM = sK;           // M_{s-1} (hi): K stage 0, free once load nl - 2 is done
   uint8_t* sDN = sK + kTile;  // dnum: K stage 1; dden in the next 64-column box (V stage 0)
 
+  // tiles of a segment are adjacent in the grid (K/V stay in L2), the heaviest first
   int bh, s, i;
   decode3(p, blockIdx.x, bh, s, i);
+  i = p.T - 1 - i;
+  const unsigned tile = (unsigned)((bh * p.S + s) * p.T + i);  // index of the partials
   const int b = bh / p.H, h = bh - b * p.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = i + 1, nl = 2 * nk, nh = 2 * nl;
@@ -747,9 +750,16 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     xs[wg * D + r] = dd;  // every thread has read den above (P_M1 needs all P_SK arrivals)
     named_bar_sync(1, 256);
     const float dden = -(xs[r] + xs[D + r]) * inv;
-    if (wg == 0)  // the 129th column of the product's right operand: (row r, column 0) of box 2
-      *reinterpret_cast<__nv_bfloat16*>(sDN + 2 * kSub + sw128((uint32_t)r, 0)) =
-          __float2bfloat16_rn(dden);
+    if (wg == 0) {
+      // columns 128 and 129 of the product's right operand, (row r, columns 0 and 1) of
+      // box 2: dden as a bf16 pair hi + lo, so that Gz keeps fp32 accuracy in dden
+      const __nv_bfloat16 hi = __float2bfloat16_rn(dden);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(dden - __bfloat162float(hi));
+      __nv_bfloat162 pr;
+      pr.x = hi;
+      pr.y = lo;
+      *reinterpret_cast<__nv_bfloat162*>(sDN + 2 * kSub + sw128((uint32_t)r, 0)) = pr;
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     mbar_arrive_warp(&bars[P_SK2]);
@@ -758,7 +768,7 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (ok) {
       tc_fence_after();
       __nv_bfloat16* dst = dq + rowi * D;
-      float* gm = GMp + ((size_t)blockIdx.x * D + r) * D;
+      float* gm = GMp + ((size_t)tile * D + r) * D;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const uint32_t col = 64 * wg + 32 * c;
@@ -789,9 +799,9 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       if (wg == 0) {
         uint32_t zv[32];
-        tmem_ld32(tmem + lane_off + 128, zv);  // column 128: sigma(Q)^T dden
+        tmem_ld32(tmem + lane_off + 128, zv);  // columns 128, 129: sigma(Q)^T dden (hi, lo)
         tmem_wait_ld();
-        Gzp[(size_t)blockIdx.x * D + r] = __uint_as_float(zv[0]);
+        Gzp[(size_t)tile * D + r] = __uint_as_float(zv[0]) + __uint_as_float(zv[1]);
         lse_out[rowi] = lse2;
         dp_out[rowi] = dpv;
       }
@@ -816,8 +826,8 @@ dq_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           a0 += red[w];
           a1 += red[8 + w];
         }
-        dot_part[blockIdx.x] = a0;
-        mem_part[blockIdx.x] = a1;
+        dot_part[tile] = a0;
+        mem_part[tile] = a1;
       }
     }
   }
