@@ -291,6 +291,25 @@ chain_bwd_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restri
 #pragma unroll
       for (int e = 0; e < 32; ++e) x[e] = 0.f;
     }
+    // GM of the next segment in the sequence (the sum of its query tiles' partials, in
+    // tile order), loaded while the current one is used
+    float nx[32];
+    auto load_gm = [&](int s) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) nx[e] = 0.f;
+      const float* src = GMp + (((size_t)bh * S + s) * T * D + r) * D + c0;
+      for (int t = 0; t < T; ++t, src += (size_t)D * D) {
+        float4 v4[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v4[e] = __ldg(reinterpret_cast<const float4*>(src + 4 * e));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          nx[4 * e] += v4[e].x; nx[4 * e + 1] += v4[e].y;
+          nx[4 * e + 2] += v4[e].z; nx[4 * e + 3] += v4[e].w;
+        }
+      }
+    };
+    if (S > 0) load_gm(S - 1);
     for (int q = 0; q < S; ++q) {
       const int s = S - 1 - q;
       {  // dM_s -> hi / lo bf16
@@ -311,18 +330,10 @@ chain_bwd_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restri
           *reinterpret_cast<uint4*>(lo + e) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
         }
       }
-      // GM_s: the segment's query tiles' partials, added in tile order
       float gm[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) gm[e] = 0.f;
-      for (int t = 0; t < T; ++t) {
-        const float* src = GMp + ((((size_t)bh * S + s) * T + t) * D + r) * D + c0;
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 v4 = __ldg(reinterpret_cast<const float4*>(src + e));
-          gm[e] += v4.x; gm[e + 1] += v4.y; gm[e + 2] += v4.z; gm[e + 3] += v4.w;
-        }
-      }
+      for (int e = 0; e < 32; ++e) gm[e] = nx[e];
+      if (s > 0) load_gm(s - 1);
       if (delta) {
         // X^T block (tf32) -> shared memory: row c, K-major, 4 boxes of 32 k
         const uint32_t kb = (uint32_t)(r >> 5), kin = (uint32_t)(r & 31);
@@ -1198,19 +1209,24 @@ dk_dz_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict__ dzs,
   }
 }
 
-// dbeta[h] = g (1 - g) sum over batch rows and segments of (sum dout * A_mem - sum D').
+// dbeta[h] = g (1 - g) sum over batch rows, segments and query tiles of (sum dout *
+// A_mem - sum D'). One warp per head: lane l takes the (batch row, tile) sums l, l+32,
+// ... in order, then a fixed shuffle tree (the result does not depend on timing).
 __global__ void dbeta_bwd_kernel(const float* __restrict__ beta, const float* __restrict__ mem_part,
                                  const float* __restrict__ dot_part, float* __restrict__ dbeta,
                                  int B, int H, int S, int T) {
-  for (int h = threadIdx.x; h < H; h += blockDim.x) {
-    double acc = 0.0;
-    for (int b = 0; b < B; ++b)
-      for (int s = 0; s < S; ++s) {
-        const size_t seg = ((size_t)b * H + h) * S + s;
-        double t = 0.0;
-        for (int i = 0; i < T; ++i) t += (double)mem_part[seg * T + i] - dot_part[seg * T + i];
-        acc += t;
-      }
+  const int h = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (h >= H) return;
+  const long long per_b = (long long)S * T, n = (long long)B * per_b;
+  double acc = 0.0;
+  for (long long x = lane; x < n; x += 32) {
+    const long long b = x / per_b, st = x - b * per_b;
+    const size_t k = ((size_t)b * H + h) * per_b + st;
+    acc += (double)mem_part[k] - (double)dot_part[k];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
     const float g = 1.f / (1.f + expf(-beta[h]));
     dbeta[h] = (float)(acc * (double)g * (1.0 - (double)g));
   }
@@ -1330,7 +1346,7 @@ cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
     const unsigned grid = (unsigned)min((units + 255) / 256, 148LL * 16);
     dk_dz_kernel<<<grid, 256, 0, stream>>>(k, dzs, dk, L, N, S, units);
   }
-  dbeta_bwd_kernel<<<1, 128, 0, stream>>>(beta, mem_part, dot_part, dbeta, B, H, S, T);
+  dbeta_bwd_kernel<<<(H + 3) / 4, 128, 0, stream>>>(beta, mem_part, dot_part, dbeta, B, H, S, T);
   return cudaGetLastError();
 }
 
