@@ -12,6 +12,8 @@ Entry points (same names as the C ABI in include/infini_attn.h):
     infini_attn_state_update(k, v, N, mode, M_in=None, z_in=None, ...)
     infini_attn_state_sum(dM, dz, M_in=None, z_in=None, ...)
     infini_attn_backward(q, k, v, beta, N, mode, dout, M_in=None, z_in=None, ...)
+    infini_attn_layer_forward(x, Wq, Wk, Wv, Wo, beta, N, mode, H, H_kv, ...)
+    infini_attn_gemm_bf16(A, B)
 q, k, v: [B, H, L, d] CUDA tensors, bf16 (d = 128) or fp32 (d <= 128);
 beta: [H] fp32; M: [B, H, d, d] fp32; z: [B, H, d] fp32.
 """
@@ -63,6 +65,8 @@ _SIGS = {
     "infini_attn_backward": [_vp] * 15 + [_i, _i, _ll, _i, _i, _i, _vp],
     "infini_attn_backward_ex": [_vp] * 15 + [_i, _i, _ll, _i, _i, _i, ctypes.POINTER(Opts), _vp],
     "infini_attn_backward_workspace_size": [_i, _i, _ll, _i, _i, _i],
+    "infini_attn_layer_forward": [_vp] * 11 + [_i, _ll, _i, _i, _i, _i, _i, _i, _vp],
+    "infini_attn_gemm_bf16": [_vp, _vp, _vp, _ll, _i, _i, _vp],
     "infini_attn_workspace_size": [_i, _i, _ll, _i, _i, _i, _i],
     "infini_attn_device_status": [],
     "infini_attn_selftest_timeout": [_ll, _vp],
@@ -297,6 +301,55 @@ def infini_attn_backward(q, k, v, beta, N, mode, dout, M_in=None, z_in=None, dM_
             o.stage_events[i] = ev.cuda_event if ev is not None else None
         _check(_lib.infini_attn_backward_ex(*args, ctypes.byref(o), _stream_handle(stream)))
     return dq, dk, dv, dbeta, dM_in, dz_in
+
+
+def infini_attn_gemm_bf16(A, B, out=None, stream=None):
+    """A [M, K] @ B [K, N] (bf16 CUDA, row-major; M, N, K multiples of 128) on the
+    tensor cores with fp32 accumulation; returns C [M, N] bf16."""
+    if A.dim() != 2 or B.dim() != 2 or A.shape[1] != B.shape[0]:
+        raise ValueError("A must be [M, K] and B [K, N]")
+    for t in (A, B):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("A and B must be contiguous bf16 CUDA tensors")
+    M, K = A.shape
+    N = B.shape[1]
+    if out is None:
+        out = torch.empty((M, N), device=A.device, dtype=torch.bfloat16)
+    _check(_lib.infini_attn_gemm_bf16(_ptr(A), _ptr(B), _ptr(out), M, N, K,
+                                      _stream_handle(stream)))
+    return out
+
+
+def infini_attn_layer_forward(x, Wq, Wk, Wv, Wo, beta, N, mode, H, H_kv=None, M_in=None,
+                              z_in=None, out=None, state_out=True, stream=None):
+    """One attention layer: x [B, L, D_model] bf16 -> projections (Wq [D_model, H*128],
+    Wk, Wv [D_model, H_kv*128]) -> grouped-head forward -> y = heads @ Wo
+    ([H*128, D_model]). Returns (y, M_out, z_out) with the state per key/value head
+    (None when state_out is False)."""
+    H_kv = H if H_kv is None else H_kv
+    if x.dim() != 3:
+        raise ValueError("x must be [B, L, D_model]")
+    B, L, D_model = x.shape
+    d = Wq.shape[1] // H
+    for t in (x, Wq, Wk, Wv, Wo):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("x and the weights must be contiguous bf16 CUDA tensors")
+    if (Wq.shape != (D_model, H * d) or Wk.shape != (D_model, H_kv * d)
+            or Wv.shape != (D_model, H_kv * d) or Wo.shape != (H * d, D_model)):
+        raise ValueError("weight shapes do not match x, H and H_kv")
+    if beta.dtype != torch.float32 or beta.numel() != H or not beta.is_cuda:
+        raise ValueError("beta must be a CUDA fp32 tensor with H elements")
+    if out is None:
+        out = torch.empty_like(x)
+    M_out = z_out = None
+    if state_out:
+        M_out = torch.empty((B, H_kv, d, d), device=x.device, dtype=torch.float32)
+        z_out = torch.empty((B, H_kv, d), device=x.device, dtype=torch.float32)
+    _check(_lib.infini_attn_layer_forward(_ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(Wo),
+                                          _ptr(beta), _ptr(M_in), _ptr(z_in), _ptr(out),
+                                          _ptr(M_out), _ptr(z_out), B, L, D_model, H, H_kv,
+                                          int(N), d, int(mode), _stream_handle(stream)))
+    return out, M_out, z_out
 
 
 def backward_workspace_size(B, H, L, N, d, mode=LINEAR) -> int:

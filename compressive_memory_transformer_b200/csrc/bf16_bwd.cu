@@ -105,7 +105,6 @@ __device__ __forceinline__ uint64_t mdesc(uint32_t base, int kk) {
 }
 constexpr uint32_t kIdKK = idesc_f32acc(1, 0, 0, 128, 128);
 constexpr uint32_t kIdKM = idesc_f32acc(1, 0, 1, 128, 128);
-constexpr uint32_t kIdMM = idesc_f32acc(1, 1, 1, 128, 128);
 
 // D (+)= A B^T: A[m][k] and B[n][k] are tiles (rows m and n, 128 k each)
 __device__ __forceinline__ void gemm_kk(uint32_t d, const uint8_t* a, const uint8_t* b, bool acc) {

@@ -75,6 +75,11 @@ cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                                  void* scratch, int CH, int CL, cudaStream_t stream,
                                  cudaEvent_t const* events = nullptr);
 
+// C [M][N] = A [M][K] B [K][N] (bf16, row-major, fp32 accumulation; bf16_gemm.cu);
+// M, N, K multiples of 128.
+cudaError_t bf16_gemm_launch(const __nv_bfloat16* A, const __nv_bfloat16* B, __nv_bfloat16* C,
+                             long long M, int N, int K, cudaStream_t stream);
+
 // Token-level decode (bf16_decode.cu): partial attention over the KV cache (rows
 // below pos) and the new rows (k, v, also written into the caches), split like flash
 // decoding, then merge + retrieval from the fp32 state + gate. `part` holds

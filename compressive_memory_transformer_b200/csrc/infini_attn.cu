@@ -23,6 +23,7 @@ __device__ unsigned long long g_wait_timeout_ns = 4000000000ull;  // 4 s per wai
 cudaError_t bf16_state_set_attributes();
 cudaError_t bf16_attn_set_attributes();
 cudaError_t bf16_bwd_set_attributes();
+cudaError_t bf16_gemm_set_attributes();
 
 namespace {
 
@@ -53,6 +54,7 @@ cudaError_t prepare_device(int* dev_out) {
   e = bf16_state_set_attributes();
   if (e == cudaSuccess) e = bf16_attn_set_attributes();
   if (e == cudaSuccess) e = bf16_bwd_set_attributes();
+  if (e == cudaSuccess) e = bf16_gemm_set_attributes();
   SideStream& sd = g_side[dev];
   if (e == cudaSuccess && !sd.stream) e = cudaStreamCreateWithFlags(&sd.stream, cudaStreamNonBlocking);
   if (e == cudaSuccess && !sd.fork) e = cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming);
@@ -439,6 +441,78 @@ int backward_impl(const void* q, const void* k, const void* v, const float* beta
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
+int gemm_checks(const void* A, const void* Bm, const void* C, long long M, int N, int K) {
+  if (!A || !Bm || !C) return INFINI_ERR_NULL;
+  if (M < 1 || N < 1 || K < 1) return INFINI_ERR_SHAPE;
+  if (M % 128 || N % 128 || K % 128) return INFINI_ERR_UNSUPPORTED;
+  if (overflows(M, K) || overflows(M * K, 2) || overflows(M, N) || overflows(M * N, 2) ||
+      overflows((long long)K, (long long)N * 2) || M / 128 * (N / 128) >= (1LL << 31))
+    return INFINI_ERR_SHAPE;
+  if (!aligned16(A) || !aligned16(Bm) || !aligned16(C)) return INFINI_ERR_ALIGN;
+  if (overlap(C, (size_t)(M * N) * 2, A, (size_t)(M * K) * 2) ||
+      overlap(C, (size_t)(M * N) * 2, Bm, (size_t)K * N * 2))
+    return INFINI_ERR_ALIAS;
+  return INFINI_OK;
+}
+
+// One attention layer: q, k, v = x W_Q, x W_K, x W_V ([B, L, heads * d], the heads'
+// columns side by side, read in place as [B, L, heads, d]), the grouped-head forward,
+// y = [A_1 ... A_H] W_O.
+int layer_forward_impl(const void* x, const void* Wq, const void* Wk, const void* Wv,
+                       const void* Wo, const float* beta, const float* M_in, const float* z_in,
+                       void* y, float* M_out, float* z_out, int B, long long L, int D_model,
+                       int H, int H_kv, int N, int d, int mode, cudaStream_t stream) {
+  if (!x || !Wq || !Wk || !Wv || !Wo || !beta || !y) return INFINI_ERR_NULL;
+  if ((M_in == nullptr) != (z_in == nullptr) || (M_out == nullptr) != (z_out == nullptr))
+    return INFINI_ERR_NULL;
+  if (B < 1 || L < 1 || D_model < 1 || H < 1 || H_kv < 1 || N < 1 || d < 1)
+    return INFINI_ERR_SHAPE;
+  if (H % H_kv != 0) return INFINI_ERR_SHAPE;
+  if (mode != INFINI_LINEAR && mode != INFINI_DELTA) return INFINI_ERR_UNSUPPORTED;
+  if (d != 128 || D_model % 128 != 0 || ((long long)B * L) % 128 != 0)
+    return INFINI_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * L;
+  if (overflows(rows, (long long)H * d * 2) || overflows(rows, (long long)D_model * 2) ||
+      L >= (1LL << 31))
+    return INFINI_ERR_SHAPE;
+  const void* ins[] = {x, Wq, Wk, Wv, Wo};
+  for (const void* q : ins)
+    if (!aligned16(q)) return INFINI_ERR_ALIGN;
+  if (!aligned16(y) || (M_in && !aligned16(M_in)) || (M_out && !aligned16(M_out)))
+    return INFINI_ERR_ALIGN;
+  const size_t ny = (size_t)(rows * D_model) * 2;
+  const size_t nw_qo = (size_t)D_model * H * d * 2, nw_kv = (size_t)D_model * H_kv * d * 2;
+  if (overlap(y, ny, x, ny) || overlap(y, ny, Wq, nw_qo) || overlap(y, ny, Wk, nw_kv) ||
+      overlap(y, ny, Wv, nw_kv) || overlap(y, ny, Wo, nw_qo))
+    return INFINI_ERR_ALIAS;
+  int dev = 0;
+  if (prepare_device(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
+  const size_t nq = (size_t)(rows * H * d), nkv = (size_t)(rows * H_kv * d);
+  Scratch sc;
+  const int st = get_scratch(sc, (2 * nq + 2 * nkv) * 2 + 256, nullptr, stream);
+  if (st != INFINI_OK) return st;
+  auto* q = static_cast<__nv_bfloat16*>(sc.ptr);
+  __nv_bfloat16* k = q + nq;
+  __nv_bfloat16* v = k + nkv;
+  __nv_bfloat16* a = v + nkv;  // the heads' outputs, [B, L, H, d]
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  cudaError_t e = bf16_gemm_launch(xb, static_cast<const __nv_bfloat16*>(Wq), q, rows, H * d,
+                                   D_model, stream);
+  if (e == cudaSuccess)
+    e = bf16_gemm_launch(xb, static_cast<const __nv_bfloat16*>(Wk), k, rows, H_kv * d, D_model,
+                         stream);
+  if (e == cudaSuccess)
+    e = bf16_gemm_launch(xb, static_cast<const __nv_bfloat16*>(Wv), v, rows, H_kv * d, D_model,
+                         stream);
+  if (e != cudaSuccess) return INFINI_ERR_CUDA;
+  const int fs = forward_impl(q, k, v, beta, M_in, z_in, a, M_out, z_out, B, H, L, N, d, mode,
+                              INFINI_DTYPE_BF16, nullptr, stream, H_kv, INFINI_LAYOUT_BLHD);
+  if (fs != INFINI_OK) return fs;
+  e = bf16_gemm_launch(a, static_cast<const __nv_bfloat16*>(Wo), static_cast<__nv_bfloat16*>(y),
+                       rows, D_model, H * d, stream);
+  return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace infini
 
@@ -570,6 +644,28 @@ size_t infini_attn_backward_workspace_size(int B, int H, long long L, int N, int
   int CH = 1, CL = N;
   bf16_state_plan((int)BH, S, N, &CH, &CL);
   return bf16_bwd_workspace_bytes((int)BH, L, S, N / 128, CH);
+}
+
+int infini_attn_gemm_bf16(const void* A, const void* B, void* C, long long M, int N, int K,
+                          void* stream) {
+  const int st = gemm_checks(A, B, C, M, N, K);
+  if (st != INFINI_OK) return st;
+  int dev = 0;
+  if (prepare_device(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
+  const cudaError_t e = bf16_gemm_launch(static_cast<const __nv_bfloat16*>(A),
+                                         static_cast<const __nv_bfloat16*>(B),
+                                         static_cast<__nv_bfloat16*>(C), M, N, K,
+                                         static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+}
+
+int infini_attn_layer_forward(const void* x, const void* Wq, const void* Wk, const void* Wv,
+                              const void* Wo, const float* beta, const float* M_in,
+                              const float* z_in, void* y, float* M_out, float* z_out, int B,
+                              long long L, int D_model, int H, int H_kv, int N, int d, int mode,
+                              void* stream) {
+  return layer_forward_impl(x, Wq, Wk, Wv, Wo, beta, M_in, z_in, y, M_out, z_out, B, L, D_model,
+                            H, H_kv, N, d, mode, static_cast<cudaStream_t>(stream));
 }
 
 int infini_attn_device_status(void) {

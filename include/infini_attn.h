@@ -227,6 +227,39 @@ int infini_attn_backward(const void* q, const void* k, const void* v, const floa
                          float* dbeta, float* dM_in, float* dz_in, int B, int H, long long L,
                          int N, int d, int mode, void* stream);
 
+/*
+ * One attention layer with its projections ("Leave No Context Behind", sections 3.1
+ * and 3.6 as quoted on llm-papers-study.pages.dev): Q = x W_Q, K = x W_K, V = x W_V
+ * (heads side by side in the columns: head h is columns [h d, h d + d)), the
+ * grouped-head forward of infini_attn_forward_gqa on them in place ([B, L, heads, d]),
+ * then y = [A_1 ... A_H] W_O.
+ *   x        device, bf16 [B, L, D_model] row-major
+ *   Wq       device, bf16 [D_model, H * d];  Wk, Wv: [D_model, H_kv * d]
+ *   Wo       device, bf16 [H * d, D_model]
+ *   beta     device, fp32 [H]; M_in/z_in, M_out/z_out as infini_attn_forward_gqa
+ *            (per key/value head: [B, H_kv, d, d] and [B, H_kv, d])
+ *   y        device, bf16 [B, L, D_model], written
+ * Requires d = 128, D_model a multiple of 128 and B * L a multiple of 128
+ * (INFINI_ERR_UNSUPPORTED otherwise), H a multiple of H_kv, 16-byte alignment; y may
+ * not overlap x or a weight. Asynchronous on `stream`; the projections' outputs
+ * (2 (H + H_kv) d bf16 per token) and the forward's scratch come from the
+ * stream-ordered allocator.
+ */
+int infini_attn_layer_forward(const void* x, const void* Wq, const void* Wk, const void* Wv,
+                              const void* Wo, const float* beta, const float* M_in,
+                              const float* z_in, void* y, float* M_out, float* z_out, int B,
+                              long long L, int D_model, int H, int H_kv, int N, int d, int mode,
+                              void* stream);
+
+/*
+ * C [M][N] = A [M][K] B [K][N]: bf16 row-major in and out, fp32 accumulation on the
+ * tensor cores (the layer's projection GEMM). M, N, K multiples of 128
+ * (INFINI_ERR_UNSUPPORTED otherwise); device pointers, 16-byte aligned; C may not
+ * overlap A or B. Asynchronous on `stream`, no scratch.
+ */
+int infini_attn_gemm_bf16(const void* A, const void* B, void* C, long long M, int N, int K,
+                          void* stream);
+
 /* fp32 q/k/v/out variants of infini_attn_forward and infini_attn_step; 1 <= d <= 128. */
 int infini_attn_forward_f32(const float* q, const float* k, const float* v, const float* beta,
                             const float* M_in, const float* z_in, float* out, float* M_out,

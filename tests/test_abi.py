@@ -208,3 +208,34 @@ def call_backward(lib, q=IN0, k=IN0 + (1 << 20), v=IN0 + (2 << 20), beta=IN0 + (
 def test_backward_rejects_bad_arguments(lib, kw, code):
     """Every argument error of the gradient entry point is reported on the host."""
     assert call_backward(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(A=None), -1), (dict(M=0), -2), (dict(K=-128), -2),
+    (dict(M=200), -3), (dict(N=96), -3), (dict(K=64), -3),
+    (dict(A=IN0 + 8), -4),
+    (dict(C=IN0 + 4096), -8),  # C over A
+])
+def test_gemm_rejects_bad_arguments(lib, kw, code):
+    a = dict(A=IN0, B=IN0 + (8 << 20), C=OUT0, M=256, N=256, K=256)
+    a.update(kw)
+    assert lib.raw_call("infini_attn_gemm_bf16", a["A"], a["B"], a["C"], a["M"], a["N"], a["K"],
+                        None) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=None), -1), (dict(Wo=None), -1), (dict(M_in=OUT0 * 2), -1),
+    (dict(B=0), -2), (dict(H=4, H_kv=3), -2), (dict(H_kv=0), -2),
+    (dict(d=64), -3), (dict(D_model=192), -3), (dict(L=100), -3), (dict(mode=2), -3),
+    (dict(y=OUT0 + 8), -4),
+    (dict(y=IN0), -8),  # y over x
+])
+def test_layer_forward_rejects_bad_arguments(lib, kw, code):
+    a = dict(x=IN0, Wq=IN0 + (8 << 20), Wk=IN0 + (9 << 20), Wv=IN0 + (10 << 20),
+             Wo=IN0 + (11 << 20), beta=IN0 + (12 << 20), M_in=None, z_in=None, y=OUT0,
+             M_out=None, z_out=None, B=1, L=128, D_model=256, H=2, H_kv=2, N=128, d=128, mode=0)
+    a.update(kw)
+    assert lib.raw_call("infini_attn_layer_forward", a["x"], a["Wq"], a["Wk"], a["Wv"], a["Wo"],
+                        a["beta"], a["M_in"], a["z_in"], a["y"], a["M_out"], a["z_out"], a["B"],
+                        a["L"], a["D_model"], a["H"], a["H_kv"], a["N"], a["d"], a["mode"],
+                        None) == code
