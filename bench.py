@@ -633,6 +633,48 @@ def run_extra(args, device):
                               "scan and the dk fix-up) and the dbeta sum; executed tensor "
                               "work is about 2.3x the algorithmic count (S and dP' are "
                               "recomputed in both attention kernels)"})
+    if which in ("layer", "all"):
+        # one attention layer with its projections on the 1B-layer shape: x [B, L, 1024]
+        # -> Q, K, V (8 heads of 128) -> forward -> W_O; and the projection GEMM alone
+        from synthetic_inputs import normal
+        Bc, Lc, Hc, Nc = 4, 32768, 8, 2048
+        Dm = Hc * D
+        x = normal((Bc, Lc, Dm), torch.bfloat16, 0, 0, device="cuda").to(device)
+        Ws = [(normal((Dm, Dm), torch.float32, 0, 1 + i, device="cuda") / Dm ** 0.5).to(
+            torch.bfloat16).to(device) for i in range(4)]
+        beta = normal((Hc,), torch.float32, 0, 5, device="cuda").to(device)
+        y = torch.empty_like(x)
+        res = {}
+        for mode, name in ((ia.LINEAR, "linear"), (ia.DELTA, "delta")):
+            def f():
+                ia.infini_attn_layer_forward(x, Ws[0], Ws[1], Ws[2], Ws[3], beta, Nc, mode, Hc,
+                                             out=y, state_out=False)
+            for _ in range(2):
+                f()
+            torch.cuda.synchronize()
+            ms = _timed(f, 5, stream)
+            res[name] = {"ms_per_call": ms, "tokens_per_s": Bc * Lc / (ms / 1e3)}
+        A2 = x.view(Bc * Lc, Dm)
+        C2 = torch.empty((Bc * Lc, Dm), device=device, dtype=torch.bfloat16)
+        g = lambda: ia.infini_attn_gemm_bf16(A2, Ws[0], out=C2)
+        for _ in range(3):
+            g()
+        torch.cuda.synchronize()
+        gms = _timed(g, 20, stream)
+        gflop = 2.0 * Bc * Lc * Dm * Dm
+        gtf = gflop / (gms / 1e3) / 1e12
+        assert ia.device_status() == 0
+        del x, Ws, y, A2, C2
+        lines.append({"config": "layer: B=4, L=32768, D_model=1024, H=H_kv=8, d=128, N=2048, "
+                                "bf16, infini_attn_layer_forward (4 projections + forward)",
+                      **res,
+                      "projection_gemm": {"shape": "[131072 x 1024] @ [1024 x 1024]",
+                                          "ms": gms, "tflops": gtf,
+                                          "roofline": {"bound": "tensor", "achieved": gtf,
+                                                       "peak": peak_burst, "unit": "TFLOP/s",
+                                                       "frac": gtf / peak_burst,
+                                                       "peak_kind": "burst (measured cuBLAS)"}},
+                      "peak_source": src})
     return lines
 
 
@@ -644,7 +686,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--config", choices=["c2", "c3", "c4", "c5", "decode", "backward", "all"],
+    ap.add_argument("--config", choices=["c2", "c3", "c4", "c5", "decode", "backward", "layer",
+                                         "all"],
                     default="c2",
                     help="c2 (default) prints the headline line; the others print one extra "
                          "line per workload of the configuration list")
