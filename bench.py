@@ -644,11 +644,13 @@ def run_extra(args, device):
             torch.bfloat16).to(device) for i in range(4)]
         beta = normal((Hc,), torch.float32, 0, 5, device="cuda").to(device)
         y = torch.empty_like(x)
+        lws = torch.empty(ia.layer_workspace_size(Bc, Lc, Dm, Hc, Hc, Nc), dtype=torch.uint8,
+                          device=device)
         res = {}
         for mode, name in ((ia.LINEAR, "linear"), (ia.DELTA, "delta")):
             def f():
                 ia.infini_attn_layer_forward(x, Ws[0], Ws[1], Ws[2], Ws[3], beta, Nc, mode, Hc,
-                                             out=y, state_out=False)
+                                             out=y, state_out=False, workspace=lws)
             for _ in range(2):
                 f()
             torch.cuda.synchronize()
@@ -663,8 +665,21 @@ def run_extra(args, device):
         gms = _timed(g, 20, stream)
         gflop = 2.0 * Bc * Lc * Dm * Dm
         gtf = gflop / (gms / 1e3) / 1e12
+        # the forward inside the layer alone: the projections' outputs read in place as
+        # [B, L, H, d]
+        qkv = [ia.infini_attn_gemm_bf16(A2, Ws[i]).view(Bc, Lc, Hc, D) for i in range(3)]
+        o4 = torch.empty_like(qkv[0])
+        for mode, name in ((ia.LINEAR, "linear"), (ia.DELTA, "delta")):
+            def fw():
+                ia.infini_attn_forward_gqa(qkv[0], qkv[1], qkv[2], beta, Nc, mode,
+                                           ia.LAYOUT_BLHD, out=o4, state_out=False)
+            for _ in range(2):
+                fw()
+            torch.cuda.synchronize()
+            res[name]["forward_part_ms"] = _timed(fw, 5, stream)
+            res[name]["projections_part_ms"] = 4 * gms
         assert ia.device_status() == 0
-        del x, Ws, y, A2, C2
+        del x, Ws, y, A2, C2, qkv, o4, lws
         lines.append({"config": "layer: B=4, L=32768, D_model=1024, H=H_kv=8, d=128, N=2048, "
                                 "bf16, infini_attn_layer_forward (4 projections + forward)",
                       **res,

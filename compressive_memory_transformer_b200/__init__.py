@@ -67,6 +67,9 @@ _SIGS = {
     "infini_attn_backward_workspace_size": [_i, _i, _ll, _i, _i, _i],
     "infini_attn_layer_forward": [_vp] * 11 + [_i, _ll, _i, _i, _i, _i, _i, _i, _vp],
     "infini_attn_gemm_bf16": [_vp, _vp, _vp, _ll, _i, _i, _vp],
+    "infini_attn_layer_forward_ex": [_vp] * 11 + [_i, _ll, _i, _i, _i, _i, _i, _i,
+                                                  ctypes.POINTER(Opts), _vp],
+    "infini_attn_layer_workspace_size": [_i, _ll, _i, _i, _i, _i, _i, _i],
     "infini_attn_workspace_size": [_i, _i, _ll, _i, _i, _i, _i],
     "infini_attn_device_status": [],
     "infini_attn_selftest_timeout": [_ll, _vp],
@@ -80,6 +83,7 @@ for _name, _args in _SIGS.items():
 _lib.infini_attn_strerror.restype = ctypes.c_char_p
 _lib.infini_attn_workspace_size.restype = ctypes.c_size_t
 _lib.infini_attn_backward_workspace_size.restype = ctypes.c_size_t
+_lib.infini_attn_layer_workspace_size.restype = ctypes.c_size_t
 
 # every symbol the header declares (checked by the CPU tests)
 EXPORTED = tuple(_SIGS)
@@ -321,11 +325,14 @@ def infini_attn_gemm_bf16(A, B, out=None, stream=None):
 
 
 def infini_attn_layer_forward(x, Wq, Wk, Wv, Wo, beta, N, mode, H, H_kv=None, M_in=None,
-                              z_in=None, out=None, state_out=True, stream=None):
+                              z_in=None, out=None, state_out=True, workspace=None,
+                              stage_events=None, stream=None):
     """One attention layer: x [B, L, D_model] bf16 -> projections (Wq [D_model, H*128],
     Wk, Wv [D_model, H_kv*128]) -> grouped-head forward -> y = heads @ Wo
     ([H*128, D_model]). Returns (y, M_out, z_out) with the state per key/value head
-    (None when state_out is False)."""
+    (None when state_out is False). workspace: optional uint8 CUDA tensor of at least
+    layer_workspace_size(...) bytes; stage_events: up to three torch.cuda.Event recorded
+    after the Q/K/V projections, after the forward and after the output projection."""
     H_kv = H if H_kv is None else H_kv
     if x.dim() != 3:
         raise ValueError("x must be [B, L, D_model]")
@@ -345,11 +352,24 @@ def infini_attn_layer_forward(x, Wq, Wk, Wv, Wo, beta, N, mode, H, H_kv=None, M_
     if state_out:
         M_out = torch.empty((B, H_kv, d, d), device=x.device, dtype=torch.float32)
         z_out = torch.empty((B, H_kv, d), device=x.device, dtype=torch.float32)
-    _check(_lib.infini_attn_layer_forward(_ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(Wo),
-                                          _ptr(beta), _ptr(M_in), _ptr(z_in), _ptr(out),
-                                          _ptr(M_out), _ptr(z_out), B, L, D_model, H, H_kv,
-                                          int(N), d, int(mode), _stream_handle(stream)))
+    args = (_ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(Wo), _ptr(beta), _ptr(M_in),
+            _ptr(z_in), _ptr(out), _ptr(M_out), _ptr(z_out), B, L, D_model, H, H_kv, int(N), d,
+            int(mode))
+    if workspace is None and stage_events is None:
+        _check(_lib.infini_attn_layer_forward(*args, _stream_handle(stream)))
+    else:
+        o = Opts()
+        if workspace is not None:
+            o.workspace = workspace.data_ptr()
+            o.workspace_bytes = workspace.numel() * workspace.element_size()
+        for i, ev in enumerate(stage_events or ()):
+            o.stage_events[i] = ev.cuda_event if ev is not None else None
+        _check(_lib.infini_attn_layer_forward_ex(*args, ctypes.byref(o), _stream_handle(stream)))
     return out, M_out, z_out
+
+
+def layer_workspace_size(B, L, D_model, H, H_kv, N, d=128, mode=LINEAR) -> int:
+    return int(_lib.infini_attn_layer_workspace_size(B, L, D_model, H, H_kv, N, d, mode))
 
 
 def backward_workspace_size(B, H, L, N, d, mode=LINEAR) -> int:

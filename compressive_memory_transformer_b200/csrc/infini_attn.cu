@@ -461,7 +461,8 @@ int gemm_checks(const void* A, const void* Bm, const void* C, long long M, int N
 int layer_forward_impl(const void* x, const void* Wq, const void* Wk, const void* Wv,
                        const void* Wo, const float* beta, const float* M_in, const float* z_in,
                        void* y, float* M_out, float* z_out, int B, long long L, int D_model,
-                       int H, int H_kv, int N, int d, int mode, cudaStream_t stream) {
+                       int H, int H_kv, int N, int d, int mode, const infini_attn_opts_t* opts,
+                       cudaStream_t stream) {
   if (!x || !Wq || !Wk || !Wv || !Wo || !beta || !y) return INFINI_ERR_NULL;
   if ((M_in == nullptr) != (z_in == nullptr) || (M_out == nullptr) != (z_out == nullptr))
     return INFINI_ERR_NULL;
@@ -488,9 +489,22 @@ int layer_forward_impl(const void* x, const void* Wq, const void* Wk, const void
   int dev = 0;
   if (prepare_device(&dev) != cudaSuccess) return INFINI_ERR_CUDA;
   const size_t nq = (size_t)(rows * H * d), nkv = (size_t)(rows * H_kv * d);
+  // the projections' outputs, then the forward's own scratch
+  const size_t proj_bytes = ((2 * nq + 2 * nkv) * 2 + 255) & ~(size_t)255;
+  const int S = (int)((L + N - 1) / N);
+  int CH = 1, CL = N;
+  bf16_state_plan(B * H_kv, S, N, &CH, &CL);
+  const size_t fwd_bytes = bf16_workspace_bytes(B * H_kv, S, CH);
   Scratch sc;
-  const int st = get_scratch(sc, (2 * nq + 2 * nkv) * 2 + 256, nullptr, stream);
+  infini_attn_opts_t ws_opts;
+  memset(&ws_opts, 0, sizeof(ws_opts));
+  if (opts) ws_opts.workspace = opts->workspace, ws_opts.workspace_bytes = opts->workspace_bytes;
+  const int st = get_scratch(sc, proj_bytes + fwd_bytes, opts ? &ws_opts : nullptr, stream);
   if (st != INFINI_OK) return st;
+  infini_attn_opts_t fwd_opts;
+  memset(&fwd_opts, 0, sizeof(fwd_opts));
+  fwd_opts.workspace = static_cast<char*>(sc.ptr) + proj_bytes;
+  fwd_opts.workspace_bytes = fwd_bytes;
   auto* q = static_cast<__nv_bfloat16*>(sc.ptr);
   __nv_bfloat16* k = q + nq;
   __nv_bfloat16* v = k + nkv;
@@ -505,11 +519,15 @@ int layer_forward_impl(const void* x, const void* Wq, const void* Wk, const void
     e = bf16_gemm_launch(xb, static_cast<const __nv_bfloat16*>(Wv), v, rows, H_kv * d, D_model,
                          stream);
   if (e != cudaSuccess) return INFINI_ERR_CUDA;
+  record(opts, 0, stream);
   const int fs = forward_impl(q, k, v, beta, M_in, z_in, a, M_out, z_out, B, H, L, N, d, mode,
-                              INFINI_DTYPE_BF16, nullptr, stream, H_kv, INFINI_LAYOUT_BLHD);
+                              INFINI_DTYPE_BF16, fwd_bytes ? &fwd_opts : nullptr, stream, H_kv,
+                              INFINI_LAYOUT_BLHD);
   if (fs != INFINI_OK) return fs;
+  record(opts, 1, stream);
   e = bf16_gemm_launch(a, static_cast<const __nv_bfloat16*>(Wo), static_cast<__nv_bfloat16*>(y),
                        rows, D_model, H * d, stream);
+  record(opts, 2, stream);
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
@@ -665,7 +683,31 @@ int infini_attn_layer_forward(const void* x, const void* Wq, const void* Wk, con
                               long long L, int D_model, int H, int H_kv, int N, int d, int mode,
                               void* stream) {
   return layer_forward_impl(x, Wq, Wk, Wv, Wo, beta, M_in, z_in, y, M_out, z_out, B, L, D_model,
-                            H, H_kv, N, d, mode, static_cast<cudaStream_t>(stream));
+                            H, H_kv, N, d, mode, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int infini_attn_layer_forward_ex(const void* x, const void* Wq, const void* Wk, const void* Wv,
+                                 const void* Wo, const float* beta, const float* M_in,
+                                 const float* z_in, void* y, float* M_out, float* z_out, int B,
+                                 long long L, int D_model, int H, int H_kv, int N, int d, int mode,
+                                 const infini_attn_opts_t* opts, void* stream) {
+  return layer_forward_impl(x, Wq, Wk, Wv, Wo, beta, M_in, z_in, y, M_out, z_out, B, L, D_model,
+                            H, H_kv, N, d, mode, opts, static_cast<cudaStream_t>(stream));
+}
+
+size_t infini_attn_layer_workspace_size(int B, long long L, int D_model, int H, int H_kv, int N,
+                                        int d, int mode) {
+  (void)mode;
+  (void)D_model;
+  if (B < 1 || L < 1 || H < 1 || H_kv < 1 || N < 1 || d != 128 || H % H_kv != 0) return 0;
+  const long long rows = (long long)B * L;
+  if (rows % 128 != 0 || L >= (1LL << 31) || overflows(rows, (long long)H * d * 2)) return 0;
+  const size_t nq = (size_t)(rows * H * d), nkv = (size_t)(rows * H_kv * d);
+  const size_t proj_bytes = ((2 * nq + 2 * nkv) * 2 + 255) & ~(size_t)255;
+  const int S = (int)((L + N - 1) / N);
+  int CH = 1, CL = N;
+  bf16_state_plan(B * H_kv, S, N, &CH, &CL);
+  return proj_bytes + bf16_workspace_bytes(B * H_kv, S, CH);
 }
 
 int infini_attn_device_status(void) {

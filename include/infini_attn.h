@@ -303,6 +303,23 @@ int infini_attn_forward_ex(const void* q, const void* k, const void* v, const fl
                            int dtype, const infini_attn_opts_t* opts, void* stream);
 
 /*
+ * infini_attn_layer_forward with options: opts->workspace (256-byte aligned, at least
+ * infini_attn_layer_workspace_size(...) bytes) holds the projections' outputs and the
+ * forward's scratch instead of the stream-ordered allocator; opts->stage_events[0..2]
+ * (cudaEvent_t or NULL) are recorded after the Q/K/V projections, after the forward
+ * and after the output projection.
+ */
+int infini_attn_layer_forward_ex(const void* x, const void* Wq, const void* Wk, const void* Wv,
+                                 const void* Wo, const float* beta, const float* M_in,
+                                 const float* z_in, void* y, float* M_out, float* z_out, int B,
+                                 long long L, int D_model, int H, int H_kv, int N, int d, int mode,
+                                 const infini_attn_opts_t* opts, void* stream);
+
+/* Scratch bytes infini_attn_layer_forward needs (0 when the sizes are not supported). */
+size_t infini_attn_layer_workspace_size(int B, long long L, int D_model, int H, int H_kv, int N,
+                                        int d, int mode);
+
+/*
  * infini_attn_backward with options: opts->workspace (256-byte aligned, at least
  * infini_attn_backward_workspace_size(...) bytes) replaces the stream-ordered
  * allocation; opts->stage_events[0..2] (cudaEvent_t or NULL) are recorded on

@@ -81,3 +81,23 @@ def test_layer_matches_oracle(ia, mode):
 def test_layer_grouped_heads_with_state(ia, mode):
     """4 query heads on 2 key/value heads, two batch rows, a carried state."""
     layer_case(ia, 2, 384, 384, 4, 2, 128, mode, seed=73, state=True)
+
+
+def test_layer_workspace_and_events_give_the_same_result(ia):
+    """A caller workspace (infini_attn_layer_forward_ex) gives bitwise the same outputs
+    as the library's own scratch, and the three stage events are recorded in order."""
+    B, L, D, H, N = 1, 256, 256, 2, 128
+    x = normal((B, L, D), torch.bfloat16, 75, 0).cuda()
+    Ws = [(normal(shape, torch.float32, 75, 1 + i) / np.sqrt(shape[0])).to(torch.bfloat16).cuda()
+          for i, shape in enumerate([(D, H * 128)] * 3 + [(H * 128, D)])]
+    beta = normal((H,), torch.float32, 75, 5).cuda()
+    a = ia.infini_attn_layer_forward(x, *Ws, beta, N, DEL, H)
+    ws = torch.empty(ia.layer_workspace_size(B, L, D, H, H, N), dtype=torch.uint8, device="cuda")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for e in evs:
+        e.record()
+    b = ia.infini_attn_layer_forward(x, *Ws, beta, N, DEL, H, workspace=ws, stage_events=evs)
+    sync_ok(ia)
+    for u, w in zip(a, b):
+        assert torch.equal(u, w)
+    assert evs[0].elapsed_time(evs[1]) >= 0 and evs[1].elapsed_time(evs[2]) >= 0
