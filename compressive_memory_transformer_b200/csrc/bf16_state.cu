@@ -368,7 +368,6 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
           for (int e = 0; e < 32; ++e) rr[e] = 0u;
         }
         if (done && ok) {
-#pragma unroll
           if (half == 1) {  // G feeds a tf32 MMA in the chain: round it here, unbiased
 #pragma unroll
             for (int e = 0; e < 32; ++e) rr[e] = tf32_rna(__uint_as_float(rr[e]));
@@ -433,7 +432,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
   uint64_t* bar_seg = bars + 4; // G_s M of a whole segment done (once per segment)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
 
-  const int bh = blockIdx.x, cb = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x, cb = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
   const int c0 = 32 * cb;
   const bool delta = mode == 1;
   if (tid == 0) {
