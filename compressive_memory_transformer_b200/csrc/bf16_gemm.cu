@@ -193,14 +193,153 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
   }
 }
 
+// The same GEMM with 128 x 256 output tiles (N a multiple of 256): each k-step of 64
+// brings A [128 m][64 k] (one 16 KB box, K-major) and B [64 k][256 n] (four 8 KB
+// boxes of 64 columns, MN-major) into a 4-stage ring; four MMAs (N = 256, K = 16)
+// per k-step into one of two 256-column accumulators. Per FLOP it streams a quarter
+// less through L2 than the 128 x 128 tiles.
+constexpr int kWStages = 4;
+constexpr int kWA = 16384, kWB = 32768, kWStage = kWA + kWB;
+constexpr int kGemmWSmem = kWStages * kWStage + 256 + 1024;
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                 __nv_bfloat16* __restrict__ C, const GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWStages * kWStage);
+  // FULL [0, 4), EMPTY [4, 8), AFULL 8-9, AEMPTY 10-11 (4 warp arrivals), DRAIN 12
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int x = 0; x < 13; ++x) mbar_init(&bars[x], (x == 10 || x == 11) ? 4u : 1u);
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      int it = 0;
+      int iss[kWStages] = {0, 0, 0, 0};
+      for (unsigned t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
+        const int tm = (int)(t / (unsigned)p.tiles_n), tn = (int)(t % (unsigned)p.tiles_n);
+        for (int ks = 0; ks < p.ksteps; ++ks, ++it) {
+          const int st = it % kWStages, use = it / kWStages;
+          if (use > 0 && !mbar_wait(&bars[4 + st], (uint32_t)((use - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + st * kWStage;
+          uint8_t* sb = sa + kWA;
+          mbar_arrive_expect_tx(&bars[st], kWStage);
+          tma_load_2d(sa, &tm_a, &bars[st], 64 * ks, 128 * tm);
+#pragma unroll
+          for (int a4 = 0; a4 < 4; ++a4)
+            tma_load_2d(sb + a4 * 8192, &tm_b, &bars[st], 256 * tn + 64 * a4, 64 * ks);
+          ++iss[st];
+        }
+      }
+      if (!ok)
+        for (int st = 0; st < kWStages; ++st)
+          if (iss[st] > 0) drain_wait_g(&bars[st], (uint32_t)((iss[st] - 1) & 1));
+    }
+  } else if (warp == 5) {
+    const uint32_t idesc = idesc_f32acc(1, 0, 1, 128, 256);
+    int it = 0, lt = 0;
+    for (unsigned t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1, use = lt >> 1;
+      if (use > 0 && !mbar_wait_warp(&bars[10 + acc], (uint32_t)((use - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      const uint32_t td = tmem + (uint32_t)acc * 256;
+      for (int ks = 0; ks < p.ksteps; ++ks, ++it) {
+        const int st = it % kWStages;
+        if (!mbar_wait_warp(&bars[st], (uint32_t)((it / kWStages) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t sa = smem_u32(smem + st * kWStage), sb = sa + kWA;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(td, sdesc(sa + (uint32_t)kk * 32, 16, 1024),
+                        sdesc(sb + (uint32_t)kk * 2048, 8192, 1024), idesc,
+                        (ks > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars[4 + st]);
+          if (ks == p.ksteps - 1) mma_commit(&bars[8 + acc]);
+        }
+        __syncwarp();
+      }
+    }
+    if (elect_one()) mma_commit(&bars[12]);
+    __syncwarp();
+    drain_wait_g(&bars[12], 0);
+  } else {
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    int lt = 0;
+    for (unsigned t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++lt) {
+      const int acc = lt & 1;
+      if (!mbar_wait_warp(&bars[8 + acc], (uint32_t)((lt >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int tm = (int)(t / (unsigned)p.tiles_n), tn = (int)(t % (unsigned)p.tiles_n);
+      __nv_bfloat16* dst = C + (size_t)(128 * tm + r) * p.ldc + 256 * tn;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t v[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_ld32(tmem + (uint32_t)acc * 256 + lane_off + 128 * hf + 32 * c,
+                    *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
+        tmem_wait_ld();
+        if (hf == 1) {
+          tc_fence_before();
+          mbar_arrive_warp(&bars[10 + acc]);  // the accumulator may take the next tile
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          *reinterpret_cast<uint4*>(dst + 128 * hf + 8 * u) = make_uint4(
+              pack_bf16x2(__uint_as_float(v[8 * u]), __uint_as_float(v[8 * u + 1])),
+              pack_bf16x2(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
+              pack_bf16x2(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
+              pack_bf16x2(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7])));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // 2-D bf16 map over a row-major [rows][cols] matrix: box 64 columns x 128 rows,
 // 128-byte swizzle (one box row is one 128-byte swizzle row).
-bool make_bf16_map2(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+bool make_bf16_map2(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows = 128) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -210,12 +349,35 @@ bool make_bf16_map2(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
 }  // namespace
 
 cudaError_t bf16_gemm_set_attributes() {
-  return cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  const cudaError_t e =
+      cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(gemm_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kGemmWSmem);
 }
 
 cudaError_t bf16_gemm_launch(const __nv_bfloat16* A, const __nv_bfloat16* B, __nv_bfloat16* C,
                              long long M, int N, int K, cudaStream_t stream) {
   if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 128) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (N % 256 == 0) {  // 128 x 256 tiles
+    CUtensorMap ma, mb;
+    if (!make_bf16_map2(&ma, A, (uint64_t)M, (uint64_t)K, 128) ||
+        !make_bf16_map2(&mb, B, (uint64_t)K, (uint64_t)N, 64))
+      return cudaErrorInvalidValue;
+    GemmParams p;
+    p.tiles_n = N / 256;
+    p.ksteps = K / 64;
+    const long long tiles = (M / 128) * (long long)(N / 256);
+    if (tiles >= (1ll << 31)) return cudaErrorInvalidValue;
+    p.tiles = (unsigned)tiles;
+    p.ldc = N;
+    const unsigned grid = p.tiles < (unsigned)sms ? p.tiles : (unsigned)sms;
+    gemm_wide_kernel<<<grid, kGemmThreads, kGemmWSmem, stream>>>(ma, mb, C, p);
+    return cudaGetLastError();
+  }
   CUtensorMap ma, mb;
   if (!make_bf16_map2(&ma, A, (uint64_t)M, (uint64_t)K) ||
       !make_bf16_map2(&mb, B, (uint64_t)K, (uint64_t)N))
@@ -227,9 +389,6 @@ cudaError_t bf16_gemm_launch(const __nv_bfloat16* A, const __nv_bfloat16* B, __n
   if (tiles >= (1ll << 31)) return cudaErrorInvalidValue;
   p.tiles = (unsigned)tiles;
   p.ldc = N;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const unsigned grid = p.tiles < (unsigned)sms ? p.tiles : (unsigned)sms;
   gemm_kernel<<<grid, kGemmThreads, kGemmSmem, stream>>>(ma, mb, C, p);
   return cudaGetLastError();
