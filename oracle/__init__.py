@@ -19,7 +19,7 @@ Every step is evaluated in float64 with numpy. Matrix products use ``@`` (a
 library matmul) as a single step; nothing is blocked, fused or reordered beyond
 what the equations state.
 
-Readings of points the pages leave open (each one is listed in the design doc):
+Readings of points the pages leave open:
   * softmax scale is 1/sqrt(d_key) of the head (section 3.1 prints sqrt(d_model);
     the section 3.8 summary and the book's SDPA call use the head width);
   * the causal mask is inside the segment and includes the diagonal;
