@@ -217,9 +217,11 @@ int infini_attn_decode(const void* q, const void* k, const void* v, const float*
  * (INFINI_ERR_UNSUPPORTED otherwise); every pointer 16-byte aligned; no output may
  * overlap an input or another output (INFINI_ERR_ALIAS). L = 0 writes dbeta = 0 and
  * passes (dM_out, dz_out) through to (dM_in, dz_in). Asynchronous on `stream`;
- * scratch (about 1.6 KB per token and head) comes from the stream-ordered
- * allocator (INFINI_ERR_NOMEM). The forward's state path runs again inside the call
- * to rebuild every segment's incoming state.
+ * scratch (infini_attn_backward_workspace_size: about 0.6 to 1.1 KB per token and
+ * head, mostly per-tile partials of the state gradients) comes from the
+ * stream-ordered allocator (INFINI_ERR_NOMEM). The forward's state path runs again
+ * inside the call to rebuild every segment's incoming state. Results are bitwise
+ * reproducible (every reduction runs in a fixed order).
  */
 int infini_attn_backward(const void* q, const void* k, const void* v, const float* beta,
                          const float* M_in, const float* z_in, const void* dout,

@@ -239,3 +239,19 @@ def test_layer_forward_rejects_bad_arguments(lib, kw, code):
                         a["beta"], a["M_in"], a["z_in"], a["y"], a["M_out"], a["z_out"], a["B"],
                         a["L"], a["D_model"], a["H"], a["H_kv"], a["N"], a["d"], a["mode"],
                         None) == code
+
+
+def test_backward_and_layer_workspace_sizes_are_host_only(lib):
+    """The scratch-size queries need no device: positive for supported sizes, 0 for
+    unsupported ones, and growing with the sequence."""
+    b1 = lib.backward_workspace_size(1, 2, 2048, 512, 128, 1)
+    b2 = lib.backward_workspace_size(1, 2, 4096, 512, 128, 1)
+    assert 0 < b1 < b2
+    assert lib.backward_workspace_size(1, 2, 2048, 192, 128, 1) == 0   # N % 128
+    assert lib.backward_workspace_size(1, 2, 1000, 512, 128, 1) == 0   # L % N
+    assert lib.backward_workspace_size(1, 2, 2048, 512, 64, 1) == 0    # d
+    l1 = lib.layer_workspace_size(1, 1024, 256, 2, 1, 256)
+    l2 = lib.layer_workspace_size(1, 1024, 256, 2, 2, 256)
+    assert 0 < l1 < l2                                                  # more key/value heads
+    assert lib.layer_workspace_size(1, 100, 256, 2, 2, 256) == 0        # B * L % 128
+    assert lib.layer_workspace_size(1, 1024, 256, 3, 2, 256) == 0       # H % H_kv
