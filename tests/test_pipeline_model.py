@@ -1,0 +1,381 @@
+"""Randomized model checks of the mbarrier protocols of the pipelined kernels (the
+backward's dq and dk/dv kernels, the projection GEMM): every role of a CTA is
+written as a step function that waits on barriers by completion index, TMA copies
+and tensor-core commits complete at random later times (commits in issue order,
+each after every product issued before it), and a random scheduler interleaves
+everything. Each run must finish (no deadlock) and no barrier may ever be more than
+one phase ahead of a waiter that still has to observe an earlier phase (a parity
+wait would then miss it). This checks the protocol as written in the kernels' loop
+structure, for every tile count they meet; it runs no GPU code."""
+import random
+
+import pytest
+
+
+class Bar:
+    def __init__(self, name, count):
+        self.name, self.count, self.pending, self.done = name, count, count, 0
+
+    def arrive(self, n=1):
+        self.pending -= n
+        assert self.pending >= 0, f"{self.name}: more arrivals than the count"
+        if self.pending == 0:
+            self.done += 1
+            self.pending = self.count
+
+
+class Sim:
+    """Roles are generators yielding ('wait', bar, k) (wait for completion k, counted
+    from 0), ('arrive', bar, n), ('tma', bar) (a copy that completes bar later),
+    ('mma',) (a product), ('commit', bar) (arrives on bar once every earlier product of
+    the CTA is done) or ('named', id, members) (a CTA-level named barrier)."""
+
+    def __init__(self, seed):
+        self.rng = random.Random(seed)
+        self.bars = {}
+        self.tma = []          # pending copies (bar)
+        self.mma_queue = []    # issued products and commits, in order
+
+    def bar(self, name, count=1):
+        self.bars[name] = Bar(name, count)
+        return self.bars[name]
+
+    def run(self, roles, max_steps=2_000_000):
+        state = {r: None for r in roles}   # the pending request of each role
+        for step in range(max_steps):
+            ready = []
+            for r, req in list(state.items()):
+                if req is None:
+                    try:
+                        req = next(roles[r])
+                    except StopIteration:
+                        del state[r]
+                        continue
+                    state[r] = req
+                if req[0] == 'wait':
+                    b, k = req[1], req[2]
+                    # a waiter for completion k must not find the barrier past k + 1:
+                    # its parity would then match a later phase
+                    assert b.done <= k + 1, f"{b.name}: phase skipped (waiter for {k}, done {b.done})"
+                    if b.done >= k + 1:
+                        ready.append(r)
+                elif req[0] == 'named':
+                    nid, members = req[1], req[2]
+                    arrived = [x for x in members if x in state and state[x] is not None
+                               and state[x][0] == 'named' and state[x][1] == nid]
+                    if len(arrived) == len(members):
+                        ready.append(r)
+                else:
+                    ready.append(r)
+            events = []  # asynchronous completions (named apart from the roles)
+            if self.tma:
+                events.append('<copy done>')
+            if self.mma_queue:
+                events.append('<product done>')
+            if not state and not self.tma and not self.mma_queue:
+                return step
+            if not ready and not events:
+                raise AssertionError("deadlock: " + ", ".join(
+                    f"{r} waits {req[1].name if hasattr(req[1], 'name') else req[1]}"
+                    f"#{req[2] if len(req) > 2 else ''}" for r, req in state.items()))
+            choice = self.rng.choice(ready + events)
+            if choice == '<copy done>':
+                b = self.tma.pop(self.rng.randrange(len(self.tma)))
+                b.arrive()
+            elif choice == '<product done>':
+                item = self.mma_queue.pop(0)   # in issue order
+                if item is not None:
+                    item.arrive()
+            else:
+                req = state[choice]
+                kind = req[0]
+                if kind == 'arrive':
+                    req[1].arrive(req[2])
+                elif kind == 'tma':
+                    self.tma.append(req[1])
+                elif kind == 'mma':
+                    self.mma_queue.append(None)
+                elif kind == 'commit':
+                    self.mma_queue.append(req[1])
+                elif kind == 'named':
+                    nid, members = req[1], req[2]
+                    for m in members:
+                        state[m] = None
+                    continue
+                state[choice] = None
+        raise AssertionError("did not finish")
+
+
+# ------------------------------------------------------------------------------
+# dq kernel: loads n = 0 .. 2 nk - 1 (two sweeps over nk key tiles), halves h = 2n + a
+# ------------------------------------------------------------------------------
+def dq_roles(sim, nk):
+    nl, nh = 2 * nk, 4 * nk
+    ONCE, X, DONE, M1, M2 = (sim.bar(n) for n in ("once", "x", "done", "m1", "m2"))
+    FULL = [sim.bar(f"full{i}") for i in range(2)]
+    FREE = [sim.bar(f"free{i}") for i in range(2)]
+    SFULL = [sim.bar(f"sfull{i}") for i in range(2)]
+    PFULL = [sim.bar(f"pfull{i}", 4) for i in range(2)]
+    SK, SK2 = sim.bar("sk", 8), sim.bar("sk2", 8)
+
+    def producer():
+        yield ('tma', ONCE)
+        for n in range(nl):
+            st = n & 1
+            if n >= 2:
+                yield ('wait', FREE[st], (n >> 1) - 1)
+            yield ('tma', FULL[st])
+        yield ('wait', FREE[0], (nl - 2) >> 1)
+        yield ('tma', X)
+
+    def mma():
+        def issue_sdp(h):
+            n, a = h >> 1, h & 1
+            st = n & 1
+            if a == 0:
+                yield ('wait', FULL[st], n >> 1)
+            yield ('mma',)
+            yield ('commit', SFULL[a])
+            if n < nk and a == 1:
+                yield ('commit', FREE[st])
+        yield ('wait', ONCE, 0)
+        yield from issue_sdp(0)
+        yield from issue_sdp(1)
+        for h in range(nh):
+            n, a = h >> 1, h & 1
+            yield ('wait', PFULL[a], n)
+            if n >= nk:
+                yield ('mma',)
+                if a == 1:
+                    yield ('commit', FREE[n & 1])
+            if h + 2 < nh:
+                yield from issue_sdp(h + 2)
+        yield ('commit', DONE)
+        yield ('wait', X, 0)
+        yield ('wait', SK, 0)
+        yield ('mma',)
+        yield ('commit', M1)
+        yield ('wait', SK2, 0)
+        yield ('mma',)
+        yield ('commit', M2)
+
+    wgs = ("wg0", "wg1")
+
+    def wg(w):
+        for n in range(nk):
+            yield ('wait', SFULL[w], n)
+            yield ('arrive', PFULL[w], 4)
+        yield ('named', 'merge', wgs)
+        for n in range(nk, nl):
+            yield ('wait', SFULL[w], n)
+            yield ('arrive', PFULL[w], 4)
+        yield ('wait', DONE, 0)
+        yield ('wait', X, 0)
+        yield ('named', 'den', wgs)
+        yield ('arrive', SK, 4)
+        yield ('wait', M1, 0)
+        yield ('named', 'dd', wgs)
+        yield ('arrive', SK2, 4)
+        yield ('wait', M2, 0)
+        yield ('named', 'sums', wgs)
+
+    return {"producer": producer(), "mma": mma(), "wg0": wg(0), "wg1": wg(1)}
+
+
+# ------------------------------------------------------------------------------
+# dk/dv kernel: loads n = 0 .. nl - 1 (query tiles at or after the key tile)
+# ------------------------------------------------------------------------------
+def dkdv_roles(sim, nl, delta):
+    nh = 2 * nl
+    sx = nl & 1
+    ONCE, X, DONE, M1, M2 = (sim.bar(n) for n in ("once", "x", "done", "m1", "m2"))
+    FULL = [sim.bar(f"full{i}") for i in range(2)]
+    FREE = [sim.bar(f"free{i}") for i in range(2)]
+    SFULL = [sim.bar(f"sfull{i}") for i in range(2)]
+    PFULL = [sim.bar(f"pfull{i}", 4) for i in range(2)]
+    SK, SK2 = sim.bar("sk", 8), sim.bar("sk2", 8)
+
+    def producer():
+        yield ('tma', ONCE)
+        for n in range(nl):
+            st = n & 1
+            if n >= 2:
+                yield ('wait', FREE[st], (n >> 1) - 1)
+            yield ('tma', FULL[st])
+        if nl >= 2:
+            yield ('wait', FREE[sx], (nl - 2) >> 1)
+        yield ('tma', X)
+
+    def mma():
+        def issue_sdp(h):
+            n, a = h >> 1, h & 1
+            if a == 0:
+                yield ('wait', FULL[n & 1], n >> 1)
+            yield ('mma',)
+            yield ('commit', SFULL[a])
+        yield ('wait', ONCE, 0)
+        yield from issue_sdp(0)
+        yield from issue_sdp(1)
+        for h in range(nh):
+            n, a = h >> 1, h & 1
+            yield ('wait', PFULL[a], n)
+            yield ('mma',)
+            if a == 1:
+                yield ('commit', FREE[n & 1])
+            if h + 2 < nh:
+                yield from issue_sdp(h + 2)
+        yield ('commit', DONE)
+        yield ('wait', X, 0)
+        yield ('wait', SK, 0)
+        yield ('mma',)
+        yield ('commit', M1)
+        if delta:
+            yield ('wait', SK2, 0)
+            yield ('mma',)
+            yield ('commit', M2)
+
+    wgs = ("wg0", "wg1")
+
+    def wg(w):
+        for n in range(nl):
+            yield ('wait', FULL[n & 1], n >> 1)
+            yield ('wait', SFULL[w], n)
+            yield ('arrive', PFULL[w], 4)
+        yield ('wait', DONE, 0)
+        if delta:
+            yield ('wait', X, 0)
+        yield ('named', 'den', wgs)
+        yield ('arrive', SK, 4)
+        if delta:
+            yield ('wait', M1, 0)
+            yield ('named', 'dd', wgs)
+            yield ('arrive', SK2, 4)
+            yield ('named', 'sdd', wgs)
+            yield ('named', 'gz', wgs)
+            yield ('wait', M2, 0)
+        else:
+            yield ('wait', M1, 0)
+
+    return {"producer": producer(), "mma": mma(), "wg0": wg(0), "wg1": wg(1)}
+
+
+# ------------------------------------------------------------------------------
+# projection GEMM: a CTA's output tiles, k-steps through a ring, two accumulators
+# ------------------------------------------------------------------------------
+def gemm_roles(sim, tiles, ksteps, stages):
+    FULL = [sim.bar(f"full{i}") for i in range(stages)]
+    EMPTY = [sim.bar(f"empty{i}") for i in range(stages)]
+    AFULL = [sim.bar(f"afull{i}") for i in range(2)]
+    AEMPTY = [sim.bar(f"aempty{i}", 4) for i in range(2)]
+
+    def producer():
+        it = 0
+        for _ in range(tiles):
+            for _ in range(ksteps):
+                st, use = it % stages, it // stages
+                if use > 0:
+                    yield ('wait', EMPTY[st], use - 1)
+                yield ('tma', FULL[st])
+                it += 1
+
+    def mma():
+        it = 0
+        for lt in range(tiles):
+            acc, use = lt & 1, lt >> 1
+            if use > 0:
+                yield ('wait', AEMPTY[acc], use - 1)
+            for ks in range(ksteps):
+                st = it % stages
+                yield ('wait', FULL[st], it // stages)
+                yield ('mma',)
+                yield ('commit', EMPTY[st])
+                if ks == ksteps - 1:
+                    yield ('commit', AFULL[acc])
+                it += 1
+
+    def epilogue():
+        for lt in range(tiles):
+            yield ('wait', AFULL[lt & 1], lt >> 1)
+            yield ('arrive', AEMPTY[lt & 1], 4)
+
+    return {"producer": producer(), "mma": mma(), "epilogue": epilogue()}
+
+
+@pytest.mark.parametrize("nk", [1, 2, 3, 4, 7, 16])
+def test_dq_pipeline_protocol(nk):
+    for seed in range(40):
+        sim = Sim(seed * 1000 + nk)
+        sim.run(dq_roles(sim, nk))
+
+
+@pytest.mark.parametrize("delta", [False, True])
+@pytest.mark.parametrize("nl", [1, 2, 3, 4, 7, 16])
+def test_dkdv_pipeline_protocol(nl, delta):
+    for seed in range(40):
+        sim = Sim(seed * 1000 + nl + 100 * delta)
+        sim.run(dkdv_roles(sim, nl, delta))
+
+
+@pytest.mark.parametrize("tiles,ksteps,stages", [(1, 1, 3), (3, 8, 3), (5, 16, 4), (2, 2, 4),
+                                                 (7, 1, 3)])
+def test_gemm_pipeline_protocol(tiles, ksteps, stages):
+    for seed in range(40):
+        sim = Sim(seed * 1000 + tiles * 10 + ksteps)
+        sim.run(gemm_roles(sim, tiles, ksteps, stages))
+
+
+def test_model_detects_a_phase_skip():
+    """Planted mistake: the dq producer no longer waits for the ring stage to be freed
+    before refilling it (FULL then completes twice before the MMA warp has seen the
+    first completion)."""
+    def broken(sim, nk):
+        roles = dq_roles(sim, nk)
+        FULL = [sim.bars["full0"], sim.bars["full1"]]
+        ONCE = sim.bars["once"]
+
+        def producer():
+            yield ('tma', ONCE)
+            for n in range(2 * nk):
+                yield ('tma', FULL[n & 1])
+        roles["producer"] = producer()
+        return roles
+    failures = 0
+    for seed in range(40):
+        sim = Sim(seed)
+        try:
+            sim.run(broken(sim, 4))
+        except AssertionError:
+            failures += 1
+    assert failures > 0
+
+
+def test_model_detects_a_deadlock():
+    """Planted mistake: the dk/dv MMA warp frees a ring stage only after the next
+    tile's scores, which wait for that stage to be refilled."""
+    def broken(sim, nl):
+        roles = dkdv_roles(sim, nl, False)
+        FULL = [sim.bars["full0"], sim.bars["full1"]]
+        FREE = [sim.bars["free0"], sim.bars["free1"]]
+        SFULL = [sim.bars["sfull0"], sim.bars["sfull1"]]
+        PFULL = [sim.bars["pfull0"], sim.bars["pfull1"]]
+        ONCE, DONE = sim.bars["once"], sim.bars["done"]
+
+        def mma():
+            yield ('wait', ONCE, 0)
+            for n in range(nl):
+                yield ('wait', FULL[n & 1], n >> 1)
+                for a in range(2):
+                    yield ('mma',)
+                    yield ('commit', SFULL[a])
+                for a in range(2):
+                    yield ('wait', PFULL[a], n)
+                    yield ('mma',)
+                if n + 2 < nl:
+                    yield ('wait', FULL[n & 1], (n + 2) >> 1)  # waits for its own refill
+                yield ('commit', FREE[n & 1])
+            yield ('commit', DONE)
+        roles["mma"] = mma()
+        return roles
+    with pytest.raises(AssertionError):
+        sim = Sim(1)
+        sim.run(broken(sim, 4))
