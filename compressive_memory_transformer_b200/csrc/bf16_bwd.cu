@@ -400,10 +400,12 @@ dz_bwd_kernel(const float* __restrict__ Gzp, const float* __restrict__ gzk, cons
 // cores compute half h + 1 (and the gradient products of half h - 1). Warp 8 is the
 // TMA producer, warp 9 allocates tensor memory and issues every MMA from one
 // elected lane. Barriers: SFULL[b] (scores of a half in buffer b ready, one
-// tcgen05.commit), PFULL[b] (the half's bf16 operand written over the buffer, four
-// warp arrivals); each completes once per use of its buffer and cannot run a phase
-// ahead of its waiter (the next use of a buffer is issued only after the previous
-// one's PFULL, and its PFULL needs the next SFULL).
+// tcgen05.commit), PFULL[b] (the warpgroup is done with the buffer: its values read
+// and, where a product follows, the half's bf16 operand written over them; four warp
+// arrivals); each completes once per use of its buffer and cannot run a phase ahead
+// of its waiter (the next use of a buffer is issued only after the previous one's
+// PFULL, and its PFULL needs the next SFULL). tests/test_pipeline_model.py checks
+// these protocols on the CPU.
 // ---------------------------------------------------------------------------
 constexpr int kPipeThreads = 320;
 constexpr uint32_t kIdN64 = idesc_f32acc(1, 0, 0, 128, 64);
