@@ -115,3 +115,13 @@ def test_backward_zero_length(ia):
     sync_ok(ia)
     assert torch.count_nonzero(r[3]) == 0
     assert torch.equal(r[4], dM) and torch.equal(r[5], dz)
+
+
+@pytest.mark.parametrize("mode", [LIN, DEL])
+@pytest.mark.parametrize("state", [False, True])
+def test_backward_single_segment(ia, mode, state):
+    """L = N (one segment, S = 1): from the zero state every row retrieves the constant 0
+    and no gradient reaches the state through the retrieval or the Delta term; with a
+    carried state both paths carry weight. Final-state gradients included."""
+    got, ref = run(ia, 1, 2, 256, 256, mode, seed=99 + mode, state=state, state_grad=True)
+    check(got, ref, f"single segment mode={mode} state={state}")
