@@ -1,5 +1,6 @@
 """Randomized model checks of the mbarrier protocols of the pipelined kernels (the
-backward's dq and dk/dv kernels, the projection GEMM): every role of a CTA is
+forward's fused attention kernel, the backward's dq and dk/dv kernels, the
+projection GEMM): every role of a CTA is
 written as a step function that waits on barriers by completion index, TMA copies
 and tensor-core commits complete at random later times (commits in issue order,
 each after every product issued before it), and a random scheduler interleaves
@@ -379,3 +380,264 @@ def test_model_detects_a_deadlock():
     with pytest.raises(AssertionError):
         sim = Sim(1)
         sim.run(broken(sim, 4))
+
+
+# ------------------------------------------------------------------------------
+# the forward attention kernel (one persistent CTA walking its list of query tiles)
+# ------------------------------------------------------------------------------
+def attn_roles(sim, tiles):
+    """tiles: list of (nkv, tma_out) per query tile of the CTA's list."""
+    QFULL, QEMPTY = sim.bar("qfull"), sim.bar("qempty", 9)   # QK commit + 8 softmax warps
+    KFULL = [sim.bar(f"kfull{i}") for i in range(2)]
+    SFREE = [sim.bar(f"sfree{i}") for i in range(2)]
+    VFULL = [sim.bar(f"vfull{i}") for i in range(2)]
+    VEMPTY = [sim.bar(f"vempty{i}") for i in range(2)]
+    SFULL = [sim.bar(f"sfull{i}") for i in range(2)]
+    PFULL, PVDONE, RDONE = sim.bar("pfull", 8), sim.bar("pvdone"), sim.bar("rdone")
+    SQFULL = sim.bar("sqfull", 8)
+    DRAIN = sim.bar("drain", 2)
+    PAIR = [sim.bar(f"pair{i}", 2) for i in range(4)]
+    OFULL = [sim.bar(f"ofull{i}", 4) for i in range(2)]
+    OFREE = [sim.bar(f"ofree{i}") for i in range(2)]
+    STORE = [sim.bar(f"storeread{i}") for i in range(2)]  # a TMA store has read its tile
+    ntiles = len(tiles)
+
+    def producer():
+        k_use, v_use = [0, 0], [0, 0]
+        kst, vst = [0], [0]
+
+        def issue_k():
+            st = kst[0]
+            if k_use[st] > 0:
+                yield ('wait', SFULL[st], k_use[st] - 1)
+            yield ('tma', KFULL[st])
+            k_use[st] += 1
+            kst[0] ^= 1
+
+        def issue_v():
+            st = vst[0]
+            if v_use[st] > 0:
+                yield ('wait', VEMPTY[st], v_use[st] - 1)
+            yield ('tma', VFULL[st])
+            v_use[st] += 1
+            vst[0] ^= 1
+        for tc, (nkv, _) in enumerate(tiles):
+            if tc > 0:
+                yield ('wait', QEMPTY, tc - 1)
+            yield ('tma', QFULL)                   # Q (and z), after the descriptor slot
+            yield from issue_k()
+            if nkv >= 2:
+                yield from issue_k()
+            yield from issue_v()                   # item 0: M_hi
+            for j in range(nkv):
+                if j + 2 < nkv:
+                    yield from issue_k()
+                yield from issue_v()               # V_j
+        if ntiles > 0:
+            yield ('wait', QEMPTY, ntiles - 1)
+        yield ('arrive', QFULL, 1)                 # the end marker
+
+    def qk():
+        n = 0
+        for tc in range(ntiles + 1):
+            yield ('wait', QFULL, tc)
+            if tc == ntiles:
+                break
+            nkv = tiles[tc][0]
+            for j in range(nkv):
+                st = n & 1
+                if n >= 2:
+                    yield ('wait', SFREE[st], (n >> 1) - 1)
+                yield ('wait', KFULL[st], n >> 1)
+                yield ('mma', 'qk')
+                yield ('commit', SFULL[st], 'qk')
+                if j == nkv - 1:
+                    yield ('commit', QEMPTY, 'qk')
+                n += 1
+        yield ('commit', DRAIN, 'qk')
+        yield ('wait', DRAIN, 0)
+
+    def pv():
+        n, vit = 0, 0
+        for tc in range(ntiles + 1):
+            yield ('wait', SQFULL, tc)
+            if tc == ntiles:
+                break
+            nkv = tiles[tc][0]
+            st = vit & 1
+            yield ('wait', VFULL[st], vit >> 1)
+            yield ('mma', 'pv')                       # R = sigma(Q) M_hi
+            yield ('commit', VEMPTY[st], 'pv')
+            yield ('commit', RDONE, 'pv')
+            vit += 1
+            for j in range(nkv):
+                st = vit & 1
+                yield ('wait', PFULL, n)
+                yield ('wait', VFULL[st], vit >> 1)
+                yield ('mma', 'pv')
+                yield ('commit', VEMPTY[st], 'pv')
+                yield ('commit', PVDONE, 'pv')
+                yield ('commit', SFREE[n & 1], 'pv')
+                vit += 1
+                n += 1
+        yield ('commit', DRAIN, 'pv')
+        yield ('wait', DRAIN, 0)
+
+    def softmax(w):
+        half, wq = w // 4, w % 4
+        issuer = wq == 0
+        kc, pph, oc, stores = 0, 0, 0, 0
+        yield ('wait', QFULL, 0)
+        if ntiles == 0:
+            yield ('arrive', SQFULL, 1)
+            return
+        yield ('arrive', QEMPTY, 1)                   # sigma(Q) of tile 0
+        yield ('arrive', SQFULL, 1)
+        for tc, (nkv, tma_out) in enumerate(tiles):
+            for j in range(nkv):
+                yield ('wait', SFULL[kc & 1], kc >> 1)
+                kc += 1
+                yield ('arrive', PAIR[wq], 1)
+                yield ('wait', PAIR[wq], pph)
+                pph += 1
+                if j > 0:
+                    yield ('wait', PVDONE, kc - 2)
+                yield ('arrive', PFULL, 1)
+            yield ('arrive', PAIR[wq], 1)              # epilogue: row sums exchanged
+            yield ('wait', PAIR[wq], pph)
+            pph += 1
+            yield ('wait', PVDONE, kc - 1)
+            yield ('wait', RDONE, tc)
+            if tma_out:
+                if oc > 0:
+                    if issuer:
+                        yield ('wait', STORE[half], stores - 1)   # its last store has read
+                        yield ('arrive', OFREE[half], 1)
+                    yield ('wait', OFREE[half], oc - 1)
+                yield ('arrive', OFULL[half], 1)
+                if issuer:
+                    yield ('wait', OFULL[half], oc)
+                    yield ('tma', STORE[half])                     # TMA store reads the tile
+                    stores += 1
+                oc += 1
+            yield ('wait', QFULL, tc + 1)
+            if tc + 1 == ntiles:
+                yield ('arrive', SQFULL, 1)            # the end marker reaches the P V warp
+            else:
+                yield ('arrive', QEMPTY, 1)            # sigma(Q) of the next tile
+                yield ('arrive', SQFULL, 1)
+
+    roles = {"producer": producer(), "qk": qk(), "pv": pv()}
+    for w in range(8):
+        roles[f"softmax{w}"] = softmax(w)
+    return roles
+
+
+class SimPerWarp(Sim):
+    """Products and commits complete in issue order per issuing warp (the two MMA
+    warps issue independently)."""
+
+    def run(self, roles, max_steps=4_000_000):
+        queues = {}
+
+        # route ('mma', who) and ('commit', bar, who) into per-warp queues
+        def gen_wrap(g):
+            for req in g:
+                if req[0] == 'mma':
+                    yield ('mma_w', req[1])
+                elif req[0] == 'commit' and len(req) == 3:
+                    yield ('commit_w', req[1], req[2])
+                else:
+                    yield req
+        roles = {k: gen_wrap(v) for k, v in roles.items()}
+        state = {r: None for r in roles}
+        for step in range(max_steps):
+            ready = []
+            for r, req in list(state.items()):
+                if req is None:
+                    try:
+                        req = next(roles[r])
+                    except StopIteration:
+                        del state[r]
+                        continue
+                    state[r] = req
+                if req[0] == 'wait':
+                    b, k = req[1], req[2]
+                    assert b.done <= k + 1, f"{b.name}: phase skipped (waiter for {k}, done {b.done})"
+                    if b.done >= k + 1:
+                        ready.append(r)
+                else:
+                    ready.append(r)
+            events = ['<copy done>'] if self.tma else []
+            events += [f'<product done {w}>' for w, q in queues.items() if q]
+            if not state and not self.tma and not any(queues.values()):
+                return step
+            if not ready and not events:
+                raise AssertionError("deadlock: " + ", ".join(
+                    f"{r} waits {req[1].name}#{req[2]}" for r, req in state.items()
+                    if req[0] == 'wait'))
+            choice = self.rng.choice(ready + events)
+            if choice == '<copy done>':
+                self.tma.pop(self.rng.randrange(len(self.tma))).arrive()
+            elif choice.startswith('<product done'):
+                w = choice[len('<product done '):-1]
+                item = queues[w].pop(0)
+                if item is not None:
+                    item.arrive()
+            else:
+                req = state[choice]
+                if req[0] == 'arrive':
+                    req[1].arrive(req[2])
+                elif req[0] == 'tma':
+                    self.tma.append(req[1])
+                elif req[0] == 'mma_w':
+                    queues.setdefault(req[1], []).append(None)
+                elif req[0] == 'commit_w':
+                    queues.setdefault(req[2], []).append(req[1])
+                state[choice] = None
+        raise AssertionError("did not finish")
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_attention_kernel_protocol(seed):
+    """Random tile lists of a persistent CTA: 0 to 6 tiles of 1 to 6 key tiles each,
+    whole tiles (TMA-stored through shared memory) and ragged ones (stored directly)."""
+    rng = random.Random(seed)
+    tiles = [(rng.randint(1, 6), rng.random() < 0.8) for _ in range(rng.randint(0, 6))]
+    sim = SimPerWarp(seed)
+    sim.run(attn_roles(sim, tiles))
+
+
+def test_attention_model_detects_a_missing_sfree_wait():
+    """Planted mistake: Q K^T no longer waits for the P V that last read its S buffer."""
+    def broken(sim, tiles):
+        roles = attn_roles(sim, tiles)
+        QFULL, KFULL = sim.bars["qfull"], [sim.bars["kfull0"], sim.bars["kfull1"]]
+        SFULL = [sim.bars["sfull0"], sim.bars["sfull1"]]
+        QEMPTY, DRAIN = sim.bars["qempty"], sim.bars["drain"]
+
+        def qk():
+            n = 0
+            for tc in range(len(tiles) + 1):
+                yield ('wait', QFULL, tc)
+                if tc == len(tiles):
+                    break
+                for j in range(tiles[tc][0]):
+                    yield ('wait', KFULL[n & 1], n >> 1)
+                    yield ('mma', 'qk')
+                    yield ('commit', SFULL[n & 1], 'qk')
+                    if j == tiles[tc][0] - 1:
+                        yield ('commit', QEMPTY, 'qk')
+                    n += 1
+            yield ('commit', DRAIN, 'qk')
+            yield ('wait', DRAIN, 0)
+        roles["qk"] = qk()
+        return roles
+    failures = 0
+    for seed in range(30):
+        sim = SimPerWarp(seed)
+        try:
+            sim.run(broken(sim, [(6, True), (5, True), (6, False)]))
+        except AssertionError:
+            failures += 1
+    assert failures > 0
