@@ -1,6 +1,6 @@
 """Randomized model checks of the mbarrier protocols of the pipelined kernels (the
-forward's fused attention kernel, the backward's dq and dk/dv kernels, the
-projection GEMM): every role of a CTA is
+forward's fused attention kernel, its state kernel and state chain, the backward's
+dq and dk/dv kernels and reverse chain, the projection GEMM): every role of a CTA is
 written as a step function that waits on barriers by completion index, TMA copies
 and tensor-core commits complete at random later times (commits in issue order,
 each after every product issued before it), and a random scheduler interleaves
@@ -641,3 +641,93 @@ def test_attention_model_detects_a_missing_sfree_wait():
         except AssertionError:
             failures += 1
     assert failures > 0
+
+
+# ------------------------------------------------------------------------------
+# the forward's state kernel (one chunk of one segment) and the state chains
+# ------------------------------------------------------------------------------
+def state_roles(sim, nslab, stages=3, conv_warps=16):
+    FULL = [sim.bar(f"full{i}") for i in range(stages)]
+    CONV = [sim.bar(f"conv{i}", conv_warps) for i in range(stages)]
+    MMA = [sim.bar(f"mma{i}") for i in range(stages)]
+    DONE = sim.bar("done")
+
+    def producer():
+        for sl in range(nslab):
+            stg = sl % stages
+            if sl >= stages:
+                yield ('wait', MMA[stg], sl // stages - 1)
+            yield ('tma', FULL[stg])
+
+    def mma():
+        for sl in range(nslab):
+            stg = sl % stages
+            yield ('wait', CONV[stg], sl // stages)
+            yield ('mma',)
+            yield ('commit', MMA[stg])
+        yield ('commit', DONE)
+
+    def converter():
+        for sl in range(nslab):
+            stg = sl % stages
+            yield ('wait', FULL[stg], sl // stages)
+            yield ('arrive', CONV[stg], 1)  # operands converted in place
+        yield ('wait', DONE, 0)
+
+    roles = {"producer": producer(), "mma": mma()}
+    for w in range(conv_warps):
+        roles[f"conv{w}"] = converter()
+    return roles
+
+
+def chain_roles(sim, S, CH, delta=True):
+    """The forward chain and the backward's reverse chain share this protocol: per
+    segment the four row warps write their block of M (or dM) transposed and arrive;
+    the MMA warp multiplies by the segment's G chunks (double-buffered TMA, the next
+    chunk's load issued before waiting for the current one) and signals the segment."""
+    G = [sim.bar(f"g{i}") for i in range(2)]
+    MT, MMA, SEG = sim.bar("mt", 4), sim.bar("mma"), sim.bar("seg")
+
+    def mma():
+        if not delta:
+            return
+        total, n = S * CH, 0
+        yield ('tma', G[0])
+        for q in range(S):
+            yield ('wait', MT, q)
+            for c in range(CH):
+                buf = n & 1
+                if n + 1 < total:
+                    yield ('tma', G[buf ^ 1])   # the other buffer's last MMA is done
+                yield ('wait', G[buf], n >> 1)
+                yield ('mma',)
+                yield ('commit', MMA)
+                if c == CH - 1:
+                    yield ('commit', SEG)
+                yield ('wait', MMA, n)
+                n += 1
+
+    def rows():
+        for q in range(S):
+            if delta:
+                yield ('arrive', MT, 1)         # the M block transposed, for G M
+                yield ('wait', SEG, q)
+
+    roles = {"mma": mma()}
+    for w in range(4):
+        roles[f"rows{w}"] = rows()
+    return roles
+
+
+@pytest.mark.parametrize("nslab", [0, 1, 2, 3, 4, 7, 32])
+def test_state_kernel_protocol(nslab):
+    for seed in range(20):
+        sim = Sim(seed * 100 + nslab)
+        sim.run(state_roles(sim, nslab))
+
+
+@pytest.mark.parametrize("S,CH", [(1, 1), (1, 8), (3, 2), (16, 1), (5, 4)])
+def test_chain_protocol(S, CH):
+    for seed in range(20):
+        sim = Sim(seed * 100 + S * 10 + CH)
+        sim.run(chain_roles(sim, S, CH))
