@@ -255,3 +255,24 @@ def test_backward_and_layer_workspace_sizes_are_host_only(lib):
     assert 0 < l1 < l2                                                  # more key/value heads
     assert lib.layer_workspace_size(1, 100, 256, 2, 2, 256) == 0        # B * L % 128
     assert lib.layer_workspace_size(1, 1024, 256, 3, 2, 256) == 0       # H % H_kv
+
+
+def test_binding_rejects_bad_tensors_before_the_library(lib):
+    """The Python binding of the gradient, the layer and the GEMM raises ValueError on
+    host tensors, wrong dtypes or mismatched shapes without calling into CUDA."""
+    import torch
+    bf = torch.zeros((1, 1, 128, 128), dtype=torch.bfloat16)
+    beta = torch.zeros(1)
+    with pytest.raises(ValueError):
+        lib.infini_attn_backward(bf, bf, bf, beta, 128, 0, bf)            # host tensors
+    with pytest.raises(ValueError):
+        lib.infini_attn_gemm_bf16(torch.zeros((128, 128), dtype=torch.bfloat16),
+                                  torch.zeros((256, 128), dtype=torch.bfloat16))  # K mismatch
+    with pytest.raises(ValueError):
+        lib.infini_attn_gemm_bf16(torch.zeros((128, 128)), torch.zeros((128, 128)))  # fp32
+    x = torch.zeros((1, 128, 256), dtype=torch.bfloat16)
+    W = torch.zeros((256, 256), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        lib.infini_attn_layer_forward(x, W, W, W, W, torch.zeros(2), 128, 0, 2)  # host tensors
+    with pytest.raises(ValueError):
+        lib.infini_attn_layer_forward(x[0], W, W, W, W, torch.zeros(2), 128, 0, 2)  # not 3-d
