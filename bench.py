@@ -8,6 +8,10 @@ modes over the same batch: infini_attn_forward in Linear mode, then in
 Linear+Delta mode (each = sigma(K) sums, z scan, per-segment state GEMMs, state
 chain, fused attention + retrieval + gate). Tokens per step = 2 * B * L.
 
+At N = 1 the line also carries, under "configs", the other full-size workloads
+timed in the same run: the 1M-token stream of 512 graph-captured step calls, the
+8B-model 500K forward and the segment-length sweep (--no-extra skips them).
+
 Prints one JSON line (rank 0). Under torchrun (N > 1) every rank runs its own
 batch (the path shards by (batch, head) with no exchange: weak scaling), the
 ranks meet at barriers around the timed region, and the time is the max over
@@ -191,7 +195,8 @@ def cpu_baseline(inp_cpu):
     heads = [(0, 0), (1, 3), (2, 5), (3, 7)]
     secs, th = oracle_sample(inp_cpu["q"], inp_cpu["k"], inp_cpu["v"], inp_cpu["beta"], heads,
                              (0, 1))
-    return {"value": (th / H) / secs, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    return {"value": (th / H) / secs, "unit": UNIT, "cores": usable_cores(),
+            "blas_threads": blas_threads(), "kind": "oracle",
             "sample": f"{len(heads)} of {B * H} heads (full L={L}) x Linear and Linear+Delta, "
                       f"fp64 numpy oracle, {secs:.1f} s; tokens = token-heads / H"}
 
@@ -312,14 +317,16 @@ def run_ours(args, rank, world, device):
         "config": {"workload": WORKLOAD, "B": B, "H": H, "d": D, "N": N, "L": L,
                    "modes": ["linear", "delta"], "per_rank_batch": B,
                    "l2": "inputs larger than L2 (q/k/v 768 MiB per forward), no flush"},
+        # the timed region is tens of milliseconds at full clocks: the burst peak is
+        # the denominator; the seconds-long power-capped figure is given beside it
         "roofline": {"kernel": "attn_kernel (fused local attention + retrieval + gate)",
-                     "bound": "tensor", "achieved": achieved, "peak": peak_sust,
-                     "unit": "TFLOP/s", "frac": achieved / peak_sust,
+                     "bound": "tensor", "achieved": achieved, "peak": peak_burst,
+                     "unit": "TFLOP/s", "frac": achieved / peak_burst,
                      "traffic": measured_traffic(
                          "compressive_memory_transformer_b200/csrc/bf16_attn.cu",
                          "attn_kernel_c2_traffic.json"),
-                     "peak_kind": f"bf16 dense, sustained, {peak_src}",
-                     "frac_of_burst_peak": achieved / peak_burst,
+                     "peak_kind": f"bf16 dense, burst, {peak_src}",
+                     "frac_of_sustained_peak": achieved / peak_sust,
                      "flops_per_launch": attn_flops_per_launch(),
                      "avg_launch_ms": avg_attn_s * 1e3},
         "modes": {
@@ -333,6 +340,12 @@ def run_ours(args, rank, world, device):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if world == 1 and not args.no_extra:
+        # the other full-size workloads of the configuration list, each timed live in
+        # this run (kernel fractions of the burst peak): they are reported beside the
+        # headline, which stays the 1B-layer step above
+        line["configs"] = {"c3_stream": extra_c3(args, device), "c4_8b_500k": extra_c4(args, device),
+                           "c5_sweep": extra_c5(args, device)}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline({"q": q.cpu(), "k": k.cpu(), "v": v.cpu(),
                                              "beta": beta.cpu()})
@@ -373,8 +386,8 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": B, "H": H, "d": D, "N": N, "L": L,
                    "modes": ["linear", "delta"]},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": usable_cores(),
+                         "blas_threads": blas_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -392,9 +405,149 @@ def _timed(fn, reps, stream):
     return a.elapsed_time(b_) / reps
 
 
+def _attn_tflops(Bc, Hc, Lc, Nc, ms):
+    """Algorithmic TFLOP/s of the fused attention kernel over ms milliseconds."""
+    return Bc * Hc * Lc * (2 * D * (Nc + 1) + 2 * D * D) / (ms / 1e3) / 1e12
+
+
+def extra_c5(args, device):
+    """Segment-length sweep: B=8, H=16, L=65536, N in {512, 1024, 2048, 4096}, both modes;
+    per forward the state path and the attention kernel timed by the library's events."""
+    import compressive_memory_transformer_b200 as ia
+    from synthetic_inputs import make_inputs
+    stream = torch.cuda.current_stream()
+    peak_burst, peak_sust, _, src = load_peaks()
+    Bc, Hc, Lc = 8, 16, 65536
+    inp = make_inputs(Bc, Hc, Lc, D, torch.bfloat16, seed=0, device=device, gen_device=device)
+    out = torch.empty_like(inp["q"])
+    res = []
+    for Nc in (512, 1024, 2048, 4096):
+        for mode in (ia.LINEAR, ia.DELTA):
+            ws = torch.empty(ia.workspace_size(Bc, Hc, Lc, Nc, D, mode), dtype=torch.uint8,
+                             device=device)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            for e in ev:
+                e.record(stream)
+
+            def f():
+                ia.infini_attn_forward_ex(inp["q"], inp["k"], inp["v"], inp["beta"], Nc, mode,
+                                          out=out, workspace=ws, stage_events=ev)
+            for _ in range(3):
+                f()
+            torch.cuda.synchronize()
+            tot = st = at = 0.0
+            reps = max(3, args.steps // 3)
+            for _ in range(reps):
+                f()
+                torch.cuda.synchronize()
+                tot += ev[0].elapsed_time(ev[2])
+                st += ev[0].elapsed_time(ev[1])
+                at += ev[1].elapsed_time(ev[2])
+            tot, st, at = tot / reps, st / reps, at / reps
+            tf = _attn_tflops(Bc, Hc, Lc, Nc, at)
+            res.append({"N": Nc, "mode": "delta" if mode else "linear",
+                        "tokens_per_s": Bc * Lc / (tot / 1e3), "forward_ms": tot,
+                        "state_ms": st, "attn_ms": at, "attn_tflops": tf,
+                        "attn_frac": tf / peak_burst, "attn_frac_sustained": tf / peak_sust,
+                        "attn_hbm_gbs": Bc * Hc * Lc * 1024 / (at / 1e3) / 1e9})
+            del ws
+    assert ia.device_status() == 0
+    del inp, out
+    torch.cuda.empty_cache()
+    return {"config": "C5 segment-length sweep: B=8, H=16, d=128, L=65536, bf16",
+            "peak": f"attn_frac of the {peak_burst} TFLOP/s burst bf16 peak ({src})",
+            "results": res}
+
+
+def extra_c4(args, device):
+    """8B-model 500K stream: B=1, H=32, L=524288, N=2048, Linear+Delta, one forward."""
+    import compressive_memory_transformer_b200 as ia
+    from synthetic_inputs import make_inputs
+    stream = torch.cuda.current_stream()
+    peak_burst, peak_sust, _, src = load_peaks()
+    Bc, Hc, Lc, Nc = 1, 32, 524288, 2048
+    inp = make_inputs(Bc, Hc, Lc, D, torch.bfloat16, seed=0, device=device, gen_device=device)
+    out = torch.empty_like(inp["q"])
+    ws = torch.empty(ia.workspace_size(Bc, Hc, Lc, Nc, D, ia.DELTA), dtype=torch.uint8,
+                     device=device)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(3)]
+    for e in (e for row in evs for e in row):
+        e.record(stream)
+    it = [0]
+
+    def f4():
+        e = evs[it[0] % 3]
+        it[0] += 1
+        ia.infini_attn_forward_ex(inp["q"], inp["k"], inp["v"], inp["beta"], Nc, ia.DELTA,
+                                  out=out, workspace=ws, stage_events=e)
+    f4()
+    f4()
+    torch.cuda.synchronize()
+    it[0] = 0
+    ms = _timed(f4, 3, stream)
+    at = sum(e[1].elapsed_time(e[2]) for e in evs) / 3
+    st = sum(e[0].elapsed_time(e[1]) for e in evs) / 3
+    tf = _attn_tflops(Bc, Hc, Lc, Nc, at)
+    assert ia.device_status() == 0
+    del inp, out, ws
+    torch.cuda.empty_cache()
+    return {"config": "C4 8B-model 500K stream: B=1, H=32, d=128, N=2048, L=524288, "
+                      "Linear+Delta, one forward",
+            "tokens_per_s": Bc * Lc / (ms / 1e3), "forward_ms": ms, "state_ms": st,
+            "attn_ms": at, "attn_tflops": tf, "attn_frac": tf / peak_burst,
+            "attn_frac_sustained": tf / peak_sust, "peak_source": src}
+
+
+def extra_c3(args, device):
+    """1M-token stream: 512 infini_attn_step calls (B=1, H=8, N=2048, Linear+Delta, the
+    state carried in place), issued back to back and captured in one CUDA graph."""
+    import compressive_memory_transformer_b200 as ia
+    from synthetic_inputs import make_inputs
+    stream = torch.cuda.current_stream()
+    peak_burst, peak_sust, _, src = load_peaks()
+    Bc, Hc, Nc, S = 1, 8, 2048, 512
+    # the stream arrives segment by segment: [S][B, H, N, d], each segment contiguous
+    seg = [make_inputs(Bc, Hc, Nc, D, torch.bfloat16, seed=1000 + i, device=device,
+                       gen_device=device) for i in range(S)]
+    beta = seg[0]["beta"]
+    M = torch.zeros((Bc, Hc, D, D), device=device)
+    z = torch.zeros((Bc, Hc, D), device=device)
+    outs = [torch.empty_like(seg[0]["q"]) for _ in range(S)]
+
+    def run_stream():
+        for i in range(S):
+            ia.infini_attn_step(seg[i]["q"], seg[i]["k"], seg[i]["v"], beta, ia.DELTA, M, z,
+                                out=outs[i], M_out=M, z_out=z)
+    run_stream()
+    torch.cuda.synchronize()
+    plain_ms = _timed(run_stream, 2, stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run_stream()
+    g.replay()
+    torch.cuda.synchronize()
+    graph_ms = _timed(g.replay, 3, stream)
+    del g
+    assert ia.device_status() == 0
+    step_ms = graph_ms / S
+    # the attention kernel's algorithmic FLOPs per step over the whole step's time (the
+    # state path runs beside it): a lower bound on the kernel's own fraction
+    tf = _attn_tflops(Bc, Hc, Nc, Nc, step_ms)
+    del seg, outs
+    torch.cuda.empty_cache()
+    return {"config": "C3 1M-token stream: B=1, H=8, d=128, N=2048, L=1048576 via 512 "
+                      "infini_attn_step calls, Linear+Delta, state carried in place",
+            "tokens_per_s_graph": Bc * S * Nc / (graph_ms / 1e3),
+            "stream_ms_graph": graph_ms, "us_per_step_graph": step_ms * 1e3,
+            "tokens_per_s_plain": Bc * S * Nc / (plain_ms / 1e3), "stream_ms_plain": plain_ms,
+            "attn_tflops_over_step": tf, "attn_frac_over_step": tf / peak_burst,
+            "peak_source": src}
+
+
 def run_extra(args, device):
     """C3: 1M-token stream through 512 infini_attn_step calls (graph-captured),
-    C4: 8B 500K single forward, C5: segment-length sweep. One JSON line each."""
+    C4: 8B 500K single forward, C5: segment-length sweep, decode, backward, layer.
+    One JSON line each."""
     import compressive_memory_transformer_b200 as ia
     from synthetic_inputs import make_inputs
     torch.cuda.set_device(device)
@@ -402,108 +555,12 @@ def run_extra(args, device):
     peak_burst, peak_sust, _, src = load_peaks()
     lines = []
     which = args.config
-
-    def attn_tflops(Bc, Hc, Lc, Nc, ms):
-        return Bc * Hc * Lc * (2 * D * (Nc + 1) + 2 * D * D) / (ms / 1e3) / 1e12
-
     if which in ("c5", "all"):
-        Bc, Hc, Lc = 8, 16, 65536
-        inp = make_inputs(Bc, Hc, Lc, D, torch.bfloat16, seed=0, device=device, gen_device=device)
-        res = []
-        for Nc in (512, 1024, 2048, 4096):
-            for mode in (ia.LINEAR, ia.DELTA):
-                ws = torch.empty(ia.workspace_size(Bc, Hc, Lc, Nc, D, mode), dtype=torch.uint8,
-                                 device=device)
-                out = torch.empty_like(inp["q"])
-                ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-                for e in ev:
-                    e.record(stream)
-
-                def f():
-                    ia.infini_attn_forward_ex(inp["q"], inp["k"], inp["v"], inp["beta"], Nc, mode,
-                                              out=out, workspace=ws, stage_events=ev)
-                for _ in range(3):
-                    f()
-                torch.cuda.synchronize()
-                tot = st = at = 0.0
-                reps = max(3, args.steps // 3)
-                for _ in range(reps):
-                    f()
-                    torch.cuda.synchronize()
-                    tot += ev[0].elapsed_time(ev[2])
-                    st += ev[0].elapsed_time(ev[1])
-                    at += ev[1].elapsed_time(ev[2])
-                tot, st, at = tot / reps, st / reps, at / reps
-                res.append({"N": Nc, "mode": "delta" if mode else "linear",
-                            "tokens_per_s": Bc * Lc / (tot / 1e3), "forward_ms": tot,
-                            "state_ms": st, "attn_ms": at,
-                            "attn_tflops": attn_tflops(Bc, Hc, Lc, Nc, at),
-                            "attn_frac_sustained": attn_tflops(Bc, Hc, Lc, Nc, at) / peak_sust,
-                            "attn_hbm_gbs": Bc * Hc * Lc * 1024 / (at / 1e3) / 1e9})
-        assert ia.device_status() == 0
-        lines.append({"config": "C5 segment-length sweep: B=8, H=16, d=128, L=65536, bf16",
-                      "peak": f"{peak_sust} TFLOP/s sustained ({src})", "results": res})
-        del inp
-        torch.cuda.empty_cache()
-
+        lines.append(extra_c5(args, device))
     if which in ("c4", "all"):
-        Bc, Hc, Lc, Nc = 1, 32, 524288, 2048
-        inp = make_inputs(Bc, Hc, Lc, D, torch.bfloat16, seed=0, device=device, gen_device=device)
-        out = torch.empty_like(inp["q"])
-        ws = torch.empty(ia.workspace_size(Bc, Hc, Lc, Nc, D, ia.DELTA), dtype=torch.uint8,
-                         device=device)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        for e in ev:
-            e.record(stream)
-
-        def f4():
-            ia.infini_attn_forward_ex(inp["q"], inp["k"], inp["v"], inp["beta"], Nc, ia.DELTA,
-                                      out=out, workspace=ws, stage_events=ev)
-        f4()
-        torch.cuda.synchronize()
-        ms = _timed(f4, 3, stream)
-        at = ev[1].elapsed_time(ev[2])
-        assert ia.device_status() == 0
-        lines.append({"config": "C4 8B-model 500K stream: B=1, H=32, d=128, N=2048, L=524288, "
-                                "Linear+Delta, one forward",
-                      "tokens_per_s": Bc * Lc / (ms / 1e3), "forward_ms": ms,
-                      "state_ms": ev[0].elapsed_time(ev[1]), "attn_ms": at,
-                      "attn_tflops": attn_tflops(Bc, Hc, Lc, Nc, at),
-                      "attn_frac_sustained": attn_tflops(Bc, Hc, Lc, Nc, at) / peak_sust})
-        del inp, out, ws
-        torch.cuda.empty_cache()
-
+        lines.append(extra_c4(args, device))
     if which in ("c3", "all"):
-        Bc, Hc, Nc, S = 1, 8, 2048, 512
-        # the stream arrives segment by segment: [S][B, H, N, d], each segment contiguous
-        seg = [make_inputs(Bc, Hc, Nc, D, torch.bfloat16, seed=1000 + i, device=device,
-                           gen_device=device) for i in range(S)]
-        beta = seg[0]["beta"]
-        M = torch.zeros((Bc, Hc, D, D), device=device)
-        z = torch.zeros((Bc, Hc, D), device=device)
-        outs = [torch.empty_like(seg[0]["q"]) for _ in range(S)]
-
-        def run_stream():
-            for i in range(S):
-                ia.infini_attn_step(seg[i]["q"], seg[i]["k"], seg[i]["v"], beta, ia.DELTA, M, z,
-                                    out=outs[i], M_out=M, z_out=z)
-        run_stream()
-        torch.cuda.synchronize()
-        plain_ms = _timed(run_stream, 2, stream)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            run_stream()
-        g.replay()
-        torch.cuda.synchronize()
-        graph_ms = _timed(g.replay, 3, stream)
-        del g
-        assert ia.device_status() == 0
-        lines.append({"config": "C3 1M-token stream: B=1, H=8, d=128, N=2048, L=1048576 via 512 "
-                                "infini_attn_step calls, Linear+Delta, state carried in place",
-                      "tokens_per_s_graph": Bc * S * Nc / (graph_ms / 1e3),
-                      "stream_ms_graph": graph_ms, "us_per_step_graph": graph_ms * 1e3 / S,
-                      "tokens_per_s_plain": Bc * S * Nc / (plain_ms / 1e3),
-                      "stream_ms_plain": plain_ms})
+        lines.append(extra_c3(args, device))
     if which in ("decode", "all"):
         # token-level streaming decode on the 1B-layer heads: one segment of N tokens fed
         # one token per infini_attn_decode call (the segment-end call also folds the
@@ -701,6 +758,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the C3 / C4 / C5 workloads reported beside the headline")
     ap.add_argument("--config", choices=["c2", "c3", "c4", "c5", "decode", "backward", "layer",
                                          "all"],
                     default="c2",

@@ -20,7 +20,7 @@
 //   warp 0     TMA producer: Q per tile (reloaded once the last Q K^T of the tile
 //              and sigma(Q) are done) together with the tile's descriptor (a shared
 //              memory slot, so no other role walks the work list); a K ring (2
-//              stages); a V ring (3 stages) whose items per tile are M_hi (the
+//              stages); a V ring (2 stages) whose items per tile are M_hi (the
 //              state rounded to bf16), then V_0, V_1, ...
 //   warp 1     tensor-memory allocation; issues the retrieval and P V products.
 //   warp 10    issues the Q K^T products (another scheduler than warp 1, so each

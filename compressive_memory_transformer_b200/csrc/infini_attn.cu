@@ -1,7 +1,8 @@
 // infini_attn.cu — the C ABI (include/infini_attn.h): argument checks, scratch
 // memory, and the launch sequence of the forward.
 //
-// bf16 (d = 128): zpart -> zscan -> state (tcgen05 tf32) -> chain -> attn (tcgen05 bf16)
+// bf16 (d = 128): zpart -> zscan -> state (tcgen05 bf16, sigma(K) as a hi/lo pair)
+//                 -> chain (Linear+Delta: G_s M_{s-1} on tcgen05 tf32) -> attn (tcgen05 bf16)
 // fp32 (d <= 128): f32_state -> f32_attn (CUDA cores)
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>

@@ -87,11 +87,18 @@ extern "C" int infini_attn_step_static(const void* q, const void* k, const void*
   if (d != 128) return INFINI_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return INFINI_ERR_ALIGN;
   if ((M_in && !aligned16(M_in)) || (M_out && !aligned16(M_out))) return INFINI_ERR_ALIGN;
+  // out may overlap none of the inputs and none of the state buffers (the same rule
+  // as infini_attn_step)
   const size_t nio = (size_t)B * H * N * d * 2;
+  const size_t nM = (size_t)B * H * d * d * sizeof(float), nz = (size_t)B * H * d * sizeof(float);
   const uintptr_t o = reinterpret_cast<uintptr_t>(out);
-  for (const void* p : {q, k, v}) {
-    const uintptr_t x = reinterpret_cast<uintptr_t>(p);
-    if (o < x + nio && x < o + nio) return INFINI_ERR_ALIAS;
+  const struct {
+    const void* p;
+    size_t n;
+  } others[] = {{q, nio}, {k, nio}, {v, nio}, {M_in, nM}, {z_in, nz}, {M_out, nM}, {z_out, nz}};
+  for (const auto& x : others) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(x.p);
+    if (x.p && o < a + x.n && a < o + nio) return INFINI_ERR_ALIAS;
   }
 
   // Token chunking of the state GEMM: as in the allocating call, but halved

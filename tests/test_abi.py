@@ -276,3 +276,22 @@ def test_binding_rejects_bad_tensors_before_the_library(lib):
         lib.infini_attn_layer_forward(x, W, W, W, W, torch.zeros(2), 128, 0, 2)  # host tensors
     with pytest.raises(ValueError):
         lib.infini_attn_layer_forward(x[0], W, W, W, W, torch.zeros(2), 128, 0, 2)  # not 3-d
+
+
+@pytest.mark.parametrize("name", ["infini_attn_step", "infini_attn_step_static"])
+@pytest.mark.parametrize("which", ["q", "k", "v", "M_in", "z_in", "M_out", "z_out"])
+def test_step_entry_points_reject_the_same_aliasing(lib, name, which):
+    """The allocating and the allocation-free step refuse the same overlaps of out with
+    an input or a state buffer (INFINI_ERR_ALIAS), on the host, before any launch."""
+    gap = 1 << 24                       # B=1, H=1, N=128, d=128: 32 KiB per operand
+    args = dict(q=FAKE, k=FAKE + gap, v=FAKE + 2 * gap, beta=FAKE + 3 * gap, M_in=None,
+                z_in=None, out=FAKE + 8 * gap, M_out=None, z_out=None)
+    inside = args["out"] + 4096         # 16-byte aligned, inside out's 32 KiB
+    partner = {"M_in": "z_in", "z_in": "M_in", "M_out": "z_out", "z_out": "M_out"}
+    args[which] = inside
+    if which in partner:                # state pointers come in pairs
+        args[partner[which]] = FAKE + 16 * gap
+    st = lib.raw_call(name, args["q"], args["k"], args["v"], args["beta"], args["M_in"],
+                      args["z_in"], args["out"], args["M_out"], args["z_out"], 1, 1, 128, 128, 0,
+                      None)
+    assert st == -8, (name, which, st)

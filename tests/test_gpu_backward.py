@@ -125,3 +125,13 @@ def test_backward_single_segment(ia, mode, state):
     carried state both paths carry weight. Final-state gradients included."""
     got, ref = run(ia, 1, 2, 256, 256, mode, seed=99 + mode, state=state, state_grad=True)
     check(got, ref, f"single segment mode={mode} state={state}")
+
+
+@pytest.mark.parametrize("mode", [LIN, DEL])
+def test_backward_at_the_benchmarked_segment_length(ia, mode):
+    """N = 2048 (16 query tiles per segment, the heaviest-first tile order and the longest
+    reverse chains of the benchmarked shape) over two segments, with a carried state and
+    final-state gradients; B * H = 2 heads, so the state rebuild splits every segment
+    into the most token chunks (8)."""
+    got, ref = run(ia, 1, 2, 4096, 2048, mode, seed=105, state=True, state_grad=True)
+    check(got, ref, f"N=2048 mode={mode}")

@@ -5,6 +5,8 @@ head), so a sampled head is compared exactly, output rows and final state.
 
 Workloads (bf16 q/k/v i.i.d. N(0,1), beta ~ N(0,1) per head, zero initial state):
   1B-LM layer:      B=4, H=8,  d=128, N=2048, L=32768, Linear and Linear+Delta
+                    (also with beta = +30 on every head: the retrieval on its own)
+  8B 500K length:   B=1, H=1,  d=128, N=2048, L=524288, beta = +30, Linear+Delta
   1M-token stream:  B=1, H=8,  d=128, N=2048, 512 infini_attn_step calls, Linear+Delta
   8B 500K stream:   B=1, H=32, d=128, N=2048, L=524288, Linear+Delta, one forward
   segment sweep:    B=8, H=16, d=128, L=65536, N in {512, 1024, 2048, 4096}, both modes
@@ -59,6 +61,41 @@ def test_1b_layer_shape(ia, mode):
     for b, h in ((0, 0), (B - 1, H - 1)):
         check_head(out, M, z, inp["q"], inp["k"], inp["v"], beta, b, h, N, mode,
                    f"1B layer mode={mode}")
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_1b_layer_shape_memory_path_isolated(ia, mode):
+    """beta = +30 on every head of the 1B-layer shape (16 segments of 2048): the output
+    is the memory retrieval (the local attention's weight is 1e-13), so the retrieval
+    with M rounded to bf16 is compared on its own at the full segment count, where z
+    has grown over 15 segments."""
+    B, H, L, N = 4, 8, 32768, 2048
+    inp = make_inputs(B, H, L, 128, torch.bfloat16, seed=0, device="cuda", gen_device="cuda",
+                      beta=[30.0] * H)
+    out, M, z = ia.infini_attn_forward(inp["q"], inp["k"], inp["v"], inp["beta"], N, mode)
+    torch.cuda.synchronize()
+    assert ia.device_status() == 0
+    beta = inp["beta"].cpu()
+    for b, h in ((0, 0), (B - 1, H - 1)):
+        check_head(out, M, z, inp["q"], inp["k"], inp["v"], beta, b, h, N, mode,
+                   f"1B layer beta=+30 mode={mode}")
+    # the first segment retrieves exactly nothing: only the 1e-13 local-attention share
+    assert float(out[:, :, :N].abs().max()) < 1e-6
+
+
+def test_8b_length_memory_path_isolated(ia):
+    """beta = +30 over the 8B 500K stream's length (256 segments of 2048, Linear+Delta),
+    one head: the retrieval after z has grown for half a million tokens."""
+    B, H, L, N, mode = 1, 1, 524288, 2048, 1
+    inp = make_inputs(B, H, L, 128, torch.bfloat16, seed=2, device="cuda", gen_device="cuda",
+                      beta=[30.0])
+    out, M, z = ia.infini_attn_forward(inp["q"], inp["k"], inp["v"], inp["beta"], N, mode)
+    torch.cuda.synchronize()
+    assert ia.device_status() == 0
+    check_head(out, M, z, inp["q"], inp["k"], inp["v"], inp["beta"].cpu(), 0, 0, N, mode,
+               "8B length beta=+30")
+    del inp, out
+    torch.cuda.empty_cache()
 
 
 def test_1m_token_stream_steps(ia):

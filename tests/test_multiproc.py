@@ -82,58 +82,136 @@ def test_reference_arm_under_torchrun_prints_once():
     assert d["e2e"]["h2d_bytes_per_step"] == 0
 
 
-def _shard_worker(rank, world, port, q):
-    """Each rank holds one range of a Linear-mode sequence; the range's state sum is
-    taken with the oracle (the GPU library's infini_attn_state_update on a GPU machine),
-    exchanged with the package's gather_states over gloo, and composed as the
-    sharded forward composes it."""
+def _oracle_library(monkeypatch_target, beta):
+    """Stand-ins for the three library calls of the sharded forward, computed by the
+    oracle in float64 on the host (this CPU test has no CUDA library to run): the
+    host logic around them (the exchange, the rank-order prefix, the validation of
+    the ranges, the final state) is the shipped code."""
+    import numpy as np
+    import oracle
+
+    def state_update(k, v, N, mode, stream=None):
+        kk, vv = k.double().numpy(), v.double().numpy()
+        _, M, z = oracle.forward(kk, kk, vv, np.zeros(k.shape[1]), N, mode)
+        return torch.from_numpy(M).float(), torch.from_numpy(z).float()
+
+    def state_sum(dM, dz, M_in=None, z_in=None, stream=None):
+        M = dM.double().sum(0) + (0 if M_in is None else M_in.double())
+        z = dz.double().sum(0) + (0 if z_in is None else z_in.double())
+        return M.float(), z.float()
+
+    def forward(q, k, v, beta_, N, mode, M_in=None, z_in=None, out=None, state_out=True,
+                stream=None):
+        f = lambda t: None if t is None else t.double().numpy()
+        o, M, z = oracle.forward(f(q), f(k), f(v), f(beta_), N, mode, f(M_in), f(z_in))
+        return torch.from_numpy(o), torch.from_numpy(M), torch.from_numpy(z)
+
+    monkeypatch_target.infini_attn_state_update = state_update
+    monkeypatch_target.infini_attn_state_sum = state_sum
+    monkeypatch_target.infini_attn_forward = forward
+
+
+def _shard_worker(rank, world, port, q, seg_per_rank, ragged):
+    """Each rank holds one range of a Linear-mode sequence and runs the package's
+    sequence_sharded_linear_forward on it (its library calls taken by the oracle)."""
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     sys.path.insert(0, ROOT)
     import numpy as np
     import oracle
-    from compressive_memory_transformer_b200.sharded import gather_states
-    from synthetic_inputs import make_inputs
+    from compressive_memory_transformer_b200 import sharded
+    from synthetic_inputs import make_inputs, normal_state
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         B, H, N, d = 1, 2, 32, 16
-        seg_per_rank = [3, 2]                   # ranges of unequal length, in rank order
-        L = N * sum(seg_per_rank)
+        lens = [N * n for n in seg_per_rank]
+        lens[-1] -= ragged                      # the last range may end mid-segment
+        L = sum(lens)
         inp = make_inputs(B, H, L, d, torch.float32, seed=61, device="cpu", gen_device="cpu")
+        M0, z0 = normal_state(B, H, d, seed=62, scale_M=2.0, scale_z=10.0)
+        _oracle_library(sharded, inp["beta"])
+        lo = sum(lens[:rank])
+        hi = lo + lens[rank]
+        part = {x: inp[x][:, :, lo:hi] for x in ("q", "k", "v")}
+        try:
+            out_r, M_end, z_end = sharded.sequence_sharded_linear_forward(
+                part["q"], part["k"], part["v"], inp["beta"], N, M0, z0)
+        except ValueError as e:
+            q.put((rank, "ValueError", str(e)))
+            return
         f = {x: inp[x].double().numpy() for x in ("q", "k", "v", "beta")}
-        lo = N * sum(seg_per_rank[:rank])
-        hi = lo + N * seg_per_rank[rank]
-        part = {x: f[x][:, :, lo:hi] for x in ("q", "k", "v")}
-        _, dM, dz = oracle.forward(part["q"], part["k"], part["v"], f["beta"], N, oracle.LINEAR)
-        dM_all, dz_all = gather_states(torch.from_numpy(dM), torch.from_numpy(dz))
-        assert dM_all.shape == (world, B, H, d, d) and dz_all.shape == (world, B, H, d)
-        M_pre = dM_all[:rank].sum(0).numpy()
-        z_pre = dz_all[:rank].sum(0).numpy()
-        out_r, _, _ = oracle.forward(part["q"], part["k"], part["v"], f["beta"], N, oracle.LINEAR,
-                                     M_pre, z_pre)
-        ref_out, ref_M, ref_z = oracle.forward(f["q"], f["k"], f["v"], f["beta"], N, oracle.LINEAR)
-        err_out = float(np.max(np.abs(out_r - ref_out[:, :, lo:hi])))
-        err_M = float(np.max(np.abs(dM_all.sum(0).numpy() - ref_M)) / np.max(np.abs(ref_M)))
-        err_z = float(np.max(np.abs(dz_all.sum(0).numpy() - ref_z)) / np.max(np.abs(ref_z)))
+        ref_out, ref_M, ref_z = oracle.forward(f["q"], f["k"], f["v"], f["beta"], N,
+                                               oracle.LINEAR, M0.double().numpy(),
+                                               z0.double().numpy())
+        err_out = float(np.max(np.abs(out_r.numpy() - ref_out[:, :, lo:hi])))
+        err_M = float(np.max(np.abs(M_end.double().numpy() - ref_M)) / np.max(np.abs(ref_M)))
+        err_z = float(np.max(np.abs(z_end.double().numpy() - ref_z)) / np.max(np.abs(ref_z)))
         q.put((rank, err_out, err_M, err_z))
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
-def test_linear_sequence_sharding_exchange():
-    """Two ranks, one all-gather of the per-range Linear state sums: every rank's
-    outputs and the final state equal the single-process forward's."""
-    world = 2
+def _run_shards(seg_per_rank, ragged):
+    world = len(seg_per_rank)
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, q, seg_per_rank, ragged))
+             for r in range(world)]
     for p in procs:
         p.start()
     res = sorted(q.get(timeout=180) for _ in range(world))
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, err_out, err_M, err_z in res:
-        assert err_out < 1e-12 and err_M < 1e-12 and err_z < 1e-12, (rank, err_out, err_M, err_z)
+    return res
+
+
+def test_linear_sequence_sharding_exchange():
+    """Two ranks of unequal length (3 and 2 segments, the last one ragged), a non-zero
+    incoming state, one all-gather of the per-range Linear state sums: every rank's
+    outputs and the final state equal the single-process forward's (the state sums
+    travel in float32, hence the 1e-6 bound)."""
+    for rank, err_out, err_M, err_z in _run_shards([3, 2], ragged=5):
+        assert err_out < 1e-5 and err_M < 1e-6 and err_z < 1e-6, (rank, err_out, err_M, err_z)
+
+
+def test_linear_sequence_sharding_rejects_a_ragged_inner_range_on_every_rank():
+    """A range that ends mid-segment on a rank other than the last raises ValueError on
+    every rank together (each learns every range's length from the one all-gather), so
+    no rank is left waiting in a collective."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bad_range_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == ["ValueError", "ValueError"], res
+    assert all("[0]" in r[2] for r in res), res
+
+
+def _bad_range_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    sys.path.insert(0, ROOT)
+    from compressive_memory_transformer_b200 import sharded
+    from synthetic_inputs import make_inputs
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        N = 32
+        L_r = N * 2 - 7 if rank == 0 else N * 2   # rank 0's range ends mid-segment
+        inp = make_inputs(1, 2, L_r, 16, torch.float32, seed=63 + rank, device="cpu")
+        _oracle_library(sharded, inp["beta"])
+        try:
+            sharded.sequence_sharded_linear_forward(inp["q"], inp["k"], inp["v"], inp["beta"], N)
+            q.put((rank, "returned", ""))
+        except ValueError as e:
+            q.put((rank, "ValueError", str(e)))
+    finally:
+        dist.destroy_process_group()
