@@ -21,7 +21,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_NAME = "libinfini_attn.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
 SOURCES = ["infini_attn.cu", "bf16_state.cu", "bf16_attn.cu", "f32_path.cu", "step_static.cu",
-           "bf16_decode.cu", "bf16_bwd.cu", "bf16_gemm.cu"]
+           "bf16_decode.cu", "bf16_bwd.cu", "bf16_gemm.cu", "bf16_step_state.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

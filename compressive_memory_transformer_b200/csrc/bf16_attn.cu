@@ -44,9 +44,12 @@
 // P V through the buffer's S-free barrier.
 // Every mbarrier is waited on in completion order and can never complete twice
 // before its waiter has seen the first completion (a parity wait would then
-// miss it): sigma(Q) and P have separate barriers; P_{j+1} is written only after
-// the softmax saw PV_j done, the next tile's sigma(Q) only after the epilogue saw
-// R and the last PV done. z_{s-1} (512 B) rides on the Q barrier.
+// miss it): sigma(Q) and P have separate barriers; P has one per S buffer (P of
+// step n + 2 needs the S of step n + 2, whose Q K^T waited for the P V of step n);
+// the next tile's sigma(Q) is written only after the epilogue saw R and the last
+// P V done. The softmax warps wait for a P V (through its S buffer's S-free
+// barrier) only before touching O: for a rescale, and in the epilogue.
+// z_{s-1} (512 B) rides on the Q barrier.
 // Online softmax keeps a per-row reference max and rescales O only when the
 // running max grows by more than 2^8 (in exp2 units). One exponential in four is
 // evaluated on the FMA pipe (ex2_poly2) to offload the MUFU unit. The retrieval
@@ -79,46 +82,129 @@ constexpr int OFF_X = 6 * kTile;     // exchange: max [2][2][128], den [2][128],
 constexpr int OFF_Z = OFF_X + 4096;   // z_{s-1} of the current tile (128 floats), loaded with Q
 constexpr int OFF_BAR = OFF_Z + 512;
 constexpr int OFF_SLOT = OFF_BAR + 256;  // two tile descriptors
-constexpr int kAttnSmem = OFF_SLOT + 128 + 1024;  // + alignment slack
+constexpr int OFF_FLAG = OFF_SLOT + 256;  // split mode: "this piece merges" broadcast
+constexpr int kAttnSmem = OFF_FLAG + 16 + 1024;  // + alignment slack
 constexpr int kThreads = 352;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kSoftmaxWarps = 8;
+// Split mode: the record a piece leaves for the tile's merge. O (128 rows x 128
+// value columns, fp32, unnormalised, against the piece's reference row max) as
+// [32 column quads][128 rows] float4, then the reference max and the row sum.
+constexpr int kRecO = 128 * 128;
+constexpr int kRecFloats = kRecO + 2 * 128;
 
 enum {
   B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_SFREE = 4 /* 2 */, B_VFULL = 6 /* 3 */, B_VEMPTY = 9 /* 3 */,
-  B_SFULL = 12, B_PFULL = 14, B_PVDONE = 15, B_DRAIN = 16, B_PAIR = 17 /* 4 */, B_RDONE = 21,
-  B_SQFULL = 22, B_OFULL = 23 /* 2 */, B_OFREE = 25 /* 2 */, B_COUNT = 27
+  B_SFULL = 12, B_PFULL = 14 /* 2 */, B_DRAIN = 16, B_PAIR = 17 /* 4 */, B_RDONE = 21,
+  B_SQFULL = 22, B_OFULL = 23 /* 2 */, B_OFREE = 25 /* 2 */, B_SPLW = 27, B_SPLF = 28,
+  B_COUNT = 29
 };
 
 struct Params {
   long long L;
   int N, S, H, T, U, BH;
-  unsigned units;  // BH * S * U, below 2^31
+  unsigned units;  // tile pairs: BH * S * U; split mode: pieces (below 2^31)
   FastDiv divU, divS, divH, divG;  // G = H / Hkv query heads per key/value head
   int Hkv;
   long long o_sb, o_sh, o_sl;  // out strides (elements): batch row, head, row
   int out32;    // out is 32-byte aligned: rows are stored as whole 32-byte sectors
   int tma_out;  // out has a TMA map: whole tiles leave through shared memory
+  // Split mode (calls with fewer tile pairs than SMs): a unit is a piece of one query
+  // tile's key range; units are taken from a device counter, heaviest first.
+  int split;
+  int C;        // most key tiles per piece
+  int Pmax;     // record slots per tile
+  unsigned BHS; // BH * S
+  FastDiv divBHS;
+  unsigned* unit_ctr;  // next unit (zeroed before the launch)
+  unsigned* tile_ctr;  // [BHS * T] pieces of each tile finished (zeroed before the launch)
+  float* rec;          // [BHS * T * Pmax] records of kRecFloats
 };
 
-// One query tile of the work list (valid = 0: the end of the CTA's list).
+// One query tile (or, in split mode, one piece of its key range) of the work list
+// (valid = 0: the end of the CTA's list).
 struct Tile {
   long long seg0;
   int bh, s, i, nkv, q_row, rows_valid, h, valid;
   int b, hk, bhk;  // batch row, key/value head, and its index b * Hkv + hk
+  int j0;          // first key tile of the piece (0 outside split mode)
+  int np, pc;      // pieces of this tile (1 outside split mode) and this piece's index
+  unsigned tid;    // split mode: the tile's index (bh * S + s) * T + i
 };
 
-// Walks the CTA's tiles: units blockIdx.x, blockIdx.x + gridDim.x, ...; unit u of
-// a segment holds tiles T-1-u and u (one tile when they coincide); tiles past the
-// end of a short final segment are skipped.
+// Fills t for query tile i of segment seg = bh * S + s; false when the tile lies past
+// the end of a short final segment.
+__device__ __forceinline__ bool fill_tile(const Params& p, unsigned seg, int i, Tile& t) {
+  const unsigned bh = p.divS.div(seg);
+  t.s = (int)(seg - bh * (unsigned)p.S);
+  t.bh = (int)bh;
+  t.seg0 = (long long)t.s * p.N;
+  const int n_s = (int)min((long long)p.N, p.L - t.seg0);
+  const int T_s = (n_s + BM - 1) / BM;
+  if (i >= T_s) return false;
+  t.i = i;
+  t.nkv = i + 1;
+  t.j0 = 0;
+  t.np = 1;
+  t.pc = 0;
+  t.tid = seg * (unsigned)p.T + (unsigned)i;
+  t.b = (int)p.divH.div((uint32_t)t.bh);
+  t.h = t.bh - t.b * p.H;
+  t.hk = (int)p.divG.div((uint32_t)t.h);
+  t.bhk = t.b * p.Hkv + t.hk;
+  t.valid = 1;
+  t.q_row = (int)(t.seg0 + (long long)i * BM);
+  t.rows_valid = min(BM, n_s - i * BM);
+  return true;
+}
+
+// Split mode, unit u -> piece. Units are ordered heaviest first: query tiles from the
+// last (T - 1, the longest key range) down to 0; tile i's i + 1 key tiles form
+// np = ceil((i + 1) / C) pieces of near-equal length; within a tile level, piece
+// index, then segment.
+__device__ __forceinline__ bool decode_piece(const Params& p, unsigned u, Tile& t) {
+  for (int i = p.T - 1; i >= 0; --i) {
+    const int np = (i + p.C) / p.C;
+    const unsigned cnt = (unsigned)np * p.BHS;
+    if (u < cnt) {
+      const int pc = (int)p.divBHS.div(u);
+      const unsigned seg = u - (unsigned)pc * p.BHS;
+      if (!fill_tile(p, seg, i, t)) return false;
+      const int j0 = pc * (i + 1) / np, j1 = (pc + 1) * (i + 1) / np;
+      t.j0 = j0;
+      t.nkv = j1 - j0;
+      t.np = np;
+      t.pc = pc;
+      return true;
+    }
+    u -= cnt;
+  }
+  return false;
+}
+
+// Walks the CTA's tiles. Tile pairs: units blockIdx.x, blockIdx.x + gridDim.x, ...;
+// unit u of a segment holds tiles T-1-u and u (one tile when they coincide); tiles
+// past the end of a short final segment are skipped. Split mode: each unit is taken
+// from the device counter when the producer is ready to load it (after it has issued
+// every copy of the previous unit), never earlier: a CTA that starts late, when the
+// SMs of a kernel running beside it free up, still finds the units that no CTA has
+// begun.
+template <bool kSplit>
 struct TileIter {
   unsigned unit;
   int k;  // 0: tile T-1-u, 1: tile u
-  __device__ void init() {
+  __device__ void init(const Params& p) {
     unit = blockIdx.x;
     k = 0;
   }
   __device__ bool next(const Params& p, Tile& t) {
+    if (kSplit) {
+      for (;;) {
+        const unsigned u = atomicAdd(p.unit_ctr, 1u);
+        if (u >= p.units) return false;
+        if (decode_piece(p, u, t)) return true;
+      }
+    }
     while (unit < p.units) {
       const unsigned seg = p.divU.div(unit);
       const int u = (int)(unit - seg * (unsigned)p.U);
@@ -129,25 +215,16 @@ struct TileIter {
       }
       const int i = kk == 0 ? p.T - 1 - u : u;
       if (kk == 1 && u >= p.T - 1 - u) continue;  // the pair collapsed to one tile
-      const unsigned bh = p.divS.div(seg);
-      t.s = (int)(seg - bh * (unsigned)p.S);
-      t.bh = (int)bh;
-      t.seg0 = (long long)t.s * p.N;
-      const int n_s = (int)min((long long)p.N, p.L - t.seg0);
-      const int T_s = (n_s + BM - 1) / BM;
-      if (i >= T_s) continue;
-      t.i = i;
-      t.nkv = i + 1;
-      t.b = (int)p.divH.div((uint32_t)t.bh);
-      t.h = t.bh - t.b * p.H;
-      t.hk = (int)p.divG.div((uint32_t)t.h);
-      t.bhk = t.b * p.Hkv + t.hk;
-      t.valid = 1;
-      t.q_row = (int)(t.seg0 + (long long)i * BM);
-      t.rows_valid = min(BM, n_s - i * BM);
-      return true;
+      if (fill_tile(p, seg, i, t)) return true;
     }
     return false;
+  }
+  // The tile the next call returns, if known without taking a unit (for prefetching;
+  // split mode does not know it).
+  __device__ bool peek(const Params& p, Tile& t) const {
+    if (kSplit) return false;
+    TileIter a = *this;
+    return a.next(p, t);
   }
 };
 
@@ -176,6 +253,9 @@ __device__ __forceinline__ constexpr uint32_t kdesc_off(int kk) {
 }
 __device__ __forceinline__ constexpr uint32_t mndesc_off(int kk) { return (uint32_t)kk * 128u; }
 
+// kSplit: split mode (a separate instantiation, so that the tile-pair kernel carries
+// none of its code).
+template <bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
@@ -204,7 +284,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     for (int b = 0; b < B_COUNT; ++b) {
       uint32_t cnt = 1;
       // arrivals are counted per warp (mbar_arrive_warp)
-      if (b == B_PFULL || b == B_SQFULL) cnt = kSoftmaxWarps;
+      if (b == B_PFULL || b == B_PFULL + 1 || b == B_SQFULL || b == B_SPLW) cnt = kSoftmaxWarps;
       // Q is free once the tile's last Q K^T is done and every softmax warp has
       // read its rows of Q for sigma(Q)
       if (b == B_QEMPTY) cnt = 1 + kSoftmaxWarps;
@@ -242,7 +322,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // the Q K^T that read this stage signalled the same stage's scores barrier
         if (k_wrapped && !mbar_wait(&bars[B_SFULL + kst], kph ^ 1u)) return false;
         mbar_arrive_expect_tx(&bars[B_KFULL + kst], kTile);
-        const int row = (int)(t.seg0 + (long long)j * BN);
+        const int row = (int)(t.seg0 + (long long)(t.j0 + j) * BN);
         uint8_t* dst = sK + kst * kTile;
         tma_load_4d(dst, &tm_k, &bars[B_KFULL + kst], 0, row, t.hk, t.b);
         tma_load_4d(dst + kSub, &tm_k, &bars[B_KFULL + kst], 64, row, t.hk, t.b);
@@ -261,7 +341,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           tma_load_3d(dst, &tm_m, &bars[B_VFULL + vst], 0, 0, zc);
           tma_load_3d(dst + kSub, &tm_m, &bars[B_VFULL + vst], 64, 0, zc);
         } else {
-          const int row = (int)(t.seg0 + (long long)(item - 1) * BN);
+          const int row = (int)(t.seg0 + (long long)(t.j0 + item - 1) * BN);
           tma_load_4d(dst, &tm_v, &bars[B_VFULL + vst], 0, row, t.hk, t.b);
           tma_load_4d(dst + kSub, &tm_v, &bars[B_VFULL + vst], 64, row, t.hk, t.b);
         }
@@ -273,8 +353,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         return true;
       };
-      TileIter it;
-      it.init();
+      TileIter<kSplit> it;
+      it.init(p);
       Tile t;
       int tc = 0;
       while (ok && it.next(p, t)) {
@@ -289,9 +369,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         bulk_load(sZ, zprev + ((size_t)t.bhk * p.S + t.s) * D, D * 4, &bars[B_QFULL]);
         ++q_iss;
         {  // the next tile's Q has a whole tile of work to reach L2
-          TileIter ahead = it;
           Tile tn;
-          if (ahead.next(p, tn)) {
+          if (it.peek(p, tn)) {
             tma_prefetch_l2_4d(&tm_q, 0, tn.q_row, tn.h, tn.b);
             tma_prefetch_l2_4d(&tm_q, 64, tn.q_row, tn.h, tn.b);
           }
@@ -336,7 +415,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       const uint64_t dV0 = mnmajor_desc(smem_u32(sV), 0);
       constexpr uint32_t kTileD = kTile >> 4;  // one tile, in descriptor units
       uint32_t vst = 0, vph = 0;  // V ring: stage and phase of the next item
-      uint32_t pb = 0;            // S buffer (and p_full parity) of the next P
+      uint32_t pn = 0;            // P products issued so far: P n sits in S buffer n & 1
       int tc = 0;
       auto v_next = [&]() {
         if (++vst == (uint32_t)kVStages) {
@@ -374,7 +453,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int j = 0; ok && j < t.nkv; ++j) {
           const uint32_t st = vst, ph = vph;
           v_next();
-          ok = mbar_wait_warp(&bars[B_PFULL], pb) && mbar_wait_warp(&bars[B_VFULL + st], ph);
+          const uint32_t pb = pn & 1u;
+          ok = mbar_wait_warp(&bars[B_PFULL + pb], (pn >> 1) & 1u) &&
+               mbar_wait_warp(&bars[B_VFULL + st], ph);
           if (!ok) break;
           tc_fence_after();
           // P_j lives in the first 64 columns of its S buffer
@@ -385,11 +466,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             for (int kk = 0; kk < BN / 16; ++kk)
               mma_bf16_ts(tO, tP + 8 * kk, dv + mndesc_off(kk), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&bars[B_VEMPTY + st]);
-            mma_commit(&bars[B_PVDONE]);
-            mma_commit(&bars[B_SFREE + pb]);  // the S buffer may take the next Q K^T
+            // P V done: the S buffer may take the next Q K^T, and O may be rescaled
+            mma_commit(&bars[B_SFREE + pb]);
           }
           __syncwarp();
-          pb ^= 1u;
+          ++pn;
         }
         if (!ok) break;
         ++tc;
@@ -461,8 +542,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     float* xden = sX + 512;      // [2 halves][128]
     float* xl = sX + 768;        // [2 halves][128]
     const float sl = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
+    volatile int* sflag = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
     long long kc = 0;
     int tc = 0;
+    int sc = 0;  // split tiles met so far (phase of the split barriers)
     bool ok = true;
     // sigma(Q) of tile number tile_no (this thread's 64 columns) -> tensor memory
     // (O + 64 half, 32 packed columns) for the retrieval MMA; partial denominator
@@ -529,7 +612,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tmem_ld32(tS + lane_off + b * BN + col0 + 32,
                   *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
         tmem_wait_ld();
-        if (j == t.i) {
+        if ((kSplit ? t.j0 : 0) + j == t.i) {  // the diagonal key tile: causal mask
 #pragma unroll
           for (int c = 0; c < 64; ++c)
             if ((int)col0 + c > r) sr[c] = __float_as_uint(-INFINITY);
@@ -585,15 +668,18 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         f2unpack(rsum2[0], r0, r1);
         f2unpack(rsum2[1], r2, r3);
         const float rs = (r0 + r1) + (r2 + r3);
-        // PV_{j-1} must be done before O is touched (a rescale). Every PV completion
-        // is consumed once, in order: PV of the previous tile's last step in its
-        // epilogue, PV_{j-1} here for j >= 1.
-        if (j > 0 && !mbar_wait_warp(&bars[B_PVDONE], (uint32_t)((kc - 2) & 1))) {
+        // A rescale of O must wait for the previous step's P V (the S-free barrier of
+        // its buffer). Only then: without a rescale nothing here touches O. The wait
+        // cannot be misread: the barrier's previous phase completed before this
+        // step's Q K^T was issued, and its next needs a P these warps have not written.
+        const bool rescale = __any_sync(0xffffffffu, need);
+        if (rescale && j > 0 &&
+            !mbar_wait_warp(&bars[B_SFREE + ((kc - 2) & 1)], (uint32_t)(((kc - 2) >> 1) & 1))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
+        if (rescale) {
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t o[32];
@@ -611,7 +697,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tmem_st32_(tS + lane_off + b * BN + 32 * half, pk);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive_warp(&bars[B_PFULL]);
+        mbar_arrive_warp(&bars[B_PFULL + b]);
       }
       if (!ok) break;
 
@@ -631,19 +717,105 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       const float g = 1.f / (1.f + expf(-bta));
       const float den_t = den + xden[(1 - half) * 128 + r];
       const float l_t = l + xl[(1 - half) * 128 + r];
-      const float go = (1.f - g) / l_t;
       const float gr = den_t != 0.f ? g / den_t : 0.f;
-      if (!mbar_wait_warp(&bars[B_PVDONE], (uint32_t)((kc - 1) & 1)) ||
+      if (!mbar_wait_warp(&bars[B_SFREE + ((kc - 1) & 1)], (uint32_t)(((kc - 1) >> 1) & 1)) ||
           !mbar_wait_warp(&bars[B_RDONE], (uint32_t)(tc & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
+      // Split mode: every piece of a tile leaves its record (O against its reference
+      // max m_use, and the row sum); the piece that finishes last merges the records
+      // in piece order (the same sums whichever piece it is) and writes the output.
+      bool emit = true;
+      float mx = m_use, l_out = l_t;
+      const float* recs = p.rec + (size_t)t.tid * p.Pmax * kRecFloats;
+      if (kSplit && t.np > 1) {
+        float* rec = p.rec + ((size_t)t.tid * p.Pmax + t.pc) * kRecFloats;
+        float4* recO = reinterpret_cast<float4*>(rec);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + col0 + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            __stcg(recO + (half * 16 + c * 8 + q) * 128 + r,
+                   make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
+                               __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3])));
+        }
+        if (half == 0) {
+          __stcg(rec + kRecO + r, m_use);
+          __stcg(rec + kRecO + 128 + r, l_t);
+        }
+        __threadfence();  // the record is visible device-wide before the count
+        mbar_arrive_warp(&bars[B_SPLW]);
+        if (warp == 2) {
+          ok = mbar_wait_warp(&bars[B_SPLW], (uint32_t)(sc & 1));
+          if (ok && lane == 0) {
+            const unsigned done = atomicAdd(p.tile_ctr + t.tid, 1u);
+            *sflag = done == (unsigned)t.np - 1u ? 1 : 0;
+            __threadfence();
+            mbar_arrive(&bars[B_SPLF]);
+          }
+          __syncwarp();
+        }
+        if (!ok || !mbar_wait_warp(&bars[B_SPLF], (uint32_t)(sc & 1))) {
+          ok = false;
+          break;
+        }
+        ++sc;
+        emit = *sflag != 0;
+        if (emit) {
+          __threadfence();  // the other pieces' records, counted before this piece's
+          for (int q = 0; q < t.np; ++q)
+            if (q != t.pc) mx = fmaxf(mx, __ldcg(recs + q * kRecFloats + kRecO + r));
+          l_out = 0.f;
+          for (int q = 0; q < t.np; ++q) {
+            const float mq = q == t.pc ? m_use : __ldcg(recs + q * kRecFloats + kRecO + r);
+            const float lq = q == t.pc ? l_t : __ldcg(recs + q * kRecFloats + kRecO + 128 + r);
+            l_out = fmaf(ex2_approx((mq - mx) * sl), lq, l_out);
+          }
+        }
+      }
+      const float go = (1.f - g) / l_out;
       uint32_t w[32];  // this row's 64 outputs, bf16 pairs
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t o[32], rr[32];
-        tmem_ld32(tO + lane_off + col0 + c * 32, o);
+        if (!emit) break;
+        uint32_t o[32];
+        if (kSplit && t.np > 1) {  // the merged O: sum over the pieces in piece order, each scaled to mx
+          float acc[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+          for (int q = 0; q < t.np; ++q) {
+            if (q == t.pc) {
+              tmem_ld32(tO + lane_off + col0 + c * 32, o);
+              tmem_wait_ld();
+              const float a = ex2_approx((m_use - mx) * sl);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) acc[e] = fmaf(a, __uint_as_float(o[e]), acc[e]);
+            } else {
+              const float* rq = recs + q * kRecFloats;
+              const float a = ex2_approx((__ldcg(rq + kRecO + r) - mx) * sl);
+              const float4* oq = reinterpret_cast<const float4*>(rq) + (half * 16 + c * 8) * 128 + r;
+#pragma unroll
+              for (int qq = 0; qq < 8; ++qq) {
+                const float4 v4 = __ldcg(oq + qq * 128);
+                acc[4 * qq] = fmaf(a, v4.x, acc[4 * qq]);
+                acc[4 * qq + 1] = fmaf(a, v4.y, acc[4 * qq + 1]);
+                acc[4 * qq + 2] = fmaf(a, v4.z, acc[4 * qq + 2]);
+                acc[4 * qq + 3] = fmaf(a, v4.w, acc[4 * qq + 3]);
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(acc[e]);
+        } else {
+          tmem_ld32(tO + lane_off + col0 + c * 32, o);
+          tmem_wait_ld();
+        }
+        uint32_t rr[32];
         tmem_ld32(tR + lane_off + col0 + c * 32, rr);
         tmem_wait_ld();
 #pragma unroll
@@ -658,8 +830,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // TMA drops them) leaves through shared memory: each half writes its 128 x 64
       // box, 128B-swizzled, and the half's first warp issues the TMA store. Before a
       // half rewrites its box, that warp has seen its previous store finish reading.
-      const bool tma_tile =
-          p.tma_out && (t.rows_valid == BM || (long long)t.q_row + t.rows_valid == p.L);
+      const bool tma_tile = emit && p.tma_out &&
+                            (t.rows_valid == BM || (long long)t.q_row + t.rows_valid == p.L);
       const bool issuer = warp == 2 + 4 * half;
       if (tma_tile) {
         if (oc > 0) {
@@ -698,7 +870,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         ok = false;
         break;
       }
-      if (!tma_tile && r < t.rows_valid) {
+      if (emit && !tma_tile && r < t.rows_valid) {
         __nv_bfloat16* orow = out + t.b * p.o_sb + t.h * p.o_sh + (t.q_row + r) * p.o_sl + col0;
         if (p.out32) {
 #pragma unroll
@@ -729,14 +901,65 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 }  // namespace
 
 cudaError_t bf16_attn_set_attributes() {
-  return cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const cudaError_t e = cudaFuncSetAttribute(attn_kernel<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               kAttnSmem);
+}
+
+namespace {
+int split_tiles(int T, int C) {  // sum over tiles i < T of ceil((i + 1) / C)
+  int n = 0;
+  for (int i = 0; i < T; ++i) n += (i + C) / C;
+  return n;
+}
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+}  // namespace
+
+Bf16AttnSplit bf16_attn_split_plan(int BH, int S, int N, long long L, int sms) {
+  Bf16AttnSplit sp;
+  if (L <= 0 || BH < 1 || S < 1) return sp;
+  const int T = (int)((min((long long)N, L) + BM - 1) / BM);
+  const long long pairs = (long long)BH * S * ((T + 1) / 2);
+  if (pairs >= sms) return sp;
+  // Fewer pairs than SMs: whole query tiles, heaviest first, one per CTA as far as they
+  // go (no records, no merge) while there are at least half as many tiles as SMs.
+  // Fewer tiles than that: pieces, the longest that still give about 1.25 units per
+  // SM (a longer piece spends less on its prologue, record and merge), at least
+  // ceil(T / 8) key tiles each.
+  if ((long long)BH * S * T * 2 >= sms) {
+    sp.C = T;
+    sp.Pmax = 1;
+    sp.units = (long long)BH * S * T;
+    return sp;
+  }
+  const int cmin = max(1, (T + 7) / 8);
+  int C = cmin;
+  for (int c = T; c >= cmin; --c)
+    if ((long long)BH * S * split_tiles(T, c) * 4 >= 5LL * sms) {
+      C = c;
+      break;
+    }
+  sp.C = C;
+  sp.Pmax = (T + C - 1) / C;
+  sp.units = (long long)BH * S * split_tiles(T, C);
+  return sp;
+}
+
+size_t bf16_attn_split_bytes(const Bf16AttnSplit& sp, int BH, int S, int N, long long L) {
+  if (sp.C == 0) return 0;
+  const int T = (int)((min((long long)N, L) + BM - 1) / BM);
+  const size_t tiles = (size_t)BH * S * T;
+  // whole tiles (Pmax 1) leave no records
+  return 256 + up256(tiles * 4) + (sp.Pmax > 1 ? tiles * sp.Pmax * kRecFloats * sizeof(float) : 0);
 }
 
 cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                              const __nv_bfloat16* v, const float* beta, __nv_bfloat16* out,
                              const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
-                             cudaStream_t stream, const Bf16Layout* lay) {
+                             cudaStream_t stream, const Bf16Layout* lay,
+                             const Bf16AttnSplit* split, void* split_ws) {
   // query head (b, h) reads key/value head (b, h / (H / H_kv)); out is laid out as q
   const Bf16Layout l = lay ? *lay : Bf16Layout::bhld(BH / H, H, L);
   if ((long long)l.B * l.H != BH || l.H_kv < 1 || l.H % l.H_kv != 0) return cudaErrorInvalidValue;
@@ -746,7 +969,7 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
       !make_bf16_map4(&mv, v, (uint64_t)L, l.H_kv, l.B, l.kv_sl, l.kv_sh, l.kv_sb, 128) ||
       !make_bf16_map(&mm, ws.Mhl, D, (uint64_t)l.B * l.H_kv * S * 2, 128))
     return cudaErrorInvalidValue;
-  Params p;
+  Params p{};
   p.L = L;
   p.N = N;
   p.S = S;
@@ -758,7 +981,22 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   p.o_sl = l.q_sl;
   p.T = (int)((min((long long)N, L) + BM - 1) / BM);
   p.U = (p.T + 1) / 2;
-  const long long units = (long long)BH * S * p.U;
+  long long units = (long long)BH * S * p.U;
+  if (split && split->C > 0 && split_ws) {
+    // counters first (zeroed here, on the launch stream), then the records
+    const size_t tiles = (size_t)BH * S * p.T;
+    if (cudaMemsetAsync(split_ws, 0, 256 + up256(tiles * 4), stream) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    p.split = 1;
+    p.C = split->C;
+    p.Pmax = split->Pmax;
+    p.BHS = (unsigned)(BH * S);
+    p.divBHS = FastDiv(p.BHS);
+    p.unit_ctr = static_cast<unsigned*>(split_ws);
+    p.tile_ctr = reinterpret_cast<unsigned*>(static_cast<char*>(split_ws) + 256);
+    p.rec = reinterpret_cast<float*>(static_cast<char*>(split_ws) + 256 + up256(tiles * 4));
+    units = split->units;
+  }
   if (units >= (1ll << 31)) return cudaErrorInvalidValue;
   p.units = (unsigned)units;
   p.divU = FastDiv((uint32_t)p.U);
@@ -773,7 +1011,13 @@ cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const unsigned grid = p.units < (unsigned)sms ? p.units : (unsigned)sms;
-  attn_kernel<<<grid, kThreads, kAttnSmem, stream>>>(mq, mk, mv, mm, mo, beta, ws.zprev, out, p);
+  if (grid == 0) return cudaSuccess;
+  if (p.split)
+    attn_kernel<true><<<grid, kThreads, kAttnSmem, stream>>>(mq, mk, mv, mm, mo, beta, ws.zprev,
+                                                             out, p);
+  else
+    attn_kernel<false><<<grid, kThreads, kAttnSmem, stream>>>(mq, mk, mv, mm, mo, beta, ws.zprev,
+                                                              out, p);
   return cudaGetLastError();
 }
 

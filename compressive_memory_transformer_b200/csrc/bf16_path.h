@@ -50,17 +50,53 @@ cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, co
                               int CL, int mode, int first, cudaStream_t stream,
                               const Bf16Layout* lay = nullptr);
 
-// Writes the workspace's first-segment M_{-1} hi/lo and z_{-1} from M_in / z_in.
+// Writes the workspace's first-segment M_{-1} hi/lo and z_{-1} from M_in / z_in, and
+// zeroes ctr[0 .. nctr) (counters of kernels launched after it).
 cudaError_t bf16_prep_first(const float* M_in, const float* z_in, const Bf16Workspace& ws,
-                            int BH, int S, cudaStream_t stream);
+                            int BH, int S, cudaStream_t stream, unsigned* ctr = nullptr,
+                            int nctr = 0);
+
+// The memory update of a call holding one segment (bf16_step_state.cu): CTAs per (head,
+// token chunk, column block) compute sigma(K)^T (V - sigma(K) M_in / den) in parallel
+// and the last CTA of each (head, column block) adds the chunks to M_in in chunk order.
+// Reads the workspace's M_{-1} hi/lo and z_{-1} (bf16_prep_first) and k, v; writes
+// M_out, z_out. step_ws holds bf16_step_state_bytes(BH, CH) bytes whose counters
+// (bf16_step_state_counters, 2 * BH of them) are zero at the launch. BH counts key/value
+// heads.
+void bf16_step_state_plan(int BH, int N, int* CH, int* CL);
+size_t bf16_step_state_bytes(int BH, int CH);
+unsigned* bf16_step_state_counters(void* step_ws, int BH, int CH);
+cudaError_t bf16_step_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                   const float* M_in, float* M_out, float* z_out,
+                                   const Bf16Workspace& ws, void* step_ws, int BH, int N, int CH,
+                                   int CL, int mode, cudaStream_t stream,
+                                   const Bf16Layout* lay = nullptr);
+
+// Split mode of the attention kernel, for calls whose query-tile pairs are fewer than
+// the SMs (one segment of a few heads, short sequences): each query tile's key range
+// is cut into pieces of at most C key tiles, the pieces are taken from a device
+// counter heaviest first, and the last piece of a tile to finish merges the pieces'
+// partial results (log-sum-exp weights, fixed piece order) into the output.
+struct Bf16AttnSplit {
+  int C = 0;             // 0: no split (tile pairs dealt out round-robin)
+  int Pmax = 0;          // most pieces of one tile
+  long long units = 0;   // pieces in the call
+};
+// BH counts query heads (B * H).
+Bf16AttnSplit bf16_attn_split_plan(int BH, int S, int N, long long L, int sms);
+// Scratch of a split call (counters and partial records; 0 without a split).
+size_t bf16_attn_split_bytes(const Bf16AttnSplit& sp, int BH, int S, int N, long long L);
 
 // The fused local-attention + retrieval + gate kernel. Reads q, k, v, beta and
 // the workspace's zprev / Mhl; writes out.
 // BH counts query heads (B * H); the workspace holds the key/value heads' states.
+// split / split_ws: a split plan and bf16_attn_split_bytes(...) bytes of scratch
+// (zeroed counters are set up on `stream` before the kernel); NULL: tile pairs.
 cudaError_t bf16_attn_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
                              const __nv_bfloat16* v, const float* beta, __nv_bfloat16* out,
                              const Bf16Workspace& ws, int BH, int H, long long L, int N, int S,
-                             cudaStream_t stream, const Bf16Layout* lay = nullptr);
+                             cudaStream_t stream, const Bf16Layout* lay = nullptr,
+                             const Bf16AttnSplit* split = nullptr, void* split_ws = nullptr);
 
 // Gradient of the bf16 forward (bf16_bwd.cu): [B, H, L, 128] contiguous, N a multiple
 // of 128, L a multiple of N. `scratch` holds bf16_bwd_workspace_bytes(...) bytes; CH /

@@ -616,10 +616,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
 // Writes what the attention kernel reads for the first segment, M_{-1} = M_in as
 // hi / lo bf16 and z_{-1} = z_in (zero when absent), exactly as chain_kernel and
 // zscan_kernel would, so that a one-segment call can run the attention beside the
-// state update.
+// state update; block (0, 0) also zeroes the counters of the kernels that follow.
 __global__ void __launch_bounds__(D) prep_first_kernel(const float* M_in, const float* z_in,
                                                        __nv_bfloat16* __restrict__ Mhl,
-                                                       float* __restrict__ zprev, int S) {
+                                                       float* __restrict__ zprev, int S,
+                                                       unsigned* ctr, int nctr) {
+  if (blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = threadIdx.x; i < nctr; i += blockDim.x) ctr[i] = 0u;
   const int bh = blockIdx.x, r = blockIdx.y * 8 + (threadIdx.x >> 4), c = (threadIdx.x & 15) * 8;
   float m[8];
   if (M_in) {
@@ -652,8 +655,9 @@ __global__ void __launch_bounds__(D) prep_first_kernel(const float* M_in, const 
 }  // namespace
 
 cudaError_t bf16_prep_first(const float* M_in, const float* z_in, const Bf16Workspace& ws,
-                            int BH, int S, cudaStream_t stream) {
-  prep_first_kernel<<<dim3(BH, D / 8), D, 0, stream>>>(M_in, z_in, ws.Mhl, ws.zprev, S);
+                            int BH, int S, cudaStream_t stream, unsigned* ctr, int nctr) {
+  prep_first_kernel<<<dim3(BH, D / 8), D, 0, stream>>>(M_in, z_in, ws.Mhl, ws.zprev, S, ctr,
+                                                       nctr);
   return cudaGetLastError();
 }
 

@@ -25,6 +25,7 @@ cudaError_t bf16_state_set_attributes();
 cudaError_t bf16_attn_set_attributes();
 cudaError_t bf16_bwd_set_attributes();
 cudaError_t bf16_gemm_set_attributes();
+cudaError_t bf16_step_state_set_attributes();
 
 namespace {
 
@@ -56,6 +57,7 @@ cudaError_t prepare_device(int* dev_out) {
   if (e == cudaSuccess) e = bf16_attn_set_attributes();
   if (e == cudaSuccess) e = bf16_bwd_set_attributes();
   if (e == cudaSuccess) e = bf16_gemm_set_attributes();
+  if (e == cudaSuccess) e = bf16_step_state_set_attributes();
   SideStream& sd = g_side[dev];
   if (e == cudaSuccess && !sd.stream) e = cudaStreamCreateWithFlags(&sd.stream, cudaStreamNonBlocking);
   if (e == cudaSuccess && !sd.fork) e = cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming);
@@ -186,6 +188,41 @@ int get_scratch(Scratch& s, size_t bytes, const infini_attn_opts_t* opts, cudaSt
   return INFINI_OK;
 }
 
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  return sms;
+}
+
+// Scratch of one bf16 forward: the state path's workspace, then (one segment) the
+// one-segment update's partial sums, then (calls with fewer query-tile pairs than
+// SMs) the attention's split scratch.
+struct FwdPlan {
+  int CH = 1, CL = 1;        // multi-segment state GEMM: token chunks
+  int sCH = 0, sCL = 0;      // one segment: token chunks of the update
+  Bf16AttnSplit split;
+  size_t state_bytes = 0, step_bytes = 0, bytes = 0;
+};
+
+FwdPlan fwd_plan(int BH, int BHkv, int S, int N, long long L) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  FwdPlan f;
+  f.CL = N;
+  bf16_state_plan(BHkv, S, N, &f.CH, &f.CL);
+  f.split = bf16_attn_split_plan(BH, S, N, L, device_sms());
+  f.state_bytes = up(bf16_workspace_bytes(BHkv, S, f.CH));
+  if (S == 1 && L > 0) {
+    bf16_step_state_plan(BHkv, (int)min((long long)N, L), &f.sCH, &f.sCL);
+    f.step_bytes = up(bf16_step_state_bytes(BHkv, f.sCH));
+  }
+  f.bytes = f.state_bytes + f.step_bytes + bf16_attn_split_bytes(f.split, BH, S, N, L);
+  return f;
+}
+
 void record(const infini_attn_opts_t* opts, int i, cudaStream_t stream) {
   if (opts && opts->stage_events[i])
     cudaEventRecord(static_cast<cudaEvent_t>(opts->stage_events[i]), stream);
@@ -237,13 +274,16 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
     record(opts, 2, stream);
     return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
   }
-  int CH = 1, CL = N;
-  bf16_state_plan(BHkv, S, N, &CH, &CL);
+  const FwdPlan fp = fwd_plan(BH, BHkv, S, N, L);
+  const int CH = fp.CH, CL = fp.CL;
   if ((long long)BHkv * S * CH >= (1LL << 31)) return INFINI_ERR_SHAPE;
   Scratch sc;
-  st = get_scratch(sc, bf16_workspace_bytes(BHkv, S, CH), opts, stream);
+  st = get_scratch(sc, fp.bytes, opts, stream);
   if (st != INFINI_OK) return st;
   const Bf16Workspace ws = bf16_workspace_carve(sc.ptr, BHkv, S, CH);
+  void* step_ws = fp.step_bytes ? static_cast<char*>(sc.ptr) + fp.state_bytes : nullptr;
+  void* split_ws =
+      fp.split.C ? static_cast<char*>(sc.ptr) + fp.state_bytes + fp.step_bytes : nullptr;
   const auto* qb = static_cast<const __nv_bfloat16*>(q);
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
   const auto* vb = static_cast<const __nv_bfloat16*>(v);
@@ -251,16 +291,30 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
   if (S == 1) {
     // One segment: the attention reads only the incoming state (M_in, z_in), so it
     // runs beside the state update, which goes to the side stream and is joined
-    // back before the call returns.
+    // back before the call returns. The update is the one-segment kernel (chunks of
+    // tokens in parallel, no chain); without M_out there is no update to make.
+    const int nseg = (int)min((long long)N, L);
+    unsigned* sctr = step_ws ? bf16_step_state_counters(step_ws, BHkv, fp.sCH) : nullptr;
+    cudaError_t e = bf16_prep_first(M_in, z_in, ws, BHkv, S, stream, sctr, sctr ? 2 * BHkv : 0);
+    if (e != cudaSuccess) return INFINI_ERR_CUDA;
+    if (!M_out) {
+      record(opts, 1, stream);
+      e = bf16_attn_launch(qb, kb, vb, beta, static_cast<__nv_bfloat16*>(out), ws, BH, H, L, N,
+                           S, stream, &lay, &fp.split, split_ws);
+      record(opts, 2, stream);
+      return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
+    }
     SideStream& sd = g_side[dev];
     std::lock_guard<std::mutex> lk(sd.mu);
-    cudaError_t e = bf16_prep_first(M_in, z_in, ws, BHkv, S, stream);
-    if (e == cudaSuccess) e = cudaEventRecord(sd.fork, stream);
+    e = cudaEventRecord(sd.fork, stream);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(sd.stream, sd.fork, 0);
     if (e != cudaSuccess) return INFINI_ERR_CUDA;
-    const cudaError_t es = bf16_state_launch(kb, vb, M_in, z_in, M_out, z_out, ws, BHkv, L, N, S,
-                                             CH, CL, mode, 1, sd.stream, &lay);
+    const cudaError_t es = bf16_step_state_launch(kb, vb, M_in, M_out, z_out, ws, step_ws, BHkv,
+                                                  nseg, fp.sCH, fp.sCL, mode, sd.stream, &lay);
     record(opts, 1, stream);
+    // Beside the state update the attention keeps its tile pairs: split units would
+    // want the SMs the update holds (measured on 8 heads of one 2048-token segment:
+    // 33.6 us per step with pairs, 36.9 with whole tiles taken from the counter).
     const cudaError_t ea = bf16_attn_launch(qb, kb, vb, beta, static_cast<__nv_bfloat16*>(out),
                                             ws, BH, H, L, N, S, stream, &lay);
     // joined even after a launch error, so that the side stream never runs ahead of
@@ -276,7 +330,7 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
   if (e != cudaSuccess) return INFINI_ERR_CUDA;
   record(opts, 1, stream);
   e = bf16_attn_launch(qb, kb, vb, beta, static_cast<__nv_bfloat16*>(out), ws, BH, H, L, N, S,
-                       stream, &lay);
+                       stream, &lay, &fp.split, split_ws);
   record(opts, 2, stream);
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
@@ -493,9 +547,7 @@ int layer_forward_impl(const void* x, const void* Wq, const void* Wk, const void
   // the projections' outputs, then the forward's own scratch
   const size_t proj_bytes = ((2 * nq + 2 * nkv) * 2 + 255) & ~(size_t)255;
   const int S = (int)((L + N - 1) / N);
-  int CH = 1, CL = N;
-  bf16_state_plan(B * H_kv, S, N, &CH, &CL);
-  const size_t fwd_bytes = bf16_workspace_bytes(B * H_kv, S, CH);
+  const size_t fwd_bytes = fwd_plan(B * H, B * H_kv, S, N, L).bytes;
   Scratch sc;
   infini_attn_opts_t ws_opts;
   memset(&ws_opts, 0, sizeof(ws_opts));
@@ -622,9 +674,7 @@ size_t infini_attn_workspace_size(int B, int H, long long L, int N, int d, int m
   const int BH = B * H;
   const int S = (int)((L + N - 1) / N);
   if (dtype == INFINI_DTYPE_F32) return f32_workspace_bytes(BH, S, d);
-  int CH = 1, CL = N;
-  bf16_state_plan(BH, S, N, &CH, &CL);
-  return bf16_workspace_bytes(BH, S, CH);
+  return fwd_plan(BH, BH, S, N, L).bytes;
 }
 
 int infini_attn_forward_ex(const void* q, const void* k, const void* v, const float* beta,
@@ -706,9 +756,7 @@ size_t infini_attn_layer_workspace_size(int B, long long L, int D_model, int H, 
   const size_t nq = (size_t)(rows * H * d), nkv = (size_t)(rows * H_kv * d);
   const size_t proj_bytes = ((2 * nq + 2 * nkv) * 2 + 255) & ~(size_t)255;
   const int S = (int)((L + N - 1) / N);
-  int CH = 1, CL = N;
-  bf16_state_plan(B * H_kv, S, N, &CH, &CL);
-  return proj_bytes + bf16_workspace_bytes(B * H_kv, S, CH);
+  return proj_bytes + fwd_plan(B * H, B * H_kv, S, N, L).bytes;
 }
 
 int infini_attn_device_status(void) {

@@ -55,9 +55,11 @@ class Sim:
                     state[r] = req
                 if req[0] == 'wait':
                     b, k = req[1], req[2]
-                    # a waiter for completion k must not find the barrier past k + 1:
-                    # its parity would then match a later phase
+                    # a waiter for completion k must not find the barrier past k + 1 (its
+                    # parity would then match a later phase) nor before k (it would match
+                    # an older one)
                     assert b.done <= k + 1, f"{b.name}: phase skipped (waiter for {k}, done {b.done})"
+                    assert b.done >= k, f"{b.name}: stale phase (waiter for {k}, done {b.done})"
                     if b.done >= k + 1:
                         ready.append(r)
                 elif req[0] == 'named':
@@ -386,20 +388,25 @@ def test_model_detects_a_deadlock():
 # the forward attention kernel (one persistent CTA walking its list of query tiles)
 # ------------------------------------------------------------------------------
 def attn_roles(sim, tiles):
-    """tiles: list of (nkv, tma_out) per query tile of the CTA's list."""
+    """tiles: list of (nkv, tma_out[, piece, merges]) per query tile of the CTA's list;
+    piece: the tile is one piece of a split key range (its record is written and
+    counted: the split barriers), merges: this piece finished last and writes the
+    merged output (otherwise it writes none)."""
     QFULL, QEMPTY = sim.bar("qfull"), sim.bar("qempty", 9)   # QK commit + 8 softmax warps
     KFULL = [sim.bar(f"kfull{i}") for i in range(2)]
     SFREE = [sim.bar(f"sfree{i}") for i in range(2)]
     VFULL = [sim.bar(f"vfull{i}") for i in range(2)]
     VEMPTY = [sim.bar(f"vempty{i}") for i in range(2)]
     SFULL = [sim.bar(f"sfull{i}") for i in range(2)]
-    PFULL, PVDONE, RDONE = sim.bar("pfull", 8), sim.bar("pvdone"), sim.bar("rdone")
+    PFULL = [sim.bar(f"pfull{i}", 8) for i in range(2)]   # one per S buffer
+    RDONE = sim.bar("rdone")
     SQFULL = sim.bar("sqfull", 8)
     DRAIN = sim.bar("drain", 2)
     PAIR = [sim.bar(f"pair{i}", 2) for i in range(4)]
     OFULL = [sim.bar(f"ofull{i}", 4) for i in range(2)]
     OFREE = [sim.bar(f"ofree{i}") for i in range(2)]
     STORE = [sim.bar(f"storeread{i}") for i in range(2)]  # a TMA store has read its tile
+    SPLW, SPLF = sim.bar("split_written", 8), sim.bar("split_flag")
     ntiles = len(tiles)
 
     def producer():
@@ -421,7 +428,8 @@ def attn_roles(sim, tiles):
             yield ('tma', VFULL[st])
             v_use[st] += 1
             vst[0] ^= 1
-        for tc, (nkv, _) in enumerate(tiles):
+        for tc, tile in enumerate(tiles):
+            nkv = tile[0]
             if tc > 0:
                 yield ('wait', QEMPTY, tc - 1)
             yield ('tma', QFULL)                   # Q (and z), after the descriptor slot
@@ -472,43 +480,55 @@ def attn_roles(sim, tiles):
             vit += 1
             for j in range(nkv):
                 st = vit & 1
-                yield ('wait', PFULL, n)
+                yield ('wait', PFULL[n & 1], n >> 1)
                 yield ('wait', VFULL[st], vit >> 1)
                 yield ('mma', 'pv')
                 yield ('commit', VEMPTY[st], 'pv')
-                yield ('commit', PVDONE, 'pv')
-                yield ('commit', SFREE[n & 1], 'pv')
+                yield ('commit', SFREE[n & 1], 'pv')       # P V done: S free, O readable
                 vit += 1
                 n += 1
         yield ('commit', DRAIN, 'pv')
         yield ('wait', DRAIN, 0)
 
+    rescale_rng = random.Random(len(tiles) * 7919 + sum(t[0] for t in tiles))
+
     def softmax(w):
         half, wq = w // 4, w % 4
+        rng = random.Random(rescale_rng.random() + w)   # each warp decides its own rescales
         issuer = wq == 0
-        kc, pph, oc, stores = 0, 0, 0, 0
+        kc, pph, oc, stores, sc = 0, 0, 0, 0, 0
         yield ('wait', QFULL, 0)
         if ntiles == 0:
             yield ('arrive', SQFULL, 1)
             return
         yield ('arrive', QEMPTY, 1)                   # sigma(Q) of tile 0
         yield ('arrive', SQFULL, 1)
-        for tc, (nkv, tma_out) in enumerate(tiles):
+        for tc, tile in enumerate(tiles):
+            nkv, tma_out = tile[0], tile[1]
+            piece = len(tile) > 2 and tile[2]
+            emit = not piece or tile[3]
             for j in range(nkv):
                 yield ('wait', SFULL[kc & 1], kc >> 1)
                 kc += 1
                 yield ('arrive', PAIR[wq], 1)
                 yield ('wait', PAIR[wq], pph)
                 pph += 1
-                if j > 0:
-                    yield ('wait', PVDONE, kc - 2)
-                yield ('arrive', PFULL, 1)
+                if j > 0 and rng.random() < 0.3:           # a rescale of O: P V of the
+                    yield ('wait', SFREE[(kc - 2) & 1], (kc - 2) >> 1)   # previous step
+                yield ('arrive', PFULL[(kc - 1) & 1], 1)
             yield ('arrive', PAIR[wq], 1)              # epilogue: row sums exchanged
             yield ('wait', PAIR[wq], pph)
             pph += 1
-            yield ('wait', PVDONE, kc - 1)
+            yield ('wait', SFREE[(kc - 1) & 1], (kc - 1) >> 1)    # the tile's last P V
             yield ('wait', RDONE, tc)
-            if tma_out:
+            if piece:                                  # record written, then counted
+                yield ('arrive', SPLW, 1)
+                if w == 0:
+                    yield ('wait', SPLW, sc)
+                    yield ('arrive', SPLF, 1)           # the merge decision, broadcast
+                yield ('wait', SPLF, sc)
+                sc += 1
+            if tma_out and emit:
                 if oc > 0:
                     if issuer:
                         yield ('wait', STORE[half], stores - 1)   # its last store has read
@@ -564,6 +584,7 @@ class SimPerWarp(Sim):
                 if req[0] == 'wait':
                     b, k = req[1], req[2]
                     assert b.done <= k + 1, f"{b.name}: phase skipped (waiter for {k}, done {b.done})"
+                    assert b.done >= k, f"{b.name}: stale phase (waiter for {k}, done {b.done})"
                     if b.done >= k + 1:
                         ready.append(r)
                 else:
@@ -606,6 +627,77 @@ def test_attention_kernel_protocol(seed):
     tiles = [(rng.randint(1, 6), rng.random() < 0.8) for _ in range(rng.randint(0, 6))]
     sim = SimPerWarp(seed)
     sim.run(attn_roles(sim, tiles))
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_attention_kernel_protocol_split_pieces(seed):
+    """Split mode: lists that mix whole tiles with pieces of split key ranges (1 to 4
+    key tiles), some of which merge and store the tile and some of which only leave
+    their record."""
+    rng = random.Random(1000 + seed)
+    tiles = []
+    for _ in range(rng.randint(1, 7)):
+        piece = rng.random() < 0.7
+        tiles.append((rng.randint(1, 4), rng.random() < 0.8, piece, rng.random() < 0.5))
+    sim = SimPerWarp(seed)
+    sim.run(attn_roles(sim, tiles))
+
+
+def test_attention_model_detects_a_wrong_split_count():
+    """Planted mistake: the records barrier counts one arrival per warp of one
+    warpgroup (4) instead of all eight softmax warps, so it completes twice per piece
+    and the counting warp's parity wait would see a later phase."""
+    def broken(sim, tiles):
+        roles = attn_roles(sim, tiles)
+        sim.bars["split_written"].count = sim.bars["split_written"].pending = 4
+        return roles
+    failures = 0
+    for seed in range(30):
+        sim = SimPerWarp(seed)
+        try:
+            sim.run(broken(sim, [(2, True, True, False), (1, True, True, True),
+                                 (3, False, True, False), (2, True, True, True)]))
+        except AssertionError:
+            failures += 1
+    assert failures > 0
+
+
+def test_attention_model_detects_a_conditional_wait_on_a_shared_pv_barrier():
+    """Planted mistake: one P-V-done barrier committed after every P V and waited only
+    when a rescale needs O. Skipped phases leave it behind the waiter's count, where a
+    parity wait would pass on an older phase (the kernel waits on the S buffer's S-free
+    barrier instead, which the Q K^T warp keeps in step)."""
+    def broken(sim, tiles):
+        roles = attn_roles(sim, tiles)
+        PV = sim.bar("pvdone_shared")
+        SFREE = [sim.bars["sfree0"], sim.bars["sfree1"]]
+        old_pv, softs = roles["pv"], {w: roles[f"softmax{w}"] for w in range(8)}
+
+        def pv():
+            for req in old_pv:
+                yield req
+                if req[0] == 'commit' and req[1] in SFREE:
+                    yield ('commit', PV, 'pv')
+
+        def soft(g):
+            count = 0
+            for req in g:
+                if req[0] == 'wait' and req[1] in SFREE:
+                    yield ('wait', PV, req[2] * 2 + SFREE.index(req[1]))
+                    continue
+                yield req
+        roles["pv"] = pv()
+        for w in range(8):
+            roles[f"softmax{w}"] = soft(softs[w])
+        return roles
+    failures = 0
+    for seed in range(30):
+        sim = SimPerWarp(seed)
+        try:
+            sim.run(broken(sim, [(6, True), (5, True), (6, False), (4, True)]))
+        except AssertionError:
+            failures += 1
+    assert failures > 0
 
 
 def test_attention_model_detects_a_missing_sfree_wait():
