@@ -16,6 +16,7 @@
 #include <cuda_bf16.h>
 #include <cuda.h>
 #include <cstdint>
+#include <cstring>
 
 #include "bf16_path.h"
 #include "sm100.cuh"
@@ -33,10 +34,21 @@ constexpr int kGemmSmem = kStages * 2 * kTile + 256 + 1024;
 enum { G_FULL = 0, G_EMPTY = 3, G_AFULL = 6, G_AEMPTY = 8, G_DRAIN = 10, G_COUNT = 11 };
 
 struct GemmParams {
-  int tiles_n;     // N / 128
-  int ksteps;      // K / 128
-  unsigned tiles;  // (M / 128) * (N / 128)
+  int tiles_n;     // N / 128 (wide kernel: N / 256, summed over the column groups)
+  int ksteps;      // K / 128 (wide kernel: K / 64)
+  unsigned tiles;  // (M / 128) * tiles_n
   long long ldc;   // N
+};
+
+// The wide kernel's column groups: C_g = A B_g for up to three B matrices that share A
+// (the layer's Q, K and V projections of the same x in one launch, so that each
+// 128-row block of A is fetched once for all of them). Group g covers the column tiles
+// [first[g], first[g + 1]) of the launch.
+struct GemmGroups {
+  int n;                     // groups (1..3)
+  int first[4];              // first column tile of each group, then the total
+  __nv_bfloat16* C[3];       // outputs
+  long long ldc[3];          // their row strides (elements)
 };
 
 __device__ __forceinline__ uint64_t kdesc_g(uint32_t base, int kk) {
@@ -202,9 +214,14 @@ constexpr int kWStages = 4;
 constexpr int kWA = 16384, kWB = 32768, kWStage = kWA + kWB;
 constexpr int kGemmWSmem = kWStages * kWStage + 256 + 1024;
 
+__device__ __forceinline__ int gemm_group(const GemmGroups& gr, int tn) {
+  return tn < gr.first[1] ? 0 : (tn < gr.first[2] ? 1 : 2);
+}
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
-gemm_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                 __nv_bfloat16* __restrict__ C, const GemmParams p) {
+gemm_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
+                 const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_b2,
+                 const GemmParams p, const GemmGroups gr) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -216,7 +233,9 @@ gemm_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     for (int x = 0; x < 13; ++x) mbar_init(&bars[x], (x == 10 || x == 11) ? 4u : 1u);
     fence_barrier_init();
     tma_prefetch_desc(&tm_a);
-    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_b0);
+    if (gr.n > 1) tma_prefetch_desc(&tm_b1);
+    if (gr.n > 2) tma_prefetch_desc(&tm_b2);
   }
   if (warp == 5) {
     tmem_alloc(tmem_slot, 512);
@@ -234,6 +253,8 @@ gemm_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
       int iss[kWStages] = {0, 0, 0, 0};
       for (unsigned t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
         const int tm = (int)(t / (unsigned)p.tiles_n), tn = (int)(t % (unsigned)p.tiles_n);
+        const int g = gemm_group(gr, tn), tl = tn - gr.first[g];
+        const CUtensorMap* tmb = g == 0 ? &tm_b0 : (g == 1 ? &tm_b1 : &tm_b2);
         for (int ks = 0; ks < p.ksteps; ++ks, ++it) {
           const int st = it % kWStages, use = it / kWStages;
           if (use > 0 && !mbar_wait(&bars[4 + st], (uint32_t)((use - 1) & 1))) {
@@ -246,7 +267,7 @@ gemm_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
           tma_load_2d(sa, &tm_a, &bars[st], 64 * ks, 128 * tm);
 #pragma unroll
           for (int a4 = 0; a4 < 4; ++a4)
-            tma_load_2d(sb + a4 * 8192, &tm_b, &bars[st], 256 * tn + 64 * a4, 64 * ks);
+            tma_load_2d(sb + a4 * 8192, tmb, &bars[st], 256 * tl + 64 * a4, 64 * ks);
           ++iss[st];
         }
       }
@@ -299,7 +320,8 @@ gemm_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
       }
       tc_fence_after();
       const int tm = (int)(t / (unsigned)p.tiles_n), tn = (int)(t % (unsigned)p.tiles_n);
-      __nv_bfloat16* dst = C + (size_t)(128 * tm + r) * p.ldc + 256 * tn;
+      const int g = gemm_group(gr, tn);
+      __nv_bfloat16* dst = gr.C[g] + (size_t)(128 * tm + r) * gr.ldc[g] + 256 * (tn - gr.first[g]);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t v[128];
@@ -356,6 +378,44 @@ cudaError_t bf16_gemm_set_attributes() {
                               kGemmWSmem);
 }
 
+cudaError_t bf16_gemm_grouped_launch(const __nv_bfloat16* A, const __nv_bfloat16* const* B,
+                                     __nv_bfloat16* const* C, const int* N, int ngroups,
+                                     long long M, int K, cudaStream_t stream) {
+  if (ngroups < 1 || ngroups > 3 || M <= 0 || K <= 0 || M % 128 || K % 128)
+    return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  CUtensorMap ma, mb[3];
+  if (!make_bf16_map2(&ma, A, (uint64_t)M, (uint64_t)K, 128)) return cudaErrorInvalidValue;
+  GemmGroups gr;
+  memset(&gr, 0, sizeof(gr));
+  gr.n = ngroups;
+  for (int g = 0; g < ngroups; ++g) {
+    if (N[g] <= 0 || N[g] % 256 != 0) return cudaErrorInvalidValue;
+    if (!make_bf16_map2(&mb[g], B[g], (uint64_t)K, (uint64_t)N[g], 64)) return cudaErrorInvalidValue;
+    gr.C[g] = C[g];
+    gr.ldc[g] = N[g];
+    gr.first[g + 1] = gr.first[g] + N[g] / 256;
+  }
+  for (int g = ngroups; g < 3; ++g) {
+    mb[g] = mb[0];
+    gr.first[g + 1] = gr.first[g];
+    gr.C[g] = C[0];
+    gr.ldc[g] = 0;
+  }
+  GemmParams p;
+  p.tiles_n = gr.first[ngroups];
+  p.ksteps = K / 64;
+  const long long tiles = (M / 128) * (long long)p.tiles_n;
+  if (tiles >= (1ll << 31)) return cudaErrorInvalidValue;
+  p.tiles = (unsigned)tiles;
+  p.ldc = 0;
+  const unsigned grid = p.tiles < (unsigned)sms ? p.tiles : (unsigned)sms;
+  gemm_wide_kernel<<<grid, kGemmThreads, kGemmWSmem, stream>>>(ma, mb[0], mb[1], mb[2], p, gr);
+  return cudaGetLastError();
+}
+
 cudaError_t bf16_gemm_launch(const __nv_bfloat16* A, const __nv_bfloat16* B, __nv_bfloat16* C,
                              long long M, int N, int K, cudaStream_t stream) {
   if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 128) return cudaErrorInvalidValue;
@@ -363,20 +423,10 @@ cudaError_t bf16_gemm_launch(const __nv_bfloat16* A, const __nv_bfloat16* B, __n
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (N % 256 == 0) {  // 128 x 256 tiles
-    CUtensorMap ma, mb;
-    if (!make_bf16_map2(&ma, A, (uint64_t)M, (uint64_t)K, 128) ||
-        !make_bf16_map2(&mb, B, (uint64_t)K, (uint64_t)N, 64))
-      return cudaErrorInvalidValue;
-    GemmParams p;
-    p.tiles_n = N / 256;
-    p.ksteps = K / 64;
-    const long long tiles = (M / 128) * (long long)(N / 256);
-    if (tiles >= (1ll << 31)) return cudaErrorInvalidValue;
-    p.tiles = (unsigned)tiles;
-    p.ldc = N;
-    const unsigned grid = p.tiles < (unsigned)sms ? p.tiles : (unsigned)sms;
-    gemm_wide_kernel<<<grid, kGemmThreads, kGemmWSmem, stream>>>(ma, mb, C, p);
-    return cudaGetLastError();
+    const __nv_bfloat16* Bs[1] = {B};
+    __nv_bfloat16* Cs[1] = {C};
+    const int Ns[1] = {N};
+    return bf16_gemm_grouped_launch(A, Bs, Cs, Ns, 1, M, K, stream);
   }
   CUtensorMap ma, mb;
   if (!make_bf16_map2(&ma, A, (uint64_t)M, (uint64_t)K) ||

@@ -115,6 +115,11 @@ cudaError_t bf16_backward_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
 // M, N, K multiples of 128.
 cudaError_t bf16_gemm_launch(const __nv_bfloat16* A, const __nv_bfloat16* B, __nv_bfloat16* C,
                              long long M, int N, int K, cudaStream_t stream);
+// C_g = A B_g (g < ngroups <= 3) in one launch: B_g [K][N_g], C_g [M][N_g] row-major, every
+// N_g a multiple of 256; each 128-row block of A is fetched once for all the groups.
+cudaError_t bf16_gemm_grouped_launch(const __nv_bfloat16* A, const __nv_bfloat16* const* B,
+                                     __nv_bfloat16* const* C, const int* N, int ngroups,
+                                     long long M, int K, cudaStream_t stream);
 
 // Token-level decode (bf16_decode.cu): partial attention over the KV cache (rows
 // below pos) and the new rows (k, v, also written into the caches), split like flash

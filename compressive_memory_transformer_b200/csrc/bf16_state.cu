@@ -148,7 +148,6 @@ __global__ void __launch_bounds__(D) zscan_kernel(const float* __restrict__ zpar
 // ---------------------------------------------------------------------------
 constexpr int kSlab = 64;
 constexpr int kStages = 3;
-constexpr int kMufuFeat = 4;  // of a converter thread's 8 features, these take the MUFU exp
 constexpr int kConvRows = 32;  // token rows converted at once (16 threads per row)
 constexpr int kBox = kSlab * 128;          // one 64-row x 64-feature box: 8 KB
 constexpr int kMat = 2 * kBox;             // one [64 x 128] bf16 matrix: 16 KB
@@ -294,22 +293,13 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
         const uint4 raw = *reinterpret_cast<const uint4*>(st + OFF_KH + off);
         float f[8];
         bf16x8_to_f32(raw, f);
-        // sigma(K): half of the exponentials on the FMA pipe (ex2_poly2), the rest on
-        // the MUFU, which the bf16 conversions below also load
+        // sigma(K), every exponential on the MUFU: the converters are bound by their
+        // instruction issue, and the FMA-pipe polynomial costs more instructions (with
+        // half of the exponentials on it the state path was 3-4% slower, measured at
+        // the 1B-layer shape in both modes)
         float den = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          if (e >= kMufuFeat) {
-            const float kLog2e = 1.4426950408889634f;
-            float p0, p1;
-            ex2_poly2(fminf(f[e], 0.f) * kLog2e, fminf(f[e + 1], 0.f) * kLog2e, p0, p1);
-            f[e] = f[e] > 0.f ? f[e] + 1.f : p0;
-            f[e + 1] = f[e + 1] > 0.f ? f[e + 1] + 1.f : p1;
-          } else {
-            f[e] = elu1(f[e]);
-            f[e + 1] = elu1(f[e + 1]);
-          }
-        }
+        for (int e = 0; e < 8; ++e) f[e] = elu1(f[e]);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           f[e] = valid ? f[e] : 0.f;

@@ -419,15 +419,21 @@ int decode_impl(const void* q, const void* k, const void* v, const float* beta, 
                          (int)BH, H, n, pos, N, sms, stream) != cudaSuccess)
     return INFINI_ERR_CUDA;
   if (pos + n < N) return INFINI_OK;
-  int CH = 1, CL = N;
-  bf16_state_plan((int)BH, 1, N, &CH, &CL);
+  // the completed segment's update, in place: the one-segment state kernel over the
+  // cache (token chunks in parallel, the chunks added to M in chunk order)
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  int sCH = 1, sCL = N;
+  bf16_step_state_plan((int)BH, N, &sCH, &sCL);
+  const size_t state_bytes = up(bf16_workspace_bytes((int)BH, 1, 1));
   Scratch sc;
-  st = get_scratch(sc, bf16_workspace_bytes((int)BH, 1, CH), nullptr, stream);
+  st = get_scratch(sc, state_bytes + bf16_step_state_bytes((int)BH, sCH), nullptr, stream);
   if (st != INFINI_OK) return st;
-  const Bf16Workspace ws = bf16_workspace_carve(sc.ptr, (int)BH, 1, CH);
-  cudaError_t e = bf16_prep_first(M, z, ws, (int)BH, 1, stream);
+  const Bf16Workspace ws = bf16_workspace_carve(sc.ptr, (int)BH, 1, 1);
+  void* step_ws = static_cast<char*>(sc.ptr) + state_bytes;
+  cudaError_t e = bf16_prep_first(M, z, ws, (int)BH, 1, stream,
+                                  bf16_step_state_counters(step_ws, (int)BH, sCH), 2 * (int)BH);
   if (e == cudaSuccess)
-    e = bf16_state_launch(kcb, vcb, M, z, M, z, ws, (int)BH, N, N, 1, CH, CL, mode, 1, stream);
+    e = bf16_step_state_launch(kcb, vcb, M, M, z, ws, step_ws, (int)BH, N, sCH, sCL, mode, stream);
   return e == cudaSuccess ? INFINI_OK : INFINI_ERR_CUDA;
 }
 
@@ -511,7 +517,8 @@ int gemm_checks(const void* A, const void* Bm, const void* C, long long M, int N
 }
 
 // One attention layer: q, k, v = x W_Q, x W_K, x W_V ([B, L, heads * d], the heads'
-// columns side by side, read in place as [B, L, heads, d]), the grouped-head forward,
+// columns side by side, read in place as [B, L, heads, d]; the three products in one
+// GEMM launch when every width is a multiple of 256), the grouped-head forward,
 // y = [A_1 ... A_H] W_O.
 int layer_forward_impl(const void* x, const void* Wq, const void* Wk, const void* Wv,
                        const void* Wo, const float* beta, const float* M_in, const float* z_in,
@@ -563,14 +570,25 @@ int layer_forward_impl(const void* x, const void* Wq, const void* Wk, const void
   __nv_bfloat16* v = k + nkv;
   __nv_bfloat16* a = v + nkv;  // the heads' outputs, [B, L, H, d]
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
-  cudaError_t e = bf16_gemm_launch(xb, static_cast<const __nv_bfloat16*>(Wq), q, rows, H * d,
-                                   D_model, stream);
-  if (e == cudaSuccess)
-    e = bf16_gemm_launch(xb, static_cast<const __nv_bfloat16*>(Wk), k, rows, H_kv * d, D_model,
+  cudaError_t e;
+  if ((H * d) % 256 == 0 && (H_kv * d) % 256 == 0) {
+    // the three projections of x in one launch (x fetched once per 128-row block)
+    const __nv_bfloat16* Ws[3] = {static_cast<const __nv_bfloat16*>(Wq),
+                                  static_cast<const __nv_bfloat16*>(Wk),
+                                  static_cast<const __nv_bfloat16*>(Wv)};
+    __nv_bfloat16* Cs[3] = {q, k, v};
+    const int Ns[3] = {H * d, H_kv * d, H_kv * d};
+    e = bf16_gemm_grouped_launch(xb, Ws, Cs, Ns, 3, rows, D_model, stream);
+  } else {
+    e = bf16_gemm_launch(xb, static_cast<const __nv_bfloat16*>(Wq), q, rows, H * d, D_model,
                          stream);
-  if (e == cudaSuccess)
-    e = bf16_gemm_launch(xb, static_cast<const __nv_bfloat16*>(Wv), v, rows, H_kv * d, D_model,
-                         stream);
+    if (e == cudaSuccess)
+      e = bf16_gemm_launch(xb, static_cast<const __nv_bfloat16*>(Wk), k, rows, H_kv * d, D_model,
+                           stream);
+    if (e == cudaSuccess)
+      e = bf16_gemm_launch(xb, static_cast<const __nv_bfloat16*>(Wv), v, rows, H_kv * d, D_model,
+                           stream);
+  }
   if (e != cudaSuccess) return INFINI_ERR_CUDA;
   record(opts, 0, stream);
   const int fs = forward_impl(q, k, v, beta, M_in, z_in, a, M_out, z_out, B, H, L, N, d, mode,

@@ -83,6 +83,20 @@ def test_layer_grouped_heads_with_state(ia, mode):
     layer_case(ia, 2, 384, 384, 4, 2, 128, mode, seed=73, state=True)
 
 
+@pytest.mark.parametrize("mode", [LIN, DEL])
+def test_layer_projection_widths_off_the_wide_tile(ia, mode):
+    """3 query heads on 1 key/value head: the projection widths (384, 128) are not
+    multiples of 256, so the three products take three launches of the 128-wide GEMM
+    instead of the one grouped launch."""
+    layer_case(ia, 1, 384, 256, 3, 1, 128, mode, seed=77)
+
+
+def test_layer_grouped_projection_many_row_blocks(ia):
+    """6 query heads on 2 key/value heads over 2 x 1024 rows: the grouped projection
+    launch spans 16 row blocks and 3 + 1 + 1 wide column tiles (more tiles than SMs)."""
+    layer_case(ia, 2, 1024, 512, 6, 2, 512, DEL, seed=79, state=True)
+
+
 def test_layer_workspace_and_events_give_the_same_result(ia):
     """A caller workspace (infini_attn_layer_forward_ex) gives bitwise the same outputs
     as the library's own scratch, and the three stage events are recorded in order."""
