@@ -205,32 +205,96 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
   }
 }
 
-// The same GEMM with 128 x 256 output tiles (N a multiple of 256): each k-step of 64
-// brings A [128 m][64 k] (one 16 KB box, K-major) and B [64 k][256 n] (four 8 KB
-// boxes of 64 columns, MN-major) into a 4-stage ring; four MMAs (N = 256, K = 16)
-// per k-step into one of two 256-column accumulators. Per FLOP it streams a quarter
-// less through L2 than the 128 x 128 tiles.
-constexpr int kWStages = 4;
-constexpr int kWA = 16384, kWB = 32768, kWStage = kWA + kWB;
-constexpr int kGemmWSmem = kWStages * kWStage + 256 + 1024;
+// The same GEMM with 256 x 256 output tiles (N a multiple of 256) on a CTA pair (a
+// cluster of two CTAs, one per SM, driving tcgen05 MMAs with cta_group::2). Each k-step
+// of 64 brings into each CTA its 128 rows of A (one 16 KB box, K-major) and its 128
+// columns of B (two 8 KB boxes of 64 columns, MN-major), into a 6-stage ring; both
+// CTAs' copies complete on the even CTA's barrier, and the even CTA issues four pair
+// MMAs (M = 256, N = 256, K = 16) per k-step into one of two 256-column accumulators,
+// each CTA's tensor memory holding its own 128 rows of the tile. Per FLOP an SM
+// streams two thirds of what a 128 x 256 tile on one SM needs through L2, and the ring
+// covers more of the latency. In both CTAs four epilogue warps drain their own rows of
+// the accumulator 64 columns at a time (tensor memory -> bf16 -> a swizzled staging
+// buffer -> a TMA store of 32 rows x 64 columns, full 128-byte lines), and release the
+// accumulator on the even CTA's barrier once it has been read.
+constexpr int kPStages = 5;
+constexpr int kPA = 16384, kPB = 16384, kPStage = kPA + kPB;
+// epilogue staging: per epilogue warp two 4 KB buffers (32 rows x 64 columns, 128-byte
+// swizzle), written from registers and sent to C by TMA stores
+constexpr int kPOut = 4 * 2 * 4096;
+constexpr int kGemmPSmem = kPStages * kPStage + kPOut + 256 + 1024;
+// FULL (the even CTA's: 1 arrival with the pair's bytes), EMPTY, AFULL (arrivals
+// multicast to both CTAs by the MMA commits), AEMPTY (the even CTA's: 4 warps of each
+// CTA), DRAIN (both CTAs: every MMA issued has completed)
+enum {
+  P_FULL = 0,
+  P_EMPTY = P_FULL + kPStages,
+  P_AFULL = P_EMPTY + kPStages,
+  P_AEMPTY = P_AFULL + 2,
+  P_DRAIN = P_AEMPTY + 2,
+  P_COUNT = P_DRAIN + 1
+};
+static_assert(P_COUNT * 8 + 4 <= 256, "barrier area");
 
 __device__ __forceinline__ int gemm_group(const GemmGroups& gr, int tn) {
   return tn < gr.first[1] ? 0 : (tn < gr.first[2] ? 1 : 2);
 }
 
+// TMA load into this CTA's shared memory whose completion is counted on an mbarrier of
+// either CTA of the pair (cluster-window address).
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* m,
+                                                 uint32_t bar_cluster, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// First row of this CTA's half of row tile tm. A half that lies wholly past the last
+// row (M an odd number of 128-row blocks) loads the last 128 rows instead: its products
+// are never stored, and every copy stays inside the matrix.
+__device__ __forceinline__ int a_row(int tm, uint32_t rank, long long M) {
+  const long long r = 256ll * tm + 128 * (long long)rank;
+  return (int)(r < M ? r : M - 128);
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* smem_src, int c0,
+                                             int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// Until at most one of this thread's bulk store groups is still reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+struct PairOut {
+  CUtensorMap c[3];  // C_g, box 64 columns x 32 rows, 128-byte swizzle
+};
+
 __global__ void __launch_bounds__(kGemmThreads, 1)
-gemm_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
                  const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_b2,
-                 const GemmParams p, const GemmGroups gr) {
+                 const __grid_constant__ PairOut out, const GemmParams p, const GemmGroups gr,
+                 const long long M) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWStages * kWStage);
-  // FULL [0, 4), EMPTY [4, 8), AFULL 8-9, AEMPTY 10-11 (4 warp arrivals), DRAIN 12
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint8_t* stage_out = smem + kPStages * kPStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stage_out + kPOut);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + P_COUNT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool lead = rank == 0;
+  const unsigned pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   if (threadIdx.x == 0) {
-    for (int x = 0; x < 13; ++x) mbar_init(&bars[x], (x == 10 || x == 11) ? 4u : 1u);
+    for (int x = 0; x < P_COUNT; ++x)
+      mbar_init(&bars[x], (x == P_AEMPTY || x == P_AEMPTY + 1) ? 8u : 1u);
     fence_barrier_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b0);
@@ -238,11 +302,11 @@ gemm_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     if (gr.n > 2) tma_prefetch_desc(&tm_b2);
   }
   if (warp == 5) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers initialised in both CTAs before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
@@ -250,106 +314,140 @@ gemm_wide_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
   if (warp == 4) {
     if (lane == 0) {
       int it = 0;
-      int iss[kWStages] = {0, 0, 0, 0};
-      for (unsigned t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
+      int iss[kPStages] = {};
+      for (unsigned t = pair; ok && t < p.tiles; t += npairs) {
         const int tm = (int)(t / (unsigned)p.tiles_n), tn = (int)(t % (unsigned)p.tiles_n);
         const int g = gemm_group(gr, tn), tl = tn - gr.first[g];
         const CUtensorMap* tmb = g == 0 ? &tm_b0 : (g == 1 ? &tm_b1 : &tm_b2);
         for (int ks = 0; ks < p.ksteps; ++ks, ++it) {
-          const int st = it % kWStages, use = it / kWStages;
-          if (use > 0 && !mbar_wait(&bars[4 + st], (uint32_t)((use - 1) & 1))) {
+          const int st = it % kPStages, use = it / kPStages;
+          if (use > 0 && !mbar_wait(&bars[P_EMPTY + st], (uint32_t)((use - 1) & 1))) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + st * kWStage;
-          uint8_t* sb = sa + kWA;
-          mbar_arrive_expect_tx(&bars[st], kWStage);
-          tma_load_2d(sa, &tm_a, &bars[st], 64 * ks, 128 * tm);
+          uint8_t* sa = smem + st * kPStage;
+          uint8_t* sb = sa + kPA;
+          if (lead) mbar_arrive_expect_tx(&bars[P_FULL + st], 2 * kPStage);
+          const uint32_t full = smem_cluster_addr(&bars[P_FULL + st], 0);
+          tma_load_2d_pair(sa, &tm_a, full, 64 * ks, a_row(tm, rank, M));
 #pragma unroll
-          for (int a4 = 0; a4 < 4; ++a4)
-            tma_load_2d(sb + a4 * 8192, tmb, &bars[st], 256 * tl + 64 * a4, 64 * ks);
+          for (int a2 = 0; a2 < 2; ++a2)
+            tma_load_2d_pair(sb + a2 * 8192, tmb, full, 256 * tl + 128 * (int)rank + 64 * a2,
+                             64 * ks);
           ++iss[st];
         }
       }
-      if (!ok)
-        for (int st = 0; st < kWStages; ++st)
-          if (iss[st] > 0) drain_wait_g(&bars[st], (uint32_t)((iss[st] - 1) & 1));
+      // every copy into this CTA's ring has landed (and every arrival on its EMPTY
+      // barriers) once the last use of each stage has been released
+      for (int st = 0; st < kPStages; ++st)
+        if (iss[st] > 0) drain_wait_g(&bars[P_EMPTY + st], (uint32_t)((iss[st] - 1) & 1));
     }
+    __syncwarp();
   } else if (warp == 5) {
-    const uint32_t idesc = idesc_f32acc(1, 0, 1, 128, 256);
-    int it = 0, lt = 0;
-    for (unsigned t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++lt) {
-      const int acc = lt & 1, use = lt >> 1;
-      if (use > 0 && !mbar_wait_warp(&bars[10 + acc], (uint32_t)((use - 1) & 1))) {
-        ok = false;
-        break;
-      }
-      const uint32_t td = tmem + (uint32_t)acc * 256;
-      for (int ks = 0; ks < p.ksteps; ++ks, ++it) {
-        const int st = it % kWStages;
-        if (!mbar_wait_warp(&bars[st], (uint32_t)((it / kWStages) & 1))) {
+    if (lead) {
+      const uint32_t idesc = idesc_f32acc(1, 0, 1, 256, 256);
+      int it = 0, lt = 0;
+      for (unsigned t = pair; ok && t < p.tiles; t += npairs, ++lt) {
+        const int acc = lt & 1, use = lt >> 1;
+        if (use > 0 && !mbar_wait_warp(&bars[P_AEMPTY + acc], (uint32_t)((use - 1) & 1))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (elect_one()) {
-          const uint32_t sa = smem_u32(smem + st * kWStage), sb = sa + kWA;
+        const uint32_t td = tmem + (uint32_t)acc * 256;
+        for (int ks = 0; ks < p.ksteps; ++ks, ++it) {
+          const int st = it % kPStages;
+          if (!mbar_wait_warp(&bars[P_FULL + st], (uint32_t)((it / kPStages) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            const uint32_t sa = smem_u32(smem + st * kPStage), sb = sa + kPA;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(td, sdesc(sa + (uint32_t)kk * 32, 16, 1024),
-                        sdesc(sb + (uint32_t)kk * 2048, 8192, 1024), idesc,
-                        (ks > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&bars[4 + st]);
-          if (ks == p.ksteps - 1) mma_commit(&bars[8 + acc]);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss_pair(td, sdesc(sa + (uint32_t)kk * 32, 16, 1024),
+                               sdesc(sb + (uint32_t)kk * 2048, 8192, 1024), idesc,
+                               (ks > 0 || kk > 0) ? 1u : 0u);
+            mma_commit_pair(&bars[P_EMPTY + st], 3);
+            if (ks == p.ksteps - 1) mma_commit_pair(&bars[P_AFULL + acc], 3);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
+      if (elect_one()) mma_commit_pair(&bars[P_DRAIN], 3);
+      __syncwarp();
+      // both CTAs' epilogues have released every accumulator use (their arrivals on
+      // this CTA's barriers have landed)
+      if (lane == 0)
+        for (int acc = 0; acc < 2; ++acc) {
+          const int uses = (lt + 1 - acc) / 2;
+          if (uses > 0) drain_wait_g(&bars[P_AEMPTY + acc], (uint32_t)((uses - 1) & 1));
+        }
+      __syncwarp();
     }
-    if (elect_one()) mma_commit(&bars[12]);
+    // no MMA into either CTA's tensor memory is in flight past this point
+    if (lane == 0) drain_wait_g(&bars[P_DRAIN], 0);
     __syncwarp();
-    drain_wait_g(&bars[12], 0);
   } else {
-    const int r = warp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    int lt = 0;
-    for (unsigned t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++lt) {
+    uint8_t* sbuf = stage_out + warp * 8192;
+    int lt = 0, chunk = 0;
+    for (unsigned t = pair; ok && t < p.tiles; t += npairs, ++lt) {
       const int acc = lt & 1;
-      if (!mbar_wait_warp(&bars[8 + acc], (uint32_t)((lt >> 1) & 1))) {
+      if (!mbar_wait_warp(&bars[P_AFULL + acc], (uint32_t)((lt >> 1) & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int tm = (int)(t / (unsigned)p.tiles_n), tn = (int)(t % (unsigned)p.tiles_n);
       const int g = gemm_group(gr, tn);
-      __nv_bfloat16* dst = gr.C[g] + (size_t)(128 * tm + r) * gr.ldc[g] + 256 * (tn - gr.first[g]);
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t v[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tmem_ld32(tmem + (uint32_t)acc * 256 + lane_off + 128 * hf + 32 * c,
-                    *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
+      const long long row0 = 256ll * tm + 128 * (int)rank + 32 * warp;  // this warp's rows
+      const int col0 = 256 * (tn - gr.first[g]);
+#pragma unroll 1
+      for (int c4 = 0; c4 < 4; ++c4, ++chunk) {
+        uint8_t* buf = sbuf + (chunk & 1) * 4096;
+        uint32_t v[64];
+        tmem_ld32(tmem + (uint32_t)acc * 256 + lane_off + 64 * c4,
+                  *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld32(tmem + (uint32_t)acc * 256 + lane_off + 64 * c4 + 32,
+                  *reinterpret_cast<uint32_t(*)[32]>(v + 32));
         tmem_wait_ld();
-        if (hf == 1) {
+        if (c4 == 3) {
           tc_fence_before();
-          mbar_arrive_warp(&bars[10 + acc]);  // the accumulator may take the next tile
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(smem_cluster_addr(&bars[P_AEMPTY + acc], 0));
         }
+        // the store that last read this buffer (two chunks back) has finished reading
+        if (lane == 0 && chunk >= 2) bulk_wait_group_read1();
+        __syncwarp();
+        const uint32_t rowb = smem_u32(buf) + (uint32_t)lane * 128;
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          *reinterpret_cast<uint4*>(dst + 128 * hf + 8 * u) = make_uint4(
-              pack_bf16x2(__uint_as_float(v[8 * u]), __uint_as_float(v[8 * u + 1])),
-              pack_bf16x2(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
-              pack_bf16x2(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
-              pack_bf16x2(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7])));
+        for (int u = 0; u < 8; ++u)
+          st_shared_v4(rowb + (uint32_t)((u ^ (lane & 7)) * 16),
+                        pack_bf16x2(__uint_as_float(v[8 * u]), __uint_as_float(v[8 * u + 1])),
+                        pack_bf16x2(__uint_as_float(v[8 * u + 2]), __uint_as_float(v[8 * u + 3])),
+                        pack_bf16x2(__uint_as_float(v[8 * u + 4]), __uint_as_float(v[8 * u + 5])),
+                        pack_bf16x2(__uint_as_float(v[8 * u + 6]), __uint_as_float(v[8 * u + 7])));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          // rows past the end of C are clipped by the store; a block wholly past it is
+          // not sent
+          if (row0 < M) tma_store_2d(&out.c[g], buf, col0 + 64 * c4, (int)row0);
+          tma_store_commit();
+        }
       }
     }
+    if (lane == 0) tma_store_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // both CTAs done with tensor memory and with each other's barriers
   if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -374,19 +472,52 @@ cudaError_t bf16_gemm_set_attributes() {
   const cudaError_t e =
       cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(gemm_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              kGemmWSmem);
+  return cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kGemmPSmem);
 }
+
+namespace {
+// CTAs of the pair kernel that can be resident at once (two per co-resident cluster),
+// looked up once per device.
+int pair_kernel_ctas() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cached[dev] > 0) return cached[dev];
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(sms & ~1));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kGemmPSmem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel, &cfg) != cudaSuccess ||
+      clusters < 1) {
+    cudaGetLastError();
+    return 0;
+  }
+  cached[dev] = 2 * clusters;
+  return cached[dev];
+}
+}  // namespace
 
 cudaError_t bf16_gemm_grouped_launch(const __nv_bfloat16* A, const __nv_bfloat16* const* B,
                                      __nv_bfloat16* const* C, const int* N, int ngroups,
                                      long long M, int K, cudaStream_t stream) {
-  if (ngroups < 1 || ngroups > 3 || M <= 0 || K <= 0 || M % 128 || K % 128)
+  if (ngroups < 1 || ngroups > 3 || M <= 0 || K <= 0 || M % 128 || K % 128 || M >= (1ll << 31))
     return cudaErrorInvalidValue;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int ctas = pair_kernel_ctas();
+  if (ctas < 2) return cudaErrorLaunchOutOfResources;
   CUtensorMap ma, mb[3];
+  PairOut out;
   if (!make_bf16_map2(&ma, A, (uint64_t)M, (uint64_t)K, 128)) return cudaErrorInvalidValue;
   GemmGroups gr;
   memset(&gr, 0, sizeof(gr));
@@ -394,12 +525,15 @@ cudaError_t bf16_gemm_grouped_launch(const __nv_bfloat16* A, const __nv_bfloat16
   for (int g = 0; g < ngroups; ++g) {
     if (N[g] <= 0 || N[g] % 256 != 0) return cudaErrorInvalidValue;
     if (!make_bf16_map2(&mb[g], B[g], (uint64_t)K, (uint64_t)N[g], 64)) return cudaErrorInvalidValue;
+    if (!make_bf16_map2(&out.c[g], C[g], (uint64_t)M, (uint64_t)N[g], 32))
+      return cudaErrorInvalidValue;
     gr.C[g] = C[g];
     gr.ldc[g] = N[g];
     gr.first[g + 1] = gr.first[g] + N[g] / 256;
   }
   for (int g = ngroups; g < 3; ++g) {
     mb[g] = mb[0];
+    out.c[g] = out.c[0];
     gr.first[g + 1] = gr.first[g];
     gr.C[g] = C[0];
     gr.ldc[g] = 0;
@@ -407,13 +541,26 @@ cudaError_t bf16_gemm_grouped_launch(const __nv_bfloat16* A, const __nv_bfloat16
   GemmParams p;
   p.tiles_n = gr.first[ngroups];
   p.ksteps = K / 64;
-  const long long tiles = (M / 128) * (long long)p.tiles_n;
+  const long long tiles = ((M + 255) / 256) * (long long)p.tiles_n;
   if (tiles >= (1ll << 31)) return cudaErrorInvalidValue;
   p.tiles = (unsigned)tiles;
   p.ldc = 0;
-  const unsigned grid = p.tiles < (unsigned)sms ? p.tiles : (unsigned)sms;
-  gemm_wide_kernel<<<grid, kGemmThreads, kGemmWSmem, stream>>>(ma, mb[0], mb[1], mb[2], p, gr);
-  return cudaGetLastError();
+  const unsigned pairs = p.tiles < (unsigned)(ctas / 2) ? p.tiles : (unsigned)(ctas / 2);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kGemmPSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ma, mb[0], mb[1], mb[2], out, p, gr, M);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t bf16_gemm_launch(const __nv_bfloat16* A, const __nv_bfloat16* B, __nv_bfloat16* C,

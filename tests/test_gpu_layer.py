@@ -35,10 +35,14 @@ def sync_ok(ia):
     assert ia.device_status() == 0, "a bounded device wait ran out"
 
 
-@pytest.mark.parametrize("M,N,K", [(256, 384, 640), (128, 128, 128), (2048, 1024, 1024)])
+@pytest.mark.parametrize("M,N,K", [(256, 384, 640), (128, 128, 128), (2048, 1024, 1024),
+                                   (640, 512, 256), (8320, 1024, 256), (4224, 768, 1152)])
 def test_gemm_matches_fp64(ia, M, N, K):
     """Several tiles in each direction, several k-steps, more tiles than SMs in the
-    largest case (each CTA takes several tiles and reuses its two accumulators)."""
+    largest cases (each CTA takes several tiles and reuses its two accumulators). N a
+    multiple of 256 takes the CTA-pair kernel (256 x 256 tiles); an odd number of
+    128-row blocks (640, 8320, 4224 rows) leaves the last tile's second half past the
+    end, and K = 256 gives fewer k-steps than ring stages."""
     A = normal((M, K), torch.bfloat16, 61, 0).cuda()
     B = (normal((K, N), torch.float32, 61, 1) / np.sqrt(K)).to(torch.bfloat16).cuda()
     C = ia.infini_attn_gemm_bf16(A, B)
