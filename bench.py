@@ -705,14 +705,29 @@ def run_extra(args, device):
                           device=device)
         res = {}
         for mode, name in ((ia.LINEAR, "linear"), (ia.DELTA, "delta")):
-            def f():
+            def f(evs=None):
                 ia.infini_attn_layer_forward(x, Ws[0], Ws[1], Ws[2], Ws[3], beta, Nc, mode, Hc,
-                                             out=y, state_out=False, workspace=lws)
+                                             out=y, state_out=False, workspace=lws,
+                                             stage_events=evs)
             for _ in range(2):
                 f()
             torch.cuda.synchronize()
             ms = _timed(f, 5, stream)
             res[name] = {"ms_per_call": ms, "tokens_per_s": Bc * Lc / (ms / 1e3)}
+            # the three stages of one call, from the events the layer records after the
+            # grouped Q/K/V projection, after the forward and after W_O (mean of 5 calls)
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            for e in evs:
+                e.record(stream)
+            parts = [0.0, 0.0, 0.0]
+            for _ in range(5):
+                evs[0].record(stream)
+                f(evs[1:])
+                torch.cuda.synchronize()
+                for i in range(3):
+                    parts[i] += evs[i].elapsed_time(evs[i + 1]) / 5
+            res[name]["stages_ms"] = {"qkv_projection": parts[0], "forward": parts[1],
+                                      "output_projection": parts[2]}
         A2 = x.view(Bc * Lc, Dm)
         C2 = torch.empty((Bc * Lc, Dm), device=device, dtype=torch.bfloat16)
         g = lambda: ia.infini_attn_gemm_bf16(A2, Ws[0], out=C2)
@@ -722,23 +737,11 @@ def run_extra(args, device):
         gms = _timed(g, 20, stream)
         gflop = 2.0 * Bc * Lc * Dm * Dm
         gtf = gflop / (gms / 1e3) / 1e12
-        # the forward inside the layer alone: the projections' outputs read in place as
-        # [B, L, H, d]
-        qkv = [ia.infini_attn_gemm_bf16(A2, Ws[i]).view(Bc, Lc, Hc, D) for i in range(3)]
-        o4 = torch.empty_like(qkv[0])
-        for mode, name in ((ia.LINEAR, "linear"), (ia.DELTA, "delta")):
-            def fw():
-                ia.infini_attn_forward_gqa(qkv[0], qkv[1], qkv[2], beta, Nc, mode,
-                                           ia.LAYOUT_BLHD, out=o4, state_out=False)
-            for _ in range(2):
-                fw()
-            torch.cuda.synchronize()
-            res[name]["forward_part_ms"] = _timed(fw, 5, stream)
-            res[name]["projections_part_ms"] = 4 * gms
         assert ia.device_status() == 0
-        del x, Ws, y, A2, C2, qkv, o4, lws
+        del x, Ws, y, A2, C2, lws
         lines.append({"config": "layer: B=4, L=32768, D_model=1024, H=H_kv=8, d=128, N=2048, "
-                                "bf16, infini_attn_layer_forward (4 projections + forward)",
+                                "bf16, infini_attn_layer_forward (Q/K/V projections in one "
+                                "grouped GEMM launch, forward, W_O)",
                       **res,
                       "projection_gemm": {"shape": "[131072 x 1024] @ [1024 x 1024]",
                                           "ms": gms, "tflops": gtf,
