@@ -1,6 +1,7 @@
 """Randomized model checks of the mbarrier protocols of the pipelined kernels (the
 forward's fused attention kernel, its state kernel and state chain, the backward's
-dq and dk/dv kernels and reverse chain, the projection GEMM): every role of a CTA is
+dq and dk/dv kernels and reverse chain, the projection GEMMs on one CTA and on a CTA
+pair): every role of a CTA is
 written as a step function that waits on barriers by completion index, TMA copies
 and tensor-core commits complete at random later times (commits in issue order,
 each after every product issued before it), and a random scheduler interleaves
@@ -17,7 +18,11 @@ class Bar:
     def __init__(self, name, count):
         self.name, self.count, self.pending, self.done = name, count, count, 0
 
-    def arrive(self, n=1):
+    def arrive(self, n=1, tag=None):
+        # a tagged arrival belongs to phase `tag` (counted from 0): it must not land
+        # while the barrier is still in an earlier phase or already in a later one
+        assert tag is None or tag == self.done, \
+            f"{self.name}: arrival for phase {tag} while in phase {self.done}"
         self.pending -= n
         assert self.pending >= 0, f"{self.name}: more arrivals than the count"
         if self.pending == 0:
@@ -27,9 +32,11 @@ class Bar:
 
 class Sim:
     """Roles are generators yielding ('wait', bar, k) (wait for completion k, counted
-    from 0), ('arrive', bar, n), ('tma', bar) (a copy that completes bar later),
-    ('mma',) (a product), ('commit', bar) (arrives on bar once every earlier product of
-    the CTA is done) or ('named', id, members) (a CTA-level named barrier)."""
+    from 0), ('arrive', bar, n[, tag]), ('tma', bar[, tag]) (a copy that completes bar
+    later), ('mma',) (a product), ('commit', bar or [bars]) (arrives on the bar, or on
+    each bar of a multicast list, once every earlier product is done) or ('named', id,
+    members) (a named barrier of the CTA, or of a cluster). An optional tag names the
+    phase an arrival belongs to (checked by Bar.arrive)."""
 
     def __init__(self, seed):
         self.rng = random.Random(seed)
@@ -83,19 +90,19 @@ class Sim:
                     f"#{req[2] if len(req) > 2 else ''}" for r, req in state.items()))
             choice = self.rng.choice(ready + events)
             if choice == '<copy done>':
-                b = self.tma.pop(self.rng.randrange(len(self.tma)))
-                b.arrive()
+                b, tag = self.tma.pop(self.rng.randrange(len(self.tma)))
+                b.arrive(1, tag)
             elif choice == '<product done>':
                 item = self.mma_queue.pop(0)   # in issue order
-                if item is not None:
-                    item.arrive()
+                for b in (item if isinstance(item, list) else [item] if item else []):
+                    b.arrive()
             else:
                 req = state[choice]
                 kind = req[0]
                 if kind == 'arrive':
-                    req[1].arrive(req[2])
+                    req[1].arrive(req[2], req[3] if len(req) > 3 else None)
                 elif kind == 'tma':
-                    self.tma.append(req[1])
+                    self.tma.append((req[1], req[2] if len(req) > 2 else None))
                 elif kind == 'mma':
                     self.mma_queue.append(None)
                 elif kind == 'commit':
@@ -302,6 +309,101 @@ def gemm_roles(sim, tiles, ksteps, stages):
             yield ('arrive', AEMPTY[lt & 1], 4)
 
     return {"producer": producer(), "mma": mma(), "epilogue": epilogue()}
+
+
+# ------------------------------------------------------------------------------
+# projection GEMM on a CTA pair (cluster of two, cta_group::2 MMAs from the even CTA):
+# each CTA's copies complete on the even CTA's FULL barrier, whose producer expects the
+# pair's bytes (count: its arrival + one completion per CTA's copies); the MMA commits
+# are multicast to both CTAs' EMPTY / AFULL / DRAIN barriers; both CTAs' epilogues
+# release an accumulator on the even CTA's AEMPTY (4 warps each); before the cluster
+# barrier every producer waits for its stages' last release and the even CTA's MMA
+# warp for the last accumulator releases.
+# ------------------------------------------------------------------------------
+def pair_gemm_roles(sim, tiles, ksteps, stages, full_count=3, empty_mask=(0, 1)):
+    FULL = [sim.bar(f"full{i}", full_count) for i in range(stages)]        # CTA 0's
+    EMPTY = [[sim.bar(f"empty{c}.{i}") for i in range(stages)] for c in range(2)]
+    AFULL = [[sim.bar(f"afull{c}.{i}") for i in range(2)] for c in range(2)]
+    AEMPTY = [sim.bar(f"aempty{i}", 8) for i in range(2)]                  # CTA 0's
+    DRAIN = [sim.bar(f"drain{c}") for c in range(2)]
+    members = [f"{r}{c}" for c in range(2) for r in ("producer", "mma", "epilogue")]
+
+    def producer(c):
+        it, last = 0, {}
+        for _ in range(tiles):
+            for _ in range(ksteps):
+                st, use = it % stages, it // stages
+                if use > 0:
+                    yield ('wait', EMPTY[c][st], use - 1)
+                if c == 0:
+                    yield ('arrive', FULL[st], 1, use)   # arrive.expect_tx (the pair's bytes)
+                yield ('tma', FULL[st], use)            # this CTA's A half and B half
+                last[st] = use
+                it += 1
+        for st, use in last.items():                     # tail: no copy still landing
+            yield ('wait', EMPTY[c][st], use)
+        yield ('named', 'cluster', members)
+
+    def mma(c):
+        if c == 0:
+            it = 0
+            for lt in range(tiles):
+                acc, use = lt & 1, lt >> 1
+                if use > 0:
+                    yield ('wait', AEMPTY[acc], use - 1)
+                for ks in range(ksteps):
+                    st = it % stages
+                    yield ('wait', FULL[st], it // stages)
+                    yield ('mma',)
+                    yield ('commit', [EMPTY[x][st] for x in empty_mask])
+                    if ks == ksteps - 1:
+                        yield ('commit', [AFULL[0][acc], AFULL[1][acc]])
+                    it += 1
+            yield ('commit', [DRAIN[0], DRAIN[1]])
+            for acc in range(2):                          # tail: the last releases landed
+                uses = (tiles + 1 - acc) // 2
+                if uses > 0:
+                    yield ('wait', AEMPTY[acc], uses - 1)
+        yield ('wait', DRAIN[c], 0)
+        yield ('named', 'cluster', members)
+
+    def epilogue(c):
+        for lt in range(tiles):
+            yield ('wait', AFULL[c][lt & 1], lt >> 1)
+            yield ('arrive', AEMPTY[lt & 1], 4)
+        yield ('named', 'cluster', members)
+
+    roles = {}
+    for c in range(2):
+        roles[f"producer{c}"] = producer(c)
+        roles[f"mma{c}"] = mma(c)
+        roles[f"epilogue{c}"] = epilogue(c)
+    return roles
+
+
+@pytest.mark.parametrize("tiles,ksteps,stages", [(1, 1, 5), (3, 16, 5), (4, 4, 5), (7, 2, 5),
+                                                 (2, 9, 3), (5, 16, 6)])
+def test_pair_gemm_pipeline_protocol(tiles, ksteps, stages):
+    for seed in range(40):
+        sim = Sim(seed * 1000 + tiles * 10 + ksteps + stages)
+        sim.run(pair_gemm_roles(sim, tiles, ksteps, stages))
+
+
+def test_pair_gemm_model_detects_a_barrier_expecting_one_cta():
+    """A FULL barrier that counts only the even CTA's copies completes early, and the
+    odd CTA's copy then lands in the next phase."""
+    with pytest.raises(AssertionError, match="arrival for phase|phase skipped|stale"):
+        for seed in range(40):
+            sim = Sim(seed)
+            sim.run(pair_gemm_roles(sim, 4, 8, 5, full_count=2))
+
+
+def test_pair_gemm_model_detects_a_commit_to_one_cta():
+    """Ring stages released only in the even CTA: the odd CTA's producer never sees
+    its stages free."""
+    with pytest.raises(AssertionError, match="deadlock"):
+        sim = Sim(1)
+        sim.run(pair_gemm_roles(sim, 3, 8, 5, empty_mask=(0,)))
 
 
 @pytest.mark.parametrize("nk", [1, 2, 3, 4, 7, 16])
@@ -823,3 +925,102 @@ def test_chain_protocol(S, CH):
     for seed in range(20):
         sim = Sim(seed * 100 + S * 10 + CH)
         sim.run(chain_roles(sim, S, CH))
+
+
+# ------------------------------------------------------------------------------
+# one-segment update (step_state_kernel): slabs n through two stages; converter group
+# g (eight warps, one arrival each) takes the slabs of stage g; Linear+Delta issues
+# R of slab n, then the update product of slab n - 1
+# ------------------------------------------------------------------------------
+def step_state_roles(sim, nslab, delta):
+    FULL = [sim.bar(f"full{i}", 2) for i in range(2)]     # expect_tx arrival + the copies
+    CONV1 = [sim.bar(f"conv1_{i}", 8) for i in range(2)]
+    RDONE = [sim.bar(f"rdone{i}") for i in range(2)]
+    CONV2 = [sim.bar(f"conv2_{i}", 8) for i in range(2)]
+    FREE = [sim.bar(f"free{i}") for i in range(2)]
+    MFULL = sim.bar("mfull", 2)
+    DONE = sim.bar("done")
+
+    def producer():
+        if delta:
+            yield ('arrive', MFULL, 1, 0)
+            yield ('tma', MFULL, 0)
+        for n in range(nslab):
+            st = n & 1
+            if n >= 2:
+                yield ('wait', FREE[st], (n >> 1) - 1)
+            yield ('arrive', FULL[st], 1, n >> 1)
+            yield ('tma', FULL[st], n >> 1)
+
+    def mma():
+        if delta and nslab > 0:
+            yield ('wait', MFULL, 0)
+        for n in range(nslab):
+            st = n & 1
+            yield ('wait', CONV1[st], n >> 1)
+            if not delta:
+                yield ('mma',)
+                yield ('commit', FREE[st])
+                continue
+            yield ('mma',)                      # R of slab n
+            yield ('commit', RDONE[st])
+            if n > 0:
+                yield ('wait', CONV2[(n - 1) & 1], (n - 1) >> 1)
+                yield ('mma',)                  # update of slab n - 1
+                yield ('commit', FREE[(n - 1) & 1])
+        if delta and nslab > 0:
+            yield ('wait', CONV2[(nslab - 1) & 1], (nslab - 1) >> 1)
+            yield ('mma',)
+            yield ('commit', FREE[(nslab - 1) & 1])
+        yield ('commit', DONE)
+
+    def converters(g):
+        for n in range(g, nslab, 2):
+            st = n & 1
+            yield ('wait', FULL[st], n >> 1)
+            yield ('arrive', CONV1[st], 8)      # sigma(K) hi/lo and 1/den written
+            if not delta:
+                continue
+            yield ('wait', CONV1[st], n >> 1)   # every warp's 1/den of the slab
+            yield ('wait', RDONE[st], n >> 1)
+            yield ('arrive', CONV2[st], 8)      # U = V - R / den written
+        yield ('wait', DONE, 0)
+
+    return {"producer": producer(), "mma": mma(), "conv0": converters(0), "conv1": converters(1)}
+
+
+@pytest.mark.parametrize("delta", [False, True])
+@pytest.mark.parametrize("nslab", [0, 1, 2, 3, 4, 7, 16])
+def test_step_state_kernel_protocol(nslab, delta):
+    for seed in range(40):
+        sim = Sim(seed * 1000 + nslab + 100 * delta)
+        sim.run(step_state_roles(sim, nslab, delta))
+
+
+def test_step_state_model_detects_a_wait_for_the_wrong_slab():
+    """The update of slab n - 1 waiting for the U of slab n's completion index: the U
+    it waits for needs an R that is issued only after that update."""
+    def broken(sim, nslab):
+        roles = step_state_roles(sim, nslab, True)
+        CONV1 = [sim.bars["conv1_0"], sim.bars["conv1_1"]]
+        CONV2 = [sim.bars["conv2_0"], sim.bars["conv2_1"]]
+        RDONE = [sim.bars["rdone0"], sim.bars["rdone1"]]
+        FREE = [sim.bars["free0"], sim.bars["free1"]]
+
+        def mma():
+            yield ('wait', sim.bars["mfull"], 0)
+            for n in range(nslab):
+                st = n & 1
+                yield ('wait', CONV1[st], n >> 1)
+                yield ('mma',)
+                yield ('commit', RDONE[st])
+                if n > 0:
+                    yield ('wait', CONV2[(n - 1) & 1], n >> 1)   # should be (n - 1) >> 1
+                    yield ('mma',)
+                    yield ('commit', FREE[(n - 1) & 1])
+            yield ('commit', sim.bars["done"])
+        roles["mma"] = mma()
+        return roles
+    with pytest.raises(AssertionError, match="deadlock|phase"):
+        sim = Sim(3)
+        sim.run(broken(sim, 8))
