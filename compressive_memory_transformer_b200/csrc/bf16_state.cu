@@ -105,19 +105,45 @@ __global__ void __launch_bounds__(256) zpart_kernel(const __nv_bfloat16* __restr
 // ---------------------------------------------------------------------------
 // zscan: grid = BH, block 128. zprev[bh][s] = z_in + sum_{r<s} dz_r; z_out = final.
 // The thread that reads z_in[k] is the one that writes z_out[k] (in-place safe).
+// In Linear mode the chain kernel runs the same scan in its otherwise idle warp.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void zscan_feature(const float* __restrict__ zpart, const float* z_in,
+                                              float* z_out, float* __restrict__ zprev, int S,
+                                              int CH, int first, int bh, int kf) {
+  float z = z_in ? z_in[(size_t)bh * D + kf] : 0.f;
+  const float* zp = zpart + (size_t)bh * S * CH * D + kf;
+  if (CH == 1) {
+    // four segments' sums loaded together (their loads do not wait on z); still added
+    // in segment order
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {
+      float t[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) t[e] = __ldcg(zp + (size_t)(s + e) * D);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (s + e >= first) zprev[((size_t)bh * S + s + e) * D + kf] = z;
+        z += t[e];
+      }
+    }
+    for (; s < S; ++s) {
+      if (s >= first) zprev[((size_t)bh * S + s) * D + kf] = z;
+      z += __ldcg(zp + (size_t)s * D);
+    }
+  } else {
+    for (int s = 0; s < S; ++s) {
+      if (s >= first) zprev[((size_t)bh * S + s) * D + kf] = z;
+      for (int c = 0; c < CH; ++c) z += __ldcg(zp + ((size_t)s * CH + c) * D);
+    }
+  }
+  if (z_out) z_out[(size_t)bh * D + kf] = z;
+}
+
 __global__ void __launch_bounds__(D) zscan_kernel(const float* __restrict__ zpart,
                                                   const float* z_in, float* z_out,
                                                   float* __restrict__ zprev, int S, int CH,
                                                   int first) {
-  const int bh = blockIdx.x, kf = threadIdx.x;
-  float z = z_in ? z_in[(size_t)bh * D + kf] : 0.f;
-  for (int s = 0; s < S; ++s) {
-    if (s >= first) zprev[((size_t)bh * S + s) * D + kf] = z;
-    const float* zp = zpart + ((size_t)bh * S + s) * CH * D + kf;
-    for (int c = 0; c < CH; ++c) z += zp[(size_t)c * D];
-  }
-  if (z_out) z_out[(size_t)bh * D + kf] = z;
+  zscan_feature(zpart, z_in, z_out, zprev, S, CH, first, blockIdx.x, threadIdx.x);
 }
 
 // ---------------------------------------------------------------------------
@@ -409,7 +435,8 @@ constexpr int kChainSmem = 2 * kGBytes + kMtBytes + 1024 + 256;
 __global__ void __launch_bounds__(kChainThreads, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__ dpart,
              const float* M_in, float* M_out, __nv_bfloat16* __restrict__ Mhl, int S, int CH,
-             int mode, int first) {
+             int mode, int first, const float* __restrict__ zpart, const float* z_in,
+             float* z_out, float* __restrict__ zprev) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -444,6 +471,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
   bool ok = true;
 
   if (warp == 4) {
+    // Linear (zpart given): this warp scans z for features [32 cb, 32 cb + 32) of the
+    // head, beside the rows' M chain (the two do not depend on each other).
+    if (!delta && zpart)
+      zscan_feature(zpart, z_in, z_out, zprev, S, CH, first, bh, c0 + (tid & 31));
     // The whole warp runs the loop and waits; one elected lane (always lane 0)
     // issues the copies, MMAs and commits.
     if (delta) {
@@ -514,54 +545,74 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
 #pragma unroll
       for (int e = 0; e < 32; ++e) m[e] = 0.f;
     }
-    // dM of the next segment, prefetched into registers. Chunk 0 is loaded by plain
-    // assignment so that nothing waits on the loads until the next segment uses
-    // them; further chunks (only when a segment is split, e.g. one-segment steps)
-    // are added at once.
-    float nx[32];
-    auto load_dm = [&](int s) {
+    // dM of a later segment, prefetched into registers. Chunk 0 is loaded by plain
+    // assignment so that nothing waits on the loads until the segment uses them;
+    // further chunks (only when a segment is split, e.g. one-segment steps) are added
+    // at once.
+    auto load_dm = [&](float (&dst)[32], int s) {
       const float* src = dpart + ((size_t)((bh * S + s) * CH) * 2) * D * D + (size_t)r * D + c0;
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
         const float4 t = __ldg(reinterpret_cast<const float4*>(src + e));
-        nx[e] = t.x; nx[e + 1] = t.y; nx[e + 2] = t.z; nx[e + 3] = t.w;
+        dst[e] = t.x; dst[e + 1] = t.y; dst[e + 2] = t.z; dst[e + 3] = t.w;
       }
       for (int c = 1; c < CH; ++c) {
         const float* sc = src + (size_t)c * 2 * D * D;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float4 t = __ldg(reinterpret_cast<const float4*>(sc + e));
-          nx[e] += t.x; nx[e + 1] += t.y; nx[e + 2] += t.z; nx[e + 3] += t.w;
+          dst[e] += t.x; dst[e + 1] += t.y; dst[e + 2] += t.z; dst[e + 3] += t.w;
         }
       }
     };
-    if (S > 0) load_dm(0);
-    for (int s = 0; s < S; ++s) {
-      // M_{s-1} -> hi / lo bf16 (segments below `first` were written by prep_first_kernel)
-      if (s >= first) {
-        __nv_bfloat16* hi = Mhl + ((size_t)bh * S + s) * 2 * D * D + (size_t)r * D + c0;
-        __nv_bfloat16* lo = hi + D * D;
+    // M_{s-1} -> hi / lo bf16 (segments below `first` were written by prep_first_kernel)
+    auto emit = [&](int s) {
+      if (s < first) return;
+      __nv_bfloat16* hi = Mhl + ((size_t)bh * S + s) * 2 * D * D + (size_t)r * D + c0;
+      __nv_bfloat16* lo = hi + D * D;
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint32_t h4[4], l4[4];
+      for (int e = 0; e < 32; e += 8) {
+        uint32_t h4[4], l4[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(m[e + 2 * q], m[e + 2 * q + 1]);
-            const float2 hf = __bfloat1622float2(h);
-            const __nv_bfloat162 l =
-                __floats2bfloat162_rn(m[e + 2 * q] - hf.x, m[e + 2 * q + 1] - hf.y);
-            h4[q] = *reinterpret_cast<const uint32_t*>(&h);
-            l4[q] = *reinterpret_cast<const uint32_t*>(&l);
-          }
-          *reinterpret_cast<uint4*>(hi + e) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-          *reinterpret_cast<uint4*>(lo + e) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+        for (int q = 0; q < 4; ++q) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(m[e + 2 * q], m[e + 2 * q + 1]);
+          const float2 hf = __bfloat1622float2(h);
+          const __nv_bfloat162 l =
+              __floats2bfloat162_rn(m[e + 2 * q] - hf.x, m[e + 2 * q + 1] - hf.y);
+          h4[q] = *reinterpret_cast<const uint32_t*>(&h);
+          l4[q] = *reinterpret_cast<const uint32_t*>(&l);
+        }
+        *reinterpret_cast<uint4*>(hi + e) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+        *reinterpret_cast<uint4*>(lo + e) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+      }
+    };
+    if (!delta) {
+      // Linear: M_s = M_{s-1} + dM_s, with two segments' dM in flight (a and b hold
+      // the even and odd segments)
+      float a[32], b[32];
+      if (S > 0) load_dm(a, 0);
+      if (S > 1) load_dm(b, 1);
+      for (int s = 0; s < S; s += 2) {
+        emit(s);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) m[e] += a[e];
+        if (s + 2 < S) load_dm(a, s + 2);
+        if (s + 1 < S) {
+          emit(s + 1);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) m[e] += b[e];
+          if (s + 3 < S) load_dm(b, s + 3);
         }
       }
-      float dm[32];
+    } else {
+      float nx[32];
+      if (S > 0) load_dm(nx, 0);
+      for (int s = 0; s < S; ++s) {
+        emit(s);
+        float dm[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) dm[e] = nx[e];
-      if (s + 1 < S) load_dm(s + 1);
-      if (delta) {
+        for (int e = 0; e < 32; ++e) dm[e] = nx[e];
+        if (s + 1 < S) load_dm(nx, s + 1);
         // M^T block (tf32) -> shared memory: row c, K-major, 4 boxes of 32 k
         const uint32_t kb = (uint32_t)(r >> 5), kin = (uint32_t)(r & 31);
 #pragma unroll
@@ -582,9 +633,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_g, const float* __restrict__
         tc_fence_before();
 #pragma unroll
         for (int e = 0; e < 32; ++e) m[e] += dm[e] - __uint_as_float(gm[e]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) m[e] += dm[e];
       }
     }
     if (M_out && ok) {
@@ -718,10 +766,12 @@ cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, co
         mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 0, Hkv);
   } else {
     // The state GEMM also produces the sums of sigma(K): always in Linear mode, and
-    // in Linear+Delta mode for a lone segment whose z_{-1} is already in place
+    // in Linear+Delta mode for a lone segment whose z_{-1} is already in place. In
+    // Linear mode the chain kernel scans z itself.
     state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(
         mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 1, Hkv);
-    zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH, first);
+    if (mode == 1)
+      zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH, first);
   }
   CUtensorMap mg;
   if (mode == 1) {
@@ -739,8 +789,10 @@ cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, co
   } else {
     memset(&mg, 0, sizeof(mg));
   }
-  chain_kernel<<<dim3(BH, 4), kChainThreads, kChainSmem, stream>>>(mg, ws.dpart, M_in, M_out,
-                                                                    ws.Mhl, S, CH, mode, first);
+  const bool fused_z = mode == 0;
+  chain_kernel<<<dim3(BH, 4), kChainThreads, kChainSmem, stream>>>(
+      mg, ws.dpart, M_in, M_out, ws.Mhl, S, CH, mode, first, fused_z ? ws.zpart : nullptr,
+      z_in, z_out, ws.zprev);
   return cudaGetLastError();
 }
 
