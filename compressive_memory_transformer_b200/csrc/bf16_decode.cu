@@ -24,11 +24,11 @@
 //                          Four more CTAs per (head, group) compute the retrieval
 //                          sigma(q) M_{s-1} (32 columns each, M read row-coalesced)
 //                          and sigma(q) z_{s-1}, beside the cache reads.
-//   decode_combine_kernel  grid (BH, query groups). Merges the splits' partials,
-//                          divides the retrieval by its denominator, applies the
-//                          gate and writes out in bf16.
-// Both kernels are compiled for query-group widths 1, 2, 4, 8 and 16, so a single
-// token carries no idle accumulators.
+//   decode_combine_kernel  grid (BH, queries). Merges the splits' partials of one
+//                          query, divides the retrieval by its denominator, applies
+//                          the gate and writes out in bf16.
+// The partial kernel is compiled for query-group widths 1, 2, 4, 8 and 16, so a
+// single token carries no idle accumulators.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -262,41 +262,59 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
   }
 }
 
-template <int NQ>
+// One CTA per query. Thread t merges feature t of the splits' partials; every thread
+// loads the splits' (max, sum) pairs too (the same addresses across the CTA, one
+// transaction per warp), so that a batch of up to 32 splits is one round of
+// independent loads and the merge needs no barrier. Batches are merged in split
+// order, each rescaled to the running maximum.
 __global__ void __launch_bounds__(kThreads)
 decode_combine_kernel(const float* __restrict__ part, const float* __restrict__ ret,
                       const float* __restrict__ beta, __nv_bfloat16* __restrict__ out,
                       const DecodeParams p) {
-  __shared__ float sml[kMaxSplits][2];  // splits' (max, sum)
-  const int bh = blockIdx.x, grp = blockIdx.y, t = threadIdx.x;
-  const int q0 = grp * kGroup;
-  const int nq = min(NQ, p.n - q0);
+  const int bh = blockIdx.x, t = threadIdx.x;
   const float bt = beta[bh % p.H];
   const float g = 1.f / (1.f + expf(-bt));
-  const float* pb = part + ((size_t)bh * p.groups + grp) * p.splits * kGroup * kPart;
-  const float* rec = ret + ((size_t)bh * p.groups + grp) * kGroup * kRet;
-  for (int i = 0; i < nq; ++i) {
-    // every split's (max, sum) in parallel, then the weights
-    for (int s = t; s < p.splits; s += kThreads) {
-      sml[s][0] = pb[(s * kGroup + i) * kPart];
-      sml[s][1] = pb[(s * kGroup + i) * kPart + 1];
-    }
-    __syncthreads();
-    float m = -INFINITY;
-    for (int s = 0; s < p.splits; ++s) m = fmaxf(m, sml[s][0]);
-    float l = 0.f, a = 0.f;
-#pragma unroll 4
-    for (int s = 0; s < p.splits; ++s) {
+  const size_t sstride = (size_t)kGroup * kPart;
+  for (int qi = blockIdx.y; qi < p.n; qi += gridDim.y) {
+    const int grp = qi / kGroup, i = qi % kGroup;
+    const float* pb = part + ((size_t)bh * p.groups + grp) * p.splits * kGroup * kPart + i * kPart;
+    const float* rec = ret + ((size_t)bh * p.groups + grp) * kGroup * kRet + i * kRet;
+    float m = -INFINITY, l = 0.f, a = 0.f;
+    for (int s0 = 0; s0 < p.splits; s0 += 32) {
+      float mx[32], sm[32], v[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        mx[u] = -INFINITY;
+        sm[u] = 0.f;
+        v[u] = 0.f;
+        if (s0 + u < p.splits) {
+          const float* ps = pb + (size_t)(s0 + u) * sstride;
+          mx[u] = ps[0];
+          sm[u] = ps[1];
+          v[u] = ps[2 + t];
+        }
+      }
+      float mb = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) mb = fmaxf(mb, mx[u]);
+      const float mn = fmaxf(m, mb);
+      if (mn == -INFINITY) continue;  // no split of this batch (or before) saw a row
+      const float sc = m == -INFINITY ? 0.f : exp2f(m - mn);
+      l *= sc;
+      a *= sc;
       // a split that saw none of the query's rows has max -inf and weight 0
-      const float f = sml[s][0] == -INFINITY ? 0.f : exp2f(sml[s][0] - m);
-      l = fmaf(sml[s][1], f, l);
-      a = fmaf(pb[(s * kGroup + i) * kPart + 2 + t], f, a);
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const float f = mx[u] == -INFINITY ? 0.f : exp2f(mx[u] - mn);
+        l = fmaf(sm[u], f, l);
+        a = fmaf(v[u], f, a);
+      }
+      m = mn;
     }
-    __syncthreads();
-    const float den = rec[i * kRet + D];
-    const float amem = den != 0.f ? rec[i * kRet + t] / den : 0.f;
+    const float den = rec[D];
+    const float amem = den != 0.f ? rec[t] / den : 0.f;
     const float adot = a / l;
-    out[((size_t)bh * p.n + q0 + i) * D + t] = __float2bfloat16(g * amem + (1.f - g) * adot);
+    out[((size_t)bh * p.n + qi) * D + t] = __float2bfloat16(g * amem + (1.f - g) * adot);
   }
 }
 
@@ -334,7 +352,7 @@ cudaError_t bf16_decode_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   p.H = H;
   p.groups = (n + kGroup - 1) / kGroup;
   decode_splits(BH, n, pos, sms, &p.splits, &p.chunks_per_split);
-  const dim3 gp(p.splits + kRetCTAs, BH, p.groups), gc(BH, p.groups);
+  const dim3 gp(p.splits + kRetCTAs, BH, p.groups), gc(BH, n < 65535 ? n : 65535);
   float* ret = part + (size_t)BH * p.groups * p.splits * kGroup * kPart;
   // the compiled width must hold the widest group: min(n, 16) queries
   const int w = n > 8 ? kGroup : n > 4 ? 8 : n > 2 ? 4 : n;
@@ -343,7 +361,7 @@ cudaError_t bf16_decode_launch(const __nv_bfloat16* q, const __nv_bfloat16* k,
   case W:                                                                                   \
     decode_partial_kernel<W><<<gp, kThreads, 0, stream>>>(q, k, v, k_cache, v_cache, M, z,    \
                                                           part, ret, p);                    \
-    decode_combine_kernel<W><<<gc, kThreads, 0, stream>>>(part, ret, beta, out, p);          \
+    decode_combine_kernel<<<gc, kThreads, 0, stream>>>(part, ret, beta, out, p);             \
     break;
     DECODE_CASE(1)
     DECODE_CASE(2)
