@@ -367,33 +367,30 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   const bool done = warp < kConvWarps ? mbar_wait_warp(bar_done, 0) : true;
   tc_fence_after();
   if (warp < kConvWarps) {
-    // epilogue: warps 0-3 write dM rows, warps 4-7 write G rows (Delta)
+    // epilogue: every converter warp drains 32 rows (its tensor-memory lane quadrant)
+    // x 32 columns of [dM | G]: column chunk (warp >> 2) of dM and, for Delta, the G
+    // chunk four further on; each thread writes its row's 128 bytes as four 256-bit
+    // stores (whole 32-byte sectors)
     const int lane_base = (warp & 3) * 32;
     const int row = lane_base + lane;
-    const int half = warp >> 2;
-    if (warp < 8 && (half == 0 || delta)) {
-      float* dst = dpart + ((size_t)idx * 2 + half) * D * D + (size_t)row * D;
+    for (int k = 0; k < (delta ? 2 : 1); ++k) {
+      const int cc = (warp >> 2) + 4 * k;  // 0..3: dM columns, 4..7: G columns
+      uint32_t rr[32];
+      if (nslab > 0) {
+        tmem_ld32(tmem_d + ((uint32_t)lane_base << 16) + (uint32_t)cc * 32, rr);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t rr[32];
-        if (nslab > 0) {
-          tmem_ld32(tmem_d + ((uint32_t)lane_base << 16) + half * 128 + cc * 32, rr);
-          tmem_wait_ld();
-        } else {
+        for (int e = 0; e < 32; ++e) rr[e] = 0u;
+      }
+      if (done && ok) {
+        if (cc >= 4) {  // G feeds a tf32 MMA in the chain: round it here, unbiased
 #pragma unroll
-          for (int e = 0; e < 32; ++e) rr[e] = 0u;
+          for (int e = 0; e < 32; ++e) rr[e] = tf32_rna(__uint_as_float(rr[e]));
         }
-        if (done && ok) {
-          if (half == 1) {  // G feeds a tf32 MMA in the chain: round it here, unbiased
+        float* dst = dpart + ((size_t)idx * 2 + (cc >> 2)) * D * D + (size_t)row * D + (cc & 3) * 32;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) rr[e] = tf32_rna(__uint_as_float(rr[e]));
-          }
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + cc * 32 + e) =
-                make_float4(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1]),
-                            __uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3]));
-        }
+        for (int e = 0; e < 32; e += 8) st_global_v8(dst + e, rr + e);
       }
     }
     if (zsum) {
