@@ -182,12 +182,22 @@ constexpr int kStageBytes = 4 * kMat;      // 64 KB
 constexpr int kConvWarps = 16;
 constexpr int kStateThreads = (kConvWarps + 2) * 32;
 constexpr int kProdWarp = kConvWarps, kMmaWarp = kConvWarps + 1;
-constexpr int kStateSmem = kStages * kStageBytes + 1024 + 256;  // + alignment, barriers
+constexpr int kZredBytes = kConvRows * 128 * 4;   // 16 KB
+constexpr int kStateSmem = kStages * kStageBytes + kZredBytes + 1024 + 256;  // + alignment, barriers
 
 __device__ __forceinline__ uint32_t tf32_rna(float x) {
   uint32_t r;
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return r;
+}
+
+// Bounded wait used only while draining after an error: ignores the error flag.
+__device__ __forceinline__ void drain_wait_s(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) break;  // 200 ms
+  }
 }
 
 __device__ __forceinline__ uint64_t slab_desc(uint32_t base, int kk) {
@@ -199,28 +209,21 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
              const float* __restrict__ zprev, float* __restrict__ dpart,
              float* __restrict__ zpart, long long L, int N, int S, int CH, int CL, int mode,
-             int zsum, int Hkv) {
+             int zsum, int Hkv, long long nunits) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  // [32][128] partial sums of sigma(K) of one unit (its own area: the ring keeps
+  // streaming the next unit meanwhile)
+  float* sZred = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kZredBytes);
   uint64_t* bar_full = bars;                 // [kStages] TMA landed
   uint64_t* bar_conv = bars + kStages;       // [kStages] operands converted (warp arrivals)
   uint64_t* bar_mma = bars + 2 * kStages;    // [kStages] MMAs of the stage done
-  uint64_t* bar_done = bars + 3 * kStages;   // all MMAs done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
-  // [32][128] partial sums of sigma(K); reuses stage memory once every MMA is done
-  float* sZred = reinterpret_cast<float*>(smem);
+  uint64_t* bar_done = bars + 3 * kStages;   // a unit's MMAs all done (once per unit)
+  uint64_t* bar_drain = bars + 3 * kStages + 1;  // every MMA of the CTA done (at the end)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 2);
 
-  const long long idx = blockIdx.x;
-  const int c = (int)(idx % CH);
-  const int s = (int)((idx / CH) % S);
-  const long long bh = idx / ((long long)CH * S);
-  const long long t0 = (long long)s * N;
-  const int n = (int)min((long long)N, L - t0);
-  const int beg = min(n, c * CL), end = min(n, (c + 1) * CL);
-  const int len = end - beg;
-  const int nslab = len > 0 ? (len + kSlab - 1) / kSlab : 0;
   const bool delta = mode == 1;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t ncols = delta ? 256u : 128u;
@@ -232,6 +235,7 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
       mbar_init(&bar_mma[i], 1);
     }
     mbar_init(bar_done, 1);
+    mbar_init(bar_drain, 1);
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -243,147 +247,195 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   bool ok = true;
-  float dz[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // Linear: sum of sigma(K)
   const int cg = tid & 15;  // this converter's 8-feature group
   const int r = tid >> 4;   // this converter's token row in each slab
 
+  // unit idx = (head, segment, token chunk): its head, first row, tokens and slabs
+  struct Unit {
+    long long bh, row0;
+    int s, len, nslab;
+  };
+  auto unit = [&](long long idx) {
+    Unit x;
+    const int c = (int)(idx % CH);
+    x.s = (int)((idx / CH) % S);
+    x.bh = idx / ((long long)CH * S);
+    const long long t0 = (long long)x.s * N;
+    const int n = (int)min((long long)N, L - t0);
+    const int beg = min(n, c * CL), end = min(n, (c + 1) * CL);
+    x.len = end - beg;
+    x.nslab = x.len > 0 ? (x.len + kSlab - 1) / kSlab : 0;
+    x.row0 = t0 + beg;
+    return x;
+  };
+
   if (warp == kProdWarp) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer: the ring runs on across units ----------------
     if (lane == 0) {
-      const int row0 = (int)(t0 + beg);
-      for (int sl = 0; sl < nslab; ++sl) {
-        const int stg = sl % kStages;
-        if (sl >= kStages &&
-            !mbar_wait(&bar_mma[stg], (uint32_t)((sl / kStages - 1) & 1))) {
-          ok = false;
-          break;
+      int g = 0;
+      int issued[kStages] = {0, 0, 0};
+      for (long long idx = blockIdx.x; ok && idx < nunits; idx += gridDim.x) {
+        const Unit x = unit(idx);
+        const int hh = (int)(x.bh % Hkv), bb = (int)(x.bh / Hkv);
+        for (int sl = 0; sl < x.nslab; ++sl, ++g) {
+          const int stg = g % kStages;
+          if (g >= kStages && !mbar_wait(&bar_mma[stg], (uint32_t)((g / kStages - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + stg * kStageBytes;
+          mbar_arrive_expect_tx(&bar_full[stg], 2 * kMat);
+          const int row = (int)(x.row0 + sl * kSlab);
+          tma_load_4d(st + OFF_KH, &tm_k, &bar_full[stg], 0, row, hh, bb);
+          tma_load_4d(st + OFF_KH + kBox, &tm_k, &bar_full[stg], 64, row, hh, bb);
+          tma_load_4d(st + OFF_V, &tm_v, &bar_full[stg], 0, row, hh, bb);
+          tma_load_4d(st + OFF_V + kBox, &tm_v, &bar_full[stg], 64, row, hh, bb);
+          ++issued[stg];
         }
-        uint8_t* st = smem + stg * kStageBytes;
-        mbar_arrive_expect_tx(&bar_full[stg], 2 * kMat);
-        const int row = row0 + sl * kSlab;
-        const int hh = (int)(bh % Hkv), bb = (int)(bh / Hkv);
-        tma_load_4d(st + OFF_KH, &tm_k, &bar_full[stg], 0, row, hh, bb);
-        tma_load_4d(st + OFF_KH + kBox, &tm_k, &bar_full[stg], 64, row, hh, bb);
-        tma_load_4d(st + OFF_V, &tm_v, &bar_full[stg], 0, row, hh, bb);
-        tma_load_4d(st + OFF_V + kBox, &tm_v, &bar_full[stg], 64, row, hh, bb);
       }
+      if (!ok)  // let the copies already issued land before the CTA exits
+        for (int st = 0; st < kStages; ++st)
+          if (issued[st] > 0) drain_wait_s(&bar_full[st], (uint32_t)((issued[st] - 1) & 1));
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     // The whole warp runs the loop and waits; one elected lane (always lane 0)
     // issues and commits, which keeps the issue path short next to the busy
-    // converter warps on the same scheduler.
+    // converter warps on the same scheduler. A unit's first product overwrites the
+    // accumulator: the converters read the previous unit's sums out of it before
+    // they convert (and signal) the first slab of this one.
     const uint32_t id256 = idesc_f32acc(1, 1, 1, 128, 256);
     const uint32_t id128 = idesc_f32acc(1, 1, 1, 128, 128);
-    for (int sl = 0; sl < nslab; ++sl) {
-      const int stg = sl % kStages;
-      if (!mbar_wait_warp(&bar_conv[stg], (uint32_t)((sl / kStages) & 1))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t base = smem_u32(smem + stg * kStageBytes);
-      if (elect_one()) {
-#pragma unroll
-        for (int kk = 0; kk < kSlab / 16; ++kk) {
-          const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t a_hi = slab_desc(base + OFF_KH, kk);
-          const uint64_t a_lo = slab_desc(base + OFF_KL, kk);
-          const uint64_t b_v = slab_desc(base + OFF_V, kk);
-          mma_bf16_ss(tmem_d, a_hi, b_v, delta ? id256 : id128, acc);  // [dM | G] += hi^T [V | GH]
-          mma_bf16_ss(tmem_d, a_lo, b_v, id128, 1u);                  // dM += lo^T V
+    int g = 0;
+    for (long long idx = blockIdx.x; ok && idx < nunits; idx += gridDim.x) {
+      const Unit x = unit(idx);
+      for (int sl = 0; sl < x.nslab; ++sl, ++g) {
+        const int stg = g % kStages;
+        if (!mbar_wait_warp(&bar_conv[stg], (uint32_t)((g / kStages) & 1))) {
+          ok = false;
+          break;
         }
-        mma_commit(&bar_mma[stg]);
+        tc_fence_after();
+        const uint32_t base = smem_u32(smem + stg * kStageBytes);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kSlab / 16; ++kk) {
+            const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t a_hi = slab_desc(base + OFF_KH, kk);
+            const uint64_t a_lo = slab_desc(base + OFF_KL, kk);
+            const uint64_t b_v = slab_desc(base + OFF_V, kk);
+            mma_bf16_ss(tmem_d, a_hi, b_v, delta ? id256 : id128, acc);  // [dM | G] += hi^T [V | GH]
+            mma_bf16_ss(tmem_d, a_lo, b_v, id128, 1u);                  // dM += lo^T V
+          }
+          mma_commit(&bar_mma[stg]);
+        }
+        __syncwarp();
       }
-      __syncwarp();
+      // the unit's sums are complete (also after an error, so that the converters never
+      // wait on a phase that cannot come). A unit without tokens has no products and
+      // no commit: two commits with no converter wait between them would let the
+      // barrier complete twice before its waiters saw the first.
+      if (x.nslab > 0) {
+        if (elect_one()) mma_commit(bar_done);
+        __syncwarp();
+      }
     }
-    if (elect_one()) mma_commit(bar_done);  // tracks every MMA issued above
+    // no product may still be running when the CTA frees tensor memory (the converters
+    // stop waiting for the units' sums after an error)
+    if (elect_one()) mma_commit(bar_drain);
     __syncwarp();
+    drain_wait_s(bar_drain, 0);
   } else {
-    // ---------------- converters (warps 0..15) ----------------
-    float zr[8];
+    // ---------------- converters (warps 0..15), then each unit's epilogue ----------------
+    int g = 0, un = 0;  // un: units with tokens so far (bar_done completes once for each)
+    for (long long idx = blockIdx.x; idx < nunits; idx += gridDim.x) {
+      const Unit x = unit(idx);
+      float dz[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // sum of sigma(K)
+      float zr[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) zr[e] = delta ? zprev[((size_t)bh * S + s) * D + cg * 8 + e] : 0.f;
-    for (int sl = 0; sl < nslab && ok; ++sl) {
-      const int stg = sl % kStages;
-      uint8_t* st = smem + stg * kStageBytes;
-      if (!mbar_wait_warp(&bar_full[stg], (uint32_t)((sl / kStages) & 1))) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int rh = 0; rh < kSlab / kConvRows; ++rh) {
-        const int row = r + kConvRows * rh;
-        const bool valid = sl * kSlab + row < len;
-        const uint32_t off = (uint32_t)(cg >> 3) * kBox + sw128(row, cg & 7);
-        const uint4 raw = *reinterpret_cast<const uint4*>(st + OFF_KH + off);
-        float f[8];
-        bf16x8_to_f32(raw, f);
-        // sigma(K), every exponential on the MUFU: the converters are bound by their
-        // instruction issue, and the FMA-pipe polynomial costs more instructions (with
-        // half of the exponentials on it the state path was 3-4% slower, measured at
-        // the 1B-layer shape in both modes)
-        float den = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = elu1(f[e]);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          f[e] = valid ? f[e] : 0.f;
-          den = fmaf(f[e], zr[e], den);
-          dz[e] += f[e];
+      for (int e = 0; e < 8; ++e)
+        zr[e] = delta ? zprev[((size_t)x.bh * S + x.s) * D + cg * 8 + e] : 0.f;
+      for (int sl = 0; sl < x.nslab && ok; ++sl, ++g) {
+        const int stg = g % kStages;
+        uint8_t* st = smem + stg * kStageBytes;
+        if (!mbar_wait_warp(&bar_full[stg], (uint32_t)((g / kStages) & 1))) {
+          ok = false;
+          break;
         }
-        uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
-          const float2 hf = __bfloat1622float2(h);
-          const __nv_bfloat162 l = __floats2bfloat162_rn(f[2 * e] - hf.x, f[2 * e + 1] - hf.y);
-          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[e] = *reinterpret_cast<const uint32_t*>(&l);
-        }
-        *reinterpret_cast<uint4*>(st + OFF_KH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(st + OFF_KL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        if (delta) {
-          // 16 lanes of a half-warp hold the 128 features of one token
+        for (int rh = 0; rh < kSlab / kConvRows; ++rh) {
+          const int row = r + kConvRows * rh;
+          const bool valid = sl * kSlab + row < x.len;
+          const uint32_t off = (uint32_t)(cg >> 3) * kBox + sw128(row, cg & 7);
+          const uint4 raw = *reinterpret_cast<const uint4*>(st + OFF_KH + off);
+          float f[8];
+          bf16x8_to_f32(raw, f);
+          // sigma(K), every exponential on the MUFU: the converters are bound by their
+          // instruction issue, and the FMA-pipe polynomial costs more instructions (with
+          // half of the exponentials on it the state path was 3-4% slower, measured at
+          // the 1B-layer shape in both modes)
+          float den = 0.f;
 #pragma unroll
-          for (int o = 8; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-          const float inv = den != 0.f ? 1.f / den : 0.f;
-          uint32_t gh[4];
+          for (int e = 0; e < 8; ++e) f[e] = elu1(f[e]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            f[e] = valid ? f[e] : 0.f;
+            den = fmaf(f[e], zr[e], den);
+            dz[e] += f[e];
+          }
+          uint32_t hi[4], lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 g = __floats2bfloat162_rn(f[2 * e] * inv, f[2 * e + 1] * inv);
-            gh[e] = *reinterpret_cast<const uint32_t*>(&g);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+            const float2 hf = __bfloat1622float2(h);
+            const __nv_bfloat162 l = __floats2bfloat162_rn(f[2 * e] - hf.x, f[2 * e + 1] - hf.y);
+            hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+            lo[e] = *reinterpret_cast<const uint32_t*>(&l);
           }
-          *reinterpret_cast<uint4*>(st + OFF_GH + off) = make_uint4(gh[0], gh[1], gh[2], gh[3]);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive_warp(&bar_conv[stg]);
-    }
-  }
-
-  // Only the converter warps wait for the MMAs: the idle lanes of the producer and
-  // MMA warps must not spin next to the lane that drives the pipeline.
-  const bool done = warp < kConvWarps ? mbar_wait_warp(bar_done, 0) : true;
-  tc_fence_after();
-  if (warp < kConvWarps) {
-    // epilogue: every converter warp drains 32 rows (its tensor-memory lane quadrant)
-    // x 32 columns of [dM | G]: column chunk (warp >> 2) of dM and, for Delta, the G
-    // chunk four further on; each thread writes its row's 128 bytes as four 256-bit
-    // stores (whole 32-byte sectors)
-    const int lane_base = (warp & 3) * 32;
-    const int row = lane_base + lane;
-    for (int k = 0; k < (delta ? 2 : 1); ++k) {
-      const int cc = (warp >> 2) + 4 * k;  // 0..3: dM columns, 4..7: G columns
-      uint32_t rr[32];
-      if (nslab > 0) {
-        tmem_ld32(tmem_d + ((uint32_t)lane_base << 16) + (uint32_t)cc * 32, rr);
-        tmem_wait_ld();
-      } else {
+          *reinterpret_cast<uint4*>(st + OFF_KH + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(st + OFF_KL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          if (delta) {
+            // 16 lanes of a half-warp hold the 128 features of one token
 #pragma unroll
-        for (int e = 0; e < 32; ++e) rr[e] = 0u;
+            for (int o = 8; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+            const float inv = den != 0.f ? 1.f / den : 0.f;
+            uint32_t gh[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 g2 = __floats2bfloat162_rn(f[2 * e] * inv, f[2 * e + 1] * inv);
+              gh[e] = *reinterpret_cast<const uint32_t*>(&g2);
+            }
+            *reinterpret_cast<uint4*>(st + OFF_GH + off) = make_uint4(gh[0], gh[1], gh[2], gh[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive_warp(&bar_conv[stg]);
       }
-      if (done && ok) {
+      if (!ok) break;
+      if (x.nslab > 0) {
+        if (!mbar_wait_warp(bar_done, (uint32_t)(un & 1))) {
+          ok = false;
+          break;
+        }
+        ++un;
+        tc_fence_after();
+      }
+      // epilogue: every converter warp drains 32 rows (its tensor-memory lane quadrant)
+      // x 32 columns of [dM | G]: column chunk (warp >> 2) of dM and, for Delta, the G
+      // chunk four further on; each thread writes its row's 128 bytes as four 256-bit
+      // stores (whole 32-byte sectors)
+      const int lane_base = (warp & 3) * 32;
+      const int row = lane_base + lane;
+      for (int k = 0; k < (delta ? 2 : 1); ++k) {
+        const int cc = (warp >> 2) + 4 * k;  // 0..3: dM columns, 4..7: G columns
+        uint32_t rr[32];
+        if (x.nslab > 0) {
+          tmem_ld32(tmem_d + ((uint32_t)lane_base << 16) + (uint32_t)cc * 32, rr);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) rr[e] = 0u;
+        }
         if (cc >= 4) {  // G feeds a tf32 MMA in the chain: round it here, unbiased
 #pragma unroll
           for (int e = 0; e < 32; ++e) rr[e] = tf32_rna(__uint_as_float(rr[e]));
@@ -392,21 +444,27 @@ state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ C
 #pragma unroll
         for (int e = 0; e < 32; e += 8) st_global_v8(dst + e, rr + e);
       }
-    }
-    if (zsum) {
-      // chunk sum of sigma(K): threads with the same feature group add up
+      // the accumulator is read: the next unit's first product may overwrite it (the
+      // MMA warp issues it only after this warp's arrival for that unit's first slab)
+      tc_fence_before();
+      if (zsum) {
+        // unit sum of sigma(K): threads with the same feature group add up
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sZred[r * 128 + cg * 8 + e] = dz[e];
+        for (int e = 0; e < 8; ++e) sZred[r * 128 + cg * 8 + e] = dz[e];
+        named_bar_sync(1, kConvWarps * 32);
+        if (tid < D) {
+          float sum = 0.f;
+#pragma unroll
+          for (int rr = 0; rr < kConvRows; ++rr) sum += sZred[rr * 128 + tid];
+          zpart[idx * D + tid] = sum;
+        }
+        named_bar_sync(1, kConvWarps * 32);  // sZred is rewritten by the next unit
+      }
     }
   }
+
   tc_fence_before();
   __syncthreads();
-  if (zsum && tid < D) {
-    float sum = 0.f;
-#pragma unroll
-    for (int rr = 0; rr < kConvRows; ++rr) sum += sZred[rr * 128 + tid];
-    zpart[idx * D + tid] = sum;
-  }
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_d, ncols);
@@ -746,6 +804,10 @@ cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, co
                               int CL, int mode, int first, cudaStream_t stream,
                               const Bf16Layout* lay) {
   const unsigned nunits = (unsigned)((long long)BH * S * CH);
+  // persistent: one CTA per SM walks the units (head, segment, token chunk)
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const unsigned grid = nunits < (unsigned)sms ? nunits : (unsigned)sms;
   // key/value head i = (batch row i / Hkv, head i % Hkv); without a layout, BH
   // contiguous [L, 128] planes
   const Bf16Layout l = lay ? *lay : Bf16Layout::bhld(BH, 1, L);
@@ -759,14 +821,14 @@ cudaError_t bf16_state_launch(const __nv_bfloat16* k, const __nv_bfloat16* v, co
     zpart_kernel<<<nunits, 256, 0, stream>>>(k, ws.zpart, L, N, S, CH, CL, Hkv, l.kv_sb, l.kv_sh,
                                              l.kv_sl);
     zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH, first);
-    state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(
-        mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 0, Hkv);
+    state_kernel<<<grid, kStateThreads, kStateSmem, stream>>>(
+        mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 0, Hkv, (long long)nunits);
   } else {
     // The state GEMM also produces the sums of sigma(K): always in Linear mode, and
     // in Linear+Delta mode for a lone segment whose z_{-1} is already in place. In
     // Linear mode the chain kernel scans z itself.
-    state_kernel<<<nunits, kStateThreads, kStateSmem, stream>>>(
-        mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 1, Hkv);
+    state_kernel<<<grid, kStateThreads, kStateSmem, stream>>>(
+        mk, mv, ws.zprev, ws.dpart, ws.zpart, L, N, S, CH, CL, mode, 1, Hkv, (long long)nunits);
     if (mode == 1)
       zscan_kernel<<<BH, D, 0, stream>>>(ws.zpart, z_in, z_out, ws.zprev, S, CH, first);
   }

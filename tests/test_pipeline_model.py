@@ -840,37 +840,62 @@ def test_attention_model_detects_a_missing_sfree_wait():
 # ------------------------------------------------------------------------------
 # the forward's state kernel (one chunk of one segment) and the state chains
 # ------------------------------------------------------------------------------
-def state_roles(sim, nslab, stages=3, conv_warps=16):
+def state_roles(sim, units, stages=3, conv_warps=16, zsum=True):
+    """The persistent state kernel: a CTA walks units (head, segment, chunk) of
+    units[i] slabs each; the ring and its barrier phases run on across units; the MMA
+    warp commits DONE once per unit with tokens and DRAIN at the end; the converters
+    wait for such a unit's DONE before draining its accumulator (a unit without
+    tokens writes zeros and waits for nothing), and (zsum) meet at a named barrier
+    twice per unit around the shared sum area."""
     FULL = [sim.bar(f"full{i}") for i in range(stages)]
     CONV = [sim.bar(f"conv{i}", conv_warps) for i in range(stages)]
     MMA = [sim.bar(f"mma{i}") for i in range(stages)]
     DONE = sim.bar("done")
+    DRAIN = sim.bar("drain")
+    convs = [f"conv{w}" for w in range(conv_warps)]
 
     def producer():
-        for sl in range(nslab):
-            stg = sl % stages
-            if sl >= stages:
-                yield ('wait', MMA[stg], sl // stages - 1)
-            yield ('tma', FULL[stg])
+        g = 0
+        for nslab in units:
+            for _ in range(nslab):
+                stg = g % stages
+                if g >= stages:
+                    yield ('wait', MMA[stg], g // stages - 1)
+                yield ('tma', FULL[stg], g // stages)
+                g += 1
 
     def mma():
-        for sl in range(nslab):
-            stg = sl % stages
-            yield ('wait', CONV[stg], sl // stages)
-            yield ('mma',)
-            yield ('commit', MMA[stg])
-        yield ('commit', DONE)
+        g = 0
+        for nslab in units:
+            for _ in range(nslab):
+                stg = g % stages
+                yield ('wait', CONV[stg], g // stages)
+                yield ('mma',)
+                yield ('commit', MMA[stg])
+                g += 1
+            if nslab > 0:
+                yield ('commit', DONE)
+        yield ('commit', DRAIN)
+        yield ('wait', DRAIN, 0)
 
     def converter():
-        for sl in range(nslab):
-            stg = sl % stages
-            yield ('wait', FULL[stg], sl // stages)
-            yield ('arrive', CONV[stg], 1)  # operands converted in place
-        yield ('wait', DONE, 0)
+        g, dn = 0, 0
+        for un, nslab in enumerate(units):
+            for _ in range(nslab):
+                stg = g % stages
+                yield ('wait', FULL[stg], g // stages)
+                yield ('arrive', CONV[stg], 1)  # operands converted in place
+                g += 1
+            if nslab > 0:
+                yield ('wait', DONE, dn)        # then the accumulator is drained
+                dn += 1
+            if zsum:
+                yield ('named', f"zred{un}a", convs)
+                yield ('named', f"zred{un}b", convs)
 
     roles = {"producer": producer(), "mma": mma()}
-    for w in range(conv_warps):
-        roles[f"conv{w}"] = converter()
+    for w in convs:
+        roles[w] = converter()
     return roles
 
 
@@ -913,11 +938,70 @@ def chain_roles(sim, S, CH, delta=True):
     return roles
 
 
-@pytest.mark.parametrize("nslab", [0, 1, 2, 3, 4, 7, 32])
-def test_state_kernel_protocol(nslab):
-    for seed in range(20):
-        sim = Sim(seed * 100 + nslab)
-        sim.run(state_roles(sim, nslab))
+@pytest.mark.parametrize("units", [[1], [8], [32], [8, 8, 8], [0, 3, 5], [2, 0], [5, 1, 7, 2],
+                                   [32, 32, 1]])
+def test_state_kernel_protocol(units):
+    for seed in range(30):
+        sim = Sim(seed * 1000 + sum(units) + len(units))
+        sim.run(state_roles(sim, units))
+
+
+def test_state_model_detects_a_commit_for_a_unit_without_tokens():
+    """DONE committed for a unit without tokens as well: the two commits of units
+    [2, 0] complete the barrier twice before the converters' first wait."""
+    def broken(sim, units):
+        roles = state_roles(sim, units, zsum=False)
+        stages = 3
+        CONV = [sim.bars[f"conv{i}"] for i in range(stages)]
+        MMA = [sim.bars[f"mma{i}"] for i in range(stages)]
+
+        def mma():
+            g = 0
+            for nslab in units:
+                for _ in range(nslab):
+                    stg = g % stages
+                    yield ('wait', CONV[stg], g // stages)
+                    yield ('mma',)
+                    yield ('commit', MMA[stg])
+                    g += 1
+                yield ('commit', sim.bars["done"])
+            yield ('commit', sim.bars["drain"])
+            yield ('wait', sim.bars["drain"], 0)
+        roles["mma"] = mma()
+        return roles
+    with pytest.raises(AssertionError, match="phase skipped"):
+        for seed in range(40):
+            sim = Sim(seed)
+            sim.run(broken(sim, [2, 0]))
+
+
+def test_state_model_detects_a_done_barrier_committed_once():
+    """DONE committed once for the whole CTA instead of once per unit: the converters'
+    wait for the second unit's sums never completes."""
+    def broken(sim, units):
+        roles = state_roles(sim, units, zsum=False)
+        stages = 3
+        FULL = [sim.bars[f"full{i}"] for i in range(stages)]
+        CONV = [sim.bars[f"conv{i}"] for i in range(stages)]
+        MMA = [sim.bars[f"mma{i}"] for i in range(stages)]
+
+        def mma():
+            g = 0
+            for nslab in units:
+                for _ in range(nslab):
+                    stg = g % stages
+                    yield ('wait', CONV[stg], g // stages)
+                    yield ('mma',)
+                    yield ('commit', MMA[stg])
+                    g += 1
+            yield ('commit', sim.bars["done"])
+            yield ('commit', sim.bars["drain"])
+            yield ('wait', sim.bars["drain"], 0)
+        roles["mma"] = mma()
+        return roles
+    with pytest.raises(AssertionError, match="deadlock"):
+        sim = Sim(5)
+        sim.run(broken(sim, [4, 4]))
 
 
 @pytest.mark.parametrize("S,CH", [(1, 1), (1, 8), (3, 2), (16, 1), (5, 4)])
