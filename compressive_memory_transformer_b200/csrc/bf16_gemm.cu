@@ -4,14 +4,18 @@
 // attention layer ("Leave No Context Behind", arXiv 2404.07143, as quoted on
 // llm-papers-study.pages.dev, sections 3.1 and 3.6).
 //
-// Persistent kernel, one CTA per SM, 192 threads: warps 0-3 drain the accumulator
-// (tensor memory -> bf16 -> global), warp 4 is the TMA producer, warp 5 allocates
-// tensor memory and issues the MMAs from one elected lane. Output tiles are 128 x 128,
-// taken in the order (m, n) with n fastest so that a 128-row block of A is reused
-// from L2 by the N/128 tiles that need it. Each k-step brings a 128 x 128 tile of A
-// (K-major) and one of B (MN-major) into a 3-stage ring; eight tcgen05 MMAs
-// (K = 16 each) accumulate into one of two 128-column accumulators, so the epilogue
-// of one tile overlaps the products of the next.
+// Two persistent kernels, 192 threads each: warps 0-3 drain the accumulator (tensor
+// memory -> bf16 -> global), warp 4 is the TMA producer, warp 5 allocates tensor
+// memory and issues the MMAs from one elected lane; output tiles are taken in the
+// order (m, n) with n fastest, so that a block of rows of A is reused from L2 by the
+// tiles that need it, and two accumulators let the epilogue of one tile overlap the
+// products of the next.
+//   gemm_pair_kernel (every N a multiple of 256): 256 x 256 tiles on CTA pairs with
+//     cta_group::2 MMAs, epilogue through shared memory and TMA stores; up to three B
+//     matrices sharing A in one launch (the layer's Q, K and V projections).
+//   gemm_kernel (otherwise): 128 x 128 tiles on one CTA per SM; each k-step brings a
+//     128 x 128 tile of A (K-major) and one of B (MN-major) into a 3-stage ring; eight
+//     tcgen05 MMAs (K = 16 each) per k-step.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda.h>
