@@ -156,7 +156,7 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
           ks = knew + src;
           vs = vnew + src;
         }
-        cp_async16(&sk[row][c * 4], ks);
+        cp_async16(&sk[row][(c ^ (row & 15)) * 4], ks);
         cp_async16(&sv[row][c * 4], vs);
       }
     }
@@ -168,39 +168,62 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
       for (int e = first * (D / 8) + t; e < nr * (D / 8); e += kThreads) {
         const int row = e / (D / 8), c = e % (D / 8);
         const size_t dst = base + (size_t)(r0 + row) * D + c * 8;
-        *reinterpret_cast<uint4*>(kc + dst) = *reinterpret_cast<const uint4*>(&sk[row][c * 4]);
+        *reinterpret_cast<uint4*>(kc + dst) =
+            *reinterpret_cast<const uint4*>(&sk[row][(c ^ (row & 15)) * 4]);
         *reinterpret_cast<uint4*>(vc + dst) = *reinterpret_cast<const uint4*>(&sv[row][c * 4]);
       }
     }
-    // scores: thread pair (2r, 2r + 1) covers row r, features [64h, 64h + 64); each
-    // key pair is read from shared memory once for all the group's queries; the pair
-    // word read at step j is rotated by 2r + h, so a warp's 32 reads fall in 32
-    // different banks
+    // scores: thread (row r, part p). With 16 queries part p takes queries [8p, 8p + 8)
+    // over all 128 features; with fewer, every query over features [64p, 64p + 64),
+    // and the two parts' sums meet in shared memory. A warp's lanes are 32 rows with
+    // the same part, so every query read is a broadcast; the rows' 16-byte chunks are
+    // stored permuted (chunk c of row r at c ^ (r & 15)), so that the 32 rows' chunk c
+    // fall in distinct banks.
     {
-      const int r = t >> 1, h = t & 1;
-      float sc[NQ];
+      constexpr int QPT = NQ == kGroup ? kGroup / 2 : NQ;  // queries per thread
+      const int r = t & (kRows - 1), pt = t >> 6;
+      const int qb = NQ == kGroup ? QPT * pt : 0;
+      const int cb = NQ == kGroup ? 0 : 8 * pt, ce = NQ == kGroup ? D / 8 : 8 * pt + 8;
+      float sc[QPT];
 #pragma unroll
-      for (int i = 0; i < NQ; ++i) sc[i] = 0.f;
+      for (int i = 0; i < QPT; ++i) sc[i] = 0.f;
       if (r < nr) {
-#pragma unroll 8
-        for (int j = 0; j < 32; ++j) {
-          const int jj = (j + 2 * r + h) & 31;
-          const uint32_t u = sk[r][32 * h + jj];
-          const float k0 = bf_lo(u), k1 = bf_hi(u);
+#pragma unroll 2
+        for (int c = cb; c < ce; ++c) {
+          const uint4 kr = *reinterpret_cast<const uint4*>(&sk[r][(c ^ (r & 15)) * 4]);
+          const float k8[8] = {bf_lo(kr.x), bf_hi(kr.x), bf_lo(kr.y), bf_hi(kr.y),
+                               bf_lo(kr.z), bf_hi(kr.z), bf_lo(kr.w), bf_hi(kr.w)};
 #pragma unroll
-          for (int i = 0; i < NQ; ++i) {
-            if (i < nq) {
-              const float2 qf = *reinterpret_cast<const float2*>(&sq[i][64 * h + 2 * jj]);
-              sc[i] = fmaf(qf.x, k0, fmaf(qf.y, k1, sc[i]));
+          for (int i = 0; i < QPT; ++i) {
+            if (qb + i < nq) {
+              const float4 qa = *reinterpret_cast<const float4*>(&sq[qb + i][8 * c]);
+              const float4 qc = *reinterpret_cast<const float4*>(&sq[qb + i][8 * c + 4]);
+              float v = fmaf(qa.x, k8[0], sc[i]);
+              v = fmaf(qa.y, k8[1], v);
+              v = fmaf(qa.z, k8[2], v);
+              v = fmaf(qa.w, k8[3], v);
+              v = fmaf(qc.x, k8[4], v);
+              v = fmaf(qc.y, k8[5], v);
+              v = fmaf(qc.z, k8[6], v);
+              sc[i] = fmaf(qc.w, k8[7], v);
             }
           }
         }
       }
+      if (NQ != kGroup && pt == 1) {
 #pragma unroll
-      for (int i = 0; i < NQ; ++i) {
-        if (i < nq) {
-          const float sv2 = sc[i] + __shfl_xor_sync(0xffffffffu, sc[i], 1);
-          if (h == 0) ss[i][r] = (r < nr && r0 + r <= p.pos + q0 + i) ? sv2 : -INFINITY;
+        for (int i = 0; i < QPT; ++i)
+          if (i < nq) ss[i][r] = sc[i];
+      }
+      __syncthreads();
+      if (NQ == kGroup || pt == 0) {
+#pragma unroll
+        for (int i = 0; i < QPT; ++i) {
+          const int qi = qb + i;
+          if (qi < nq) {
+            const float v = NQ == kGroup ? sc[i] : sc[i] + ss[qi][r];
+            ss[qi][r] = (r < nr && r0 + r <= p.pos + q0 + qi) ? v : -INFINITY;
+          }
         }
       }
     }
@@ -239,8 +262,27 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
 #pragma unroll
       for (int i = 0; i < NQ; ++i)
         if (i < nq) acc[i] *= sm_a[i];
-#pragma unroll 4
-      for (int r = 0; r < nr; ++r) {
+      // four rows per step: each query's four probabilities are one 128-bit broadcast
+      int r = 0;
+      for (; r + 4 <= nr; r += 4) {
+        float vf[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t u = sv[r + k][t >> 1];
+          vf[k] = (t & 1) ? bf_hi(u) : bf_lo(u);
+        }
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+          if (i < nq) {
+            const float4 p4 = *reinterpret_cast<const float4*>(&ss[i][r]);
+            float v = fmaf(p4.x, vf[0], acc[i]);
+            v = fmaf(p4.y, vf[1], v);
+            v = fmaf(p4.z, vf[2], v);
+            acc[i] = fmaf(p4.w, vf[3], v);
+          }
+        }
+      }
+      for (; r < nr; ++r) {
         const uint32_t u = sv[r][t >> 1];
         const float vf = (t & 1) ? bf_hi(u) : bf_lo(u);
 #pragma unroll
