@@ -21,9 +21,9 @@
 //                          its group against the chunk (two threads per row, 64
 //                          features each) and keeps one online-softmax partial
 //                          (max, sum, 128 accumulators) per query in exp2 units.
-//                          Four more CTAs per (head, group) compute the retrieval
-//                          sigma(q) M_{s-1} (32 columns each, M read row-coalesced)
-//                          and sigma(q) z_{s-1}, beside the cache reads.
+//                          One more CTA per (head, group) computes the retrieval
+//                          sigma(q) M_{s-1} (a column per thread, M read
+//                          row-coalesced) and sigma(q) z_{s-1}, beside the cache reads.
 //   decode_combine_kernel  grid (BH, queries). Merges the splits' partials of one
 //                          query, divides the retrieval by its denominator, applies
 //                          the gate and writes out in bf16.
@@ -45,7 +45,7 @@ constexpr int kGroup = 16;    // queries per CTA
 constexpr int kThreads = 128;
 constexpr int kPart = 2 + D;  // one partial: max, sum, 128 accumulators
 constexpr int kMaxSplits = 512;
-constexpr int kRetCTAs = 4;   // retrieval CTAs per (head, group), 32 columns of M each
+constexpr int kRetCTAs = 1;   // retrieval CTAs per (head, group): thread t forms column t
 constexpr int kRet = D + 1;   // one retrieval record: sigma(q) M (128), sigma(q) z
 
 struct DecodeParams {
@@ -75,47 +75,39 @@ decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* 
   const float sl = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
 
   if (split >= p.splits) {
-    // retrieval CTA cb: columns [32 cb, 32 cb + 32) of sigma(q) M_{s-1}; cb 0 also
-    // forms sigma(q) z_{s-1}
-    const int cb = split - p.splits, lane = t & 31, w = t >> 5;
+    // the retrieval CTA: thread t forms column t of sigma(q) M_{s-1} (M read
+    // row-coalesced, 32 rows' loads in flight), and the CTA the denominators
+    // sigma(q) z_{s-1}. One such CTA per (head, group) keeps a one-token call within
+    // one wave of CTAs beside the cache splits.
+    const int lane = t & 31, w = t >> 5;
     float (*sphi)[D] = sq;
     for (int i = 0; i < nq; ++i)
       sphi[i][t] = elu1(__bfloat162float(q[((size_t)bh * p.n + q0 + i) * D + t]));
     __syncthreads();
     float* rec = ret + ((size_t)bh * p.groups + grp) * kGroup * kRet;
-    if (cb == 0) {
-      const float zt = z[(size_t)bh * D + t];
-      for (int i = 0; i < nq; ++i) {
-        float dp = sphi[i][t] * zt;
+    const float zt = z[(size_t)bh * D + t];
+    for (int i = 0; i < nq; ++i) {
+      float dp = sphi[i][t] * zt;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) dp += __shfl_xor_sync(0xffffffffu, dp, o);
-        if (lane == 0) ss[i][w] = dp;
-      }
+      for (int o = 16; o > 0; o >>= 1) dp += __shfl_xor_sync(0xffffffffu, dp, o);
+      if (lane == 0) ss[i][w] = dp;
     }
     float acc[NQ];
 #pragma unroll
     for (int i = 0; i < NQ; ++i) acc[i] = 0.f;
-    const float* Mc = M + (size_t)bh * D * D + 32 * cb + lane;
-#pragma unroll 8
-    for (int k = w; k < D; k += kThreads / 32) {
-      const float m = Mc[(size_t)k * D];
+    const float* Mc = M + (size_t)bh * D * D + t;
+#pragma unroll 32
+    for (int k = 0; k < D; ++k) {
+      const float m = __ldg(Mc + (size_t)k * D);
 #pragma unroll
       for (int i = 0; i < NQ; ++i)
         if (i < nq) acc[i] = fmaf(sphi[i][k], m, acc[i]);
     }
-    float (*red)[NQ][32] = reinterpret_cast<float (*)[NQ][32]>(&sk[0][0]);
 #pragma unroll
     for (int i = 0; i < NQ; ++i)
-      if (i < nq) red[w][i][lane] = acc[i];
+      if (i < nq) rec[i * kRet + t] = acc[i];
     __syncthreads();
-    if (w == 0) {
-#pragma unroll
-      for (int i = 0; i < NQ; ++i)
-        if (i < nq)
-          rec[i * kRet + 32 * cb + lane] = (red[0][i][lane] + red[1][i][lane]) +
-                                           (red[2][i][lane] + red[3][i][lane]);
-    }
-    if (cb == 0 && t < nq) rec[t * kRet + D] = (ss[t][0] + ss[t][1]) + (ss[t][2] + ss[t][3]);
+    if (t < nq) rec[t * kRet + D] = (ss[t][0] + ss[t][1]) + (ss[t][2] + ss[t][3]);
     return;
   }
 
@@ -360,12 +352,13 @@ decode_combine_kernel(const float* __restrict__ part, const float* __restrict__ 
   }
 }
 
-// Cache split: one 64-row chunk per CTA while that keeps the grid within four CTAs
-// per SM, more chunks per CTA beyond; at most kMaxSplits splits.
+// Cache split: one 64-row chunk per CTA while the splits and the retrieval CTA of
+// every (head, group) fit one wave of four CTAs per SM, more chunks per CTA beyond;
+// at most kMaxSplits splits.
 void decode_splits(int BH, int n, int pos, int sms, int* splits, int* cps) {
   const int groups = (n + kGroup - 1) / kGroup;
   const int chunks = (pos + n + kRows - 1) / kRows;
-  const long long want = (4LL * sms + (long long)BH * groups - 1) / ((long long)BH * groups);
+  const long long want = 4LL * sms / ((long long)BH * groups) - kRetCTAs;
   int s = want < 1 ? 1 : (want > kMaxSplits ? kMaxSplits : (int)want);
   if (s > chunks) s = chunks;
   *cps = (chunks + s - 1) / s;
