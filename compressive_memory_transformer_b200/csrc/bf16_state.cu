@@ -147,9 +147,12 @@ __global__ void __launch_bounds__(D) zscan_kernel(const float* __restrict__ zpar
 }
 
 // ---------------------------------------------------------------------------
-// state_kernel: grid = BH * S * CH, one CTA per (head, segment, chunk of tokens).
+// state_kernel: persistent, min(BH * S * CH, SMs) CTAs; each walks the units (head,
+// segment, chunk of tokens) blockIdx.x, blockIdx.x + gridDim.x, ... with its ring and
+// barrier phases running on from one unit to the next, so the next unit's copies
+// stream while the converter warps drain the last unit's sums.
 //
-// For the chunk's tokens it accumulates, in tensor memory,
+// For a unit's tokens it accumulates, in tensor memory,
 //   columns   0..127: dM = sigma(K)^T V
 //   columns 128..255: G  = sigma(K)^T diag(inv) sigma(K)      (Delta only)
 // with bf16 tcgen05 MMAs (fp32 accumulation). sigma(K) is split into
@@ -169,8 +172,8 @@ __global__ void __launch_bounds__(D) zscan_kernel(const float* __restrict__ zpar
 // adjacent so that hi^T [V | GH] is one N = 256 MMA.
 // Warps 0..15 convert (one 8-feature group of two tokens each per slab: 64-token
 // slabs measured ~6% faster for this kernel than 32-token ones with twice the
-// stages, the per-slab waits and arrivals being paid on twice the work), warp 16
-// issues the TMA copies, warp 17 issues the MMAs.
+// stages, the per-slab waits and arrivals being paid on twice the work) and drain
+// each unit's sums, warp 16 issues the TMA copies, warp 17 issues the MMAs.
 // ---------------------------------------------------------------------------
 constexpr int kSlab = 64;
 constexpr int kStages = 3;
