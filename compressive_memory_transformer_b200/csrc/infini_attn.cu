@@ -1,8 +1,12 @@
 // infini_attn.cu — the C ABI (include/infini_attn.h): argument checks, scratch
 // memory, and the launch sequence of the forward.
 //
-// bf16 (d = 128): zpart -> zscan -> state (tcgen05 bf16, sigma(K) as a hi/lo pair)
-//                 -> chain (Linear+Delta: G_s M_{s-1} on tcgen05 tf32) -> attn (tcgen05 bf16)
+// bf16 (d = 128), several segments:
+//   Linear+Delta: zpart -> zscan -> state (tcgen05 bf16, sigma(K) as a hi/lo pair)
+//                 -> chain (G_s M_{s-1} on tcgen05 tf32) -> attn (tcgen05 bf16)
+//   Linear:       state (also the sums of sigma(K)) -> chain (with the z scan) -> attn
+// one segment (every step call): prep_first, then the one-segment update (a second
+//   stream) beside attn
 // fp32 (d <= 128): f32_state -> f32_attn (CUDA cores)
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
