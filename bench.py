@@ -42,9 +42,9 @@ UNIT = "tokens/s"
 B, H, D, N, L = 4, 8, 128, 2048, 32768
 WORKLOAD = (f"1B-LM layer shape: B={B}, H={H}, d={D}, N={N}, L={L} ({L // N} segments), "
             "bf16 q/k/v, fp32 state from zero; step = Linear forward + Linear+Delta forward")
-# kernels per forward of the workload (several segments): Linear state, zscan, chain,
-# attn; Linear+Delta zpart, zscan, state, chain, attn
-LAUNCHES_PER_STEP = 4 + 5
+# kernels per forward of the workload (several segments): Linear state, chain (which
+# also scans z), attn; Linear+Delta zpart, zscan, state, chain, attn
+LAUNCHES_PER_STEP = 3 + 5
 
 
 def attn_flops_per_launch():
