@@ -283,6 +283,9 @@ int infini_attn_step_f32(const float* q, const float* k, const float* v, const f
  *     state and the state update runs beside it on a second stream of the
  *     library (forked from and joined back into `stream` within the call):
  *     event 1 then marks the fork, event 2 the point where both are done.
+ *     That second stream is one per device for the whole process: one-segment
+ *     calls from several host threads take turns on it (a mutex keeps each
+ *     fork..join sequence whole), so their state updates run one after another.
  */
 typedef struct {
   void* workspace;
