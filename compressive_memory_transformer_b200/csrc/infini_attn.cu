@@ -509,6 +509,7 @@ int backward_impl(const void* q, const void* k, const void* v, const float* beta
 int gemm_checks(const void* A, const void* Bm, const void* C, long long M, int N, int K) {
   if (!A || !Bm || !C) return INFINI_ERR_NULL;
   if (M < 1 || N < 1 || K < 1) return INFINI_ERR_SHAPE;
+  if (M >= (1LL << 31)) return INFINI_ERR_SHAPE;  // tensor-map row coordinates are 32-bit
   if (M % 128 || N % 128 || K % 128) return INFINI_ERR_UNSUPPORTED;
   if (overflows(M, K) || overflows(M * K, 2) || overflows(M, N) || overflows(M * N, 2) ||
       overflows((long long)K, (long long)N * 2) || M / 128 * (N / 128) >= (1LL << 31))
@@ -540,7 +541,7 @@ int layer_forward_impl(const void* x, const void* Wq, const void* Wk, const void
     return INFINI_ERR_UNSUPPORTED;
   const long long rows = (long long)B * L;
   if (overflows(rows, (long long)H * d * 2) || overflows(rows, (long long)D_model * 2) ||
-      L >= (1LL << 31))
+      L >= (1LL << 31) || rows >= (1LL << 31))  // the projections' row coordinates are 32-bit
     return INFINI_ERR_SHAPE;
   const void* ins[] = {x, Wq, Wk, Wv, Wo};
   for (const void* q : ins)
@@ -774,7 +775,9 @@ size_t infini_attn_layer_workspace_size(int B, long long L, int D_model, int H, 
   (void)D_model;
   if (B < 1 || L < 1 || H < 1 || H_kv < 1 || N < 1 || d != 128 || H % H_kv != 0) return 0;
   const long long rows = (long long)B * L;
-  if (rows % 128 != 0 || L >= (1LL << 31) || overflows(rows, (long long)H * d * 2)) return 0;
+  if (rows % 128 != 0 || L >= (1LL << 31) || rows >= (1LL << 31) ||
+      overflows(rows, (long long)H * d * 2))
+    return 0;
   const size_t nq = (size_t)(rows * H * d), nkv = (size_t)(rows * H_kv * d);
   const size_t proj_bytes = ((2 * nq + 2 * nkv) * 2 + 255) & ~(size_t)255;
   const int S = (int)((L + N - 1) / N);

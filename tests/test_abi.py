@@ -212,6 +212,7 @@ def test_backward_rejects_bad_arguments(lib, kw, code):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(A=None), -1), (dict(M=0), -2), (dict(K=-128), -2),
+    (dict(M=1 << 31, N=128, K=128), -2),  # rows past 32-bit tensor-map coordinates
     (dict(M=200), -3), (dict(N=96), -3), (dict(K=64), -3),
     (dict(A=IN0 + 8), -4),
     (dict(C=IN0 + 4096), -8),  # C over A
@@ -226,6 +227,7 @@ def test_gemm_rejects_bad_arguments(lib, kw, code):
 @pytest.mark.parametrize("kw,code", [
     (dict(x=None), -1), (dict(Wo=None), -1), (dict(M_in=OUT0 * 2), -1),
     (dict(B=0), -2), (dict(H=4, H_kv=3), -2), (dict(H_kv=0), -2),
+    (dict(B=2, L=1 << 30), -2),  # B * L rows past 32-bit tensor-map coordinates
     (dict(d=64), -3), (dict(D_model=192), -3), (dict(L=100), -3), (dict(mode=2), -3),
     (dict(y=OUT0 + 8), -4),
     (dict(y=IN0), -8),  # y over x
@@ -255,6 +257,7 @@ def test_backward_and_layer_workspace_sizes_are_host_only(lib):
     assert 0 < l1 < l2                                                  # more key/value heads
     assert lib.layer_workspace_size(1, 100, 256, 2, 2, 256) == 0        # B * L % 128
     assert lib.layer_workspace_size(1, 1024, 256, 3, 2, 256) == 0       # H % H_kv
+    assert lib.layer_workspace_size(2, 1 << 30, 256, 2, 2, 2048) == 0   # B * L >= 2^31
 
 
 def test_binding_rejects_bad_tensors_before_the_library(lib):
