@@ -393,6 +393,8 @@ int decode_impl(const void* q, const void* k, const void* v, const float* beta, 
   if (d != 128) return INFINI_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
   if (BH > (1LL << 30) || overflows(BH, (long long)N * d * 2)) return INFINI_ERR_SHAPE;
+  // the decode grid has a row per head and a layer per group of 16 new tokens
+  if (BH > 65535 || (n + 15) / 16 > 65535) return INFINI_ERR_SHAPE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(k_cache) ||
       !aligned16(v_cache) || !aligned16(M) || !aligned16(z))
     return INFINI_ERR_ALIGN;

@@ -183,9 +183,10 @@ int infini_attn_state_sum(const float* dM, const float* dz, int count, const flo
  *                      causal softmax attention over cache rows 0..t and A_mem the
  *                      retrieval from (M, z) as passed in. Every token gets what
  *                      infini_attn_forward gives it on the same stream of tokens.
- * Requires d == 128, n >= 1, pos >= 0, pos + n <= N, mode 0 or 1, 16-byte aligned
- * pointers and no overlap between out, the caches, the state and the inputs
- * (INFINI_ERR_NULL / SHAPE / UNSUPPORTED / ALIGN / ALIAS before any launch).
+ * Requires d == 128, n >= 1, pos >= 0, pos + n <= N, B * H <= 65535, n <= 1048560
+ * (65535 groups of 16 tokens), mode 0 or 1, 16-byte aligned pointers and no overlap
+ * between out, the caches, the state and the inputs (INFINI_ERR_NULL / SHAPE /
+ * UNSUPPORTED / ALIGN / ALIAS before any launch).
  * Scratch comes from the stream-ordered allocator on `stream` (INFINI_ERR_NOMEM).
  * Built for small n; a whole segment at once is cheaper through infini_attn_step.
  */

@@ -117,6 +117,7 @@ def call_decode(lib, q=FAKE, k=FAKE + 4096, v=FAKE + 8192, beta=FAKE + 12288, k_
     (dict(out=None), -1),
     (dict(B=0), -2), (dict(H=0), -2), (dict(n=0), -2), (dict(pos=-1), -2), (dict(N=0), -2),
     (dict(pos=120, n=9), -2),             # pos + n > N
+    (dict(B=256, H=256), -2),             # more heads than the grid's rows hold
     (dict(d=64), -3), (dict(mode=2), -3),
     (dict(q=FAKE + 8), -4), (dict(k_cache=FAKE * 3 + 8), -4), (dict(M=FAKE * 4 + 4), -4),
     (dict(out=FAKE), -8),                 # out is q
