@@ -239,6 +239,8 @@ int forward_impl(const void* q, const void* k, const void* v, const float* beta,
                  int layout = INFINI_LAYOUT_BHLD) {
   if (dtype != INFINI_DTYPE_BF16 && dtype != INFINI_DTYPE_F32) return INFINI_ERR_UNSUPPORTED;
   if (H_kv == 0) H_kv = H;
+  // the fp32 path's attention grid has a row per head
+  if (dtype == INFINI_DTYPE_F32 && (long long)B * H > 65535) return INFINI_ERR_SHAPE;
   const size_t esize = dtype == INFINI_DTYPE_BF16 ? 2 : 4;
   int st = check_common(q, k, v, beta, M_in, z_in, out, M_out, z_out, B, H, L, N, d, mode, esize,
                         H_kv);

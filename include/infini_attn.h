@@ -257,13 +257,15 @@ int infini_attn_layer_forward(const void* x, const void* Wq, const void* Wk, con
 /*
  * C [M][N] = A [M][K] B [K][N]: bf16 row-major in and out, fp32 accumulation on the
  * tensor cores (the layer's projection GEMM). M, N, K multiples of 128
- * (INFINI_ERR_UNSUPPORTED otherwise); device pointers, 16-byte aligned; C may not
+ * (INFINI_ERR_UNSUPPORTED otherwise), M < 2^31 (INFINI_ERR_SHAPE); device pointers,
+ * 16-byte aligned; C may not
  * overlap A or B. Asynchronous on `stream`, no scratch.
  */
 int infini_attn_gemm_bf16(const void* A, const void* B, void* C, long long M, int N, int K,
                           void* stream);
 
-/* fp32 q/k/v/out variants of infini_attn_forward and infini_attn_step; 1 <= d <= 128. */
+/* fp32 q/k/v/out variants of infini_attn_forward and infini_attn_step; 1 <= d <= 128,
+ * B * H <= 65535 (INFINI_ERR_SHAPE beyond). */
 int infini_attn_forward_f32(const float* q, const float* k, const float* v, const float* beta,
                             const float* M_in, const float* z_in, float* out, float* M_out,
                             float* z_out, int B, int H, long long L, int N, int d, int mode,

@@ -68,6 +68,8 @@ def test_forward_rejects_bad_arguments(lib, kw, code):
 def test_f32_rejects_wide_heads(lib):
     assert call_fwd(lib, d=129, name="infini_attn_forward_f32") == -3
     assert call_fwd(lib, d=0, name="infini_attn_forward_f32") == -2
+    # more heads than the fp32 attention grid's rows hold
+    assert call_fwd(lib, B=256, H=256, name="infini_attn_forward_f32") == -2
 
 
 def test_step_rejects_bad_arguments(lib):
