@@ -38,13 +38,13 @@ constexpr int kGemmSmem = kStages * 2 * kTile + 256 + 1024;
 enum { G_FULL = 0, G_EMPTY = 3, G_AFULL = 6, G_AEMPTY = 8, G_DRAIN = 10, G_COUNT = 11 };
 
 struct GemmParams {
-  int tiles_n;     // N / 128 (wide kernel: N / 256, summed over the column groups)
-  int ksteps;      // K / 128 (wide kernel: K / 64)
+  int tiles_n;     // N / 128 (pair kernel: N / 256, summed over the column groups)
+  int ksteps;      // K / 128 (pair kernel: K / 64)
   unsigned tiles;  // (M / 128) * tiles_n
   long long ldc;   // N
 };
 
-// The wide kernel's column groups: C_g = A B_g for up to three B matrices that share A
+// The pair kernel's column groups: C_g = A B_g for up to three B matrices that share A
 // (the layer's Q, K and V projections of the same x in one launch, so that each
 // 128-row block of A is fetched once for all of them). Group g covers the column tiles
 // [first[g], first[g + 1]) of the launch.
