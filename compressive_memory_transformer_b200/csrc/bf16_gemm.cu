@@ -40,8 +40,8 @@ enum { G_FULL = 0, G_EMPTY = 3, G_AFULL = 6, G_AEMPTY = 8, G_DRAIN = 10, G_COUNT
 struct GemmParams {
   int tiles_n;     // N / 128 (pair kernel: N / 256, summed over the column groups)
   int ksteps;      // K / 128 (pair kernel: K / 64)
-  unsigned tiles;  // (M / 128) * tiles_n
-  long long ldc;   // N
+  unsigned tiles;  // (M / 128) * tiles_n (pair kernel: ceil(M / 256) * tiles_n)
+  long long ldc;   // N (pair kernel: unused, row strides per group)
 };
 
 // The pair kernel's column groups: C_g = A B_g for up to three B matrices that share A
