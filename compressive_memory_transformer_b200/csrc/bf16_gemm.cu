@@ -228,7 +228,7 @@ constexpr int kPA = 16384, kPB = 16384, kPStage = kPA + kPB;
 constexpr int kPOut = 4 * 2 * 4096;
 constexpr int kGemmPSmem = kPStages * kPStage + kPOut + 256 + 1024;
 // FULL (the even CTA's: 1 arrival with the pair's bytes), EMPTY, AFULL (arrivals
-// multicast to both CTAs by the MMA commits), AEMPTY (the even CTA's: 4 warps of each
+// sent to both CTAs by the MMA commits), AEMPTY (the even CTA's: 4 warps of each
 // CTA), DRAIN (both CTAs: every MMA issued has completed)
 enum {
   P_FULL = 0,

@@ -122,7 +122,7 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 }
 
 // ----------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor); no TMA or bulk load in this library multicasts
+// TMA tensor copies: every load lands in the issuing CTA's own shared memory
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
